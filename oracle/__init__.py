@@ -1,0 +1,297 @@
+"""CPU oracle for the gated delta-rule recurrence -- TEST INFRASTRUCTURE ONLY.
+
+Only tests/, __graft_entry__.smoke() and bench.py's CPU-baseline leg may
+import this package. It shares no code with the CUDA path
+(gated_delta_rule_147_b200/); the only module both sides use is the seeded
+input generator gated_delta_rule_147_b200.inputs, which holds none of the
+recurrence's arithmetic.
+
+Every route computes, per head, in fp64, on inputs already rounded to the
+device dtype and then widened:
+
+    S_t = (I - k_t^T (b_t . k_t)) Diag(alpha_t) S_{t-1} + (w_t . k_t)^T v_t
+    o_t = q_t S_t
+
+Routes (each follows a different passage, so they pin each other):
+  recurrence            C token loop (gdr_oracle.c), the oracle proper.
+  recurrence_py         the same definition as a numpy token loop (small cases).
+  unrolled_contributions  S_t = sum_i C_i^(t) with explicit d_k x d_k
+                        transition matrices ("How Linear Attention Remembers",
+                        Analytical Framework).
+  masked_matrix         erase-free case b = 0 as a structured masked matrix
+                        ("The Eraser Trilogy", "The Rosetta Stone").
+  delta_three_line      tied gates b = w = beta written as read / delta /
+                        write-back ("Recurrent Memory: Write, Erase, Decay,
+                        Read", section 03) with decay (section 04).
+  unified_decay_after_erase  the section-05 unified equation with decay applied
+                        after the erase (the page's own order).
+
+Parity: every route is pinned by the tests in tests/test_oracle_pins.py.
+"""
+from __future__ import annotations
+
+import ctypes
+import os
+import subprocess
+import threading
+
+import numpy as np
+
+_HERE = os.path.dirname(os.path.abspath(__file__))
+_SRC = os.path.join(_HERE, "gdr_oracle.c")
+_SO = os.path.join(_HERE, "libgdr_oracle.so")
+_lock = threading.Lock()
+_lib_handle = None
+
+
+def build(force: bool = False) -> str:
+    """Compile the C oracle into oracle/libgdr_oracle.so (gcc, OpenMP)."""
+    if force or not os.path.exists(_SO) or os.path.getmtime(_SO) < os.path.getmtime(_SRC):
+        cmd = ["gcc", "-O2", "-fopenmp", "-fPIC", "-shared", "-o", _SO, _SRC]
+        subprocess.run(cmd, check=True)
+    return _SO
+
+
+def _lib():
+    global _lib_handle
+    with _lock:
+        if _lib_handle is None:
+            build()
+            _lib_handle = load_library(_SO)
+        return _lib_handle
+
+
+def max_threads() -> int:
+    return int(_lib().gdr_oracle_max_threads())
+
+
+def f64(x):
+    """Widen a torch tensor or numpy array (any float dtype) to contiguous fp64 numpy."""
+    if x is None:
+        return None
+    if hasattr(x, "detach"):
+        x = x.detach().to("cpu")
+        import torch
+        x = x.to(torch.float64).numpy()
+    return np.ascontiguousarray(np.asarray(x, dtype=np.float64))
+
+
+def _ptr(a):
+    if a is None:
+        return None
+    return a.ctypes.data_as(ctypes.POINTER(ctypes.c_double))
+
+
+def _resolve_gates(alpha, b, w, gates):
+    """Returns (alpha, alpha_pc, b, b_pc, w, w_pc) with 'tied' resolved to w := b."""
+    g = dict(gates or {})
+    ka, kb, kw = g.get("alpha", "none"), g.get("b", "none"), g.get("w", "none")
+    alpha = None if ka == "none" else f64(alpha)
+    b = None if kb == "none" else f64(b)
+    if kw == "tied":
+        w, kw = b, kb
+    else:
+        w = None if kw == "none" else f64(w)
+    return alpha, int(ka == "channel"), b, int(kb == "channel"), w, int(kw == "channel")
+
+
+def load_library(path: str):
+    """Load another build of gdr_oracle.c (tests compile deliberately broken
+    copies to check that the pins catch each mistake)."""
+    lib = ctypes.CDLL(path)
+    dp = ctypes.POINTER(ctypes.c_double)
+    lib.gdr_oracle_forward.argtypes = [ctypes.c_int] * 5 + [dp, dp, dp, dp, ctypes.c_int,
+                                                            dp, ctypes.c_int, dp, ctypes.c_int,
+                                                            dp, dp, dp, ctypes.c_int]
+    lib.gdr_oracle_forward.restype = ctypes.c_int
+    lib.gdr_oracle_max_threads.restype = ctypes.c_int
+    return lib
+
+
+def recurrence(q, k, v, alpha=None, b=None, w=None, S0=None, gates=None, nthreads: int = 0,
+               lib=None):
+    """Token-by-token recurrence (the C oracle). Returns (o, S_T) in fp64.
+
+    q,k [B,T,H,dk]; v [B,T,H,dv]; gates scalar [B,T,H] or channel [B,T,H,dk];
+    S0 [B,H,dk,dv] or None. gates = {"alpha": kind, "b": kind, "w": kind},
+    kinds "none" (alpha=1, b=0, w=1), "scalar", "channel", and for w "tied".
+    """
+    q, k, v = f64(q), f64(k), f64(v)
+    B, T, H, dk = q.shape
+    dv = v.shape[-1]
+    a, apc, bb, bpc, ww, wpc = _resolve_gates(alpha, b, w, gates)
+    S0 = f64(S0)
+    o = np.zeros((B, T, H, dv), dtype=np.float64)
+    S_T = np.zeros((B, H, dk, dv), dtype=np.float64)
+    rc = (lib or _lib()).gdr_oracle_forward(B, T, H, dk, dv, _ptr(q), _ptr(k), _ptr(v), _ptr(a), apc,
+                                   _ptr(bb), bpc, _ptr(ww), wpc, _ptr(S0), _ptr(o), _ptr(S_T),
+                                   int(nthreads))
+    if rc != 0:
+        raise RuntimeError(f"gdr_oracle_forward returned {rc}")
+    return o, S_T
+
+
+def decode_step(q, k, v, alpha, b, w, S, gates=None, nthreads: int = 0):
+    """One decode token per head: the recurrence with T = 1 and the state
+    carried between calls. q,k [B,H,dk]; v [B,H,dv]; gates [B,H] or [B,H,dk];
+    S [B,H,dk,dv]. Returns (o [B,H,dv], S_new)."""
+    q, k, v = f64(q)[:, None], f64(k)[:, None], f64(v)[:, None]
+    ex = lambda g: None if g is None else f64(g)[:, None]
+    o, S_new = recurrence(q, k, v, ex(alpha), ex(b), ex(w), f64(S), gates, nthreads)
+    return o[:, 0], S_new
+
+
+# ---------------------------------------------------------------------------
+# Independent routes used to pin the oracle (small inputs only).
+# ---------------------------------------------------------------------------
+
+def _full_gates(alpha, b, w, gates, B, T, H, dk):
+    """Materialise all three gates as [B,T,H,dk] fp64 arrays (broadcasting only)."""
+    a, apc, bb, bpc, ww, wpc = _resolve_gates(alpha, b, w, gates)
+
+    def full(g, pc, dflt):
+        if g is None:
+            return np.full((B, T, H, dk), dflt)
+        return np.broadcast_to(g if pc else g[..., None], (B, T, H, dk)).copy()
+    return full(a, apc, 1.0), full(bb, bpc, 0.0), full(ww, wpc, 1.0)
+
+
+def recurrence_py(q, k, v, alpha=None, b=None, w=None, S0=None, gates=None):
+    """The definition again, as a numpy token loop (spec form:
+    decay, then erase read with b.k, erase along k, write with key w.k)."""
+    q, k, v = f64(q), f64(k), f64(v)
+    B, T, H, dk = q.shape
+    dv = v.shape[-1]
+    A, Bg, W = _full_gates(alpha, b, w, gates, B, T, H, dk)
+    S0 = f64(S0)
+    o = np.zeros((B, T, H, dv))
+    ST = np.zeros((B, H, dk, dv))
+    for bi in range(B):
+        for h in range(H):
+            S = np.zeros((dk, dv)) if S0 is None else S0[bi, h].copy()
+            for t in range(T):
+                kt = k[bi, t, h]
+                S = A[bi, t, h][:, None] * S
+                r = (Bg[bi, t, h] * kt) @ S
+                S = S - np.outer(kt, r) + np.outer(W[bi, t, h] * kt, v[bi, t, h])
+                o[bi, t, h] = q[bi, t, h] @ S
+            ST[bi, h] = S
+    return o, ST
+
+
+def unrolled_contributions(q, k, v, alpha=None, b=None, w=None, S0=None, gates=None):
+    """State as a sum of per-position contributions ("How Linear Attention
+    Remembers", Analytical Framework): S_t = T_t(S_{t-1}) + W_t with the
+    linear map T_t(S) = M_t S, M_t = (I - k_t^T (b_t . k_t)) Diag(alpha_t)
+    materialised as a d_k x d_k matrix, and the write W_t = (w_t . k_t)^T v_t.
+    Then S_t = P_{t,0} S0 + sum_{i<=t} C_i^(t), C_i^(t) = P_{t,i} W_i with
+    P_{t,i} = M_t M_{t-1} ... M_{i+1} (the product of transitions after i).
+    o_t = q_t S_t. Cost O(T^2 d_k^2 (d_k + d_v)): tiny inputs only."""
+    q, k, v = f64(q), f64(k), f64(v)
+    B, T, H, dk = q.shape
+    dv = v.shape[-1]
+    A, Bg, Wg = _full_gates(alpha, b, w, gates, B, T, H, dk)
+    S0 = f64(S0)
+    I = np.eye(dk)
+    o = np.zeros((B, T, H, dv))
+    ST = np.zeros((B, H, dk, dv))
+    for bi in range(B):
+        for h in range(H):
+            M = [(I - np.outer(k[bi, t, h], Bg[bi, t, h] * k[bi, t, h])) @ np.diag(A[bi, t, h])
+                 for t in range(T)]
+            Wr = [np.outer(Wg[bi, t, h] * k[bi, t, h], v[bi, t, h]) for t in range(T)]
+            for t in range(T):
+                S = np.zeros((dk, dv))
+                for i in range(t + 1):
+                    P = I.copy()
+                    for j in range(i + 1, t + 1):
+                        P = M[j] @ P
+                    S += P @ Wr[i]
+                if S0 is not None:
+                    P = I.copy()
+                    for j in range(0, t + 1):
+                        P = M[j] @ P
+                    S += P @ S0[bi, h]
+                o[bi, t, h] = q[bi, t, h] @ S
+                if t == T - 1:
+                    ST[bi, h] = S
+    return o, ST
+
+
+def masked_matrix(q, k, v, alpha=None, w=None, gates=None):
+    """Erase-free case (b = 0) read as a structured masked matrix ("The Eraser
+    Trilogy", "The Rosetta Stone"): with gamma_t = prod_{j<=t} alpha_j (per
+    channel), o_t = sum_{i<=t} [sum_c q_{t,c} (gamma_{t,c}/gamma_{i,c})
+    w_{i,c} k_{i,c}] v_i. The decay ratio is formed as a product of alphas over
+    (i, t], never as a quotient, so any alpha in (0, 1] works. S0 = 0."""
+    q, k, v = f64(q), f64(k), f64(v)
+    B, T, H, dk = q.shape
+    dv = v.shape[-1]
+    g = dict(gates or {})
+    g["b"] = "none"
+    A, _, W = _full_gates(alpha, None, w, g, B, T, H, dk)
+    o = np.zeros((B, T, H, dv))
+    for bi in range(B):
+        for h in range(H):
+            Mk = np.zeros((T, T))
+            for t in range(T):
+                ratio = np.ones(dk)
+                for i in range(t, -1, -1):
+                    Mk[t, i] = np.sum(q[bi, t, h] * ratio * W[bi, i, h] * k[bi, i, h])
+                    ratio = ratio * A[bi, i, h]
+            o[bi, :, h] = Mk @ v[bi, :, h]
+    return o
+
+
+def delta_three_line(q, k, v, alpha=None, beta=None, S0=None, alpha_kind="scalar"):
+    """Tied gates b = w = beta (scalar per token-head) in the read / delta /
+    write-back form ("Recurrent Memory: Write, Erase, Decay, Read", section 03)
+    with the decay of section 04 applied to the carried state first:
+        S'    = Diag(alpha_t) S_{t-1}
+        v_old = k_t S'
+        u_t   = beta_t (v_t - v_old)
+        S_t   = S' + k_t^T u_t,     o_t = q_t S_t
+    alpha [B,T,H] (scalar) or [B,T,H,dk] (channel), or None (alpha = 1)."""
+    q, k, v = f64(q), f64(k), f64(v)
+    B, T, H, dk = q.shape
+    dv = v.shape[-1]
+    beta = f64(beta)
+    alpha = None if alpha is None else f64(alpha)
+    S0 = f64(S0)
+    o = np.zeros((B, T, H, dv))
+    ST = np.zeros((B, H, dk, dv))
+    for bi in range(B):
+        for h in range(H):
+            S = np.zeros((dk, dv)) if S0 is None else S0[bi, h].copy()
+            for t in range(T):
+                if alpha is not None:
+                    a = alpha[bi, t, h]
+                    S = (a[:, None] if alpha_kind == "channel" else a) * S
+                v_old = k[bi, t, h] @ S
+                u = beta[bi, t, h] * (v[bi, t, h] - v_old)
+                S = S + np.outer(k[bi, t, h], u)
+                o[bi, t, h] = q[bi, t, h] @ S
+            ST[bi, h] = S
+    return o, ST
+
+
+def unified_decay_after_erase(q, k, v, alpha, beta, S0=None):
+    """The unified equation in the order the section-05 equation of "Recurrent
+    Memory: Write, Erase, Decay, Read" prints it: S_t = Diag(alpha_t)
+    (I - beta_t k_t^T k_t) S_{t-1} + beta_t k_t^T v_t (decay after erase).
+    alpha channel [B,T,H,dk]; beta scalar [B,T,H]."""
+    q, k, v, alpha, beta = f64(q), f64(k), f64(v), f64(alpha), f64(beta)
+    B, T, H, dk = q.shape
+    dv = v.shape[-1]
+    S0 = f64(S0)
+    o = np.zeros((B, T, H, dv))
+    I = np.eye(dk)
+    for bi in range(B):
+        for h in range(H):
+            S = np.zeros((dk, dv)) if S0 is None else S0[bi, h].copy()
+            for t in range(T):
+                kt = k[bi, t, h]
+                S = np.diag(alpha[bi, t, h]) @ (I - beta[bi, t, h] * np.outer(kt, kt)) @ S \
+                    + beta[bi, t, h] * np.outer(kt, v[bi, t, h])
+                o[bi, t, h] = q[bi, t, h] @ S
+    return o
