@@ -1,0 +1,387 @@
+#!/usr/bin/env python
+"""Benchmark of the gated delta-rule hot path on B200.
+
+    python bench.py [--gpus N] [--steps K] [--warmup W] [--impl ours|reference]
+
+A step is one gdr_chunk_fwd over the Gated DeltaNet workload (B=4, H=16,
+T=4096, d_k=d_v=128, bf16, scalar decay, tied scalar beta, chunk 64): the
+whole chunkwise path (load and log-decay scan, intra-chunk products, WY/UT
+transform, inter-chunk state propagation, write-back). Inputs (274 MB) are
+larger than the 126 MB L2, so no flush is needed between steps. The decode
+step (256 x 32 heads, d = 128, 1000 sequential steps, fp32 state in HBM) is
+measured in the same run and reported under "decode"; the KDA and Gated
+DeltaNet-2 chunk workloads under "other_workloads".
+
+With N > 1 (torchrun, one process per GPU) every rank runs its own copy of
+the workload (heads are independent; no collective on the data path), the
+timed region is bracketed by barriers and the time is the max over ranks.
+
+--impl reference times the fp64 CPU oracle (the only reference this project
+has) on a bounded sample of the same workload on the host cores.
+"""
+from __future__ import annotations
+
+import argparse
+import json
+import os
+import statistics
+import subprocess
+import sys
+import tempfile
+import time
+
+ROOT = os.path.dirname(os.path.abspath(__file__))
+sys.path.insert(0, ROOT)
+
+METRIC = "gated-delta-rule fwd tokens/s and % roofline; decode state GB/s vs HBM peak"
+# Algorithmic work per token-head (2 flops per multiply-add) of the chunkwise
+# contractions at C = 64, d = 128: general gates and tied scalar beta.
+FLOPS_PER_TOKEN_HEAD = {"general": 281259, "tied": 182955}
+L2_BYTES = 126 * 2**20
+
+
+def peaks():
+    p = os.path.join(ROOT, "MEASURED_PEAKS.json")
+    if os.path.exists(p):
+        d = json.load(open(p))
+        return {"hbm_gbs": d["hbm_gbs"], "bf16_tflops": d["bf16_tflops"],
+                "bf16_tflops_sustained": d.get("bf16_tflops_sustained"), "source": "measured"}
+    return {"hbm_gbs": 6650.0, "bf16_tflops": 1590.0, "bf16_tflops_sustained": 1400.0,
+            "source": "fallback"}
+
+
+def workload_bytes(wl):
+    """Bytes that must cross HBM once: inputs read, o written, S0 read if
+    given, S_T written."""
+    el = 2 if wl.dtype == "bf16" else 4
+    th = wl.B * wl.T * wl.H
+    gate = lambda kind: 0 if kind in ("none", "tied") else (th if kind == "scalar" else th * wl.dk)
+    n = th * (2 * wl.dk + 2 * wl.dv) + gate(wl.alpha) + gate(wl.b) + gate(wl.w)
+    state = wl.B * wl.H * wl.dk * wl.dv * 4
+    return n * el + state * (1 + int(wl.s0))
+
+
+def workload_flops(wl):
+    kind = "tied" if wl.w == "tied" and wl.b == "scalar" else "general"
+    return FLOPS_PER_TOKEN_HEAD[kind] * wl.B * wl.T * wl.H
+
+
+class ClockSampler:
+    """nvidia-smi clocks and throttle reasons sampled during the timed region."""
+
+    FIELDS = ("index,clocks.sm,clocks.max.sm,power.draw,clocks_event_reasons.active,"
+              "clocks_event_reasons.hw_slowdown,clocks_event_reasons.hw_thermal_slowdown,"
+              "clocks_event_reasons.sw_thermal_slowdown,clocks_event_reasons.sw_power_cap")
+
+    def __init__(self, device_index: int):
+        self.idx = device_index
+        self.proc = None
+        self.path = None
+
+    def __enter__(self):
+        fd, self.path = tempfile.mkstemp(suffix=".csv")
+        os.close(fd)
+        try:
+            self.proc = subprocess.Popen(
+                ["nvidia-smi", f"--id={self.idx}", f"--query-gpu={self.FIELDS}",
+                 "--format=csv,noheader,nounits", "-lms", "100"],
+                stdout=open(self.path, "w"), stderr=subprocess.DEVNULL)
+            time.sleep(0.3)
+        except OSError:
+            self.proc = None
+        return self
+
+    def __exit__(self, *exc):
+        if self.proc is not None:
+            self.proc.terminate()
+            try:
+                self.proc.wait(timeout=5)
+            except subprocess.TimeoutExpired:
+                self.proc.kill()
+
+    def summary(self):
+        rows = []
+        if self.path and os.path.exists(self.path):
+            for line in open(self.path):
+                parts = [x.strip() for x in line.split(",")]
+                if len(parts) >= 9 and parts[1].replace(".", "").isdigit():
+                    rows.append(parts)
+            os.unlink(self.path)
+        if not rows:
+            return {"sm_mhz": None, "sm_max_mhz": None, "reasons": ["unsampled"], "samples": 0}
+        sm = [float(r[1]) for r in rows]
+        names = ["hw_slowdown", "hw_thermal_slowdown", "sw_thermal_slowdown", "sw_power_cap"]
+        reasons = sorted({names[i] for r in rows for i in range(4) if r[5 + i].lower() == "active"})
+        return {"sm_mhz": statistics.median(sm), "sm_max_mhz": float(rows[0][2]),
+                "reasons": reasons, "samples": len(rows),
+                "power_w_max": max(float(r[3]) for r in rows if r[3].replace(".", "").isdigit())}
+
+
+def dist_env():
+    ws = int(os.environ.get("WORLD_SIZE", "1"))
+    return ws, int(os.environ.get("RANK", "0")), int(os.environ.get("LOCAL_RANK", "0"))
+
+
+# ------------------------------------------------------------------ ours ---
+def prepare_chunk(wl, dev):
+    import torch
+    from gated_delta_rule_147_b200.inputs import make_chunk_inputs
+    inp = make_chunk_inputs(wl)
+    d = {k: (v.to(dev) if hasattr(v, "to") else v) for k, v in inp.items()}
+    return inp, d
+
+
+def chunk_call(d, wl, o, ST, stream):
+    from gated_delta_rule_147_b200 import TIED, chunk_fwd
+    w = TIED if wl.w == "tied" else d["w"]
+    chunk_fwd(d["q"], d["k"], d["v"], d["alpha"], d["b"], w, d["S0"], out=o, S_T=ST, stream=stream)
+
+
+def time_chunk(wl, dev, steps, warmup, barrier):
+    """Device time per launch (CUDA events on the launching stream)."""
+    import torch
+    inp, d = prepare_chunk(wl, dev)
+    o = torch.empty((wl.B, wl.T, wl.H, wl.dv), dtype=d["v"].dtype, device=dev)
+    ST = torch.empty((wl.B, wl.H, wl.dk, wl.dv), dtype=torch.float32, device=dev)
+    stream = torch.cuda.current_stream()
+    for _ in range(warmup):
+        chunk_call(d, wl, o, ST, stream)
+    torch.cuda.synchronize()
+    barrier()
+    ev = [torch.cuda.Event(enable_timing=True) for _ in range(steps + 1)]
+    ev[0].record(stream)
+    for i in range(steps):
+        chunk_call(d, wl, o, ST, stream)
+        ev[i + 1].record(stream)
+    torch.cuda.synchronize()
+    per = [ev[i].elapsed_time(ev[i + 1]) for i in range(steps)]
+    total = ev[0].elapsed_time(ev[steps])
+    barrier()
+    return inp, d, total, per
+
+
+def time_chunk_e2e(inp, wl, dev, steps, warmup):
+    """Same metric through the public API with host buffers: every step copies
+    its inputs from pinned host memory to the device and reads o back."""
+    import torch
+    host = {k: (v.pin_memory() if hasattr(v, "pin_memory") else v) for k, v in inp.items()}
+    dbuf = {k: (torch.empty_like(v, device=dev) if hasattr(v, "pin_memory") else v) for k, v in host.items()}
+    o = torch.empty((wl.B, wl.T, wl.H, wl.dv), dtype=host["v"].dtype, device=dev)
+    o_host = torch.empty(o.shape, dtype=o.dtype, pin_memory=True)
+    stream = torch.cuda.current_stream()
+    tensors = [k for k, v in host.items() if hasattr(v, "pin_memory")]
+    h2d = sum(host[k].numel() * host[k].element_size() for k in tensors)
+    d2h = o.numel() * o.element_size()
+
+    def step():
+        for k in tensors:
+            dbuf[k].copy_(host[k], non_blocking=True)
+        chunk_call(dbuf, wl, o, None, stream)
+        o_host.copy_(o, non_blocking=True)
+
+    for _ in range(warmup):
+        step()
+    torch.cuda.synchronize()
+    e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    e0.record(stream)
+    for _ in range(steps):
+        step()
+    e1.record(stream)
+    torch.cuda.synchronize()
+    return e0.elapsed_time(e1), h2d, d2h
+
+
+def time_decode(dev, nsteps, warmup):
+    import torch
+    from gated_delta_rule_147_b200 import decode_step
+    from gated_delta_rule_147_b200.inputs import DECODE, make_decode_state, make_decode_steps
+    dw = DECODE
+    S = make_decode_state(dw).to(dev)
+    steps = []
+    for s0 in range(0, nsteps, 100):
+        for st in make_decode_steps(dw, range(s0, min(s0 + 100, nsteps)), threads=os.cpu_count() or 8):
+            steps.append({k: v.to(dev) for k, v in st.items()})
+    o = torch.empty((dw.B, dw.H, dw.dv), dtype=torch.bfloat16, device=dev)
+    stream = torch.cuda.current_stream()
+
+    def run(i):
+        d = steps[i % len(steps)]
+        decode_step(d["q"], d["k"], d["v"], d["alpha"], d["b"], d["w"], S, out=o, stream=stream)
+
+    for i in range(warmup):
+        run(i)
+    torch.cuda.synchronize()
+    e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    e0.record(stream)
+    for i in range(nsteps):
+        run(i)
+    e1.record(stream)
+    torch.cuda.synchronize()
+    ms = e0.elapsed_time(e1) / nsteps
+    state = dw.B * dw.H * dw.dk * dw.dv * 4
+    tok = dw.B * dw.H * (2 * dw.dk + dw.dv + 3 * dw.dk + dw.dv) * 2
+    return {"workload": f"decode B={dw.B} H={dw.H} d_k=d_v={dw.dk} bf16 tokens, fp32 state, "
+                        f"GDN-2 channel gates, {nsteps} sequential steps",
+            "ms_per_step": ms, "launches": nsteps,
+            "state_gbs": 2 * state / (ms * 1e-3) / 1e9,
+            "total_gbs": (2 * state + tok) / (ms * 1e-3) / 1e9}
+
+
+def cpu_baseline(wl, budget_s=15.0):
+    """The oracle, untuned, on host cores over a bounded sample of heads (full
+    sequence each); value in tokens/s of the same workload."""
+    import oracle
+    from gated_delta_rule_147_b200.inputs import make_chunk_inputs
+    cores = len(os.sched_getaffinity(0))
+    small = wl.with_(B=1, H=1, T=512)
+    inp = make_chunk_inputs(small)
+    t = time.perf_counter()
+    oracle.recurrence(inp["q"], inp["k"], inp["v"], inp["alpha"], inp["b"], inp["w"], inp["S0"],
+                      inp["gates"], nthreads=1)
+    per_head_token = (time.perf_counter() - t) / small.T
+    heads = max(1, min(wl.B * wl.H, int(budget_s * cores / (per_head_token * wl.T))))
+    heads = max(cores, heads) if heads >= cores else heads
+    sample = wl.with_(B=1, H=heads)
+    inp = make_chunk_inputs(sample)
+    t = time.perf_counter()
+    oracle.recurrence(inp["q"], inp["k"], inp["v"], inp["alpha"], inp["b"], inp["w"], inp["S0"],
+                      inp["gates"], nthreads=cores)
+    dt = time.perf_counter() - t
+    token_heads = heads * wl.T
+    return {"value": token_heads / wl.H / dt, "unit": "tokens/s", "cores": min(cores, heads),
+            "kind": "oracle",
+            "sample": f"{heads} of {wl.B * wl.H} heads of the same workload, full T={wl.T}, "
+                      f"fp64 token loop, {dt:.1f} s"}
+
+
+def run_ours(args):
+    import torch
+    import torch.distributed as dist
+    from gated_delta_rule_147_b200.inputs import WORKLOADS
+    ws, rank, local = dist_env()
+    torch.cuda.set_device(local)
+    dev = torch.device("cuda", local)
+    if ws > 1:
+        import datetime
+        dist.init_process_group("nccl", timeout=datetime.timedelta(seconds=120))
+        barrier = lambda: dist.barrier(device_ids=[local])
+    else:
+        barrier = lambda: None
+    pk = peaks()
+    wl = WORKLOADS["gdn"]
+    with ClockSampler(local) as clk:
+        inp, d, total_ms, per = time_chunk(wl, dev, args.steps, args.warmup, barrier)
+    clocks = clk.summary()
+    t = torch.tensor([total_ms], device=dev)
+    if ws > 1:
+        dist.all_reduce(t, op=dist.ReduceOp.MAX)
+    total_ms = float(t.item())
+    tokens = wl.B * wl.T
+    value = ws * tokens * args.steps / (total_ms * 1e-3)
+    bytes_ = workload_bytes(wl)
+    flops = workload_flops(wl)
+    avg_ms = statistics.fmean(per)
+    t_hbm = bytes_ / (pk["hbm_gbs"] * 1e9)
+    t_tc = flops / (pk["bf16_tflops"] * 1e12)
+    bound = "hbm" if t_hbm >= t_tc else "tensor"
+    achieved_gbs = bytes_ / (avg_ms * 1e-3) / 1e9
+    result = None
+    if rank == 0:
+        e2e_ms, h2d, d2h = time_chunk_e2e(inp, wl, dev, max(3, args.steps // 2), args.warmup)
+        e2e_steps = max(3, args.steps // 2)
+        other = {}
+        for name in ("kda", "gdn2"):
+            w2 = WORKLOADS[name]
+            _, _, tot2, per2 = time_chunk(w2, dev, max(3, args.steps // 2), args.warmup, lambda: None)
+            a2 = statistics.fmean(per2)
+            b2, f2 = workload_bytes(w2), workload_flops(w2)
+            rt = max(b2 / (pk["hbm_gbs"] * 1e9), f2 / (pk["bf16_tflops"] * 1e12))
+            other[name] = {"workload": f"{name} B={w2.B} H={w2.H} T={w2.T} d={w2.dk} bf16 alpha={w2.alpha} "
+                                       f"b={w2.b} w={w2.w} S0={'random' if w2.s0 else 'zero'}",
+                           "tokens_per_s": w2.B * w2.T / (a2 * 1e-3), "ms_per_launch": a2,
+                           "hbm_gbs": b2 / (a2 * 1e-3) / 1e9, "roofline_frac": rt / (a2 * 1e-3)}
+            torch.cuda.empty_cache()
+        dec = time_decode(dev, 1000, 10)
+        dec["frac_of_hbm"] = dec["total_gbs"] / pk["hbm_gbs"]
+        dec["peak_gbs"] = pk["hbm_gbs"]
+        cpu = cpu_baseline(wl) if ws == 1 else None
+        result = {
+            "metric": METRIC, "value": value, "unit": "tokens/s", "n_gpus": ws, "steps": args.steps,
+            "warmup": args.warmup, "ms_per_step": total_ms / args.steps, "higher_is_better": True,
+            "scaling": "weak", "vs_baseline": None, "dtype": "bf16", "data": "synthetic",
+            "config": {"workload": f"Gated DeltaNet chunk forward B={wl.B} H={wl.H} T={wl.T} "
+                                   f"d_k=d_v={wl.dk} bf16, scalar alpha, tied scalar beta, chunk 64",
+                       "global_batch": wl.B * ws, "seq_len": wl.T, "parallelism": f"replicas x{ws}",
+                       "l2": f"inputs {bytes_ / 1e6:.0f} MB > 126 MB L2, no flush"},
+            "roofline": {"bound": bound, "achieved": achieved_gbs if bound == "hbm" else flops / (avg_ms * 1e-3) / 1e12,
+                         "peak": pk["hbm_gbs"] if bound == "hbm" else pk["bf16_tflops"],
+                         "unit": "GB/s" if bound == "hbm" else "TFLOP/s",
+                         "frac": (max(t_hbm, t_tc)) / (avg_ms * 1e-3), "traffic": None,
+                         "kernel": "gdr::chunk::chunk_fwd_kernel<true>",
+                         "algorithmic_bytes": bytes_, "algorithmic_flops": flops,
+                         "tensor_tflops": flops / (avg_ms * 1e-3) / 1e12,
+                         "ms_per_launch": avg_ms, "peak_source": pk["source"]},
+            "e2e": {"value": tokens * e2e_steps / (e2e_ms * 1e-3), "unit": "tokens/s",
+                    "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": d2h},
+            "gpu_launches": args.steps,
+            "clocks": clocks,
+            "decode": dec,
+            "other_workloads": other,
+            "cpu_baseline": cpu,
+        }
+    if ws > 1:
+        dist.barrier(device_ids=[local])
+        dist.destroy_process_group()
+    return result
+
+
+def run_reference(args):
+    ws, rank, _ = dist_env()
+    if rank != 0:
+        return None
+    import oracle
+    from gated_delta_rule_147_b200.inputs import WORKLOADS, make_chunk_inputs
+    wl = WORKLOADS["gdn"]
+    cores = len(os.sched_getaffinity(0))
+    heads = max(1, min(cores, wl.B * wl.H))
+    sample = wl.with_(B=1, H=heads, T=1024)
+    inp = make_chunk_inputs(sample)
+    call = lambda: oracle.recurrence(inp["q"], inp["k"], inp["v"], inp["alpha"], inp["b"], inp["w"],
+                                     inp["S0"], inp["gates"], nthreads=cores)
+    for _ in range(args.warmup):
+        call()
+    t = time.perf_counter()
+    for _ in range(args.steps):
+        call()
+    dt = time.perf_counter() - t
+    value = heads * sample.T * args.steps / wl.H / dt
+    desc = (f"{heads} heads x T={sample.T} of the Gated DeltaNet workload per step, fp64 token "
+            f"loop, OpenMP over heads")
+    return {"impl": "reference", "metric": METRIC, "value": value, "unit": "tokens/s", "n_gpus": ws,
+            "steps": args.steps, "warmup": args.warmup, "ms_per_step": dt * 1e3 / args.steps,
+            "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "f64",
+            "data": "synthetic",
+            "config": {"workload": f"Gated DeltaNet chunk forward B={wl.B} H={wl.H} T={wl.T} "
+                                   f"d_k=d_v={wl.dk} bf16, scalar alpha, tied scalar beta, chunk 64",
+                       "global_batch": wl.B, "seq_len": wl.T, "parallelism": "cpu"},
+            "cpu_baseline": {"value": value, "unit": "tokens/s", "cores": cores, "kind": "oracle",
+                             "sample": desc},
+            "e2e": {"value": value, "unit": "tokens/s", "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0}}
+
+
+def main():
+    ap = argparse.ArgumentParser()
+    ap.add_argument("--gpus", type=int, default=1)
+    ap.add_argument("--steps", type=int, default=20)
+    ap.add_argument("--warmup", type=int, default=5)
+    ap.add_argument("--impl", choices=["ours", "reference"], default="ours")
+    args = ap.parse_args()
+    if args.warmup < 3:
+        args.warmup = 3
+    res = run_reference(args) if args.impl == "reference" else run_ours(args)
+    if res is not None:
+        print(json.dumps(res), flush=True)
+
+
+if __name__ == "__main__":
+    main()

@@ -1,0 +1,79 @@
+"""B200-native gated delta-rule linear attention.
+
+    S_t = (I - k_t^T (b_t . k_t)) Diag(alpha_t) S_{t-1} + (w_t . k_t)^T v_t,
+    o_t = q_t S_t
+
+Entry points (CUDA, sm_100a, through the C ABI in include/gdr.h):
+  gdr_chunk_fwd / chunk_fwd     whole-sequence forward, chunkwise on tcgen05
+  gdr_decode_step / decode_step one token per head, state updated in place
+
+torch is used for device memory and streams only; every step of the
+recurrence runs in the library's kernels. Importing this package does not
+load the library; the first call does (and fails loudly if it cannot).
+"""
+from __future__ import annotations
+
+from ._lib import (GATE_CHANNEL, GATE_NONE, GATE_SCALAR, GATE_TIED, GDR_BF16, GDR_FP32,
+                   GDR_DEVICE_DECAY_RANGE, GDR_DEVICE_TIMEOUT, GdrError, gdr_chunk_fwd,
+                   gdr_decode_step, load)
+
+TIED = "tied"
+_KIND = {"none": GATE_NONE, "scalar": GATE_SCALAR, "channel": GATE_CHANNEL, "tied": GATE_TIED}
+
+
+def _dtype_code(t):
+    import torch
+    if t.dtype == torch.bfloat16:
+        return GDR_BF16
+    if t.dtype == torch.float32:
+        return GDR_FP32
+    raise TypeError(f"unsupported dtype {t.dtype}; use bfloat16 or float32")
+
+
+def _check(*ts):
+    for t in ts:
+        if t is not None and not isinstance(t, str) and not t.is_contiguous():
+            raise ValueError("tensors passed to the library must be contiguous")
+
+
+def _gate_kind(g, ndim_scalar: int):
+    if g is None:
+        return GATE_NONE
+    if isinstance(g, str):
+        if g != TIED:
+            raise ValueError(g)
+        return GATE_TIED
+    return GATE_SCALAR if g.dim() == ndim_scalar else GATE_CHANNEL
+
+
+def chunk_fwd(q, k, v, alpha=None, b=None, w=None, S0=None, *, out=None, final_state=True,
+              S_T=None, chunk: int = 64, d_status=None, stream=None):
+    """Forward over [B,T,H,*] inputs. alpha/b/w: None, a [B,T,H] tensor
+    (scalar gate), a [B,T,H,d_k] tensor (channel gate); w may be TIED (w := b).
+    Returns (o, S_T) with S_T None when final_state is False."""
+    import torch
+    _check(q, k, v, alpha, b, w, S0, out, S_T)
+    B, T, H, dk = q.shape
+    dv = v.shape[-1]
+    o = out if out is not None else torch.empty((B, T, H, dv), dtype=v.dtype, device=v.device)
+    if final_state and S_T is None:
+        S_T = torch.empty((B, H, dk, dv), dtype=torch.float32, device=v.device)
+    gdr_chunk_fwd(q, k, v, alpha, b, None if isinstance(w, str) else w, _gate_kind(alpha, 3),
+                  _gate_kind(b, 3), _gate_kind(w, 3), S0, o, S_T if final_state else None, B, T, H,
+                  dk, dv, chunk, _dtype_code(q), d_status, stream)
+    return o, (S_T if final_state else None)
+
+
+def decode_step(q, k, v, alpha, b, w, S, *, out=None, d_status=None, stream=None):
+    """One token per head: q,k [B,H,d_k]; v [B,H,d_v]; gates [B,H] or
+    [B,H,d_k] (w may be TIED); S [B,H,d_k,d_v] fp32 updated in place.
+    Returns o [B,H,d_v]."""
+    import torch
+    _check(q, k, v, alpha, b, w, S, out)
+    B, H, dk = q.shape
+    dv = v.shape[-1]
+    o = out if out is not None else torch.empty((B, H, dv), dtype=v.dtype, device=v.device)
+    gdr_decode_step(q, k, v, alpha, b, None if isinstance(w, str) else w, _gate_kind(alpha, 2),
+                    _gate_kind(b, 2), _gate_kind(w, 2), S, o, B, H, dk, dv, _dtype_code(q),
+                    d_status, stream)
+    return o

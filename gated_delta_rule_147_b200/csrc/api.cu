@@ -1,0 +1,166 @@
+// C ABI entry points (include/gdr.h): argument checks on the host, TMA tensor
+// maps for the tensor-core path, and dispatch to the kernels.
+#include <cudaTypedefs.h>
+
+#include <cstdint>
+#include <mutex>
+
+#include "common.cuh"
+
+namespace gdr {
+cudaError_t launch_decode(const void* q, const void* k, const void* v, const void* a, const void* b,
+                          const void* w, int ak, int bk, int wk, float* S, void* o, int BH, int dk,
+                          int dv, int dtype, cudaStream_t st);
+int decode_rows_per_thread(int dk, int dv);
+cudaError_t launch_recurrent(const void* q, const void* k, const void* v, const void* a,
+                             const void* b, const void* w, int ak, int bk, int wk, const float* S0,
+                             void* o, float* ST, int B, int T, int H, int dk, int dv, int dtype,
+                             cudaStream_t st);
+cudaError_t launch_chunk_sm100(const CUtensorMap* maps, const void* alpha, const void* b,
+                               const void* w, int akind, int bkind, int wkind, bool tied,
+                               const float* S0, void* o, float* ST, int* d_status, int B, int T,
+                               int H, int dv, cudaStream_t st);
+}  // namespace gdr
+
+namespace {
+
+PFN_cuTensorMapEncodeTiled_v12000 g_encode = nullptr;
+std::once_flag g_encode_once;
+
+PFN_cuTensorMapEncodeTiled_v12000 encoder() {
+    std::call_once(g_encode_once, [] {
+        void* fn = nullptr;
+        cudaDriverEntryPointQueryResult q;
+        if (cudaGetDriverEntryPoint("cuTensorMapEncodeTiled", &fn, cudaEnableDefault, &q) ==
+                cudaSuccess &&
+            q == cudaDriverEntryPointSuccess)
+            g_encode = reinterpret_cast<PFN_cuTensorMapEncodeTiled_v12000>(fn);
+    });
+    return g_encode;
+}
+
+bool aligned16(const void* p) { return (reinterpret_cast<uintptr_t>(p) & 15u) == 0; }
+
+bool kind_ok(int kind, bool allow_tied) {
+    return kind == GDR_GATE_NONE || kind == GDR_GATE_SCALAR || kind == GDR_GATE_CHANNEL ||
+           (allow_tied && kind == GDR_GATE_TIED);
+}
+
+// Pointer must be NULL exactly when the gate carries no data of its own.
+bool gate_ptr_ok(int kind, const void* p) {
+    bool needs = kind == GDR_GATE_SCALAR || kind == GDR_GATE_CHANNEL;
+    return needs ? p != nullptr : p == nullptr;
+}
+
+// 4-D map over a [B, T, H, d] bf16 tensor, box {64 (d), 1 (H), 64 (T), 1 (B)},
+// 128-byte swizzle, zero fill outside the tensor (masks the last chunk).
+bool make_map(CUtensorMap* m, const void* base, int B, int T, int H, int d) {
+    auto enc = encoder();
+    if (!enc) return false;
+    cuuint64_t dims[4] = {(cuuint64_t)d, (cuuint64_t)H, (cuuint64_t)T, (cuuint64_t)B};
+    cuuint64_t strides[3] = {(cuuint64_t)d * 2, (cuuint64_t)H * d * 2, (cuuint64_t)T * H * d * 2};
+    cuuint32_t box[4] = {64, 1, 64, 1};
+    cuuint32_t estr[4] = {1, 1, 1, 1};
+    CUresult r = enc(m, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 4, const_cast<void*>(base), dims, strides,
+                     box, estr, CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B,
+                     CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
+    return r == CUDA_SUCCESS;
+}
+
+}  // namespace
+
+extern "C" {
+
+const char* gdr_status_string(int s) {
+    switch (s) {
+        case GDR_OK: return "GDR_OK";
+        case GDR_ERR_INVALID_ARG: return "GDR_ERR_INVALID_ARG";
+        case GDR_ERR_UNSUPPORTED: return "GDR_ERR_UNSUPPORTED";
+        case GDR_ERR_MISALIGNED: return "GDR_ERR_MISALIGNED";
+        case GDR_ERR_LAUNCH: return "GDR_ERR_LAUNCH";
+        case GDR_ERR_NO_DEVICE: return "GDR_ERR_NO_DEVICE";
+        default: return "GDR_ERR_UNKNOWN";
+    }
+}
+
+int gdr_version(void) { return (1 << 16) | 0; }
+
+gdr_status gdr_chunk_fwd(const void* q, const void* k, const void* v, const void* alpha,
+                         const void* b, const void* w, int alpha_kind, int b_kind, int w_kind,
+                         const float* S0, void* o, float* S_T, int B, int T, int H, int d_k,
+                         int d_v, int chunk, int dtype, int* d_status, void* stream) {
+    if (B < 1 || H < 1 || T < 0 || d_k < 1 || d_v < 1) return GDR_ERR_INVALID_ARG;
+    if (dtype != GDR_BF16 && dtype != GDR_FP32) return GDR_ERR_INVALID_ARG;
+    if (!kind_ok(alpha_kind, false) || !kind_ok(b_kind, false) || !kind_ok(w_kind, true))
+        return GDR_ERR_INVALID_ARG;
+    if (!gate_ptr_ok(alpha_kind, alpha) || !gate_ptr_ok(b_kind, b) || !gate_ptr_ok(w_kind, w))
+        return GDR_ERR_INVALID_ARG;
+    if (w_kind == GDR_GATE_TIED && b_kind == GDR_GATE_NONE) return GDR_ERR_INVALID_ARG;
+    if (T > 0 && (!q || !k || !v || !o)) return GDR_ERR_INVALID_ARG;
+    if (chunk != 64) return GDR_ERR_UNSUPPORTED;
+    cudaStream_t st = reinterpret_cast<cudaStream_t>(stream);
+    const size_t state_bytes = (size_t)B * H * d_k * d_v * sizeof(float);
+    if (T == 0) {
+        if (!S_T) return GDR_OK;
+        cudaError_t e = S0 ? (S0 == S_T ? cudaSuccess
+                                        : cudaMemcpyAsync(S_T, S0, state_bytes,
+                                                          cudaMemcpyDeviceToDevice, st))
+                           : cudaMemsetAsync(S_T, 0, state_bytes, st);
+        return e == cudaSuccess ? GDR_OK : GDR_ERR_LAUNCH;
+    }
+    const bool tc_path = dtype == GDR_BF16 && d_k == 128 && d_v % 64 == 0;
+    if (!tc_path && (d_k > 128 || d_v > 1024)) return GDR_ERR_UNSUPPORTED;
+    if (!aligned16(q) || !aligned16(k) || !aligned16(v) || !aligned16(o) ||
+        (S0 && !aligned16(S0)) || (S_T && !aligned16(S_T)))
+        return GDR_ERR_MISALIGNED;
+    if ((alpha_kind == GDR_GATE_CHANNEL && !aligned16(alpha)) ||
+        (b_kind == GDR_GATE_CHANNEL && !aligned16(b)) ||
+        (w_kind == GDR_GATE_CHANNEL && !aligned16(w)))
+        return GDR_ERR_MISALIGNED;
+
+    cudaError_t e;
+    if (tc_path) {
+        if (!encoder()) return GDR_ERR_NO_DEVICE;
+        CUtensorMap maps[6];
+        // unused maps point at q so every kernel argument is a valid map
+        const void* amap = alpha_kind == GDR_GATE_CHANNEL ? alpha : q;
+        const void* bmap = b_kind == GDR_GATE_CHANNEL ? b : q;
+        const void* wmap = w_kind == GDR_GATE_CHANNEL ? w : q;
+        if (!make_map(&maps[0], q, B, T, H, d_k) || !make_map(&maps[1], k, B, T, H, d_k) ||
+            !make_map(&maps[2], v, B, T, H, d_v) || !make_map(&maps[3], amap, B, T, H, d_k) ||
+            !make_map(&maps[4], bmap, B, T, H, d_k) || !make_map(&maps[5], wmap, B, T, H, d_k))
+            return GDR_ERR_INVALID_ARG;
+        const bool tied = w_kind == GDR_GATE_TIED && b_kind == GDR_GATE_SCALAR;
+        e = gdr::launch_chunk_sm100(maps, alpha, b, w, alpha_kind, b_kind, w_kind, tied, S0, o, S_T,
+                                    d_status, B, T, H, d_v, st);
+    } else {
+        e = gdr::launch_recurrent(q, k, v, alpha, b, w, alpha_kind, b_kind, w_kind, S0, o, S_T, B,
+                                  T, H, d_k, d_v, dtype, st);
+    }
+    return e == cudaSuccess ? GDR_OK : GDR_ERR_LAUNCH;
+}
+
+gdr_status gdr_decode_step(const void* q, const void* k, const void* v, const void* alpha,
+                           const void* b, const void* w, int alpha_kind, int b_kind, int w_kind,
+                           float* S, void* o, int B, int H, int d_k, int d_v, int dtype,
+                           int* d_status, void* stream) {
+    (void)d_status;  // the decode kernel has no bounded waits
+    if (B < 1 || H < 1 || d_k < 1 || d_v < 1) return GDR_ERR_INVALID_ARG;
+    if (dtype != GDR_BF16 && dtype != GDR_FP32) return GDR_ERR_INVALID_ARG;
+    if (!kind_ok(alpha_kind, false) || !kind_ok(b_kind, false) || !kind_ok(w_kind, true))
+        return GDR_ERR_INVALID_ARG;
+    if (!gate_ptr_ok(alpha_kind, alpha) || !gate_ptr_ok(b_kind, b) || !gate_ptr_ok(w_kind, w))
+        return GDR_ERR_INVALID_ARG;
+    if (w_kind == GDR_GATE_TIED && b_kind == GDR_GATE_NONE) return GDR_ERR_INVALID_ARG;
+    if (!q || !k || !v || !S || !o) return GDR_ERR_INVALID_ARG;
+    if (d_k > 256 || !(d_v == 16 || d_v == 32 || d_v == 64 || d_v == 128 || d_v == 256) ||
+        gdr::decode_rows_per_thread(d_k, d_v) > 32)
+        return GDR_ERR_UNSUPPORTED;
+    if (!aligned16(S) || !aligned16(o) || !aligned16(q) || !aligned16(k) || !aligned16(v))
+        return GDR_ERR_MISALIGNED;
+    cudaError_t e = gdr::launch_decode(q, k, v, alpha, b, w, alpha_kind, b_kind, w_kind, S, o, B * H,
+                                       d_k, d_v, dtype, reinterpret_cast<cudaStream_t>(stream));
+    return e == cudaSuccess ? GDR_OK : GDR_ERR_LAUNCH;
+}
+
+}  // extern "C"

@@ -1,0 +1,148 @@
+/*
+ * gdr.h -- C ABI of the B200 (sm_100a) gated delta-rule library.
+ *
+ * The library runs, per head, the gated delta-rule linear-attention recurrence
+ *
+ *   S_t = (I - k_t^T (b_t . k_t)) Diag(alpha_t) S_{t-1} + (w_t . k_t)^T v_t
+ *   o_t = q_t S_t
+ *
+ * with row vectors q_t, k_t, alpha_t, b_t, w_t of length d_k, v_t and o_t of
+ * length d_v, "." the elementwise product, and a d_k x d_v state S kept in
+ * fp32. Sources for the operation:
+ *   - write S <- S + k^T v and read o = q S, row vectors:
+ *     "Recurrent Memory: Write, Erase, Decay, Read", section 01;
+ *   - erase (delta rule, I - beta k^T k): same page, section 03, and
+ *     "The Eraser Trilogy", "Eraser two";
+ *   - decay Diag(alpha), scalar (Gated DeltaNet) or per channel (KDA), and the
+ *     unified equation: same page, sections 04-05; "The Eraser Trilogy",
+ *     "Eraser three";
+ *   - channel-wise erase gate b and write gate w, collapsing to one scalar
+ *     beta for KDA and Gated DeltaNet, decay absorbed into the erase factor:
+ *     "Erase-then-Delta Attention" (Gated DeltaNet-2), abstract;
+ *   - chunkwise-parallel evaluation: "Recurrent Memory", sections 03-04
+ *     (reassociation into chunks; decay as a prefix sum of logs), and the
+ *     chunkwise WY algorithm named in the Gated DeltaNet-2 abstract.
+ *
+ * Conventions shared by every entry point
+ * ---------------------------------------
+ * Pointers: every array argument is a DEVICE pointer (memory the CUDA device
+ *   can read/write). The caller owns every buffer; the library allocates no
+ *   memory, keeps no state between calls and never frees caller memory.
+ * Layouts (contiguous, row-major, innermost last):
+ *   q, k        [B, T, H, d_k]       chunk forward;  [B, H, d_k] decode
+ *   v, o        [B, T, H, d_v]                       [B, H, d_v]
+ *   scalar gate [B, T, H]                            [B, H]
+ *   channel gate[B, T, H, d_k]                       [B, H, d_k]
+ *   S0, S_T, S  [B, H, d_k, d_v] fp32
+ * Element type: q, k, v, o and the gates all have type `dtype`
+ *   (GDR_BF16 = bfloat16, GDR_FP32 = float). The state is always fp32 and
+ *   all arithmetic accumulates in fp32.
+ * Gates: alpha (decay) must lie in (0, 1]; b (erase) and w (write) are
+ *   meant to lie in [0, 1] (not enforced). Kinds:
+ *   GDR_GATE_NONE     the pointer must be NULL; alpha = 1, b = 0, w = 1.
+ *   GDR_GATE_SCALAR   one value per token-head, used for every channel.
+ *   GDR_GATE_CHANNEL  one value per token-head and key channel.
+ *   GDR_GATE_TIED     w only: w := b (same values, pointer must be NULL);
+ *                     b = w = beta is the KDA / Gated DeltaNet form.
+ * Streams: `stream` is a cudaStream_t (NULL = the legacy default stream).
+ *   Calls are asynchronous: GDR_OK means the work was launched. Faults
+ *   surface at the caller's next synchronisation.
+ * Device status: `d_status`, if not NULL, is a device int the kernels OR
+ *   GDR_DEVICE_* flags into (the caller zeroes it). Kernels never trap: every
+ *   wait on the tensor-memory / TMA pipeline is bounded and, on expiry, sets
+ *   GDR_DEVICE_TIMEOUT and ends the block cleanly.
+ * Errors: argument problems are detected on the host before any launch and
+ *   returned as gdr_status; nothing is launched in that case.
+ */
+#ifndef GDR_H
+#define GDR_H
+
+#ifdef __cplusplus
+extern "C" {
+#endif
+
+typedef enum {
+    GDR_OK = 0,
+    GDR_ERR_INVALID_ARG = 1,   /* bad size, NULL where data is required, bad enum */
+    GDR_ERR_UNSUPPORTED = 2,   /* valid request this build does not implement */
+    GDR_ERR_MISALIGNED = 3,    /* a pointer is not 16-byte aligned */
+    GDR_ERR_LAUNCH = 4,        /* the CUDA launch itself failed */
+    GDR_ERR_NO_DEVICE = 5      /* no usable CUDA device / driver entry point */
+} gdr_status;
+
+/* Flags ORed into *d_status by the kernels. */
+#define GDR_DEVICE_TIMEOUT 1       /* a bounded pipeline wait expired; results invalid */
+#define GDR_DEVICE_DECAY_RANGE 2   /* chunk decay span outside the tensor-core path's range */
+
+typedef enum { GDR_BF16 = 0, GDR_FP32 = 1 } gdr_dtype;
+
+typedef enum {
+    GDR_GATE_NONE = 0,
+    GDR_GATE_SCALAR = 1,
+    GDR_GATE_CHANNEL = 2,
+    GDR_GATE_TIED = 3
+} gdr_gate_kind;
+
+/*
+ * gdr_chunk_fwd -- forward pass over whole sequences (prefill / training
+ * forward), evaluated chunk by chunk.
+ *
+ * Computes o_t for t = 0..T-1 of every (b, h) head, starting from S0 (or a
+ * zero state when S0 is NULL), and writes the final state S_T when S_T is not
+ * NULL. S_T may alias S0 (S0 is read once, before any write). o must not
+ * alias any input.
+ *
+ * chunk: the chunk length of the chunkwise evaluation; 64 is the supported
+ * value. The result does not depend on it beyond rounding.
+ * Paths: dtype GDR_BF16 with d_k = 128 and d_v a multiple of 64 runs the
+ * tcgen05 tensor-core chunk kernel (bf16 operands, fp32 accumulation, fp32
+ * state on chip). Its decay range: within every chunk and channel the
+ * summed -log(alpha) over the chunk's tokens after the first must not exceed
+ * 160 (outside it the kernel sets GDR_DEVICE_DECAY_RANGE). Every other
+ * supported shape (fp32, or 1 <= d_k, d_v <= 128 otherwise) runs an exact
+ * fp32 token-by-token CUDA kernel.
+ * Alignment: q, k, v, o and channel gates must be 16-byte aligned and, on
+ * the tensor-core path, d_k and d_v rows 16-byte multiples (given by the
+ * shape rules above).
+ * Returns GDR_OK, GDR_ERR_INVALID_ARG (B, H < 1, T < 0, bad kinds, NULL
+ * data), GDR_ERR_UNSUPPORTED (chunk != 64, shape beyond the limits above),
+ * GDR_ERR_MISALIGNED, GDR_ERR_LAUNCH or GDR_ERR_NO_DEVICE. T = 0 writes S_T
+ * := S0 (or zeros) and launches nothing else.
+ */
+gdr_status gdr_chunk_fwd(const void* q, const void* k, const void* v,
+                         const void* alpha, const void* b, const void* w,
+                         int alpha_kind, int b_kind, int w_kind,
+                         const float* S0, void* o, float* S_T,
+                         int B, int T, int H, int d_k, int d_v, int chunk,
+                         int dtype, int* d_status, void* stream);
+
+/*
+ * gdr_decode_step -- one token per head (autoregressive decoding).
+ *
+ * Applies one step of the recurrence to every (b, h) head: S is read and
+ * overwritten in place with S_new, and o = q S_new is written. One pass over
+ * S: the two column reductions (b.k.alpha) S and (q.alpha) S are taken while
+ * S is read, and S_new is written from registers.
+ * q, k [B, H, d_k]; v, o [B, H, d_v]; gates [B, H] or [B, H, d_k];
+ * S [B, H, d_k, d_v] fp32. o must not alias S or the inputs.
+ * Supported: 1 <= d_k <= 256, d_v a multiple of 4 with 4 <= d_v <= 256.
+ * Alignment: S, o, q, k, v and channel gates must be 16-byte aligned.
+ * Returns as gdr_chunk_fwd.
+ */
+gdr_status gdr_decode_step(const void* q, const void* k, const void* v,
+                           const void* alpha, const void* b, const void* w,
+                           int alpha_kind, int b_kind, int w_kind,
+                           float* S, void* o, int B, int H, int d_k, int d_v,
+                           int dtype, int* d_status, void* stream);
+
+/* Human-readable name of a gdr_status value (static storage, never NULL). */
+const char* gdr_status_string(int status);
+
+/* Library ABI version: (major << 16) | minor. */
+int gdr_version(void);
+
+#ifdef __cplusplus
+}
+#endif
+
+#endif /* GDR_H */

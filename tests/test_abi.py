@@ -1,0 +1,103 @@
+"""The C ABI without a GPU: the library loads, exports what include/gdr.h
+declares, and rejects bad arguments on the host before any launch."""
+import ctypes
+import os
+import re
+
+import pytest
+
+from gated_delta_rule_147_b200 import _lib
+
+ROOT = os.path.dirname(os.path.dirname(os.path.abspath(__file__)))
+HEADER = os.path.join(ROOT, "include", "gdr.h")
+
+# fake, 16-byte aligned device addresses: validation fails before they are used
+P = 1 << 20
+NULL = None
+
+
+def declared_functions():
+    src = open(HEADER).read()
+    src = re.sub(r"/\*.*?\*/", "", src, flags=re.S)
+    return sorted(set(re.findall(r"^\s*(?:gdr_status|const char\*|int)\s+(gdr_\w+)\s*\(", src, flags=re.M)))
+
+
+def test_header_declares_the_entry_points():
+    assert declared_functions() == sorted(_lib.EXPORTS)
+
+
+def test_library_loads_and_exports_every_declared_symbol():
+    lib = _lib.load()
+    for name in declared_functions():
+        assert hasattr(lib, name), name
+    assert lib.gdr_version() == (1 << 16)
+    assert _lib.status_string(0) == "GDR_OK"
+    assert _lib.status_string(3) == "GDR_ERR_MISALIGNED"
+
+
+def test_library_is_in_tree():
+    assert os.path.dirname(_lib.library_path()) == os.path.join(ROOT, "gated_delta_rule_147_b200")
+
+
+def chunk(**kw):
+    a = dict(q=P, k=P, v=P, alpha=P, b=P, w=NULL, ak=1, bk=1, wk=3, S0=NULL, o=P, ST=P, B=1, T=64,
+             H=1, dk=128, dv=128, chunk=64, dtype=0)
+    a.update(kw)
+    lib = _lib.load()
+    return lib.gdr_chunk_fwd(a["q"], a["k"], a["v"], a["alpha"], a["b"], a["w"], a["ak"], a["bk"],
+                             a["wk"], a["S0"], a["o"], a["ST"], a["B"], a["T"], a["H"], a["dk"],
+                             a["dv"], a["chunk"], a["dtype"], None, None)
+
+
+@pytest.mark.parametrize("kw,expect", [
+    (dict(B=0), _lib.GDR_ERR_INVALID_ARG),
+    (dict(H=0), _lib.GDR_ERR_INVALID_ARG),
+    (dict(T=-1), _lib.GDR_ERR_INVALID_ARG),
+    (dict(dk=0), _lib.GDR_ERR_INVALID_ARG),
+    (dict(dtype=7), _lib.GDR_ERR_INVALID_ARG),
+    (dict(ak=9), _lib.GDR_ERR_INVALID_ARG),
+    (dict(ak=3), _lib.GDR_ERR_INVALID_ARG),             # alpha cannot be tied
+    (dict(alpha=NULL), _lib.GDR_ERR_INVALID_ARG),        # scalar alpha needs data
+    (dict(ak=0), _lib.GDR_ERR_INVALID_ARG),              # NONE alpha must be NULL
+    (dict(w=P), _lib.GDR_ERR_INVALID_ARG),               # tied w must be NULL
+    (dict(bk=0, b=NULL), _lib.GDR_ERR_INVALID_ARG),      # tied to an absent b
+    (dict(q=NULL), _lib.GDR_ERR_INVALID_ARG),
+    (dict(o=NULL), _lib.GDR_ERR_INVALID_ARG),
+    (dict(chunk=32), _lib.GDR_ERR_UNSUPPORTED),
+    (dict(dtype=1, dk=256), _lib.GDR_ERR_UNSUPPORTED),
+    (dict(q=P + 8), _lib.GDR_ERR_MISALIGNED),
+    (dict(o=P + 2), _lib.GDR_ERR_MISALIGNED),
+    (dict(ST=P + 4), _lib.GDR_ERR_MISALIGNED),
+    (dict(ak=2, alpha=P + 2), _lib.GDR_ERR_MISALIGNED),
+])
+def test_chunk_fwd_rejects_bad_arguments(kw, expect):
+    assert chunk(**kw) == expect
+
+
+def decode(**kw):
+    a = dict(q=P, k=P, v=P, alpha=P, b=P, w=P, ak=2, bk=2, wk=2, S=P, o=P, B=2, H=2, dk=128, dv=128,
+             dtype=0)
+    a.update(kw)
+    return _lib.load().gdr_decode_step(a["q"], a["k"], a["v"], a["alpha"], a["b"], a["w"], a["ak"],
+                                       a["bk"], a["wk"], a["S"], a["o"], a["B"], a["H"], a["dk"],
+                                       a["dv"], a["dtype"], None, None)
+
+
+@pytest.mark.parametrize("kw,expect", [
+    (dict(B=0), _lib.GDR_ERR_INVALID_ARG),
+    (dict(S=NULL), _lib.GDR_ERR_INVALID_ARG),
+    (dict(wk=3), _lib.GDR_ERR_INVALID_ARG),              # tied w must be NULL
+    (dict(bk=5), _lib.GDR_ERR_INVALID_ARG),
+    (dict(dv=48), _lib.GDR_ERR_UNSUPPORTED),
+    (dict(dk=512), _lib.GDR_ERR_UNSUPPORTED),
+    (dict(dv=256, dk=256), _lib.GDR_ERR_UNSUPPORTED),     # too many state rows per thread
+    (dict(S=P + 4), _lib.GDR_ERR_MISALIGNED),
+])
+def test_decode_step_rejects_bad_arguments(kw, expect):
+    assert decode(**kw) == expect
+
+
+def test_binding_raises_on_error_status():
+    with pytest.raises(_lib.GdrError):
+        _lib.gdr_chunk_fwd(P, P, P, P, P, None, 1, 1, 3, None, P, P, 0, 64, 1, 128, 128, 64, 0,
+                           stream=0)

@@ -1,0 +1,157 @@
+"""GPU parity of gdr_chunk_fwd against the fp64 oracle.
+
+Tolerances (max-abs error relative to max|ref|, for o and for S_T): 2e-2 for
+bf16 inputs with fp32 accumulation, 1e-4 for fp32 inputs.
+"""
+import numpy as np
+import pytest
+import torch
+
+from gated_delta_rule_147_b200 import GDR_DEVICE_DECAY_RANGE, chunk_fwd
+from gated_delta_rule_147_b200.inputs import WORKLOADS, make_chunk_inputs
+from gpu_util import TOL, assert_close, gather_heads, run_chunk, run_oracle
+
+pytestmark = pytest.mark.gpu
+
+FAMILIES = ["gdn", "kda", "gdn2"]
+
+
+def small(family, **kw):
+    base = dict(B=2, H=3, T=200)
+    base.update(kw)
+    return WORKLOADS[family].with_(**base)
+
+
+@pytest.mark.parametrize("family", FAMILIES)
+@pytest.mark.parametrize("T", [1, 64, 65, 200])
+def test_small_ragged(cuda_device, family, T):
+    """Several chunks and a ragged tail, two 64-column slices of d_v."""
+    wl = small(family, T=T, s0=True, seed=100 + T)
+    inp = make_chunk_inputs(wl)
+    o, ST = run_chunk(inp, cuda_device)
+    o_ref, ST_ref = run_oracle(inp)
+    assert_close(o, o_ref, TOL["bf16"], "o")
+    assert_close(ST, ST_ref, TOL["bf16"], "S_T")
+
+
+@pytest.mark.parametrize("family", FAMILIES)
+def test_slow_decay_carries_state_across_chunks(cuda_device, family):
+    """alpha close to 1: the state survives many chunks, so inter-chunk
+    propagation (and its bf16 operand rounding) is exercised."""
+    wl = small(family, T=640, H=2, s0=True, seed=7)
+    inp = make_chunk_inputs(wl)
+    inp["alpha"] = (inp["alpha"].float() ** 0.02).to(inp["alpha"].dtype)
+    o, ST = run_chunk(inp, cuda_device)
+    o_ref, ST_ref = run_oracle(inp)
+    assert_close(o, o_ref, TOL["bf16"], "o")
+    assert_close(ST, ST_ref, TOL["bf16"], "S_T")
+
+
+@pytest.mark.parametrize("gates", [
+    {"alpha": "none", "b": "none", "w": "none"},          # linear attention
+    {"alpha": "scalar", "b": "none", "w": "channel"},     # gated linear attention (no erase)
+    {"alpha": "none", "b": "scalar", "w": "tied"},        # DeltaNet
+    {"alpha": "channel", "b": "channel", "w": "tied"},    # channel b with w := b
+    {"alpha": "scalar", "b": "scalar", "w": "scalar"},    # untied scalar gates
+])
+def test_gate_forms(cuda_device, gates):
+    wl = small("gdn2", T=150, alpha=gates["alpha"], b=gates["b"], w=gates["w"], s0=True, seed=3)
+    inp = make_chunk_inputs(wl)
+    o, ST = run_chunk(inp, cuda_device)
+    o_ref, ST_ref = run_oracle(inp)
+    assert_close(o, o_ref, TOL["bf16"], "o")
+    assert_close(ST, ST_ref, TOL["bf16"], "S_T")
+
+
+def test_tiny_fp32(cuda_device):
+    """B=1,H=1,T=64,d=16 fp32, channel alpha, independent b,w ~ U(0,1)."""
+    inp = make_chunk_inputs(WORKLOADS["tiny"])
+    o, ST = run_chunk(inp, cuda_device)
+    o_ref, ST_ref = run_oracle(inp)
+    assert_close(o, o_ref, TOL["fp32"], "o")
+    assert_close(ST, ST_ref, TOL["fp32"], "S_T")
+
+
+@pytest.mark.parametrize("family", FAMILIES)
+def test_fp32_path_d128(cuda_device, family):
+    wl = small(family, T=97, dtype="fp32", s0=True, seed=5)
+    inp = make_chunk_inputs(wl)
+    o, ST = run_chunk(inp, cuda_device)
+    o_ref, ST_ref = run_oracle(inp)
+    assert_close(o, o_ref, TOL["fp32"], "o")
+    assert_close(ST, ST_ref, TOL["fp32"], "S_T")
+
+
+def test_bf16_other_shapes_use_exact_path(cuda_device):
+    wl = small("kda", T=70, dk=64, dv=48, s0=True, seed=9)
+    inp = make_chunk_inputs(wl)
+    o, ST = run_chunk(inp, cuda_device)
+    o_ref, ST_ref = run_oracle(inp)
+    assert_close(o, o_ref, TOL["bf16"], "o")
+    assert_close(ST, ST_ref, TOL["bf16"], "S_T")
+
+
+def test_split_sequence_resumes(cuda_device):
+    """Two calls with S0 := S_T of the first equal one call."""
+    wl = small("gdn2", T=256, s0=True, seed=11)
+    inp = make_chunk_inputs(wl)
+    dev = cuda_device
+    o_full, ST_full = run_chunk(inp, dev)
+    first = {k: (v[:, :128] if hasattr(v, "dim") and k not in ("S0",) else v) for k, v in inp.items()}
+    second = {k: (v[:, 128:] if hasattr(v, "dim") and k not in ("S0",) else v) for k, v in inp.items()}
+    o1, S1 = run_chunk(first, dev)
+    second["S0"] = torch.from_numpy(S1)
+    o2, S2 = run_chunk(second, dev)
+    assert_close(np.concatenate([o1, o2], axis=1), o_full, 1e-2, "o (split)")
+    assert_close(S2, ST_full, 1e-2, "S_T (split)")
+
+
+def test_zero_length_copies_initial_state(cuda_device):
+    wl = small("kda", T=0, s0=True)
+    inp = make_chunk_inputs(wl)
+    o, ST = run_chunk(inp, cuda_device)
+    assert o.shape == (2, 0, 3, 128)
+    np.testing.assert_array_equal(ST, inp["S0"].numpy())
+
+
+def test_final_state_in_place(cuda_device):
+    """S_T may alias S0."""
+    wl = small("kda", T=130, s0=True, seed=12)
+    inp = make_chunk_inputs(wl)
+    dev = cuda_device
+    S = inp["S0"].to(dev).clone()
+    q, k, v = (inp[x].to(dev) for x in ("q", "k", "v"))
+    o, ST = chunk_fwd(q, k, v, inp["alpha"].to(dev), inp["b"].to(dev), "tied", S, S_T=S)
+    torch.cuda.synchronize()
+    o_ref, ST_ref = run_oracle(inp)
+    assert_close(S.cpu().numpy(), ST_ref, TOL["bf16"], "S_T in place")
+
+
+def test_decay_range_flag(cuda_device):
+    """A chunk whose decay span exceeds the tensor-core path's range is
+    reported through d_status; in-range inputs leave it zero."""
+    wl = small("kda", T=64, H=1, B=1, seed=13)
+    inp = make_chunk_inputs(wl)
+    st = torch.zeros(1, dtype=torch.int32, device=cuda_device)
+    run_chunk(inp, cuda_device, d_status=st)
+    assert int(st.item()) == 0
+    inp["alpha"] = torch.full_like(inp["alpha"], 0.01)   # 63 x 4.6 nats > 160
+    run_chunk(inp, cuda_device, d_status=st)
+    assert int(st.item()) & GDR_DEVICE_DECAY_RANGE
+
+
+@pytest.mark.parametrize("family", FAMILIES)
+def test_full_size_sampled_heads(cuda_device, family):
+    """The full workload in the launch configuration the benchmark times;
+    the oracle checks a seeded sample of heads over the whole sequence."""
+    wl = WORKLOADS[family]
+    inp = make_chunk_inputs(wl)
+    o, ST = run_chunk(inp, cuda_device)
+    rng = np.random.default_rng(2024)
+    nh = 3 if family == "gdn2" else 4
+    heads = sorted({(int(rng.integers(wl.B)), int(rng.integers(wl.H))) for _ in range(nh)})
+    o_ref, ST_ref = run_oracle(inp, heads)
+    o_s, ST_s = gather_heads(o, ST, heads)
+    assert_close(o_s, o_ref, TOL["bf16"], f"o {heads}")
+    assert_close(ST_s, ST_ref, TOL["bf16"], f"S_T {heads}")
+    assert np.all(np.isfinite(o))
