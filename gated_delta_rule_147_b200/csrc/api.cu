@@ -93,7 +93,9 @@ gdr_status gdr_chunk_fwd(const void* q, const void* k, const void* v, const void
     if (dtype != GDR_BF16 && dtype != GDR_FP32) return GDR_ERR_INVALID_ARG;
     if (!kind_ok(alpha_kind, false) || !kind_ok(b_kind, false) || !kind_ok(w_kind, true))
         return GDR_ERR_INVALID_ARG;
-    if (!gate_ptr_ok(alpha_kind, alpha) || !gate_ptr_ok(b_kind, b) || !gate_ptr_ok(w_kind, w))
+    // with T = 0 there are no token arrays (zero-length buffers may be NULL)
+    if (T > 0 && (!gate_ptr_ok(alpha_kind, alpha) || !gate_ptr_ok(b_kind, b) ||
+                  !gate_ptr_ok(w_kind, w)))
         return GDR_ERR_INVALID_ARG;
     if (w_kind == GDR_GATE_TIED && b_kind == GDR_GATE_NONE) return GDR_ERR_INVALID_ARG;
     if (T > 0 && (!q || !k || !v || !o)) return GDR_ERR_INVALID_ARG;
