@@ -5,30 +5,34 @@
 // reassociation into chunks and the prefix sum of log decays; "Erase-then-
 // Delta Attention" abstract for the chunkwise WY form with the decay absorbed
 // into the erase factors):
-//   l_r   = sum_{j<=r} log2 alpha_j (per channel), g_r = 2^l_r
-//   ref   = (l_0 + l_{n-1}) / 2 per channel; rowf_r = 2^(l_r - ref),
-//           colf_r = 2^(ref - l_r) (so rowf_r colf_j = g_r / g_j, both bounded)
-//   A  = strict_lower[(b.k.rowf)(k.colf)^T]     Bm = strict_lower[(b.k.rowf)(w.k.colf)^T]
-//   Aq = lower[(q.rowf)(k.colf)^T]              Bq = lower[(q.rowf)(w.k.colf)^T]
-//   T  = (I + A)^-1                               (unit lower triangular solve)
-//   E_top = T [b.k.g | Bm],  E_bot = [q.g | Bq] - Aq E_top
-//   [-U ; O] = [E_top ; E_bot] [S ; V]            (O is the chunk's output)
-//   S_new = Diag(g_{n-1}) S + Diag(2^(l_{n-1}-ref)) [(k.colf)^T U + (w.k.colf)^T V]
-// With tied scalar gates b = w = beta, Bm = A Diag(beta) and the V columns
-// simplify to E = [ [T b.k.g, -T Diag(beta)] ; [q.g - Aq T b.k.g, Aq T Diag(beta)] ],
-// U becomes U + Diag(beta) V and the state update needs only (k.colf)^T U.
+//   l_r   = sum_{j<=r} log2 alpha_j (per channel),   g_r = 2^l_r
+//   ref   = (l_0 + l_{n-1}) / 2 per channel,  rowf_r = 2^(l_r - ref),
+//           colf_r = 2^(ref - l_r)  (rowf_r colf_j = g_r / g_j; both bounded)
+//   Kb = b.k.rowf, Qs = q.rowf, Ks = k.colf, Kws = w.k.colf
+//   A  = strict_lower(Kb Ks^T)   Bm = strict_lower(Kb Kws^T)
+//   Aq = lower(Qs Ks^T)          Bq = lower(Qs Kws^T)
+//   T  = (I + A)^-1                                  (unit lower triangular)
+//   W  = T Kb . 2^ref            (the rows of b.k.g, mapped through T)
+//   U  = -W S - T Bm V                               (per-chunk "new values")
+//   O  = (Qs . 2^ref) S + Aq U + Bq V                (the chunk's outputs)
+//   S' = Diag(g_{n-1}) S + Diag(2^(l_{n-1}-ref)) (Ks^T U + Kws^T V)
+// With tied scalar gates b = w = beta: Bm = A Diag(beta), Bq = Aq Diag(beta),
+// U + Diag(beta) V = T Diag(beta) V - W S, and only Ks^T (U + beta V) enters S'.
 //
-// One CTA (128 threads) owns one (batch, head, 64-column slice of d_v) and
-// walks the chunks in order; the state slice stays on chip (fp32 registers,
-// a bf16 copy in shared memory as the MMA operand). Per chunk five tcgen05
-// MMAs run with fp32 accumulators in tensor memory:
-//   P1  D1 = [b.k.rowf ; q.rowf] x [k.colf ; w.k.colf]^T        (A, Aq, Bm, Bq)
-//   P2  D2 = [[T,0],[0,I]] x [ [b.k.g ; q.g] | X ]               (E_top, copy of bottom)
-//   P3  D2 += [0 ; -Aq] x E_top                                  (E_bot)
-//   S1  D3 = E x [S ; V]                                         (-U, O)
-//   S2  D4 = [k.colf ; w.k.colf]^T x [U ; V]                     (state increment)
+// One CTA (256 threads, two warpgroups that split every phase) owns one
+// (batch, head, 64-column slice of d_v) and walks the chunks in order; its
+// state slice stays on chip (fp32 registers: one row and half the columns per
+// thread; a bf16 copy in shared memory as an MMA operand). Per chunk the tcgen05
+// MMAs (fp32 accumulators in tensor memory) are:
+//   P1  D1  = [Kb ; Qs] x [Ks ; Kws]^T                   -> A, Aq (Bm, Bq)
+//   P2  D2  = [T ; 0] x [Kb | Bm]                         -> W (and T Bm)
+//   P3  D3  = [T Diag(beta) ; 0] x V   or   [-T Bm ; Bq] x V    (pre-load)
+//   S1  D3 += [-W ; Qs.2^ref] x S                         -> U, O partial
+//   S2  D3 += [0 ; Aq] x U   and   D4 = [Ks ; Kws]^T x [U ; V]
 // q, k, v and channel gates arrive by TMA (128-byte swizzle) straight into
-// the operand layout the MMAs read.
+// the operand layout the MMAs read. The unit lower triangular solve runs on
+// CUDA cores in fp32 (16 x 16 diagonal blocks by forward substitution, then
+// recursive halving: 16 -> 32 -> 64).
 #include "common.cuh"
 
 namespace gdr {
@@ -37,34 +41,51 @@ namespace chunk {
 constexpr int C = 64;     // chunk length
 constexpr int DK = 128;   // key dimension handled by this kernel
 constexpr int NV = 64;    // value columns per CTA
-constexpr int NT = 128;   // threads per CTA
+constexpr int NT = 256;   // threads per CTA (two warpgroups)
 
 // Shared memory map (bytes from a 1024-aligned base).
-constexpr uint32_t OFF_QIN = 0;        // q chunk   [64 x 128] bf16, 2 column blocks of 8 KB
+constexpr uint32_t OFF_QIN = 0;        // q chunk [64 x 128] bf16: 2 column blocks of 8 KB
 constexpr uint32_t OFF_KIN = 16384;    // k chunk
 constexpr uint32_t OFF_GA = 32768;     // channel alpha chunk
 constexpr uint32_t OFF_GB = 49152;     // channel b chunk
 constexpr uint32_t OFF_GW = 65536;     // channel w chunk
-//   after the operands are built the input region is reused:
-constexpr uint32_t OFF_A32 = 0;        // A fp32 [64 x 64] (float4-swizzled rows)
+//   reused once the operands are built:
+constexpr uint32_t OFF_A32 = 0;        // A fp32 [64 x 64] (float4 groups swizzled by row)
 constexpr uint32_t OFF_T32 = 16384;    // T fp32 [64 x 64]
-constexpr uint32_t OFF_AP = 32768;     // [0 ; -Aq] bf16 [128 x 64]
-constexpr uint32_t OFF_L = 49152;      // [[T,0],[0,I]] bf16 [128 x 128]
-constexpr uint32_t OFF_V = 81920;      // v slice [64 x 64] bf16, two buffers of 8 KB
-constexpr uint32_t OFF_ROP = 98304;    // [b.k.rowf ; q.rowf] bf16 [128 x 128]
-constexpr uint32_t OFF_X = 131072;     // [Bm ; Bq] or [-Diag(beta) ; 0] bf16 [128 x 64]
-constexpr uint32_t OFF_E = 98304;      // E bf16 [128 x 192] (over ROP and X, after P2)
-constexpr uint32_t OFF_P32 = 98304;    // solve scratch fp32 3 x [16 x 16] (over ROP, after P1)
-constexpr uint32_t OFF_SCAN = 131072;  // scan scratch fp32 (over X, during the build)
-constexpr uint32_t OFF_RG = 147456;    // [b.k.g ; q.g] bf16 [128 x 128]
-constexpr uint32_t OFF_U = 147456;     // U bf16 [64 x 64] (over RG, after P2)
-constexpr uint32_t OFF_COP = 180224;   // [k.colf ; w.k.colf] bf16 [64 or 128 x 128]
-constexpr uint32_t OFF_SBF = 212992;   // S bf16 [128 x 64]
-constexpr uint32_t OFF_SMALL = 229376; // per-token scalars, per-channel factors, barriers
-constexpr uint32_t SMEM_BYTES = 229376 + 2048 + 1024;  // + small area + alignment slack
+constexpr uint32_t OFF_X = 32768;      // Bm bf16 [64 x 64] (general gates)
+constexpr uint32_t OFF_P32 = 40960;    // solve scratch fp32 3 x [16 x 16]
+constexpr uint32_t OFF_L = 49152;      // [T ; 0] bf16 [128 x 64]
+constexpr uint32_t OFF_V = 81920;      // v slice [64 x 64] bf16, two buffers
+constexpr uint32_t OFF_ROP = 98304;    // [Kb ; Qs] bf16 [128 x 128], later [-W ; Qs.2^ref]
+constexpr uint32_t OFF_COP = 131072;   // [Ks ; Kws] bf16 [64 or 128 x 128]
+constexpr uint32_t OFF_APRE = 163840;  // [T Diag(beta) ; 0] or [-T Bm ; Bq] bf16 [128 x 64]
+constexpr uint32_t OFF_AQ = 180224;    // [0 ; Aq] bf16 [128 x 64]
+constexpr uint32_t OFF_SBF = 196608;   // S bf16 [128 x 64]
+constexpr uint32_t OFF_U = 212992;     // U bf16 [64 x 64]
+constexpr uint32_t OFF_SCAN = 212992;  // scan scratch fp32 [17 x 128] (over U, during the build)
+constexpr uint32_t OFF_SMALL = 225792; // per-token / per-channel scalars, barriers
+constexpr uint32_t SMALL_BYTES = 4096;
+constexpr uint32_t SMEM_BYTES = OFF_SMALL + SMALL_BYTES + 1024;  // + alignment slack
 
 // TMEM columns
-constexpr uint32_t TM_D1 = 0, TM_D2 = 0, TM_D3 = 192, TM_D4 = 256, TM_COLS = 512;
+constexpr uint32_t TM_D1 = 0, TM_D2 = 128, TM_D3 = 320, TM_D4 = 384, TM_COLS = 512;
+
+// Optional phase tracing (build with -DGDR_TRACE_PHASES): thread 0 of the
+// first CTA stamps clock64() at each phase boundary of its first 64 chunks;
+// gdr_trace_read() copies the stamps out. Compiled out by default.
+#ifdef GDR_TRACE_PHASES
+__device__ unsigned long long g_trace[64 * 16];
+#define GDR_TRACE(k)                                                                          \
+    do {                                                                                     \
+        if (blockIdx.x == 0 && blockIdx.y == 0 && blockIdx.z == 0 && threadIdx.x == 0 &&   \
+            ci < 64)                                                                         \
+            g_trace[ci * 16 + (k)] = clock64();                                              \
+    } while (0)
+#else
+#define GDR_TRACE(k) \
+    do {            \
+    } while (0)
+#endif
 
 struct Params {
     const void* alpha;  // scalar gates are read with plain loads
@@ -78,10 +99,6 @@ struct Params {
     int akind, bkind, wkind;
 };
 
-__device__ __forceinline__ float ld_bf16_smem(const uint8_t* base, uint32_t off) {
-    return __bfloat162float(*reinterpret_cast<const __nv_bfloat16*>(base + off));
-}
-
 // fp32 [64 x 64] scratch with rows of 16 float4 groups XOR-swizzled by row.
 __device__ __forceinline__ float* f32_at(float* base, int r, int c) {
     return base + r * 64 + ((((c >> 2) ^ (r & 15))) << 2) + (c & 3);
@@ -94,6 +111,10 @@ __device__ __forceinline__ void st_chunk(uint8_t* base, uint32_t off, const floa
     u.z = pack_bf16x2(x8[4], x8[5]);
     u.w = pack_bf16x2(x8[6], x8[7]);
     *reinterpret_cast<uint4*>(base + off) = u;
+}
+
+__device__ __forceinline__ void st_zero_chunk(uint8_t* base, uint32_t off) {
+    *reinterpret_cast<uint4*>(base + off) = make_uint4(0u, 0u, 0u, 0u);
 }
 
 __device__ __forceinline__ void ld_chunk(const uint8_t* base, uint32_t off, float* x8) {
@@ -116,30 +137,33 @@ __global__ void __launch_bounds__(NT, 1) chunk_fwd_kernel(
     extern __shared__ uint8_t smem_raw[];
     uint8_t* sm = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) &
                                              ~uintptr_t(1023));
-    const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
+    const int tid = threadIdx.x, warp = tid >> 5;
+    const int wg = warp >> 2;          // warpgroup: which half of the columns it handles
+    const int row = tid & 127;         // TMEM lane this thread reads (warp % 4 selects the quarter)
     const int vt = blockIdx.x, h = blockIdx.y, bb = blockIdx.z;
     const int v0 = vt * NV;
     const int T = p.T, H = p.H;
     const int nchunks = (T + C - 1) / C;
     const bool ach = p.akind == GDR_GATE_CHANNEL, bch = p.bkind == GDR_GATE_CHANNEL,
                wch = p.wkind == GDR_GATE_CHANNEL;
-    constexpr int N1 = TIED ? 64 : 128;  // rows of [k.colf ; w.k.colf]
+    constexpr int N1 = TIED ? 64 : 128;  // rows of [Ks ; Kws]
 
-    float* s_ascal = reinterpret_cast<float*>(sm + OFF_SMALL);          // [64] scalar alpha
-    float* s_bscal = s_ascal + 64;                                       // [64] scalar b
-    float* s_wscal = s_ascal + 128;                                      // [64] scalar w
-    float* s_gC = s_ascal + 192;                                         // [128] g_{n-1}
-    float* s_fS = s_ascal + 320;                                         // [128] 2^(l_{n-1}-ref)
-    uint64_t* bar_tma = reinterpret_cast<uint64_t*>(sm + OFF_SMALL + 1920);
+    float* s_ascal = reinterpret_cast<float*>(sm + OFF_SMALL);  // [64] scalar alpha
+    float* s_bscal = s_ascal + 64;                              // [64] scalar b
+    float* s_wscal = s_ascal + 128;                             // [64] scalar w
+    float* s_rowf = s_ascal + 192;                              // [64] scalar-decay rowf
+    float* s_colf = s_ascal + 256;                              // [64] scalar-decay colf
+    float* s_eref = s_ascal + 320;                              // [128] 2^ref
+    float* s_gC = s_ascal + 448;                                // [128] g_{n-1}
+    float* s_fS = s_ascal + 576;                                // [128] 2^(l_{n-1}-ref)
+    uint64_t* bar_tma = reinterpret_cast<uint64_t*>(sm + OFF_SMALL + 3072);
     uint64_t* bar_mma = bar_tma + 1;
-    uint32_t* s_tmem = reinterpret_cast<uint32_t*>(sm + OFF_SMALL + 1936);
-    int* s_flag = reinterpret_cast<int*>(sm + OFF_SMALL + 1940);
+    uint32_t* s_tmem = reinterpret_cast<uint32_t*>(sm + OFF_SMALL + 3088);
 
     if (tid == 0) {
         mbar_init(bar_tma, 1);
         mbar_init(bar_mma, 1);
         fence_barrier_init();
-        *s_flag = 0;
         prefetch_tmap(&tm_q);
         prefetch_tmap(&tm_k);
         prefetch_tmap(&tm_v);
@@ -149,11 +173,11 @@ __global__ void __launch_bounds__(NT, 1) chunk_fwd_kernel(
     __syncthreads();
     tc_fence_after();
     const uint32_t tmem = *s_tmem;
-    const uint32_t lane_base = (uint32_t)(warp * 32) << 16;
+    const uint32_t lane_base = (uint32_t)((warp & 3) * 32) << 16;
     uint32_t ph_tma = 0, ph_mma = 0;
     bool ok = true;
-
     const uint32_t sbase = smem_u32(sm);
+
     auto issue_loads = [&](int ci) {
         const int t0 = ci * C;
         const uint32_t bytes = (uint32_t)(4 + 1 + 2 * (ach + bch + wch)) * 8192u;
@@ -177,17 +201,25 @@ __global__ void __launch_bounds__(NT, 1) chunk_fwd_kernel(
         }
     };
 
-    // ---- initial state: row `tid` of the slice, fp32 in registers ----------
-    float S[NV];
+    // ---- initial state: row `row`, columns [32 wg, 32 wg + 32) of the slice ----
+    constexpr int NH = NV / 2;  // state columns per thread
+    float S[NH];
     {
-        const float* s0 = p.S0 ? p.S0 + (((size_t)bb * H + h) * DK + tid) * p.dv + v0 : nullptr;
+        const float* s0 = p.S0 ? p.S0 + (((size_t)bb * H + h) * DK + row) * p.dv + v0 + wg * NH : nullptr;
 #pragma unroll
-        for (int j = 0; j < NV; j += 4) {
+        for (int j = 0; j < NH; j += 4) {
             float4 x = s0 ? *reinterpret_cast<const float4*>(s0 + j) : make_float4(0.f, 0.f, 0.f, 0.f);
             S[j] = x.x; S[j + 1] = x.y; S[j + 2] = x.z; S[j + 3] = x.w;
         }
 #pragma unroll
-        for (int ch = 0; ch < 8; ++ch) st_chunk(sm + OFF_SBF, sw128_chunk(tid, ch, DK), &S[8 * ch]);
+        for (int ch = 0; ch < 4; ++ch) st_chunk(sm + OFF_SBF, sw128_chunk(row, wg * 4 + ch, DK), &S[8 * ch]);
+        if (tid < 64) {  // AQ rows 0..63 stay zero; with tied gates so do APRE rows 64..127
+#pragma unroll
+            for (int ch = 0; ch < 8; ++ch) {
+                st_zero_chunk(sm + OFF_AQ, sw128_chunk(tid, ch, 128));
+                if (TIED) st_zero_chunk(sm + OFF_APRE, sw128_chunk(64 + tid, ch, 128));
+            }
+        }
     }
     if (tid == 0 && nchunks > 0) issue_loads(0);
 
@@ -197,10 +229,18 @@ __global__ void __launch_bounds__(NT, 1) chunk_fwd_kernel(
         ph ^= 1u;                                                           \
         if (!__syncthreads_and(w_ok)) { ok = false; goto finish; }          \
     } while (0)
+#define GDR_BEFORE_MMA()    \
+    do {                    \
+        fence_proxy_async(); \
+        tc_fence_before();  \
+        __syncthreads();    \
+    } while (0)
 
     for (int ci = 0; ci < nchunks; ++ci) {
         const int t0 = ci * C;
         const int n = min(C, T - t0);
+        const uint32_t vbuf = sbase + OFF_V + (ci & 1) * 8192u;
+        GDR_TRACE(0);
         // ---- scalar gates of this chunk (plain loads) ----------------------
         if (tid < C) {
             const int t = t0 + tid;
@@ -210,82 +250,111 @@ __global__ void __launch_bounds__(NT, 1) chunk_fwd_kernel(
             const __nv_bfloat16* bp = (const __nv_bfloat16*)p.bg;
             const __nv_bfloat16* wp = (const __nv_bfloat16*)p.wg;
             s_ascal[tid] = (p.akind == GDR_GATE_SCALAR && valid) ? __bfloat162float(ap[gi]) : 1.f;
-            s_bscal[tid] = (p.bkind == GDR_GATE_SCALAR && valid) ? __bfloat162float(bp[gi])
-                           : (p.bkind == GDR_GATE_NONE ? 0.f : 0.f);
+            s_bscal[tid] = (p.bkind == GDR_GATE_SCALAR && valid) ? __bfloat162float(bp[gi]) : 0.f;
             s_wscal[tid] = (p.wkind == GDR_GATE_SCALAR && valid) ? __bfloat162float(wp[gi])
                            : (p.wkind == GDR_GATE_NONE ? 1.f : 0.f);
         }
         GDR_WAIT(bar_tma, ph_tma);
+        GDR_TRACE(1);
 
         // ---- build: log-decay scan and scaled operands --------------------
-        // thread = (channel group cg of 8 channels, token group rg of 8 tokens)
+        // thread = (channel group cg: 8 channels, token group rg: 4 tokens)
         {
             const int cg = tid & 15, rg = tid >> 4;
             const int ch0 = cg * 8;
-            float lg[8][8];  // [token i][channel e]: log2 alpha, then inclusive prefix
-            float loc[8];
+            float* scan = reinterpret_cast<float*>(sm + OFF_SCAN);  // [16 rg][128 ch] + [128]
+            float lrow[4][8];  // channel decay: l_r - ref
+            if (!ach) {
+                // one decay per token: warp 0 scans the 64 tokens (2 per lane)
+                if (warp == 0) {
+                    const int lane = tid;
+                    const float la0 = (2 * lane < n) ? lg2_approx(s_ascal[2 * lane]) : 0.f;
+                    const float la1 = (2 * lane + 1 < n) ? lg2_approx(s_ascal[2 * lane + 1]) : 0.f;
+                    float x = la0 + la1;
 #pragma unroll
-            for (int e = 0; e < 8; ++e) loc[e] = 0.f;
+                    for (int off = 1; off < 32; off <<= 1) {
+                        float y = __shfl_up_sync(0xffffffffu, x, off);
+                        if (lane >= off) x += y;
+                    }
+                    const float l1 = x, l0v = x - la1;  // inclusive prefix at tokens 2 lane + 1, 2 lane
+                    const float first = __shfl_sync(0xffffffffu, l0v, 0);
+                    const float last = __shfl_sync(0xffffffffu, l1, 31);
+                    const float ref = 0.5f * (first + last);
+                    s_rowf[2 * lane] = ex2_approx(l0v - ref);
+                    s_rowf[2 * lane + 1] = ex2_approx(l1 - ref);
+                    s_colf[2 * lane] = ex2_approx(ref - l0v);
+                    s_colf[2 * lane + 1] = ex2_approx(ref - l1);
+                    if (lane == 0) {
+                        scan[0] = ex2_approx(ref);
+                        scan[1] = ex2_approx(last);
+                        scan[2] = ex2_approx(last - ref);
+                        if (first - last > 230.f) flag_status(p.d_status, GDR_DEVICE_DECAY_RANGE);
+                    }
+                }
+                __syncthreads();
+                if (tid < 128) {
+                    s_eref[tid] = scan[0];
+                    s_gC[tid] = scan[1];
+                    s_fS[tid] = scan[2];
+                }
+            } else {
+                float loc[8];
 #pragma unroll
-            for (int i = 0; i < 8; ++i) {
-                const int r = rg * 8 + i;
-                float a8[8];
-                if (ach) {
+                for (int e = 0; e < 8; ++e) loc[e] = 0.f;
+#pragma unroll
+                for (int i = 0; i < 4; ++i) {
+                    const int r = rg * 4 + i;
+                    float a8[8];
                     ld_chunk(sm + OFF_GA, sw128_chunk(r, cg, C), a8);
-                } else {
 #pragma unroll
-                    for (int e = 0; e < 8; ++e) a8[e] = s_ascal[r];
+                    for (int e = 0; e < 8; ++e) {
+                        loc[e] += (r < n) ? lg2_approx(a8[e]) : 0.f;
+                        lrow[i][e] = loc[e];
+                    }
+                }
+#pragma unroll
+                for (int e = 0; e < 8; ++e) scan[rg * 128 + ch0 + e] = loc[e];
+                if (rg == 0) {
+#pragma unroll
+                    for (int e = 0; e < 8; ++e) scan[2048 + ch0 + e] = lrow[0][e];
+                }
+                __syncthreads();
+                float pre[8], tot[8], ref[8];
+                bool bad = false;
+#pragma unroll
+                for (int e = 0; e < 8; ++e) { pre[e] = 0.f; tot[e] = 0.f; }
+#pragma unroll
+                for (int g = 0; g < 16; ++g) {
+                    const float4 xa = *reinterpret_cast<const float4*>(scan + g * 128 + ch0);
+                    const float4 xb = *reinterpret_cast<const float4*>(scan + g * 128 + ch0 + 4);
+                    const float xs[8] = {xa.x, xa.y, xa.z, xa.w, xb.x, xb.y, xb.z, xb.w};
+#pragma unroll
+                    for (int e = 0; e < 8; ++e) {
+                        if (g < rg) pre[e] += xs[e];
+                        tot[e] += xs[e];
+                    }
                 }
 #pragma unroll
                 for (int e = 0; e < 8; ++e) {
-                    float la = (r < n) ? lg2_approx(a8[e]) : 0.f;
-                    loc[e] += la;
-                    lg[i][e] = loc[e];
+                    const float l0 = scan[2048 + ch0 + e];
+                    ref[e] = 0.5f * (l0 + tot[e]);  // tot = l_{n-1} (padding adds 0)
+                    bad |= (l0 - tot[e]) > 230.f;
+#pragma unroll
+                    for (int i = 0; i < 4; ++i) lrow[i][e] += pre[e] - ref[e];
                 }
-            }
-            float* scan = reinterpret_cast<float*>(sm + OFF_SCAN);  // [8 rg][128 ch] totals
+                if (bad) flag_status(p.d_status, GDR_DEVICE_DECAY_RANGE);
+                if (rg == 0) {
 #pragma unroll
-            for (int e = 0; e < 8; ++e) scan[rg * 128 + ch0 + e] = loc[e];
-            __syncthreads();
-            float pre[8], tot[8], l0[8];
-#pragma unroll
-            for (int e = 0; e < 8; ++e) { pre[e] = 0.f; tot[e] = 0.f; }
-#pragma unroll
-            for (int g = 0; g < 8; ++g) {
-#pragma unroll
-                for (int e = 0; e < 8; ++e) {
-                    float x = scan[g * 128 + ch0 + e];
-                    if (g < rg) pre[e] += x;
-                    tot[e] += x;
-                }
-            }
-            // l_0 = log2 alpha_0 = first token's value (token group 0's first entry)
-            __syncthreads();
-            if (rg == 0) {
-#pragma unroll
-                for (int e = 0; e < 8; ++e) scan[1024 + ch0 + e] = lg[0][e];
-            }
-            __syncthreads();
-#pragma unroll
-            for (int e = 0; e < 8; ++e) l0[e] = scan[1024 + ch0 + e];
-            float ref[8];
-            bool bad = false;
-#pragma unroll
-            for (int e = 0; e < 8; ++e) {
-                ref[e] = 0.5f * (l0[e] + tot[e]);  // tot = l_{n-1} (padding adds 0)
-                bad |= (l0[e] - tot[e]) > 230.f;
-            }
-            if (bad) flag_status(p.d_status, GDR_DEVICE_DECAY_RANGE);
-            if (rg == 0) {
-#pragma unroll
-                for (int e = 0; e < 8; ++e) {
-                    s_gC[ch0 + e] = ex2_approx(tot[e]);
-                    s_fS[ch0 + e] = ex2_approx(tot[e] - ref[e]);
+                    for (int e = 0; e < 8; ++e) {
+                        s_eref[ch0 + e] = ex2_approx(ref[e]);
+                        s_gC[ch0 + e] = ex2_approx(tot[e]);
+                        s_fS[ch0 + e] = ex2_approx(tot[e] - ref[e]);
+                    }
                 }
             }
 #pragma unroll
-            for (int i = 0; i < 8; ++i) {
-                const int r = rg * 8 + i;
+            for (int i = 0; i < 4; ++i) {
+                const int r = rg * 4 + i;
                 float k8[8], q8[8], b8[8], w8[8];
                 ld_chunk(sm + OFF_KIN, sw128_chunk(r, cg, C), k8);
                 ld_chunk(sm + OFF_QIN, sw128_chunk(r, cg, C), q8);
@@ -305,47 +374,30 @@ __global__ void __launch_bounds__(NT, 1) chunk_fwd_kernel(
                         for (int e = 0; e < 8; ++e) w8[e] = s_wscal[r];
                     }
                 }
-                float rop_k[8], rop_q[8], rg_k[8], rg_q[8], cop_k[8], cop_w[8];
+                float rop_k[8], rop_q[8], cop_k[8], cop_w[8];
+                const bool valid = r < n;
+                const float rs = ach ? 0.f : s_rowf[r], cs = ach ? 0.f : s_colf[r];
 #pragma unroll
                 for (int e = 0; e < 8; ++e) {
-                    const float l = lg[i][e] + pre[e];
-                    const float rowf = ex2_approx(l - ref[e]);
-                    const float colf = ex2_approx(ref[e] - l);
-                    const float g = ex2_approx(l);
-                    const float kk = (r < n) ? k8[e] : 0.f;
-                    const float qq = (r < n) ? q8[e] : 0.f;
+                    const float rowf = ach ? ex2_approx(lrow[i][e]) : rs;
+                    const float colf = ach ? ex2_approx(-lrow[i][e]) : cs;
+                    const float kk = valid ? k8[e] : 0.f;
+                    const float qq = valid ? q8[e] : 0.f;
                     rop_k[e] = b8[e] * kk * rowf;
                     rop_q[e] = qq * rowf;
-                    rg_k[e] = b8[e] * kk * g;
-                    rg_q[e] = qq * g;
                     cop_k[e] = kk * colf;
                     cop_w[e] = TIED ? 0.f : w8[e] * kk * colf;
                 }
                 st_chunk(sm + OFF_ROP, sw128_chunk(r, cg, 128), rop_k);
                 st_chunk(sm + OFF_ROP, sw128_chunk(64 + r, cg, 128), rop_q);
-                st_chunk(sm + OFF_RG, sw128_chunk(r, cg, 128), rg_k);
-                st_chunk(sm + OFF_RG, sw128_chunk(64 + r, cg, 128), rg_q);
                 st_chunk(sm + OFF_COP, sw128_chunk(r, cg, N1), cop_k);
                 if (!TIED) st_chunk(sm + OFF_COP, sw128_chunk(64 + r, cg, N1), cop_w);
             }
         }
-        __syncthreads();  // scan scratch (over X) is dead from here on
-        if (TIED) {
-            // X = [-Diag(beta) ; 0]: row t, 8 chunks of 8 columns
-            float z[8];
-#pragma unroll
-            for (int c8 = 0; c8 < 8; ++c8) {
-#pragma unroll
-                for (int e = 0; e < 8; ++e)
-                    z[e] = (tid < 64 && c8 * 8 + e == tid) ? -s_bscal[tid] : 0.f;
-                st_chunk(sm + OFF_X, sw128_chunk(tid, c8, 128), z);
-            }
-        }
-        fence_proxy_async();
-        tc_fence_before();
-        __syncthreads();
+        GDR_BEFORE_MMA();
+        GDR_TRACE(2);
 
-        // ---- P1: D1 = Rop x Cop^T ------------------------------------------
+        // ---- P1: D1 = [Kb ; Qs] x [Ks ; Kws]^T --------------------------------
         if (tid == 0) {
             tc_fence_after();
             const uint32_t id = idesc_bf16(128, N1, 0, 0);
@@ -360,250 +412,325 @@ __global__ void __launch_bounds__(NT, 1) chunk_fwd_kernel(
         }
         GDR_WAIT(bar_mma, ph_mma);
         tc_fence_after();
+        GDR_TRACE(3);
 
-        // ---- unload D1: A (fp32), [0 ; -Aq] (bf16), X for general gates ------
+        // ---- unload D1 (each warpgroup one half of the columns): A (fp32),
+        //      Aq -> AQ rows 64..127; general gates: Bm -> X, Bq -> APRE rows 64..127 ----
         {
-            const int r = tid & 63;
-            float d[64];
-            tmem_ld32(tmem + lane_base + TM_D1, d);
-            tmem_ld32(tmem + lane_base + TM_D1 + 32, d + 32);
-            if (tid < 64) {
+            const int r = row & 63;
+            float d[32];
+            tmem_ld32(tmem + lane_base + TM_D1 + wg * 32, d);
+            if (row < 64) {
                 float* A32 = reinterpret_cast<float*>(sm + OFF_A32);
 #pragma unroll
-                for (int j = 0; j < 64; j += 4) {
-                    float4 x = make_float4(j < r ? d[j] : 0.f, j + 1 < r ? d[j + 1] : 0.f,
-                                           j + 2 < r ? d[j + 2] : 0.f, j + 3 < r ? d[j + 3] : 0.f);
+                for (int j4 = 0; j4 < 32; j4 += 4) {
+                    const int j = wg * 32 + j4;
+                    float4 x = make_float4(j < r ? d[j4] : 0.f, j + 1 < r ? d[j4 + 1] : 0.f,
+                                           j + 2 < r ? d[j4 + 2] : 0.f, j + 3 < r ? d[j4 + 3] : 0.f);
                     *reinterpret_cast<float4*>(f32_at(A32, r, j)) = x;
                 }
-                float z[8];
-#pragma unroll
-                for (int e = 0; e < 8; ++e) z[e] = 0.f;
-#pragma unroll
-                for (int c8 = 0; c8 < 8; ++c8) st_chunk(sm + OFF_AP, sw128_chunk(tid, c8, 128), z);
             } else {
                 float x[8];
 #pragma unroll
-                for (int c8 = 0; c8 < 8; ++c8) {
+                for (int c8 = 0; c8 < 4; ++c8) {
 #pragma unroll
-                    for (int e = 0; e < 8; ++e) {
-                        const int j = c8 * 8 + e;
-                        x[e] = j <= r ? -d[j] : 0.f;
-                    }
-                    st_chunk(sm + OFF_AP, sw128_chunk(tid, c8, 128), x);
+                    for (int e = 0; e < 8; ++e) x[e] = (wg * 32 + c8 * 8 + e <= r) ? d[c8 * 8 + e] : 0.f;
+                    st_chunk(sm + OFF_AQ, sw128_chunk(row, wg * 4 + c8, 128), x);
                 }
             }
             if (!TIED) {
-                tmem_ld32(tmem + lane_base + TM_D1 + 64, d);
-                tmem_ld32(tmem + lane_base + TM_D1 + 96, d + 32);
+                tmem_ld32(tmem + lane_base + TM_D1 + 64 + wg * 32, d);
                 float x[8];
 #pragma unroll
-                for (int c8 = 0; c8 < 8; ++c8) {
+                for (int c8 = 0; c8 < 4; ++c8) {
 #pragma unroll
                     for (int e = 0; e < 8; ++e) {
-                        const int j = c8 * 8 + e;
-                        x[e] = (tid < 64 ? j < r : j <= r) ? d[j] : 0.f;
+                        const int j = wg * 32 + c8 * 8 + e;
+                        x[e] = (row < 64 ? j < r : j <= r) ? d[c8 * 8 + e] : 0.f;
                     }
-                    st_chunk(sm + OFF_X, sw128_chunk(tid, c8, 128), x);
+                    if (row < 64) st_chunk(sm + OFF_X, sw128_chunk(r, wg * 4 + c8, 64), x);   // Bm
+                    else st_chunk(sm + OFF_APRE, sw128_chunk(row, wg * 4 + c8, 128), x);     // Bq
                 }
             }
         }
-        tc_fence_before();
         __syncthreads();
+        GDR_TRACE(4);
 
-        // ---- solve T = (I + A)^-1, 16x16 blocks -------------------------------
+        // ---- solve T = (I + A)^-1 (fp32) by recursive halving:
+        //      16x16 diagonal blocks by forward substitution, then
+        //      T_(I+1)I = -T_(I+1)(I+1) A_(I+1)I T_II for the pairs (1,0), (3,2),
+        //      then T_bot,top = -T_bot A_bot,top T_top for the 32x32 halves ----------
         {
             float* A32 = reinterpret_cast<float*>(sm + OFF_A32);
             float* T32 = reinterpret_cast<float*>(sm + OFF_T32);
-            float* P32 = reinterpret_cast<float*>(sm + OFF_P32);
+            float* X16 = reinterpret_cast<float*>(sm + OFF_P32);          // [2][16 x 16]
+            float* Y32 = reinterpret_cast<float*>(sm + OFF_P32 + 2048);   // [32 x 32]
             if (tid < 64) {
-                // diagonal block I, column c: forward substitution
                 const int I = tid >> 4, c = tid & 15;
                 float x[16];
 #pragma unroll
-                for (int rr = 0; rr < 16; ++rr) {
-                    float s = (rr == c) ? 1.f : 0.f;
+                for (int j = 0; j < 16; ++j) x[j] = 0.f;
 #pragma unroll
-                    for (int j = 0; j < rr; ++j) s -= *f32_at(A32, 16 * I + rr, 16 * I + j) * x[j];
-                    x[rr] = s;
+                for (int rr = 0; rr < 16; ++rr) {
+                    float a[16];
+#pragma unroll
+                    for (int j4 = 0; j4 < 16; j4 += 4) {
+                        const float4 v4 = *reinterpret_cast<const float4*>(f32_at(A32, 16 * I + rr, 16 * I + j4));
+                        a[j4] = v4.x; a[j4 + 1] = v4.y; a[j4 + 2] = v4.z; a[j4 + 3] = v4.w;
+                    }
+                    float s0 = 0.f, s1 = 0.f, s2 = 0.f, s3 = 0.f;
+#pragma unroll
+                    for (int j = 0; j < rr; j += 4) {
+                        s0 += a[j] * x[j];
+                        if (j + 1 < rr) s1 += a[j + 1] * x[j + 1];
+                        if (j + 2 < rr) s2 += a[j + 2] * x[j + 2];
+                        if (j + 3 < rr) s3 += a[j + 3] * x[j + 3];
+                    }
+                    x[rr] = ((rr == c) ? 1.f : 0.f) - ((s0 + s1) + (s2 + s3));
                 }
 #pragma unroll
                 for (int rr = 0; rr < 16; ++rr) *f32_at(T32, 16 * I + rr, 16 * I + c) = x[rr];
-            } else {
-                // zero the strictly upper blocks of T (rows 0..47)
-                const int u = tid - 64;  // 64 threads
-                for (int idx = u; idx < 6 * 256; idx += 64) {
-                    const int blk = idx >> 8, e = idx & 255;
-                    // upper blocks (I,J) with J > I: (0,1)(0,2)(0,3)(1,2)(1,3)(2,3)
-                    const int I = blk < 3 ? 0 : (blk < 5 ? 1 : 2);
-                    const int J = blk < 3 ? blk + 1 : (blk < 5 ? blk - 1 : 3);
-                    *f32_at(T32, 16 * I + (e >> 4), 16 * J + (e & 15)) = 0.f;
+            } else if (tid < 128) {
+                // the strictly upper 16x16 blocks inside each 32x32 diagonal half are zero
+                const int u = tid - 64;                        // 64 threads, 2 blocks x 16 rows x 4 float4
+                for (int idx = u; idx < 128; idx += 64) {
+                    const int blk = idx >> 6, rr = (idx >> 2) & 15, c4 = (idx & 3) * 4;
+                    *reinterpret_cast<float4*>(f32_at(T32, 32 * blk + rr, 32 * blk + 16 + c4)) =
+                        make_float4(0.f, 0.f, 0.f, 0.f);
                 }
             }
             __syncthreads();
-            for (int dlev = 1; dlev <= 3; ++dlev) {
-                const int nb = 4 - dlev;
-                // stage a: P_IJ = sum_{K=J}^{I-1} A_IK T_KJ, units of 2 rows x 4 cols
-                for (int u = tid; u < nb * 32; u += NT) {
-                    const int bi = u >> 5, rr = ((u >> 2) & 7) * 2, c4 = (u & 3) * 4;
-                    const int I = dlev + bi, J = bi;
-                    float acc0[4] = {0.f, 0.f, 0.f, 0.f}, acc1[4] = {0.f, 0.f, 0.f, 0.f};
-                    for (int K = J; K < I; ++K) {
+            GDR_TRACE(12);
+            // X_b = A_(2b+1)(2b) T_(2b)(2b), b = 0, 1: units of (row, 4 columns), 128 units
+            if (tid < 128) {
+                const int b = tid >> 6, rr = (tid >> 2) & 15, c4 = (tid & 3) * 4;
+                const int R = 32 * b + 16, Cc = 32 * b;
+                float acc[4] = {0.f, 0.f, 0.f, 0.f};
 #pragma unroll
-                        for (int m = 0; m < 16; ++m) {
-                            const float a0 = *f32_at(A32, 16 * I + rr, 16 * K + m);
-                            const float a1 = *f32_at(A32, 16 * I + rr + 1, 16 * K + m);
-                            const float4 t4 = *reinterpret_cast<const float4*>(f32_at(T32, 16 * K + m, 16 * J + c4));
-                            acc0[0] += a0 * t4.x; acc0[1] += a0 * t4.y; acc0[2] += a0 * t4.z; acc0[3] += a0 * t4.w;
-                            acc1[0] += a1 * t4.x; acc1[1] += a1 * t4.y; acc1[2] += a1 * t4.z; acc1[3] += a1 * t4.w;
-                        }
-                    }
-                    float* pb = P32 + bi * 256;
+                for (int m4 = 0; m4 < 16; m4 += 4) {
+                    const float4 a4 = *reinterpret_cast<const float4*>(f32_at(A32, R + rr, Cc + m4));
+                    const float av[4] = {a4.x, a4.y, a4.z, a4.w};
 #pragma unroll
-                    for (int e = 0; e < 4; ++e) {
-                        pb[rr * 16 + c4 + e] = acc0[e];
-                        pb[(rr + 1) * 16 + c4 + e] = acc1[e];
+                    for (int mm = 0; mm < 4; ++mm) {
+                        const float4 t4 = *reinterpret_cast<const float4*>(f32_at(T32, Cc + m4 + mm, Cc + c4));
+                        acc[0] += av[mm] * t4.x; acc[1] += av[mm] * t4.y; acc[2] += av[mm] * t4.z; acc[3] += av[mm] * t4.w;
                     }
                 }
-                __syncthreads();
-                // stage b: T_IJ = -T_II P_IJ
-                for (int u = tid; u < nb * 32; u += NT) {
-                    const int bi = u >> 5, rr = ((u >> 2) & 7) * 2, c4 = (u & 3) * 4;
-                    const int I = dlev + bi, J = bi;
-                    const float* pb = P32 + bi * 256;
-                    float acc0[4] = {0.f, 0.f, 0.f, 0.f}, acc1[4] = {0.f, 0.f, 0.f, 0.f};
-#pragma unroll
-                    for (int m = 0; m < 16; ++m) {
-                        const float t0v = *f32_at(T32, 16 * I + rr, 16 * I + m);
-                        const float t1v = *f32_at(T32, 16 * I + rr + 1, 16 * I + m);
-                        const float4 p4 = *reinterpret_cast<const float4*>(pb + m * 16 + c4);
-                        acc0[0] += t0v * p4.x; acc0[1] += t0v * p4.y; acc0[2] += t0v * p4.z; acc0[3] += t0v * p4.w;
-                        acc1[0] += t1v * p4.x; acc1[1] += t1v * p4.y; acc1[2] += t1v * p4.z; acc1[3] += t1v * p4.w;
-                    }
-                    *reinterpret_cast<float4*>(f32_at(T32, 16 * I + rr, 16 * J + c4)) =
-                        make_float4(-acc0[0], -acc0[1], -acc0[2], -acc0[3]);
-                    *reinterpret_cast<float4*>(f32_at(T32, 16 * I + rr + 1, 16 * J + c4)) =
-                        make_float4(-acc1[0], -acc1[1], -acc1[2], -acc1[3]);
-                }
-                __syncthreads();
+                *reinterpret_cast<float4*>(X16 + b * 256 + rr * 16 + c4) = make_float4(acc[0], acc[1], acc[2], acc[3]);
             }
-            // L = [[T, 0], [0, I]] as bf16 [128 x 128]: thread = row
+            __syncthreads();
+            // T_(2b+1)(2b) = -T_(2b+1)(2b+1) X_b
+            if (tid < 128) {
+                const int b = tid >> 6, rr = (tid >> 2) & 15, c4 = (tid & 3) * 4;
+                const int R = 32 * b + 16, Cc = 32 * b;
+                float acc[4] = {0.f, 0.f, 0.f, 0.f};
+#pragma unroll
+                for (int m4 = 0; m4 < 16; m4 += 4) {
+                    const float4 t4 = *reinterpret_cast<const float4*>(f32_at(T32, R + rr, R + m4));
+                    const float tv[4] = {t4.x, t4.y, t4.z, t4.w};
+#pragma unroll
+                    for (int mm = 0; mm < 4; ++mm) {
+                        const float4 x4 = *reinterpret_cast<const float4*>(X16 + b * 256 + (m4 + mm) * 16 + c4);
+                        acc[0] += tv[mm] * x4.x; acc[1] += tv[mm] * x4.y; acc[2] += tv[mm] * x4.z; acc[3] += tv[mm] * x4.w;
+                    }
+                }
+                *reinterpret_cast<float4*>(f32_at(T32, R + rr, Cc + c4)) = make_float4(-acc[0], -acc[1], -acc[2], -acc[3]);
+            }
+            __syncthreads();
+            GDR_TRACE(13);
+            // Y = A[32:64, 0:32] T[0:32, 0:32]: 256 units of (row, 4 columns)
             {
-                float x[8];
+                const int rr = tid >> 3, c4 = (tid & 7) * 4;
+                float acc[4] = {0.f, 0.f, 0.f, 0.f};
 #pragma unroll
-                for (int c8 = 0; c8 < 16; ++c8) {
+                for (int m4 = 0; m4 < 32; m4 += 4) {
+                    const float4 a4 = *reinterpret_cast<const float4*>(f32_at(A32, 32 + rr, m4));
+                    const float av[4] = {a4.x, a4.y, a4.z, a4.w};
 #pragma unroll
-                    for (int e = 0; e < 8; ++e) {
-                        const int j = c8 * 8 + e;
-                        if (tid < 64) x[e] = j < 64 ? *f32_at(T32, tid, j) : 0.f;
-                        else x[e] = (j == tid) ? 1.f : 0.f;
+                    for (int mm = 0; mm < 4; ++mm) {
+                        const float4 t4 = *reinterpret_cast<const float4*>(f32_at(T32, m4 + mm, c4));
+                        acc[0] += av[mm] * t4.x; acc[1] += av[mm] * t4.y; acc[2] += av[mm] * t4.z; acc[3] += av[mm] * t4.w;
                     }
-                    st_chunk(sm + OFF_L, sw128_chunk(tid, c8, 128), x);
                 }
+                *reinterpret_cast<float4*>(Y32 + rr * 32 + c4) = make_float4(acc[0], acc[1], acc[2], acc[3]);
             }
-        }
-        fence_proxy_async();
-        tc_fence_before();
-        __syncthreads();
-
-        // ---- P2: D2 = L x [Rg | X] -------------------------------------------
-        if (tid == 0) {
-            tc_fence_after();
-            const uint32_t idA = idesc_bf16(128, 128, 0, 1);
-            const uint32_t idX = idesc_bf16(128, 64, 0, 1);
+            __syncthreads();
+            // T[32:64, 0:32] = -T[32:64, 32:64] Y
+            {
+                const int rr = tid >> 3, c4 = (tid & 7) * 4;
+                float acc[4] = {0.f, 0.f, 0.f, 0.f};
 #pragma unroll
-            for (int ks = 0; ks < 8; ++ks) {
-                const uint64_t ad = sdesc_sw128(sbase + OFF_L + (ks >> 2) * 16384u + (ks & 3) * 32u, 16, 1024);
-                mma_bf16(tmem + TM_D2, ad, sdesc_sw128(sbase + OFF_RG + ks * 2048u, 16384, 1024), idA, ks > 0);
-                mma_bf16(tmem + TM_D2 + 128, ad, sdesc_sw128(sbase + OFF_X + ks * 2048u, 16384, 1024), idX, ks > 0);
+                for (int m4 = 0; m4 < 32; m4 += 4) {
+                    const float4 t4 = *reinterpret_cast<const float4*>(f32_at(T32, 32 + rr, 32 + m4));
+                    const float tv[4] = {t4.x, t4.y, t4.z, t4.w};
+#pragma unroll
+                    for (int mm = 0; mm < 4; ++mm) {
+                        const float4 y4 = *reinterpret_cast<const float4*>(Y32 + (m4 + mm) * 32 + c4);
+                        acc[0] += tv[mm] * y4.x; acc[1] += tv[mm] * y4.y; acc[2] += tv[mm] * y4.z; acc[3] += tv[mm] * y4.w;
+                    }
+                }
+                *reinterpret_cast<float4*>(f32_at(T32, 32 + rr, c4)) = make_float4(-acc[0], -acc[1], -acc[2], -acc[3]);
             }
-            mma_commit(bar_mma);
-        }
-        GDR_WAIT(bar_mma, ph_mma);
-        tc_fence_after();
-
-        // next chunk's inputs may now overwrite the input region (A32, T32, L
-        // were last read above / by P2) -- except AP, read by P3 below.
-        // ---- E_top = D2 rows 0..63 -> bf16 ----------------------------------
-        if (tid < 64) {
-            float d[32];
-#pragma unroll
-            for (int cb = 0; cb < 6; ++cb) {
-                tmem_ld32(tmem + lane_base + TM_D2 + cb * 32, d);
-#pragma unroll
-                for (int c4 = 0; c4 < 4; ++c4) st_chunk(sm + OFF_E, sw128_chunk(tid, cb * 4 + c4, 128), d + 8 * c4);
-            }
-        }
-        fence_proxy_async();
-        tc_fence_before();
-        __syncthreads();
-
-        // ---- P3: D2 += [0 ; -Aq] x E_top --------------------------------------
-        if (tid == 0) {
-            tc_fence_after();
-            const uint32_t id = idesc_bf16(128, 192, 0, 1);
-#pragma unroll
-            for (int ks = 0; ks < 4; ++ks)
-                mma_bf16(tmem + TM_D2, sdesc_sw128(sbase + OFF_AP + ks * 32u, 16, 1024),
-                         sdesc_sw128(sbase + OFF_E + ks * 2048u, 16384, 1024), id, 1);
-            mma_commit(bar_mma);
-        }
-        GDR_WAIT(bar_mma, ph_mma);
-        tc_fence_after();
-        if (tid == 0 && ci + 1 < nchunks) {
-            fence_proxy_async();
-            issue_loads(ci + 1);
-        }
-
-        // ---- E_bot = D2 rows 64..127 -> bf16 ----------------------------------
-        if (tid >= 64) {
-            float d[32];
-#pragma unroll
-            for (int cb = 0; cb < 6; ++cb) {
-                tmem_ld32(tmem + lane_base + TM_D2 + cb * 32, d);
-#pragma unroll
-                for (int c4 = 0; c4 < 4; ++c4) st_chunk(sm + OFF_E, sw128_chunk(tid, cb * 4 + c4, 128), d + 8 * c4);
-            }
-        }
-        fence_proxy_async();
-        tc_fence_before();
-        __syncthreads();
-
-        // ---- S1: D3 = E x [S ; V] ---------------------------------------------
-        const uint32_t vbuf = sbase + OFF_V + (ci & 1) * 8192u;
-        if (tid == 0) {
-            tc_fence_after();
-            const uint32_t id = idesc_bf16(128, NV, 0, 1);
-#pragma unroll
-            for (int ks = 0; ks < 12; ++ks) {
-                const uint64_t ad = sdesc_sw128(sbase + OFF_E + (ks >> 2) * 16384u + (ks & 3) * 32u, 16, 1024);
-                const uint64_t bd = ks < 8 ? sdesc_sw128(sbase + OFF_SBF + ks * 2048u, 8192, 1024)
-                                           : sdesc_sw128(vbuf + (ks - 8) * 2048u, 8192, 1024);
-                mma_bf16(tmem + TM_D3, ad, bd, id, ks > 0);
-            }
-            mma_commit(bar_mma);
-        }
-        GDR_WAIT(bar_mma, ph_mma);
-        tc_fence_after();
-
-        // ---- epilogue: U -> smem, O -> global -----------------------------------
-        {
-            float d[64];
-            tmem_ld32(tmem + lane_base + TM_D3, d);
-            tmem_ld32(tmem + lane_base + TM_D3 + 32, d + 32);
-            if (tid < 64) {
+            __syncthreads();
+            GDR_TRACE(14);
+            // L = [T ; 0] (bf16, 128 x 64); tied: APRE rows 0..63 = T Diag(beta)
+            if (tid < 128) {
                 float x[8];
 #pragma unroll
                 for (int c8 = 0; c8 < 8; ++c8) {
+                    if (tid < 64) {
 #pragma unroll
-                    for (int e = 0; e < 8; ++e) x[e] = -d[c8 * 8 + e];
-                    st_chunk(sm + OFF_U, sw128_chunk(tid, c8, 64), x);
+                        for (int e4 = 0; e4 < 8; e4 += 4) {
+                            const int j = c8 * 8 + e4;
+                            // T is lower triangular: the upper-right 32x32 block is zero
+                            float4 t4 = (j < 32 || tid >= 32)
+                                            ? *reinterpret_cast<const float4*>(f32_at(T32, tid, j))
+                                            : make_float4(0.f, 0.f, 0.f, 0.f);
+                            x[e4] = t4.x; x[e4 + 1] = t4.y; x[e4 + 2] = t4.z; x[e4 + 3] = t4.w;
+                        }
+                        st_chunk(sm + OFF_L, sw128_chunk(tid, c8, 128), x);
+                        if (TIED) {
+#pragma unroll
+                            for (int e = 0; e < 8; ++e) x[e] *= s_bscal[c8 * 8 + e];
+                            st_chunk(sm + OFF_APRE, sw128_chunk(tid, c8, 128), x);
+                        }
+                    } else {
+                        st_zero_chunk(sm + OFF_L, sw128_chunk(tid, c8, 128));
+                    }
                 }
-            } else {
-                const int t = t0 + tid - 64;
-                if (t < T) {
-                    __nv_bfloat16* op = p.o + (((size_t)bb * T + t) * H + h) * p.dv + v0;
+            }
+        }
+        GDR_BEFORE_MMA();
+        GDR_TRACE(5);
+
+        // ---- P2: D2 = [T ; 0] x [Kb | Bm];  tied: P3 D3 = [T Diag(beta) ; 0] x V ----
+        if (tid == 0) {
+            tc_fence_after();
+            const uint32_t idW = idesc_bf16(128, 128, 0, 1);
+            const uint32_t id64 = idesc_bf16(128, 64, 0, 1);
 #pragma unroll
-                    for (int c8 = 0; c8 < 8; ++c8) {
+            for (int ks = 0; ks < 4; ++ks) {
+                const uint64_t ad = sdesc_sw128(sbase + OFF_L + ks * 32u, 16, 1024);
+                mma_bf16(tmem + TM_D2, ad, sdesc_sw128(sbase + OFF_ROP + ks * 2048u, 16384, 1024), idW, ks > 0);
+                if (!TIED)
+                    mma_bf16(tmem + TM_D2 + 128, ad, sdesc_sw128(sbase + OFF_X + ks * 2048u, 8192, 1024), id64, ks > 0);
+            }
+            if (TIED) {
+#pragma unroll
+                for (int ks = 0; ks < 4; ++ks)
+                    mma_bf16(tmem + TM_D3, sdesc_sw128(sbase + OFF_APRE + ks * 32u, 16, 1024),
+                             sdesc_sw128(vbuf + ks * 2048u, 8192, 1024), id64, ks > 0);
+            }
+            mma_commit(bar_mma);
+        }
+        GDR_WAIT(bar_mma, ph_mma);
+        tc_fence_after();
+        GDR_TRACE(6);
+        // the input region (A, T, L, Bm) is free: prefetch the next chunk
+        if (tid == 0 && ci + 1 < nchunks) issue_loads(ci + 1);
+
+        // ---- W -> [-W ; Qs.2^ref] in place of [Kb ; Qs]; general: -T Bm -> APRE -----
+        if (row < 64) {
+            float d[32];
+#pragma unroll
+            for (int cb = 0; cb < 2; ++cb) {
+                const int col = wg * 64 + cb * 32;
+                tmem_ld32(tmem + lane_base + TM_D2 + col, d);
+#pragma unroll
+                for (int c4 = 0; c4 < 4; ++c4) {
+                    float x[8];
+#pragma unroll
+                    for (int e = 0; e < 8; ++e) x[e] = -d[c4 * 8 + e] * s_eref[col + c4 * 8 + e];
+                    st_chunk(sm + OFF_ROP, sw128_chunk(row, col / 8 + c4, 128), x);
+                }
+            }
+            if (!TIED) {
+                tmem_ld32(tmem + lane_base + TM_D2 + 128 + wg * 32, d);
+#pragma unroll
+                for (int c4 = 0; c4 < 4; ++c4) {
+                    float x[8];
+#pragma unroll
+                    for (int e = 0; e < 8; ++e) x[e] = -d[c4 * 8 + e];
+                    st_chunk(sm + OFF_APRE, sw128_chunk(row, wg * 4 + c4, 128), x);
+                }
+            }
+        } else {
+#pragma unroll
+            for (int c = 0; c < 8; ++c) {
+                const int ch = wg * 8 + c;
+                float x[8];
+                const uint32_t off = sw128_chunk(row, ch, 128);
+                ld_chunk(sm + OFF_ROP, off, x);
+#pragma unroll
+                for (int e = 0; e < 8; ++e) x[e] *= s_eref[ch * 8 + e];
+                st_chunk(sm + OFF_ROP, off, x);
+            }
+        }
+        GDR_BEFORE_MMA();
+        GDR_TRACE(7);
+
+        // ---- general: P3 D3 = [-T Bm ; Bq] x V;  S1: D3 += [-W ; Qs.2^ref] x S -----
+        if (tid == 0) {
+            tc_fence_after();
+            const uint32_t id64 = idesc_bf16(128, NV, 0, 1);
+            if (!TIED) {
+#pragma unroll
+                for (int ks = 0; ks < 4; ++ks)
+                    mma_bf16(tmem + TM_D3, sdesc_sw128(sbase + OFF_APRE + ks * 32u, 16, 1024),
+                             sdesc_sw128(vbuf + ks * 2048u, 8192, 1024), id64, ks > 0);
+            }
+#pragma unroll
+            for (int ks = 0; ks < 8; ++ks)
+                mma_bf16(tmem + TM_D3, sdesc_sw128(sbase + OFF_ROP + (ks >> 2) * 16384u + (ks & 3) * 32u, 16, 1024),
+                         sdesc_sw128(sbase + OFF_SBF + ks * 2048u, 8192, 1024), id64, 1);
+            mma_commit(bar_mma);
+        }
+        GDR_WAIT(bar_mma, ph_mma);
+        tc_fence_after();
+        GDR_TRACE(8);
+
+        // ---- U (rows 0..63 of D3) -> bf16 ---------------------------------------
+        if (row < 64) {
+            float d[32];
+            tmem_ld32(tmem + lane_base + TM_D3 + wg * 32, d);
+#pragma unroll
+            for (int c8 = 0; c8 < 4; ++c8) st_chunk(sm + OFF_U, sw128_chunk(row, wg * 4 + c8, 64), d + 8 * c8);
+        }
+        GDR_BEFORE_MMA();
+        GDR_TRACE(9);
+
+        // ---- S2: D3 += [0 ; Aq] x U ;  D4 = [Ks ; Kws]^T x [U ; V] -----------------
+        if (tid == 0) {
+            tc_fence_after();
+            const uint32_t idK = idesc_bf16(128, NV, 0, 1);
+            const uint32_t idM = idesc_bf16(128, NV, 1, 1);
+#pragma unroll
+            for (int ks = 0; ks < 4; ++ks)
+                mma_bf16(tmem + TM_D3, sdesc_sw128(sbase + OFF_AQ + ks * 32u, 16, 1024),
+                         sdesc_sw128(sbase + OFF_U + ks * 2048u, 8192, 1024), idK, 1);
+#pragma unroll
+            for (int ks = 0; ks < N1 / 16; ++ks) {
+                const uint64_t ad = sdesc_sw128(sbase + OFF_COP + ks * 2048u, N1 * 128, 1024);
+                const uint64_t bd = ks < 4 ? sdesc_sw128(sbase + OFF_U + ks * 2048u, 8192, 1024)
+                                           : sdesc_sw128(vbuf + (ks - 4) * 2048u, 8192, 1024);
+                mma_bf16(tmem + TM_D4, ad, bd, idM, ks > 0);
+            }
+            mma_commit(bar_mma);
+        }
+        GDR_WAIT(bar_mma, ph_mma);
+        tc_fence_after();
+        GDR_TRACE(10);
+
+        // ---- O (rows 64..127 of D3) -> global; state update from D4 -----------------
+        {
+            float d[32];
+            if (row >= 64) {
+                tmem_ld32(tmem + lane_base + TM_D3 + wg * 32, d);
+                const int t = t0 + row - 64;
+                if (t < T) {
+                    __nv_bfloat16* op = p.o + (((size_t)bb * T + t) * H + h) * p.dv + v0 + wg * 32;
+#pragma unroll
+                    for (int c8 = 0; c8 < 4; ++c8) {
                         uint4 u;
                         u.x = pack_bf16x2(d[c8 * 8 + 0], d[c8 * 8 + 1]);
                         u.y = pack_bf16x2(d[c8 * 8 + 2], d[c8 * 8 + 3]);
@@ -613,46 +740,22 @@ __global__ void __launch_bounds__(NT, 1) chunk_fwd_kernel(
                     }
                 }
             }
-        }
-        fence_proxy_async();
-        tc_fence_before();
-        __syncthreads();
-
-        // ---- S2: D4 = Cop^T x [U ; V] ------------------------------------------
-        if (tid == 0) {
-            tc_fence_after();
-            const uint32_t id = idesc_bf16(128, NV, 1, 1);
+            tmem_ld32(tmem + lane_base + TM_D4 + wg * 32, d);
+            const float gC = s_gC[row], fS = s_fS[row];
 #pragma unroll
-            for (int ks = 0; ks < N1 / 16; ++ks) {
-                const uint64_t ad = sdesc_sw128(sbase + OFF_COP + ks * 2048u, N1 * 128, 1024);
-                const uint64_t bd = ks < 4 ? sdesc_sw128(sbase + OFF_U + ks * 2048u, 8192, 1024)
-                                           : sdesc_sw128(vbuf + (ks - 4) * 2048u, 8192, 1024);
-                mma_bf16(tmem + TM_D4, ad, bd, id, ks > 0);
-            }
-            mma_commit(bar_mma);
-        }
-        GDR_WAIT(bar_mma, ph_mma);
-        tc_fence_after();
-
-        // ---- state update: S = Diag(g) S + Diag(f) D4 ------------------------
-        {
-            float d[64];
-            tmem_ld32(tmem + lane_base + TM_D4, d);
-            tmem_ld32(tmem + lane_base + TM_D4 + 32, d + 32);
-            const float gC = s_gC[tid], fS = s_fS[tid];
+            for (int j = 0; j < NH; ++j) S[j] = gC * S[j] + fS * d[j];
 #pragma unroll
-            for (int j = 0; j < NV; ++j) S[j] = gC * S[j] + fS * d[j];
-#pragma unroll
-            for (int ch = 0; ch < 8; ++ch) st_chunk(sm + OFF_SBF, sw128_chunk(tid, ch, DK), &S[8 * ch]);
+            for (int ch = 0; ch < 4; ++ch) st_chunk(sm + OFF_SBF, sw128_chunk(row, wg * 4 + ch, DK), &S[8 * ch]);
         }
         tc_fence_before();
         __syncthreads();
+        GDR_TRACE(11);
     }
 
     if (p.ST) {
-        float* st = p.ST + (((size_t)bb * H + h) * DK + tid) * p.dv + v0;
+        float* st = p.ST + (((size_t)bb * H + h) * DK + row) * p.dv + v0 + wg * NH;
 #pragma unroll
-        for (int j = 0; j < NV; j += 4) *reinterpret_cast<float4*>(st + j) = make_float4(S[j], S[j + 1], S[j + 2], S[j + 3]);
+        for (int j = 0; j < NH; j += 4) *reinterpret_cast<float4*>(st + j) = make_float4(S[j], S[j + 1], S[j + 2], S[j + 3]);
     }
 
 finish:
@@ -661,6 +764,7 @@ finish:
     __syncthreads();
     if (warp == 0) tmem_dealloc(tmem, TM_COLS);
 #undef GDR_WAIT
+#undef GDR_BEFORE_MMA
 }
 
 }  // namespace chunk
@@ -690,3 +794,9 @@ cudaError_t launch_chunk_sm100(const CUtensorMap* maps, const void* alpha, const
 }
 
 }  // namespace gdr
+
+#ifdef GDR_TRACE_PHASES
+extern "C" int gdr_trace_read(unsigned long long* host, int n) {
+    return (int)cudaMemcpyFromSymbol(host, gdr::chunk::g_trace, sizeof(unsigned long long) * n);
+}
+#endif
