@@ -53,7 +53,7 @@ constexpr uint32_t OFF_GW = 65536;     // channel w chunk
 constexpr uint32_t OFF_A32 = 0;        // A fp32 [64 x 64] (float4 groups swizzled by row)
 constexpr uint32_t OFF_T32 = 16384;    // T fp32 [64 x 64]
 constexpr uint32_t OFF_X = 32768;      // Bm bf16 [64 x 64] (general gates)
-constexpr uint32_t OFF_P32 = 40960;    // solve scratch fp32 3 x [16 x 16]
+constexpr uint32_t OFF_P32 = 40960;    // solve scratch fp32 (8 KB)
 constexpr uint32_t OFF_L = 49152;      // [T ; 0] bf16 [128 x 64]
 constexpr uint32_t OFF_V = 81920;      // v slice [64 x 64] bf16, two buffers
 constexpr uint32_t OFF_ROP = 98304;    // [Kb ; Qs] bf16 [128 x 128], later [-W ; Qs.2^ref]
@@ -221,7 +221,21 @@ __global__ void __launch_bounds__(NT, 1) chunk_fwd_kernel(
             }
         }
     }
+    // scalar gates travel in registers of threads 0..63 one chunk ahead
+    float g_a = 1.f, g_b = 0.f, g_w = 1.f;
+    auto load_scalar_gates = [&](int ci) {
+        if (tid < C) {
+            const int t = ci * C + tid;
+            const bool valid = t < T;
+            const size_t gi = ((size_t)bb * T + t) * H + h;
+            g_a = (p.akind == GDR_GATE_SCALAR && valid) ? __bfloat162float(((const __nv_bfloat16*)p.alpha)[gi]) : 1.f;
+            g_b = (p.bkind == GDR_GATE_SCALAR && valid) ? __bfloat162float(((const __nv_bfloat16*)p.bg)[gi]) : 0.f;
+            g_w = (p.wkind == GDR_GATE_SCALAR && valid) ? __bfloat162float(((const __nv_bfloat16*)p.wg)[gi])
+                  : (p.wkind == GDR_GATE_NONE ? 1.f : 0.f);
+        }
+    };
     if (tid == 0 && nchunks > 0) issue_loads(0);
+    if (nchunks > 0) load_scalar_gates(0);
 
 #define GDR_WAIT(bar, ph)                                                   \
     do {                                                                    \
@@ -241,18 +255,11 @@ __global__ void __launch_bounds__(NT, 1) chunk_fwd_kernel(
         const int n = min(C, T - t0);
         const uint32_t vbuf = sbase + OFF_V + (ci & 1) * 8192u;
         GDR_TRACE(0);
-        // ---- scalar gates of this chunk (plain loads) ----------------------
+        // ---- scalar gates of this chunk (loaded one chunk ahead) -----------
         if (tid < C) {
-            const int t = t0 + tid;
-            const bool valid = t < T;
-            const size_t gi = ((size_t)bb * T + t) * H + h;
-            const __nv_bfloat16* ap = (const __nv_bfloat16*)p.alpha;
-            const __nv_bfloat16* bp = (const __nv_bfloat16*)p.bg;
-            const __nv_bfloat16* wp = (const __nv_bfloat16*)p.wg;
-            s_ascal[tid] = (p.akind == GDR_GATE_SCALAR && valid) ? __bfloat162float(ap[gi]) : 1.f;
-            s_bscal[tid] = (p.bkind == GDR_GATE_SCALAR && valid) ? __bfloat162float(bp[gi]) : 0.f;
-            s_wscal[tid] = (p.wkind == GDR_GATE_SCALAR && valid) ? __bfloat162float(wp[gi])
-                           : (p.wkind == GDR_GATE_NONE ? 1.f : 0.f);
+            s_ascal[tid] = g_a;
+            s_bscal[tid] = g_b;
+            s_wscal[tid] = g_w;
         }
         GDR_WAIT(bar_tma, ph_tma);
         GDR_TRACE(1);
@@ -463,8 +470,6 @@ __global__ void __launch_bounds__(NT, 1) chunk_fwd_kernel(
         {
             float* A32 = reinterpret_cast<float*>(sm + OFF_A32);
             float* T32 = reinterpret_cast<float*>(sm + OFF_T32);
-            float* X16 = reinterpret_cast<float*>(sm + OFF_P32);          // [2][16 x 16]
-            float* Y32 = reinterpret_cast<float*>(sm + OFF_P32 + 2048);   // [32 x 32]
             if (tid < 64) {
                 const int I = tid >> 4, c = tid & 15;
                 float x[16];
@@ -501,101 +506,106 @@ __global__ void __launch_bounds__(NT, 1) chunk_fwd_kernel(
             }
             __syncthreads();
             GDR_TRACE(12);
-            // X_b = A_(2b+1)(2b) T_(2b)(2b), b = 0, 1: units of (row, 4 columns), 128 units
-            if (tid < 128) {
-                const int b = tid >> 6, rr = (tid >> 2) & 15, c4 = (tid & 3) * 4;
-                const int R = 32 * b + 16, Cc = 32 * b;
-                float acc[4] = {0.f, 0.f, 0.f, 0.f};
+            // Merges on warp-level tensor cores (tf32 operands, fp32 accumulate).
+            // One warp computes a 16 x 8 tile
+            //   D[i][j] = sum_k A[rA + i][cA + k] B[rB + k][cB + j],  k < 8 ksteps,
+            // reading A and B from the swizzled fp32 tiles (f32_at) or from a
+            // plain scratch tile with rows of kPad floats.
+            constexpr int kPad = 40;
+            const int lane = tid & 31, gq = lane >> 2, tq = lane & 3;
+            auto tile_mma = [&](float* Am, bool swzA, int rA, int cA, float* Bm, bool swzB, int rB,
+                                int cB, int ksteps, float* acc) {
 #pragma unroll
-                for (int m4 = 0; m4 < 16; m4 += 4) {
-                    const float4 a4 = *reinterpret_cast<const float4*>(f32_at(A32, R + rr, Cc + m4));
-                    const float av[4] = {a4.x, a4.y, a4.z, a4.w};
-#pragma unroll
-                    for (int mm = 0; mm < 4; ++mm) {
-                        const float4 t4 = *reinterpret_cast<const float4*>(f32_at(T32, Cc + m4 + mm, Cc + c4));
-                        acc[0] += av[mm] * t4.x; acc[1] += av[mm] * t4.y; acc[2] += av[mm] * t4.z; acc[3] += av[mm] * t4.w;
-                    }
+                for (int e = 0; e < 4; ++e) acc[e] = 0.f;
+                auto ldA = [&](int r, int c) { return swzA ? *f32_at(Am, r, c) : Am[r * kPad + c]; };
+                auto ldB = [&](int r, int c) { return swzB ? *f32_at(Bm, r, c) : Bm[r * kPad + c]; };
+                for (int ks = 0; ks < ksteps; ++ks) {
+                    const int k = 8 * ks;
+                    uint32_t a[4], b[2];
+                    a[0] = to_tf32(ldA(rA + gq, cA + k + tq));
+                    a[1] = to_tf32(ldA(rA + gq + 8, cA + k + tq));
+                    a[2] = to_tf32(ldA(rA + gq, cA + k + tq + 4));
+                    a[3] = to_tf32(ldA(rA + gq + 8, cA + k + tq + 4));
+                    b[0] = to_tf32(ldB(rB + k + tq, cB + gq));
+                    b[1] = to_tf32(ldB(rB + k + tq + 4, cB + gq));
+                    mma_tf32_m16n8k8(acc, a, b);
                 }
-                *reinterpret_cast<float4*>(X16 + b * 256 + rr * 16 + c4) = make_float4(acc[0], acc[1], acc[2], acc[3]);
+            };
+            float* XY = reinterpret_cast<float*>(sm + OFF_P32);  // X: [2][16 x kPad], later Y: [32 x kPad]
+            // 16 -> 32: X_b = A_(2b+1)(2b) T_(2b)(2b) (b = 0, 1), four 16 x 8 tiles
+            if (warp < 4) {
+                const int b = warp >> 1, nt = warp & 1;
+                const int R = 32 * b + 16, Cc = 32 * b;
+                float acc[4];
+                tile_mma(A32, true, R, Cc, T32, true, Cc, Cc + 8 * nt, 2, acc);
+                float* X = XY + b * 16 * kPad;
+                X[gq * kPad + 8 * nt + 2 * tq] = acc[0];
+                X[gq * kPad + 8 * nt + 2 * tq + 1] = acc[1];
+                X[(gq + 8) * kPad + 8 * nt + 2 * tq] = acc[2];
+                X[(gq + 8) * kPad + 8 * nt + 2 * tq + 1] = acc[3];
             }
             __syncthreads();
             // T_(2b+1)(2b) = -T_(2b+1)(2b+1) X_b
-            if (tid < 128) {
-                const int b = tid >> 6, rr = (tid >> 2) & 15, c4 = (tid & 3) * 4;
+            if (warp < 4) {
+                const int b = warp >> 1, nt = warp & 1;
                 const int R = 32 * b + 16, Cc = 32 * b;
-                float acc[4] = {0.f, 0.f, 0.f, 0.f};
-#pragma unroll
-                for (int m4 = 0; m4 < 16; m4 += 4) {
-                    const float4 t4 = *reinterpret_cast<const float4*>(f32_at(T32, R + rr, R + m4));
-                    const float tv[4] = {t4.x, t4.y, t4.z, t4.w};
-#pragma unroll
-                    for (int mm = 0; mm < 4; ++mm) {
-                        const float4 x4 = *reinterpret_cast<const float4*>(X16 + b * 256 + (m4 + mm) * 16 + c4);
-                        acc[0] += tv[mm] * x4.x; acc[1] += tv[mm] * x4.y; acc[2] += tv[mm] * x4.z; acc[3] += tv[mm] * x4.w;
-                    }
-                }
-                *reinterpret_cast<float4*>(f32_at(T32, R + rr, Cc + c4)) = make_float4(-acc[0], -acc[1], -acc[2], -acc[3]);
+                float acc[4];
+                tile_mma(T32, true, R, R, XY + b * 16 * kPad, false, 0, 8 * nt, 2, acc);
+                *f32_at(T32, R + gq, Cc + 8 * nt + 2 * tq) = -acc[0];
+                *f32_at(T32, R + gq, Cc + 8 * nt + 2 * tq + 1) = -acc[1];
+                *f32_at(T32, R + gq + 8, Cc + 8 * nt + 2 * tq) = -acc[2];
+                *f32_at(T32, R + gq + 8, Cc + 8 * nt + 2 * tq + 1) = -acc[3];
             }
             __syncthreads();
             GDR_TRACE(13);
-            // Y = A[32:64, 0:32] T[0:32, 0:32]: 256 units of (row, 4 columns)
+            // 32 -> 64: Y = A[32:64, 0:32] T[0:32, 0:32], eight 16 x 8 tiles (one per warp)
             {
-                const int rr = tid >> 3, c4 = (tid & 7) * 4;
-                float acc[4] = {0.f, 0.f, 0.f, 0.f};
-#pragma unroll
-                for (int m4 = 0; m4 < 32; m4 += 4) {
-                    const float4 a4 = *reinterpret_cast<const float4*>(f32_at(A32, 32 + rr, m4));
-                    const float av[4] = {a4.x, a4.y, a4.z, a4.w};
-#pragma unroll
-                    for (int mm = 0; mm < 4; ++mm) {
-                        const float4 t4 = *reinterpret_cast<const float4*>(f32_at(T32, m4 + mm, c4));
-                        acc[0] += av[mm] * t4.x; acc[1] += av[mm] * t4.y; acc[2] += av[mm] * t4.z; acc[3] += av[mm] * t4.w;
-                    }
-                }
-                *reinterpret_cast<float4*>(Y32 + rr * 32 + c4) = make_float4(acc[0], acc[1], acc[2], acc[3]);
+                const int mt = warp >> 2, nt = warp & 3;
+                float acc[4];
+                tile_mma(A32, true, 32 + 16 * mt, 0, T32, true, 0, 8 * nt, 4, acc);
+                XY[(16 * mt + gq) * kPad + 8 * nt + 2 * tq] = acc[0];
+                XY[(16 * mt + gq) * kPad + 8 * nt + 2 * tq + 1] = acc[1];
+                XY[(16 * mt + gq + 8) * kPad + 8 * nt + 2 * tq] = acc[2];
+                XY[(16 * mt + gq + 8) * kPad + 8 * nt + 2 * tq + 1] = acc[3];
             }
             __syncthreads();
             // T[32:64, 0:32] = -T[32:64, 32:64] Y
             {
-                const int rr = tid >> 3, c4 = (tid & 7) * 4;
-                float acc[4] = {0.f, 0.f, 0.f, 0.f};
-#pragma unroll
-                for (int m4 = 0; m4 < 32; m4 += 4) {
-                    const float4 t4 = *reinterpret_cast<const float4*>(f32_at(T32, 32 + rr, 32 + m4));
-                    const float tv[4] = {t4.x, t4.y, t4.z, t4.w};
-#pragma unroll
-                    for (int mm = 0; mm < 4; ++mm) {
-                        const float4 y4 = *reinterpret_cast<const float4*>(Y32 + (m4 + mm) * 32 + c4);
-                        acc[0] += tv[mm] * y4.x; acc[1] += tv[mm] * y4.y; acc[2] += tv[mm] * y4.z; acc[3] += tv[mm] * y4.w;
-                    }
-                }
-                *reinterpret_cast<float4*>(f32_at(T32, 32 + rr, c4)) = make_float4(-acc[0], -acc[1], -acc[2], -acc[3]);
+                const int mt = warp >> 2, nt = warp & 3;
+                float acc[4];
+                tile_mma(T32, true, 32 + 16 * mt, 32, XY, false, 0, 8 * nt, 4, acc);
+                *f32_at(T32, 32 + 16 * mt + gq, 8 * nt + 2 * tq) = -acc[0];
+                *f32_at(T32, 32 + 16 * mt + gq, 8 * nt + 2 * tq + 1) = -acc[1];
+                *f32_at(T32, 32 + 16 * mt + gq + 8, 8 * nt + 2 * tq) = -acc[2];
+                *f32_at(T32, 32 + 16 * mt + gq + 8, 8 * nt + 2 * tq + 1) = -acc[3];
             }
             __syncthreads();
             GDR_TRACE(14);
-            // L = [T ; 0] (bf16, 128 x 64); tied: APRE rows 0..63 = T Diag(beta)
-            if (tid < 128) {
-                float x[8];
+            // L = [T ; 0] (bf16, 128 x 64); tied: APRE rows 0..63 = T Diag(beta).
+            // Thread (row r = tid & 63, half = tid >> 6 of 4): chunks 2*half, 2*half+1.
+            {
+                const int r = tid & 63, q4 = tid >> 6;
 #pragma unroll
-                for (int c8 = 0; c8 < 8; ++c8) {
-                    if (tid < 64) {
+                for (int cc = 0; cc < 2; ++cc) {
+                    const int c8 = q4 * 2 + cc;
+                    float x[8];
 #pragma unroll
-                        for (int e4 = 0; e4 < 8; e4 += 4) {
-                            const int j = c8 * 8 + e4;
-                            // T is lower triangular: the upper-right 32x32 block is zero
-                            float4 t4 = (j < 32 || tid >= 32)
-                                            ? *reinterpret_cast<const float4*>(f32_at(T32, tid, j))
-                                            : make_float4(0.f, 0.f, 0.f, 0.f);
-                            x[e4] = t4.x; x[e4 + 1] = t4.y; x[e4 + 2] = t4.z; x[e4 + 3] = t4.w;
-                        }
-                        st_chunk(sm + OFF_L, sw128_chunk(tid, c8, 128), x);
-                        if (TIED) {
-#pragma unroll
-                            for (int e = 0; e < 8; ++e) x[e] *= s_bscal[c8 * 8 + e];
-                            st_chunk(sm + OFF_APRE, sw128_chunk(tid, c8, 128), x);
-                        }
-                    } else {
-                        st_zero_chunk(sm + OFF_L, sw128_chunk(tid, c8, 128));
+                    for (int e4 = 0; e4 < 8; e4 += 4) {
+                        const int j = c8 * 8 + e4;
+                        // T is lower triangular: the upper-right 32x32 block is zero
+                        float4 t4 = (j < 32 || r >= 32)
+                                        ? *reinterpret_cast<const float4*>(f32_at(T32, r, j))
+                                        : make_float4(0.f, 0.f, 0.f, 0.f);
+                        x[e4] = t4.x; x[e4 + 1] = t4.y; x[e4 + 2] = t4.z; x[e4 + 3] = t4.w;
+                    }
+                    st_chunk(sm + OFF_L, sw128_chunk(r, c8, 128), x);
+                    st_zero_chunk(sm + OFF_L, sw128_chunk(64 + r, c8, 128));
+                    if (TIED) {
+                        const float4 b0 = *reinterpret_cast<const float4*>(s_bscal + c8 * 8);
+                        const float4 b1 = *reinterpret_cast<const float4*>(s_bscal + c8 * 8 + 4);
+                        x[0] *= b0.x; x[1] *= b0.y; x[2] *= b0.z; x[3] *= b0.w;
+                        x[4] *= b1.x; x[5] *= b1.y; x[6] *= b1.z; x[7] *= b1.w;
+                        st_chunk(sm + OFF_APRE, sw128_chunk(r, c8, 128), x);
                     }
                 }
             }
@@ -628,6 +638,7 @@ __global__ void __launch_bounds__(NT, 1) chunk_fwd_kernel(
         GDR_TRACE(6);
         // the input region (A, T, L, Bm) is free: prefetch the next chunk
         if (tid == 0 && ci + 1 < nchunks) issue_loads(ci + 1);
+        if (ci + 1 < nchunks) load_scalar_gates(ci + 1);
 
         // ---- W -> [-W ; Qs.2^ref] in place of [Kb ; Qs]; general: -T Bm -> APRE -----
         if (row < 64) {
