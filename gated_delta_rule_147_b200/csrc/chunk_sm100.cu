@@ -53,7 +53,7 @@ constexpr uint32_t OFF_GW = 65536;     // channel w chunk
 constexpr uint32_t OFF_A32 = 0;        // A fp32 [64 x 64] (float4 groups swizzled by row)
 constexpr uint32_t OFF_T32 = 16384;    // T fp32 [64 x 64]
 constexpr uint32_t OFF_X = 32768;      // Bm bf16 [64 x 64] (general gates)
-constexpr uint32_t OFF_P32 = 40960;    // solve scratch fp32 (8 KB)
+constexpr uint32_t OFF_P32 = 40960;    // solve scratch fp32 (8 KB): transposed diagonal blocks, then X / Y
 constexpr uint32_t OFF_L = 49152;      // [T ; 0] bf16 [128 x 64]
 constexpr uint32_t OFF_V = 81920;      // v slice [64 x 64] bf16, two buffers
 constexpr uint32_t OFF_ROP = 98304;    // [Kb ; Qs] bf16 [128 x 128], later [-W ; Qs.2^ref]
@@ -62,7 +62,7 @@ constexpr uint32_t OFF_APRE = 163840;  // [T Diag(beta) ; 0] or [-T Bm ; Bq] bf1
 constexpr uint32_t OFF_AQ = 180224;    // [0 ; Aq] bf16 [128 x 64]
 constexpr uint32_t OFF_SBF = 196608;   // S bf16 [128 x 64]
 constexpr uint32_t OFF_U = 212992;     // U bf16 [64 x 64]
-constexpr uint32_t OFF_SCAN = 212992;  // scan scratch fp32 [17 x 128] (over U, during the build)
+constexpr uint32_t OFF_SCAN = 212992;  // scan scratch fp32 [9 x 128] (over U, during the build)
 constexpr uint32_t OFF_SMALL = 225792; // per-token / per-channel scalars, barriers
 constexpr uint32_t SMALL_BYTES = 4096;
 constexpr uint32_t SMEM_BYTES = OFF_SMALL + SMALL_BYTES + 1024;  // + alignment slack
@@ -128,7 +128,7 @@ __device__ __forceinline__ void ld_chunk(const uint8_t* base, uint32_t off, floa
     }
 }
 
-template <bool TIED>
+template <bool TIED, bool ACH>
 __global__ void __launch_bounds__(NT, 1) chunk_fwd_kernel(
     const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ CUtensorMap tm_k,
     const __grid_constant__ CUtensorMap tm_v, const __grid_constant__ CUtensorMap tm_a,
@@ -144,7 +144,8 @@ __global__ void __launch_bounds__(NT, 1) chunk_fwd_kernel(
     const int v0 = vt * NV;
     const int T = p.T, H = p.H;
     const int nchunks = (T + C - 1) / C;
-    const bool ach = p.akind == GDR_GATE_CHANNEL, bch = p.bkind == GDR_GATE_CHANNEL,
+    constexpr bool ach = ACH;  // channel-wise decay
+    const bool bch = p.bkind == GDR_GATE_CHANNEL,
                wch = p.wkind == GDR_GATE_CHANNEL;
     constexpr int N1 = TIED ? 64 : 128;  // rows of [Ks ; Kws]
 
@@ -221,19 +222,19 @@ __global__ void __launch_bounds__(NT, 1) chunk_fwd_kernel(
             }
         }
     }
-    // scalar gates travel in registers of threads 0..63 one chunk ahead
-    float g_a = 1.f, g_b = 0.f, g_w = 1.f;
+    // scalar gates travel as raw bf16 bits in registers of threads 0..63, loaded
+    // one chunk ahead from a clamped address and converted when the chunk starts
+    unsigned short g_a = 0, g_b = 0, g_w = 0;
     auto load_scalar_gates = [&](int ci) {
         if (tid < C) {
-            const int t = ci * C + tid;
-            const bool valid = t < T;
+            const int t = min(ci * C + tid, T - 1);
             const size_t gi = ((size_t)bb * T + t) * H + h;
-            g_a = (p.akind == GDR_GATE_SCALAR && valid) ? __bfloat162float(((const __nv_bfloat16*)p.alpha)[gi]) : 1.f;
-            g_b = (p.bkind == GDR_GATE_SCALAR && valid) ? __bfloat162float(((const __nv_bfloat16*)p.bg)[gi]) : 0.f;
-            g_w = (p.wkind == GDR_GATE_SCALAR && valid) ? __bfloat162float(((const __nv_bfloat16*)p.wg)[gi])
-                  : (p.wkind == GDR_GATE_NONE ? 1.f : 0.f);
+            if (p.akind == GDR_GATE_SCALAR) g_a = ((const unsigned short*)p.alpha)[gi];
+            if (p.bkind == GDR_GATE_SCALAR) g_b = ((const unsigned short*)p.bg)[gi];
+            if (p.wkind == GDR_GATE_SCALAR) g_w = ((const unsigned short*)p.wg)[gi];
         }
     };
+    auto bits_to_f32 = [](unsigned short u) { return __uint_as_float((uint32_t)u << 16); };
     if (tid == 0 && nchunks > 0) issue_loads(0);
     if (nchunks > 0) load_scalar_gates(0);
 
@@ -257,20 +258,39 @@ __global__ void __launch_bounds__(NT, 1) chunk_fwd_kernel(
         GDR_TRACE(0);
         // ---- scalar gates of this chunk (loaded one chunk ahead) -----------
         if (tid < C) {
-            s_ascal[tid] = g_a;
-            s_bscal[tid] = g_b;
-            s_wscal[tid] = g_w;
+            const bool valid = t0 + tid < T;
+            s_ascal[tid] = (p.akind == GDR_GATE_SCALAR && valid) ? bits_to_f32(g_a) : 1.f;
+            s_bscal[tid] = (p.bkind == GDR_GATE_SCALAR && valid) ? bits_to_f32(g_b) : 0.f;
+            s_wscal[tid] = (p.wkind == GDR_GATE_SCALAR && valid) ? bits_to_f32(g_w)
+                           : (p.wkind == GDR_GATE_NONE ? 1.f : 0.f);
         }
         GDR_WAIT(bar_tma, ph_tma);
         GDR_TRACE(1);
 
         // ---- build: log-decay scan and scaled operands --------------------
-        // thread = (channel group cg: 8 channels, token group rg: 4 tokens)
+        // thread = (token group rg = warp: 8 tokens, channel group cg = lane: 4 channels);
+        // a warp reads whole 256-byte token rows (conflict-free 8-byte pieces)
         {
-            const int cg = tid & 15, rg = tid >> 4;
-            const int ch0 = cg * 8;
-            float* scan = reinterpret_cast<float*>(sm + OFF_SCAN);  // [16 rg][128 ch] + [128]
-            float lrow[4][8];  // channel decay: l_r - ref
+            const int cg = tid & 31, rg = warp;
+            const int ch0 = cg * 4;
+            auto piece = [&](int r, int rows) {  // byte offset of channels ch0..ch0+3 of row r
+                return sw128_chunk(r, cg >> 1, rows) + (uint32_t)(cg & 1) * 8u;
+            };
+            auto ld4 = [&](uint32_t base, int r, float* x4) {
+                const uint2 u = *reinterpret_cast<const uint2*>(sm + base + piece(r, C));
+                const float2 f0 = __bfloat1622float2(*reinterpret_cast<const __nv_bfloat162*>(&u.x));
+                const float2 f1 = __bfloat1622float2(*reinterpret_cast<const __nv_bfloat162*>(&u.y));
+                x4[0] = f0.x; x4[1] = f0.y; x4[2] = f1.x; x4[3] = f1.y;
+            };
+            auto st4 = [&](uint32_t base, int r, int rows, const float* x4) {
+                uint2 u;
+                u.x = pack_bf16x2(x4[0], x4[1]);
+                u.y = pack_bf16x2(x4[2], x4[3]);
+                *reinterpret_cast<uint2*>(sm + base + piece(r, rows)) = u;
+            };
+            float* scan = reinterpret_cast<float*>(sm + OFF_SCAN);  // [8 rg][128 ch] + [128]
+            float lrow[8][4];  // channel decay: l_r - ref
+            float aval[8][4];  // channel decay: alpha of this thread's tokens
             if (!ach) {
                 // one decay per token: warp 0 scans the 64 tokens (2 per lane)
                 if (warp == 0) {
@@ -305,100 +325,103 @@ __global__ void __launch_bounds__(NT, 1) chunk_fwd_kernel(
                     s_fS[tid] = scan[2];
                 }
             } else {
-                float loc[8];
+                float loc[4] = {0.f, 0.f, 0.f, 0.f};
 #pragma unroll
-                for (int e = 0; e < 8; ++e) loc[e] = 0.f;
+                for (int i = 0; i < 8; ++i) {
+                    const int r = rg * 8 + i;
+                    ld4(OFF_GA, r, aval[i]);
 #pragma unroll
-                for (int i = 0; i < 4; ++i) {
-                    const int r = rg * 4 + i;
-                    float a8[8];
-                    ld_chunk(sm + OFF_GA, sw128_chunk(r, cg, C), a8);
-#pragma unroll
-                    for (int e = 0; e < 8; ++e) {
-                        loc[e] += (r < n) ? lg2_approx(a8[e]) : 0.f;
+                    for (int e = 0; e < 4; ++e) {
+                        if (r >= n) aval[i][e] = 1.f;  // padding tokens do not decay
+                        loc[e] += lg2_approx(aval[i][e]);
                         lrow[i][e] = loc[e];
                     }
                 }
-#pragma unroll
-                for (int e = 0; e < 8; ++e) scan[rg * 128 + ch0 + e] = loc[e];
-                if (rg == 0) {
-#pragma unroll
-                    for (int e = 0; e < 8; ++e) scan[2048 + ch0 + e] = lrow[0][e];
-                }
+                *reinterpret_cast<float4*>(scan + rg * 128 + ch0) = make_float4(loc[0], loc[1], loc[2], loc[3]);
+                if (rg == 0)
+                    *reinterpret_cast<float4*>(scan + 1024 + ch0) =
+                        make_float4(lrow[0][0], lrow[0][1], lrow[0][2], lrow[0][3]);
                 __syncthreads();
-                float pre[8], tot[8], ref[8];
-                bool bad = false;
+                float pre[4] = {0.f, 0.f, 0.f, 0.f}, tot[4] = {0.f, 0.f, 0.f, 0.f};
 #pragma unroll
-                for (int e = 0; e < 8; ++e) { pre[e] = 0.f; tot[e] = 0.f; }
+                for (int g = 0; g < 8; ++g) {
+                    const float4 x = *reinterpret_cast<const float4*>(scan + g * 128 + ch0);
+                    const float xs[4] = {x.x, x.y, x.z, x.w};
 #pragma unroll
-                for (int g = 0; g < 16; ++g) {
-                    const float4 xa = *reinterpret_cast<const float4*>(scan + g * 128 + ch0);
-                    const float4 xb = *reinterpret_cast<const float4*>(scan + g * 128 + ch0 + 4);
-                    const float xs[8] = {xa.x, xa.y, xa.z, xa.w, xb.x, xb.y, xb.z, xb.w};
-#pragma unroll
-                    for (int e = 0; e < 8; ++e) {
+                    for (int e = 0; e < 4; ++e) {
                         if (g < rg) pre[e] += xs[e];
                         tot[e] += xs[e];
                     }
                 }
+                const float4 l04 = *reinterpret_cast<const float4*>(scan + 1024 + ch0);
+                const float l0[4] = {l04.x, l04.y, l04.z, l04.w};
+                bool bad = false;
+                float ref[4];
 #pragma unroll
-                for (int e = 0; e < 8; ++e) {
-                    const float l0 = scan[2048 + ch0 + e];
-                    ref[e] = 0.5f * (l0 + tot[e]);  // tot = l_{n-1} (padding adds 0)
-                    bad |= (l0 - tot[e]) > 230.f;
+                for (int e = 0; e < 4; ++e) {
+                    ref[e] = 0.5f * (l0[e] + tot[e]);  // tot = l_{n-1} (padding adds 0)
+                    bad |= (l0[e] - tot[e]) > 230.f;
 #pragma unroll
-                    for (int i = 0; i < 4; ++i) lrow[i][e] += pre[e] - ref[e];
+                    for (int i = 0; i < 8; ++i) lrow[i][e] += pre[e] - ref[e];
                 }
                 if (bad) flag_status(p.d_status, GDR_DEVICE_DECAY_RANGE);
                 if (rg == 0) {
 #pragma unroll
-                    for (int e = 0; e < 8; ++e) {
+                    for (int e = 0; e < 4; ++e) {
                         s_eref[ch0 + e] = ex2_approx(ref[e]);
                         s_gC[ch0 + e] = ex2_approx(tot[e]);
                         s_fS[ch0 + e] = ex2_approx(tot[e] - ref[e]);
                     }
                 }
             }
+            float rowf_c[4];
 #pragma unroll
-            for (int i = 0; i < 4; ++i) {
-                const int r = rg * 4 + i;
-                float k8[8], q8[8], b8[8], w8[8];
-                ld_chunk(sm + OFF_KIN, sw128_chunk(r, cg, C), k8);
-                ld_chunk(sm + OFF_QIN, sw128_chunk(r, cg, C), q8);
-                if (bch) ld_chunk(sm + OFF_GB, sw128_chunk(r, cg, C), b8);
+            for (int i = 0; i < 8; ++i) {
+                const int r = rg * 8 + i;
+                float k4[4], q4[4], b4[4], w4[4];
+                ld4(OFF_KIN, r, k4);
+                ld4(OFF_QIN, r, q4);
+                if (bch) ld4(OFF_GB, r, b4);
                 else {
 #pragma unroll
-                    for (int e = 0; e < 8; ++e) b8[e] = s_bscal[r];
+                    for (int e = 0; e < 4; ++e) b4[e] = s_bscal[r];
                 }
                 if (!TIED) {
                     if (p.wkind == GDR_GATE_TIED) {
 #pragma unroll
-                        for (int e = 0; e < 8; ++e) w8[e] = b8[e];
+                        for (int e = 0; e < 4; ++e) w4[e] = b4[e];
                     } else if (wch) {
-                        ld_chunk(sm + OFF_GW, sw128_chunk(r, cg, C), w8);
+                        ld4(OFF_GW, r, w4);
                     } else {
 #pragma unroll
-                        for (int e = 0; e < 8; ++e) w8[e] = s_wscal[r];
+                        for (int e = 0; e < 4; ++e) w4[e] = s_wscal[r];
                     }
                 }
-                float rop_k[8], rop_q[8], cop_k[8], cop_w[8];
+                float rop_k[4], rop_q[4], cop_k[4], cop_w[4];
                 const bool valid = r < n;
                 const float rs = ach ? 0.f : s_rowf[r], cs = ach ? 0.f : s_colf[r];
+                if (ach) {
+                    // rowf by a multiply chain over this thread's 8 tokens (one exp2 per
+                    // chain), colf = 1 / rowf by Newton iterations on the FMA pipe
 #pragma unroll
-                for (int e = 0; e < 8; ++e) {
-                    const float rowf = ach ? ex2_approx(lrow[i][e]) : rs;
-                    const float colf = ach ? ex2_approx(-lrow[i][e]) : cs;
-                    const float kk = valid ? k8[e] : 0.f;
-                    const float qq = valid ? q8[e] : 0.f;
-                    rop_k[e] = b8[e] * kk * rowf;
+                    for (int e = 0; e < 4; ++e)
+                        rowf_c[e] = (i == 0) ? ex2_approx(lrow[0][e]) : rowf_c[e] * aval[i][e];
+                }
+#pragma unroll
+                for (int e = 0; e < 4; ++e) {
+                    const float rowf = ach ? rowf_c[e] : rs;
+                    const float colf = ach ? rcp_newton(rowf) : cs;
+                    const float kk = valid ? k4[e] : 0.f;
+                    const float qq = valid ? q4[e] : 0.f;
+                    rop_k[e] = b4[e] * kk * rowf;
                     rop_q[e] = qq * rowf;
                     cop_k[e] = kk * colf;
-                    cop_w[e] = TIED ? 0.f : w8[e] * kk * colf;
+                    cop_w[e] = TIED ? 0.f : w4[e] * kk * colf;
                 }
-                st_chunk(sm + OFF_ROP, sw128_chunk(r, cg, 128), rop_k);
-                st_chunk(sm + OFF_ROP, sw128_chunk(64 + r, cg, 128), rop_q);
-                st_chunk(sm + OFF_COP, sw128_chunk(r, cg, N1), cop_k);
-                if (!TIED) st_chunk(sm + OFF_COP, sw128_chunk(64 + r, cg, N1), cop_w);
+                st4(OFF_ROP, r, 128, rop_k);
+                st4(OFF_ROP, 64 + r, 128, rop_q);
+                st4(OFF_COP, r, N1, cop_k);
+                if (!TIED) st4(OFF_COP, 64 + r, N1, cop_w);
             }
         }
         GDR_BEFORE_MMA();
@@ -425,8 +448,10 @@ __global__ void __launch_bounds__(NT, 1) chunk_fwd_kernel(
         //      Aq -> AQ rows 64..127; general gates: Bm -> X, Bq -> APRE rows 64..127 ----
         {
             const int r = row & 63;
-            float d[32];
-            tmem_ld32(tmem + lane_base + TM_D1 + wg * 32, d);
+            float d[32], d2[32];
+            tmem_ld32_async(tmem + lane_base + TM_D1 + wg * 32, d);
+            if (!TIED) tmem_ld32_async(tmem + lane_base + TM_D1 + 64 + wg * 32, d2);
+            tmem_wait_ld();
             if (row < 64) {
                 float* A32 = reinterpret_cast<float*>(sm + OFF_A32);
 #pragma unroll
@@ -435,6 +460,19 @@ __global__ void __launch_bounds__(NT, 1) chunk_fwd_kernel(
                     float4 x = make_float4(j < r ? d[j4] : 0.f, j + 1 < r ? d[j4 + 1] : 0.f,
                                            j + 2 < r ? d[j4 + 2] : 0.f, j + 3 < r ? d[j4 + 3] : 0.f);
                     *reinterpret_cast<float4*>(f32_at(A32, r, j)) = x;
+                }
+                // transposed diagonal block: AT[I][j][rr] = A[16 I + rr][16 I + j]
+                const int I = r >> 4, rr = r & 15;
+                if ((I >> 1) == wg) {
+                    float* at = reinterpret_cast<float*>(sm + OFF_P32) + I * 272;
+                    // the block's 16 columns start at d[0] (even I) or d[16] (odd I)
+                    if (I & 1) {
+#pragma unroll
+                        for (int j = 0; j < 16; ++j) at[j * 16 + rr] = j < rr ? d[16 + j] : 0.f;
+                    } else {
+#pragma unroll
+                        for (int j = 0; j < 16; ++j) at[j * 16 + rr] = j < rr ? d[j] : 0.f;
+                    }
                 }
             } else {
                 float x[8];
@@ -446,14 +484,13 @@ __global__ void __launch_bounds__(NT, 1) chunk_fwd_kernel(
                 }
             }
             if (!TIED) {
-                tmem_ld32(tmem + lane_base + TM_D1 + 64 + wg * 32, d);
                 float x[8];
 #pragma unroll
                 for (int c8 = 0; c8 < 4; ++c8) {
 #pragma unroll
                     for (int e = 0; e < 8; ++e) {
                         const int j = wg * 32 + c8 * 8 + e;
-                        x[e] = (row < 64 ? j < r : j <= r) ? d[c8 * 8 + e] : 0.f;
+                        x[e] = (row < 64 ? j < r : j <= r) ? d2[c8 * 8 + e] : 0.f;
                     }
                     if (row < 64) st_chunk(sm + OFF_X, sw128_chunk(r, wg * 4 + c8, 64), x);   // Bm
                     else st_chunk(sm + OFF_APRE, sw128_chunk(row, wg * 4 + c8, 128), x);     // Bq
@@ -471,27 +508,24 @@ __global__ void __launch_bounds__(NT, 1) chunk_fwd_kernel(
             float* A32 = reinterpret_cast<float*>(sm + OFF_A32);
             float* T32 = reinterpret_cast<float*>(sm + OFF_T32);
             if (tid < 64) {
+                // diagonal block I, column c: right-looking substitution; column j
+                // of the block is a contiguous row of the transposed copy AT
                 const int I = tid >> 4, c = tid & 15;
-                float x[16];
+                const float* at = reinterpret_cast<const float*>(sm + OFF_P32) + I * 272;
+                float acc[16], x[16];
 #pragma unroll
-                for (int j = 0; j < 16; ++j) x[j] = 0.f;
+                for (int rr = 0; rr < 16; ++rr) acc[rr] = 0.f;
 #pragma unroll
-                for (int rr = 0; rr < 16; ++rr) {
+                for (int j = 0; j < 16; ++j) {
+                    x[j] = ((j == c) ? 1.f : 0.f) - acc[j];
                     float a[16];
 #pragma unroll
-                    for (int j4 = 0; j4 < 16; j4 += 4) {
-                        const float4 v4 = *reinterpret_cast<const float4*>(f32_at(A32, 16 * I + rr, 16 * I + j4));
-                        a[j4] = v4.x; a[j4 + 1] = v4.y; a[j4 + 2] = v4.z; a[j4 + 3] = v4.w;
+                    for (int r4 = 0; r4 < 16; r4 += 4) {
+                        const float4 v4 = *reinterpret_cast<const float4*>(at + j * 16 + r4);
+                        a[r4] = v4.x; a[r4 + 1] = v4.y; a[r4 + 2] = v4.z; a[r4 + 3] = v4.w;
                     }
-                    float s0 = 0.f, s1 = 0.f, s2 = 0.f, s3 = 0.f;
 #pragma unroll
-                    for (int j = 0; j < rr; j += 4) {
-                        s0 += a[j] * x[j];
-                        if (j + 1 < rr) s1 += a[j + 1] * x[j + 1];
-                        if (j + 2 < rr) s2 += a[j + 2] * x[j + 2];
-                        if (j + 3 < rr) s3 += a[j + 3] * x[j + 3];
-                    }
-                    x[rr] = ((rr == c) ? 1.f : 0.f) - ((s0 + s1) + (s2 + s3));
+                    for (int rr = j + 1; rr < 16; ++rr) acc[rr] += a[rr] * x[j];
                 }
 #pragma unroll
                 for (int rr = 0; rr < 16; ++rr) *f32_at(T32, 16 * I + rr, 16 * I + c) = x[rr];
@@ -633,6 +667,32 @@ __global__ void __launch_bounds__(NT, 1) chunk_fwd_kernel(
             }
             mma_commit(bar_mma);
         }
+        // ---- while P2 runs: Qs.2^ref in place (rows 64..127 of [Kb ; Qs], not read by P2)
+        auto load_eref = [&](int c0, float* er) {
+            if (ach) {
+                const float4 e0 = *reinterpret_cast<const float4*>(s_eref + c0);
+                const float4 e1 = *reinterpret_cast<const float4*>(s_eref + c0 + 4);
+                er[0] = e0.x; er[1] = e0.y; er[2] = e0.z; er[3] = e0.w;
+                er[4] = e1.x; er[5] = e1.y; er[6] = e1.z; er[7] = e1.w;
+            } else {
+                const float e = s_eref[0];
+#pragma unroll
+                for (int i = 0; i < 8; ++i) er[i] = e;
+            }
+        };
+        if (row >= 64) {
+#pragma unroll
+            for (int c = 0; c < 8; ++c) {
+                const int ch = wg * 8 + c;
+                float x[8], er[8];
+                const uint32_t off = sw128_chunk(row, ch, 128);
+                ld_chunk(sm + OFF_ROP, off, x);
+                load_eref(ch * 8, er);
+#pragma unroll
+                for (int e = 0; e < 8; ++e) x[e] *= er[e];
+                st_chunk(sm + OFF_ROP, off, x);
+            }
+        }
         GDR_WAIT(bar_mma, ph_mma);
         tc_fence_after();
         GDR_TRACE(6);
@@ -640,41 +700,34 @@ __global__ void __launch_bounds__(NT, 1) chunk_fwd_kernel(
         if (tid == 0 && ci + 1 < nchunks) issue_loads(ci + 1);
         if (ci + 1 < nchunks) load_scalar_gates(ci + 1);
 
-        // ---- W -> [-W ; Qs.2^ref] in place of [Kb ; Qs]; general: -T Bm -> APRE -----
+        // ---- W -> -W.2^ref in place of Kb (rows 0..63); general: -T Bm -> APRE -----
         if (row < 64) {
-            float d[32];
+            float d[32], d1[32], d2[32];
+            tmem_ld32_async(tmem + lane_base + TM_D2 + wg * 64, d);
+            tmem_ld32_async(tmem + lane_base + TM_D2 + wg * 64 + 32, d1);
+            if (!TIED) tmem_ld32_async(tmem + lane_base + TM_D2 + 128 + wg * 32, d2);
+            tmem_wait_ld();
 #pragma unroll
             for (int cb = 0; cb < 2; ++cb) {
                 const int col = wg * 64 + cb * 32;
-                tmem_ld32(tmem + lane_base + TM_D2 + col, d);
+                const float* dd = cb ? d1 : d;
 #pragma unroll
                 for (int c4 = 0; c4 < 4; ++c4) {
-                    float x[8];
+                    float x[8], er[8];
+                    load_eref(col + c4 * 8, er);
 #pragma unroll
-                    for (int e = 0; e < 8; ++e) x[e] = -d[c4 * 8 + e] * s_eref[col + c4 * 8 + e];
+                    for (int e = 0; e < 8; ++e) x[e] = -dd[c4 * 8 + e] * er[e];
                     st_chunk(sm + OFF_ROP, sw128_chunk(row, col / 8 + c4, 128), x);
                 }
             }
             if (!TIED) {
-                tmem_ld32(tmem + lane_base + TM_D2 + 128 + wg * 32, d);
 #pragma unroll
                 for (int c4 = 0; c4 < 4; ++c4) {
                     float x[8];
 #pragma unroll
-                    for (int e = 0; e < 8; ++e) x[e] = -d[c4 * 8 + e];
+                    for (int e = 0; e < 8; ++e) x[e] = -d2[c4 * 8 + e];
                     st_chunk(sm + OFF_APRE, sw128_chunk(row, wg * 4 + c4, 128), x);
                 }
-            }
-        } else {
-#pragma unroll
-            for (int c = 0; c < 8; ++c) {
-                const int ch = wg * 8 + c;
-                float x[8];
-                const uint32_t off = sw128_chunk(row, ch, 128);
-                ld_chunk(sm + OFF_ROP, off, x);
-#pragma unroll
-                for (int e = 0; e < 8; ++e) x[e] *= s_eref[ch * 8 + e];
-                st_chunk(sm + OFF_ROP, off, x);
             }
         }
         GDR_BEFORE_MMA();
@@ -734,9 +787,11 @@ __global__ void __launch_bounds__(NT, 1) chunk_fwd_kernel(
 
         // ---- O (rows 64..127 of D3) -> global; state update from D4 -----------------
         {
-            float d[32];
+            float d[32], dS[32];
+            if (row >= 64) tmem_ld32_async(tmem + lane_base + TM_D3 + wg * 32, d);
+            tmem_ld32_async(tmem + lane_base + TM_D4 + wg * 32, dS);
+            tmem_wait_ld();
             if (row >= 64) {
-                tmem_ld32(tmem + lane_base + TM_D3 + wg * 32, d);
                 const int t = t0 + row - 64;
                 if (t < T) {
                     __nv_bfloat16* op = p.o + (((size_t)bb * T + t) * H + h) * p.dv + v0 + wg * 32;
@@ -751,10 +806,9 @@ __global__ void __launch_bounds__(NT, 1) chunk_fwd_kernel(
                     }
                 }
             }
-            tmem_ld32(tmem + lane_base + TM_D4 + wg * 32, d);
             const float gC = s_gC[row], fS = s_fS[row];
 #pragma unroll
-            for (int j = 0; j < NH; ++j) S[j] = gC * S[j] + fS * d[j];
+            for (int j = 0; j < NH; ++j) S[j] = gC * S[j] + fS * dS[j];
 #pragma unroll
             for (int ch = 0; ch < 4; ++ch) st_chunk(sm + OFF_SBF, sw128_chunk(row, wg * 4 + ch, DK), &S[8 * ch]);
         }
@@ -791,16 +845,17 @@ cudaError_t launch_chunk_sm100(const CUtensorMap* maps, const void* alpha, const
     p.B = B; p.T = T; p.H = H; p.dv = dv;
     p.akind = akind; p.bkind = bkind; p.wkind = wkind;
     dim3 grid(dv / chunk::NV, H, B);
+    const bool ach = akind == GDR_GATE_CHANNEL;
+    auto launch = [&](auto kern) -> cudaError_t {
+        cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, chunk::SMEM_BYTES);
+        if (e != cudaSuccess) return e;
+        kern<<<grid, chunk::NT, chunk::SMEM_BYTES, st>>>(maps[0], maps[1], maps[2], maps[3], maps[4], maps[5], p);
+        return cudaSuccess;
+    };
     cudaError_t e;
-    if (tied) {
-        e = cudaFuncSetAttribute(chunk::chunk_fwd_kernel<true>, cudaFuncAttributeMaxDynamicSharedMemorySize, chunk::SMEM_BYTES);
-        if (e != cudaSuccess) return e;
-        chunk::chunk_fwd_kernel<true><<<grid, chunk::NT, chunk::SMEM_BYTES, st>>>(maps[0], maps[1], maps[2], maps[3], maps[4], maps[5], p);
-    } else {
-        e = cudaFuncSetAttribute(chunk::chunk_fwd_kernel<false>, cudaFuncAttributeMaxDynamicSharedMemorySize, chunk::SMEM_BYTES);
-        if (e != cudaSuccess) return e;
-        chunk::chunk_fwd_kernel<false><<<grid, chunk::NT, chunk::SMEM_BYTES, st>>>(maps[0], maps[1], maps[2], maps[3], maps[4], maps[5], p);
-    }
+    if (tied) e = ach ? launch(chunk::chunk_fwd_kernel<true, true>) : launch(chunk::chunk_fwd_kernel<true, false>);
+    else e = ach ? launch(chunk::chunk_fwd_kernel<false, true>) : launch(chunk::chunk_fwd_kernel<false, false>);
+    if (e != cudaSuccess) return e;
     return cudaGetLastError();
 }
 

@@ -48,6 +48,17 @@ __device__ __forceinline__ float lg2_approx(float x) {
     return y;
 }
 
+// 1/a for positive normal a by Newton-Raphson, x <- x (2 - a x), from a seed
+// that flips the exponent bits (relative error of the seed below 1/8, so
+// three steps reach fp32 precision). Runs on the FMA pipe.
+__device__ __forceinline__ float rcp_newton(float a) {
+    float x = __int_as_float(0x7EF311C7 - __float_as_int(a));
+    x = x * fmaf(-a, x, 2.f);
+    x = x * fmaf(-a, x, 2.f);
+    x = x * fmaf(-a, x, 2.f);
+    return x;
+}
+
 __device__ __forceinline__ uint32_t pack_bf16x2(float lo, float hi) {
     __nv_bfloat162 h = __floats2bfloat162_rn(lo, hi);
     return *reinterpret_cast<uint32_t*>(&h);
@@ -185,8 +196,9 @@ __device__ __forceinline__ void mma_commit(uint64_t* bar) {
         : "memory");
 }
 
-// Loads 32 consecutive fp32 columns of this thread's TMEM lane.
-__device__ __forceinline__ void tmem_ld32(uint32_t taddr, float* v) {
+// Starts a load of 32 consecutive fp32 columns of this thread's TMEM lane;
+// the registers are valid after tmem_wait_ld().
+__device__ __forceinline__ void tmem_ld32_async(uint32_t taddr, float* v) {
     uint32_t r[32];
     asm volatile(
         "tcgen05.ld.sync.aligned.32x32b.x32.b32"
@@ -198,9 +210,18 @@ __device__ __forceinline__ void tmem_ld32(uint32_t taddr, float* v) {
           "=r"(r[20]), "=r"(r[21]), "=r"(r[22]), "=r"(r[23]), "=r"(r[24]), "=r"(r[25]),
           "=r"(r[26]), "=r"(r[27]), "=r"(r[28]), "=r"(r[29]), "=r"(r[30]), "=r"(r[31])
         : "r"(taddr));
-    asm volatile("tcgen05.wait::ld.sync.aligned;" ::: "memory");
 #pragma unroll
     for (int i = 0; i < 32; ++i) v[i] = __uint_as_float(r[i]);
+}
+
+__device__ __forceinline__ void tmem_wait_ld() {
+    asm volatile("tcgen05.wait::ld.sync.aligned;" ::: "memory");
+}
+
+// Loads 32 consecutive fp32 columns of this thread's TMEM lane and waits.
+__device__ __forceinline__ void tmem_ld32(uint32_t taddr, float* v) {
+    tmem_ld32_async(taddr, v);
+    tmem_wait_ld();
 }
 
 // Warp-level D += A * B with tf32 operands and fp32 accumulation (m16n8k8).
