@@ -17,7 +17,8 @@ GDR_DEVICE_TIMEOUT, GDR_DEVICE_DECAY_RANGE = 1, 2
 GDR_BF16, GDR_FP32 = 0, 1
 GATE_NONE, GATE_SCALAR, GATE_CHANNEL, GATE_TIED = 0, 1, 2, 3
 
-EXPORTS = ("gdr_chunk_fwd", "gdr_decode_step", "gdr_status_string", "gdr_version")
+EXPORTS = ("gdr_chunk_fwd", "gdr_decode_step", "gdr_selftest_bounded_wait", "gdr_status_string",
+           "gdr_version")
 
 _lock = threading.Lock()
 _handle = None
@@ -52,6 +53,8 @@ def load(build_if_missing: bool = True) -> ctypes.CDLL:
         lib.gdr_status_string.argtypes = [ip]
         lib.gdr_status_string.restype = ctypes.c_char_p
         lib.gdr_version.restype = ip
+        lib.gdr_selftest_bounded_wait.argtypes = [vp, vp]
+        lib.gdr_selftest_bounded_wait.restype = ip
         _handle = lib
         return lib
 
@@ -93,3 +96,9 @@ def gdr_decode_step(q, k, v, alpha, b, w, alpha_kind, b_kind, w_kind, S, o, B, H
                                 _stream(stream))
     if st != GDR_OK:
         raise GdrError("gdr_decode_step", st)
+
+
+def gdr_selftest_bounded_wait(d_status, stream=None) -> None:
+    st = load().gdr_selftest_bounded_wait(_p(d_status), _stream(stream))
+    if st != GDR_OK:
+        raise GdrError("gdr_selftest_bounded_wait", st)

@@ -128,6 +128,123 @@ __device__ __forceinline__ void ld_chunk(const uint8_t* base, uint32_t off, floa
     }
 }
 
+// T = (I + A)^-1 for the strictly lower 64 x 64 matrix A (fp32, swizzled rows,
+// with its 16 x 16 diagonal blocks also stored transposed at scr[I * 272 +
+// j * 16 + rr]) into T32: right-looking forward substitution on the diagonal
+// blocks, then recursive halving 16 -> 32 -> 64 on warp-level tensor cores.
+// Called by all 256 threads; ends with a block barrier.
+__device__ __forceinline__ void solve_unit_lower(float* A32, float* T32, float* scr, int tid, int warp,
+                                                 int ci) {
+    (void)ci;
+    if (tid < 64) {
+        // diagonal block I, column c: right-looking substitution; column j
+        // of the block is a contiguous row of the transposed copy AT
+        const int I = tid >> 4, c = tid & 15;
+        const float* at = scr + I * 272;
+        float acc[16], x[16];
+#pragma unroll
+        for (int rr = 0; rr < 16; ++rr) acc[rr] = 0.f;
+#pragma unroll
+        for (int j = 0; j < 16; ++j) {
+            x[j] = ((j == c) ? 1.f : 0.f) - acc[j];
+            float a[16];
+#pragma unroll
+            for (int r4 = 0; r4 < 16; r4 += 4) {
+                const float4 v4 = *reinterpret_cast<const float4*>(at + j * 16 + r4);
+                a[r4] = v4.x; a[r4 + 1] = v4.y; a[r4 + 2] = v4.z; a[r4 + 3] = v4.w;
+            }
+#pragma unroll
+            for (int rr = j + 1; rr < 16; ++rr) acc[rr] += a[rr] * x[j];
+        }
+#pragma unroll
+        for (int rr = 0; rr < 16; ++rr) *f32_at(T32, 16 * I + rr, 16 * I + c) = x[rr];
+    } else if (tid < 128) {
+        // the strictly upper 16x16 blocks inside each 32x32 diagonal half are zero
+        const int u = tid - 64;                        // 64 threads, 2 blocks x 16 rows x 4 float4
+        for (int idx = u; idx < 128; idx += 64) {
+            const int blk = idx >> 6, rr = (idx >> 2) & 15, c4 = (idx & 3) * 4;
+            *reinterpret_cast<float4*>(f32_at(T32, 32 * blk + rr, 32 * blk + 16 + c4)) =
+                make_float4(0.f, 0.f, 0.f, 0.f);
+        }
+    }
+    __syncthreads();
+    GDR_TRACE(12);
+    // Merges on warp-level tensor cores (tf32 operands, fp32 accumulate).
+    // One warp computes a 16 x 8 tile
+    //   D[i][j] = sum_k A[rA + i][cA + k] B[rB + k][cB + j],  k < 8 ksteps,
+    // reading A and B from the swizzled fp32 tiles (f32_at) or from a
+    // plain scratch tile with rows of kPad floats.
+    constexpr int kPad = 40;
+    const int lane = tid & 31, gq = lane >> 2, tq = lane & 3;
+    auto tile_mma = [&](float* Am, bool swzA, int rA, int cA, float* Bm, bool swzB, int rB,
+                        int cB, int ksteps, float* acc) {
+#pragma unroll
+        for (int e = 0; e < 4; ++e) acc[e] = 0.f;
+        auto ldA = [&](int r, int c) { return swzA ? *f32_at(Am, r, c) : Am[r * kPad + c]; };
+        auto ldB = [&](int r, int c) { return swzB ? *f32_at(Bm, r, c) : Bm[r * kPad + c]; };
+        for (int ks = 0; ks < ksteps; ++ks) {
+            const int k = 8 * ks;
+            uint32_t a[4], b[2];
+            a[0] = to_tf32(ldA(rA + gq, cA + k + tq));
+            a[1] = to_tf32(ldA(rA + gq + 8, cA + k + tq));
+            a[2] = to_tf32(ldA(rA + gq, cA + k + tq + 4));
+            a[3] = to_tf32(ldA(rA + gq + 8, cA + k + tq + 4));
+            b[0] = to_tf32(ldB(rB + k + tq, cB + gq));
+            b[1] = to_tf32(ldB(rB + k + tq + 4, cB + gq));
+            mma_tf32_m16n8k8(acc, a, b);
+        }
+    };
+    float* XY = scr;  // X: [2][16 x kPad], later Y: [32 x kPad]
+    // 16 -> 32: X_b = A_(2b+1)(2b) T_(2b)(2b) (b = 0, 1), four 16 x 8 tiles
+    if (warp < 4) {
+        const int b = warp >> 1, nt = warp & 1;
+        const int R = 32 * b + 16, Cc = 32 * b;
+        float acc[4];
+        tile_mma(A32, true, R, Cc, T32, true, Cc, Cc + 8 * nt, 2, acc);
+        float* X = XY + b * 16 * kPad;
+        X[gq * kPad + 8 * nt + 2 * tq] = acc[0];
+        X[gq * kPad + 8 * nt + 2 * tq + 1] = acc[1];
+        X[(gq + 8) * kPad + 8 * nt + 2 * tq] = acc[2];
+        X[(gq + 8) * kPad + 8 * nt + 2 * tq + 1] = acc[3];
+    }
+    __syncthreads();
+    // T_(2b+1)(2b) = -T_(2b+1)(2b+1) X_b
+    if (warp < 4) {
+        const int b = warp >> 1, nt = warp & 1;
+        const int R = 32 * b + 16, Cc = 32 * b;
+        float acc[4];
+        tile_mma(T32, true, R, R, XY + b * 16 * kPad, false, 0, 8 * nt, 2, acc);
+        *f32_at(T32, R + gq, Cc + 8 * nt + 2 * tq) = -acc[0];
+        *f32_at(T32, R + gq, Cc + 8 * nt + 2 * tq + 1) = -acc[1];
+        *f32_at(T32, R + gq + 8, Cc + 8 * nt + 2 * tq) = -acc[2];
+        *f32_at(T32, R + gq + 8, Cc + 8 * nt + 2 * tq + 1) = -acc[3];
+    }
+    __syncthreads();
+    GDR_TRACE(13);
+    // 32 -> 64: Y = A[32:64, 0:32] T[0:32, 0:32], eight 16 x 8 tiles (one per warp)
+    {
+        const int mt = warp >> 2, nt = warp & 3;
+        float acc[4];
+        tile_mma(A32, true, 32 + 16 * mt, 0, T32, true, 0, 8 * nt, 4, acc);
+        XY[(16 * mt + gq) * kPad + 8 * nt + 2 * tq] = acc[0];
+        XY[(16 * mt + gq) * kPad + 8 * nt + 2 * tq + 1] = acc[1];
+        XY[(16 * mt + gq + 8) * kPad + 8 * nt + 2 * tq] = acc[2];
+        XY[(16 * mt + gq + 8) * kPad + 8 * nt + 2 * tq + 1] = acc[3];
+    }
+    __syncthreads();
+    // T[32:64, 0:32] = -T[32:64, 32:64] Y
+    {
+        const int mt = warp >> 2, nt = warp & 3;
+        float acc[4];
+        tile_mma(T32, true, 32 + 16 * mt, 32, XY, false, 0, 8 * nt, 4, acc);
+        *f32_at(T32, 32 + 16 * mt + gq, 8 * nt + 2 * tq) = -acc[0];
+        *f32_at(T32, 32 + 16 * mt + gq, 8 * nt + 2 * tq + 1) = -acc[1];
+        *f32_at(T32, 32 + 16 * mt + gq + 8, 8 * nt + 2 * tq) = -acc[2];
+        *f32_at(T32, 32 + 16 * mt + gq + 8, 8 * nt + 2 * tq + 1) = -acc[3];
+    }
+    __syncthreads();
+}
+
 template <bool TIED, bool ACH>
 __global__ void __launch_bounds__(NT, 1) chunk_fwd_kernel(
     const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ CUtensorMap tm_k,
@@ -507,113 +624,7 @@ __global__ void __launch_bounds__(NT, 1) chunk_fwd_kernel(
         {
             float* A32 = reinterpret_cast<float*>(sm + OFF_A32);
             float* T32 = reinterpret_cast<float*>(sm + OFF_T32);
-            if (tid < 64) {
-                // diagonal block I, column c: right-looking substitution; column j
-                // of the block is a contiguous row of the transposed copy AT
-                const int I = tid >> 4, c = tid & 15;
-                const float* at = reinterpret_cast<const float*>(sm + OFF_P32) + I * 272;
-                float acc[16], x[16];
-#pragma unroll
-                for (int rr = 0; rr < 16; ++rr) acc[rr] = 0.f;
-#pragma unroll
-                for (int j = 0; j < 16; ++j) {
-                    x[j] = ((j == c) ? 1.f : 0.f) - acc[j];
-                    float a[16];
-#pragma unroll
-                    for (int r4 = 0; r4 < 16; r4 += 4) {
-                        const float4 v4 = *reinterpret_cast<const float4*>(at + j * 16 + r4);
-                        a[r4] = v4.x; a[r4 + 1] = v4.y; a[r4 + 2] = v4.z; a[r4 + 3] = v4.w;
-                    }
-#pragma unroll
-                    for (int rr = j + 1; rr < 16; ++rr) acc[rr] += a[rr] * x[j];
-                }
-#pragma unroll
-                for (int rr = 0; rr < 16; ++rr) *f32_at(T32, 16 * I + rr, 16 * I + c) = x[rr];
-            } else if (tid < 128) {
-                // the strictly upper 16x16 blocks inside each 32x32 diagonal half are zero
-                const int u = tid - 64;                        // 64 threads, 2 blocks x 16 rows x 4 float4
-                for (int idx = u; idx < 128; idx += 64) {
-                    const int blk = idx >> 6, rr = (idx >> 2) & 15, c4 = (idx & 3) * 4;
-                    *reinterpret_cast<float4*>(f32_at(T32, 32 * blk + rr, 32 * blk + 16 + c4)) =
-                        make_float4(0.f, 0.f, 0.f, 0.f);
-                }
-            }
-            __syncthreads();
-            GDR_TRACE(12);
-            // Merges on warp-level tensor cores (tf32 operands, fp32 accumulate).
-            // One warp computes a 16 x 8 tile
-            //   D[i][j] = sum_k A[rA + i][cA + k] B[rB + k][cB + j],  k < 8 ksteps,
-            // reading A and B from the swizzled fp32 tiles (f32_at) or from a
-            // plain scratch tile with rows of kPad floats.
-            constexpr int kPad = 40;
-            const int lane = tid & 31, gq = lane >> 2, tq = lane & 3;
-            auto tile_mma = [&](float* Am, bool swzA, int rA, int cA, float* Bm, bool swzB, int rB,
-                                int cB, int ksteps, float* acc) {
-#pragma unroll
-                for (int e = 0; e < 4; ++e) acc[e] = 0.f;
-                auto ldA = [&](int r, int c) { return swzA ? *f32_at(Am, r, c) : Am[r * kPad + c]; };
-                auto ldB = [&](int r, int c) { return swzB ? *f32_at(Bm, r, c) : Bm[r * kPad + c]; };
-                for (int ks = 0; ks < ksteps; ++ks) {
-                    const int k = 8 * ks;
-                    uint32_t a[4], b[2];
-                    a[0] = to_tf32(ldA(rA + gq, cA + k + tq));
-                    a[1] = to_tf32(ldA(rA + gq + 8, cA + k + tq));
-                    a[2] = to_tf32(ldA(rA + gq, cA + k + tq + 4));
-                    a[3] = to_tf32(ldA(rA + gq + 8, cA + k + tq + 4));
-                    b[0] = to_tf32(ldB(rB + k + tq, cB + gq));
-                    b[1] = to_tf32(ldB(rB + k + tq + 4, cB + gq));
-                    mma_tf32_m16n8k8(acc, a, b);
-                }
-            };
-            float* XY = reinterpret_cast<float*>(sm + OFF_P32);  // X: [2][16 x kPad], later Y: [32 x kPad]
-            // 16 -> 32: X_b = A_(2b+1)(2b) T_(2b)(2b) (b = 0, 1), four 16 x 8 tiles
-            if (warp < 4) {
-                const int b = warp >> 1, nt = warp & 1;
-                const int R = 32 * b + 16, Cc = 32 * b;
-                float acc[4];
-                tile_mma(A32, true, R, Cc, T32, true, Cc, Cc + 8 * nt, 2, acc);
-                float* X = XY + b * 16 * kPad;
-                X[gq * kPad + 8 * nt + 2 * tq] = acc[0];
-                X[gq * kPad + 8 * nt + 2 * tq + 1] = acc[1];
-                X[(gq + 8) * kPad + 8 * nt + 2 * tq] = acc[2];
-                X[(gq + 8) * kPad + 8 * nt + 2 * tq + 1] = acc[3];
-            }
-            __syncthreads();
-            // T_(2b+1)(2b) = -T_(2b+1)(2b+1) X_b
-            if (warp < 4) {
-                const int b = warp >> 1, nt = warp & 1;
-                const int R = 32 * b + 16, Cc = 32 * b;
-                float acc[4];
-                tile_mma(T32, true, R, R, XY + b * 16 * kPad, false, 0, 8 * nt, 2, acc);
-                *f32_at(T32, R + gq, Cc + 8 * nt + 2 * tq) = -acc[0];
-                *f32_at(T32, R + gq, Cc + 8 * nt + 2 * tq + 1) = -acc[1];
-                *f32_at(T32, R + gq + 8, Cc + 8 * nt + 2 * tq) = -acc[2];
-                *f32_at(T32, R + gq + 8, Cc + 8 * nt + 2 * tq + 1) = -acc[3];
-            }
-            __syncthreads();
-            GDR_TRACE(13);
-            // 32 -> 64: Y = A[32:64, 0:32] T[0:32, 0:32], eight 16 x 8 tiles (one per warp)
-            {
-                const int mt = warp >> 2, nt = warp & 3;
-                float acc[4];
-                tile_mma(A32, true, 32 + 16 * mt, 0, T32, true, 0, 8 * nt, 4, acc);
-                XY[(16 * mt + gq) * kPad + 8 * nt + 2 * tq] = acc[0];
-                XY[(16 * mt + gq) * kPad + 8 * nt + 2 * tq + 1] = acc[1];
-                XY[(16 * mt + gq + 8) * kPad + 8 * nt + 2 * tq] = acc[2];
-                XY[(16 * mt + gq + 8) * kPad + 8 * nt + 2 * tq + 1] = acc[3];
-            }
-            __syncthreads();
-            // T[32:64, 0:32] = -T[32:64, 32:64] Y
-            {
-                const int mt = warp >> 2, nt = warp & 3;
-                float acc[4];
-                tile_mma(T32, true, 32 + 16 * mt, 32, XY, false, 0, 8 * nt, 4, acc);
-                *f32_at(T32, 32 + 16 * mt + gq, 8 * nt + 2 * tq) = -acc[0];
-                *f32_at(T32, 32 + 16 * mt + gq, 8 * nt + 2 * tq + 1) = -acc[1];
-                *f32_at(T32, 32 + 16 * mt + gq + 8, 8 * nt + 2 * tq) = -acc[2];
-                *f32_at(T32, 32 + 16 * mt + gq + 8, 8 * nt + 2 * tq + 1) = -acc[3];
-            }
-            __syncthreads();
+            solve_unit_lower(A32, T32, reinterpret_cast<float*>(sm + OFF_P32), tid, warp, ci);
             GDR_TRACE(14);
             // L = [T ; 0] (bf16, 128 x 64); tied: APRE rows 0..63 = T Diag(beta).
             // Thread (row r = tid & 63, half = tid >> 6 of 4): chunks 2*half, 2*half+1.
@@ -832,6 +843,463 @@ finish:
 #undef GDR_BEFORE_MMA
 }
 
+// ---------------------------------------------------------------------------
+// Gated DeltaNet form: scalar decay per token, tied scalar b = w = beta.
+// Every scale factor is per token, so it folds into MMA outputs or into the
+// small T-derived operands and the raw q / k tiles from TMA are the MMA
+// operands (no operand build):
+//   A  = Diag(beta rowf) (K K^T) Diag(colf)  (strict lower)     [D1 unload]
+//   Aq = Diag(rowf) (Q K^T) Diag(colf)       (lower)            [D1 unload]
+//   W  = T Diag(beta g) K                     (P2, A = [T Diag(beta g) ; 0])
+//   U  = T Diag(beta) V - W S                 (P3 pre-load + S1)
+//   O  = Diag(g) (Q S) + Aq U                 (S1 gives Q S, S2 gives Aq U)
+//   S' = g_{n-1} S + (Diag(g_{n-1}/g) K)^T U  (K copy scaled per token, S2)
+// with g_r = 2^l_r and rowf_r colf_j = g_r / g_j around the chunk's reference.
+// Inputs are double-buffered: the next chunk's TMA is issued as a chunk starts.
+namespace gdn {
+constexpr uint32_t OFF_QK = 0;          // [K ; Q] bf16 [128 x 128], 2 buffers; rows 0..63 become -W
+constexpr uint32_t OFF_K2 = 65536;      // K bf16 [64 x 128], 2 buffers; scaled by g_{n-1}/g per token
+constexpr uint32_t OFF_V = 98304;       // V slice bf16 [64 x 64], 2 buffers
+constexpr uint32_t OFF_L = 114688;      // [T Diag(beta g) ; 0] bf16 [128 x 64]
+constexpr uint32_t OFF_APRE = 131072;   // [T Diag(beta) ; 0] bf16 [128 x 64]
+constexpr uint32_t OFF_AQ = 147456;     // [0 ; Aq] bf16 [128 x 64]
+constexpr uint32_t OFF_SBF = 163840;    // S bf16 [128 x 64]
+constexpr uint32_t OFF_U = 180224;      // U bf16 [64 x 64]
+constexpr uint32_t OFF_A32 = 188416;    // A fp32 [64 x 64]
+constexpr uint32_t OFF_T32 = 204800;    // T fp32 [64 x 64]
+constexpr uint32_t OFF_SCR = 221184;    // solve scratch fp32 (5 KB)
+constexpr uint32_t OFF_SMALL = 226304;  // per-token scalars, barriers
+constexpr uint32_t SMEM_BYTES = OFF_SMALL + 3072 + 1024;
+constexpr uint32_t TM_D1 = 0, TM_D2 = 64, TM_D3 = 192, TM_D4 = 256, TM_D5 = 320, TM_COLS = 512;
+}  // namespace gdn
+
+__global__ void __launch_bounds__(NT, 1) chunk_fwd_gdn_kernel(
+    const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ CUtensorMap tm_k,
+    const __grid_constant__ CUtensorMap tm_v, const Params p) {
+    extern __shared__ uint8_t smem_raw[];
+    uint8_t* sm = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) &
+                                             ~uintptr_t(1023));
+    const int tid = threadIdx.x, warp = tid >> 5;
+    const int wg = warp >> 2;
+    const int row = tid & 127;
+    const int vt = blockIdx.x, h = blockIdx.y, bb = blockIdx.z;
+    const int v0 = vt * NV;
+    const int T = p.T, H = p.H;
+    const int nchunks = (T + C - 1) / C;
+
+    // per-token factors, double-buffered by chunk parity (the next chunk's are
+    // computed while the current chunk's last MMA runs): [2][64] each
+    float* s_beta2 = reinterpret_cast<float*>(sm + gdn::OFF_SMALL);
+    float* s_rowf2 = s_beta2 + 128;
+    float* s_colf2 = s_beta2 + 256;
+    float* s_g2 = s_beta2 + 384;
+    float* s_gcr2 = s_beta2 + 512;
+    float* s_misc2 = s_beta2 + 640;   // [2][4]: g_{n-1}
+    float* s_alpha = s_beta2 + 648;   // [64] staging of the next chunk's decays
+    uint64_t* bar_tma = reinterpret_cast<uint64_t*>(sm + gdn::OFF_SMALL + 2880);  // [2]
+    uint64_t* bar_mma = bar_tma + 2;
+    uint32_t* s_tmem = reinterpret_cast<uint32_t*>(sm + gdn::OFF_SMALL + 2912);
+    if (tid == 0) {
+        mbar_init(&bar_tma[0], 1);
+        mbar_init(&bar_tma[1], 1);
+        mbar_init(bar_mma, 1);
+        fence_barrier_init();
+        prefetch_tmap(&tm_q);
+        prefetch_tmap(&tm_k);
+        prefetch_tmap(&tm_v);
+    }
+    if (warp == 0) tmem_alloc(s_tmem, gdn::TM_COLS);
+    tc_fence_before();
+    __syncthreads();
+    tc_fence_after();
+    const uint32_t tmem = *s_tmem;
+    const uint32_t lane_base = (uint32_t)((warp & 3) * 32) << 16;
+    uint32_t ph_tma0 = 0u, ph_tma1 = 0u, ph_mma = 0;
+    bool ok = true;
+    const uint32_t sbase = smem_u32(sm);
+
+    auto issue_loads = [&](int ci) {
+        const int t0 = ci * C, buf = ci & 1;
+        uint8_t* qk = sm + gdn::OFF_QK + buf * 32768;
+        uint8_t* k2 = sm + gdn::OFF_K2 + buf * 16384;
+        mbar_expect_tx(&bar_tma[buf], 7u * 8192u);
+        // [K ; Q]: each 64-column block holds 128 rows (k rows 0..63, q rows 64..127)
+        tma_load_4d(qk, &tm_k, &bar_tma[buf], 0, h, t0, bb);
+        tma_load_4d(qk + 16384, &tm_k, &bar_tma[buf], 64, h, t0, bb);
+        tma_load_4d(qk + 8192, &tm_q, &bar_tma[buf], 0, h, t0, bb);
+        tma_load_4d(qk + 16384 + 8192, &tm_q, &bar_tma[buf], 64, h, t0, bb);
+        tma_load_4d(k2, &tm_k, &bar_tma[buf], 0, h, t0, bb);
+        tma_load_4d(k2 + 8192, &tm_k, &bar_tma[buf], 64, h, t0, bb);
+        tma_load_4d(sm + gdn::OFF_V + buf * 8192, &tm_v, &bar_tma[buf], v0, h, t0, bb);
+    };
+
+    // ---- initial state; constant zero blocks ----------------------------------
+    constexpr int NH = NV / 2;
+    float S[NH];
+    {
+        const float* s0 = p.S0 ? p.S0 + (((size_t)bb * H + h) * DK + row) * p.dv + v0 + wg * NH : nullptr;
+#pragma unroll
+        for (int j = 0; j < NH; j += 4) {
+            float4 x = s0 ? *reinterpret_cast<const float4*>(s0 + j) : make_float4(0.f, 0.f, 0.f, 0.f);
+            S[j] = x.x; S[j + 1] = x.y; S[j + 2] = x.z; S[j + 3] = x.w;
+        }
+#pragma unroll
+        for (int ch = 0; ch < 4; ++ch) st_chunk(sm + gdn::OFF_SBF, sw128_chunk(row, wg * 4 + ch, DK), &S[8 * ch]);
+        if (tid < 64) {  // AQ rows 0..63, L and APRE rows 64..127 stay zero
+#pragma unroll
+            for (int ch = 0; ch < 8; ++ch) {
+                st_zero_chunk(sm + gdn::OFF_AQ, sw128_chunk(tid, ch, 128));
+                st_zero_chunk(sm + gdn::OFF_L, sw128_chunk(64 + tid, ch, 128));
+                st_zero_chunk(sm + gdn::OFF_APRE, sw128_chunk(64 + tid, ch, 128));
+            }
+        }
+    }
+    unsigned short g_a = 0, g_b = 0;
+    auto load_scalar_gates = [&](int ci) {
+        if (tid < C) {
+            const int t = min(ci * C + tid, T - 1);
+            const size_t gi = ((size_t)bb * T + t) * H + h;
+            g_a = ((const unsigned short*)p.alpha)[gi];
+            g_b = ((const unsigned short*)p.bg)[gi];
+        }
+    };
+    auto bits_to_f32 = [](unsigned short u) { return __uint_as_float((uint32_t)u << 16); };
+    // one warp: prefix sum of log2 alpha over the chunk's 64 tokens (2 per lane),
+    // then the bounded factors around the reference and the decay products
+    auto decay_scan = [&](int ci, int lane) {
+        const int par = ci & 1;
+        const int n = min(C, T - ci * C);
+        const float la0 = (2 * lane < n) ? lg2_approx(s_alpha[2 * lane]) : 0.f;
+        const float la1 = (2 * lane + 1 < n) ? lg2_approx(s_alpha[2 * lane + 1]) : 0.f;
+        float x = la0 + la1;
+#pragma unroll
+        for (int off = 1; off < 32; off <<= 1) {
+            const float y = __shfl_up_sync(0xffffffffu, x, off);
+            if (lane >= off) x += y;
+        }
+        const float l1 = x, l0v = x - la1;
+        const float first = __shfl_sync(0xffffffffu, l0v, 0);
+        const float last = __shfl_sync(0xffffffffu, l1, 31);
+        const float ref = 0.5f * (first + last);
+        float* rf = s_rowf2 + par * 64;
+        float* cf = s_colf2 + par * 64;
+        float* g = s_g2 + par * 64;
+        float* gcr = s_gcr2 + par * 64;
+        rf[2 * lane] = ex2_approx(l0v - ref);
+        rf[2 * lane + 1] = ex2_approx(l1 - ref);
+        cf[2 * lane] = ex2_approx(ref - l0v);
+        cf[2 * lane + 1] = ex2_approx(ref - l1);
+        g[2 * lane] = ex2_approx(l0v);
+        g[2 * lane + 1] = ex2_approx(l1);
+        gcr[2 * lane] = ex2_approx(last - l0v);
+        gcr[2 * lane + 1] = ex2_approx(last - l1);
+        if (lane == 0) {
+            s_misc2[par * 4] = ex2_approx(last);
+            if (first - last > 230.f) flag_status(p.d_status, GDR_DEVICE_DECAY_RANGE);
+        }
+    };
+    // stage chunk ci's gates (threads 0..63 hold them in g_a, g_b)
+    auto stage_gates = [&](int ci) {
+        if (tid < C) {
+            const bool valid = ci * C + tid < T;
+            s_alpha[tid] = valid ? bits_to_f32(g_a) : 1.f;
+            s_beta2[(ci & 1) * 64 + tid] = valid ? bits_to_f32(g_b) : 0.f;
+        }
+    };
+    if (tid == 0 && nchunks > 0) issue_loads(0);
+    if (nchunks > 0) {
+        load_scalar_gates(0);
+        stage_gates(0);
+        __syncthreads();
+        if (warp == 7) decay_scan(0, tid & 31);
+        __syncthreads();
+    }
+
+#define GDR_WAIT(bar, ph)                                                   \
+    do {                                                                    \
+        bool w_ok = mbar_wait(bar, ph);                                     \
+        ph ^= 1u;                                                           \
+        if (!__syncthreads_and(w_ok)) { ok = false; goto finish; }          \
+    } while (0)
+#define GDR_BEFORE_MMA()    \
+    do {                    \
+        fence_proxy_async(); \
+        tc_fence_before();  \
+        __syncthreads();    \
+    } while (0)
+
+    for (int ci = 0; ci < nchunks; ++ci) {
+        const int t0 = ci * C;
+        const int n = min(C, T - t0);
+        const int buf = ci & 1;
+        const uint32_t qkb = sbase + gdn::OFF_QK + buf * 32768u;
+        const uint32_t k2b = sbase + gdn::OFF_K2 + buf * 16384u;
+        const uint32_t vbuf = sbase + gdn::OFF_V + buf * 8192u;
+        GDR_TRACE(0);
+        if (tid == 0 && ci + 1 < nchunks) issue_loads(ci + 1);  // its buffers were freed by chunk ci-1
+        if (ci + 1 < nchunks) load_scalar_gates(ci + 1);         // consumed before S2 of this chunk
+        const int par = ci & 1;
+        const float* s_beta = s_beta2 + par * 64;
+        const float* s_rowf = s_rowf2 + par * 64;
+        const float* s_colf = s_colf2 + par * 64;
+        const float* s_g = s_g2 + par * 64;
+        const float* s_gcr = s_gcr2 + par * 64;
+        const float* s_misc = s_misc2 + par * 4;
+        if (buf == 0) GDR_WAIT(&bar_tma[0], ph_tma0);
+        else GDR_WAIT(&bar_tma[1], ph_tma1);
+        GDR_TRACE(1);
+        GDR_TRACE(2);
+
+        // ---- P1: D1 = [K ; Q] x K^T -----------------------------------------------
+        if (tid == 0) {
+            tc_fence_after();
+            const uint32_t id = idesc_bf16(128, 64, 0, 0);
+#pragma unroll
+            for (int ks = 0; ks < 8; ++ks) {
+                const uint32_t koff = (ks >> 2) * 16384u + (ks & 3) * 32u;
+                mma_bf16(tmem + gdn::TM_D1, sdesc_sw128(qkb + koff, 16, 1024), sdesc_sw128(qkb + koff, 16, 1024),
+                         id, ks > 0);
+            }
+            mma_commit(bar_mma);
+        }
+        // while P1 runs: scale the K copy's rows by g_{n-1} / g_r (rows of S2's operand)
+        {
+            const int r = tid >> 2, c4 = (tid & 3) * 4;  // 64 rows x 4 threads x 4 chunks
+            const float f = s_gcr[r];
+#pragma unroll
+            for (int cc = 0; cc < 4; ++cc) {
+                float x[8];
+                const uint32_t off = sw128_chunk(r, c4 + cc, 64);
+                ld_chunk(sm + gdn::OFF_K2 + buf * 16384, off, x);
+#pragma unroll
+                for (int e = 0; e < 8; ++e) x[e] *= f;
+                st_chunk(sm + gdn::OFF_K2 + buf * 16384, off, x);
+            }
+        }
+        GDR_WAIT(bar_mma, ph_mma);
+        tc_fence_after();
+        GDR_TRACE(3);
+
+        // ---- unload D1: A (fp32) and its transposed diagonal blocks; Aq -> AQ ---------
+        {
+            const int r = row & 63;
+            float d[32];
+            tmem_ld32(tmem + lane_base + gdn::TM_D1 + wg * 32, d);
+            const float rf = s_rowf[r] * (row < 64 ? s_beta[r] : 1.f);
+            float cf[32];
+#pragma unroll
+            for (int j4 = 0; j4 < 32; j4 += 4) {
+                const float4 c4v = *reinterpret_cast<const float4*>(s_colf + wg * 32 + j4);
+                cf[j4] = c4v.x; cf[j4 + 1] = c4v.y; cf[j4 + 2] = c4v.z; cf[j4 + 3] = c4v.w;
+            }
+            if (row < 64) {
+                float* A32 = reinterpret_cast<float*>(sm + gdn::OFF_A32);
+#pragma unroll
+                for (int j4 = 0; j4 < 32; j4 += 4) {
+                    const int j = wg * 32 + j4;
+                    float4 x;
+                    x.x = j < r ? rf * cf[j4] * d[j4] : 0.f;
+                    x.y = j + 1 < r ? rf * cf[j4 + 1] * d[j4 + 1] : 0.f;
+                    x.z = j + 2 < r ? rf * cf[j4 + 2] * d[j4 + 2] : 0.f;
+                    x.w = j + 3 < r ? rf * cf[j4 + 3] * d[j4 + 3] : 0.f;
+                    d[j4] = x.x; d[j4 + 1] = x.y; d[j4 + 2] = x.z; d[j4 + 3] = x.w;
+                    *reinterpret_cast<float4*>(f32_at(A32, r, j)) = x;
+                }
+                const int I = r >> 4, rr = r & 15;
+                if ((I >> 1) == wg) {
+                    float* at = reinterpret_cast<float*>(sm + gdn::OFF_SCR) + I * 272;
+                    if (I & 1) {
+#pragma unroll
+                        for (int j = 0; j < 16; ++j) at[j * 16 + rr] = d[16 + j];
+                    } else {
+#pragma unroll
+                        for (int j = 0; j < 16; ++j) at[j * 16 + rr] = d[j];
+                    }
+                }
+            } else {
+                float x[8];
+#pragma unroll
+                for (int c8 = 0; c8 < 4; ++c8) {
+#pragma unroll
+                    for (int e = 0; e < 8; ++e) {
+                        const int jl = c8 * 8 + e;
+                        x[e] = (wg * 32 + jl <= r) ? rf * cf[jl] * d[jl] : 0.f;
+                    }
+                    st_chunk(sm + gdn::OFF_AQ, sw128_chunk(row, wg * 4 + c8, 128), x);
+                }
+            }
+        }
+        __syncthreads();
+        GDR_TRACE(4);
+
+        // ---- solve; L = T Diag(beta g), APRE = T Diag(beta) (rows 0..63) ------------
+        {
+            float* A32 = reinterpret_cast<float*>(sm + gdn::OFF_A32);
+            float* T32 = reinterpret_cast<float*>(sm + gdn::OFF_T32);
+            solve_unit_lower(A32, T32, reinterpret_cast<float*>(sm + gdn::OFF_SCR), tid, warp, ci);
+            GDR_TRACE(14);
+            const int r = tid & 63, q4 = tid >> 6;
+#pragma unroll
+            for (int cc = 0; cc < 2; ++cc) {
+                const int c8 = q4 * 2 + cc;
+                float x[8], y[8];
+#pragma unroll
+                for (int e4 = 0; e4 < 8; e4 += 4) {
+                    const int j = c8 * 8 + e4;
+                    float4 t4 = (j < 32 || r >= 32) ? *reinterpret_cast<const float4*>(f32_at(T32, r, j))
+                                                    : make_float4(0.f, 0.f, 0.f, 0.f);
+                    const float4 b4 = *reinterpret_cast<const float4*>(s_beta + j);
+                    const float4 g4 = *reinterpret_cast<const float4*>(s_g + j);
+                    y[e4] = t4.x * b4.x; y[e4 + 1] = t4.y * b4.y; y[e4 + 2] = t4.z * b4.z; y[e4 + 3] = t4.w * b4.w;
+                    x[e4] = y[e4] * g4.x; x[e4 + 1] = y[e4 + 1] * g4.y; x[e4 + 2] = y[e4 + 2] * g4.z;
+                    x[e4 + 3] = y[e4 + 3] * g4.w;
+                }
+                st_chunk(sm + gdn::OFF_L, sw128_chunk(r, c8, 128), x);
+                st_chunk(sm + gdn::OFF_APRE, sw128_chunk(r, c8, 128), y);
+            }
+        }
+        GDR_BEFORE_MMA();
+        GDR_TRACE(5);
+
+        // ---- P2: D2 = [T Diag(beta g) ; 0] x K;  P3: D3 = [T Diag(beta) ; 0] x V ----
+        if (tid == 0) {
+            tc_fence_after();
+            const uint32_t idW = idesc_bf16(128, 128, 0, 1);
+            const uint32_t id64 = idesc_bf16(128, 64, 0, 1);
+#pragma unroll
+            for (int ks = 0; ks < 4; ++ks)
+                mma_bf16(tmem + gdn::TM_D2, sdesc_sw128(sbase + gdn::OFF_L + ks * 32u, 16, 1024),
+                         sdesc_sw128(qkb + ks * 2048u, 16384, 1024), idW, ks > 0);
+#pragma unroll
+            for (int ks = 0; ks < 4; ++ks)
+                mma_bf16(tmem + gdn::TM_D3, sdesc_sw128(sbase + gdn::OFF_APRE + ks * 32u, 16, 1024),
+                         sdesc_sw128(vbuf + ks * 2048u, 8192, 1024), id64, ks > 0);
+            mma_commit(bar_mma);
+        }
+        GDR_WAIT(bar_mma, ph_mma);
+        tc_fence_after();
+        GDR_TRACE(6);
+
+        // ---- -W -> rows 0..63 of [K ; Q] (K is no longer read from this tile) ----------
+        if (row < 64) {
+            float d[32], d1[32];
+            tmem_ld32_async(tmem + lane_base + gdn::TM_D2 + wg * 64, d);
+            tmem_ld32_async(tmem + lane_base + gdn::TM_D2 + wg * 64 + 32, d1);
+            tmem_wait_ld();
+#pragma unroll
+            for (int cb = 0; cb < 2; ++cb) {
+                const int col = wg * 64 + cb * 32;
+                const float* dd = cb ? d1 : d;
+#pragma unroll
+                for (int c4 = 0; c4 < 4; ++c4) {
+                    float x[8];
+#pragma unroll
+                    for (int e = 0; e < 8; ++e) x[e] = -dd[c4 * 8 + e];
+                    st_chunk(sm + gdn::OFF_QK + buf * 32768, sw128_chunk(row, col / 8 + c4, 128), x);
+                }
+            }
+        }
+        GDR_BEFORE_MMA();
+        GDR_TRACE(7);
+
+        // ---- S1: D3 += [-W ; Q] x S ------------------------------------------------
+        if (tid == 0) {
+            tc_fence_after();
+            const uint32_t id64 = idesc_bf16(128, NV, 0, 1);
+#pragma unroll
+            for (int ks = 0; ks < 8; ++ks)
+                mma_bf16(tmem + gdn::TM_D3, sdesc_sw128(qkb + (ks >> 2) * 16384u + (ks & 3) * 32u, 16, 1024),
+                         sdesc_sw128(sbase + gdn::OFF_SBF + ks * 2048u, 8192, 1024), id64, 1);
+            mma_commit(bar_mma);
+        }
+        GDR_WAIT(bar_mma, ph_mma);
+        tc_fence_after();
+        GDR_TRACE(8);
+
+        // ---- U (rows 0..63 of D3) -> bf16 -------------------------------------------
+        if (row < 64) {
+            float d[32];
+            tmem_ld32(tmem + lane_base + gdn::TM_D3 + wg * 32, d);
+#pragma unroll
+            for (int c8 = 0; c8 < 4; ++c8) st_chunk(sm + gdn::OFF_U, sw128_chunk(row, wg * 4 + c8, 64), d + 8 * c8);
+        }
+        if (ci + 1 < nchunks) stage_gates(ci + 1);
+        GDR_BEFORE_MMA();
+        GDR_TRACE(9);
+
+        // ---- S2: D5 = [0 ; Aq] x U ;  D4 = (Diag(g_{n-1}/g) K)^T x U ------------------
+        if (tid == 0) {
+            tc_fence_after();
+            const uint32_t idK = idesc_bf16(128, NV, 0, 1);
+            const uint32_t idM = idesc_bf16(128, NV, 1, 1);
+#pragma unroll
+            for (int ks = 0; ks < 4; ++ks) {
+                mma_bf16(tmem + gdn::TM_D5, sdesc_sw128(sbase + gdn::OFF_AQ + ks * 32u, 16, 1024),
+                         sdesc_sw128(sbase + gdn::OFF_U + ks * 2048u, 8192, 1024), idK, ks > 0);
+                mma_bf16(tmem + gdn::TM_D4, sdesc_sw128(k2b + ks * 2048u, 8192, 1024),
+                         sdesc_sw128(sbase + gdn::OFF_U + ks * 2048u, 8192, 1024), idM, ks > 0);
+            }
+            mma_commit(bar_mma);
+        }
+        if (warp == 7 && ci + 1 < nchunks) decay_scan(ci + 1, tid & 31);  // overlaps S2
+        GDR_WAIT(bar_mma, ph_mma);
+        tc_fence_after();
+        GDR_TRACE(10);
+
+        // ---- O = g Q S + Aq U (rows 64..127) -> global; S = g_{n-1} S + D4 ----------
+        {
+            float d[32], d5[32], dS[32];
+            if (row >= 64) {
+                tmem_ld32_async(tmem + lane_base + gdn::TM_D3 + wg * 32, d);
+                tmem_ld32_async(tmem + lane_base + gdn::TM_D5 + wg * 32, d5);
+            }
+            tmem_ld32_async(tmem + lane_base + gdn::TM_D4 + wg * 32, dS);
+            tmem_wait_ld();
+            if (row >= 64) {
+                const int t = t0 + row - 64;
+                if (t < T) {
+                    const float gr = s_g[row - 64];
+                    __nv_bfloat16* op = p.o + (((size_t)bb * T + t) * H + h) * p.dv + v0 + wg * 32;
+#pragma unroll
+                    for (int c8 = 0; c8 < 4; ++c8) {
+                        float y[8];
+#pragma unroll
+                        for (int e = 0; e < 8; ++e) y[e] = fmaf(gr, d[c8 * 8 + e], d5[c8 * 8 + e]);
+                        uint4 u;
+                        u.x = pack_bf16x2(y[0], y[1]);
+                        u.y = pack_bf16x2(y[2], y[3]);
+                        u.z = pack_bf16x2(y[4], y[5]);
+                        u.w = pack_bf16x2(y[6], y[7]);
+                        *reinterpret_cast<uint4*>(op + c8 * 8) = u;
+                    }
+                }
+            }
+            const float gC = s_misc[0];
+#pragma unroll
+            for (int j = 0; j < NH; ++j) S[j] = fmaf(gC, S[j], dS[j]);
+#pragma unroll
+            for (int ch = 0; ch < 4; ++ch) st_chunk(sm + gdn::OFF_SBF, sw128_chunk(row, wg * 4 + ch, DK), &S[8 * ch]);
+        }
+        tc_fence_before();
+        __syncthreads();
+        GDR_TRACE(11);
+    }
+
+    if (p.ST) {
+        float* st = p.ST + (((size_t)bb * H + h) * DK + row) * p.dv + v0 + wg * NH;
+#pragma unroll
+        for (int j = 0; j < NH; j += 4) *reinterpret_cast<float4*>(st + j) = make_float4(S[j], S[j + 1], S[j + 2], S[j + 3]);
+    }
+
+finish:
+    if (!ok && tid == 0) flag_status(p.d_status, GDR_DEVICE_TIMEOUT);
+    tc_fence_before();
+    __syncthreads();
+    if (warp == 0) tmem_dealloc(tmem, gdn::TM_COLS);
+#undef GDR_WAIT
+#undef GDR_BEFORE_MMA
+}
+
 }  // namespace chunk
 
 // Host-side launch (tensor maps are built by the caller).
@@ -853,7 +1321,11 @@ cudaError_t launch_chunk_sm100(const CUtensorMap* maps, const void* alpha, const
         return cudaSuccess;
     };
     cudaError_t e;
-    if (tied) e = ach ? launch(chunk::chunk_fwd_kernel<true, true>) : launch(chunk::chunk_fwd_kernel<true, false>);
+    if (tied && akind == GDR_GATE_SCALAR) {
+        e = cudaFuncSetAttribute(chunk::chunk_fwd_gdn_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, chunk::gdn::SMEM_BYTES);
+        if (e != cudaSuccess) return e;
+        chunk::chunk_fwd_gdn_kernel<<<grid, chunk::NT, chunk::gdn::SMEM_BYTES, st>>>(maps[0], maps[1], maps[2], p);
+    } else if (tied) e = ach ? launch(chunk::chunk_fwd_kernel<true, true>) : launch(chunk::chunk_fwd_kernel<true, false>);
     else e = ach ? launch(chunk::chunk_fwd_kernel<false, true>) : launch(chunk::chunk_fwd_kernel<false, false>);
     if (e != cudaSuccess) return e;
     return cudaGetLastError();

@@ -135,6 +135,19 @@ gdr_status gdr_decode_step(const void* q, const void* k, const void* v,
                            float* S, void* o, int B, int H, int d_k, int d_v,
                            int dtype, int* d_status, void* stream);
 
+/*
+ * gdr_selftest_bounded_wait -- diagnostic for the kernels' bounded waits.
+ *
+ * Launches one block that waits, with the bounded mbarrier wait used by the
+ * tensor-core kernels (poll count and a 2 s %globaltimer limit), on a barrier
+ * that nothing ever completes. The block gives up, ORs GDR_DEVICE_TIMEOUT
+ * into *d_status (device int, required) and ends; the CUDA context stays
+ * usable. Asynchronous on `stream`. Returns GDR_OK, GDR_ERR_INVALID_ARG
+ * (NULL d_status) or GDR_ERR_LAUNCH. No page source defines this; it tests
+ * the library's own failure handling.
+ */
+gdr_status gdr_selftest_bounded_wait(int* d_status, void* stream);
+
 /* Human-readable name of a gdr_status value (static storage, never NULL). */
 const char* gdr_status_string(int status);
 
