@@ -40,6 +40,45 @@ FLOPS_PER_TOKEN_HEAD = {"general": 281259, "tied": 182955}
 L2_BYTES = 126 * 2**20
 
 
+# Sources of the kernel each workload runs; a recorded DRAM traffic figure is
+# used only while these files are unchanged since the capture.
+_CSRC = "gated_delta_rule_147_b200/csrc/"
+KERNEL_SOURCES = {
+    "general": (_CSRC + "chunk_sm100.cu", _CSRC + "common.cuh"),
+    "erasefree": (_CSRC + "chunk_erasefree_sm100.cu", _CSRC + "chunk_common.cuh",
+                  _CSRC + "common.cuh"),
+}
+
+
+def kernel_family(wl) -> str:
+    return "erasefree" if wl.b == "none" else "general"
+
+
+def kernel_source_hash(family: str) -> str:
+    import hashlib
+    h = hashlib.sha256()
+    for rel in KERNEL_SOURCES[family]:
+        with open(os.path.join(ROOT, rel), "rb") as f:
+            h.update(f.read())
+    return h.hexdigest()
+
+
+def measured_traffic(workload: str):
+    """DRAM bytes per launch (dram__bytes_read.sum + dram__bytes_write.sum) of
+    the chunk kernel from the committed ncu summary, or None when the summary
+    is missing or was taken on different kernel sources."""
+    path = os.path.join(ROOT, "profiles", "chunk_fwd_traffic.json")
+    try:
+        d = json.load(open(path))
+    except (OSError, ValueError):
+        return None
+    from gated_delta_rule_147_b200.inputs import WORKLOADS
+    w = d.get("workloads", {}).get(workload)
+    if w is None or w.get("source_sha256") != kernel_source_hash(kernel_family(WORKLOADS[workload])):
+        return None
+    return w.get("dram_bytes_per_launch")
+
+
 def peaks():
     p = os.path.join(ROOT, "MEASURED_PEAKS.json")
     if os.path.exists(p):
@@ -62,6 +101,11 @@ def workload_bytes(wl):
 
 
 def workload_flops(wl):
+    if wl.b == "none":
+        # erase-free chunk form: (q.g) S, Bq V, the state increment and Bq itself
+        C = 64
+        per = 2 * (2 * wl.dk * wl.dv + C * wl.dv + C * wl.dk // 2)
+        return per * wl.B * wl.T * wl.H
     kind = "tied" if wl.w == "tied" and wl.b == "scalar" else "general"
     return FLOPS_PER_TOKEN_HEAD[kind] * wl.B * wl.T * wl.H
 
@@ -290,16 +334,17 @@ def run_ours(args):
         e2e_ms, h2d, d2h = time_chunk_e2e(inp, wl, dev, max(3, args.steps // 2), args.warmup)
         e2e_steps = max(3, args.steps // 2)
         other = {}
-        for name in ("kda", "gdn2"):
+        for name in ("kda", "gdn2", "gla"):
             w2 = WORKLOADS[name]
             _, _, tot2, per2 = time_chunk(w2, dev, max(3, args.steps // 2), args.warmup, lambda: None)
             a2 = statistics.fmean(per2)
             b2, f2 = workload_bytes(w2), workload_flops(w2)
             rt = max(b2 / (pk["hbm_gbs"] * 1e9), f2 / (pk["bf16_tflops"] * 1e12))
-            other[name] = {"workload": f"{name} B={w2.B} H={w2.H} T={w2.T} d={w2.dk} bf16 alpha={w2.alpha} "
+            other[name] = {"workload": f"{name} B={w2.B} H={w2.H} T={w2.T} d_k={w2.dk} d_v={w2.dv} bf16 alpha={w2.alpha} "
                                        f"b={w2.b} w={w2.w} S0={'random' if w2.s0 else 'zero'}",
                            "tokens_per_s": w2.B * w2.T / (a2 * 1e-3), "ms_per_launch": a2,
-                           "hbm_gbs": b2 / (a2 * 1e-3) / 1e9, "roofline_frac": rt / (a2 * 1e-3)}
+                           "hbm_gbs": b2 / (a2 * 1e-3) / 1e9, "roofline_frac": rt / (a2 * 1e-3),
+                           "traffic": measured_traffic(name)}
             torch.cuda.empty_cache()
         dec = time_decode(dev, 1000, 10)
         dec["frac_of_hbm"] = dec["total_gbs"] / pk["hbm_gbs"]
@@ -316,8 +361,8 @@ def run_ours(args):
             "roofline": {"bound": bound, "achieved": achieved_gbs if bound == "hbm" else flops / (avg_ms * 1e-3) / 1e12,
                          "peak": pk["hbm_gbs"] if bound == "hbm" else pk["bf16_tflops"],
                          "unit": "GB/s" if bound == "hbm" else "TFLOP/s",
-                         "frac": (max(t_hbm, t_tc)) / (avg_ms * 1e-3), "traffic": None,
-                         "kernel": "gdr::chunk::chunk_fwd_kernel<true>",
+                         "frac": (max(t_hbm, t_tc)) / (avg_ms * 1e-3), "traffic": measured_traffic("gdn"),
+                         "kernel": "gdr::chunk::chunk_fwd_gdn_kernel",
                          "algorithmic_bytes": bytes_, "algorithmic_flops": flops,
                          "tensor_tflops": flops / (avg_ms * 1e-3) / 1e12,
                          "ms_per_launch": avg_ms, "peak_source": pk["source"]},

@@ -16,6 +16,9 @@ cudaError_t launch_recurrent(const void* q, const void* k, const void* v, const 
                              const void* b, const void* w, int ak, int bk, int wk, const float* S0,
                              void* o, float* ST, int B, int T, int H, int dk, int dv, int dtype,
                              cudaStream_t st);
+cudaError_t launch_chunk_erasefree_sm100(const CUtensorMap* maps, const void* alpha, const void* w,
+                                         int akind, int wkind, const float* S0, void* o, float* ST,
+                                         int* d_status, int B, int T, int H, int dv, cudaStream_t st);
 cudaError_t launch_chunk_sm100(const CUtensorMap* maps, const void* alpha, const void* b,
                                const void* w, int akind, int bkind, int wkind, bool tied,
                                const float* S0, void* o, float* ST, int* d_status, int B, int T,
@@ -133,8 +136,12 @@ gdr_status gdr_chunk_fwd(const void* q, const void* k, const void* v, const void
             !make_map(&maps[4], bmap, B, T, H, d_k) || !make_map(&maps[5], wmap, B, T, H, d_k))
             return GDR_ERR_INVALID_ARG;
         const bool tied = w_kind == GDR_GATE_TIED && b_kind == GDR_GATE_SCALAR;
-        e = gdr::launch_chunk_sm100(maps, alpha, b, w, alpha_kind, b_kind, w_kind, tied, S0, o, S_T,
-                                    d_status, B, T, H, d_v, st);
+        if (b_kind == GDR_GATE_NONE)  // no erase: no triangular solve
+            e = gdr::launch_chunk_erasefree_sm100(maps, alpha, w, alpha_kind, w_kind, S0, o, S_T,
+                                                  d_status, B, T, H, d_v, st);
+        else
+            e = gdr::launch_chunk_sm100(maps, alpha, b, w, alpha_kind, b_kind, w_kind, tied, S0, o,
+                                        S_T, d_status, B, T, H, d_v, st);
     } else {
         e = gdr::launch_recurrent(q, k, v, alpha, b, w, alpha_kind, b_kind, w_kind, S0, o, S_T, B,
                                   T, H, d_k, d_v, dtype, st);

@@ -20,6 +20,8 @@ settings; "Erase-then-Delta Attention" abstract for the independent b/w gates;
          b,w channel, independent, ~ sigmoid(N(0,1)); S0 = 0; seed 3
   decode B=256,H=32,d=128; fp32 state ~ N(0, 0.02^2); per step one bf16 token
          with gdn2 gates; 1000 steps; state from seed 4, step s from (4, s)
+  gla    B=4,H=16,T=4096,d_k=128,d_v=256 bf16; q,k L2-normalised; channel
+         alpha; no erase (b = 0), w = 1; S0 = 0; seed 5 (erase-free path)
 
 Value recipes: q,k,v ~ N(0,1); alpha = exp(-softplus(x)), x ~ N(0,1);
 sigmoid gates = 1/(1+exp(-x)), x ~ N(0,1). L2 normalisation is
@@ -74,6 +76,10 @@ WORKLOADS = {
                          True, True, True, "sigmoid", 2),
     "gdn2": ChunkWorkload("gdn2", 1, 16, 32768, 128, 128, "bf16", "channel", "channel", "channel",
                           True, True, False, "sigmoid", 3),
+    # erase-free gated linear attention with the GLA head shape d_k=128, d_v=256
+    # ("How Linear Attention Remembers", Table 1); q, k L2-normalised
+    "gla": ChunkWorkload("gla", 4, 16, 4096, 128, 256, "bf16", "channel", "none", "none",
+                         True, True, False, "sigmoid", 5),
 }
 
 

@@ -155,3 +155,29 @@ def test_full_size_sampled_heads(cuda_device, family):
     assert_close(o_s, o_ref, TOL["bf16"], f"o {heads}")
     assert_close(ST_s, ST_ref, TOL["bf16"], f"S_T {heads}")
     assert np.all(np.isfinite(o))
+
+
+@pytest.mark.parametrize("akind,wkind", [("channel", "none"), ("scalar", "scalar"), ("none", "channel"),
+                                         ("channel", "channel"), ("none", "none")])
+@pytest.mark.parametrize("dv,T", [(64, 130), (256, 64), (128, 1)])
+def test_erase_free_path(cuda_device, akind, wkind, dv, T):
+    """b = 0 (no erase) runs the erase-free kernel: linear attention, gated
+    linear attention and Mamba-2 shapes, with or without a write gate."""
+    wl = small("gdn2", T=T, dv=dv, alpha=akind, b="none", w=wkind, s0=True, seed=40 + dv + T)
+    inp = make_chunk_inputs(wl)
+    o, ST = run_chunk(inp, cuda_device)
+    o_ref, ST_ref = run_oracle(inp)
+    assert_close(o, o_ref, TOL["bf16"], "o")
+    assert_close(ST, ST_ref, TOL["bf16"], "S_T")
+
+
+def test_gla_full_size_sampled_heads(cuda_device):
+    """The erase-free workload (GLA head shape d_v = 256) at full size."""
+    wl = WORKLOADS["gla"]
+    inp = make_chunk_inputs(wl)
+    o, ST = run_chunk(inp, cuda_device)
+    heads = [(0, 3), (2, 11), (3, 15)]
+    o_ref, ST_ref = run_oracle(inp, heads)
+    o_s, ST_s = gather_heads(o, ST, heads)
+    assert_close(o_s, o_ref, TOL["bf16"], f"o {heads}")
+    assert_close(ST_s, ST_ref, TOL["bf16"], f"S_T {heads}")

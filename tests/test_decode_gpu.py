@@ -81,3 +81,30 @@ def test_decode_full_size_sampled_heads(cuda_device):
     assert o_err_max <= TOL["bf16"] * o_ref_max, (o_err_max, o_ref_max)
     worst = assert_close(S_dev[rows].cpu().numpy(), S_ref, TOL["bf16"], "S after 1000 steps")
     assert np.all(np.isfinite(S_dev.cpu().numpy()))
+
+
+@pytest.mark.parametrize("family", ["gdn", "kda", "gdn2"])
+def test_prefill_then_decode_continues_the_sequence(cuda_device, family):
+    """The chunk forward's final state is the decode step's state layout:
+    prefill T tokens, then decode m more from S_T; the decode outputs equal
+    the oracle's outputs for tokens T..T+m-1 of one T+m sequence."""
+    from gated_delta_rule_147_b200 import chunk_fwd
+    from gated_delta_rule_147_b200.inputs import WORKLOADS, make_chunk_inputs
+    T, m = 130, 6
+    wl = WORKLOADS[family].with_(B=2, H=2, T=T + m, s0=True, seed=31)
+    inp = make_chunk_inputs(wl)
+    g = inp["gates"]
+    dev = cuda_device
+    pre = lambda x: None if x is None else x[:, :T].contiguous().to(dev)
+    w_arg = TIED if g["w"] == "tied" else pre(inp["w"])
+    _, S = chunk_fwd(pre(inp["q"]), pre(inp["k"]), pre(inp["v"]), pre(inp["alpha"]), pre(inp["b"]),
+                     w_arg, inp["S0"].to(dev))
+    o_ref, _ = oracle.recurrence(inp["q"], inp["k"], inp["v"], inp["alpha"], inp["b"], inp["w"],
+                                 inp["S0"], g)
+    for t in range(T, T + m):
+        tok = lambda x: None if x is None else x[:, t].contiguous().to(dev)
+        w_t = TIED if g["w"] == "tied" else tok(inp["w"])
+        o = decode_step(tok(inp["q"]), tok(inp["k"]), tok(inp["v"]), tok(inp["alpha"]), tok(inp["b"]),
+                        w_t, S)
+        torch.cuda.synchronize()
+        assert_close(o.float().cpu().numpy(), o_ref[:, t], TOL["bf16"], f"decode token {t}")
