@@ -44,14 +44,28 @@ L2_BYTES = 126 * 2**20
 # used only while these files are unchanged since the capture.
 _CSRC = "gated_delta_rule_147_b200/csrc/"
 KERNEL_SOURCES = {
-    "general": (_CSRC + "chunk_sm100.cu", _CSRC + "common.cuh"),
+    "general": (_CSRC + "chunk_sm100.cu", _CSRC + "chunk_common.cuh", _CSRC + "common.cuh"),
+    "twopass": (_CSRC + "chunk_twopass_sm100.cu", _CSRC + "chunk_common.cuh", _CSRC + "common.cuh"),
     "erasefree": (_CSRC + "chunk_erasefree_sm100.cu", _CSRC + "chunk_common.cuh",
                   _CSRC + "common.cuh"),
 }
 
 
+KERNEL_NAMES = {
+    "general": "gdr::chunk::chunk_fwd_kernel / chunk_fwd_gdn_kernel (single pass)",
+    "twopass": "gdr::twopass::prep_gdn_kernel + gdr::twopass::state_gdn_kernel (one call, two launches)",
+    "erasefree": "gdr::erasefree::chunk_fwd_erasefree_kernel",
+}
+LAUNCHES_PER_CALL = {"general": 1, "twopass": 2, "erasefree": 1}
+
+
 def kernel_family(wl) -> str:
-    return "erasefree" if wl.b == "none" else "general"
+    if wl.b == "none":
+        return "erasefree"
+    if (wl.dtype == "bf16" and wl.dk == 128 and wl.dv in (64, 128) and wl.alpha == "scalar"
+            and wl.b == "scalar" and wl.w == "tied"):
+        return "twopass"
+    return "general"
 
 
 def kernel_source_hash(family: str) -> str:
@@ -175,10 +189,20 @@ def prepare_chunk(wl, dev):
     return inp, d
 
 
-def chunk_call(d, wl, o, ST, stream):
+def alloc_workspace(d, wl):
+    """The two-pass path's scratch (None when the gate form has no such path)."""
+    import torch
+    from gated_delta_rule_147_b200 import TIED, workspace_bytes
+    w = TIED if wl.w == "tied" else d["w"]
+    n = workspace_bytes(d["q"], d["v"], d["alpha"], d["b"], w)
+    return torch.empty(n, dtype=torch.uint8, device=d["q"].device) if n else None
+
+
+def chunk_call(d, wl, o, ST, stream, ws):
     from gated_delta_rule_147_b200 import TIED, chunk_fwd
     w = TIED if wl.w == "tied" else d["w"]
-    chunk_fwd(d["q"], d["k"], d["v"], d["alpha"], d["b"], w, d["S0"], out=o, S_T=ST, stream=stream)
+    chunk_fwd(d["q"], d["k"], d["v"], d["alpha"], d["b"], w, d["S0"], out=o, S_T=ST, stream=stream,
+              workspace=ws)
 
 
 def time_chunk(wl, dev, steps, warmup, barrier):
@@ -188,14 +212,15 @@ def time_chunk(wl, dev, steps, warmup, barrier):
     o = torch.empty((wl.B, wl.T, wl.H, wl.dv), dtype=d["v"].dtype, device=dev)
     ST = torch.empty((wl.B, wl.H, wl.dk, wl.dv), dtype=torch.float32, device=dev)
     stream = torch.cuda.current_stream()
+    ws = alloc_workspace(d, wl)
     for _ in range(warmup):
-        chunk_call(d, wl, o, ST, stream)
+        chunk_call(d, wl, o, ST, stream, ws)
     torch.cuda.synchronize()
     barrier()
     ev = [torch.cuda.Event(enable_timing=True) for _ in range(steps + 1)]
     ev[0].record(stream)
     for i in range(steps):
-        chunk_call(d, wl, o, ST, stream)
+        chunk_call(d, wl, o, ST, stream, ws)
         ev[i + 1].record(stream)
     torch.cuda.synchronize()
     per = [ev[i].elapsed_time(ev[i + 1]) for i in range(steps)]
@@ -216,11 +241,12 @@ def time_chunk_e2e(inp, wl, dev, steps, warmup):
     tensors = [k for k, v in host.items() if hasattr(v, "pin_memory")]
     h2d = sum(host[k].numel() * host[k].element_size() for k in tensors)
     d2h = o.numel() * o.element_size()
+    ws = alloc_workspace(dbuf, wl)
 
     def step():
         for k in tensors:
             dbuf[k].copy_(host[k], non_blocking=True)
-        chunk_call(dbuf, wl, o, None, stream)
+        chunk_call(dbuf, wl, o, None, stream, ws)
         o_host.copy_(o, non_blocking=True)
 
     for _ in range(warmup):
@@ -362,13 +388,13 @@ def run_ours(args):
                          "peak": pk["hbm_gbs"] if bound == "hbm" else pk["bf16_tflops"],
                          "unit": "GB/s" if bound == "hbm" else "TFLOP/s",
                          "frac": (max(t_hbm, t_tc)) / (avg_ms * 1e-3), "traffic": measured_traffic("gdn"),
-                         "kernel": "gdr::chunk::chunk_fwd_gdn_kernel",
+                         "kernel": KERNEL_NAMES[kernel_family(wl)],
                          "algorithmic_bytes": bytes_, "algorithmic_flops": flops,
                          "tensor_tflops": flops / (avg_ms * 1e-3) / 1e12,
                          "ms_per_launch": avg_ms, "peak_source": pk["source"]},
             "e2e": {"value": tokens * e2e_steps / (e2e_ms * 1e-3), "unit": "tokens/s",
                     "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": d2h},
-            "gpu_launches": args.steps,
+            "gpu_launches": args.steps * LAUNCHES_PER_CALL[kernel_family(wl)],
             "clocks": clocks,
             "decode": dec,
             "other_workloads": other,

@@ -15,7 +15,7 @@ from __future__ import annotations
 
 from ._lib import (GATE_CHANNEL, GATE_NONE, GATE_SCALAR, GATE_TIED, GDR_BF16, GDR_FP32,
                    GDR_DEVICE_DECAY_RANGE, GDR_DEVICE_TIMEOUT, GdrError, gdr_chunk_fwd,
-                   gdr_decode_step, load)
+                   gdr_chunk_fwd_workspace_size, gdr_decode_step, load)
 
 TIED = "tied"
 _KIND = {"none": GATE_NONE, "scalar": GATE_SCALAR, "channel": GATE_CHANNEL, "tied": GATE_TIED}
@@ -46,11 +46,22 @@ def _gate_kind(g, ndim_scalar: int):
     return GATE_SCALAR if g.dim() == ndim_scalar else GATE_CHANNEL
 
 
+def workspace_bytes(q, v, alpha=None, b=None, w=None) -> int:
+    """Scratch bytes the two-pass chunk path wants for these inputs (0 when
+    the shape / gate form has no two-pass path)."""
+    B, T, H, dk = q.shape
+    return gdr_chunk_fwd_workspace_size(B, T, H, dk, v.shape[-1], _gate_kind(alpha, 3),
+                                        _gate_kind(b, 3), _gate_kind(w, 3), _dtype_code(q))
+
+
 def chunk_fwd(q, k, v, alpha=None, b=None, w=None, S0=None, *, out=None, final_state=True,
-              S_T=None, chunk: int = 64, d_status=None, stream=None):
+              S_T=None, chunk: int = 64, workspace="auto", d_status=None, stream=None):
     """Forward over [B,T,H,*] inputs. alpha/b/w: None, a [B,T,H] tensor
     (scalar gate), a [B,T,H,d_k] tensor (channel gate); w may be TIED (w := b).
-    Returns (o, S_T) with S_T None when final_state is False."""
+    workspace: "auto" allocates the two-pass path's scratch with torch when
+    the inputs have such a path; a uint8 device tensor supplies it; None runs
+    the single-pass kernels. Returns (o, S_T) with S_T None when final_state
+    is False."""
     import torch
     _check(q, k, v, alpha, b, w, S0, out, S_T)
     B, T, H, dk = q.shape
@@ -58,9 +69,15 @@ def chunk_fwd(q, k, v, alpha=None, b=None, w=None, S0=None, *, out=None, final_s
     o = out if out is not None else torch.empty((B, T, H, dv), dtype=v.dtype, device=v.device)
     if final_state and S_T is None:
         S_T = torch.empty((B, H, dk, dv), dtype=torch.float32, device=v.device)
+    if isinstance(workspace, str):
+        if workspace != "auto":
+            raise ValueError(workspace)
+        nbytes = workspace_bytes(q, v, alpha, b, w)
+        workspace = torch.empty(nbytes, dtype=torch.uint8, device=v.device) if nbytes else None
+    ws_bytes = 0 if workspace is None else workspace.numel() * workspace.element_size()
     gdr_chunk_fwd(q, k, v, alpha, b, None if isinstance(w, str) else w, _gate_kind(alpha, 3),
-                  _gate_kind(b, 3), _gate_kind(w, 3), S0, o, S_T if final_state else None, B, T, H,
-                  dk, dv, chunk, _dtype_code(q), d_status, stream)
+                  _gate_kind(b, 3), _gate_kind(w, 3), S0, o, S_T if final_state else None,
+                  workspace, ws_bytes, B, T, H, dk, dv, chunk, _dtype_code(q), d_status, stream)
     return o, (S_T if final_state else None)
 
 

@@ -17,7 +17,7 @@ GDR_DEVICE_TIMEOUT, GDR_DEVICE_DECAY_RANGE = 1, 2
 GDR_BF16, GDR_FP32 = 0, 1
 GATE_NONE, GATE_SCALAR, GATE_CHANNEL, GATE_TIED = 0, 1, 2, 3
 
-EXPORTS = ("gdr_chunk_fwd", "gdr_decode_step", "gdr_selftest_bounded_wait", "gdr_status_string",
+EXPORTS = ("gdr_chunk_fwd", "gdr_chunk_fwd_workspace_size", "gdr_decode_step", "gdr_selftest_bounded_wait", "gdr_status_string",
            "gdr_version")
 
 _lock = threading.Lock()
@@ -46,8 +46,11 @@ def load(build_if_missing: bool = True) -> ctypes.CDLL:
             raise OSError(f"CUDA library {path} is missing; run python -m gated_delta_rule_147_b200.build")
         lib = ctypes.CDLL(path)
         vp, ip = ctypes.c_void_p, ctypes.c_int
-        lib.gdr_chunk_fwd.argtypes = [vp] * 6 + [ip] * 3 + [vp, vp, vp] + [ip] * 7 + [vp, vp]
+        sz = ctypes.c_size_t
+        lib.gdr_chunk_fwd.argtypes = [vp] * 6 + [ip] * 3 + [vp, vp, vp, vp, sz] + [ip] * 7 + [vp, vp]
         lib.gdr_chunk_fwd.restype = ip
+        lib.gdr_chunk_fwd_workspace_size.argtypes = [ip] * 9
+        lib.gdr_chunk_fwd_workspace_size.restype = sz
         lib.gdr_decode_step.argtypes = [vp] * 6 + [ip] * 3 + [vp, vp] + [ip] * 5 + [vp, vp]
         lib.gdr_decode_step.restype = ip
         lib.gdr_status_string.argtypes = [ip]
@@ -79,14 +82,20 @@ def _stream(stream):
     return stream if isinstance(stream, int) else stream.cuda_stream
 
 
-def gdr_chunk_fwd(q, k, v, alpha, b, w, alpha_kind, b_kind, w_kind, S0, o, S_T, B, T, H, d_k, d_v,
-                  chunk, dtype, d_status=None, stream=None) -> None:
+def gdr_chunk_fwd(q, k, v, alpha, b, w, alpha_kind, b_kind, w_kind, S0, o, S_T, workspace,
+                  workspace_bytes, B, T, H, d_k, d_v, chunk, dtype, d_status=None,
+                  stream=None) -> None:
     """Same arguments as the C entry point; tensors are passed by device pointer."""
     st = load().gdr_chunk_fwd(_p(q), _p(k), _p(v), _p(alpha), _p(b), _p(w), alpha_kind, b_kind,
-                              w_kind, _p(S0), _p(o), _p(S_T), B, T, H, d_k, d_v, chunk, dtype,
-                              _p(d_status), _stream(stream))
+                              w_kind, _p(S0), _p(o), _p(S_T), _p(workspace), int(workspace_bytes),
+                              B, T, H, d_k, d_v, chunk, dtype, _p(d_status), _stream(stream))
     if st != GDR_OK:
         raise GdrError("gdr_chunk_fwd", st)
+
+
+def gdr_chunk_fwd_workspace_size(B, T, H, d_k, d_v, alpha_kind, b_kind, w_kind, dtype) -> int:
+    return int(load().gdr_chunk_fwd_workspace_size(B, T, H, d_k, d_v, alpha_kind, b_kind, w_kind,
+                                                   dtype))
 
 
 def gdr_decode_step(q, k, v, alpha, b, w, alpha_kind, b_kind, w_kind, S, o, B, H, d_k, d_v, dtype,

@@ -19,6 +19,11 @@ cudaError_t launch_recurrent(const void* q, const void* k, const void* v, const 
 cudaError_t launch_chunk_erasefree_sm100(const CUtensorMap* maps, const void* alpha, const void* w,
                                          int akind, int wkind, const float* S0, void* o, float* ST,
                                          int* d_status, int B, int T, int H, int dv, cudaStream_t st);
+size_t twopass_workspace_bytes(int B, int T, int H, int dv);
+cudaError_t launch_chunk_twopass_gdn(const CUtensorMap* maps, const CUtensorMap* ws_maps, void* ws,
+                                     const void* alpha, const void* beta, const float* S0, void* o,
+                                     float* ST, int* d_status, int B, int T, int H, int dv,
+                                     cudaStream_t st);
 cudaError_t launch_chunk_sm100(const CUtensorMap* maps, const void* alpha, const void* b,
                                const void* w, int akind, int bkind, int wkind, bool tied,
                                const float* S0, void* o, float* ST, int* d_status, int B, int T,
@@ -70,9 +75,23 @@ bool make_map(CUtensorMap* m, const void* base, int B, int T, int H, int d) {
     return r == CUDA_SUCCESS;
 }
 
+// The two-pass path (per-chunk factors for all chunks in parallel, then the
+// state pass) exists for the tensor-core shape with scalar decay and tied
+// scalar beta, d_v <= 128.
+bool twopass_applies(int T, int d_k, int d_v, int ak, int bk, int wk, int dtype) {
+    return T > 0 && dtype == GDR_BF16 && d_k == 128 && (d_v == 64 || d_v == 128) &&
+           ak == GDR_GATE_SCALAR && bk == GDR_GATE_SCALAR && wk == GDR_GATE_TIED;
+}
+
 }  // namespace
 
 extern "C" {
+
+size_t gdr_chunk_fwd_workspace_size(int B, int T, int H, int d_k, int d_v, int alpha_kind,
+                                    int b_kind, int w_kind, int dtype) {
+    if (B < 1 || H < 1 || !twopass_applies(T, d_k, d_v, alpha_kind, b_kind, w_kind, dtype)) return 0;
+    return gdr::twopass_workspace_bytes(B, T, H, d_v);
+}
 
 const char* gdr_status_string(int s) {
     switch (s) {
@@ -90,8 +109,9 @@ int gdr_version(void) { return (1 << 16) | 0; }
 
 gdr_status gdr_chunk_fwd(const void* q, const void* k, const void* v, const void* alpha,
                          const void* b, const void* w, int alpha_kind, int b_kind, int w_kind,
-                         const float* S0, void* o, float* S_T, int B, int T, int H, int d_k,
-                         int d_v, int chunk, int dtype, int* d_status, void* stream) {
+                         const float* S0, void* o, float* S_T, void* workspace,
+                         size_t workspace_bytes, int B, int T, int H, int d_k, int d_v, int chunk,
+                         int dtype, int* d_status, void* stream) {
     if (B < 1 || H < 1 || T < 0 || d_k < 1 || d_v < 1) return GDR_ERR_INVALID_ARG;
     if (dtype != GDR_BF16 && dtype != GDR_FP32) return GDR_ERR_INVALID_ARG;
     if (!kind_ok(alpha_kind, false) || !kind_ok(b_kind, false) || !kind_ok(w_kind, true))
@@ -123,6 +143,13 @@ gdr_status gdr_chunk_fwd(const void* q, const void* k, const void* v, const void
         (w_kind == GDR_GATE_CHANNEL && !aligned16(w)))
         return GDR_ERR_MISALIGNED;
 
+    const bool twopass = workspace != nullptr && twopass_applies(T, d_k, d_v, alpha_kind, b_kind,
+                                                                 w_kind, dtype);
+    if (twopass) {
+        if (workspace_bytes < gdr::twopass_workspace_bytes(B, T, H, d_v)) return GDR_ERR_INVALID_ARG;
+        if ((reinterpret_cast<uintptr_t>(workspace) & 255u) != 0) return GDR_ERR_MISALIGNED;
+    }
+
     cudaError_t e;
     if (tc_path) {
         if (!encoder()) return GDR_ERR_NO_DEVICE;
@@ -136,7 +163,16 @@ gdr_status gdr_chunk_fwd(const void* q, const void* k, const void* v, const void
             !make_map(&maps[4], bmap, B, T, H, d_k) || !make_map(&maps[5], wmap, B, T, H, d_k))
             return GDR_ERR_INVALID_ARG;
         const bool tied = w_kind == GDR_GATE_TIED && b_kind == GDR_GATE_SCALAR;
-        if (b_kind == GDR_GATE_NONE)  // no erase: no triangular solve
+        if (twopass) {
+            CUtensorMap ws_maps[2];
+            const uint8_t* pbase = reinterpret_cast<const uint8_t*>(workspace) +
+                                   (size_t)B * T * H * d_k * sizeof(uint16_t);
+            if (!make_map(&ws_maps[0], workspace, B, T, H, d_k) ||
+                !make_map(&ws_maps[1], pbase, B, T, H, d_v))
+                return GDR_ERR_INVALID_ARG;
+            e = gdr::launch_chunk_twopass_gdn(maps, ws_maps, workspace, alpha, b, S0, o, S_T,
+                                              d_status, B, T, H, d_v, st);
+        } else if (b_kind == GDR_GATE_NONE)  // no erase: no triangular solve
             e = gdr::launch_chunk_erasefree_sm100(maps, alpha, w, alpha_kind, w_kind, S0, o, S_T,
                                                   d_status, B, T, H, d_v, st);
         else

@@ -56,5 +56,134 @@ __device__ __forceinline__ void st4(uint8_t* base, uint32_t off, const float* x4
     *reinterpret_cast<uint2*>(base + off) = u;
 }
 
+// fp32 [64 x 64] scratch with rows of 16 float4 groups XOR-swizzled by row.
+__device__ __forceinline__ float* f32_at(float* base, int r, int c) {
+    return base + r * 64 + ((((c >> 2) ^ (r & 15))) << 2) + (c & 3);
+}
+
+__device__ __forceinline__ void ld_chunk(const uint8_t* base, uint32_t off, float* x8) {
+    uint4 u = *reinterpret_cast<const uint4*>(base + off);
+    const __nv_bfloat162* h = reinterpret_cast<const __nv_bfloat162*>(&u);
+#pragma unroll
+    for (int i = 0; i < 4; ++i) {
+        float2 f = __bfloat1622float2(h[i]);
+        x8[2 * i] = f.x;
+        x8[2 * i + 1] = f.y;
+    }
+}
+
+// T = (I + A)^-1 for the strictly lower 64 x 64 matrix A (fp32, swizzled rows,
+// with its 16 x 16 diagonal blocks also stored transposed at scr[I * 272 +
+// j * 16 + rr]) into T32: right-looking forward substitution on the diagonal
+// blocks, then recursive halving 16 -> 32 -> 64 on warp-level tensor cores.
+// Called by all 256 threads; ends with a block barrier.
+__device__ __forceinline__ void solve_unit_lower(float* A32, float* T32, float* scr, int tid, int warp) {
+    if (tid < 64) {
+        // diagonal block I, column c: right-looking substitution; column j
+        // of the block is a contiguous row of the transposed copy AT
+        const int I = tid >> 4, c = tid & 15;
+        const float* at = scr + I * 272;
+        float acc[16], x[16];
+#pragma unroll
+        for (int rr = 0; rr < 16; ++rr) acc[rr] = 0.f;
+#pragma unroll
+        for (int j = 0; j < 16; ++j) {
+            x[j] = ((j == c) ? 1.f : 0.f) - acc[j];
+            float a[16];
+#pragma unroll
+            for (int r4 = 0; r4 < 16; r4 += 4) {
+                const float4 v4 = *reinterpret_cast<const float4*>(at + j * 16 + r4);
+                a[r4] = v4.x; a[r4 + 1] = v4.y; a[r4 + 2] = v4.z; a[r4 + 3] = v4.w;
+            }
+#pragma unroll
+            for (int rr = j + 1; rr < 16; ++rr) acc[rr] += a[rr] * x[j];
+        }
+#pragma unroll
+        for (int rr = 0; rr < 16; ++rr) *f32_at(T32, 16 * I + rr, 16 * I + c) = x[rr];
+    } else if (tid < 128) {
+        // the strictly upper 16x16 blocks inside each 32x32 diagonal half are zero
+        const int u = tid - 64;                        // 64 threads, 2 blocks x 16 rows x 4 float4
+        for (int idx = u; idx < 128; idx += 64) {
+            const int blk = idx >> 6, rr = (idx >> 2) & 15, c4 = (idx & 3) * 4;
+            *reinterpret_cast<float4*>(f32_at(T32, 32 * blk + rr, 32 * blk + 16 + c4)) =
+                make_float4(0.f, 0.f, 0.f, 0.f);
+        }
+    }
+    __syncthreads();
+    // Merges on warp-level tensor cores (tf32 operands, fp32 accumulate).
+    // One warp computes a 16 x 8 tile
+    //   D[i][j] = sum_k A[rA + i][cA + k] B[rB + k][cB + j],  k < 8 ksteps,
+    // reading A and B from the swizzled fp32 tiles (f32_at) or from a
+    // plain scratch tile with rows of kPad floats.
+    constexpr int kPad = 40;
+    const int lane = tid & 31, gq = lane >> 2, tq = lane & 3;
+    auto tile_mma = [&](float* Am, bool swzA, int rA, int cA, float* Bm, bool swzB, int rB,
+                        int cB, int ksteps, float* acc) {
+#pragma unroll
+        for (int e = 0; e < 4; ++e) acc[e] = 0.f;
+        auto ldA = [&](int r, int c) { return swzA ? *f32_at(Am, r, c) : Am[r * kPad + c]; };
+        auto ldB = [&](int r, int c) { return swzB ? *f32_at(Bm, r, c) : Bm[r * kPad + c]; };
+        for (int ks = 0; ks < ksteps; ++ks) {
+            const int k = 8 * ks;
+            uint32_t a[4], b[2];
+            a[0] = to_tf32(ldA(rA + gq, cA + k + tq));
+            a[1] = to_tf32(ldA(rA + gq + 8, cA + k + tq));
+            a[2] = to_tf32(ldA(rA + gq, cA + k + tq + 4));
+            a[3] = to_tf32(ldA(rA + gq + 8, cA + k + tq + 4));
+            b[0] = to_tf32(ldB(rB + k + tq, cB + gq));
+            b[1] = to_tf32(ldB(rB + k + tq + 4, cB + gq));
+            mma_tf32_m16n8k8(acc, a, b);
+        }
+    };
+    float* XY = scr;  // X: [2][16 x kPad], later Y: [32 x kPad]
+    // 16 -> 32: X_b = A_(2b+1)(2b) T_(2b)(2b) (b = 0, 1), four 16 x 8 tiles
+    if (warp < 4) {
+        const int b = warp >> 1, nt = warp & 1;
+        const int R = 32 * b + 16, Cc = 32 * b;
+        float acc[4];
+        tile_mma(A32, true, R, Cc, T32, true, Cc, Cc + 8 * nt, 2, acc);
+        float* X = XY + b * 16 * kPad;
+        X[gq * kPad + 8 * nt + 2 * tq] = acc[0];
+        X[gq * kPad + 8 * nt + 2 * tq + 1] = acc[1];
+        X[(gq + 8) * kPad + 8 * nt + 2 * tq] = acc[2];
+        X[(gq + 8) * kPad + 8 * nt + 2 * tq + 1] = acc[3];
+    }
+    __syncthreads();
+    // T_(2b+1)(2b) = -T_(2b+1)(2b+1) X_b
+    if (warp < 4) {
+        const int b = warp >> 1, nt = warp & 1;
+        const int R = 32 * b + 16, Cc = 32 * b;
+        float acc[4];
+        tile_mma(T32, true, R, R, XY + b * 16 * kPad, false, 0, 8 * nt, 2, acc);
+        *f32_at(T32, R + gq, Cc + 8 * nt + 2 * tq) = -acc[0];
+        *f32_at(T32, R + gq, Cc + 8 * nt + 2 * tq + 1) = -acc[1];
+        *f32_at(T32, R + gq + 8, Cc + 8 * nt + 2 * tq) = -acc[2];
+        *f32_at(T32, R + gq + 8, Cc + 8 * nt + 2 * tq + 1) = -acc[3];
+    }
+    __syncthreads();
+    // 32 -> 64: Y = A[32:64, 0:32] T[0:32, 0:32], eight 16 x 8 tiles (one per warp)
+    {
+        const int mt = warp >> 2, nt = warp & 3;
+        float acc[4];
+        tile_mma(A32, true, 32 + 16 * mt, 0, T32, true, 0, 8 * nt, 4, acc);
+        XY[(16 * mt + gq) * kPad + 8 * nt + 2 * tq] = acc[0];
+        XY[(16 * mt + gq) * kPad + 8 * nt + 2 * tq + 1] = acc[1];
+        XY[(16 * mt + gq + 8) * kPad + 8 * nt + 2 * tq] = acc[2];
+        XY[(16 * mt + gq + 8) * kPad + 8 * nt + 2 * tq + 1] = acc[3];
+    }
+    __syncthreads();
+    // T[32:64, 0:32] = -T[32:64, 32:64] Y
+    {
+        const int mt = warp >> 2, nt = warp & 3;
+        float acc[4];
+        tile_mma(T32, true, 32 + 16 * mt, 32, XY, false, 0, 8 * nt, 4, acc);
+        *f32_at(T32, 32 + 16 * mt + gq, 8 * nt + 2 * tq) = -acc[0];
+        *f32_at(T32, 32 + 16 * mt + gq, 8 * nt + 2 * tq + 1) = -acc[1];
+        *f32_at(T32, 32 + 16 * mt + gq + 8, 8 * nt + 2 * tq) = -acc[2];
+        *f32_at(T32, 32 + 16 * mt + gq + 8, 8 * nt + 2 * tq + 1) = -acc[3];
+    }
+    __syncthreads();
+}
+
 }  // namespace chunkc
 }  // namespace gdr

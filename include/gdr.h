@@ -57,6 +57,8 @@
 #ifndef GDR_H
 #define GDR_H
 
+#include <stddef.h>
+
 #ifdef __cplusplus
 extern "C" {
 #endif
@@ -104,17 +106,39 @@ typedef enum {
  * Alignment: q, k, v, o and channel gates must be 16-byte aligned and, on
  * the tensor-core path, d_k and d_v rows 16-byte multiples (given by the
  * shape rules above).
+ * workspace, workspace_bytes: optional caller-owned device scratch (NULL, 0
+ * for none). When gdr_chunk_fwd_workspace_size() is non-zero for the call's
+ * shape and gate form and workspace is not NULL, the forward runs in two
+ * passes: first the per-chunk WY factors of every chunk of every head in
+ * parallel (written to the workspace), then the state pass over the chunks.
+ * Otherwise one kernel does both per chunk. Both give the same result up to
+ * rounding. The workspace must be 256-byte aligned and hold at least the
+ * queried size; its contents on entry are ignored and on exit undefined.
  * Returns GDR_OK, GDR_ERR_INVALID_ARG (B, H < 1, T < 0, bad kinds, NULL
- * data), GDR_ERR_UNSUPPORTED (chunk != 64, shape beyond the limits above),
- * GDR_ERR_MISALIGNED, GDR_ERR_LAUNCH or GDR_ERR_NO_DEVICE. T = 0 writes S_T
- * := S0 (or zeros) and launches nothing else.
+ * data, workspace smaller than required), GDR_ERR_UNSUPPORTED (chunk != 64,
+ * shape beyond the limits above), GDR_ERR_MISALIGNED, GDR_ERR_LAUNCH or
+ * GDR_ERR_NO_DEVICE. T = 0 writes S_T := S0 (or zeros) and launches nothing
+ * else.
  */
 gdr_status gdr_chunk_fwd(const void* q, const void* k, const void* v,
                          const void* alpha, const void* b, const void* w,
                          int alpha_kind, int b_kind, int w_kind,
                          const float* S0, void* o, float* S_T,
+                         void* workspace, size_t workspace_bytes,
                          int B, int T, int H, int d_k, int d_v, int chunk,
                          int dtype, int* d_status, void* stream);
+
+/*
+ * gdr_chunk_fwd_workspace_size -- bytes of scratch gdr_chunk_fwd's two-pass
+ * path needs for this shape and gate form, or 0 when it has none. Two-pass
+ * forms: dtype GDR_BF16, d_k = 128, d_v in {64, 128}, scalar alpha, tied
+ * scalar beta (Gated DeltaNet). Size: B*T*H*(d_k + d_v) bf16 values (the
+ * per-token rows of -W = -T Diag(beta g) K and of T Diag(beta) V).
+ * Host-only; launches nothing.
+ */
+size_t gdr_chunk_fwd_workspace_size(int B, int T, int H, int d_k, int d_v,
+                                    int alpha_kind, int b_kind, int w_kind,
+                                    int dtype);
 
 /*
  * gdr_decode_step -- one token per head (autoregressive decoding).

@@ -12,13 +12,15 @@ def to_dev(x, dev):
     return None if x is None else x.to(dev).contiguous()
 
 
-def run_chunk(inp, dev, S0="inp", final_state=True, d_status=None):
+def run_chunk(inp, dev, S0="inp", final_state=True, d_status=None, workspace="auto"):
+    """chunk_fwd on the device; workspace="auto" takes the two-pass path where
+    the gate form has one, None forces the single-pass kernels."""
     g = inp["gates"]
     w = TIED if g["w"] == "tied" else to_dev(inp["w"], dev)
     s0 = inp["S0"] if isinstance(S0, str) else S0
     o, ST = chunk_fwd(to_dev(inp["q"], dev), to_dev(inp["k"], dev), to_dev(inp["v"], dev),
                       to_dev(inp["alpha"], dev), to_dev(inp["b"], dev), w, to_dev(s0, dev),
-                      final_state=final_state, d_status=d_status)
+                      final_state=final_state, d_status=d_status, workspace=workspace)
     torch.cuda.synchronize()
     return o.float().cpu().numpy(), (None if ST is None else ST.cpu().numpy())
 

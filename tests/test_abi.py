@@ -19,7 +19,7 @@ NULL = None
 def declared_functions():
     src = open(HEADER).read()
     src = re.sub(r"/\*.*?\*/", "", src, flags=re.S)
-    return sorted(set(re.findall(r"^\s*(?:gdr_status|const char\*|int)\s+(gdr_\w+)\s*\(", src, flags=re.M)))
+    return sorted(set(re.findall(r"^\s*(?:gdr_status|const char\*|int|size_t)\s+(gdr_\w+)\s*\(", src, flags=re.M)))
 
 
 def test_header_declares_the_entry_points():
@@ -40,13 +40,13 @@ def test_library_is_in_tree():
 
 
 def chunk(**kw):
-    a = dict(q=P, k=P, v=P, alpha=P, b=P, w=NULL, ak=1, bk=1, wk=3, S0=NULL, o=P, ST=P, B=1, T=64,
-             H=1, dk=128, dv=128, chunk=64, dtype=0)
+    a = dict(q=P, k=P, v=P, alpha=P, b=P, w=NULL, ak=1, bk=1, wk=3, S0=NULL, o=P, ST=P, ws=NULL,
+             ws_bytes=0, B=1, T=64, H=1, dk=128, dv=128, chunk=64, dtype=0)
     a.update(kw)
     lib = _lib.load()
     return lib.gdr_chunk_fwd(a["q"], a["k"], a["v"], a["alpha"], a["b"], a["w"], a["ak"], a["bk"],
-                             a["wk"], a["S0"], a["o"], a["ST"], a["B"], a["T"], a["H"], a["dk"],
-                             a["dv"], a["chunk"], a["dtype"], None, None)
+                             a["wk"], a["S0"], a["o"], a["ST"], a["ws"], a["ws_bytes"], a["B"],
+                             a["T"], a["H"], a["dk"], a["dv"], a["chunk"], a["dtype"], None, None)
 
 
 @pytest.mark.parametrize("kw,expect", [
@@ -69,6 +69,8 @@ def chunk(**kw):
     (dict(o=P + 2), _lib.GDR_ERR_MISALIGNED),
     (dict(ST=P + 4), _lib.GDR_ERR_MISALIGNED),
     (dict(ak=2, alpha=P + 2), _lib.GDR_ERR_MISALIGNED),
+    (dict(ws=P, ws_bytes=1024), _lib.GDR_ERR_INVALID_ARG),          # workspace too small
+    (dict(ws=P + 16, ws_bytes=1 << 30), _lib.GDR_ERR_MISALIGNED),   # workspace not 256-aligned
 ])
 def test_chunk_fwd_rejects_bad_arguments(kw, expect):
     assert chunk(**kw) == expect
@@ -99,5 +101,18 @@ def test_decode_step_rejects_bad_arguments(kw, expect):
 
 def test_binding_raises_on_error_status():
     with pytest.raises(_lib.GdrError):
-        _lib.gdr_chunk_fwd(P, P, P, P, P, None, 1, 1, 3, None, P, P, 0, 64, 1, 128, 128, 64, 0,
-                           stream=0)
+        _lib.gdr_chunk_fwd(P, P, P, P, P, None, 1, 1, 3, None, P, P, None, 0, 0, 64, 1, 128, 128,
+                           64, 0, stream=0)
+
+
+@pytest.mark.parametrize("shape,kinds,expect", [
+    ((4, 4096, 16, 128, 128), (1, 1, 3), 4 * 4096 * 16 * (128 + 128) * 2),   # GDN form
+    ((1, 100, 2, 128, 64), (1, 1, 3), 1 * 100 * 2 * (128 + 64) * 2),
+    ((1, 64, 1, 128, 256), (1, 1, 3), 0),          # d_v > 128: single pass only
+    ((1, 64, 1, 128, 128), (2, 1, 3), 0),          # channel decay: single pass only
+    ((1, 64, 1, 64, 64), (1, 1, 3), 0),            # not the tensor-core shape
+    ((1, 0, 1, 128, 128), (1, 1, 3), 0),
+])
+def test_workspace_size(shape, kinds, expect):
+    B, T, H, dk, dv = shape
+    assert _lib.gdr_chunk_fwd_workspace_size(B, T, H, dk, dv, *kinds, 0) == expect

@@ -7,7 +7,7 @@ import numpy as np
 import pytest
 import torch
 
-from gated_delta_rule_147_b200 import GDR_DEVICE_DECAY_RANGE, chunk_fwd
+from gated_delta_rule_147_b200 import GDR_DEVICE_DECAY_RANGE, TIED, chunk_fwd
 from gated_delta_rule_147_b200.inputs import WORKLOADS, make_chunk_inputs
 from gpu_util import TOL, assert_close, gather_heads, run_chunk, run_oracle
 
@@ -181,3 +181,55 @@ def test_gla_full_size_sampled_heads(cuda_device):
     o_s, ST_s = gather_heads(o, ST, heads)
     assert_close(o_s, o_ref, TOL["bf16"], f"o {heads}")
     assert_close(ST_s, ST_ref, TOL["bf16"], f"S_T {heads}")
+
+
+# ---- two-pass path (per-chunk factors in parallel, then the state pass) -----
+# The Gated DeltaNet form (scalar alpha, tied beta, d_v <= 128) takes it by
+# default; these also run the same inputs through the single-pass kernel.
+
+@pytest.mark.parametrize("T", [1, 63, 64, 65, 200, 1000])
+@pytest.mark.parametrize("dv", [64, 128])
+def test_two_pass_matches_oracle_and_single_pass(cuda_device, T, dv):
+    wl = small("gdn", T=T, dv=dv, s0=True, seed=300 + T + dv)
+    inp = make_chunk_inputs(wl)
+    o2, S2 = run_chunk(inp, cuda_device)                      # two-pass
+    o1, S1 = run_chunk(inp, cuda_device, workspace=None)      # single pass
+    o_ref, ST_ref = run_oracle(inp)
+    assert_close(o2, o_ref, TOL["bf16"], "o (two-pass)")
+    assert_close(S2, ST_ref, TOL["bf16"], "S_T (two-pass)")
+    assert_close(o1, o_ref, TOL["bf16"], "o (single pass)")
+    assert_close(S1, ST_ref, TOL["bf16"], "S_T (single pass)")
+
+
+def test_two_pass_workspace_is_used(cuda_device):
+    """The two-pass path writes the per-token rows of -W and P into the
+    caller's workspace: row t of -W is -(T Diag(beta g) K)_t, so a token whose
+    beta is 0 gets a zero row in both."""
+    wl = small("gdn", T=130, B=1, H=2, seed=17)
+    inp = make_chunk_inputs(wl)
+    inp["b"][0, 5, 1] = 0.0
+    dev = cuda_device
+    q, k, v, a, b = (inp[x].to(dev) for x in ("q", "k", "v", "alpha", "b"))
+    from gated_delta_rule_147_b200 import workspace_bytes
+    nbytes = workspace_bytes(q, v, a, b, TIED)
+    assert nbytes == 1 * 130 * 2 * (128 + 128) * 2
+    ws = torch.full((nbytes,), 0x7F, dtype=torch.uint8, device=dev)
+    chunk_fwd(q, k, v, a, b, TIED, None, workspace=ws)
+    torch.cuda.synchronize()
+    half = 130 * 2 * 128
+    wneg = ws[: half * 2].view(torch.bfloat16).view(1, 130, 2, 128).float().cpu()
+    p = ws[half * 2:].view(torch.bfloat16).view(1, 130, 2, 128).float().cpu()
+    assert torch.all(wneg[0, 5, 1] == 0) and torch.all(p[0, 5, 1] == 0)
+    assert torch.isfinite(wneg).all() and torch.isfinite(p).all()
+    assert wneg.abs().sum() > 0 and p.abs().sum() > 0
+
+
+def test_two_pass_full_size_matches_single_pass(cuda_device):
+    """Full Gated DeltaNet workload: the two paths agree everywhere (both
+    were checked against the oracle on sampled heads above)."""
+    wl = WORKLOADS["gdn"]
+    inp = make_chunk_inputs(wl)
+    o2, S2 = run_chunk(inp, cuda_device)
+    o1, S1 = run_chunk(inp, cuda_device, workspace=None)
+    assert_close(o2, o1, 2e-2, "o two-pass vs single pass")
+    assert_close(S2, S1, 2e-2, "S_T two-pass vs single pass")
