@@ -46,6 +46,8 @@ _CSRC = "gated_delta_rule_147_b200/csrc/"
 KERNEL_SOURCES = {
     "general": (_CSRC + "chunk_sm100.cu", _CSRC + "chunk_common.cuh", _CSRC + "common.cuh"),
     "twopass": (_CSRC + "chunk_twopass_sm100.cu", _CSRC + "chunk_common.cuh", _CSRC + "common.cuh"),
+    "twopass_general": (_CSRC + "chunk_twopass_general_sm100.cu", _CSRC + "chunk_common.cuh",
+                        _CSRC + "common.cuh"),
     "erasefree": (_CSRC + "chunk_erasefree_sm100.cu", _CSRC + "chunk_common.cuh",
                   _CSRC + "common.cuh"),
 }
@@ -55,16 +57,18 @@ KERNEL_NAMES = {
     "general": "gdr::chunk::chunk_fwd_kernel / chunk_fwd_gdn_kernel (single pass)",
     "twopass": "gdr::twopass::prep_gdn_kernel + gdr::twopass::state_gdn_kernel (one call, two launches)",
     "erasefree": "gdr::erasefree::chunk_fwd_erasefree_kernel",
+    "twopass_general": "gdr::twopass_g::prep_general_kernel + state_general_kernel (one call, two launches)",
 }
-LAUNCHES_PER_CALL = {"general": 1, "twopass": 2, "erasefree": 1}
+LAUNCHES_PER_CALL = {"general": 1, "twopass": 2, "erasefree": 1, "twopass_general": 2}
 
 
 def kernel_family(wl) -> str:
     if wl.b == "none":
         return "erasefree"
-    if (wl.dtype == "bf16" and wl.dk == 128 and wl.dv in (64, 128) and wl.alpha == "scalar"
-            and wl.b == "scalar" and wl.w == "tied"):
-        return "twopass"
+    if wl.dtype == "bf16" and wl.dk == 128 and wl.dv in (64, 128) and wl.T > 0:
+        if wl.alpha == "scalar" and wl.b == "scalar" and wl.w == "tied":
+            return "twopass"
+        return "twopass_general"
     return "general"
 
 
@@ -370,7 +374,7 @@ def run_ours(args):
                                        f"b={w2.b} w={w2.w} S0={'random' if w2.s0 else 'zero'}",
                            "tokens_per_s": w2.B * w2.T / (a2 * 1e-3), "ms_per_launch": a2,
                            "hbm_gbs": b2 / (a2 * 1e-3) / 1e9, "roofline_frac": rt / (a2 * 1e-3),
-                           "traffic": measured_traffic(name)}
+                           "traffic": measured_traffic(name), "kernel": KERNEL_NAMES[kernel_family(w2)]}
             torch.cuda.empty_cache()
         dec = time_decode(dev, 1000, 10)
         dec["frac_of_hbm"] = dec["total_gbs"] / pk["hbm_gbs"]

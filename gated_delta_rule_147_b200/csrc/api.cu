@@ -24,6 +24,14 @@ cudaError_t launch_chunk_twopass_gdn(const CUtensorMap* maps, const CUtensorMap*
                                      const void* alpha, const void* beta, const float* S0, void* o,
                                      float* ST, int* d_status, int B, int T, int H, int dv,
                                      cudaStream_t st);
+size_t twopass_general_workspace_bytes(int B, int T, int H, int dv, bool untied);
+cudaError_t launch_chunk_twopass_general(const CUtensorMap* maps,
+                                         bool (*make_map)(CUtensorMap*, const void*, int, int, int, int),
+                                         void* ws, const void* q, const void* k, const void* alpha,
+                                         const void* b, const void* w, int akind, int bkind,
+                                         int wkind, const float* S0, void* o, float* ST,
+                                         int* d_status, int B, int T, int H, int dv,
+                                         cudaStream_t st);
 cudaError_t launch_chunk_sm100(const CUtensorMap* maps, const void* alpha, const void* b,
                                const void* w, int akind, int bkind, int wkind, bool tied,
                                const float* S0, void* o, float* ST, int* d_status, int B, int T,
@@ -75,12 +83,25 @@ bool make_map(CUtensorMap* m, const void* base, int B, int T, int H, int d) {
     return r == CUDA_SUCCESS;
 }
 
-// The two-pass path (per-chunk factors for all chunks in parallel, then the
-// state pass) exists for the tensor-core shape with scalar decay and tied
-// scalar beta, d_v <= 128.
-bool twopass_applies(int T, int d_k, int d_v, int ak, int bk, int wk, int dtype) {
-    return T > 0 && dtype == GDR_BF16 && d_k == 128 && (d_v == 64 || d_v == 128) &&
-           ak == GDR_GATE_SCALAR && bk == GDR_GATE_SCALAR && wk == GDR_GATE_TIED;
+// Two-pass paths (per-chunk factors of all chunks in parallel, then the state
+// pass) exist for the tensor-core shape with an erase gate and d_v <= 128:
+// the Gated DeltaNet form (scalar decay, tied scalar beta) has its own pair of
+// kernels, every other gate form the general pair.
+enum TwoPass { TP_NONE = 0, TP_GDN = 1, TP_GENERAL = 2 };
+
+TwoPass twopass_kind(int T, int d_k, int d_v, int ak, int bk, int wk, int dtype) {
+    if (T <= 0 || dtype != GDR_BF16 || d_k != 128 || !(d_v == 64 || d_v == 128)) return TP_NONE;
+    if (bk == GDR_GATE_NONE) return TP_NONE;  // erase-free: single pass, no solve
+    if (ak == GDR_GATE_SCALAR && bk == GDR_GATE_SCALAR && wk == GDR_GATE_TIED) return TP_GDN;
+    return TP_GENERAL;
+}
+
+size_t twopass_bytes(TwoPass kind, int B, int T, int H, int d_v, int bk, int wk) {
+    if (kind == TP_GDN) return gdr::twopass_workspace_bytes(B, T, H, d_v);
+    if (kind == TP_GENERAL)
+        return gdr::twopass_general_workspace_bytes(B, T, H, d_v,
+                                                    !(wk == GDR_GATE_TIED && bk == GDR_GATE_SCALAR));
+    return 0;
 }
 
 }  // namespace
@@ -89,8 +110,9 @@ extern "C" {
 
 size_t gdr_chunk_fwd_workspace_size(int B, int T, int H, int d_k, int d_v, int alpha_kind,
                                     int b_kind, int w_kind, int dtype) {
-    if (B < 1 || H < 1 || !twopass_applies(T, d_k, d_v, alpha_kind, b_kind, w_kind, dtype)) return 0;
-    return gdr::twopass_workspace_bytes(B, T, H, d_v);
+    if (B < 1 || H < 1) return 0;
+    return twopass_bytes(twopass_kind(T, d_k, d_v, alpha_kind, b_kind, w_kind, dtype), B, T, H, d_v,
+                         b_kind, w_kind);
 }
 
 const char* gdr_status_string(int s) {
@@ -143,10 +165,11 @@ gdr_status gdr_chunk_fwd(const void* q, const void* k, const void* v, const void
         (w_kind == GDR_GATE_CHANNEL && !aligned16(w)))
         return GDR_ERR_MISALIGNED;
 
-    const bool twopass = workspace != nullptr && twopass_applies(T, d_k, d_v, alpha_kind, b_kind,
-                                                                 w_kind, dtype);
-    if (twopass) {
-        if (workspace_bytes < gdr::twopass_workspace_bytes(B, T, H, d_v)) return GDR_ERR_INVALID_ARG;
+    const TwoPass tp = workspace != nullptr
+                           ? twopass_kind(T, d_k, d_v, alpha_kind, b_kind, w_kind, dtype)
+                           : TP_NONE;
+    if (tp != TP_NONE) {
+        if (workspace_bytes < twopass_bytes(tp, B, T, H, d_v, b_kind, w_kind)) return GDR_ERR_INVALID_ARG;
         if ((reinterpret_cast<uintptr_t>(workspace) & 255u) != 0) return GDR_ERR_MISALIGNED;
     }
 
@@ -163,7 +186,11 @@ gdr_status gdr_chunk_fwd(const void* q, const void* k, const void* v, const void
             !make_map(&maps[4], bmap, B, T, H, d_k) || !make_map(&maps[5], wmap, B, T, H, d_k))
             return GDR_ERR_INVALID_ARG;
         const bool tied = w_kind == GDR_GATE_TIED && b_kind == GDR_GATE_SCALAR;
-        if (twopass) {
+        if (tp == TP_GENERAL) {
+            e = gdr::launch_chunk_twopass_general(maps, make_map, workspace, q, k, alpha, b, w,
+                                                  alpha_kind, b_kind, w_kind, S0, o, S_T, d_status,
+                                                  B, T, H, d_v, st);
+        } else if (tp == TP_GDN) {
             CUtensorMap ws_maps[2];
             const uint8_t* pbase = reinterpret_cast<const uint8_t*>(workspace) +
                                    (size_t)B * T * H * d_k * sizeof(uint16_t);

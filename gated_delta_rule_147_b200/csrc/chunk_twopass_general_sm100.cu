@@ -1,0 +1,845 @@
+// Two-pass chunkwise forward for channel-wise decay and for independent erase
+// / write gates (Kimi Delta Attention and Gated DeltaNet-2 forms) on sm_100a.
+//
+// Same chunk algebra as the single-pass kernel ("Recurrent Memory: Write,
+// Erase, Decay, Read" sections 03-05; "Erase-then-Delta Attention" abstract),
+// with l_r the per-channel prefix sum of log2 alpha over the chunk, ref the
+// chunk's reference, rowf = 2^(l - ref), colf = 2^(ref - l), g = 2^l:
+//   Kb = b.k.rowf   Qs = q.rowf   Ks = k.colf   Kws = w.k.colf
+//   A  = strict_lower(Kb Ks^T)    Bm = strict_lower(Kb Kws^T)
+//   Aq = lower(Qs Ks^T)           Bq = lower(Qs Kws^T)
+//   T  = (I + A)^-1,  W = T Kb . 2^ref
+// Everything that does not involve the state is formed in pass 1, one CTA per
+// chunk, all chunks of all heads in parallel, into a workspace:
+//   WN = -W          QG = q.g               K2 = k.g_{n-1}/g    AQ = Aq
+//   P  = T Diag(beta) V (tied beta)  or  -T Bm V (independent gates)
+//   KW2 = w.k.g_{n-1}/g,  BQ = Bq    (independent gates only)
+//   GC = g_{n-1}  (fp32, per chunk and channel)
+// Pass 2 walks the chunks of one (batch, head, 64 columns of d_v) in order:
+//   U  = P + WN S
+//   O  = QG S + AQ U (+ BQ V)
+//   S' = Diag(GC) S + K2^T U (+ KW2^T V)
+// With tied beta, Bm = A Diag(beta) and Bq = Aq Diag(beta), so U + Diag(beta) V
+// = T Diag(beta) V - W S replaces U and the V terms drop out.
+#include "chunk_common.cuh"
+
+namespace gdr {
+namespace twopass_g {
+
+using namespace chunkc;
+
+// ---- pass 1 shared memory (bytes from a 1024-aligned base) ----------------
+// M = 128 MMAs read A rows 64..127 beyond each 64-row operand; those rows
+// land in the next region (garbage rows whose outputs are never read).
+constexpr uint32_t G_OFF_ROP = 0;       // [Kb ; Qs] bf16 [128 x 128] (two 16 KB column blocks);
+                                        // after P1 the Qs rows hold the V tiles
+constexpr uint32_t G_OFF_COP = 32768;   // [Ks ; Kws] bf16 [64 | 128 x 128]; after P1: A32, T32
+constexpr uint32_t G_OFF_A32 = 32768;   // A fp32 [64 x 64]
+constexpr uint32_t G_OFF_T32 = 49152;   // T fp32 [64 x 64]
+constexpr uint32_t G_OFF_SCR = 65536;   // decay-scan scratch in the build, solve scratch after (5 KB)
+constexpr uint32_t G_OFF_APRE = 71680;  // T Diag(beta) (tied) or -T Bm, bf16 [64 x 64]
+constexpr uint32_t G_OFF_L = 79872;     // T bf16 [64 x 64]
+constexpr uint32_t G_OFF_X = 88064;     // Bm bf16 [64 x 64]
+constexpr uint32_t G_OFF_SMALL = 96256;
+constexpr uint32_t G_SMEM_BYTES = G_OFF_SMALL + 3072 + 1024;
+constexpr uint32_t G_TM_COLS = 256;
+
+struct GPrepParams {
+    const __nv_bfloat16* q;
+    const __nv_bfloat16* k;
+    const __nv_bfloat16* alpha;
+    const __nv_bfloat16* bg;
+    const __nv_bfloat16* wg;
+    __nv_bfloat16 *wn, *qg, *k2, *kw2, *aq, *bq, *p;  // [B, T, H, d]
+    float* gc;                                        // [B, H, nchunks, 128]
+    int* d_status;
+    int T, H, dv, akind, bkind, wkind;
+};
+
+__device__ __forceinline__ void ld8b(const __nv_bfloat16* p, uint2& u) {
+    u = *reinterpret_cast<const uint2*>(p);
+}
+__device__ __forceinline__ void unpack4(const uint2& u, float* x4) {
+    const float2 f0 = __bfloat1622float2(*reinterpret_cast<const __nv_bfloat162*>(&u.x));
+    const float2 f1 = __bfloat1622float2(*reinterpret_cast<const __nv_bfloat162*>(&u.y));
+    x4[0] = f0.x; x4[1] = f0.y; x4[2] = f1.x; x4[3] = f1.y;
+}
+__device__ __forceinline__ void st8b(__nv_bfloat16* p, const float* x4) {
+    uint2 u;
+    u.x = pack_bf16x2(x4[0], x4[1]);
+    u.y = pack_bf16x2(x4[2], x4[3]);
+    *reinterpret_cast<uint2*>(p) = u;
+}
+// 32 consecutive fp32 values (one thread's TMEM row slice) -> bf16 in global
+__device__ __forceinline__ void st32_bf16(__nv_bfloat16* p, const float* x, float sign) {
+#pragma unroll
+    for (int c8 = 0; c8 < 4; ++c8) {
+        uint4 u;
+        u.x = pack_bf16x2(sign * x[c8 * 8 + 0], sign * x[c8 * 8 + 1]);
+        u.y = pack_bf16x2(sign * x[c8 * 8 + 2], sign * x[c8 * 8 + 3]);
+        u.z = pack_bf16x2(sign * x[c8 * 8 + 4], sign * x[c8 * 8 + 5]);
+        u.w = pack_bf16x2(sign * x[c8 * 8 + 6], sign * x[c8 * 8 + 7]);
+        *reinterpret_cast<uint4*>(p + c8 * 8) = u;
+    }
+}
+
+template <bool TIED, bool ACH>
+__global__ void __launch_bounds__(NT, 2) prep_general_kernel(const __grid_constant__ CUtensorMap tm_v,
+                                                             const GPrepParams pp) {
+    extern __shared__ uint8_t smem_raw[];
+    uint8_t* sm = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) &
+                                             ~uintptr_t(1023));
+    const int tid = threadIdx.x, warp = tid >> 5, wg = warp >> 2, row = tid & 127;
+    const int ci = blockIdx.x, h = blockIdx.y, bb = blockIdx.z;
+    const int T = pp.T, H = pp.H, dv = pp.dv;
+    const int nchunks = (T + C - 1) / C;
+    const int t0 = ci * C;
+    const int n = min(C, T - t0);
+    const int nvt = dv / 64;
+    const bool bch = pp.bkind == GDR_GATE_CHANNEL, wch = pp.wkind == GDR_GATE_CHANNEL;
+    constexpr int N1 = TIED ? 64 : 128;  // rows of [Ks ; Kws]
+
+    float* s_ascal = reinterpret_cast<float*>(sm + G_OFF_SMALL);
+    float* s_bscal = s_ascal + 64;
+    float* s_wscal = s_ascal + 128;
+    float* s_rowf = s_ascal + 192;
+    float* s_colf = s_ascal + 256;
+    float* s_eref = s_ascal + 320;   // [128] 2^ref
+    float* s_gC = s_ascal + 448;     // [128] g_{n-1}
+    float* s_fS = s_ascal + 576;     // [128] 2^(l_{n-1} - ref)
+    uint64_t* bar_v = reinterpret_cast<uint64_t*>(sm + G_OFF_SMALL + 2816);
+    uint64_t* bar_mma = bar_v + 1;
+    uint32_t* s_tmem = reinterpret_cast<uint32_t*>(sm + G_OFF_SMALL + 2832);
+    const uint32_t sbase = smem_u32(sm);
+
+    if (tid == 0) {
+        mbar_init(bar_v, 1);
+        mbar_init(bar_mma, 1);
+        fence_barrier_init();
+        prefetch_tmap(&tm_v);
+    }
+    if (warp == 0) tmem_alloc(s_tmem, G_TM_COLS);
+    if (tid < C) {
+        const bool valid = tid < n;
+        const size_t gi = ((size_t)bb * T + (valid ? t0 + tid : t0)) * H + h;
+        s_ascal[tid] = (pp.akind == GDR_GATE_SCALAR && valid) ? to_f32(pp.alpha[gi]) : 1.f;
+        s_bscal[tid] = (pp.bkind == GDR_GATE_SCALAR && valid) ? to_f32(pp.bg[gi]) : 0.f;
+        s_wscal[tid] = (pp.wkind == GDR_GATE_SCALAR && valid) ? to_f32(pp.wg[gi])
+                       : (pp.wkind == GDR_GATE_NONE ? 1.f : 0.f);
+    }
+    tc_fence_before();
+    __syncthreads();
+    tc_fence_after();
+    const uint32_t tmem = *s_tmem;
+    const uint32_t lane_base = (uint32_t)((warp & 3) * 32) << 16;
+    uint32_t ph_v = 0, ph_mma = 0;
+    bool ok = true;
+
+#define GDR_WAIT(bar, ph)                                                   \
+    do {                                                                    \
+        bool w_ok = mbar_wait(bar, ph);                                     \
+        ph ^= 1u;                                                           \
+        if (!__syncthreads_and(w_ok)) { ok = false; goto finish; }          \
+    } while (0)
+#define GDR_BEFORE_MMA()    \
+    do {                    \
+        fence_proxy_async(); \
+        tc_fence_before();  \
+        __syncthreads();    \
+    } while (0)
+
+    // ---- build: thread = 8 tokens (rg = warp) x 4 channels (cg = lane) --------
+    {
+        const int cg = tid & 31, rg = warp;
+        const int ch0 = cg * 4;
+        // issue every global load of this thread first
+        uint2 qa[8], ka[8], aa[8], ba[8], wa[8];
+#pragma unroll
+        for (int i = 0; i < 8; ++i) {
+            const int r = rg * 8 + i;
+            const int t = t0 + min(r, n - 1);
+            const size_t e = (((size_t)bb * T + t) * H + h) * DK + ch0;
+            ld8b(pp.q + e, qa[i]);
+            ld8b(pp.k + e, ka[i]);
+            if (ACH) ld8b(pp.alpha + e, aa[i]);
+            if (bch) ld8b(pp.bg + e, ba[i]);
+            if (!TIED && wch) ld8b(pp.wg + e, wa[i]);
+        }
+        float* scan = reinterpret_cast<float*>(sm + G_OFF_SCR);  // [8 rg][128 ch] + [128]
+        float lrow0[4];   // channel decay: l at this thread's first token - ref
+        float aval[8][4];
+        if (!ACH) {
+            if (warp == 0) {
+                const int lane = tid;
+                const float la0 = (2 * lane < n) ? lg2_approx(s_ascal[2 * lane]) : 0.f;
+                const float la1 = (2 * lane + 1 < n) ? lg2_approx(s_ascal[2 * lane + 1]) : 0.f;
+                float x = la0 + la1;
+#pragma unroll
+                for (int off = 1; off < 32; off <<= 1) {
+                    const float y = __shfl_up_sync(0xffffffffu, x, off);
+                    if (lane >= off) x += y;
+                }
+                const float l1 = x, l0v = x - la1;
+                const float first = __shfl_sync(0xffffffffu, l0v, 0);
+                const float last = __shfl_sync(0xffffffffu, l1, 31);
+                const float ref = 0.5f * (first + last);
+                s_rowf[2 * lane] = ex2_approx(l0v - ref);
+                s_rowf[2 * lane + 1] = ex2_approx(l1 - ref);
+                s_colf[2 * lane] = ex2_approx(ref - l0v);
+                s_colf[2 * lane + 1] = ex2_approx(ref - l1);
+                if (lane == 0) {
+                    scan[0] = ex2_approx(ref);
+                    scan[1] = ex2_approx(last);
+                    scan[2] = ex2_approx(last - ref);
+                    if (first - last > 230.f) flag_status(pp.d_status, GDR_DEVICE_DECAY_RANGE);
+                }
+            }
+            __syncthreads();
+            if (tid < 128) {
+                s_eref[tid] = scan[0];
+                s_gC[tid] = scan[1];
+                s_fS[tid] = scan[2];
+            }
+            __syncthreads();
+        } else {
+            float loc[4] = {0.f, 0.f, 0.f, 0.f};
+#pragma unroll
+            for (int i = 0; i < 8; ++i) {
+                const int r = rg * 8 + i;
+                unpack4(aa[i], aval[i]);
+#pragma unroll
+                for (int e = 0; e < 4; ++e) {
+                    if (r >= n) aval[i][e] = 1.f;  // padding tokens do not decay
+                    loc[e] += lg2_approx(aval[i][e]);
+                    if (i == 0) lrow0[e] = loc[e];
+                }
+            }
+            *reinterpret_cast<float4*>(scan + rg * 128 + ch0) = make_float4(loc[0], loc[1], loc[2], loc[3]);
+            if (rg == 0)
+                *reinterpret_cast<float4*>(scan + 1024 + ch0) = make_float4(lrow0[0], lrow0[1], lrow0[2], lrow0[3]);
+            __syncthreads();
+            float pre[4] = {0.f, 0.f, 0.f, 0.f}, tot[4] = {0.f, 0.f, 0.f, 0.f};
+#pragma unroll
+            for (int g = 0; g < 8; ++g) {
+                const float4 x = *reinterpret_cast<const float4*>(scan + g * 128 + ch0);
+                const float xs[4] = {x.x, x.y, x.z, x.w};
+#pragma unroll
+                for (int e = 0; e < 4; ++e) {
+                    if (g < rg) pre[e] += xs[e];
+                    tot[e] += xs[e];
+                }
+            }
+            const float4 l04 = *reinterpret_cast<const float4*>(scan + 1024 + ch0);
+            const float l0[4] = {l04.x, l04.y, l04.z, l04.w};
+            bool bad = false;
+#pragma unroll
+            for (int e = 0; e < 4; ++e) {
+                const float ref = 0.5f * (l0[e] + tot[e]);  // tot = l_{n-1} (padding adds 0)
+                bad |= (l0[e] - tot[e]) > 230.f;
+                lrow0[e] += pre[e] - ref;
+                if (rg == 0) {
+                    s_eref[ch0 + e] = ex2_approx(ref);
+                    s_gC[ch0 + e] = ex2_approx(tot[e]);
+                    s_fS[ch0 + e] = ex2_approx(tot[e] - ref);
+                }
+            }
+            if (bad) flag_status(pp.d_status, GDR_DEVICE_DECAY_RANGE);
+            __syncthreads();  // every channel's eref / fS is needed below
+        }
+        float er[4], fs[4];
+        {
+            const float4 e4 = *reinterpret_cast<const float4*>(s_eref + ch0);
+            const float4 f4 = *reinterpret_cast<const float4*>(s_fS + ch0);
+            er[0] = e4.x; er[1] = e4.y; er[2] = e4.z; er[3] = e4.w;
+            fs[0] = f4.x; fs[1] = f4.y; fs[2] = f4.z; fs[3] = f4.w;
+        }
+        if (rg == 0) {
+            const float4 g4 = *reinterpret_cast<const float4*>(s_gC + ch0);
+            *reinterpret_cast<float4*>(pp.gc + (((size_t)bb * H + h) * nchunks + ci) * DK + ch0) = g4;
+        }
+        float rowf_c[4];
+#pragma unroll
+        for (int i = 0; i < 8; ++i) {
+            const int r = rg * 8 + i;
+            const bool valid = r < n;
+            float k4[4], q4[4], b4[4], w4[4];
+            unpack4(ka[i], k4);
+            unpack4(qa[i], q4);
+            if (bch) unpack4(ba[i], b4);
+            else {
+#pragma unroll
+                for (int e = 0; e < 4; ++e) b4[e] = s_bscal[r];
+            }
+            if (!TIED) {
+                if (pp.wkind == GDR_GATE_TIED) {
+#pragma unroll
+                    for (int e = 0; e < 4; ++e) w4[e] = b4[e];
+                } else if (wch) {
+                    unpack4(wa[i], w4);
+                } else {
+#pragma unroll
+                    for (int e = 0; e < 4; ++e) w4[e] = s_wscal[r];
+                }
+            }
+            if (ACH) {
+#pragma unroll
+                for (int e = 0; e < 4; ++e)
+                    rowf_c[e] = (i == 0) ? ex2_approx(lrow0[e]) : rowf_c[e] * aval[i][e];
+            }
+            const float rs = ACH ? 0.f : s_rowf[r], cs = ACH ? 0.f : s_colf[r];
+            float kb[4], qs[4], ks[4], kws[4], qg[4], k2[4], kw2[4];
+#pragma unroll
+            for (int e = 0; e < 4; ++e) {
+                const float rowf = ACH ? rowf_c[e] : rs;
+                const float colf = ACH ? rcp_newton(rowf) : cs;
+                const float kk = valid ? k4[e] : 0.f;
+                const float qq = valid ? q4[e] : 0.f;
+                kb[e] = b4[e] * kk * rowf;
+                qs[e] = qq * rowf;
+                ks[e] = kk * colf;
+                kws[e] = TIED ? 0.f : w4[e] * kk * colf;
+                qg[e] = qs[e] * er[e];
+                k2[e] = ks[e] * fs[e];
+                kw2[e] = kws[e] * fs[e];
+            }
+            st4(sm + G_OFF_ROP, piece4(r, cg, 128), kb);
+            st4(sm + G_OFF_ROP, piece4(64 + r, cg, 128), qs);
+            st4(sm + G_OFF_COP, piece4(r, cg, N1), ks);
+            if (!TIED) st4(sm + G_OFF_COP, piece4(64 + r, cg, N1), kws);
+            if (valid) {
+                const size_t e = (((size_t)bb * T + t0 + r) * H + h) * DK + ch0;
+                st8b(pp.qg + e, qg);
+                st8b(pp.k2 + e, k2);
+                if (!TIED) st8b(pp.kw2 + e, kw2);
+            }
+        }
+    }
+    GDR_BEFORE_MMA();
+
+    // ---- P1: D1 = [Kb ; Qs] x [Ks ; Kws]^T ---------------------------------------
+    if (tid == 0) {
+        tc_fence_after();
+        const uint32_t id = idesc_bf16(128, N1, 0, 0);
+#pragma unroll
+        for (int ks = 0; ks < 8; ++ks) {
+            const uint32_t koff = (ks >> 2) * 16384u + (ks & 3) * 32u;
+            const uint32_t koffb = (ks >> 2) * (uint32_t)(N1 * 128) + (ks & 3) * 32u;
+            mma_bf16(tmem, sdesc_sw128(sbase + G_OFF_ROP + koff, 16, 1024),
+                     sdesc_sw128(sbase + G_OFF_COP + koffb, 16, 1024), id, ks > 0);
+        }
+        mma_commit(bar_mma);
+    }
+    GDR_WAIT(bar_mma, ph_mma);
+    tc_fence_after();
+    // the Qs rows are consumed: V's tiles go there (column block vt, rows 64..127)
+    if (tid == 0) {
+        mbar_expect_tx(bar_v, (uint32_t)nvt * 8192u);
+        for (int vt = 0; vt < nvt; ++vt)
+            tma_load_4d(sm + G_OFF_ROP + vt * 16384 + 8192, &tm_v, bar_v, vt * 64, h, t0, bb);
+    }
+
+    // ---- unload D1: A (fp32) + transposed diagonal blocks; Bm -> X; Aq, Bq -> workspace
+    {
+        const int r = row & 63;
+        float d[32], d2[32];
+        tmem_ld32_async(tmem + lane_base + wg * 32, d);
+        if (!TIED) tmem_ld32_async(tmem + lane_base + 64 + wg * 32, d2);
+        tmem_wait_ld();
+        if (row < 64) {
+            float* A32 = reinterpret_cast<float*>(sm + G_OFF_A32);
+#pragma unroll
+            for (int j4 = 0; j4 < 32; j4 += 4) {
+                const int j = wg * 32 + j4;
+                const float4 x = make_float4(j < r ? d[j4] : 0.f, j + 1 < r ? d[j4 + 1] : 0.f,
+                                             j + 2 < r ? d[j4 + 2] : 0.f, j + 3 < r ? d[j4 + 3] : 0.f);
+                *reinterpret_cast<float4*>(f32_at(A32, r, j)) = x;
+            }
+            const int I = r >> 4, rr = r & 15;
+            if ((I >> 1) == wg) {
+                float* at = reinterpret_cast<float*>(sm + G_OFF_SCR) + I * 272;
+                if (I & 1) {
+#pragma unroll
+                    for (int j = 0; j < 16; ++j) at[j * 16 + rr] = j < rr ? d[16 + j] : 0.f;
+                } else {
+#pragma unroll
+                    for (int j = 0; j < 16; ++j) at[j * 16 + rr] = j < rr ? d[j] : 0.f;
+                }
+            }
+            if (!TIED) {
+#pragma unroll
+                for (int c8 = 0; c8 < 4; ++c8) {
+                    float x[8];
+#pragma unroll
+                    for (int e = 0; e < 8; ++e) x[e] = (wg * 32 + c8 * 8 + e < r) ? d2[c8 * 8 + e] : 0.f;
+                    st_chunk(sm + G_OFF_X, sw128_chunk(r, wg * 4 + c8, 64), x);
+                }
+            }
+        } else if (r < n) {
+            const size_t tok = ((size_t)bb * T + t0 + r) * H + h;
+#pragma unroll
+            for (int j = 0; j < 32; ++j) {
+                const bool keep = wg * 32 + j <= r;
+                d[j] = keep ? d[j] : 0.f;
+                if (!TIED) d2[j] = keep ? d2[j] : 0.f;
+            }
+            st32_bf16(pp.aq + tok * 64 + wg * 32, d, 1.f);
+            if (!TIED) st32_bf16(pp.bq + tok * 64 + wg * 32, d2, 1.f);
+        }
+    }
+    __syncthreads();
+
+    // ---- T = (I + A)^-1; L = T (bf16); tied: APRE = T Diag(beta) ------------------
+    {
+        float* A32 = reinterpret_cast<float*>(sm + G_OFF_A32);
+        float* T32 = reinterpret_cast<float*>(sm + G_OFF_T32);
+        solve_unit_lower(A32, T32, reinterpret_cast<float*>(sm + G_OFF_SCR), tid, warp);
+        const int r = tid & 63, q4 = tid >> 6;
+#pragma unroll
+        for (int cc = 0; cc < 2; ++cc) {
+            const int c8 = q4 * 2 + cc;
+            float x[8];
+#pragma unroll
+            for (int e4 = 0; e4 < 8; e4 += 4) {
+                const int j = c8 * 8 + e4;
+                // the block T[0:32, 32:64] is never written by the solve: it is zero
+                const float4 t4 = (j < 32 || r >= 32) ? *reinterpret_cast<const float4*>(f32_at(T32, r, j))
+                                                      : make_float4(0.f, 0.f, 0.f, 0.f);
+                x[e4] = t4.x; x[e4 + 1] = t4.y; x[e4 + 2] = t4.z; x[e4 + 3] = t4.w;
+            }
+            st_chunk(sm + G_OFF_L, sw128_chunk(r, c8, 64), x);
+            if (TIED) {
+                const float4 b0 = *reinterpret_cast<const float4*>(s_bscal + c8 * 8);
+                const float4 b1 = *reinterpret_cast<const float4*>(s_bscal + c8 * 8 + 4);
+                x[0] *= b0.x; x[1] *= b0.y; x[2] *= b0.z; x[3] *= b0.w;
+                x[4] *= b1.x; x[5] *= b1.y; x[6] *= b1.z; x[7] *= b1.w;
+                st_chunk(sm + G_OFF_APRE, sw128_chunk(r, c8, 64), x);
+            }
+        }
+    }
+    GDR_BEFORE_MMA();
+    GDR_WAIT(bar_v, ph_v);  // V arrived during the solve
+
+    // ---- P2: D2 = T Kb (cols 0..127);  tied: D3 = T Diag(beta) V (cols 128..);
+    //      general: T Bm (cols 128..191) ----------------------------------------------
+    if (tid == 0) {
+        tc_fence_after();
+        const uint32_t idW = idesc_bf16(128, 128, 0, 1);
+        const uint32_t idP = idesc_bf16(128, dv, 0, 1);
+        const uint32_t id64 = idesc_bf16(128, 64, 0, 1);
+#pragma unroll
+        for (int ks = 0; ks < 4; ++ks) {
+            const uint64_t ad = sdesc_sw128(sbase + G_OFF_L + ks * 32u, 16, 1024);
+            mma_bf16(tmem, ad, sdesc_sw128(sbase + G_OFF_ROP + ks * 2048u, 16384, 1024), idW, ks > 0);
+            if (TIED)
+                mma_bf16(tmem + 128, sdesc_sw128(sbase + G_OFF_APRE + ks * 32u, 16, 1024),
+                         sdesc_sw128(sbase + G_OFF_ROP + 8192 + ks * 2048u, 16384, 1024), idP, ks > 0);
+            else
+                mma_bf16(tmem + 128, ad, sdesc_sw128(sbase + G_OFF_X + ks * 2048u, 8192, 1024), id64, ks > 0);
+        }
+        mma_commit(bar_mma);
+    }
+    GDR_WAIT(bar_mma, ph_mma);
+    tc_fence_after();
+
+    // ---- WN = -W 2^ref (rows 0..63) -> workspace; tied: P -> workspace;
+    //      general: -T Bm -> APRE -----------------------------------------------------
+    if (row < 64) {
+        const int r = row;
+        const size_t tok = ((size_t)bb * T + t0 + r) * H + h;
+        float d[32], d1[32];
+        tmem_ld32_async(tmem + lane_base + wg * 64, d);
+        tmem_ld32_async(tmem + lane_base + wg * 64 + 32, d1);
+        tmem_wait_ld();
+#pragma unroll
+        for (int j4 = 0; j4 < 32; j4 += 4) {
+            const float4 e0 = *reinterpret_cast<const float4*>(s_eref + wg * 64 + j4);
+            const float4 e1 = *reinterpret_cast<const float4*>(s_eref + wg * 64 + 32 + j4);
+            d[j4] *= e0.x; d[j4 + 1] *= e0.y; d[j4 + 2] *= e0.z; d[j4 + 3] *= e0.w;
+            d1[j4] *= e1.x; d1[j4 + 1] *= e1.y; d1[j4 + 2] *= e1.z; d1[j4 + 3] *= e1.w;
+        }
+        if (r < n) {
+            st32_bf16(pp.wn + tok * DK + wg * 64, d, -1.f);
+            st32_bf16(pp.wn + tok * DK + wg * 64 + 32, d1, -1.f);
+        }
+        if (TIED) {
+            const int half = dv >> 1;
+            tmem_ld32_async(tmem + lane_base + 128 + wg * half, d);
+            if (half == 64) tmem_ld32_async(tmem + lane_base + 128 + wg * half + 32, d1);
+            tmem_wait_ld();
+            if (r < n) {
+                st32_bf16(pp.p + tok * dv + wg * half, d, 1.f);
+                if (half == 64) st32_bf16(pp.p + tok * dv + wg * half + 32, d1, 1.f);
+            }
+        } else {
+            tmem_ld32(tmem + lane_base + 128 + wg * 32, d);
+#pragma unroll
+            for (int c8 = 0; c8 < 4; ++c8) {
+                float x[8];
+#pragma unroll
+                for (int e = 0; e < 8; ++e) x[e] = -d[c8 * 8 + e];
+                st_chunk(sm + G_OFF_APRE, sw128_chunk(r, wg * 4 + c8, 64), x);
+            }
+        }
+    }
+    if (!TIED) {
+        GDR_BEFORE_MMA();
+        // ---- P3: D3 = (-T Bm) V -> P ------------------------------------------------
+        if (tid == 0) {
+            tc_fence_after();
+            const uint32_t idP = idesc_bf16(128, dv, 0, 1);
+#pragma unroll
+            for (int ks = 0; ks < 4; ++ks)
+                mma_bf16(tmem, sdesc_sw128(sbase + G_OFF_APRE + ks * 32u, 16, 1024),
+                         sdesc_sw128(sbase + G_OFF_ROP + 8192 + ks * 2048u, 16384, 1024), idP, ks > 0);
+            mma_commit(bar_mma);
+        }
+        GDR_WAIT(bar_mma, ph_mma);
+        tc_fence_after();
+        if (row < 64) {
+            const int r = row;
+            const size_t tok = ((size_t)bb * T + t0 + r) * H + h;
+            const int half = dv >> 1;
+            float d[32], d1[32];
+            tmem_ld32_async(tmem + lane_base + wg * half, d);
+            if (half == 64) tmem_ld32_async(tmem + lane_base + wg * half + 32, d1);
+            tmem_wait_ld();
+            if (r < n) {
+                st32_bf16(pp.p + tok * dv + wg * half, d, 1.f);
+                if (half == 64) st32_bf16(pp.p + tok * dv + wg * half + 32, d1, 1.f);
+            }
+        }
+    }
+
+finish:
+    if (!ok && tid == 0) flag_status(pp.d_status, GDR_DEVICE_TIMEOUT);
+    tc_fence_before();
+    __syncthreads();
+    if (warp == 0) tmem_dealloc(tmem, G_TM_COLS);
+#undef GDR_WAIT
+#undef GDR_BEFORE_MMA
+}
+
+// ---- pass 2 ------------------------------------------------------------------
+template <bool UNTIED>
+struct StateLayout {
+    static constexpr uint32_t WQ = 0;                    // [WN ; QG] bf16 [128 x 128], 2 x 32 KB
+    static constexpr uint32_t K2 = 65536;                // K2 bf16 [64 x 128], 2 x 16 KB
+    static constexpr uint32_t AQU = 98304;               // [U ; AQ] bf16 [128 x 64], 2 x 16 KB
+    static constexpr uint32_t P = 131072;                // P slice bf16 [64 x 64], 2 x 8 KB
+    static constexpr uint32_t KW2 = 147456;              // KW2 bf16 [64 x 128], 2 x 16 KB (untied)
+    static constexpr uint32_t BQ = UNTIED ? 180224 : 0;  // BQ bf16 [64 x 64], 2 x 8 KB (untied)
+    static constexpr uint32_t V = UNTIED ? 196608 : 0;   // V slice bf16 [64 x 64], 2 x 8 KB (untied)
+    static constexpr uint32_t SBF = UNTIED ? 212992 : 147456;  // S bf16 [128 x 64]
+    static constexpr uint32_t SMALL = SBF + 16384;             // barriers, TMEM slot (1 KB)
+    static constexpr uint32_t BYTES = SMALL + 1024 + 1024;
+};
+// D3 (U, QG S) and D5 (AQ U, BQ V) alternate between two column sets by chunk parity.
+constexpr uint32_t GS_TM_D3 = 0, GS_TM_D5 = 128, GS_TM_D4 = 256, GS_TM_COLS = 512;
+
+struct GStateParams {
+    const float* S0;
+    const float* gc;
+    __nv_bfloat16* o;
+    float* ST;
+    int* d_status;
+    int T, H, dv;
+};
+
+template <bool UNTIED>
+__global__ void __launch_bounds__(NT, 1) state_general_kernel(
+    const __grid_constant__ CUtensorMap tm_wn, const __grid_constant__ CUtensorMap tm_qg,
+    const __grid_constant__ CUtensorMap tm_k2, const __grid_constant__ CUtensorMap tm_aq,
+    const __grid_constant__ CUtensorMap tm_p, const __grid_constant__ CUtensorMap tm_kw2,
+    const __grid_constant__ CUtensorMap tm_bq, const __grid_constant__ CUtensorMap tm_v,
+    const GStateParams p) {
+    using Lay = StateLayout<UNTIED>;
+    extern __shared__ uint8_t smem_raw[];
+    uint8_t* sm = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) &
+                                             ~uintptr_t(1023));
+    const int tid = threadIdx.x, warp = tid >> 5, wg = warp >> 2, row = tid & 127;
+    const int vt = blockIdx.x, h = blockIdx.y, bb = blockIdx.z;
+    const int v0 = vt * NV;
+    const int T = p.T, H = p.H;
+    const int nchunks = (T + C - 1) / C;
+
+    uint64_t* bar_tma = reinterpret_cast<uint64_t*>(sm + Lay::SMALL);  // [2]
+    uint64_t* bar_mma = bar_tma + 2;
+    uint32_t* s_tmem = reinterpret_cast<uint32_t*>(sm + Lay::SMALL + 32);
+    if (tid == 0) {
+        mbar_init(&bar_tma[0], 1);
+        mbar_init(&bar_tma[1], 1);
+        mbar_init(bar_mma, 1);
+        fence_barrier_init();
+    }
+    if (warp == 0) tmem_alloc(s_tmem, GS_TM_COLS);
+    tc_fence_before();
+    __syncthreads();
+    tc_fence_after();
+    const uint32_t tmem = *s_tmem;
+    const uint32_t lane_base = (uint32_t)((warp & 3) * 32) << 16;
+    uint32_t ph_tma0 = 0u, ph_tma1 = 0u, ph_mma = 0;
+    bool ok = true;
+    const uint32_t sbase = smem_u32(sm);
+
+    auto issue_loads = [&](int ci) {
+        const int t0 = ci * C, buf = ci & 1;
+        uint64_t* bar = &bar_tma[buf];
+        uint8_t* wq = sm + Lay::WQ + buf * 32768;
+        mbar_expect_tx(bar, (UNTIED ? 12u : 8u) * 8192u);
+        tma_load_4d(wq, &tm_wn, bar, 0, h, t0, bb);
+        tma_load_4d(wq + 16384, &tm_wn, bar, 64, h, t0, bb);
+        tma_load_4d(wq + 8192, &tm_qg, bar, 0, h, t0, bb);
+        tma_load_4d(wq + 16384 + 8192, &tm_qg, bar, 64, h, t0, bb);
+        tma_load_4d(sm + Lay::K2 + buf * 16384, &tm_k2, bar, 0, h, t0, bb);
+        tma_load_4d(sm + Lay::K2 + buf * 16384 + 8192, &tm_k2, bar, 64, h, t0, bb);
+        tma_load_4d(sm + Lay::AQU + buf * 16384 + 8192, &tm_aq, bar, 0, h, t0, bb);
+        tma_load_4d(sm + Lay::P + buf * 8192, &tm_p, bar, v0, h, t0, bb);
+        if (UNTIED) {
+            tma_load_4d(sm + Lay::KW2 + buf * 16384, &tm_kw2, bar, 0, h, t0, bb);
+            tma_load_4d(sm + Lay::KW2 + buf * 16384 + 8192, &tm_kw2, bar, 64, h, t0, bb);
+            tma_load_4d(sm + Lay::BQ + buf * 8192, &tm_bq, bar, 0, h, t0, bb);
+            tma_load_4d(sm + Lay::V + buf * 8192, &tm_v, bar, v0, h, t0, bb);
+        }
+    };
+
+    constexpr int NH = NV / 2;
+    float S[NH];
+    {
+        const float* s0 = p.S0 ? p.S0 + (((size_t)bb * H + h) * DK + row) * p.dv + v0 + wg * NH : nullptr;
+#pragma unroll
+        for (int j = 0; j < NH; j += 4) {
+            float4 x = s0 ? *reinterpret_cast<const float4*>(s0 + j) : make_float4(0.f, 0.f, 0.f, 0.f);
+            S[j] = x.x; S[j + 1] = x.y; S[j + 2] = x.z; S[j + 3] = x.w;
+        }
+#pragma unroll
+        for (int ch = 0; ch < 4; ++ch) st_chunk(sm + Lay::SBF, sw128_chunk(row, wg * 4 + ch, DK), &S[8 * ch]);
+    }
+    const float* gcp = p.gc + ((size_t)bb * H + h) * nchunks * DK + row;
+    float gC_next = nchunks > 0 ? gcp[0] : 0.f;
+    if (tid == 0 && nchunks > 0) issue_loads(0);
+
+    auto store_o = [&](int cj) {
+        const int pj = cj & 1;
+        const int t = cj * C + row - 64;
+        float d[32], d5[32];
+        tmem_ld32_async(tmem + lane_base + GS_TM_D3 + pj * 64 + wg * 32, d);
+        tmem_ld32_async(tmem + lane_base + GS_TM_D5 + pj * 64 + wg * 32, d5);
+        tmem_wait_ld();
+        if (t < T) {
+#pragma unroll
+            for (int j = 0; j < 32; ++j) d[j] += d5[j];
+            st32_bf16(p.o + (((size_t)bb * T + t) * H + h) * p.dv + v0 + wg * 32, d, 1.f);
+        }
+    };
+
+#define GDR_WAIT(bar, ph)                                                   \
+    do {                                                                    \
+        bool w_ok = mbar_wait(bar, ph);                                     \
+        ph ^= 1u;                                                           \
+        if (!__syncthreads_and(w_ok)) { ok = false; goto finish; }          \
+    } while (0)
+#define GDR_BEFORE_MMA()    \
+    do {                    \
+        fence_proxy_async(); \
+        tc_fence_before();  \
+        __syncthreads();    \
+    } while (0)
+
+    for (int ci = 0; ci < nchunks; ++ci) {
+        const int buf = ci & 1, par = ci & 1;
+        const uint32_t wqb = sbase + Lay::WQ + buf * 32768u;
+        const uint32_t k2b = sbase + Lay::K2 + buf * 16384u;
+        const uint32_t aqub = sbase + Lay::AQU + buf * 16384u;
+        const uint32_t d3 = GS_TM_D3 + (uint32_t)par * 64u, d5 = GS_TM_D5 + (uint32_t)par * 64u;
+        const float gC = gC_next;
+        if (ci + 1 < nchunks) gC_next = gcp[(size_t)(ci + 1) * DK];
+        if (buf == 0) GDR_WAIT(&bar_tma[0], ph_tma0);
+        else GDR_WAIT(&bar_tma[1], ph_tma1);
+
+        // ---- batch 1: D3 = [WN ; QG] S;  untied: D4 = KW2^T V, D5 = [. ; BQ] V --------
+        if (tid == 0) {
+            tc_fence_after();
+            const uint32_t idS = idesc_bf16(128, NV, 0, 1);
+            const uint32_t idM = idesc_bf16(128, NV, 1, 1);
+#pragma unroll
+            for (int ks = 0; ks < 8; ++ks) {
+                const uint32_t koff = (ks >> 2) * 16384u + (ks & 3) * 32u;
+                mma_bf16(tmem + d3, sdesc_sw128(wqb + koff, 16, 1024),
+                         sdesc_sw128(sbase + Lay::SBF + ks * 2048u, 8192, 1024), idS, ks > 0);
+            }
+            if (UNTIED) {
+                const uint32_t vb = sbase + Lay::V + buf * 8192u;
+                const uint32_t bqa = sbase + Lay::BQ + buf * 8192u - 8192u;  // BQ = rows 64..127
+#pragma unroll
+                for (int ks = 0; ks < 4; ++ks) {
+                    mma_bf16(tmem + GS_TM_D4, sdesc_sw128(sbase + Lay::KW2 + buf * 16384u + ks * 2048u, 8192, 1024),
+                             sdesc_sw128(vb + ks * 2048u, 8192, 1024), idM, ks > 0);
+                    mma_bf16(tmem + d5, sdesc_sw128(bqa + ks * 32u, 16, 1024),
+                             sdesc_sw128(vb + ks * 2048u, 8192, 1024), idS, ks > 0);
+                }
+            }
+            mma_commit(bar_mma);
+        }
+        // chunk ci + 1's inputs go to the buffers chunk ci - 1 has released
+        if (tid == 32 && ci + 1 < nchunks) issue_loads(ci + 1);
+        // the previous chunk's outputs, while batch 1 runs
+        if (row >= 64 && ci > 0) store_o(ci - 1);
+        GDR_WAIT(bar_mma, ph_mma);
+        tc_fence_after();
+
+        // ---- U = P + WN S (rows 0..63) -> rows 0..63 of [U ; AQ] ------------------------
+        if (row < 64) {
+            float d[32];
+            tmem_ld32(tmem + lane_base + d3 + wg * 32, d);
+#pragma unroll
+            for (int c8 = 0; c8 < 4; ++c8) {
+                float x[8];
+                ld_chunk(sm + Lay::P + buf * 8192, sw128_chunk(row, wg * 4 + c8, 64), x);
+#pragma unroll
+                for (int e = 0; e < 8; ++e) x[e] += d[c8 * 8 + e];
+                st_chunk(sm + Lay::AQU + buf * 16384, sw128_chunk(row, wg * 4 + c8, 128), x);
+            }
+        }
+        GDR_BEFORE_MMA();
+
+        // ---- batch 2: D5 (+)= [U ; AQ] U (rows 64..127: AQ U);  D4 (+)= K2^T U ----------
+        if (tid == 0) {
+            tc_fence_after();
+            const uint32_t idK = idesc_bf16(128, NV, 0, 1);
+            const uint32_t idM = idesc_bf16(128, NV, 1, 1);
+#pragma unroll
+            for (int ks = 0; ks < 4; ++ks) {
+                const uint32_t acc = UNTIED ? 1u : (uint32_t)(ks > 0);
+                mma_bf16(tmem + d5, sdesc_sw128(aqub + ks * 32u, 16, 1024),
+                         sdesc_sw128(aqub + ks * 2048u, 8192, 1024), idK, acc);
+                mma_bf16(tmem + GS_TM_D4, sdesc_sw128(k2b + ks * 2048u, 8192, 1024),
+                         sdesc_sw128(aqub + ks * 2048u, 8192, 1024), idM, acc);
+            }
+            mma_commit(bar_mma);
+        }
+        GDR_WAIT(bar_mma, ph_mma);
+        tc_fence_after();
+
+        // ---- S = Diag(GC) S + D4 ---------------------------------------------------------
+        {
+            float dS[32];
+            tmem_ld32(tmem + lane_base + GS_TM_D4 + wg * 32, dS);
+#pragma unroll
+            for (int j = 0; j < NH; ++j) S[j] = fmaf(gC, S[j], dS[j]);
+#pragma unroll
+            for (int ch = 0; ch < 4; ++ch) st_chunk(sm + Lay::SBF, sw128_chunk(row, wg * 4 + ch, DK), &S[8 * ch]);
+        }
+        tc_fence_before();
+        __syncthreads();
+    }
+    if (row >= 64 && nchunks > 0) store_o(nchunks - 1);
+
+    if (p.ST) {
+        float* st = p.ST + (((size_t)bb * H + h) * DK + row) * p.dv + v0 + wg * NH;
+#pragma unroll
+        for (int j = 0; j < NH; j += 4) *reinterpret_cast<float4*>(st + j) = make_float4(S[j], S[j + 1], S[j + 2], S[j + 3]);
+    }
+
+finish:
+    if (!ok && tid == 0) flag_status(p.d_status, GDR_DEVICE_TIMEOUT);
+    tc_fence_before();
+    __syncthreads();
+    if (warp == 0) tmem_dealloc(tmem, GS_TM_COLS);
+#undef GDR_WAIT
+#undef GDR_BEFORE_MMA
+}
+
+}  // namespace twopass_g
+
+// Workspace of the general two-pass path: sub-buffers in this order, each
+// rounded up to 256 bytes: WN, QG, K2, AQ, P, [KW2, BQ], GC.
+struct GeneralWorkspace {
+    size_t off[8];
+    size_t total;
+};
+
+static GeneralWorkspace general_workspace_layout(int B, int T, int H, int dv, bool untied) {
+    auto up = [](size_t x) { return (x + 255) & ~(size_t)255; };
+    const size_t tok = (size_t)B * T * H;
+    const size_t nchunks = ((size_t)T + 63) / 64;
+    const size_t sizes[8] = {tok * 128 * 2, tok * 128 * 2, tok * 128 * 2, tok * 64 * 2,
+                             tok * (size_t)dv * 2, untied ? tok * 128 * 2 : 0, untied ? tok * 64 * 2 : 0,
+                             (size_t)B * H * nchunks * 128 * 4};
+    GeneralWorkspace w;
+    size_t o = 0;
+    for (int i = 0; i < 8; ++i) {
+        w.off[i] = o;
+        o += up(sizes[i]);
+    }
+    w.total = o;
+    return w;
+}
+
+size_t twopass_general_workspace_bytes(int B, int T, int H, int dv, bool untied) {
+    return general_workspace_layout(B, T, H, dv, untied).total;
+}
+
+using MapFn = bool (*)(CUtensorMap*, const void*, int, int, int, int);
+
+// maps: q, k, v (of the call). alpha/b/w kinds as in the C ABI.
+cudaError_t launch_chunk_twopass_general(const CUtensorMap* maps, MapFn make_map, void* ws,
+                                         const void* q, const void* k, const void* alpha,
+                                         const void* b, const void* w, int akind, int bkind,
+                                         int wkind, const float* S0, void* o, float* ST,
+                                         int* d_status, int B, int T, int H, int dv,
+                                         cudaStream_t st) {
+    using namespace twopass_g;
+    const bool tied = wkind == GDR_GATE_TIED && bkind == GDR_GATE_SCALAR;
+    const bool ach = akind == GDR_GATE_CHANNEL;
+    const GeneralWorkspace lay = general_workspace_layout(B, T, H, dv, !tied);
+    uint8_t* base = reinterpret_cast<uint8_t*>(ws);
+    auto at = [&](int i) { return reinterpret_cast<__nv_bfloat16*>(base + lay.off[i]); };
+
+    GPrepParams pp;
+    pp.q = reinterpret_cast<const __nv_bfloat16*>(q);
+    pp.k = reinterpret_cast<const __nv_bfloat16*>(k);
+    pp.alpha = reinterpret_cast<const __nv_bfloat16*>(alpha);
+    pp.bg = reinterpret_cast<const __nv_bfloat16*>(b);
+    pp.wg = reinterpret_cast<const __nv_bfloat16*>(w);
+    pp.wn = at(0); pp.qg = at(1); pp.k2 = at(2); pp.aq = at(3); pp.p = at(4);
+    pp.kw2 = at(5); pp.bq = at(6);
+    pp.gc = reinterpret_cast<float*>(base + lay.off[7]);
+    pp.d_status = d_status;
+    pp.T = T; pp.H = H; pp.dv = dv;
+    pp.akind = akind; pp.bkind = bkind; pp.wkind = wkind;
+    const int nchunks = (T + C - 1) / C;
+    const dim3 pgrid(nchunks, H, B);
+    auto prep = [&](auto kern) -> cudaError_t {
+        cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, G_SMEM_BYTES);
+        if (e != cudaSuccess) return e;
+        kern<<<pgrid, NT, G_SMEM_BYTES, st>>>(maps[2], pp);
+        return cudaGetLastError();
+    };
+    cudaError_t e = tied ? (ach ? prep(prep_general_kernel<true, true>) : prep(prep_general_kernel<true, false>))
+                         : (ach ? prep(prep_general_kernel<false, true>) : prep(prep_general_kernel<false, false>));
+    if (e != cudaSuccess) return e;
+
+    CUtensorMap sm_maps[8];
+    const int dims[7] = {128, 128, 128, 64, dv, 128, 64};
+    for (int i = 0; i < 7; ++i) {
+        const void* ptr = (i >= 5 && tied) ? base + lay.off[0] : base + lay.off[i];
+        const int d = (i >= 5 && tied) ? 128 : dims[i];
+        if (!make_map(&sm_maps[i], ptr, B, T, H, d)) return cudaErrorInvalidValue;
+    }
+    sm_maps[7] = maps[2];
+    GStateParams sp;
+    sp.S0 = S0; sp.gc = pp.gc; sp.o = reinterpret_cast<__nv_bfloat16*>(o); sp.ST = ST;
+    sp.d_status = d_status; sp.T = T; sp.H = H; sp.dv = dv;
+    const dim3 sgrid(dv / NV, H, B);
+    auto state = [&](auto kern, uint32_t bytes) -> cudaError_t {
+        cudaError_t e2 = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, bytes);
+        if (e2 != cudaSuccess) return e2;
+        kern<<<sgrid, NT, bytes, st>>>(sm_maps[0], sm_maps[1], sm_maps[2], sm_maps[3], sm_maps[4],
+                                       sm_maps[5], sm_maps[6], sm_maps[7], sp);
+        return cudaGetLastError();
+    };
+    return tied ? state(state_general_kernel<false>, StateLayout<false>::BYTES)
+                : state(state_general_kernel<true>, StateLayout<true>::BYTES);
+}
+
+}  // namespace gdr

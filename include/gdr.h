@@ -131,9 +131,15 @@ gdr_status gdr_chunk_fwd(const void* q, const void* k, const void* v,
 /*
  * gdr_chunk_fwd_workspace_size -- bytes of scratch gdr_chunk_fwd's two-pass
  * path needs for this shape and gate form, or 0 when it has none. Two-pass
- * forms: dtype GDR_BF16, d_k = 128, d_v in {64, 128}, scalar alpha, tied
- * scalar beta (Gated DeltaNet). Size: B*T*H*(d_k + d_v) bf16 values (the
- * per-token rows of -W = -T Diag(beta g) K and of T Diag(beta) V).
+ * shapes: dtype GDR_BF16, d_k = 128, d_v in {64, 128}, T >= 1, an erase gate
+ * (b_kind != GDR_GATE_NONE). Sizes, in bytes, with N = B*T*H:
+ *   scalar alpha, tied scalar beta (Gated DeltaNet): 2 N (d_k + d_v)
+ *     (per-token rows of -W = -T Diag(beta g) K and of T Diag(beta) V);
+ *   every other form: the per-token rows of -W 2^ref, q.g, k.g_{n-1}/g,
+ *     the masked (q.rowf)(k.colf)^T block row and P (plus, with independent
+ *     b and w, w.k.g_{n-1}/g and the masked (q.rowf)(w.k.colf)^T row), in
+ *     bf16, and g_{n-1} per chunk and channel in fp32, each sub-buffer
+ *     rounded up to 256 bytes.
  * Host-only; launches nothing.
  */
 size_t gdr_chunk_fwd_workspace_size(int B, int T, int H, int d_k, int d_v,

@@ -184,13 +184,16 @@ def test_gla_full_size_sampled_heads(cuda_device):
 
 
 # ---- two-pass path (per-chunk factors in parallel, then the state pass) -----
-# The Gated DeltaNet form (scalar alpha, tied beta, d_v <= 128) takes it by
-# default; these also run the same inputs through the single-pass kernel.
+# Every erase-gated bf16 form with d_k = 128, d_v <= 128 takes it by default;
+# these also run the same inputs through the single-pass kernels.
 
+@pytest.mark.parametrize("family", FAMILIES)
 @pytest.mark.parametrize("T", [1, 63, 64, 65, 200, 1000])
 @pytest.mark.parametrize("dv", [64, 128])
-def test_two_pass_matches_oracle_and_single_pass(cuda_device, T, dv):
-    wl = small("gdn", T=T, dv=dv, s0=True, seed=300 + T + dv)
+def test_two_pass_matches_oracle_and_single_pass(cuda_device, family, T, dv):
+    """Gated DeltaNet form: its own pair of kernels; KDA and GDN-2 forms: the
+    general pair (channel decay, independent b and w)."""
+    wl = small(family, T=T, dv=dv, s0=True, seed=300 + T + dv)
     inp = make_chunk_inputs(wl)
     o2, S2 = run_chunk(inp, cuda_device)                      # two-pass
     o1, S1 = run_chunk(inp, cuda_device, workspace=None)      # single pass
@@ -224,10 +227,11 @@ def test_two_pass_workspace_is_used(cuda_device):
     assert wneg.abs().sum() > 0 and p.abs().sum() > 0
 
 
-def test_two_pass_full_size_matches_single_pass(cuda_device):
-    """Full Gated DeltaNet workload: the two paths agree everywhere (both
-    were checked against the oracle on sampled heads above)."""
-    wl = WORKLOADS["gdn"]
+@pytest.mark.parametrize("family", FAMILIES)
+def test_two_pass_full_size_matches_single_pass(cuda_device, family):
+    """Full workloads: the two paths agree everywhere (both were checked
+    against the oracle on sampled heads above)."""
+    wl = WORKLOADS[family]
     inp = make_chunk_inputs(wl)
     o2, S2 = run_chunk(inp, cuda_device)
     o1, S1 = run_chunk(inp, cuda_device, workspace=None)
