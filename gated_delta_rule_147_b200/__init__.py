@@ -15,7 +15,7 @@ from __future__ import annotations
 
 from ._lib import (GATE_CHANNEL, GATE_NONE, GATE_SCALAR, GATE_TIED, GDR_BF16, GDR_FP32,
                    GDR_DEVICE_DECAY_RANGE, GDR_DEVICE_TIMEOUT, GdrError, gdr_chunk_fwd,
-                   gdr_chunk_fwd_workspace_size, gdr_decode_step, load)
+                   gdr_chunk_fwd_static, gdr_chunk_fwd_workspace_size, gdr_decode_step, load)
 
 TIED = "tied"
 _KIND = {"none": GATE_NONE, "scalar": GATE_SCALAR, "channel": GATE_CHANNEL, "tied": GATE_TIED}
@@ -59,7 +59,8 @@ def chunk_fwd(q, k, v, alpha=None, b=None, w=None, S0=None, *, out=None, final_s
     """Forward over [B,T,H,*] inputs. alpha/b/w: None, a [B,T,H] tensor
     (scalar gate), a [B,T,H,d_k] tensor (channel gate); w may be TIED (w := b).
     workspace: "auto" allocates the two-pass path's scratch with torch when
-    the inputs have such a path; a uint8 device tensor supplies it; None runs
+    the inputs have such a path; a uint8 device tensor supplies it; "static"
+    uses the library's own scratch array (gdr_chunk_fwd_static); None runs
     the single-pass kernels. Returns (o, S_T) with S_T None when final_state
     is False."""
     import torch
@@ -69,6 +70,12 @@ def chunk_fwd(q, k, v, alpha=None, b=None, w=None, S0=None, *, out=None, final_s
     o = out if out is not None else torch.empty((B, T, H, dv), dtype=v.dtype, device=v.device)
     if final_state and S_T is None:
         S_T = torch.empty((B, H, dk, dv), dtype=torch.float32, device=v.device)
+    if isinstance(workspace, str) and workspace == "static":
+        gdr_chunk_fwd_static(q, k, v, alpha, b, None if isinstance(w, str) else w,
+                             _gate_kind(alpha, 3), _gate_kind(b, 3), _gate_kind(w, 3), S0, o,
+                             S_T if final_state else None, B, T, H, dk, dv, chunk, _dtype_code(q),
+                             d_status, stream)
+        return o, (S_T if final_state else None)
     if isinstance(workspace, str):
         if workspace != "auto":
             raise ValueError(workspace)

@@ -17,7 +17,8 @@ GDR_DEVICE_TIMEOUT, GDR_DEVICE_DECAY_RANGE = 1, 2
 GDR_BF16, GDR_FP32 = 0, 1
 GATE_NONE, GATE_SCALAR, GATE_CHANNEL, GATE_TIED = 0, 1, 2, 3
 
-EXPORTS = ("gdr_chunk_fwd", "gdr_chunk_fwd_workspace_size", "gdr_decode_step", "gdr_selftest_bounded_wait", "gdr_status_string",
+EXPORTS = ("gdr_chunk_fwd", "gdr_chunk_fwd_workspace_size", "gdr_chunk_fwd_static",
+           "gdr_chunk_fwd_static_capacity", "gdr_decode_step", "gdr_selftest_bounded_wait", "gdr_status_string",
            "gdr_version")
 
 _lock = threading.Lock()
@@ -51,6 +52,10 @@ def load(build_if_missing: bool = True) -> ctypes.CDLL:
         lib.gdr_chunk_fwd.restype = ip
         lib.gdr_chunk_fwd_workspace_size.argtypes = [ip] * 9
         lib.gdr_chunk_fwd_workspace_size.restype = sz
+        lib.gdr_chunk_fwd_static.argtypes = [vp] * 6 + [ip] * 3 + [vp, vp, vp] + [ip] * 7 + [vp, vp]
+        lib.gdr_chunk_fwd_static.restype = ip
+        lib.gdr_chunk_fwd_static_capacity.argtypes = []
+        lib.gdr_chunk_fwd_static_capacity.restype = sz
         lib.gdr_decode_step.argtypes = [vp] * 6 + [ip] * 3 + [vp, vp] + [ip] * 5 + [vp, vp]
         lib.gdr_decode_step.restype = ip
         lib.gdr_status_string.argtypes = [ip]
@@ -91,6 +96,20 @@ def gdr_chunk_fwd(q, k, v, alpha, b, w, alpha_kind, b_kind, w_kind, S0, o, S_T, 
                               B, T, H, d_k, d_v, chunk, dtype, _p(d_status), _stream(stream))
     if st != GDR_OK:
         raise GdrError("gdr_chunk_fwd", st)
+
+
+def gdr_chunk_fwd_static(q, k, v, alpha, b, w, alpha_kind, b_kind, w_kind, S0, o, S_T, B, T, H,
+                         d_k, d_v, chunk, dtype, d_status=None, stream=None) -> None:
+    """gdr_chunk_fwd with the library's own scratch array (no workspace argument)."""
+    st = load().gdr_chunk_fwd_static(_p(q), _p(k), _p(v), _p(alpha), _p(b), _p(w), alpha_kind,
+                                     b_kind, w_kind, _p(S0), _p(o), _p(S_T), B, T, H, d_k, d_v,
+                                     chunk, dtype, _p(d_status), _stream(stream))
+    if st != GDR_OK:
+        raise GdrError("gdr_chunk_fwd_static", st)
+
+
+def gdr_chunk_fwd_static_capacity() -> int:
+    return int(load().gdr_chunk_fwd_static_capacity())
 
 
 def gdr_chunk_fwd_workspace_size(B, T, H, d_k, d_v, alpha_kind, b_kind, w_kind, dtype) -> int:

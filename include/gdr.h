@@ -147,6 +147,35 @@ size_t gdr_chunk_fwd_workspace_size(int B, int T, int H, int d_k, int d_v,
                                     int dtype);
 
 /*
+ * gdr_chunk_fwd_static -- gdr_chunk_fwd without a caller workspace: the
+ * two-pass path's scratch is a fixed device array inside the library
+ * (gdr_chunk_fwd_static_capacity() bytes, one per device). The pages define
+ * no such call; it exists so a caller can run the two-pass path while
+ * allocating nothing.
+ *
+ * Arguments, layouts and results are those of gdr_chunk_fwd (which it calls
+ * with that array as the workspace). Forms without a two-pass path use no
+ * scratch. Returns GDR_ERR_UNSUPPORTED when the workspace the call needs
+ * (gdr_chunk_fwd_workspace_size) exceeds the capacity, before touching the
+ * device; otherwise as gdr_chunk_fwd.
+ * Ownership and concurrency: the array is shared by every call on a device,
+ * so calls whose executions overlap (different streams, threads or graphs
+ * running concurrently) race on it and corrupt each other's results;
+ * serialise them. The first call on each device looks the array up
+ * (cudaGetSymbolAddress, which may load the module): make it before any
+ * stream capture that records later calls.
+ */
+gdr_status gdr_chunk_fwd_static(const void* q, const void* k, const void* v,
+                                const void* alpha, const void* b, const void* w,
+                                int alpha_kind, int b_kind, int w_kind,
+                                const float* S0, void* o, float* S_T,
+                                int B, int T, int H, int d_k, int d_v, int chunk,
+                                int dtype, int* d_status, void* stream);
+
+/* Bytes of the device array gdr_chunk_fwd_static uses (64 MiB). Host-only. */
+size_t gdr_chunk_fwd_static_capacity(void);
+
+/*
  * gdr_decode_step -- one token per head (autoregressive decoding).
  *
  * Applies one step of the recurrence to every (b, h) head: S is read and
