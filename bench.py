@@ -180,8 +180,8 @@ class ClockSampler:
 
 
 def dist_env():
-    ws = int(os.environ.get("WORLD_SIZE", "1"))
-    return ws, int(os.environ.get("RANK", "0")), int(os.environ.get("LOCAL_RANK", "0"))
+    from gated_delta_rule_147_b200.dist_util import dist_env as env
+    return env()
 
 
 # ------------------------------------------------------------------ ours ---
@@ -341,15 +341,15 @@ def run_ours(args):
         barrier = lambda: dist.barrier(device_ids=[local])
     else:
         barrier = lambda: None
+    from gated_delta_rule_147_b200.dist_util import max_over_ranks, shard_seed
     pk = peaks()
     wl = WORKLOADS["gdn"]
+    # each rank processes its own shard of the global batch (disjoint sequences)
+    wl_rank = wl.with_(seed=shard_seed(wl.seed, rank))
     with ClockSampler(local) as clk:
-        inp, d, total_ms, per = time_chunk(wl, dev, args.steps, args.warmup, barrier)
+        inp, d, total_ms, per = time_chunk(wl_rank, dev, args.steps, args.warmup, barrier)
     clocks = clk.summary()
-    t = torch.tensor([total_ms], device=dev)
-    if ws > 1:
-        dist.all_reduce(t, op=dist.ReduceOp.MAX)
-    total_ms = float(t.item())
+    total_ms = max_over_ranks(total_ms, device=dev)
     tokens = wl.B * wl.T
     value = ws * tokens * args.steps / (total_ms * 1e-3)
     bytes_ = workload_bytes(wl)
