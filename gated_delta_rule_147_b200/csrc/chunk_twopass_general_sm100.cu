@@ -21,12 +21,30 @@
 //   S' = Diag(GC) S + K2^T U (+ KW2^T V)
 // With tied beta, Bm = A Diag(beta) and Bq = Aq Diag(beta), so U + Diag(beta) V
 // = T Diag(beta) V - W S replaces U and the V terms drop out.
+#include <mutex>
+
 #include "chunk_common.cuh"
 
 namespace gdr {
 namespace twopass_g {
 
 using namespace chunkc;
+
+// Optional phase tracing (build with -DGDR_TRACE_PHASES): clock64() stamps of
+// thread 0 of the pass-1 CTAs of head (0, 0), chunks 0..63 (16 slots each);
+// gdr_trace_general_read() copies them out.
+#ifdef GDR_TRACE_PHASES
+__device__ unsigned long long g_trace3[64 * 16];
+#define GDR_TRACE_G(k)                                                                     \
+    do {                                                                                  \
+        if (blockIdx.y == 0 && blockIdx.z == 0 && threadIdx.x == 0 && blockIdx.x < 64)    \
+            g_trace3[blockIdx.x * 16 + (k)] = clock64();                                  \
+    } while (0)
+#else
+#define GDR_TRACE_G(k) \
+    do {              \
+    } while (0)
+#endif
 
 // ---- pass 1 shared memory (bytes from a 1024-aligned base) ----------------
 // M = 128 MMAs read A rows 64..127 beyond each 64-row operand; those rows
@@ -45,6 +63,7 @@ constexpr uint32_t G_SMEM_BYTES = G_OFF_SMALL + 3072 + 1024;
 constexpr uint32_t G_TM_COLS = 256;
 
 struct GPrepParams {
+    int c_begin;  // chunk index of blockIdx.x = 0
     const __nv_bfloat16* q;
     const __nv_bfloat16* k;
     const __nv_bfloat16* alpha;
@@ -84,13 +103,15 @@ __device__ __forceinline__ void st32_bf16(__nv_bfloat16* p, const float* x, floa
 }
 
 template <bool TIED, bool ACH>
-__global__ void __launch_bounds__(NT, 2) prep_general_kernel(const __grid_constant__ CUtensorMap tm_v,
-                                                             const GPrepParams pp) {
+__global__ void __launch_bounds__(NT, 2) prep_general_kernel(
+    const __grid_constant__ CUtensorMap tm_v, const __grid_constant__ CUtensorMap tm_wn,
+    const __grid_constant__ CUtensorMap tm_aq, const __grid_constant__ CUtensorMap tm_p,
+    const __grid_constant__ CUtensorMap tm_bq, const GPrepParams pp) {
     extern __shared__ uint8_t smem_raw[];
     uint8_t* sm = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) &
                                              ~uintptr_t(1023));
     const int tid = threadIdx.x, warp = tid >> 5, wg = warp >> 2, row = tid & 127;
-    const int ci = blockIdx.x, h = blockIdx.y, bb = blockIdx.z;
+    const int ci = pp.c_begin + (int)blockIdx.x, h = blockIdx.y, bb = blockIdx.z;
     const int T = pp.T, H = pp.H, dv = pp.dv;
     const int nchunks = (T + C - 1) / C;
     const int t0 = ci * C;
@@ -98,6 +119,39 @@ __global__ void __launch_bounds__(NT, 2) prep_general_kernel(const __grid_consta
     const int nvt = dv / 64;
     const bool bch = pp.bkind == GDR_GATE_CHANNEL, wch = pp.wkind == GDR_GATE_CHANNEL;
     constexpr int N1 = TIED ? 64 : 128;  // rows of [Ks ; Kws]
+    const int cg = tid & 31, rg = warp;  // build: thread = 8 tokens (rg) x 4 channels (cg)
+    const int ch0 = cg * 4;
+
+    // ---- global loads first: scalar gates (raw bf16 bits), channel decay of the
+    //      thread's 8 tokens, and q, k, b, w of its first 4 tokens ----------------
+    unsigned short g_a = 0, g_b = 0, g_w = 0;
+    if (tid < C) {
+        const size_t gi = ((size_t)bb * T + t0 + min(tid, n - 1)) * H + h;
+        if (pp.akind == GDR_GATE_SCALAR) g_a = reinterpret_cast<const unsigned short*>(pp.alpha)[gi];
+        if (pp.bkind == GDR_GATE_SCALAR) g_b = reinterpret_cast<const unsigned short*>(pp.bg)[gi];
+        if (pp.wkind == GDR_GATE_SCALAR) g_w = reinterpret_cast<const unsigned short*>(pp.wg)[gi];
+    }
+    auto elem = [&](int r) {  // element index of (token row r, channel ch0)
+        return (((size_t)bb * T + t0 + min(r, n - 1)) * H + h) * DK + ch0;
+    };
+    uint2 aa[8];
+    if (ACH) {
+#pragma unroll
+        for (int i = 0; i < 8; ++i) ld8b(pp.alpha + elem(rg * 8 + i), aa[i]);
+    }
+    // q, k, b, w of token rg * 8 + i live in slot i % 4: tokens 0..3 now, token
+    // i + 4 is loaded into the slot as soon as token i has been unpacked
+    uint2 qa[4], ka[4], ba[4], wa[4];
+    auto load_token = [&](int i) {
+        const size_t e = elem(rg * 8 + i);
+        const int sl = i & 3;
+        ld8b(pp.q + e, qa[sl]);
+        ld8b(pp.k + e, ka[sl]);
+        if (bch) ld8b(pp.bg + e, ba[sl]);
+        if (!TIED && wch) ld8b(pp.wg + e, wa[sl]);
+    };
+#pragma unroll
+    for (int i = 0; i < 4; ++i) load_token(i);
 
     float* s_ascal = reinterpret_cast<float*>(sm + G_OFF_SMALL);
     float* s_bscal = s_ascal + 64;
@@ -111,7 +165,9 @@ __global__ void __launch_bounds__(NT, 2) prep_general_kernel(const __grid_consta
     uint64_t* bar_mma = bar_v + 1;
     uint32_t* s_tmem = reinterpret_cast<uint32_t*>(sm + G_OFF_SMALL + 2832);
     const uint32_t sbase = smem_u32(sm);
+    auto bits_to_f32 = [](unsigned short u) { return __uint_as_float((uint32_t)u << 16); };
 
+    GDR_TRACE_G(0);
     if (tid == 0) {
         mbar_init(bar_v, 1);
         mbar_init(bar_mma, 1);
@@ -121,10 +177,9 @@ __global__ void __launch_bounds__(NT, 2) prep_general_kernel(const __grid_consta
     if (warp == 0) tmem_alloc(s_tmem, G_TM_COLS);
     if (tid < C) {
         const bool valid = tid < n;
-        const size_t gi = ((size_t)bb * T + (valid ? t0 + tid : t0)) * H + h;
-        s_ascal[tid] = (pp.akind == GDR_GATE_SCALAR && valid) ? to_f32(pp.alpha[gi]) : 1.f;
-        s_bscal[tid] = (pp.bkind == GDR_GATE_SCALAR && valid) ? to_f32(pp.bg[gi]) : 0.f;
-        s_wscal[tid] = (pp.wkind == GDR_GATE_SCALAR && valid) ? to_f32(pp.wg[gi])
+        s_ascal[tid] = (pp.akind == GDR_GATE_SCALAR && valid) ? bits_to_f32(g_a) : 1.f;
+        s_bscal[tid] = (pp.bkind == GDR_GATE_SCALAR && valid) ? bits_to_f32(g_b) : 0.f;
+        s_wscal[tid] = (pp.wkind == GDR_GATE_SCALAR && valid) ? bits_to_f32(g_w)
                        : (pp.wkind == GDR_GATE_NONE ? 1.f : 0.f);
     }
     tc_fence_before();
@@ -134,6 +189,7 @@ __global__ void __launch_bounds__(NT, 2) prep_general_kernel(const __grid_consta
     const uint32_t lane_base = (uint32_t)((warp & 3) * 32) << 16;
     uint32_t ph_v = 0, ph_mma = 0;
     bool ok = true;
+    GDR_TRACE_G(1);
 
 #define GDR_WAIT(bar, ph)                                                   \
     do {                                                                    \
@@ -148,26 +204,10 @@ __global__ void __launch_bounds__(NT, 2) prep_general_kernel(const __grid_consta
         __syncthreads();    \
     } while (0)
 
-    // ---- build: thread = 8 tokens (rg = warp) x 4 channels (cg = lane) --------
+    // ---- build ------------------------------------------------------------------
     {
-        const int cg = tid & 31, rg = warp;
-        const int ch0 = cg * 4;
-        // issue every global load of this thread first
-        uint2 qa[8], ka[8], aa[8], ba[8], wa[8];
-#pragma unroll
-        for (int i = 0; i < 8; ++i) {
-            const int r = rg * 8 + i;
-            const int t = t0 + min(r, n - 1);
-            const size_t e = (((size_t)bb * T + t) * H + h) * DK + ch0;
-            ld8b(pp.q + e, qa[i]);
-            ld8b(pp.k + e, ka[i]);
-            if (ACH) ld8b(pp.alpha + e, aa[i]);
-            if (bch) ld8b(pp.bg + e, ba[i]);
-            if (!TIED && wch) ld8b(pp.wg + e, wa[i]);
-        }
         float* scan = reinterpret_cast<float*>(sm + G_OFF_SCR);  // [8 rg][128 ch] + [128]
         float lrow0[4];   // channel decay: l at this thread's first token - ref
-        float aval[8][4];
         if (!ACH) {
             if (warp == 0) {
                 const int lane = tid;
@@ -206,11 +246,11 @@ __global__ void __launch_bounds__(NT, 2) prep_general_kernel(const __grid_consta
 #pragma unroll
             for (int i = 0; i < 8; ++i) {
                 const int r = rg * 8 + i;
-                unpack4(aa[i], aval[i]);
+                float av[4];
+                unpack4(aa[i], av);
 #pragma unroll
                 for (int e = 0; e < 4; ++e) {
-                    if (r >= n) aval[i][e] = 1.f;  // padding tokens do not decay
-                    loc[e] += lg2_approx(aval[i][e]);
+                    loc[e] += r < n ? lg2_approx(av[e]) : 0.f;  // padding tokens do not decay
                     if (i == 0) lrow0[e] = loc[e];
                 }
             }
@@ -246,6 +286,7 @@ __global__ void __launch_bounds__(NT, 2) prep_general_kernel(const __grid_consta
             if (bad) flag_status(pp.d_status, GDR_DEVICE_DECAY_RANGE);
             __syncthreads();  // every channel's eref / fS is needed below
         }
+        GDR_TRACE_G(2);
         float er[4], fs[4];
         {
             const float4 e4 = *reinterpret_cast<const float4*>(s_eref + ch0);
@@ -260,61 +301,69 @@ __global__ void __launch_bounds__(NT, 2) prep_general_kernel(const __grid_consta
         float rowf_c[4];
 #pragma unroll
         for (int i = 0; i < 8; ++i) {
-            const int r = rg * 8 + i;
-            const bool valid = r < n;
-            float k4[4], q4[4], b4[4], w4[4];
-            unpack4(ka[i], k4);
-            unpack4(qa[i], q4);
-            if (bch) unpack4(ba[i], b4);
-            else {
+            {
+                const int sl = i & 3;
+                const int r = rg * 8 + i;
+                const bool valid = r < n;
+                float k4[4], q4[4], b4[4], w4[4];
+                unpack4(ka[sl], k4);
+                unpack4(qa[sl], q4);
+                if (bch) unpack4(ba[sl], b4);
+                else {
 #pragma unroll
-                for (int e = 0; e < 4; ++e) b4[e] = s_bscal[r];
-            }
-            if (!TIED) {
-                if (pp.wkind == GDR_GATE_TIED) {
-#pragma unroll
-                    for (int e = 0; e < 4; ++e) w4[e] = b4[e];
-                } else if (wch) {
-                    unpack4(wa[i], w4);
-                } else {
-#pragma unroll
-                    for (int e = 0; e < 4; ++e) w4[e] = s_wscal[r];
+                    for (int e = 0; e < 4; ++e) b4[e] = s_bscal[r];
                 }
-            }
-            if (ACH) {
+                if (!TIED) {
+                    if (pp.wkind == GDR_GATE_TIED) {
 #pragma unroll
-                for (int e = 0; e < 4; ++e)
-                    rowf_c[e] = (i == 0) ? ex2_approx(lrow0[e]) : rowf_c[e] * aval[i][e];
-            }
-            const float rs = ACH ? 0.f : s_rowf[r], cs = ACH ? 0.f : s_colf[r];
-            float kb[4], qs[4], ks[4], kws[4], qg[4], k2[4], kw2[4];
+                        for (int e = 0; e < 4; ++e) w4[e] = b4[e];
+                    } else if (wch) {
+                        unpack4(wa[sl], w4);
+                    } else {
 #pragma unroll
-            for (int e = 0; e < 4; ++e) {
-                const float rowf = ACH ? rowf_c[e] : rs;
-                const float colf = ACH ? rcp_newton(rowf) : cs;
-                const float kk = valid ? k4[e] : 0.f;
-                const float qq = valid ? q4[e] : 0.f;
-                kb[e] = b4[e] * kk * rowf;
-                qs[e] = qq * rowf;
-                ks[e] = kk * colf;
-                kws[e] = TIED ? 0.f : w4[e] * kk * colf;
-                qg[e] = qs[e] * er[e];
-                k2[e] = ks[e] * fs[e];
-                kw2[e] = kws[e] * fs[e];
-            }
-            st4(sm + G_OFF_ROP, piece4(r, cg, 128), kb);
-            st4(sm + G_OFF_ROP, piece4(64 + r, cg, 128), qs);
-            st4(sm + G_OFF_COP, piece4(r, cg, N1), ks);
-            if (!TIED) st4(sm + G_OFF_COP, piece4(64 + r, cg, N1), kws);
-            if (valid) {
-                const size_t e = (((size_t)bb * T + t0 + r) * H + h) * DK + ch0;
-                st8b(pp.qg + e, qg);
-                st8b(pp.k2 + e, k2);
-                if (!TIED) st8b(pp.kw2 + e, kw2);
+                        for (int e = 0; e < 4; ++e) w4[e] = s_wscal[r];
+                    }
+                }
+                if (i < 4) load_token(i + 4);
+                if (ACH) {
+                    // rowf by a multiply chain over the thread's 8 tokens (one exp2)
+                    float av[4];
+                    unpack4(aa[i], av);
+#pragma unroll
+                    for (int e = 0; e < 4; ++e)
+                        rowf_c[e] = (i == 0) ? ex2_approx(lrow0[e]) : rowf_c[e] * (valid ? av[e] : 1.f);
+                }
+                const float rs = ACH ? 0.f : s_rowf[r], cs = ACH ? 0.f : s_colf[r];
+                float kb[4], qs[4], ks[4], kws[4], qg[4], k2[4], kw2[4];
+#pragma unroll
+                for (int e = 0; e < 4; ++e) {
+                    const float rowf = ACH ? rowf_c[e] : rs;
+                    const float colf = ACH ? rcp_newton(rowf) : cs;
+                    const float kk = valid ? k4[e] : 0.f;
+                    const float qq = valid ? q4[e] : 0.f;
+                    kb[e] = b4[e] * kk * rowf;
+                    qs[e] = qq * rowf;
+                    ks[e] = kk * colf;
+                    kws[e] = TIED ? 0.f : w4[e] * kk * colf;
+                    qg[e] = qs[e] * er[e];
+                    k2[e] = ks[e] * fs[e];
+                    kw2[e] = kws[e] * fs[e];
+                }
+                st4(sm + G_OFF_ROP, piece4(r, cg, 128), kb);
+                st4(sm + G_OFF_ROP, piece4(64 + r, cg, 128), qs);
+                st4(sm + G_OFF_COP, piece4(r, cg, N1), ks);
+                if (!TIED) st4(sm + G_OFF_COP, piece4(64 + r, cg, N1), kws);
+                if (valid) {
+                    const size_t e = (((size_t)bb * T + t0 + r) * H + h) * DK + ch0;
+                    st8b(pp.qg + e, qg);
+                    st8b(pp.k2 + e, k2);
+                    if (!TIED) st8b(pp.kw2 + e, kw2);
+                }
             }
         }
     }
     GDR_BEFORE_MMA();
+    GDR_TRACE_G(3);
 
     // ---- P1: D1 = [Kb ; Qs] x [Ks ; Kws]^T ---------------------------------------
     if (tid == 0) {
@@ -331,6 +380,7 @@ __global__ void __launch_bounds__(NT, 2) prep_general_kernel(const __grid_consta
     }
     GDR_WAIT(bar_mma, ph_mma);
     tc_fence_after();
+    GDR_TRACE_G(4);
     // the Qs rows are consumed: V's tiles go there (column block vt, rows 64..127)
     if (tid == 0) {
         mbar_expect_tx(bar_v, (uint32_t)nvt * 8192u);
@@ -338,7 +388,8 @@ __global__ void __launch_bounds__(NT, 2) prep_general_kernel(const __grid_consta
             tma_load_4d(sm + G_OFF_ROP + vt * 16384 + 8192, &tm_v, bar_v, vt * 64, h, t0, bb);
     }
 
-    // ---- unload D1: A (fp32) + transposed diagonal blocks; Bm -> X; Aq, Bq -> workspace
+    // ---- unload D1: A (fp32) + transposed diagonal blocks; Bm -> X;
+    //      Aq (Bq) -> staging in L (APRE) -> workspace by bulk tensor store ----------
     {
         const int r = row & 63;
         float d[32], d2[32];
@@ -374,25 +425,39 @@ __global__ void __launch_bounds__(NT, 2) prep_general_kernel(const __grid_consta
                     st_chunk(sm + G_OFF_X, sw128_chunk(r, wg * 4 + c8, 64), x);
                 }
             }
-        } else if (r < n) {
-            const size_t tok = ((size_t)bb * T + t0 + r) * H + h;
+        } else {
 #pragma unroll
-            for (int j = 0; j < 32; ++j) {
-                const bool keep = wg * 32 + j <= r;
-                d[j] = keep ? d[j] : 0.f;
-                if (!TIED) d2[j] = keep ? d2[j] : 0.f;
+            for (int c8 = 0; c8 < 4; ++c8) {
+                float x[8], y[8];
+#pragma unroll
+                for (int e = 0; e < 8; ++e) {
+                    const bool keep = wg * 32 + c8 * 8 + e <= r;
+                    x[e] = keep ? d[c8 * 8 + e] : 0.f;
+                    y[e] = keep && !TIED ? d2[c8 * 8 + e] : 0.f;
+                }
+                st_chunk(sm + G_OFF_L, sw128_chunk(r, wg * 4 + c8, 64), x);
+                if (!TIED) st_chunk(sm + G_OFF_APRE, sw128_chunk(r, wg * 4 + c8, 64), y);
             }
-            st32_bf16(pp.aq + tok * 64 + wg * 32, d, 1.f);
-            if (!TIED) st32_bf16(pp.bq + tok * 64 + wg * 32, d2, 1.f);
         }
     }
+    fence_proxy_async();
     __syncthreads();
+    if (tid == 0) {
+        tma_store_4d(&tm_aq, sm + G_OFF_L, 0, h, t0, bb);
+        if (!TIED) tma_store_4d(&tm_bq, sm + G_OFF_APRE, 0, h, t0, bb);
+        bulk_commit_group();
+    }
+    GDR_TRACE_G(5);
 
     // ---- T = (I + A)^-1; L = T (bf16); tied: APRE = T Diag(beta) ------------------
     {
         float* A32 = reinterpret_cast<float*>(sm + G_OFF_A32);
         float* T32 = reinterpret_cast<float*>(sm + G_OFF_T32);
         solve_unit_lower(A32, T32, reinterpret_cast<float*>(sm + G_OFF_SCR), tid, warp);
+        // the Aq / Bq stores have read their staging tiles before L, APRE are rewritten
+        if (tid == 0) bulk_wait_group_read0();
+        __syncthreads();
+        GDR_TRACE_G(6);
         const int r = tid & 63, q4 = tid >> 6;
 #pragma unroll
         for (int cc = 0; cc < 2; ++cc) {
@@ -417,7 +482,9 @@ __global__ void __launch_bounds__(NT, 2) prep_general_kernel(const __grid_consta
         }
     }
     GDR_BEFORE_MMA();
+    GDR_TRACE_G(7);
     GDR_WAIT(bar_v, ph_v);  // V arrived during the solve
+    GDR_TRACE_G(8);
 
     // ---- P2: D2 = T Kb (cols 0..127);  tied: D3 = T Diag(beta) V (cols 128..);
     //      general: T Bm (cols 128..191) ----------------------------------------------
@@ -440,35 +507,36 @@ __global__ void __launch_bounds__(NT, 2) prep_general_kernel(const __grid_consta
     }
     GDR_WAIT(bar_mma, ph_mma);
     tc_fence_after();
+    GDR_TRACE_G(9);
 
-    // ---- WN = -W 2^ref (rows 0..63) -> workspace; tied: P -> workspace;
-    //      general: -T Bm -> APRE -----------------------------------------------------
+    // ---- WN = -W 2^ref -> staging (A32 region); tied: P -> staging (T32 region);
+    //      general: -T Bm -> APRE ------------------------------------------------------
     if (row < 64) {
         const int r = row;
-        const size_t tok = ((size_t)bb * T + t0 + r) * H + h;
         float d[32], d1[32];
         tmem_ld32_async(tmem + lane_base + wg * 64, d);
         tmem_ld32_async(tmem + lane_base + wg * 64 + 32, d1);
         tmem_wait_ld();
 #pragma unroll
-        for (int j4 = 0; j4 < 32; j4 += 4) {
-            const float4 e0 = *reinterpret_cast<const float4*>(s_eref + wg * 64 + j4);
-            const float4 e1 = *reinterpret_cast<const float4*>(s_eref + wg * 64 + 32 + j4);
-            d[j4] *= e0.x; d[j4 + 1] *= e0.y; d[j4 + 2] *= e0.z; d[j4 + 3] *= e0.w;
-            d1[j4] *= e1.x; d1[j4 + 1] *= e1.y; d1[j4 + 2] *= e1.z; d1[j4 + 3] *= e1.w;
-        }
-        if (r < n) {
-            st32_bf16(pp.wn + tok * DK + wg * 64, d, -1.f);
-            st32_bf16(pp.wn + tok * DK + wg * 64 + 32, d1, -1.f);
+        for (int c8 = 0; c8 < 8; ++c8) {
+            float x[8];
+            const float* dd = c8 < 4 ? d + c8 * 8 : d1 + (c8 - 4) * 8;
+            const float4 e0 = *reinterpret_cast<const float4*>(s_eref + wg * 64 + c8 * 8);
+            const float4 e1 = *reinterpret_cast<const float4*>(s_eref + wg * 64 + c8 * 8 + 4);
+            x[0] = -dd[0] * e0.x; x[1] = -dd[1] * e0.y; x[2] = -dd[2] * e0.z; x[3] = -dd[3] * e0.w;
+            x[4] = -dd[4] * e1.x; x[5] = -dd[5] * e1.y; x[6] = -dd[6] * e1.z; x[7] = -dd[7] * e1.w;
+            st_chunk(sm + G_OFF_A32, sw128_chunk(r, wg * 8 + c8, 64), x);
         }
         if (TIED) {
             const int half = dv >> 1;
             tmem_ld32_async(tmem + lane_base + 128 + wg * half, d);
             if (half == 64) tmem_ld32_async(tmem + lane_base + 128 + wg * half + 32, d1);
             tmem_wait_ld();
-            if (r < n) {
-                st32_bf16(pp.p + tok * dv + wg * half, d, 1.f);
-                if (half == 64) st32_bf16(pp.p + tok * dv + wg * half + 32, d1, 1.f);
+#pragma unroll
+            for (int c8 = 0; c8 < 8; ++c8) {
+                if (c8 * 8 >= half) break;
+                const float* dd = c8 < 4 ? d + c8 * 8 : d1 + (c8 - 4) * 8;
+                st_chunk(sm + G_OFF_T32, sw128_chunk(r, (wg * half) / 8 + c8, 64), dd);
             }
         } else {
             tmem_ld32(tmem + lane_base + 128 + wg * 32, d);
@@ -481,9 +549,17 @@ __global__ void __launch_bounds__(NT, 2) prep_general_kernel(const __grid_consta
             }
         }
     }
+    GDR_BEFORE_MMA();
+    if (tid == 0) {
+        tma_store_4d(&tm_wn, sm + G_OFF_A32, 0, h, t0, bb);
+        tma_store_4d(&tm_wn, sm + G_OFF_A32 + 8192, 64, h, t0, bb);
+        if (TIED)
+            for (int vt = 0; vt < nvt; ++vt) tma_store_4d(&tm_p, sm + G_OFF_T32 + vt * 8192, vt * 64, h, t0, bb);
+        bulk_commit_group();
+    }
+    GDR_TRACE_G(10);
     if (!TIED) {
-        GDR_BEFORE_MMA();
-        // ---- P3: D3 = (-T Bm) V -> P ------------------------------------------------
+        // ---- P3: D3 = (-T Bm) V -> P --------------------------------------------------
         if (tid == 0) {
             tc_fence_after();
             const uint32_t idP = idesc_bf16(128, dv, 0, 1);
@@ -497,21 +573,30 @@ __global__ void __launch_bounds__(NT, 2) prep_general_kernel(const __grid_consta
         tc_fence_after();
         if (row < 64) {
             const int r = row;
-            const size_t tok = ((size_t)bb * T + t0 + r) * H + h;
             const int half = dv >> 1;
             float d[32], d1[32];
             tmem_ld32_async(tmem + lane_base + wg * half, d);
             if (half == 64) tmem_ld32_async(tmem + lane_base + wg * half + 32, d1);
             tmem_wait_ld();
-            if (r < n) {
-                st32_bf16(pp.p + tok * dv + wg * half, d, 1.f);
-                if (half == 64) st32_bf16(pp.p + tok * dv + wg * half + 32, d1, 1.f);
+#pragma unroll
+            for (int c8 = 0; c8 < 8; ++c8) {
+                if (c8 * 8 >= half) break;
+                const float* dd = c8 < 4 ? d + c8 * 8 : d1 + (c8 - 4) * 8;
+                st_chunk(sm + G_OFF_T32, sw128_chunk(r, (wg * half) / 8 + c8, 64), dd);
             }
         }
+        fence_proxy_async();
+        __syncthreads();
+        if (tid == 0) {
+            for (int vt = 0; vt < nvt; ++vt) tma_store_4d(&tm_p, sm + G_OFF_T32 + vt * 8192, vt * 64, h, t0, bb);
+            bulk_commit_group();
+        }
     }
+    GDR_TRACE_G(11);
 
 finish:
     if (!ok && tid == 0) flag_status(pp.d_status, GDR_DEVICE_TIMEOUT);
+    if (tid == 0) bulk_wait_group0();
     tc_fence_before();
     __syncthreads();
     if (warp == 0) tmem_dealloc(tmem, G_TM_COLS);
@@ -537,12 +622,13 @@ struct StateLayout {
 constexpr uint32_t GS_TM_D3 = 0, GS_TM_D5 = 128, GS_TM_D4 = 256, GS_TM_COLS = 512;
 
 struct GStateParams {
-    const float* S0;
+    const float* S0;  // state at chunk c_begin (NULL: zero)
     const float* gc;
     __nv_bfloat16* o;
-    float* ST;
+    float* ST;        // state after chunk c_end - 1 (NULL: not written); may alias S0
     int* d_status;
     int T, H, dv;
+    int c_begin, c_end;  // chunk range of this launch
 };
 
 template <bool UNTIED>
@@ -614,9 +700,10 @@ __global__ void __launch_bounds__(NT, 1) state_general_kernel(
 #pragma unroll
         for (int ch = 0; ch < 4; ++ch) st_chunk(sm + Lay::SBF, sw128_chunk(row, wg * 4 + ch, DK), &S[8 * ch]);
     }
+    const int c_begin = p.c_begin, c_end = p.c_end;
     const float* gcp = p.gc + ((size_t)bb * H + h) * nchunks * DK + row;
-    float gC_next = nchunks > 0 ? gcp[0] : 0.f;
-    if (tid == 0 && nchunks > 0) issue_loads(0);
+    float gC_next = c_begin < c_end ? gcp[(size_t)c_begin * DK] : 0.f;
+    if (tid == 0 && c_begin < c_end) issue_loads(c_begin);
 
     auto store_o = [&](int cj) {
         const int pj = cj & 1;
@@ -645,14 +732,14 @@ __global__ void __launch_bounds__(NT, 1) state_general_kernel(
         __syncthreads();    \
     } while (0)
 
-    for (int ci = 0; ci < nchunks; ++ci) {
+    for (int ci = c_begin; ci < c_end; ++ci) {
         const int buf = ci & 1, par = ci & 1;
         const uint32_t wqb = sbase + Lay::WQ + buf * 32768u;
         const uint32_t k2b = sbase + Lay::K2 + buf * 16384u;
         const uint32_t aqub = sbase + Lay::AQU + buf * 16384u;
         const uint32_t d3 = GS_TM_D3 + (uint32_t)par * 64u, d5 = GS_TM_D5 + (uint32_t)par * 64u;
         const float gC = gC_next;
-        if (ci + 1 < nchunks) gC_next = gcp[(size_t)(ci + 1) * DK];
+        if (ci + 1 < c_end) gC_next = gcp[(size_t)(ci + 1) * DK];
         if (buf == 0) GDR_WAIT(&bar_tma[0], ph_tma0);
         else GDR_WAIT(&bar_tma[1], ph_tma1);
 
@@ -681,9 +768,9 @@ __global__ void __launch_bounds__(NT, 1) state_general_kernel(
             mma_commit(bar_mma);
         }
         // chunk ci + 1's inputs go to the buffers chunk ci - 1 has released
-        if (tid == 32 && ci + 1 < nchunks) issue_loads(ci + 1);
+        if (tid == 32 && ci + 1 < c_end) issue_loads(ci + 1);
         // the previous chunk's outputs, while batch 1 runs
-        if (row >= 64 && ci > 0) store_o(ci - 1);
+        if (row >= 64 && ci > c_begin) store_o(ci - 1);
         GDR_WAIT(bar_mma, ph_mma);
         tc_fence_after();
 
@@ -732,7 +819,7 @@ __global__ void __launch_bounds__(NT, 1) state_general_kernel(
         tc_fence_before();
         __syncthreads();
     }
-    if (row >= 64 && nchunks > 0) store_o(nchunks - 1);
+    if (row >= 64 && c_begin < c_end) store_o(c_end - 1);
 
     if (p.ST) {
         float* st = p.ST + (((size_t)bb * H + h) * DK + row) * p.dv + v0 + wg * NH;
@@ -752,9 +839,10 @@ finish:
 }  // namespace twopass_g
 
 // Workspace of the general two-pass path: sub-buffers in this order, each
-// rounded up to 256 bytes: WN, QG, K2, AQ, P, [KW2, BQ], GC.
+// rounded up to 256 bytes: WN, QG, K2, AQ, P, [KW2, BQ], GC, and the fp32
+// state carried between the segments of a segmented state pass.
 struct GeneralWorkspace {
-    size_t off[8];
+    size_t off[9];
     size_t total;
 };
 
@@ -762,12 +850,12 @@ static GeneralWorkspace general_workspace_layout(int B, int T, int H, int dv, bo
     auto up = [](size_t x) { return (x + 255) & ~(size_t)255; };
     const size_t tok = (size_t)B * T * H;
     const size_t nchunks = ((size_t)T + 63) / 64;
-    const size_t sizes[8] = {tok * 128 * 2, tok * 128 * 2, tok * 128 * 2, tok * 64 * 2,
+    const size_t sizes[9] = {tok * 128 * 2, tok * 128 * 2, tok * 128 * 2, tok * 64 * 2,
                              tok * (size_t)dv * 2, untied ? tok * 128 * 2 : 0, untied ? tok * 64 * 2 : 0,
-                             (size_t)B * H * nchunks * 128 * 4};
+                             (size_t)B * H * nchunks * 128 * 4, (size_t)B * H * 128 * (size_t)dv * 4};
     GeneralWorkspace w;
     size_t o = 0;
-    for (int i = 0; i < 8; ++i) {
+    for (int i = 0; i < 9; ++i) {
         w.off[i] = o;
         o += up(sizes[i]);
     }
@@ -780,6 +868,30 @@ size_t twopass_general_workspace_bytes(int B, int T, int H, int dv, bool untied)
 }
 
 using MapFn = bool (*)(CUtensorMap*, const void*, int, int, int, int);
+
+// Segmented state pass: segments of at least kSegMin chunks, at most
+// kMaxSegments. The auxiliary stream and events are created on the first
+// segmented call on a device and kept for the process.
+constexpr int kSegMin = 32;
+constexpr int kMaxSegments = 8;
+
+static bool aux_resources(int dev, cudaStream_t* aux, cudaEvent_t** evs) {
+    static std::mutex mu;
+    static cudaStream_t streams[64] = {};
+    static cudaEvent_t events[64][kMaxSegments + 1] = {};
+    if (dev < 0 || dev >= 64) return false;
+    std::lock_guard<std::mutex> lock(mu);
+    if (!streams[dev]) {
+        cudaStream_t s = nullptr;
+        if (cudaStreamCreateWithFlags(&s, cudaStreamNonBlocking) != cudaSuccess) return false;
+        for (int i = 0; i <= kMaxSegments; ++i)
+            if (cudaEventCreateWithFlags(&events[dev][i], cudaEventDisableTiming) != cudaSuccess) return false;
+        streams[dev] = s;
+    }
+    *aux = streams[dev];
+    *evs = events[dev];
+    return true;
+}
 
 // maps: q, k, v (of the call). alpha/b/w kinds as in the C ABI.
 cudaError_t launch_chunk_twopass_general(const CUtensorMap* maps, MapFn make_map, void* ws,
@@ -807,18 +919,6 @@ cudaError_t launch_chunk_twopass_general(const CUtensorMap* maps, MapFn make_map
     pp.d_status = d_status;
     pp.T = T; pp.H = H; pp.dv = dv;
     pp.akind = akind; pp.bkind = bkind; pp.wkind = wkind;
-    const int nchunks = (T + C - 1) / C;
-    const dim3 pgrid(nchunks, H, B);
-    auto prep = [&](auto kern) -> cudaError_t {
-        cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, G_SMEM_BYTES);
-        if (e != cudaSuccess) return e;
-        kern<<<pgrid, NT, G_SMEM_BYTES, st>>>(maps[2], pp);
-        return cudaGetLastError();
-    };
-    cudaError_t e = tied ? (ach ? prep(prep_general_kernel<true, true>) : prep(prep_general_kernel<true, false>))
-                         : (ach ? prep(prep_general_kernel<false, true>) : prep(prep_general_kernel<false, false>));
-    if (e != cudaSuccess) return e;
-
     CUtensorMap sm_maps[8];
     const int dims[7] = {128, 128, 128, 64, dv, 128, 64};
     for (int i = 0; i < 7; ++i) {
@@ -827,19 +927,81 @@ cudaError_t launch_chunk_twopass_general(const CUtensorMap* maps, MapFn make_map
         if (!make_map(&sm_maps[i], ptr, B, T, H, d)) return cudaErrorInvalidValue;
     }
     sm_maps[7] = maps[2];
+    // the untied maps stand in for the tied form's unused Bq output
+    const CUtensorMap& bq_map = tied ? sm_maps[3] : sm_maps[6];
+
+    const int nchunks = (T + C - 1) / C;
+    auto prep_range = [&](int c0, int c1, cudaStream_t stream) -> cudaError_t {
+        GPrepParams pr = pp;
+        pr.c_begin = c0;
+        const dim3 pgrid(c1 - c0, H, B);
+        auto go = [&](auto kern) -> cudaError_t {
+            cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, G_SMEM_BYTES);
+            if (e != cudaSuccess) return e;
+            kern<<<pgrid, NT, G_SMEM_BYTES, stream>>>(maps[2], sm_maps[0], sm_maps[3], sm_maps[4], bq_map, pr);
+            return cudaGetLastError();
+        };
+        return tied ? (ach ? go(prep_general_kernel<true, true>) : go(prep_general_kernel<true, false>))
+                    : (ach ? go(prep_general_kernel<false, true>) : go(prep_general_kernel<false, false>));
+    };
     GStateParams sp;
-    sp.S0 = S0; sp.gc = pp.gc; sp.o = reinterpret_cast<__nv_bfloat16*>(o); sp.ST = ST;
+    sp.gc = pp.gc; sp.o = reinterpret_cast<__nv_bfloat16*>(o);
     sp.d_status = d_status; sp.T = T; sp.H = H; sp.dv = dv;
     const dim3 sgrid(dv / NV, H, B);
-    auto state = [&](auto kern, uint32_t bytes) -> cudaError_t {
-        cudaError_t e2 = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, bytes);
-        if (e2 != cudaSuccess) return e2;
-        kern<<<sgrid, NT, bytes, st>>>(sm_maps[0], sm_maps[1], sm_maps[2], sm_maps[3], sm_maps[4],
-                                       sm_maps[5], sm_maps[6], sm_maps[7], sp);
-        return cudaGetLastError();
+    auto state_range = [&](int c0, int c1, const float* s_in, float* s_out) -> cudaError_t {
+        GStateParams sr = sp;
+        sr.c_begin = c0; sr.c_end = c1; sr.S0 = s_in; sr.ST = s_out;
+        auto go = [&](auto kern, uint32_t bytes) -> cudaError_t {
+            cudaError_t e2 = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, bytes);
+            if (e2 != cudaSuccess) return e2;
+            kern<<<sgrid, NT, bytes, st>>>(sm_maps[0], sm_maps[1], sm_maps[2], sm_maps[3], sm_maps[4],
+                                           sm_maps[5], sm_maps[6], sm_maps[7], sr);
+            return cudaGetLastError();
+        };
+        return tied ? go(state_general_kernel<false>, StateLayout<false>::BYTES)
+                    : go(state_general_kernel<true>, StateLayout<true>::BYTES);
     };
-    return tied ? state(state_general_kernel<false>, StateLayout<false>::BYTES)
-                : state(state_general_kernel<true>, StateLayout<true>::BYTES);
+
+    // With few state CTAs (few heads, long sequences) most SMs would idle during
+    // the state pass: split the chunks into segments and let pass 1 of later
+    // segments run on an auxiliary stream while the state pass works through
+    // earlier ones (ordered by events only).
+    int nseg = 1;
+    cudaStream_t aux = nullptr;
+    cudaEvent_t* evs = nullptr;
+    int dev = 0, nsm = 0;
+    if (cudaGetDevice(&dev) == cudaSuccess &&
+        cudaDeviceGetAttribute(&nsm, cudaDevAttrMultiProcessorCount, dev) == cudaSuccess &&
+        (int)(sgrid.x * sgrid.y * sgrid.z) * 2 <= nsm && nchunks >= 2 * kSegMin) {
+        nseg = min(kMaxSegments, nchunks / kSegMin);
+        if (!aux_resources(dev, &aux, &evs)) nseg = 1;
+    }
+    if (nseg == 1) {
+        cudaError_t e = prep_range(0, nchunks, st);
+        if (e != cudaSuccess) return e;
+        return state_range(0, nchunks, S0, ST);
+    }
+    float* carry = reinterpret_cast<float*>(base + lay.off[8]);
+    cudaError_t e = cudaEventRecord(evs[kMaxSegments], st);
+    if (e == cudaSuccess) e = cudaStreamWaitEvent(aux, evs[kMaxSegments], 0);
+    for (int sgi = 0; sgi < nseg && e == cudaSuccess; ++sgi) {
+        const int c0 = (int)((long long)nchunks * sgi / nseg), c1 = (int)((long long)nchunks * (sgi + 1) / nseg);
+        e = prep_range(c0, c1, sgi == 0 ? st : aux);
+        if (e == cudaSuccess && sgi > 0) e = cudaEventRecord(evs[sgi], aux);
+    }
+    for (int sgi = 0; sgi < nseg && e == cudaSuccess; ++sgi) {
+        const int c0 = (int)((long long)nchunks * sgi / nseg), c1 = (int)((long long)nchunks * (sgi + 1) / nseg);
+        if (sgi > 0) e = cudaStreamWaitEvent(st, evs[sgi], 0);
+        if (e == cudaSuccess)
+            e = state_range(c0, c1, sgi == 0 ? S0 : carry, sgi == nseg - 1 ? ST : carry);
+    }
+    return e;
 }
 
 }  // namespace gdr
+
+#ifdef GDR_TRACE_PHASES
+extern "C" int gdr_trace_general_read(unsigned long long* host, int n) {
+    return (int)cudaMemcpyFromSymbol(host, gdr::twopass_g::g_trace3, sizeof(unsigned long long) * n);
+}
+#endif

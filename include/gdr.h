@@ -138,8 +138,14 @@ gdr_status gdr_chunk_fwd(const void* q, const void* k, const void* v,
  *   every other form: the per-token rows of -W 2^ref, q.g, k.g_{n-1}/g,
  *     the masked (q.rowf)(k.colf)^T block row and P (plus, with independent
  *     b and w, w.k.g_{n-1}/g and the masked (q.rowf)(w.k.colf)^T row), in
- *     bf16, and g_{n-1} per chunk and channel in fp32, each sub-buffer
- *     rounded up to 256 bytes.
+ *     bf16, g_{n-1} per chunk and channel in fp32, and one fp32 state
+ *     [B, H, d_k, d_v] carried between the segments of a segmented state
+ *     pass, each sub-buffer rounded up to 256 bytes.
+ * With few (batch, head, 64-column) state tiles and long sequences the
+ * general form splits the state pass into segments and runs the first pass of
+ * later segments on an auxiliary stream while the state pass works through
+ * earlier ones; the library then keeps that stream and a few events per
+ * device for the rest of the process.
  * Host-only; launches nothing.
  */
 size_t gdr_chunk_fwd_workspace_size(int B, int T, int H, int d_k, int d_v,

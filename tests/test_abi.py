@@ -109,8 +109,8 @@ def test_binding_raises_on_error_status():
     ((4, 4096, 16, 128, 128), (1, 1, 3), 4 * 4096 * 16 * (128 + 128) * 2),   # GDN form
     ((1, 100, 2, 128, 64), (1, 1, 3), 1 * 100 * 2 * (128 + 64) * 2),
     ((1, 64, 1, 128, 256), (1, 1, 3), 0),          # d_v > 128: single pass only
-    ((1, 64, 1, 128, 128), (2, 1, 3), 3 * 16384 + 8192 + 16384 + 512),   # KDA form (general)
-    ((1, 100, 2, 128, 64), (2, 2, 2), 4 * 51200 + 3 * 25600 + 2048),      # GDN-2 form (general)
+    ((1, 64, 1, 128, 128), (2, 1, 3), 3 * 16384 + 8192 + 16384 + 512 + 65536),   # KDA form
+    ((1, 100, 2, 128, 64), (2, 2, 2), 4 * 51200 + 3 * 25600 + 2048 + 65536),      # GDN-2 form
     ((1, 64, 1, 128, 128), (2, 0, 0), 0),          # no erase: single pass only
     ((1, 64, 1, 64, 64), (1, 1, 3), 0),            # not the tensor-core shape
     ((1, 0, 1, 128, 128), (1, 1, 3), 0),

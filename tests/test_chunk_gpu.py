@@ -237,3 +237,19 @@ def test_two_pass_full_size_matches_single_pass(cuda_device, family):
     o1, S1 = run_chunk(inp, cuda_device, workspace=None)
     assert_close(o2, o1, 2e-2, "o two-pass vs single pass")
     assert_close(S2, S1, 2e-2, "S_T two-pass vs single pass")
+
+
+@pytest.mark.parametrize("family", ["kda", "gdn2"])
+@pytest.mark.parametrize("T", [4200, 9000])
+def test_two_pass_segmented_state_pass(cuda_device, family, T):
+    """Few heads and a long sequence: the general form splits the state pass
+    into segments (the first pass of later segments overlaps earlier state
+    segments on a second stream, the state carried between them)."""
+    wl = WORKLOADS[family].with_(B=1, H=2, T=T, s0=True, seed=900 + T)
+    inp = make_chunk_inputs(wl)
+    o2, S2 = run_chunk(inp, cuda_device)
+    o1, S1 = run_chunk(inp, cuda_device, workspace=None)
+    o_ref, ST_ref = run_oracle(inp)
+    assert_close(o2, o_ref, TOL["bf16"], "o (segmented two-pass)")
+    assert_close(S2, ST_ref, TOL["bf16"], "S_T (segmented two-pass)")
+    assert_close(o2, o1, 2e-2, "o two-pass vs single pass")
