@@ -700,6 +700,10 @@ __global__ void __launch_bounds__(NT, 1) state_general_kernel(
 #pragma unroll
         for (int ch = 0; ch < 4; ++ch) st_chunk(sm + Lay::SBF, sw128_chunk(row, wg * 4 + ch, DK), &S[8 * ch]);
     }
+    // the state's bf16 copy is read by the first MMA batch (async proxy)
+    fence_proxy_async();
+    tc_fence_before();
+    __syncthreads();
     const int c_begin = p.c_begin, c_end = p.c_end;
     const float* gcp = p.gc + ((size_t)bb * H + h) * nchunks * DK + row;
     float gC_next = c_begin < c_end ? gcp[(size_t)c_begin * DK] : 0.f;
@@ -731,6 +735,18 @@ __global__ void __launch_bounds__(NT, 1) state_general_kernel(
         tc_fence_before();  \
         __syncthreads();    \
     } while (0)
+    // Waits inside the chunk loop are per thread; a timed-out wait is carried in
+    // w_ok to the next block barrier, where the block leaves together.
+    bool w_ok = true;
+#define GDR_WAIT_SOLO(bar, ph)              \
+    do {                                    \
+        w_ok = mbar_wait(bar, ph) && w_ok;  \
+        ph ^= 1u;                           \
+    } while (0)
+#define GDR_SYNC_CHECK()                                            \
+    do {                                                            \
+        if (!__syncthreads_and(w_ok)) { ok = false; goto finish; }  \
+    } while (0)
 
     for (int ci = c_begin; ci < c_end; ++ci) {
         const int buf = ci & 1, par = ci & 1;
@@ -740,8 +756,8 @@ __global__ void __launch_bounds__(NT, 1) state_general_kernel(
         const uint32_t d3 = GS_TM_D3 + (uint32_t)par * 64u, d5 = GS_TM_D5 + (uint32_t)par * 64u;
         const float gC = gC_next;
         if (ci + 1 < c_end) gC_next = gcp[(size_t)(ci + 1) * DK];
-        if (buf == 0) GDR_WAIT(&bar_tma[0], ph_tma0);
-        else GDR_WAIT(&bar_tma[1], ph_tma1);
+        if (buf == 0) GDR_WAIT_SOLO(&bar_tma[0], ph_tma0);
+        else GDR_WAIT_SOLO(&bar_tma[1], ph_tma1);
 
         // ---- batch 1: D3 = [WN ; QG] S;  untied: D4 = KW2^T V, D5 = [. ; BQ] V --------
         if (tid == 0) {
@@ -771,7 +787,7 @@ __global__ void __launch_bounds__(NT, 1) state_general_kernel(
         if (tid == 32 && ci + 1 < c_end) issue_loads(ci + 1);
         // the previous chunk's outputs, while batch 1 runs
         if (row >= 64 && ci > c_begin) store_o(ci - 1);
-        GDR_WAIT(bar_mma, ph_mma);
+        GDR_WAIT_SOLO(bar_mma, ph_mma);
         tc_fence_after();
 
         // ---- U = P + WN S (rows 0..63) -> rows 0..63 of [U ; AQ] ------------------------
@@ -787,7 +803,9 @@ __global__ void __launch_bounds__(NT, 1) state_general_kernel(
                 st_chunk(sm + Lay::AQU + buf * 16384, sw128_chunk(row, wg * 4 + c8, 128), x);
             }
         }
-        GDR_BEFORE_MMA();
+        fence_proxy_async();
+        tc_fence_before();
+        GDR_SYNC_CHECK();
 
         // ---- batch 2: D5 (+)= [U ; AQ] U (rows 64..127: AQ U);  D4 (+)= K2^T U ----------
         if (tid == 0) {
@@ -804,7 +822,7 @@ __global__ void __launch_bounds__(NT, 1) state_general_kernel(
             }
             mma_commit(bar_mma);
         }
-        GDR_WAIT(bar_mma, ph_mma);
+        GDR_WAIT_SOLO(bar_mma, ph_mma);
         tc_fence_after();
 
         // ---- S = Diag(GC) S + D4 ---------------------------------------------------------
@@ -816,8 +834,9 @@ __global__ void __launch_bounds__(NT, 1) state_general_kernel(
 #pragma unroll
             for (int ch = 0; ch < 4; ++ch) st_chunk(sm + Lay::SBF, sw128_chunk(row, wg * 4 + ch, DK), &S[8 * ch]);
         }
+        fence_proxy_async();  // the state copy feeds the next chunk's MMAs
         tc_fence_before();
-        __syncthreads();
+        GDR_SYNC_CHECK();
     }
     if (row >= 64 && c_begin < c_end) store_o(c_end - 1);
 
@@ -834,6 +853,8 @@ finish:
     if (warp == 0) tmem_dealloc(tmem, GS_TM_COLS);
 #undef GDR_WAIT
 #undef GDR_BEFORE_MMA
+#undef GDR_WAIT_SOLO
+#undef GDR_SYNC_CHECK
 }
 
 }  // namespace twopass_g

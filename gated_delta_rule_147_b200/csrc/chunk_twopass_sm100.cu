@@ -446,6 +446,10 @@ __global__ void __launch_bounds__(NT, 1) state_gdn_kernel(
 #pragma unroll
         for (int ch = 0; ch < 4; ++ch) st_chunk(sm + S_OFF_SBF, sw128_chunk(row, wg * 4 + ch, DK), &S[8 * ch]);
     }
+    // the state's bf16 copy is read by the first MMA batch (async proxy)
+    fence_proxy_async();
+    tc_fence_before();
+    __syncthreads();
     unsigned short g_a = 0;
     auto load_alpha = [&](int ci) {
         if (tid < C) {
@@ -513,6 +517,18 @@ __global__ void __launch_bounds__(NT, 1) state_gdn_kernel(
         tc_fence_before();  \
         __syncthreads();    \
     } while (0)
+    // Waits inside the chunk loop are per thread; a timed-out wait is carried in
+    // w_ok to the next block barrier, where the block leaves together.
+    bool w_ok = true;
+#define GDR_WAIT_SOLO(bar, ph)              \
+    do {                                    \
+        w_ok = mbar_wait(bar, ph) && w_ok;  \
+        ph ^= 1u;                           \
+    } while (0)
+#define GDR_SYNC_CHECK()                                            \
+    do {                                                            \
+        if (!__syncthreads_and(w_ok)) { ok = false; goto finish; }  \
+    } while (0)
 
     // O rows (64..127 of D3 / D5 in the column set of chunk cj) -> global
     auto store_o = [&](int cj) {
@@ -553,9 +569,9 @@ __global__ void __launch_bounds__(NT, 1) state_gdn_kernel(
         const float* s_colf = s_colf2 + par * 64;
         const float* s_gcr = s_gcr2 + par * 64;
         const float* s_misc = s_misc2 + par * 4;
-        if (buf == 0) GDR_WAIT(&bar_tma[0], ph_tma0);
-        else if (buf == 1) GDR_WAIT(&bar_tma[1], ph_tma1);
-        else GDR_WAIT(&bar_tma[2], ph_tma2);
+        if (buf == 0) GDR_WAIT_SOLO(&bar_tma[0], ph_tma0);
+        else if (buf == 1) GDR_WAIT_SOLO(&bar_tma[1], ph_tma1);
+        else GDR_WAIT_SOLO(&bar_tma[2], ph_tma2);
         GDR_TRACE_S(1);
 
         // ---- batch 1: D3 = [-W ; Q] S;  D1 = [-W ; Q] K^T (rows 64..127: Q K^T) ------
@@ -594,7 +610,7 @@ __global__ void __launch_bounds__(NT, 1) state_gdn_kernel(
                 st_chunk(sm + S_OFF_K2, off, x);
             }
         }
-        GDR_WAIT(bar_mma, ph_mma);
+        GDR_WAIT_SOLO(bar_mma, ph_mma);
         tc_fence_after();
         GDR_TRACE_S(2);
 
@@ -630,7 +646,9 @@ __global__ void __launch_bounds__(NT, 1) state_gdn_kernel(
             }
         }
         if (ci + 1 < nchunks) stage_alpha(ci + 1);
-        GDR_BEFORE_MMA();
+        fence_proxy_async();
+        tc_fence_before();
+        GDR_SYNC_CHECK();
         GDR_TRACE_S(3);
 
         // ---- batch 2: D5 = [U ; Aq] U (rows 64..127: Aq U);  D4 = (Diag(g_{n-1}/g) K)^T U --
@@ -648,7 +666,7 @@ __global__ void __launch_bounds__(NT, 1) state_gdn_kernel(
             mma_commit(bar_mma);
         }
         if (warp == 7 && ci + 1 < nchunks) decay_scan(ci + 1, tid & 31);  // overlaps batch 2
-        GDR_WAIT(bar_mma, ph_mma);
+        GDR_WAIT_SOLO(bar_mma, ph_mma);
         tc_fence_after();
         GDR_TRACE_S(4);
 
@@ -663,8 +681,9 @@ __global__ void __launch_bounds__(NT, 1) state_gdn_kernel(
             for (int ch = 0; ch < 4; ++ch) st_chunk(sm + S_OFF_SBF, sw128_chunk(row, wg * 4 + ch, DK), &S[8 * ch]);
         }
         GDR_TRACE_S(6);
+        fence_proxy_async();  // the state copy feeds the next chunk's MMAs
         tc_fence_before();
-        __syncthreads();
+        GDR_SYNC_CHECK();
         GDR_TRACE_S(5);
     }
     if (row >= 64 && nchunks > 0) store_o(nchunks - 1);
@@ -682,6 +701,8 @@ finish:
     if (warp == 0) tmem_dealloc(tmem, S_TM_COLS);
 #undef GDR_WAIT
 #undef GDR_BEFORE_MMA
+#undef GDR_WAIT_SOLO
+#undef GDR_SYNC_CHECK
 }
 
 }  // namespace twopass
