@@ -15,7 +15,8 @@ from __future__ import annotations
 
 from ._lib import (GATE_CHANNEL, GATE_NONE, GATE_SCALAR, GATE_TIED, GDR_BF16, GDR_FP32,
                    GDR_DEVICE_DECAY_RANGE, GDR_DEVICE_TIMEOUT, GdrError, gdr_chunk_fwd,
-                   gdr_chunk_fwd_static, gdr_chunk_fwd_workspace_size, gdr_decode_step, load)
+                   gdr_chunk_fwd_grouped, gdr_chunk_fwd_static, gdr_chunk_fwd_workspace_size,
+                   gdr_decode_step, gdr_decode_step_grouped, load)
 
 TIED = "tied"
 _KIND = {"none": GATE_NONE, "scalar": GATE_SCALAR, "channel": GATE_CHANNEL, "tied": GATE_TIED}
@@ -49,7 +50,8 @@ def _gate_kind(g, ndim_scalar: int):
 def workspace_bytes(q, v, alpha=None, b=None, w=None) -> int:
     """Scratch bytes the two-pass chunk path wants for these inputs (0 when
     the shape / gate form has no two-pass path)."""
-    B, T, H, dk = q.shape
+    B, T, _, dk = q.shape
+    H = v.shape[2]
     return gdr_chunk_fwd_workspace_size(B, T, H, dk, v.shape[-1], _gate_kind(alpha, 3),
                                         _gate_kind(b, 3), _gate_kind(w, 3), _dtype_code(q))
 
@@ -58,6 +60,8 @@ def chunk_fwd(q, k, v, alpha=None, b=None, w=None, S0=None, *, out=None, final_s
               S_T=None, chunk: int = 64, workspace="auto", d_status=None, stream=None):
     """Forward over [B,T,H,*] inputs. alpha/b/w: None, a [B,T,H] tensor
     (scalar gate), a [B,T,H,d_k] tensor (channel gate); w may be TIED (w := b).
+    q and k may have fewer heads than v (grouped heads: H a multiple of
+    H_qk, value head h reads q/k head h // (H // H_qk)).
     workspace: "auto" allocates the two-pass path's scratch with torch when
     the inputs have such a path; a uint8 device tensor supplies it; "static"
     uses the library's own scratch array (gdr_chunk_fwd_static); None runs
@@ -65,12 +69,14 @@ def chunk_fwd(q, k, v, alpha=None, b=None, w=None, S0=None, *, out=None, final_s
     is False."""
     import torch
     _check(q, k, v, alpha, b, w, S0, out, S_T)
-    B, T, H, dk = q.shape
-    dv = v.shape[-1]
+    B, T, Hq, dk = q.shape
+    H, dv = v.shape[2], v.shape[-1]
     o = out if out is not None else torch.empty((B, T, H, dv), dtype=v.dtype, device=v.device)
     if final_state and S_T is None:
         S_T = torch.empty((B, H, dk, dv), dtype=torch.float32, device=v.device)
     if isinstance(workspace, str) and workspace == "static":
+        if Hq != H:
+            raise ValueError("the static-scratch call takes ungrouped heads")
         gdr_chunk_fwd_static(q, k, v, alpha, b, None if isinstance(w, str) else w,
                              _gate_kind(alpha, 3), _gate_kind(b, 3), _gate_kind(w, 3), S0, o,
                              S_T if final_state else None, B, T, H, dk, dv, chunk, _dtype_code(q),
@@ -82,9 +88,10 @@ def chunk_fwd(q, k, v, alpha=None, b=None, w=None, S0=None, *, out=None, final_s
         nbytes = workspace_bytes(q, v, alpha, b, w)
         workspace = torch.empty(nbytes, dtype=torch.uint8, device=v.device) if nbytes else None
     ws_bytes = 0 if workspace is None else workspace.numel() * workspace.element_size()
-    gdr_chunk_fwd(q, k, v, alpha, b, None if isinstance(w, str) else w, _gate_kind(alpha, 3),
-                  _gate_kind(b, 3), _gate_kind(w, 3), S0, o, S_T if final_state else None,
-                  workspace, ws_bytes, B, T, H, dk, dv, chunk, _dtype_code(q), d_status, stream)
+    gdr_chunk_fwd_grouped(q, k, v, alpha, b, None if isinstance(w, str) else w,
+                          _gate_kind(alpha, 3), _gate_kind(b, 3), _gate_kind(w, 3), S0, o,
+                          S_T if final_state else None, workspace, ws_bytes, B, T, Hq, H, dk, dv,
+                          chunk, _dtype_code(q), d_status, stream)
     return o, (S_T if final_state else None)
 
 
@@ -94,10 +101,10 @@ def decode_step(q, k, v, alpha, b, w, S, *, out=None, d_status=None, stream=None
     Returns o [B,H,d_v]."""
     import torch
     _check(q, k, v, alpha, b, w, S, out)
-    B, H, dk = q.shape
-    dv = v.shape[-1]
+    B, Hq, dk = q.shape
+    H, dv = v.shape[1], v.shape[-1]
     o = out if out is not None else torch.empty((B, H, dv), dtype=v.dtype, device=v.device)
-    gdr_decode_step(q, k, v, alpha, b, None if isinstance(w, str) else w, _gate_kind(alpha, 2),
-                    _gate_kind(b, 2), _gate_kind(w, 2), S, o, B, H, dk, dv, _dtype_code(q),
-                    d_status, stream)
+    gdr_decode_step_grouped(q, k, v, alpha, b, None if isinstance(w, str) else w,
+                            _gate_kind(alpha, 2), _gate_kind(b, 2), _gate_kind(w, 2), S, o, B, Hq,
+                            H, dk, dv, _dtype_code(q), d_status, stream)
     return o

@@ -17,8 +17,9 @@ GDR_DEVICE_TIMEOUT, GDR_DEVICE_DECAY_RANGE = 1, 2
 GDR_BF16, GDR_FP32 = 0, 1
 GATE_NONE, GATE_SCALAR, GATE_CHANNEL, GATE_TIED = 0, 1, 2, 3
 
-EXPORTS = ("gdr_chunk_fwd", "gdr_chunk_fwd_workspace_size", "gdr_chunk_fwd_static",
-           "gdr_chunk_fwd_static_capacity", "gdr_decode_step", "gdr_selftest_bounded_wait", "gdr_status_string",
+EXPORTS = ("gdr_chunk_fwd", "gdr_chunk_fwd_grouped", "gdr_chunk_fwd_workspace_size",
+           "gdr_chunk_fwd_static", "gdr_chunk_fwd_static_capacity", "gdr_decode_step",
+           "gdr_decode_step_grouped", "gdr_selftest_bounded_wait", "gdr_status_string",
            "gdr_version")
 
 _lock = threading.Lock()
@@ -50,6 +51,10 @@ def load(build_if_missing: bool = True) -> ctypes.CDLL:
         sz = ctypes.c_size_t
         lib.gdr_chunk_fwd.argtypes = [vp] * 6 + [ip] * 3 + [vp, vp, vp, vp, sz] + [ip] * 7 + [vp, vp]
         lib.gdr_chunk_fwd.restype = ip
+        lib.gdr_chunk_fwd_grouped.argtypes = [vp] * 6 + [ip] * 3 + [vp, vp, vp, vp, sz] + [ip] * 8 + [vp, vp]
+        lib.gdr_chunk_fwd_grouped.restype = ip
+        lib.gdr_decode_step_grouped.argtypes = [vp] * 6 + [ip] * 3 + [vp, vp] + [ip] * 6 + [vp, vp]
+        lib.gdr_decode_step_grouped.restype = ip
         lib.gdr_chunk_fwd_workspace_size.argtypes = [ip] * 9
         lib.gdr_chunk_fwd_workspace_size.restype = sz
         lib.gdr_chunk_fwd_static.argtypes = [vp] * 6 + [ip] * 3 + [vp, vp, vp] + [ip] * 7 + [vp, vp]
@@ -96,6 +101,26 @@ def gdr_chunk_fwd(q, k, v, alpha, b, w, alpha_kind, b_kind, w_kind, S0, o, S_T, 
                               B, T, H, d_k, d_v, chunk, dtype, _p(d_status), _stream(stream))
     if st != GDR_OK:
         raise GdrError("gdr_chunk_fwd", st)
+
+
+def gdr_chunk_fwd_grouped(q, k, v, alpha, b, w, alpha_kind, b_kind, w_kind, S0, o, S_T, workspace,
+                          workspace_bytes, B, T, H_qk, H, d_k, d_v, chunk, dtype, d_status=None,
+                          stream=None) -> None:
+    st = load().gdr_chunk_fwd_grouped(_p(q), _p(k), _p(v), _p(alpha), _p(b), _p(w), alpha_kind,
+                                      b_kind, w_kind, _p(S0), _p(o), _p(S_T), _p(workspace),
+                                      int(workspace_bytes), B, T, H_qk, H, d_k, d_v, chunk, dtype,
+                                      _p(d_status), _stream(stream))
+    if st != GDR_OK:
+        raise GdrError("gdr_chunk_fwd_grouped", st)
+
+
+def gdr_decode_step_grouped(q, k, v, alpha, b, w, alpha_kind, b_kind, w_kind, S, o, B, H_qk, H,
+                            d_k, d_v, dtype, d_status=None, stream=None) -> None:
+    st = load().gdr_decode_step_grouped(_p(q), _p(k), _p(v), _p(alpha), _p(b), _p(w), alpha_kind,
+                                        b_kind, w_kind, _p(S), _p(o), B, H_qk, H, d_k, d_v, dtype,
+                                        _p(d_status), _stream(stream))
+    if st != GDR_OK:
+        raise GdrError("gdr_decode_step_grouped", st)
 
 
 def gdr_chunk_fwd_static(q, k, v, alpha, b, w, alpha_kind, b_kind, w_kind, S0, o, S_T, B, T, H,

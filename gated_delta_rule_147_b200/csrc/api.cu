@@ -10,19 +10,20 @@
 namespace gdr {
 cudaError_t launch_decode(const void* q, const void* k, const void* v, const void* a, const void* b,
                           const void* w, int ak, int bk, int wk, float* S, void* o, int BH, int dk,
-                          int dv, int dtype, cudaStream_t st);
+                          int dv, int dtype, int group, cudaStream_t st);
 int decode_rows_per_thread(int dk, int dv);
 cudaError_t launch_recurrent(const void* q, const void* k, const void* v, const void* a,
                              const void* b, const void* w, int ak, int bk, int wk, const float* S0,
                              void* o, float* ST, int B, int T, int H, int dk, int dv, int dtype,
-                             cudaStream_t st);
+                             int group, cudaStream_t st);
 cudaError_t launch_chunk_erasefree_sm100(const CUtensorMap* maps, const void* alpha, const void* w,
                                          int akind, int wkind, const float* S0, void* o, float* ST,
-                                         int* d_status, int B, int T, int H, int dv, cudaStream_t st);
+                                         int* d_status, int B, int T, int H, int dv, int group,
+                                         cudaStream_t st);
 size_t twopass_workspace_bytes(int B, int T, int H, int dv);
 cudaError_t launch_chunk_twopass_gdn(const CUtensorMap* maps, const CUtensorMap* ws_maps, void* ws,
                                      const void* alpha, const void* beta, const float* S0, void* o,
-                                     float* ST, int* d_status, int B, int T, int H, int dv,
+                                     float* ST, int* d_status, int B, int T, int H, int dv, int group,
                                      cudaStream_t st);
 size_t twopass_general_workspace_bytes(int B, int T, int H, int dv, bool untied);
 cudaError_t launch_chunk_twopass_general(const CUtensorMap* maps,
@@ -30,12 +31,12 @@ cudaError_t launch_chunk_twopass_general(const CUtensorMap* maps,
                                          void* ws, const void* q, const void* k, const void* alpha,
                                          const void* b, const void* w, int akind, int bkind,
                                          int wkind, const float* S0, void* o, float* ST,
-                                         int* d_status, int B, int T, int H, int dv,
+                                         int* d_status, int B, int T, int H, int dv, int group,
                                          cudaStream_t st);
 cudaError_t launch_chunk_sm100(const CUtensorMap* maps, const void* alpha, const void* b,
                                const void* w, int akind, int bkind, int wkind, bool tied,
                                const float* S0, void* o, float* ST, int* d_status, int B, int T,
-                               int H, int dv, cudaStream_t st);
+                               int H, int dv, int group, cudaStream_t st);
 }  // namespace gdr
 
 namespace {
@@ -129,12 +130,14 @@ const char* gdr_status_string(int s) {
 
 int gdr_version(void) { return (1 << 16) | 0; }
 
-gdr_status gdr_chunk_fwd(const void* q, const void* k, const void* v, const void* alpha,
-                         const void* b, const void* w, int alpha_kind, int b_kind, int w_kind,
-                         const float* S0, void* o, float* S_T, void* workspace,
-                         size_t workspace_bytes, int B, int T, int H, int d_k, int d_v, int chunk,
-                         int dtype, int* d_status, void* stream) {
+gdr_status gdr_chunk_fwd_grouped(const void* q, const void* k, const void* v, const void* alpha,
+                                 const void* b, const void* w, int alpha_kind, int b_kind,
+                                 int w_kind, const float* S0, void* o, float* S_T, void* workspace,
+                                 size_t workspace_bytes, int B, int T, int H_qk, int H, int d_k,
+                                 int d_v, int chunk, int dtype, int* d_status, void* stream) {
     if (B < 1 || H < 1 || T < 0 || d_k < 1 || d_v < 1) return GDR_ERR_INVALID_ARG;
+    if (H_qk < 1 || H % H_qk != 0) return GDR_ERR_INVALID_ARG;
+    const int group = H / H_qk;
     if (dtype != GDR_BF16 && dtype != GDR_FP32) return GDR_ERR_INVALID_ARG;
     if (!kind_ok(alpha_kind, false) || !kind_ok(b_kind, false) || !kind_ok(w_kind, true))
         return GDR_ERR_INVALID_ARG;
@@ -181,7 +184,7 @@ gdr_status gdr_chunk_fwd(const void* q, const void* k, const void* v, const void
         const void* amap = alpha_kind == GDR_GATE_CHANNEL ? alpha : q;
         const void* bmap = b_kind == GDR_GATE_CHANNEL ? b : q;
         const void* wmap = w_kind == GDR_GATE_CHANNEL ? w : q;
-        if (!make_map(&maps[0], q, B, T, H, d_k) || !make_map(&maps[1], k, B, T, H, d_k) ||
+        if (!make_map(&maps[0], q, B, T, H_qk, d_k) || !make_map(&maps[1], k, B, T, H_qk, d_k) ||
             !make_map(&maps[2], v, B, T, H, d_v) || !make_map(&maps[3], amap, B, T, H, d_k) ||
             !make_map(&maps[4], bmap, B, T, H, d_k) || !make_map(&maps[5], wmap, B, T, H, d_k))
             return GDR_ERR_INVALID_ARG;
@@ -189,7 +192,7 @@ gdr_status gdr_chunk_fwd(const void* q, const void* k, const void* v, const void
         if (tp == TP_GENERAL) {
             e = gdr::launch_chunk_twopass_general(maps, make_map, workspace, q, k, alpha, b, w,
                                                   alpha_kind, b_kind, w_kind, S0, o, S_T, d_status,
-                                                  B, T, H, d_v, st);
+                                                  B, T, H, d_v, group, st);
         } else if (tp == TP_GDN) {
             CUtensorMap ws_maps[2];
             const uint8_t* pbase = reinterpret_cast<const uint8_t*>(workspace) +
@@ -198,26 +201,37 @@ gdr_status gdr_chunk_fwd(const void* q, const void* k, const void* v, const void
                 !make_map(&ws_maps[1], pbase, B, T, H, d_v))
                 return GDR_ERR_INVALID_ARG;
             e = gdr::launch_chunk_twopass_gdn(maps, ws_maps, workspace, alpha, b, S0, o, S_T,
-                                              d_status, B, T, H, d_v, st);
+                                              d_status, B, T, H, d_v, group, st);
         } else if (b_kind == GDR_GATE_NONE)  // no erase: no triangular solve
             e = gdr::launch_chunk_erasefree_sm100(maps, alpha, w, alpha_kind, w_kind, S0, o, S_T,
-                                                  d_status, B, T, H, d_v, st);
+                                                  d_status, B, T, H, d_v, group, st);
         else
             e = gdr::launch_chunk_sm100(maps, alpha, b, w, alpha_kind, b_kind, w_kind, tied, S0, o,
-                                        S_T, d_status, B, T, H, d_v, st);
+                                        S_T, d_status, B, T, H, d_v, group, st);
     } else {
         e = gdr::launch_recurrent(q, k, v, alpha, b, w, alpha_kind, b_kind, w_kind, S0, o, S_T, B,
-                                  T, H, d_k, d_v, dtype, st);
+                                  T, H, d_k, d_v, dtype, group, st);
     }
     return e == cudaSuccess ? GDR_OK : GDR_ERR_LAUNCH;
 }
 
-gdr_status gdr_decode_step(const void* q, const void* k, const void* v, const void* alpha,
-                           const void* b, const void* w, int alpha_kind, int b_kind, int w_kind,
-                           float* S, void* o, int B, int H, int d_k, int d_v, int dtype,
-                           int* d_status, void* stream) {
+gdr_status gdr_chunk_fwd(const void* q, const void* k, const void* v, const void* alpha,
+                         const void* b, const void* w, int alpha_kind, int b_kind, int w_kind,
+                         const float* S0, void* o, float* S_T, void* workspace,
+                         size_t workspace_bytes, int B, int T, int H, int d_k, int d_v, int chunk,
+                         int dtype, int* d_status, void* stream) {
+    return gdr_chunk_fwd_grouped(q, k, v, alpha, b, w, alpha_kind, b_kind, w_kind, S0, o, S_T,
+                                 workspace, workspace_bytes, B, T, H, H, d_k, d_v, chunk, dtype,
+                                 d_status, stream);
+}
+
+gdr_status gdr_decode_step_grouped(const void* q, const void* k, const void* v, const void* alpha,
+                                   const void* b, const void* w, int alpha_kind, int b_kind,
+                                   int w_kind, float* S, void* o, int B, int H_qk, int H, int d_k,
+                                   int d_v, int dtype, int* d_status, void* stream) {
     (void)d_status;  // the decode kernel has no bounded waits
     if (B < 1 || H < 1 || d_k < 1 || d_v < 1) return GDR_ERR_INVALID_ARG;
+    if (H_qk < 1 || H % H_qk != 0) return GDR_ERR_INVALID_ARG;
     if (dtype != GDR_BF16 && dtype != GDR_FP32) return GDR_ERR_INVALID_ARG;
     if (!kind_ok(alpha_kind, false) || !kind_ok(b_kind, false) || !kind_ok(w_kind, true))
         return GDR_ERR_INVALID_ARG;
@@ -231,8 +245,16 @@ gdr_status gdr_decode_step(const void* q, const void* k, const void* v, const vo
     if (!aligned16(S) || !aligned16(o) || !aligned16(q) || !aligned16(k) || !aligned16(v))
         return GDR_ERR_MISALIGNED;
     cudaError_t e = gdr::launch_decode(q, k, v, alpha, b, w, alpha_kind, b_kind, w_kind, S, o, B * H,
-                                       d_k, d_v, dtype, reinterpret_cast<cudaStream_t>(stream));
+                                       d_k, d_v, dtype, H / H_qk, reinterpret_cast<cudaStream_t>(stream));
     return e == cudaSuccess ? GDR_OK : GDR_ERR_LAUNCH;
+}
+
+gdr_status gdr_decode_step(const void* q, const void* k, const void* v, const void* alpha,
+                           const void* b, const void* w, int alpha_kind, int b_kind, int w_kind,
+                           float* S, void* o, int B, int H, int d_k, int d_v, int dtype,
+                           int* d_status, void* stream) {
+    return gdr_decode_step_grouped(q, k, v, alpha, b, w, alpha_kind, b_kind, w_kind, S, o, B, H, H,
+                                   d_k, d_v, dtype, d_status, stream);
 }
 
 }  // extern "C"

@@ -22,6 +22,7 @@ struct Params {
     int* d_status;
     int B, T, H, dv;
     int akind, bkind, wkind;
+    int group;  // value heads per q/k head: q, k have H / group heads, read at h / group
 };
 
 __device__ __forceinline__ void st_chunk(uint8_t* base, uint32_t off, const float* x8) {

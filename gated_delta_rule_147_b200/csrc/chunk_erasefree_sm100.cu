@@ -81,10 +81,10 @@ __global__ void __launch_bounds__(NT, 1) chunk_fwd_erasefree_kernel(
     auto issue_loads = [&](int ci) {
         const int t0 = ci * C;
         mbar_expect_tx(bar_tma, (uint32_t)(5 + 2 * (ACH + wch)) * 8192u);
-        tma_load_4d(sm + OFF_QIN, &tm_q, bar_tma, 0, h, t0, bb);
-        tma_load_4d(sm + OFF_QIN + 8192, &tm_q, bar_tma, 64, h, t0, bb);
-        tma_load_4d(sm + OFF_KIN, &tm_k, bar_tma, 0, h, t0, bb);
-        tma_load_4d(sm + OFF_KIN + 8192, &tm_k, bar_tma, 64, h, t0, bb);
+        tma_load_4d(sm + OFF_QIN, &tm_q, bar_tma, 0, h / p.group, t0, bb);
+        tma_load_4d(sm + OFF_QIN + 8192, &tm_q, bar_tma, 64, h / p.group, t0, bb);
+        tma_load_4d(sm + OFF_KIN, &tm_k, bar_tma, 0, h / p.group, t0, bb);
+        tma_load_4d(sm + OFF_KIN + 8192, &tm_k, bar_tma, 64, h / p.group, t0, bb);
         tma_load_4d(sm + OFF_V + (ci & 1) * 8192, &tm_v, bar_tma, v0, h, t0, bb);
         if (ACH) {
             tma_load_4d(sm + OFF_GA, &tm_a, bar_tma, 0, h, t0, bb);
@@ -390,12 +390,14 @@ finish:
 // maps: q, k, v, alpha (channel) or q, w (channel) or q
 cudaError_t launch_chunk_erasefree_sm100(const CUtensorMap* maps, const void* alpha, const void* w,
                                          int akind, int wkind, const float* S0, void* o, float* ST,
-                                         int* d_status, int B, int T, int H, int dv, cudaStream_t st) {
+                                         int* d_status, int B, int T, int H, int dv, int group,
+                                         cudaStream_t st) {
     chunkc::Params p;
     p.alpha = alpha; p.bg = nullptr; p.wg = w;
     p.S0 = S0; p.o = (__nv_bfloat16*)o; p.ST = ST; p.d_status = d_status;
     p.B = B; p.T = T; p.H = H; p.dv = dv;
     p.akind = akind; p.bkind = GDR_GATE_NONE; p.wkind = wkind;
+    p.group = group;
     dim3 grid(dv / chunkc::NV, H, B);
     auto launch = [&](auto kern) -> cudaError_t {
         cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, erasefree::SMEM_BYTES);

@@ -139,10 +139,10 @@ __global__ void __launch_bounds__(NT, 1) chunk_fwd_kernel(
         const int t0 = ci * C;
         const uint32_t bytes = (uint32_t)(4 + 1 + 2 * (ach + bch + wch)) * 8192u;
         mbar_expect_tx(bar_tma, bytes);
-        tma_load_4d(sm + OFF_QIN, &tm_q, bar_tma, 0, h, t0, bb);
-        tma_load_4d(sm + OFF_QIN + 8192, &tm_q, bar_tma, 64, h, t0, bb);
-        tma_load_4d(sm + OFF_KIN, &tm_k, bar_tma, 0, h, t0, bb);
-        tma_load_4d(sm + OFF_KIN + 8192, &tm_k, bar_tma, 64, h, t0, bb);
+        tma_load_4d(sm + OFF_QIN, &tm_q, bar_tma, 0, h / p.group, t0, bb);
+        tma_load_4d(sm + OFF_QIN + 8192, &tm_q, bar_tma, 64, h / p.group, t0, bb);
+        tma_load_4d(sm + OFF_KIN, &tm_k, bar_tma, 0, h / p.group, t0, bb);
+        tma_load_4d(sm + OFF_KIN + 8192, &tm_k, bar_tma, 64, h / p.group, t0, bb);
         tma_load_4d(sm + OFF_V + (ci & 1) * 8192, &tm_v, bar_tma, v0, h, t0, bb);
         if (ach) {
             tma_load_4d(sm + OFF_GA, &tm_a, bar_tma, 0, h, t0, bb);
@@ -763,12 +763,12 @@ __global__ void __launch_bounds__(NT, 1) chunk_fwd_gdn_kernel(
         uint8_t* k2 = sm + gdn::OFF_K2 + buf * 16384;
         mbar_expect_tx(&bar_tma[buf], 7u * 8192u);
         // [K ; Q]: each 64-column block holds 128 rows (k rows 0..63, q rows 64..127)
-        tma_load_4d(qk, &tm_k, &bar_tma[buf], 0, h, t0, bb);
-        tma_load_4d(qk + 16384, &tm_k, &bar_tma[buf], 64, h, t0, bb);
-        tma_load_4d(qk + 8192, &tm_q, &bar_tma[buf], 0, h, t0, bb);
-        tma_load_4d(qk + 16384 + 8192, &tm_q, &bar_tma[buf], 64, h, t0, bb);
-        tma_load_4d(k2, &tm_k, &bar_tma[buf], 0, h, t0, bb);
-        tma_load_4d(k2 + 8192, &tm_k, &bar_tma[buf], 64, h, t0, bb);
+        tma_load_4d(qk, &tm_k, &bar_tma[buf], 0, h / p.group, t0, bb);
+        tma_load_4d(qk + 16384, &tm_k, &bar_tma[buf], 64, h / p.group, t0, bb);
+        tma_load_4d(qk + 8192, &tm_q, &bar_tma[buf], 0, h / p.group, t0, bb);
+        tma_load_4d(qk + 16384 + 8192, &tm_q, &bar_tma[buf], 64, h / p.group, t0, bb);
+        tma_load_4d(k2, &tm_k, &bar_tma[buf], 0, h / p.group, t0, bb);
+        tma_load_4d(k2 + 8192, &tm_k, &bar_tma[buf], 64, h / p.group, t0, bb);
         tma_load_4d(sm + gdn::OFF_V + buf * 8192, &tm_v, &bar_tma[buf], v0, h, t0, bb);
     };
 
@@ -1145,12 +1145,13 @@ finish:
 cudaError_t launch_chunk_sm100(const CUtensorMap* maps, const void* alpha, const void* b,
                                const void* w, int akind, int bkind, int wkind, bool tied,
                                const float* S0, void* o, float* ST, int* d_status, int B, int T,
-                               int H, int dv, cudaStream_t st) {
+                               int H, int dv, int group, cudaStream_t st) {
     chunk::Params p;
     p.alpha = alpha; p.bg = b; p.wg = w;
     p.S0 = S0; p.o = (__nv_bfloat16*)o; p.ST = ST; p.d_status = d_status;
     p.B = B; p.T = T; p.H = H; p.dv = dv;
     p.akind = akind; p.bkind = bkind; p.wkind = wkind;
+    p.group = group;
     dim3 grid(dv / chunk::NV, H, B);
     const bool ach = akind == GDR_GATE_CHANNEL;
     auto launch = [&](auto kern) -> cudaError_t {

@@ -73,6 +73,7 @@ struct GPrepParams {
     float* gc;                                        // [B, H, nchunks, 128]
     int* d_status;
     int T, H, dv, akind, bkind, wkind;
+    int group;  // value heads per q/k head (q, k read at token-head index / group)
 };
 
 __device__ __forceinline__ void ld8b(const __nv_bfloat16* p, uint2& u) {
@@ -144,9 +145,10 @@ __global__ void __launch_bounds__(NT, 2) prep_general_kernel(
     uint2 qa[4], ka[4], ba[4], wa[4];
     auto load_token = [&](int i) {
         const size_t e = elem(rg * 8 + i);
+        const size_t eq = (e / DK) / pp.group * DK + ch0;  // q, k row of this value head
         const int sl = i & 3;
-        ld8b(pp.q + e, qa[sl]);
-        ld8b(pp.k + e, ka[sl]);
+        ld8b(pp.q + eq, qa[sl]);
+        ld8b(pp.k + eq, ka[sl]);
         if (bch) ld8b(pp.bg + e, ba[sl]);
         if (!TIED && wch) ld8b(pp.wg + e, wa[sl]);
     };
@@ -919,7 +921,7 @@ cudaError_t launch_chunk_twopass_general(const CUtensorMap* maps, MapFn make_map
                                          const void* q, const void* k, const void* alpha,
                                          const void* b, const void* w, int akind, int bkind,
                                          int wkind, const float* S0, void* o, float* ST,
-                                         int* d_status, int B, int T, int H, int dv,
+                                         int* d_status, int B, int T, int H, int dv, int group,
                                          cudaStream_t st) {
     using namespace twopass_g;
     const bool tied = wkind == GDR_GATE_TIED && bkind == GDR_GATE_SCALAR;
@@ -940,6 +942,7 @@ cudaError_t launch_chunk_twopass_general(const CUtensorMap* maps, MapFn make_map
     pp.d_status = d_status;
     pp.T = T; pp.H = H; pp.dv = dv;
     pp.akind = akind; pp.bkind = bkind; pp.wkind = wkind;
+    pp.group = group;
     CUtensorMap sm_maps[8];
     const int dims[7] = {128, 128, 128, 64, dv, 128, 64};
     for (int i = 0; i < 7; ++i) {

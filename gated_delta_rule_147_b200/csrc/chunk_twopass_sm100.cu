@@ -77,6 +77,7 @@ struct PrepParams {
     const void* beta;
     int* d_status;
     int T, H, dv, nitems;
+    int group;  // value heads per k head (k read at head h / group)
 };
 
 __global__ void __launch_bounds__(NT, 2) prep_gdn_kernel(const __grid_constant__ CUtensorMap tm_k,
@@ -113,8 +114,8 @@ __global__ void __launch_bounds__(NT, 2) prep_gdn_kernel(const __grid_constant__
         coords(item, ci, h, bb);
         const int t0 = ci * C;
         mbar_expect_tx(&bar_tma[buf], (uint32_t)(2 + nvt) * 8192u);
-        tma_load_4d(sm + P_OFF_K + buf * 16384, &tm_k, &bar_tma[buf], 0, h, t0, bb);
-        tma_load_4d(sm + P_OFF_K + buf * 16384 + 8192, &tm_k, &bar_tma[buf], 64, h, t0, bb);
+        tma_load_4d(sm + P_OFF_K + buf * 16384, &tm_k, &bar_tma[buf], 0, h / pp.group, t0, bb);
+        tma_load_4d(sm + P_OFF_K + buf * 16384 + 8192, &tm_k, &bar_tma[buf], 64, h / pp.group, t0, bb);
         for (int vt = 0; vt < nvt; ++vt)
             tma_load_4d(sm + P_OFF_V + buf * 16384 + vt * 8192, &tm_v, &bar_tma[buf], vt * 64, h, t0, bb);
     };
@@ -427,10 +428,10 @@ __global__ void __launch_bounds__(NT, 1) state_gdn_kernel(
         // [-W ; Q]: each 64-column block holds 128 rows (-W rows 0..63, q rows 64..127)
         tma_load_4d(wq, &tm_w, &bar_tma[buf], 0, h, t0, bb);
         tma_load_4d(wq + 16384, &tm_w, &bar_tma[buf], 64, h, t0, bb);
-        tma_load_4d(wq + 8192, &tm_q, &bar_tma[buf], 0, h, t0, bb);
-        tma_load_4d(wq + 16384 + 8192, &tm_q, &bar_tma[buf], 64, h, t0, bb);
-        tma_load_4d(kk, &tm_k, &bar_tma[buf], 0, h, t0, bb);
-        tma_load_4d(kk + 8192, &tm_k, &bar_tma[buf], 64, h, t0, bb);
+        tma_load_4d(wq + 8192, &tm_q, &bar_tma[buf], 0, h / p.group, t0, bb);
+        tma_load_4d(wq + 16384 + 8192, &tm_q, &bar_tma[buf], 64, h / p.group, t0, bb);
+        tma_load_4d(kk, &tm_k, &bar_tma[buf], 0, h / p.group, t0, bb);
+        tma_load_4d(kk + 8192, &tm_k, &bar_tma[buf], 64, h / p.group, t0, bb);
         tma_load_4d(sm + S_OFF_P + buf * 8192, &tm_p, &bar_tma[buf], v0, h, t0, bb);
     };
 
@@ -714,13 +715,14 @@ size_t twopass_workspace_bytes(int B, int T, int H, int dv) {
 // maps: q, k, v, then the workspace maps -W ([B,T,H,128]) and P ([B,T,H,d_v]).
 cudaError_t launch_chunk_twopass_gdn(const CUtensorMap* maps, const CUtensorMap* ws_maps, void* ws,
                                      const void* alpha, const void* beta, const float* S0, void* o,
-                                     float* ST, int* d_status, int B, int T, int H, int dv,
+                                     float* ST, int* d_status, int B, int T, int H, int dv, int group,
                                      cudaStream_t st) {
     using namespace twopass;
     PrepParams pp;
     pp.alpha = alpha; pp.beta = beta;
     pp.d_status = d_status;
     pp.T = T; pp.H = H; pp.dv = dv;
+    pp.group = group;
     const int nchunks = (T + C - 1) / C;
     pp.nitems = nchunks * H * B;
     cudaError_t e = cudaFuncSetAttribute(prep_gdn_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, P_SMEM_BYTES);
@@ -738,6 +740,7 @@ cudaError_t launch_chunk_twopass_gdn(const CUtensorMap* maps, const CUtensorMap*
     p.S0 = S0; p.o = (__nv_bfloat16*)o; p.ST = ST; p.d_status = d_status;
     p.B = B; p.T = T; p.H = H; p.dv = dv;
     p.akind = GDR_GATE_SCALAR; p.bkind = GDR_GATE_SCALAR; p.wkind = GDR_GATE_TIED;
+    p.group = group;
     e = cudaFuncSetAttribute(state_gdn_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, S_SMEM_BYTES);
     if (e != cudaSuccess) return e;
     state_gdn_kernel<<<dim3(dv / NV, H, B), NT, S_SMEM_BYTES, st>>>(maps[0], maps[1], ws_maps[0], ws_maps[1], p);

@@ -18,7 +18,7 @@ template <typename TI, int DV, int NR>
 __global__ void __launch_bounds__(256) decode_step_kernel(
     const TI* __restrict__ q, const TI* __restrict__ k, const TI* __restrict__ v,
     const TI* __restrict__ alpha, const TI* __restrict__ bg, const TI* __restrict__ wg, int akind,
-    int bkind, int wkind, float* __restrict__ S, TI* __restrict__ o, int dk) {
+    int bkind, int wkind, float* __restrict__ S, TI* __restrict__ o, int dk, int group) {
     constexpr int TPR = DV / 4;
     constexpr int RPP = 256 / TPR;
     const int bh = blockIdx.x;
@@ -28,9 +28,10 @@ __global__ void __launch_bounds__(256) decode_step_kernel(
     __shared__ float4 s_red[2][RPP][TPR];
     __shared__ float s_dots[2];
 
+    const size_t bhq = (size_t)(bh / group);  // q, k have H / group heads
     for (int i = tid; i < dk; i += 256) {
         const size_t gi = (size_t)bh * dk + i;
-        float ki = to_f32(k[gi]), qi = to_f32(q[gi]);
+        float ki = to_f32(k[bhq * dk + i]), qi = to_f32(q[bhq * dk + i]);
         float a = akind == GDR_GATE_NONE ? 1.f
                   : akind == GDR_GATE_SCALAR ? to_f32(alpha[bh]) : to_f32(alpha[gi]);
         float bb = bkind == GDR_GATE_NONE ? 0.f
@@ -49,7 +50,7 @@ __global__ void __launch_bounds__(256) decode_step_kernel(
     if (tid < 32) {
         float d1 = 0.f, d2 = 0.f;
         for (int i = tid; i < dk; i += 32) {
-            float qi = to_f32(q[(size_t)bh * dk + i]);
+            float qi = to_f32(q[bhq * dk + i]);
             d1 += qi * s_k[i];
             d2 += qi * s_wk[i];
         }
@@ -125,13 +126,13 @@ __global__ void __launch_bounds__(256) decode_step_kernel(
 template <typename TI, int DV>
 static cudaError_t launch_decode_dv(const void* q, const void* k, const void* v, const void* a,
                                     const void* b, const void* w, int ak, int bk, int wk, float* S,
-                                    void* o, int BH, int dk, cudaStream_t st) {
+                                    void* o, int BH, int dk, int group, cudaStream_t st) {
     constexpr int RPP = 256 / (DV / 4);
     const int nr = (dk + RPP - 1) / RPP;
 #define GDR_DEC(NRV)                                                                              \
     decode_step_kernel<TI, DV, NRV><<<BH, 256, 0, st>>>(                                          \
         (const TI*)q, (const TI*)k, (const TI*)v, (const TI*)a, (const TI*)b, (const TI*)w, ak, bk, \
-        wk, S, (TI*)o, dk)
+        wk, S, (TI*)o, dk, group)
     if (nr <= 4) GDR_DEC(4);
     else if (nr <= 8) GDR_DEC(8);
     else if (nr <= 16) GDR_DEC(16);
@@ -150,23 +151,23 @@ int decode_rows_per_thread(int dk, int dv) {
 template <typename TI>
 static cudaError_t launch_decode_t(const void* q, const void* k, const void* v, const void* a,
                                    const void* b, const void* w, int ak, int bk, int wk, float* S,
-                                   void* o, int BH, int dk, int dv, cudaStream_t st) {
+                                   void* o, int BH, int dk, int dv, int group, cudaStream_t st) {
     switch (dv) {
-        case 16: return launch_decode_dv<TI, 16>(q, k, v, a, b, w, ak, bk, wk, S, o, BH, dk, st);
-        case 32: return launch_decode_dv<TI, 32>(q, k, v, a, b, w, ak, bk, wk, S, o, BH, dk, st);
-        case 64: return launch_decode_dv<TI, 64>(q, k, v, a, b, w, ak, bk, wk, S, o, BH, dk, st);
-        case 128: return launch_decode_dv<TI, 128>(q, k, v, a, b, w, ak, bk, wk, S, o, BH, dk, st);
-        case 256: return launch_decode_dv<TI, 256>(q, k, v, a, b, w, ak, bk, wk, S, o, BH, dk, st);
+        case 16: return launch_decode_dv<TI, 16>(q, k, v, a, b, w, ak, bk, wk, S, o, BH, dk, group, st);
+        case 32: return launch_decode_dv<TI, 32>(q, k, v, a, b, w, ak, bk, wk, S, o, BH, dk, group, st);
+        case 64: return launch_decode_dv<TI, 64>(q, k, v, a, b, w, ak, bk, wk, S, o, BH, dk, group, st);
+        case 128: return launch_decode_dv<TI, 128>(q, k, v, a, b, w, ak, bk, wk, S, o, BH, dk, group, st);
+        case 256: return launch_decode_dv<TI, 256>(q, k, v, a, b, w, ak, bk, wk, S, o, BH, dk, group, st);
         default: return cudaErrorInvalidValue;
     }
 }
 
 cudaError_t launch_decode(const void* q, const void* k, const void* v, const void* a, const void* b,
                           const void* w, int ak, int bk, int wk, float* S, void* o, int BH, int dk,
-                          int dv, int dtype, cudaStream_t st) {
+                          int dv, int dtype, int group, cudaStream_t st) {
     if (dtype == GDR_BF16)
-        return launch_decode_t<__nv_bfloat16>(q, k, v, a, b, w, ak, bk, wk, S, o, BH, dk, dv, st);
-    return launch_decode_t<float>(q, k, v, a, b, w, ak, bk, wk, S, o, BH, dk, dv, st);
+        return launch_decode_t<__nv_bfloat16>(q, k, v, a, b, w, ak, bk, wk, S, o, BH, dk, dv, group, st);
+    return launch_decode_t<float>(q, k, v, a, b, w, ak, bk, wk, S, o, BH, dk, dv, group, st);
 }
 
 }  // namespace gdr

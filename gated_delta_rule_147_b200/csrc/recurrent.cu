@@ -20,7 +20,7 @@ __global__ void __launch_bounds__(kRecCols) recurrent_fwd_kernel(
     const TI* __restrict__ q, const TI* __restrict__ k, const TI* __restrict__ v,
     const TI* __restrict__ alpha, const TI* __restrict__ bg, const TI* __restrict__ wg, int akind,
     int bkind, int wkind, const float* __restrict__ S0, TI* __restrict__ o, float* __restrict__ ST,
-    int T, int H, int dk, int dv) {
+    int T, int H, int dk, int dv, int group) {
     const int b = blockIdx.z, h = blockIdx.y;
     const int j = blockIdx.x * kRecCols + threadIdx.x;
     const bool col_ok = j < dv;
@@ -36,9 +36,11 @@ __global__ void __launch_bounds__(kRecCols) recurrent_fwd_kernel(
     for (int t = 0; t < T; ++t) {
         const int buf = t & 1;
         const size_t tok = ((size_t)b * T + t) * H + h;
+        const size_t tokq = tok / group;  // q, k have H / group heads
         for (int i = threadIdx.x; i < dk; i += kRecCols) {
             const size_t gi = tok * dk + i;
-            float ki = to_f32(k[gi]);
+            const size_t qi = tokq * dk + i;
+            float ki = to_f32(k[qi]);
             float a = akind == GDR_GATE_NONE ? 1.f
                       : akind == GDR_GATE_SCALAR ? to_f32(alpha[tok]) : to_f32(alpha[gi]);
             float bb = bkind == GDR_GATE_NONE ? 0.f
@@ -50,7 +52,7 @@ __global__ void __launch_bounds__(kRecCols) recurrent_fwd_kernel(
             s_bk[buf][i] = bb * ki;
             s_k[buf][i] = ki;
             s_wk[buf][i] = ww * ki;
-            s_q[buf][i] = to_f32(q[gi]);
+            s_q[buf][i] = to_f32(q[qi]);
         }
         __syncthreads();  // double buffering makes one barrier per token enough
         const float vj = col_ok ? to_f32(v[tok * dv + j]) : 0.f;
@@ -82,17 +84,17 @@ __global__ void __launch_bounds__(kRecCols) recurrent_fwd_kernel(
 cudaError_t launch_recurrent(const void* q, const void* k, const void* v, const void* a,
                              const void* b, const void* w, int ak, int bk, int wk, const float* S0,
                              void* o, float* ST, int B, int T, int H, int dk, int dv, int dtype,
-                             cudaStream_t st) {
+                             int group, cudaStream_t st) {
     dim3 grid((dv + kRecCols - 1) / kRecCols, H, B);
     if (dtype == GDR_BF16)
         recurrent_fwd_kernel<__nv_bfloat16><<<grid, kRecCols, 0, st>>>(
             (const __nv_bfloat16*)q, (const __nv_bfloat16*)k, (const __nv_bfloat16*)v,
             (const __nv_bfloat16*)a, (const __nv_bfloat16*)b, (const __nv_bfloat16*)w, ak, bk, wk,
-            S0, (__nv_bfloat16*)o, ST, T, H, dk, dv);
+            S0, (__nv_bfloat16*)o, ST, T, H, dk, dv, group);
     else
         recurrent_fwd_kernel<float><<<grid, kRecCols, 0, st>>>(
             (const float*)q, (const float*)k, (const float*)v, (const float*)a, (const float*)b,
-            (const float*)w, ak, bk, wk, S0, (float*)o, ST, T, H, dk, dv);
+            (const float*)w, ak, bk, wk, S0, (float*)o, ST, T, H, dk, dv, group);
     return cudaGetLastError();
 }
 

@@ -129,6 +129,24 @@ gdr_status gdr_chunk_fwd(const void* q, const void* k, const void* v,
                          int dtype, int* d_status, void* stream);
 
 /*
+ * gdr_chunk_fwd_grouped -- gdr_chunk_fwd with grouped query/key heads
+ * ("How Linear Attention Remembers", Table 1: 16 q/k heads serving 32 value
+ * heads). q and k are [B, T, H_qk, d_k]; v, o, the gates and the states have
+ * H heads, and value head h reads q/k head h / (H / H_qk), so consecutive
+ * value heads share one q/k head. Everything else is as gdr_chunk_fwd, which
+ * is this call with H_qk = H; the workspace size does not depend on H_qk.
+ * Returns GDR_ERR_INVALID_ARG also when H_qk < 1 or H is not a multiple of
+ * H_qk.
+ */
+gdr_status gdr_chunk_fwd_grouped(const void* q, const void* k, const void* v,
+                                 const void* alpha, const void* b, const void* w,
+                                 int alpha_kind, int b_kind, int w_kind,
+                                 const float* S0, void* o, float* S_T,
+                                 void* workspace, size_t workspace_bytes,
+                                 int B, int T, int H_qk, int H, int d_k, int d_v,
+                                 int chunk, int dtype, int* d_status, void* stream);
+
+/*
  * gdr_chunk_fwd_workspace_size -- bytes of scratch gdr_chunk_fwd's two-pass
  * path needs for this shape and gate form, or 0 when it has none. Two-pass
  * shapes: dtype GDR_BF16, d_k = 128, d_v in {64, 128}, T >= 1, an erase gate
@@ -199,6 +217,19 @@ gdr_status gdr_decode_step(const void* q, const void* k, const void* v,
                            int alpha_kind, int b_kind, int w_kind,
                            float* S, void* o, int B, int H, int d_k, int d_v,
                            int dtype, int* d_status, void* stream);
+
+/*
+ * gdr_decode_step_grouped -- gdr_decode_step with grouped query/key heads:
+ * q, k are [B, H_qk, d_k], v, o, gates and S have H heads, value head h reads
+ * q/k head h / (H / H_qk). gdr_decode_step is this call with H_qk = H.
+ * Returns GDR_ERR_INVALID_ARG also when H_qk < 1 or H % H_qk != 0.
+ */
+gdr_status gdr_decode_step_grouped(const void* q, const void* k, const void* v,
+                                   const void* alpha, const void* b, const void* w,
+                                   int alpha_kind, int b_kind, int w_kind,
+                                   float* S, void* o, int B, int H_qk, int H,
+                                   int d_k, int d_v, int dtype, int* d_status,
+                                   void* stream);
 
 /*
  * gdr_selftest_bounded_wait -- diagnostic for the kernels' bounded waits.

@@ -118,3 +118,16 @@ def test_binding_raises_on_error_status():
 def test_workspace_size(shape, kinds, expect):
     B, T, H, dk, dv = shape
     assert _lib.gdr_chunk_fwd_workspace_size(B, T, H, dk, dv, *kinds, 0) == expect
+
+
+def test_grouped_entry_points_reject_bad_head_counts():
+    lib = _lib.load()
+    st = lib.gdr_chunk_fwd_grouped(P, P, P, P, P, None, 1, 1, 3, None, P, P, None, 0,
+                                   1, 64, 3, 4, 128, 128, 64, 0, None, None)   # 4 % 3 != 0
+    assert st == _lib.GDR_ERR_INVALID_ARG
+    st = lib.gdr_chunk_fwd_grouped(P, P, P, P, P, None, 1, 1, 3, None, P, P, None, 0,
+                                   1, 64, 0, 4, 128, 128, 64, 0, None, None)   # H_qk = 0
+    assert st == _lib.GDR_ERR_INVALID_ARG
+    st = lib.gdr_decode_step_grouped(P, P, P, P, P, P, 2, 2, 2, P, P, 2, 3, 4, 128, 128, 0,
+                                     None, None)
+    assert st == _lib.GDR_ERR_INVALID_ARG

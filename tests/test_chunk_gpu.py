@@ -253,3 +253,53 @@ def test_two_pass_segmented_state_pass(cuda_device, family, T):
     assert_close(o2, o_ref, TOL["bf16"], "o (segmented two-pass)")
     assert_close(S2, ST_ref, TOL["bf16"], "S_T (segmented two-pass)")
     assert_close(o2, o1, 2e-2, "o two-pass vs single pass")
+
+
+# ---- grouped q/k heads ------------------------------------------------------
+
+def _expand_heads(x, group):
+    """q or k with H_qk heads -> H = H_qk * group heads (value head h reads h // group)."""
+    return None if x is None else x.repeat_interleave(group, dim=2).contiguous()
+
+
+@pytest.mark.parametrize("family,dv,workspace", [
+    ("gdn", 128, "auto"), ("kda", 128, "auto"), ("gdn2", 64, "auto"),   # two-pass paths
+    ("gdn", 128, None), ("kda", 64, None), ("gdn2", 128, None),         # single-pass kernels
+    ("gla", 256, "auto"),                                               # erase-free kernel
+])
+def test_grouped_heads_equal_expanded_heads(cuda_device, family, dv, workspace):
+    """16 q/k heads for 32 value heads in small: H_qk = 2, H = 4. The grouped
+    call reads q/k head h // 2 and must equal, bit for bit, the ungrouped call
+    with q, k repeated per value head (same kernels, same data); the result
+    is also checked against the oracle."""
+    wl = WORKLOADS[family].with_(B=2, H=4, T=150, dv=dv, s0=True, seed=77)
+    inp = make_chunk_inputs(wl)
+    dev = cuda_device
+    qg = inp["q"][:, :, ::2].contiguous()     # H_qk = 2 q/k heads
+    kg = inp["k"][:, :, ::2].contiguous()
+    full = dict(inp, q=_expand_heads(qg, 2), k=_expand_heads(kg, 2))
+    o_ref_dev, S_ref_dev = run_chunk(full, dev, workspace=workspace)
+    w = TIED if inp["gates"]["w"] == "tied" else (None if inp["w"] is None else inp["w"].to(dev))
+    a = None if inp["alpha"] is None else inp["alpha"].to(dev)
+    b = None if inp["b"] is None else inp["b"].to(dev)
+    s0 = None if inp["S0"] is None else inp["S0"].to(dev)
+    o, ST = chunk_fwd(qg.to(dev), kg.to(dev), inp["v"].to(dev), a, b, w, s0, workspace=workspace)
+    torch.cuda.synchronize()
+    assert torch.equal(o.cpu().view(torch.int16), torch.from_numpy(o_ref_dev).to(o.dtype).view(torch.int16))
+    assert np.array_equal(ST.cpu().numpy(), S_ref_dev)
+    o_or, S_or = run_oracle(full)
+    assert_close(o.float().cpu().numpy(), o_or, TOL["bf16"], "o (grouped)")
+    assert_close(ST.cpu().numpy(), S_or, TOL["bf16"], "S_T (grouped)")
+
+
+def test_grouped_heads_fp32_exact_path(cuda_device):
+    wl = WORKLOADS["kda"].with_(B=1, H=4, T=70, dtype="fp32", s0=True, seed=78)
+    inp = make_chunk_inputs(wl)
+    dev = cuda_device
+    qg, kg = inp["q"][:, :, ::2].contiguous(), inp["k"][:, :, ::2].contiguous()
+    full = dict(inp, q=_expand_heads(qg, 2), k=_expand_heads(kg, 2))
+    o_ref, S_ref = run_chunk(full, dev)
+    o, ST = chunk_fwd(qg.to(dev), kg.to(dev), inp["v"].to(dev), inp["alpha"].to(dev),
+                      inp["b"].to(dev), TIED, inp["S0"].to(dev))
+    torch.cuda.synchronize()
+    assert np.array_equal(o.cpu().numpy(), o_ref) and np.array_equal(ST.cpu().numpy(), S_ref)

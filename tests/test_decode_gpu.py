@@ -6,7 +6,7 @@ import torch
 
 import oracle
 from gated_delta_rule_147_b200 import TIED, decode_step
-from gated_delta_rule_147_b200.inputs import DECODE, make_decode_state, make_decode_steps
+from gated_delta_rule_147_b200.inputs import DECODE, DecodeWorkload, make_decode_state, make_decode_step, make_decode_steps
 from gpu_util import TOL, assert_close
 
 pytestmark = pytest.mark.gpu
@@ -108,3 +108,21 @@ def test_prefill_then_decode_continues_the_sequence(cuda_device, family):
                         w_t, S)
         torch.cuda.synchronize()
         assert_close(o.float().cpu().numpy(), o_ref[:, t], TOL["bf16"], f"decode token {t}")
+
+
+def test_grouped_decode_equals_expanded(cuda_device):
+    """Grouped q/k heads (H_qk = 2 for H = 4): equal, bit for bit, to the
+    ungrouped step with q, k repeated per value head."""
+    from gated_delta_rule_147_b200 import decode_step
+    dw = DecodeWorkload(B=3, H=4, steps=1, seed=31)
+    dev = cuda_device
+    S1 = make_decode_state(dw).to(dev)
+    S2 = S1.clone()
+    st = {k: v.to(dev) for k, v in make_decode_step(dw, 0).items()}
+    qg, kg = st["q"][:, ::2].contiguous(), st["k"][:, ::2].contiguous()
+    o1 = decode_step(qg.repeat_interleave(2, dim=1).contiguous(), kg.repeat_interleave(2, dim=1).contiguous(),
+                     st["v"], st["alpha"], st["b"], st["w"], S1)
+    o2 = decode_step(qg, kg, st["v"], st["alpha"], st["b"], st["w"], S2)
+    torch.cuda.synchronize()
+    assert torch.equal(o1.view(torch.int16), o2.view(torch.int16))
+    assert torch.equal(S1, S2)
