@@ -113,7 +113,7 @@ def workload_bytes(wl):
     el = 2 if wl.dtype == "bf16" else 4
     th = wl.B * wl.T * wl.H
     gate = lambda kind: 0 if kind in ("none", "tied") else (th if kind == "scalar" else th * wl.dk)
-    n = th * (2 * wl.dk + 2 * wl.dv) + gate(wl.alpha) + gate(wl.b) + gate(wl.w)
+    n = wl.B * wl.T * wl.Hq * 2 * wl.dk + th * 2 * wl.dv + gate(wl.alpha) + gate(wl.b) + gate(wl.w)
     state = wl.B * wl.H * wl.dk * wl.dv * 4
     return n * el + state * (1 + int(wl.s0))
 
@@ -364,13 +364,13 @@ def run_ours(args):
         e2e_ms, h2d, d2h = time_chunk_e2e(inp, wl, dev, max(3, args.steps // 2), args.warmup)
         e2e_steps = max(3, args.steps // 2)
         other = {}
-        for name in ("kda", "gdn2", "gla"):
+        for name in ("kda", "gdn2", "gla", "gdn_gqa"):
             w2 = WORKLOADS[name]
             _, _, tot2, per2 = time_chunk(w2, dev, max(3, args.steps // 2), args.warmup, lambda: None)
             a2 = statistics.fmean(per2)
             b2, f2 = workload_bytes(w2), workload_flops(w2)
             rt = max(b2 / (pk["hbm_gbs"] * 1e9), f2 / (pk["bf16_tflops"] * 1e12))
-            other[name] = {"workload": f"{name} B={w2.B} H={w2.H} T={w2.T} d_k={w2.dk} d_v={w2.dv} bf16 alpha={w2.alpha} "
+            other[name] = {"workload": f"{name} B={w2.B} H={w2.H} (q/k heads {w2.Hq}) T={w2.T} d_k={w2.dk} d_v={w2.dv} bf16 alpha={w2.alpha} "
                                        f"b={w2.b} w={w2.w} S0={'random' if w2.s0 else 'zero'}",
                            "tokens_per_s": w2.B * w2.T / (a2 * 1e-3), "ms_per_launch": a2,
                            "hbm_gbs": b2 / (a2 * 1e-3) / 1e9, "roofline_frac": rt / (a2 * 1e-3),

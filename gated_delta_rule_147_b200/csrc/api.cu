@@ -159,7 +159,7 @@ gdr_status gdr_chunk_fwd_grouped(const void* q, const void* k, const void* v, co
         return e == cudaSuccess ? GDR_OK : GDR_ERR_LAUNCH;
     }
     const bool tc_path = dtype == GDR_BF16 && d_k == 128 && d_v % 64 == 0;
-    if (!tc_path && (d_k > 128 || d_v > 1024)) return GDR_ERR_UNSUPPORTED;
+    if (!tc_path && (d_k > 256 || d_v > 1024)) return GDR_ERR_UNSUPPORTED;
     if (!aligned16(q) || !aligned16(k) || !aligned16(v) || !aligned16(o) ||
         (S0 && !aligned16(S0)) || (S_T && !aligned16(S_T)))
         return GDR_ERR_MISALIGNED;

@@ -44,6 +44,7 @@ __global__ void __launch_bounds__(NT, 1) chunk_fwd_erasefree_kernel(
                                              ~uintptr_t(1023));
     const int tid = threadIdx.x, warp = tid >> 5, wg = warp >> 2, row = tid & 127;
     const int vt = blockIdx.x, h = blockIdx.y, bb = blockIdx.z;
+    const int hq = h / p.group;  // q / k head of this value head
     const int v0 = vt * NV;
     const int T = p.T, H = p.H;
     const int nchunks = (T + C - 1) / C;
@@ -81,10 +82,10 @@ __global__ void __launch_bounds__(NT, 1) chunk_fwd_erasefree_kernel(
     auto issue_loads = [&](int ci) {
         const int t0 = ci * C;
         mbar_expect_tx(bar_tma, (uint32_t)(5 + 2 * (ACH + wch)) * 8192u);
-        tma_load_4d(sm + OFF_QIN, &tm_q, bar_tma, 0, h / p.group, t0, bb);
-        tma_load_4d(sm + OFF_QIN + 8192, &tm_q, bar_tma, 64, h / p.group, t0, bb);
-        tma_load_4d(sm + OFF_KIN, &tm_k, bar_tma, 0, h / p.group, t0, bb);
-        tma_load_4d(sm + OFF_KIN + 8192, &tm_k, bar_tma, 64, h / p.group, t0, bb);
+        tma_load_4d(sm + OFF_QIN, &tm_q, bar_tma, 0, hq, t0, bb);
+        tma_load_4d(sm + OFF_QIN + 8192, &tm_q, bar_tma, 64, hq, t0, bb);
+        tma_load_4d(sm + OFF_KIN, &tm_k, bar_tma, 0, hq, t0, bb);
+        tma_load_4d(sm + OFF_KIN + 8192, &tm_k, bar_tma, 64, hq, t0, bb);
         tma_load_4d(sm + OFF_V + (ci & 1) * 8192, &tm_v, bar_tma, v0, h, t0, bb);
         if (ACH) {
             tma_load_4d(sm + OFF_GA, &tm_a, bar_tma, 0, h, t0, bb);

@@ -97,6 +97,7 @@ __global__ void __launch_bounds__(NT, 1) chunk_fwd_kernel(
     const int wg = warp >> 2;          // warpgroup: which half of the columns it handles
     const int row = tid & 127;         // TMEM lane this thread reads (warp % 4 selects the quarter)
     const int vt = blockIdx.x, h = blockIdx.y, bb = blockIdx.z;
+    const int hq = h / p.group;  // q / k head of this value head
     const int v0 = vt * NV;
     const int T = p.T, H = p.H;
     const int nchunks = (T + C - 1) / C;
@@ -139,10 +140,10 @@ __global__ void __launch_bounds__(NT, 1) chunk_fwd_kernel(
         const int t0 = ci * C;
         const uint32_t bytes = (uint32_t)(4 + 1 + 2 * (ach + bch + wch)) * 8192u;
         mbar_expect_tx(bar_tma, bytes);
-        tma_load_4d(sm + OFF_QIN, &tm_q, bar_tma, 0, h / p.group, t0, bb);
-        tma_load_4d(sm + OFF_QIN + 8192, &tm_q, bar_tma, 64, h / p.group, t0, bb);
-        tma_load_4d(sm + OFF_KIN, &tm_k, bar_tma, 0, h / p.group, t0, bb);
-        tma_load_4d(sm + OFF_KIN + 8192, &tm_k, bar_tma, 64, h / p.group, t0, bb);
+        tma_load_4d(sm + OFF_QIN, &tm_q, bar_tma, 0, hq, t0, bb);
+        tma_load_4d(sm + OFF_QIN + 8192, &tm_q, bar_tma, 64, hq, t0, bb);
+        tma_load_4d(sm + OFF_KIN, &tm_k, bar_tma, 0, hq, t0, bb);
+        tma_load_4d(sm + OFF_KIN + 8192, &tm_k, bar_tma, 64, hq, t0, bb);
         tma_load_4d(sm + OFF_V + (ci & 1) * 8192, &tm_v, bar_tma, v0, h, t0, bb);
         if (ach) {
             tma_load_4d(sm + OFF_GA, &tm_a, bar_tma, 0, h, t0, bb);
@@ -722,6 +723,7 @@ __global__ void __launch_bounds__(NT, 1) chunk_fwd_gdn_kernel(
     const int wg = warp >> 2;
     const int row = tid & 127;
     const int vt = blockIdx.x, h = blockIdx.y, bb = blockIdx.z;
+    const int hq = h / p.group;  // q / k head of this value head
     const int v0 = vt * NV;
     const int T = p.T, H = p.H;
     const int nchunks = (T + C - 1) / C;
@@ -763,12 +765,12 @@ __global__ void __launch_bounds__(NT, 1) chunk_fwd_gdn_kernel(
         uint8_t* k2 = sm + gdn::OFF_K2 + buf * 16384;
         mbar_expect_tx(&bar_tma[buf], 7u * 8192u);
         // [K ; Q]: each 64-column block holds 128 rows (k rows 0..63, q rows 64..127)
-        tma_load_4d(qk, &tm_k, &bar_tma[buf], 0, h / p.group, t0, bb);
-        tma_load_4d(qk + 16384, &tm_k, &bar_tma[buf], 64, h / p.group, t0, bb);
-        tma_load_4d(qk + 8192, &tm_q, &bar_tma[buf], 0, h / p.group, t0, bb);
-        tma_load_4d(qk + 16384 + 8192, &tm_q, &bar_tma[buf], 64, h / p.group, t0, bb);
-        tma_load_4d(k2, &tm_k, &bar_tma[buf], 0, h / p.group, t0, bb);
-        tma_load_4d(k2 + 8192, &tm_k, &bar_tma[buf], 64, h / p.group, t0, bb);
+        tma_load_4d(qk, &tm_k, &bar_tma[buf], 0, hq, t0, bb);
+        tma_load_4d(qk + 16384, &tm_k, &bar_tma[buf], 64, hq, t0, bb);
+        tma_load_4d(qk + 8192, &tm_q, &bar_tma[buf], 0, hq, t0, bb);
+        tma_load_4d(qk + 16384 + 8192, &tm_q, &bar_tma[buf], 64, hq, t0, bb);
+        tma_load_4d(k2, &tm_k, &bar_tma[buf], 0, hq, t0, bb);
+        tma_load_4d(k2 + 8192, &tm_k, &bar_tma[buf], 64, hq, t0, bb);
         tma_load_4d(sm + gdn::OFF_V + buf * 8192, &tm_v, &bar_tma[buf], v0, h, t0, bb);
     };
 

@@ -135,6 +135,10 @@ __global__ void __launch_bounds__(NT, 2) prep_general_kernel(
     auto elem = [&](int r) {  // element index of (token row r, channel ch0)
         return (((size_t)bb * T + t0 + min(r, n - 1)) * H + h) * DK + ch0;
     };
+    const int Hq = H / pp.group, hq = h / pp.group;  // q / k heads; this value head's
+    auto elem_qk = [&](int r) {
+        return (((size_t)bb * T + t0 + min(r, n - 1)) * Hq + hq) * DK + ch0;
+    };
     uint2 aa[8];
     if (ACH) {
 #pragma unroll
@@ -145,7 +149,7 @@ __global__ void __launch_bounds__(NT, 2) prep_general_kernel(
     uint2 qa[4], ka[4], ba[4], wa[4];
     auto load_token = [&](int i) {
         const size_t e = elem(rg * 8 + i);
-        const size_t eq = (e / DK) / pp.group * DK + ch0;  // q, k row of this value head
+        const size_t eq = elem_qk(rg * 8 + i);
         const int sl = i & 3;
         ld8b(pp.q + eq, qa[sl]);
         ld8b(pp.k + eq, ka[sl]);

@@ -112,10 +112,11 @@ __global__ void __launch_bounds__(NT, 2) prep_gdn_kernel(const __grid_constant__
     auto issue_loads = [&](int item, int buf) {
         int ci, h, bb;
         coords(item, ci, h, bb);
+        const int hq = h / pp.group;
         const int t0 = ci * C;
         mbar_expect_tx(&bar_tma[buf], (uint32_t)(2 + nvt) * 8192u);
-        tma_load_4d(sm + P_OFF_K + buf * 16384, &tm_k, &bar_tma[buf], 0, h / pp.group, t0, bb);
-        tma_load_4d(sm + P_OFF_K + buf * 16384 + 8192, &tm_k, &bar_tma[buf], 64, h / pp.group, t0, bb);
+        tma_load_4d(sm + P_OFF_K + buf * 16384, &tm_k, &bar_tma[buf], 0, hq, t0, bb);
+        tma_load_4d(sm + P_OFF_K + buf * 16384 + 8192, &tm_k, &bar_tma[buf], 64, hq, t0, bb);
         for (int vt = 0; vt < nvt; ++vt)
             tma_load_4d(sm + P_OFF_V + buf * 16384 + vt * 8192, &tm_v, &bar_tma[buf], vt * 64, h, t0, bb);
     };
@@ -385,6 +386,7 @@ __global__ void __launch_bounds__(NT, 1) state_gdn_kernel(
     const int wg = warp >> 2;
     const int row = tid & 127;
     const int vt = blockIdx.x, h = blockIdx.y, bb = blockIdx.z;
+    const int hq = h / p.group;  // q / k head of this value head
     const int v0 = vt * NV;
     const int T = p.T, H = p.H;
     const int nchunks = (T + C - 1) / C;
@@ -428,10 +430,10 @@ __global__ void __launch_bounds__(NT, 1) state_gdn_kernel(
         // [-W ; Q]: each 64-column block holds 128 rows (-W rows 0..63, q rows 64..127)
         tma_load_4d(wq, &tm_w, &bar_tma[buf], 0, h, t0, bb);
         tma_load_4d(wq + 16384, &tm_w, &bar_tma[buf], 64, h, t0, bb);
-        tma_load_4d(wq + 8192, &tm_q, &bar_tma[buf], 0, h / p.group, t0, bb);
-        tma_load_4d(wq + 16384 + 8192, &tm_q, &bar_tma[buf], 64, h / p.group, t0, bb);
-        tma_load_4d(kk, &tm_k, &bar_tma[buf], 0, h / p.group, t0, bb);
-        tma_load_4d(kk + 8192, &tm_k, &bar_tma[buf], 64, h / p.group, t0, bb);
+        tma_load_4d(wq + 8192, &tm_q, &bar_tma[buf], 0, hq, t0, bb);
+        tma_load_4d(wq + 16384 + 8192, &tm_q, &bar_tma[buf], 64, hq, t0, bb);
+        tma_load_4d(kk, &tm_k, &bar_tma[buf], 0, hq, t0, bb);
+        tma_load_4d(kk + 8192, &tm_k, &bar_tma[buf], 64, hq, t0, bb);
         tma_load_4d(sm + S_OFF_P + buf * 8192, &tm_p, &bar_tma[buf], v0, h, t0, bb);
     };
 

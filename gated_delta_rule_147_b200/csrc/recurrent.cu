@@ -12,10 +12,11 @@
 
 namespace gdr {
 
-constexpr int kRecMaxDK = 128;
 constexpr int kRecCols = 64;  // threads (state columns) per block
 
-template <typename TI>
+// MAXDK: the state column a thread holds in registers (128, or 256 for the
+// wider heads, where part of it lives in local memory).
+template <typename TI, int kRecMaxDK>
 __global__ void __launch_bounds__(kRecCols) recurrent_fwd_kernel(
     const TI* __restrict__ q, const TI* __restrict__ k, const TI* __restrict__ v,
     const TI* __restrict__ alpha, const TI* __restrict__ bg, const TI* __restrict__ wg, int akind,
@@ -36,7 +37,7 @@ __global__ void __launch_bounds__(kRecCols) recurrent_fwd_kernel(
     for (int t = 0; t < T; ++t) {
         const int buf = t & 1;
         const size_t tok = ((size_t)b * T + t) * H + h;
-        const size_t tokq = tok / group;  // q, k have H / group heads
+        const size_t tokq = ((size_t)b * T + t) * (H / group) + h / group;  // q, k have H / group heads
         for (int i = threadIdx.x; i < dk; i += kRecCols) {
             const size_t gi = tok * dk + i;
             const size_t qi = tokq * dk + i;
@@ -86,15 +87,19 @@ cudaError_t launch_recurrent(const void* q, const void* k, const void* v, const 
                              void* o, float* ST, int B, int T, int H, int dk, int dv, int dtype,
                              int group, cudaStream_t st) {
     dim3 grid((dv + kRecCols - 1) / kRecCols, H, B);
-    if (dtype == GDR_BF16)
-        recurrent_fwd_kernel<__nv_bfloat16><<<grid, kRecCols, 0, st>>>(
-            (const __nv_bfloat16*)q, (const __nv_bfloat16*)k, (const __nv_bfloat16*)v,
-            (const __nv_bfloat16*)a, (const __nv_bfloat16*)b, (const __nv_bfloat16*)w, ak, bk, wk,
-            S0, (__nv_bfloat16*)o, ST, T, H, dk, dv, group);
-    else
-        recurrent_fwd_kernel<float><<<grid, kRecCols, 0, st>>>(
-            (const float*)q, (const float*)k, (const float*)v, (const float*)a, (const float*)b,
-            (const float*)w, ak, bk, wk, S0, (float*)o, ST, T, H, dk, dv, group);
+    auto go = [&](auto kern, auto tag) {
+        using TI = decltype(tag);
+        kern<<<grid, kRecCols, 0, st>>>((const TI*)q, (const TI*)k, (const TI*)v, (const TI*)a,
+                                        (const TI*)b, (const TI*)w, ak, bk, wk, S0, (TI*)o, ST, T, H,
+                                        dk, dv, group);
+    };
+    if (dtype == GDR_BF16) {
+        if (dk <= 128) go(recurrent_fwd_kernel<__nv_bfloat16, 128>, __nv_bfloat16{});
+        else go(recurrent_fwd_kernel<__nv_bfloat16, 256>, __nv_bfloat16{});
+    } else {
+        if (dk <= 128) go(recurrent_fwd_kernel<float, 128>, float{});
+        else go(recurrent_fwd_kernel<float, 256>, float{});
+    }
     return cudaGetLastError();
 }
 

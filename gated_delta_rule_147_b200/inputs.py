@@ -22,6 +22,8 @@ settings; "Erase-then-Delta Attention" abstract for the independent b/w gates;
          with gdn2 gates; 1000 steps; state from seed 4, step s from (4, s)
   gla    B=4,H=16,T=4096,d_k=128,d_v=256 bf16; q,k L2-normalised; channel
          alpha; no erase (b = 0), w = 1; S0 = 0; seed 5 (erase-free path)
+  gdn_gqa B=2,H=32 value heads with 16 q/k heads (value head h reads q/k
+         head h // 2),T=4096,d=128 bf16; gdn gates per value head; seed 6
 
 Value recipes: q,k,v ~ N(0,1); alpha = exp(-softplus(x)), x ~ N(0,1);
 sigmoid gates = 1/(1+exp(-x)), x ~ N(0,1). L2 normalisation is
@@ -58,9 +60,14 @@ class ChunkWorkload:
     bw_dist: str        # "sigmoid" | "uniform"
     seed: int
     chunk: int = 64
+    hq: int = 0         # q/k heads (grouped heads); 0 means H
 
     def with_(self, **kw) -> "ChunkWorkload":
         return replace(self, **kw)
+
+    @property
+    def Hq(self) -> int:
+        return self.hq or self.H
 
     @property
     def tokens(self) -> int:
@@ -80,6 +87,10 @@ WORKLOADS = {
     # ("How Linear Attention Remembers", Table 1); q, k L2-normalised
     "gla": ChunkWorkload("gla", 4, 16, 4096, 128, 256, "bf16", "channel", "none", "none",
                          True, True, False, "sigmoid", 5),
+    # Gated DeltaNet gates with grouped heads: 16 q/k heads serving 32 value heads
+    # ("How Linear Attention Remembers", Table 1)
+    "gdn_gqa": ChunkWorkload("gdn_gqa", 2, 32, 4096, 128, 128, "bf16", "scalar", "scalar", "tied",
+                             False, True, False, "sigmoid", 6, hq=16),
 }
 
 
@@ -142,13 +153,14 @@ def make_chunk_inputs(wl: ChunkWorkload) -> dict:
     """Draw one workload's inputs; returns CPU torch tensors already in the
     device dtype (what the GPU consumes; the oracle widens these to fp64).
 
-    Layout: q,k [B,T,H,dk]; v [B,T,H,dv]; scalar gates [B,T,H]; channel gates
-    [B,T,H,dk]; S0 [B,H,dk,dv] fp32 or None.
+    Layout: q,k [B,T,Hq,dk] (Hq = H unless the heads are grouped); v
+    [B,T,H,dv]; scalar gates [B,T,H]; channel gates [B,T,H,dk]; S0
+    [B,H,dk,dv] fp32 or None.
     """
     rng = np.random.Generator(np.random.PCG64(wl.seed))
     B, T, H, dk, dv = wl.B, wl.T, wl.H, wl.dk, wl.dv
-    q = _normal(rng, (B, T, H, dk))
-    k = _normal(rng, (B, T, H, dk))
+    q = _normal(rng, (B, T, wl.Hq, dk))
+    k = _normal(rng, (B, T, wl.Hq, dk))
     v = _normal(rng, (B, T, H, dv))
     if wl.q_norm:
         q = _l2norm(q)

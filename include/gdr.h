@@ -101,8 +101,8 @@ typedef enum {
  * state on chip). Its decay range: within every chunk and channel the
  * summed -log(alpha) over the chunk's tokens after the first must not exceed
  * 160 (outside it the kernel sets GDR_DEVICE_DECAY_RANGE). Every other
- * supported shape (fp32, or 1 <= d_k, d_v <= 128 otherwise) runs an exact
- * fp32 token-by-token CUDA kernel.
+ * supported shape (fp32, or 1 <= d_k <= 256 and 1 <= d_v <= 1024 otherwise)
+ * runs an exact fp32 token-by-token CUDA kernel.
  * Alignment: q, k, v, o and channel gates must be 16-byte aligned and, on
  * the tensor-core path, d_k and d_v rows 16-byte multiples (given by the
  * shape rules above).

@@ -27,8 +27,12 @@ def run_chunk(inp, dev, S0="inp", final_state=True, d_status=None, workspace="au
 
 def run_oracle(inp, heads=None):
     """Oracle on all heads, or on a list of (b, h) pairs (returned stacked as
-    [n, T, 1, dv] / [n, 1, dk, dv])."""
+    [n, T, 1, dv] / [n, 1, dk, dv]). Grouped q/k heads are repeated per value
+    head first (value head h reads q/k head h // group)."""
     g = inp["gates"]
+    G = inp["v"].shape[2] // inp["q"].shape[2]
+    if G > 1:
+        inp = dict(inp, q=inp["q"].repeat_interleave(G, dim=2), k=inp["k"].repeat_interleave(G, dim=2))
     if heads is None:
         return oracle.recurrence(inp["q"], inp["k"], inp["v"], inp["alpha"], inp["b"], inp["w"],
                                  inp["S0"], g)

@@ -64,7 +64,7 @@ def chunk(**kw):
     (dict(q=NULL), _lib.GDR_ERR_INVALID_ARG),
     (dict(o=NULL), _lib.GDR_ERR_INVALID_ARG),
     (dict(chunk=32), _lib.GDR_ERR_UNSUPPORTED),
-    (dict(dtype=1, dk=256), _lib.GDR_ERR_UNSUPPORTED),
+    (dict(dtype=1, dk=512), _lib.GDR_ERR_UNSUPPORTED),
     (dict(q=P + 8), _lib.GDR_ERR_MISALIGNED),
     (dict(o=P + 2), _lib.GDR_ERR_MISALIGNED),
     (dict(ST=P + 4), _lib.GDR_ERR_MISALIGNED),

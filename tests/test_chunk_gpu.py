@@ -303,3 +303,27 @@ def test_grouped_heads_fp32_exact_path(cuda_device):
                       inp["b"].to(dev), TIED, inp["S0"].to(dev))
     torch.cuda.synchronize()
     assert np.array_equal(o.cpu().numpy(), o_ref) and np.array_equal(ST.cpu().numpy(), S_ref)
+
+
+@pytest.mark.parametrize("dtype,dv", [("bf16", 64), ("fp32", 128), ("bf16", 256)])
+def test_dk256_exact_path(cuda_device, dtype, dv):
+    """d_k = 256 heads (GDN-340M width) run on the exact token-by-token path."""
+    wl = WORKLOADS["kda"].with_(B=1, H=2, T=70, dk=256, dv=dv, dtype=dtype, s0=True, seed=81)
+    inp = make_chunk_inputs(wl)
+    o, ST = run_chunk(inp, cuda_device)
+    o_ref, ST_ref = run_oracle(inp)
+    assert_close(o, o_ref, TOL[dtype], "o")
+    assert_close(ST, ST_ref, TOL[dtype], "S_T")
+
+
+def test_grouped_workload_full_size_sampled_heads(cuda_device):
+    """The grouped-heads workload the benchmark times (32 value heads, 16 q/k
+    heads, Gated DeltaNet gates) at full size, sampled heads against the oracle."""
+    wl = WORKLOADS["gdn_gqa"]
+    inp = make_chunk_inputs(wl)
+    o, ST = run_chunk(inp, cuda_device)
+    heads = [(0, 0), (0, 1), (1, 30)]
+    o_ref, ST_ref = run_oracle(inp, heads)
+    o_s, ST_s = gather_heads(o, ST, heads)
+    assert_close(o_s, o_ref, TOL["bf16"], f"o {heads}")
+    assert_close(ST_s, ST_ref, TOL["bf16"], f"S_T {heads}")
