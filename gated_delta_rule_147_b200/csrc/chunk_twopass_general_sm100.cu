@@ -613,15 +613,21 @@ finish:
 // ---- pass 2 ------------------------------------------------------------------
 template <bool UNTIED>
 struct StateLayout {
-    static constexpr uint32_t WQ = 0;                    // [WN ; QG] bf16 [128 x 128], 2 x 32 KB
-    static constexpr uint32_t K2 = 65536;                // K2 bf16 [64 x 128], 2 x 16 KB
-    static constexpr uint32_t AQU = 98304;               // [U ; AQ] bf16 [128 x 64], 2 x 16 KB
-    static constexpr uint32_t P = 131072;                // P slice bf16 [64 x 64], 2 x 8 KB
-    static constexpr uint32_t KW2 = 147456;              // KW2 bf16 [64 x 128], 2 x 16 KB (untied)
-    static constexpr uint32_t BQ = UNTIED ? 180224 : 0;  // BQ bf16 [64 x 64], 2 x 8 KB (untied)
-    static constexpr uint32_t V = UNTIED ? 196608 : 0;   // V slice bf16 [64 x 64], 2 x 8 KB (untied)
-    static constexpr uint32_t SBF = UNTIED ? 212992 : 147456;  // S bf16 [128 x 64]
-    static constexpr uint32_t SMALL = SBF + 16384;             // barriers, TMEM slot (1 KB)
+    // inputs are triple-buffered with tied gates (chunk ci + 2 loads while chunk
+    // ci runs), double-buffered with independent gates (more inputs per chunk)
+    static constexpr int NBUF = UNTIED ? 2 : 3;
+    static constexpr uint32_t WQ = 0;                          // [WN ; QG] bf16 [128 x 128], 32 KB each
+    static constexpr uint32_t K2 = WQ + NBUF * 32768;          // K2 bf16 [64 x 128], 16 KB each
+    static constexpr uint32_t P = K2 + NBUF * 16384;           // P slice bf16 [64 x 64], 8 KB each
+    static constexpr uint32_t AQ = P + NBUF * 8192;            // AQ bf16 [64 x 64], 8 KB each: rows
+                                                               // 64..127 of an M = 128 operand whose
+                                                               // rows 0..63 (the 8 KB before) are unused
+    static constexpr uint32_t KW2 = AQ + NBUF * 8192;          // KW2 bf16 [64 x 128], 16 KB each (untied)
+    static constexpr uint32_t BQ = KW2 + (UNTIED ? NBUF * 16384 : 0);  // BQ bf16 [64 x 64] (untied)
+    static constexpr uint32_t V = BQ + (UNTIED ? NBUF * 8192 : 0);     // V slice bf16 [64 x 64] (untied)
+    static constexpr uint32_t U = V + (UNTIED ? NBUF * 8192 : 0);      // U bf16 [64 x 64]
+    static constexpr uint32_t SBF = U + 8192;                          // S bf16 [128 x 64]
+    static constexpr uint32_t SMALL = SBF + 16384;                     // barriers, TMEM slot (1 KB)
     static constexpr uint32_t BYTES = SMALL + 1024 + 1024;
 };
 // D3 (U, QG S) and D5 (AQ U, BQ V) alternate between two column sets by chunk parity.
@@ -654,12 +660,14 @@ __global__ void __launch_bounds__(NT, 1) state_general_kernel(
     const int T = p.T, H = p.H;
     const int nchunks = (T + C - 1) / C;
 
-    uint64_t* bar_tma = reinterpret_cast<uint64_t*>(sm + Lay::SMALL);  // [2]
-    uint64_t* bar_mma = bar_tma + 2;
+    constexpr int NBUF = Lay::NBUF;
+    uint64_t* bar_tma = reinterpret_cast<uint64_t*>(sm + Lay::SMALL);  // [NBUF]
+    uint64_t* bar_mma = bar_tma + 3;
     uint32_t* s_tmem = reinterpret_cast<uint32_t*>(sm + Lay::SMALL + 32);
     if (tid == 0) {
         mbar_init(&bar_tma[0], 1);
         mbar_init(&bar_tma[1], 1);
+        mbar_init(&bar_tma[2], 1);
         mbar_init(bar_mma, 1);
         fence_barrier_init();
     }
@@ -669,12 +677,12 @@ __global__ void __launch_bounds__(NT, 1) state_general_kernel(
     tc_fence_after();
     const uint32_t tmem = *s_tmem;
     const uint32_t lane_base = (uint32_t)((warp & 3) * 32) << 16;
-    uint32_t ph_tma0 = 0u, ph_tma1 = 0u, ph_mma = 0;
+    uint32_t ph_tma0 = 0u, ph_tma1 = 0u, ph_tma2 = 0u, ph_mma = 0;
     bool ok = true;
     const uint32_t sbase = smem_u32(sm);
 
     auto issue_loads = [&](int ci) {
-        const int t0 = ci * C, buf = ci & 1;
+        const int t0 = ci * C, buf = ci % NBUF;
         uint64_t* bar = &bar_tma[buf];
         uint8_t* wq = sm + Lay::WQ + buf * 32768;
         mbar_expect_tx(bar, (UNTIED ? 12u : 8u) * 8192u);
@@ -684,7 +692,7 @@ __global__ void __launch_bounds__(NT, 1) state_general_kernel(
         tma_load_4d(wq + 16384 + 8192, &tm_qg, bar, 64, h, t0, bb);
         tma_load_4d(sm + Lay::K2 + buf * 16384, &tm_k2, bar, 0, h, t0, bb);
         tma_load_4d(sm + Lay::K2 + buf * 16384 + 8192, &tm_k2, bar, 64, h, t0, bb);
-        tma_load_4d(sm + Lay::AQU + buf * 16384 + 8192, &tm_aq, bar, 0, h, t0, bb);
+        tma_load_4d(sm + Lay::AQ + buf * 8192, &tm_aq, bar, 0, h, t0, bb);
         tma_load_4d(sm + Lay::P + buf * 8192, &tm_p, bar, v0, h, t0, bb);
         if (UNTIED) {
             tma_load_4d(sm + Lay::KW2 + buf * 16384, &tm_kw2, bar, 0, h, t0, bb);
@@ -713,7 +721,10 @@ __global__ void __launch_bounds__(NT, 1) state_general_kernel(
     const int c_begin = p.c_begin, c_end = p.c_end;
     const float* gcp = p.gc + ((size_t)bb * H + h) * nchunks * DK + row;
     float gC_next = c_begin < c_end ? gcp[(size_t)c_begin * DK] : 0.f;
-    if (tid == 0 && c_begin < c_end) issue_loads(c_begin);
+    if (tid == 0) {
+        if (c_begin < c_end) issue_loads(c_begin);
+        if (NBUF == 3 && c_begin + 1 < c_end) issue_loads(c_begin + 1);
+    }
 
     auto store_o = [&](int cj) {
         const int pj = cj & 1;
@@ -755,15 +766,17 @@ __global__ void __launch_bounds__(NT, 1) state_general_kernel(
     } while (0)
 
     for (int ci = c_begin; ci < c_end; ++ci) {
-        const int buf = ci & 1, par = ci & 1;
+        const int buf = ci % NBUF, par = ci & 1;
         const uint32_t wqb = sbase + Lay::WQ + buf * 32768u;
         const uint32_t k2b = sbase + Lay::K2 + buf * 16384u;
-        const uint32_t aqub = sbase + Lay::AQU + buf * 16384u;
+        const uint32_t aqa = sbase + Lay::AQ + buf * 8192u - 8192u;  // AQ = rows 64..127
+        const uint32_t ub = sbase + Lay::U;
         const uint32_t d3 = GS_TM_D3 + (uint32_t)par * 64u, d5 = GS_TM_D5 + (uint32_t)par * 64u;
         const float gC = gC_next;
         if (ci + 1 < c_end) gC_next = gcp[(size_t)(ci + 1) * DK];
         if (buf == 0) GDR_WAIT_SOLO(&bar_tma[0], ph_tma0);
-        else GDR_WAIT_SOLO(&bar_tma[1], ph_tma1);
+        else if (buf == 1) GDR_WAIT_SOLO(&bar_tma[1], ph_tma1);
+        else GDR_WAIT_SOLO(&bar_tma[2], ph_tma2);
 
         // ---- batch 1: D3 = [WN ; QG] S;  untied: D4 = KW2^T V, D5 = [. ; BQ] V --------
         if (tid == 0) {
@@ -789,8 +802,8 @@ __global__ void __launch_bounds__(NT, 1) state_general_kernel(
             }
             mma_commit(bar_mma);
         }
-        // chunk ci + 1's inputs go to the buffers chunk ci - 1 has released
-        if (tid == 32 && ci + 1 < c_end) issue_loads(ci + 1);
+        // chunk ci + NBUF - 1's inputs go to the buffers chunk ci - 1 has released
+        if (tid == 32 && ci + NBUF - 1 < c_end) issue_loads(ci + NBUF - 1);
         // the previous chunk's outputs, while batch 1 runs
         if (row >= 64 && ci > c_begin) store_o(ci - 1);
         GDR_WAIT_SOLO(bar_mma, ph_mma);
@@ -806,7 +819,7 @@ __global__ void __launch_bounds__(NT, 1) state_general_kernel(
                 ld_chunk(sm + Lay::P + buf * 8192, sw128_chunk(row, wg * 4 + c8, 64), x);
 #pragma unroll
                 for (int e = 0; e < 8; ++e) x[e] += d[c8 * 8 + e];
-                st_chunk(sm + Lay::AQU + buf * 16384, sw128_chunk(row, wg * 4 + c8, 128), x);
+                st_chunk(sm + Lay::U, sw128_chunk(row, wg * 4 + c8, 64), x);
             }
         }
         fence_proxy_async();
@@ -821,10 +834,10 @@ __global__ void __launch_bounds__(NT, 1) state_general_kernel(
 #pragma unroll
             for (int ks = 0; ks < 4; ++ks) {
                 const uint32_t acc = UNTIED ? 1u : (uint32_t)(ks > 0);
-                mma_bf16(tmem + d5, sdesc_sw128(aqub + ks * 32u, 16, 1024),
-                         sdesc_sw128(aqub + ks * 2048u, 8192, 1024), idK, acc);
+                mma_bf16(tmem + d5, sdesc_sw128(aqa + ks * 32u, 16, 1024),
+                         sdesc_sw128(ub + ks * 2048u, 8192, 1024), idK, acc);
                 mma_bf16(tmem + GS_TM_D4, sdesc_sw128(k2b + ks * 2048u, 8192, 1024),
-                         sdesc_sw128(aqub + ks * 2048u, 8192, 1024), idM, acc);
+                         sdesc_sw128(ub + ks * 2048u, 8192, 1024), idM, acc);
             }
             mma_commit(bar_mma);
         }
