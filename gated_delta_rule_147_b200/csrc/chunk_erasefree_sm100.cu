@@ -27,14 +27,21 @@ constexpr uint32_t OFF_GW = 49152;     // channel w
 constexpr uint32_t OFF_AQG = 65536;    // [q.g ; q.rowf] bf16 [128 x 128]
 constexpr uint32_t OFF_KWS = 98304;    // w.k.colf bf16 [64 x 128]
 constexpr uint32_t OFF_BQ = 114688;    // [Bq ; 0] bf16 [128 x 64]
-constexpr uint32_t OFF_V = 131072;     // v slice [64 x 64] bf16, two buffers
-constexpr uint32_t OFF_SBF = 147456;   // S bf16 [128 x 64]
-constexpr uint32_t OFF_SCAN = 163840;  // scan scratch fp32 [9 x 128]
-constexpr uint32_t OFF_SMALL = 169984; // scalars, barriers
-constexpr uint32_t SMEM_BYTES = OFF_SMALL + 3072 + 1024;
-constexpr uint32_t TM_D1 = 0, TM_D3 = 64, TM_D4 = 128, TM_COLS = 256;
+constexpr uint32_t OFF_V = 131072;     // v slice [64 x NVT] bf16 (NVT / 64 tiles of 8 KB), two buffers
+// The CTA's value columns NVT (64 or 128; 128 halves the CTA count where there
+// are more 64-column tiles than SMs) size the rest of the map:
+template <int NVT>
+struct Lay {
+    static constexpr uint32_t VBUF = NVT / 64 * 8192;          // one V buffer
+    static constexpr uint32_t SBF = OFF_V + 2 * VBUF;          // S bf16 [128 x NVT] (16 KB per 64 columns)
+    static constexpr uint32_t SCAN = SBF + NVT / 64 * 16384;   // scan scratch fp32 [9 x 128]
+    static constexpr uint32_t SMALL = SCAN + 6144;             // scalars, barriers
+    static constexpr uint32_t BYTES = SMALL + 3072 + 1024;
+    static constexpr uint32_t TM_D1 = 0, TM_D3 = 64, TM_D4 = 64 + NVT;
+    static constexpr uint32_t TM_COLS = NVT == 64 ? 256 : 512;
+};
 
-template <bool ACH>
+template <bool ACH, int NVT>
 __global__ void __launch_bounds__(NT, 1) chunk_fwd_erasefree_kernel(
     const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ CUtensorMap tm_k,
     const __grid_constant__ CUtensorMap tm_v, const __grid_constant__ CUtensorMap tm_a,
@@ -45,7 +52,10 @@ __global__ void __launch_bounds__(NT, 1) chunk_fwd_erasefree_kernel(
     const int tid = threadIdx.x, warp = tid >> 5, wg = warp >> 2, row = tid & 127;
     const int vt = blockIdx.x, h = blockIdx.y, bb = blockIdx.z;
     const int hq = h / p.group;  // q / k head of this value head
-    const int v0 = vt * NV;
+    const int v0 = vt * NVT;
+    using L = Lay<NVT>;
+    constexpr uint32_t OFF_SBF = L::SBF, OFF_SCAN = L::SCAN, OFF_SMALL = L::SMALL;
+    constexpr uint32_t TM_D1 = L::TM_D1, TM_D3 = L::TM_D3, TM_D4 = L::TM_D4, TM_COLS = L::TM_COLS;
     const int T = p.T, H = p.H;
     const int nchunks = (T + C - 1) / C;
     const bool wch = p.wkind == GDR_GATE_CHANNEL;
@@ -81,12 +91,14 @@ __global__ void __launch_bounds__(NT, 1) chunk_fwd_erasefree_kernel(
 
     auto issue_loads = [&](int ci) {
         const int t0 = ci * C;
-        mbar_expect_tx(bar_tma, (uint32_t)(5 + 2 * (ACH + wch)) * 8192u);
+        mbar_expect_tx(bar_tma, (uint32_t)(4 + NVT / 64 + 2 * (ACH + wch)) * 8192u);
         tma_load_4d(sm + OFF_QIN, &tm_q, bar_tma, 0, hq, t0, bb);
         tma_load_4d(sm + OFF_QIN + 8192, &tm_q, bar_tma, 64, hq, t0, bb);
         tma_load_4d(sm + OFF_KIN, &tm_k, bar_tma, 0, hq, t0, bb);
         tma_load_4d(sm + OFF_KIN + 8192, &tm_k, bar_tma, 64, hq, t0, bb);
-        tma_load_4d(sm + OFF_V + (ci & 1) * 8192, &tm_v, bar_tma, v0, h, t0, bb);
+#pragma unroll
+        for (int i = 0; i < NVT / 64; ++i)
+            tma_load_4d(sm + OFF_V + (ci & 1) * L::VBUF + i * 8192, &tm_v, bar_tma, v0 + 64 * i, h, t0, bb);
         if (ACH) {
             tma_load_4d(sm + OFF_GA, &tm_a, bar_tma, 0, h, t0, bb);
             tma_load_4d(sm + OFF_GA + 8192, &tm_a, bar_tma, 64, h, t0, bb);
@@ -97,7 +109,7 @@ __global__ void __launch_bounds__(NT, 1) chunk_fwd_erasefree_kernel(
         }
     };
 
-    constexpr int NH = NV / 2;
+    constexpr int NH = NVT / 2;
     float S[NH];
     {
         const float* s0 = p.S0 ? p.S0 + (((size_t)bb * H + h) * DK + row) * p.dv + v0 + wg * NH : nullptr;
@@ -107,7 +119,7 @@ __global__ void __launch_bounds__(NT, 1) chunk_fwd_erasefree_kernel(
             S[j] = x.x; S[j + 1] = x.y; S[j + 2] = x.z; S[j + 3] = x.w;
         }
 #pragma unroll
-        for (int ch = 0; ch < 4; ++ch) st_chunk(sm + OFF_SBF, sw128_chunk(row, wg * 4 + ch, DK), &S[8 * ch]);
+        for (int ch = 0; ch < NH / 8; ++ch) st_chunk(sm + OFF_SBF, sw128_chunk(row, wg * (NH / 8) + ch, DK), &S[8 * ch]);
         if (tid < 64) {  // rows 64..127 of [Bq ; 0] stay zero
 #pragma unroll
             for (int ch = 0; ch < 8; ++ch) st_zero_chunk(sm + OFF_BQ, sw128_chunk(64 + tid, ch, 128));
@@ -142,7 +154,7 @@ __global__ void __launch_bounds__(NT, 1) chunk_fwd_erasefree_kernel(
     for (int ci = 0; ci < nchunks; ++ci) {
         const int t0 = ci * C;
         const int n = min(C, T - t0);
-        const uint32_t vbuf = sbase + OFF_V + (ci & 1) * 8192u;
+        const uint32_t vbuf = sbase + OFF_V + (ci & 1) * L::VBUF;
         if (tid < C) {
             const bool valid = t0 + tid < T;
             s_a[tid] = (p.akind == GDR_GATE_SCALAR && valid) ? bits_to_f32(g_a) : 1.f;
@@ -292,8 +304,8 @@ __global__ void __launch_bounds__(NT, 1) chunk_fwd_erasefree_kernel(
         if (tid == 0) {
             tc_fence_after();
             const uint32_t id64 = idesc_bf16(128, 64, 0, 0);
-            const uint32_t idS = idesc_bf16(128, NV, 0, 1);
-            const uint32_t idM = idesc_bf16(128, NV, 1, 1);
+            const uint32_t idS = idesc_bf16(128, NVT, 0, 1);
+            const uint32_t idM = idesc_bf16(128, NVT, 1, 1);
 #pragma unroll
             for (int ks = 0; ks < 8; ++ks) {
                 const uint32_t koff = (ks >> 2) * 16384u + (ks & 3) * 32u;
@@ -301,7 +313,7 @@ __global__ void __launch_bounds__(NT, 1) chunk_fwd_erasefree_kernel(
                 mma_bf16(tmem + TM_D1, sdesc_sw128(sbase + OFF_AQG + koff, 16, 1024),
                          sdesc_sw128(sbase + OFF_KWS + koffk, 16, 1024), id64, ks > 0);
                 mma_bf16(tmem + TM_D3, sdesc_sw128(sbase + OFF_AQG + koff, 16, 1024),
-                         sdesc_sw128(sbase + OFF_SBF + ks * 2048u, 8192, 1024), idS, ks > 0);
+                         sdesc_sw128(sbase + OFF_SBF + ks * 2048u, 16384, 1024), idS, ks > 0);
             }
 #pragma unroll
             for (int ks = 0; ks < 4; ++ks)
@@ -330,7 +342,7 @@ __global__ void __launch_bounds__(NT, 1) chunk_fwd_erasefree_kernel(
         // ---- O += Bq V -------------------------------------------------------------
         if (tid == 0) {
             tc_fence_after();
-            const uint32_t idS = idesc_bf16(128, NV, 0, 1);
+            const uint32_t idS = idesc_bf16(128, NVT, 0, 1);
 #pragma unroll
             for (int ks = 0; ks < 4; ++ks)
                 mma_bf16(tmem + TM_D3, sdesc_sw128(sbase + OFF_BQ + ks * 32u, 16, 1024),
@@ -340,32 +352,36 @@ __global__ void __launch_bounds__(NT, 1) chunk_fwd_erasefree_kernel(
         GDR_WAIT(bar_mma, ph_mma);
         tc_fence_after();
 
-        // ---- O (rows 0..63 of D3) -> global; S = g S + f D4 -------------------------
+        // ---- O (rows 0..63 of D3) -> global; S = g S + f D4 (32 columns at a time) ----
         {
-            float d[32], dS[32];
-            if (row < 64) tmem_ld32_async(tmem + lane_base + TM_D3 + wg * 32, d);
-            tmem_ld32_async(tmem + lane_base + TM_D4 + wg * 32, dS);
-            tmem_wait_ld();
-            if (row < 64) {
-                const int t = t0 + row;
-                if (t < T) {
-                    __nv_bfloat16* op = p.o + (((size_t)bb * T + t) * H + h) * p.dv + v0 + wg * 32;
-#pragma unroll
-                    for (int c8 = 0; c8 < 4; ++c8) {
-                        uint4 u;
-                        u.x = pack_bf16x2(d[c8 * 8 + 0], d[c8 * 8 + 1]);
-                        u.y = pack_bf16x2(d[c8 * 8 + 2], d[c8 * 8 + 3]);
-                        u.z = pack_bf16x2(d[c8 * 8 + 4], d[c8 * 8 + 5]);
-                        u.w = pack_bf16x2(d[c8 * 8 + 6], d[c8 * 8 + 7]);
-                        *reinterpret_cast<uint4*>(op + c8 * 8) = u;
-                    }
-                }
-            }
             const float gC = s_gC[row], fS = s_fS[row];
 #pragma unroll
-            for (int j = 0; j < NH; ++j) S[j] = gC * S[j] + fS * dS[j];
+            for (int hf = 0; hf < NH / 32; ++hf) {
+                float d[32], dS[32];
+                const uint32_t col = wg * NH + hf * 32;
+                if (row < 64) tmem_ld32_async(tmem + lane_base + TM_D3 + col, d);
+                tmem_ld32_async(tmem + lane_base + TM_D4 + col, dS);
+                tmem_wait_ld();
+                if (row < 64) {
+                    const int t = t0 + row;
+                    if (t < T) {
+                        __nv_bfloat16* op = p.o + (((size_t)bb * T + t) * H + h) * p.dv + v0 + col;
 #pragma unroll
-            for (int ch = 0; ch < 4; ++ch) st_chunk(sm + OFF_SBF, sw128_chunk(row, wg * 4 + ch, DK), &S[8 * ch]);
+                        for (int c8 = 0; c8 < 4; ++c8) {
+                            uint4 u;
+                            u.x = pack_bf16x2(d[c8 * 8 + 0], d[c8 * 8 + 1]);
+                            u.y = pack_bf16x2(d[c8 * 8 + 2], d[c8 * 8 + 3]);
+                            u.z = pack_bf16x2(d[c8 * 8 + 4], d[c8 * 8 + 5]);
+                            u.w = pack_bf16x2(d[c8 * 8 + 6], d[c8 * 8 + 7]);
+                            *reinterpret_cast<uint4*>(op + c8 * 8) = u;
+                        }
+                    }
+                }
+#pragma unroll
+                for (int j = 0; j < 32; ++j) S[hf * 32 + j] = gC * S[hf * 32 + j] + fS * dS[j];
+            }
+#pragma unroll
+            for (int ch = 0; ch < NH / 8; ++ch) st_chunk(sm + OFF_SBF, sw128_chunk(row, wg * (NH / 8) + ch, DK), &S[8 * ch]);
         }
         tc_fence_before();
         __syncthreads();
@@ -399,15 +415,25 @@ cudaError_t launch_chunk_erasefree_sm100(const CUtensorMap* maps, const void* al
     p.B = B; p.T = T; p.H = H; p.dv = dv;
     p.akind = akind; p.bkind = GDR_GATE_NONE; p.wkind = wkind;
     p.group = group;
-    dim3 grid(dv / chunkc::NV, H, B);
-    auto launch = [&](auto kern) -> cudaError_t {
-        cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, erasefree::SMEM_BYTES);
+    // 128 value columns per CTA when there are more 64-column tiles than SMs
+    // (one wave instead of two); the MMAs cost the same to issue at N = 128
+    int dev = 0, nsm = 0;
+    cudaError_t e0 = cudaGetDevice(&dev);
+    if (e0 == cudaSuccess) e0 = cudaDeviceGetAttribute(&nsm, cudaDevAttrMultiProcessorCount, dev);
+    if (e0 != cudaSuccess) return e0;
+    const bool wide = dv % 128 == 0 && (long long)(dv / 64) * H * B > nsm;
+    auto launch = [&](auto kern, int nvt, uint32_t bytes) -> cudaError_t {
+        cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, bytes);
         if (e != cudaSuccess) return e;
-        kern<<<grid, chunkc::NT, erasefree::SMEM_BYTES, st>>>(maps[0], maps[1], maps[2], maps[3], maps[5], p);
+        kern<<<dim3(dv / nvt, H, B), chunkc::NT, bytes, st>>>(maps[0], maps[1], maps[2], maps[3], maps[5], p);
         return cudaGetLastError();
     };
-    return akind == GDR_GATE_CHANNEL ? launch(erasefree::chunk_fwd_erasefree_kernel<true>)
-                                     : launch(erasefree::chunk_fwd_erasefree_kernel<false>);
+    using namespace erasefree;
+    if (wide)
+        return akind == GDR_GATE_CHANNEL ? launch(chunk_fwd_erasefree_kernel<true, 128>, 128, Lay<128>::BYTES)
+                                         : launch(chunk_fwd_erasefree_kernel<false, 128>, 128, Lay<128>::BYTES);
+    return akind == GDR_GATE_CHANNEL ? launch(chunk_fwd_erasefree_kernel<true, 64>, 64, Lay<64>::BYTES)
+                                     : launch(chunk_fwd_erasefree_kernel<false, 64>, 64, Lay<64>::BYTES);
 }
 
 }  // namespace gdr

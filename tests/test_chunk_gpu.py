@@ -327,3 +327,15 @@ def test_grouped_workload_full_size_sampled_heads(cuda_device):
     o_s, ST_s = gather_heads(o, ST, heads)
     assert_close(o_s, o_ref, TOL["bf16"], f"o {heads}")
     assert_close(ST_s, ST_ref, TOL["bf16"], f"S_T {heads}")
+
+
+@pytest.mark.parametrize("dv,akind,wkind", [(256, "channel", "none"), (128, "scalar", "channel")])
+def test_erase_free_wide_ctas(cuda_device, dv, akind, wkind):
+    """More 64-column tiles than SMs: the erase-free kernel carries 128 value
+    columns per CTA (one wave of CTAs)."""
+    wl = WORKLOADS["gla"].with_(B=2, H=40, T=200, dv=dv, alpha=akind, w=wkind, s0=True, seed=61)
+    inp = make_chunk_inputs(wl)
+    o, ST = run_chunk(inp, cuda_device)
+    o_ref, ST_ref = run_oracle(inp)
+    assert_close(o, o_ref, TOL["bf16"], "o")
+    assert_close(ST, ST_ref, TOL["bf16"], "S_T")
