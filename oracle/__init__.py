@@ -14,6 +14,9 @@ device dtype and then widened:
 
 Routes (each follows a different passage, so they pin each other):
   recurrence            C token loop (gdr_oracle.c), the oracle proper.
+  recurrence_bwd        its reverse-mode gradient (C, all states kept),
+                        pinned by finite differences of `recurrence` and by
+                        the linear-attention closed form.
   recurrence_py         the same definition as a numpy token loop (small cases).
   unrolled_contributions  S_t = sum_i C_i^(t) with explicit d_k x d_k
                         transition matrices ("How Linear Attention Remembers",
@@ -104,6 +107,11 @@ def load_library(path: str):
                                                             dp, ctypes.c_int, dp, ctypes.c_int,
                                                             dp, dp, dp, ctypes.c_int]
     lib.gdr_oracle_forward.restype = ctypes.c_int
+    lib.gdr_oracle_backward.argtypes = [ctypes.c_int] * 5 + [dp, dp, dp, dp, ctypes.c_int,
+                                                             dp, ctypes.c_int, dp, ctypes.c_int,
+                                                             dp, dp, dp, dp, dp, dp, dp, dp, dp, dp,
+                                                             ctypes.c_int]
+    lib.gdr_oracle_backward.restype = ctypes.c_int
     lib.gdr_oracle_max_threads.restype = ctypes.c_int
     return lib
 
@@ -129,6 +137,41 @@ def recurrence(q, k, v, alpha=None, b=None, w=None, S0=None, gates=None, nthread
     if rc != 0:
         raise RuntimeError(f"gdr_oracle_forward returned {rc}")
     return o, S_T
+
+
+def recurrence_bwd(q, k, v, alpha=None, b=None, w=None, S0=None, gates=None, dO=None, dS_T=None,
+                   nthreads: int = 0, lib=None):
+    """Gradients of L = sum(o * dO) + sum(S_T * dS_T) with respect to every
+    input of `recurrence` (the C oracle's reverse-mode token loop), in fp64.
+
+    Returns a dict: dq, dk [B,T,H,dk]; dv [B,T,H,dv]; dalpha, db, dw shaped like
+    their gates (None for an absent gate; with w "tied", db holds the whole
+    gradient of the shared beta and dw is None); dS0 [B,H,dk,dv] (the gradient
+    with respect to the initial state, zero-state runs included).
+    """
+    q, k, v = f64(q), f64(k), f64(v)
+    B, T, H, dk = q.shape
+    dv = v.shape[-1]
+    g = dict(gates or {})
+    tied = g.get("w") == "tied"
+    a, apc, bb, bpc, ww, wpc = _resolve_gates(alpha, b, w, gates)
+    S0, dO, dS_T = f64(S0), f64(dO), f64(dS_T)
+    gshape = lambda pc: (B, T, H, dk) if pc else (B, T, H)
+    out = {"dq": np.zeros((B, T, H, dk)), "dk": np.zeros((B, T, H, dk)),
+           "dv": np.zeros((B, T, H, dv)), "dS0": np.zeros((B, H, dk, dv))}
+    da = None if a is None else np.zeros(gshape(apc))
+    dbb = None if bb is None else np.zeros(gshape(bpc))
+    dww = None if ww is None else np.zeros(gshape(wpc))
+    rc = (lib or _lib()).gdr_oracle_backward(
+        B, T, H, dk, dv, _ptr(q), _ptr(k), _ptr(v), _ptr(a), apc, _ptr(bb), bpc, _ptr(ww), wpc,
+        _ptr(S0), _ptr(dO), _ptr(dS_T), _ptr(out["dq"]), _ptr(out["dk"]), _ptr(out["dv"]),
+        _ptr(da), _ptr(dbb), _ptr(dww), _ptr(out["dS0"]), int(nthreads))
+    if rc != 0:
+        raise RuntimeError(f"gdr_oracle_backward returned {rc}")
+    if tied:
+        dbb, dww = dbb + dww, None
+    out.update(dalpha=da, db=dbb, dw=dww)
+    return out
 
 
 def decode_step(q, k, v, alpha, b, w, S, gates=None, nthreads: int = 0):

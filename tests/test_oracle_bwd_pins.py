@@ -1,0 +1,113 @@
+"""Pins for the oracle's backward pass (no GPU).
+
+The pages name a gate-aware backward pass ("Erase-then-Delta Attention"
+(Gated DeltaNet-2), abstract) without a formula, so the gradient is fixed by
+the mathematics alone: it must equal the derivative of the forward oracle
+(central finite differences of `oracle.recurrence`, itself pinned in
+test_oracle_pins.py), and it must reduce to closed forms where the forward is
+a plain masked matrix product ("The Eraser Trilogy", "The Rosetta Stone").
+"""
+import zlib
+
+import numpy as np
+import pytest
+
+import oracle
+from test_oracle_pins import rand_inputs
+
+GRAD_OF = {"q": "dq", "k": "dk", "v": "dv", "alpha": "dalpha", "b": "db", "w": "dw", "S0": "dS0"}
+
+
+def loss(args, gates, dO, dS_T, lib=None):
+    o, ST = oracle.recurrence(args["q"], args["k"], args["v"], args["alpha"], args["b"],
+                              args["w"], args["S0"], gates, lib=lib)
+    return float((o * dO).sum() + (0.0 if dS_T is None else (ST * dS_T).sum()))
+
+
+def finite_difference(args, gates, dO, dS_T, name, eps=1e-6, lib=None):
+    x = args[name]
+    fd = np.zeros_like(x)
+    for idx in np.ndindex(x.shape):
+        a = dict(args)
+        xp, xm = x.copy(), x.copy()
+        xp[idx] += eps
+        xm[idx] -= eps
+        a[name] = xp
+        lp = loss(a, gates, dO, dS_T, lib)
+        a[name] = xm
+        lm = loss(a, gates, dO, dS_T, lib)
+        fd[idx] = (lp - lm) / (2 * eps)
+    return fd
+
+
+def fd_mismatch(gates, s0, dst, seed, lib=None, T=5, dk=3, dv=4):
+    """Largest |analytic - finite difference| / (1 + max|fd|) over every input."""
+    rng = np.random.default_rng(seed)
+    q, k, v, a, b, w, S0 = rand_inputs(rng, 1, T, 2, dk, dv, gates, s0=s0, k_unit=False)
+    args = dict(q=q, k=k, v=v, alpha=a, b=b, w=w, S0=S0 if s0 else np.zeros((1, 2, dk, dv)))
+    dO = rng.standard_normal(v.shape)
+    dS_T = rng.standard_normal((1, 2, dk, dv)) if dst else None
+    g = oracle.recurrence_bwd(q, k, v, a, b, w, args["S0"], gates, dO, dS_T, lib=lib)
+    worst = 0.0
+    for name, x in args.items():
+        if x is None:
+            assert g[GRAD_OF[name]] is None
+            continue
+        fd = finite_difference(args, gates, dO, dS_T, name, lib=lib)
+        worst = max(worst, float(np.abs(fd - g[GRAD_OF[name]]).max() / (1 + np.abs(fd).max())))
+    return worst
+
+
+@pytest.mark.parametrize("gates", [
+    {"alpha": "channel", "b": "channel", "w": "channel"},    # Gated DeltaNet-2
+    {"alpha": "channel", "b": "scalar", "w": "tied"},        # KDA
+    {"alpha": "scalar", "b": "scalar", "w": "tied"},         # Gated DeltaNet
+    {"alpha": "none", "b": "scalar", "w": "tied"},           # DeltaNet
+    {"alpha": "channel", "b": "none", "w": "none"},          # GLA (erase-free)
+    {"alpha": "scalar", "b": "channel", "w": "scalar"},
+    {"alpha": "none", "b": "none", "w": "none"},             # linear attention
+])
+@pytest.mark.parametrize("s0,dst", [(True, True), (False, False)])
+def test_gradient_equals_finite_difference(gates, s0, dst):
+    assert fd_mismatch(gates, s0, dst, seed=zlib.crc32(f"{gates}{s0}".encode()) % 1000) < 1e-7
+
+
+def test_linear_attention_closed_form():
+    """alpha = 1, b = 0, w = 1, S0 = 0: o = tril(Q K^T) V, so
+    dQ = tril(dO V^T) K, dK = tril(dO V^T)^T Q, dV = tril(Q K^T)^T dO."""
+    rng = np.random.default_rng(3)
+    T, dk, dv = 37, 6, 5
+    q, k, v = (rng.standard_normal((1, T, 1, d)) for d in (dk, dk, dv))
+    dO = rng.standard_normal((1, T, 1, dv))
+    none = {"alpha": "none", "b": "none", "w": "none"}
+    g = oracle.recurrence_bwd(q, k, v, gates=none, dO=dO)
+    Q, K, V, D = q[0, :, 0], k[0, :, 0], v[0, :, 0], dO[0, :, 0]
+    np.testing.assert_allclose(g["dq"][0, :, 0], np.tril(D @ V.T) @ K, atol=1e-11)
+    np.testing.assert_allclose(g["dk"][0, :, 0], np.tril(D @ V.T).T @ Q, atol=1e-11)
+    np.testing.assert_allclose(g["dv"][0, :, 0], np.tril(Q @ K.T).T @ D, atol=1e-11)
+    np.testing.assert_allclose(g["dS0"][0, 0], Q.T @ D, atol=1e-11)
+
+
+def test_erase_free_initial_state_gradient_closed_form():
+    """b = 0: S_t = Diag(gamma_t) S0 + (terms without S0), gamma_t the running
+    product of alpha, so dS0 = sum_t (q_t . gamma_t)^T dO_t + Diag(gamma_T) dS_T
+    ("Recurrent Memory", section 04: survival factor of a stored entry)."""
+    rng = np.random.default_rng(4)
+    T, dk, dv = 23, 5, 4
+    gates = {"alpha": "channel", "b": "none", "w": "channel"}
+    q, k, v, a, b, w, S0 = rand_inputs(rng, 1, T, 1, dk, dv, gates, s0=True)
+    dO = rng.standard_normal(v.shape)
+    dS_T = rng.standard_normal(S0.shape)
+    g = oracle.recurrence_bwd(q, k, v, a, None, w, S0, gates, dO, dS_T)
+    gamma = np.cumprod(a[0, :, 0], axis=0)
+    want = (q[0, :, 0] * gamma).T @ dO[0, :, 0] + gamma[-1][:, None] * dS_T[0, 0]
+    np.testing.assert_allclose(g["dS0"][0, 0], want, atol=1e-11)
+
+
+def test_zero_length_gradient_is_dS_T():
+    rng = np.random.default_rng(5)
+    dS_T = rng.standard_normal((2, 3, 4, 5))
+    z = lambda *s: np.zeros(s)
+    g = oracle.recurrence_bwd(z(2, 0, 3, 4), z(2, 0, 3, 4), z(2, 0, 3, 5), gates={},
+                              S0=z(2, 3, 4, 5), dO=z(2, 0, 3, 5), dS_T=dS_T)
+    np.testing.assert_array_equal(g["dS0"], dS_T)

@@ -82,3 +82,34 @@ def test_unmodified_oracle_passes_pins(tmp_path):
 @pytest.mark.parametrize("name", sorted(MUTANTS))
 def test_pins_reject_mutant(tmp_path, name):
     assert not _pins_pass(_build_variant(tmp_path, name, MUTANTS[name]))
+
+
+# Mistakes planted in the backward pass (gdr_oracle_backward); the pins are the
+# finite-difference and closed-form checks of test_oracle_bwd_pins.py.
+BWD_MUTANTS = {
+    "bwd_dq_from_previous_state": [("acc += St[i * dv + j] * dot[j];", "acc += Sp[i * dv + j] * dot[j];")],
+    "bwd_drops_erase_term": [("double dsd = G[i * dv + j] + e * dr[j];", "double dsd = G[i * dv + j];")],
+    "bwd_dalpha_decayed_state": [("dal += dsd * Sp[i * dv + j];", "dal += dsd * Sd[i * dv + j];")],
+    "bwd_state_grad_not_decayed": [("G[i * dv + j] = a * dsd;", "G[i * dv + j] = dsd;")],
+    "bwd_dk_sign": [("dk_out[tok * dk + i] = -acck;", "dk_out[tok * dk + i] = acck;")],
+    "bwd_gates_swapped_in_dk": [("+= bi_ * de[i] + wi * du[i];", "+= wi * de[i] + bi_ * du[i];")],
+    "bwd_dv_key_without_w": [("accv += u * G[i * dv + j];", "accv += kt[i] * G[i * dv + j];")],
+    "bwd_dr_sign": [("dr[j] = -accr;", "dr[j] = accr;")],
+    "bwd_drops_write_key_grad": [("accu += G[i * dv + j] * vt[j];", "accu += 0.0 * vt[j];")],
+}
+
+
+def _bwd_pins_pass(lib) -> bool:
+    from test_oracle_bwd_pins import fd_mismatch
+    ok = fd_mismatch({"alpha": "channel", "b": "channel", "w": "channel"}, True, True, 7, lib=lib) < 1e-7
+    ok &= fd_mismatch({"alpha": "scalar", "b": "scalar", "w": "scalar"}, False, False, 8, lib=lib) < 1e-7
+    return bool(ok)
+
+
+def test_unmodified_backward_passes_pins(tmp_path):
+    assert _bwd_pins_pass(_build_variant(tmp_path, "clean_bwd", []))
+
+
+@pytest.mark.parametrize("name", sorted(BWD_MUTANTS))
+def test_backward_pins_reject_mutant(tmp_path, name):
+    assert not _bwd_pins_pass(_build_variant(tmp_path, name, BWD_MUTANTS[name]))
