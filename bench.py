@@ -265,6 +265,59 @@ def time_chunk_e2e(inp, wl, dev, steps, warmup):
     return e0.elapsed_time(e1), h2d, d2h
 
 
+# fp32 CUDA-core peak: 148 SMs x 128 FP32 lanes x 2 flop (FMA) x 1965 MHz
+ALU_FP32_TFLOPS = 148 * 128 * 2 * 1965e6 / 1e12
+# reverse-mode step per state element and token: forward step (decay, erase
+# read, erase, write: 4 multiply-adds) + reverse step (dq, G += q^T dO, dv, dr,
+# du, dk, de, dS', dalpha: 9 multiply-adds), 2 flop each
+BWD_FLOPS_PER_ELEMENT = 2 * 13
+
+
+def time_backward(dev, steps, warmup, pk):
+    """The backward pass (gdr_chunk_bwd) on the Gated DeltaNet workload: CUDA
+    events per call, both launches."""
+    import torch
+    from gated_delta_rule_147_b200 import TIED, chunk_bwd, gdr_chunk_bwd_workspace_size
+    from gated_delta_rule_147_b200.inputs import WORKLOADS, make_cotangents
+    wl = WORKLOADS["gdn"]
+    _, d = prepare_chunk(wl, dev)
+    cot = make_cotangents(wl)
+    dO, dST = cot["dO"].to(dev), cot["dS_T"].to(dev)
+    ws = torch.empty(gdr_chunk_bwd_workspace_size(wl.B, wl.T, wl.H, wl.dk, wl.dv), dtype=torch.uint8,
+                     device=dev)
+    stream = torch.cuda.current_stream()
+
+    def call():
+        chunk_bwd(d["q"], d["k"], d["v"], d["alpha"], d["b"], TIED, d["S0"], dO=dO, dS_T=dST,
+                  workspace=ws, stream=stream)
+
+    for _ in range(warmup):
+        call()
+    torch.cuda.synchronize()
+    ev = [torch.cuda.Event(enable_timing=True) for _ in range(steps + 1)]
+    ev[0].record(stream)
+    for i in range(steps):
+        call()
+        ev[i + 1].record(stream)
+    torch.cuda.synchronize()
+    ms = statistics.fmean(ev[i].elapsed_time(ev[i + 1]) for i in range(steps))
+    th = wl.B * wl.T * wl.H
+    state = wl.B * wl.H * wl.dk * wl.dv * 4
+    # read q, k, v, dO (bf16), alpha, beta (bf16), dS_T; write dq, dk, dv (fp32), dalpha, dbeta, dS0
+    bytes_ = th * (2 * (2 * wl.dk + 2 * wl.dv) + 2 * 2 + 4 * (2 * wl.dk + wl.dv) + 2 * 4) + 2 * state
+    flops = BWD_FLOPS_PER_ELEMENT * wl.dk * wl.dv * th
+    achieved = flops / (ms * 1e-3) / 1e12
+    return {"workload": f"Gated DeltaNet backward B={wl.B} H={wl.H} T={wl.T} d_k=d_v={wl.dk} bf16 "
+                        f"inputs, fp32 gradients, dO and dS_T ~ N(0, 1)",
+            "ms_per_call": ms, "tokens_per_s": wl.B * wl.T / (ms * 1e-3), "launches_per_call": 2,
+            "kernel": "gdr::bwd::bwd_ckpt_kernel + gdr::bwd::bwd_main_kernel (cluster of d_v/16 CTAs)",
+            "roofline": {"bound": "alu", "achieved": achieved, "peak": ALU_FP32_TFLOPS,
+                         "unit": "TFLOP/s", "frac": achieved / ALU_FP32_TFLOPS,
+                         "peak_source": "derived: 148 SMs x 128 fp32 lanes x 2 x 1965 MHz",
+                         "algorithmic_flops": flops, "algorithmic_bytes": bytes_,
+                         "hbm_frac": bytes_ / (ms * 1e-3) / 1e9 / pk["hbm_gbs"]}}
+
+
 def time_decode(dev, nsteps, warmup):
     import torch
     from gated_delta_rule_147_b200 import decode_step
@@ -376,6 +429,8 @@ def run_ours(args):
                            "hbm_gbs": b2 / (a2 * 1e-3) / 1e9, "roofline_frac": rt / (a2 * 1e-3),
                            "traffic": measured_traffic(name), "kernel": KERNEL_NAMES[kernel_family(w2)]}
             torch.cuda.empty_cache()
+        bwd = time_backward(dev, max(3, args.steps // 2), args.warmup, pk)
+        torch.cuda.empty_cache()
         dec = time_decode(dev, 1000, 10)
         dec["frac_of_hbm"] = dec["total_gbs"] / pk["hbm_gbs"]
         dec["peak_gbs"] = pk["hbm_gbs"]
@@ -401,6 +456,7 @@ def run_ours(args):
             "gpu_launches": args.steps * LAUNCHES_PER_CALL[kernel_family(wl)],
             "clocks": clocks,
             "decode": dec,
+            "backward": bwd,
             "other_workloads": other,
             "cpu_baseline": cpu,
         }

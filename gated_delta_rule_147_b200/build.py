@@ -12,6 +12,7 @@ HERE = os.path.dirname(os.path.abspath(__file__))
 ROOT = os.path.dirname(HERE)
 CSRC = os.path.join(HERE, "csrc")
 SOURCES = ["api.cu", "decode.cu", "recurrent.cu", "chunk_sm100.cu", "chunk_erasefree_sm100.cu",
+           "chunk_bwd.cu",
            "chunk_twopass_sm100.cu", "chunk_twopass_general_sm100.cu", "selftest.cu",
            "static_scratch.cu"]
 HEADERS = ["common.cuh", "chunk_common.cuh"]

@@ -180,6 +180,18 @@ def make_chunk_inputs(wl: ChunkWorkload) -> dict:
     }
 
 
+def make_cotangents(wl: ChunkWorkload, with_dS_T: bool = True) -> dict:
+    """Upstream gradients for a backward pass over `wl`, seed (wl.seed, 1):
+    dO ~ N(0, 1) [B,T,H,dv] in the device dtype, then dS_T ~ N(0, 1)
+    [B,H,dk,dv] fp32 (None when with_dS_T is False; still drawn, so dO does
+    not depend on the flag)."""
+    rng = np.random.Generator(np.random.PCG64(np.random.SeedSequence([wl.seed, 1])))
+    dO = _normal(rng, (wl.B, wl.T, wl.H, wl.dv))
+    dS_T = _normal(rng, (wl.B, wl.H, wl.dk, wl.dv))
+    return {"dO": _to_dev_dtype(dO, wl.dtype),
+            "dS_T": torch.from_numpy(dS_T) if with_dS_T else None}
+
+
 def make_decode_state(dw: DecodeWorkload = DECODE) -> torch.Tensor:
     """Initial decode state S [B,H,dk,dv] fp32 ~ N(0, 0.02^2), seed (dw.seed)."""
     rng = np.random.Generator(np.random.PCG64(dw.seed))

@@ -200,6 +200,62 @@ gdr_status gdr_chunk_fwd_static(const void* q, const void* k, const void* v,
 size_t gdr_chunk_fwd_static_capacity(void);
 
 /*
+ * gdr_chunk_bwd -- backward pass of gdr_chunk_fwd: the gradients of a scalar
+ * loss L with respect to every input, given dO = dL/do and dS_T = dL/dS_T.
+ *
+ * The pages call for a gate-aware backward pass that keeps training
+ * parallel ("Erase-then-Delta Attention" (Gated DeltaNet-2), abstract) but
+ * print no formula; the result is the exact derivative of the recurrence in
+ * the file comment, taken in reverse token order with G = dL/dS_t
+ * (e = b.k, u = w.k, S' = Diag(alpha_t) S_{t-1}, r_t = e S'):
+ *   dq_t = dO_t S_t^T;  G += q_t^T dO_t;  dv_t = u G;  dr = -k G;
+ *   dk_t = -G r_t^T + b.(S' dr^T) + w.(G v_t^T);
+ *   db_t = k.(S' dr^T);  dw_t = k.(G v_t^T);
+ *   dalpha_t = rowsum((G + e^T dr) . S_{t-1});  G <- Diag(alpha_t)(G + e^T dr);
+ * and finally dS0 = G. Scalar gates get the sum over channels of the
+ * per-channel gradient; with w tied to b, db holds the whole gradient of the
+ * shared beta (both terms) and dw must be NULL.
+ *
+ * Inputs: q, k, v, alpha, b, w, kinds, S0 (NULL = zero state), dtype exactly
+ *   as given to gdr_chunk_fwd; dO [B, T, H, d_v] in `dtype`; dS_T
+ *   [B, H, d_k, d_v] fp32 or NULL (= 0).
+ * Outputs, all fp32 and written completely (no accumulation into them):
+ *   dq, dk [B, T, H, d_k]; dv [B, T, H, d_v]; dalpha, db, dw in the layout of
+ *   their gate ([B, T, H] scalar, [B, T, H, d_k] channel), NULL exactly when
+ *   the gate has no data of its own (kind NONE, or w TIED); dS0
+ *   [B, H, d_k, d_v] or NULL (not written).
+ * workspace: caller-owned device scratch of at least
+ *   gdr_chunk_bwd_workspace_size() bytes, 256-byte aligned (the forward
+ *   state at the start of every 64-token chunk, fp32).
+ * Method: fp32 arithmetic for both dtypes. A first kernel runs the forward
+ *   and stores the chunk-start states; a second walks the chunks backwards,
+ *   recomputing each chunk's states from its checkpoint, with one
+ *   thread-block cluster of d_v / 16 CTAs per head (16 state columns each)
+ *   adding the per-row partial sums over columns through distributed shared
+ *   memory. d_status is not used (no bounded waits on this path).
+ * Supported: chunk = 64, 1 <= d_k <= 128, d_v a multiple of 16 up to 128.
+ *   Every pointer 16-byte aligned.
+ * Returns GDR_OK, GDR_ERR_INVALID_ARG (bad sizes or kinds, a NULL array that
+ * is required, a gradient pointer that does not match its gate, workspace
+ * missing or too small), GDR_ERR_UNSUPPORTED, GDR_ERR_MISALIGNED or
+ * GDR_ERR_LAUNCH. T = 0 writes dS0 := dS_T (or zeros) and launches nothing
+ * else.
+ */
+gdr_status gdr_chunk_bwd(const void* q, const void* k, const void* v,
+                         const void* alpha, const void* b, const void* w,
+                         int alpha_kind, int b_kind, int w_kind,
+                         const float* S0, const void* dO, const float* dS_T,
+                         float* dq, float* dk, float* dv,
+                         float* dalpha, float* db, float* dw, float* dS0,
+                         void* workspace, size_t workspace_bytes,
+                         int B, int T, int H, int d_k, int d_v, int chunk,
+                         int dtype, int* d_status, void* stream);
+
+/* Bytes of workspace gdr_chunk_bwd needs: B * H * ceil(T / 64) * d_k * d_v *
+ * 4 (0 for T < 1 or bad sizes). Host-only; launches nothing. */
+size_t gdr_chunk_bwd_workspace_size(int B, int T, int H, int d_k, int d_v);
+
+/*
  * gdr_decode_step -- one token per head (autoregressive decoding).
  *
  * Applies one step of the recurrence to every (b, h) head: S is read and

@@ -131,3 +131,48 @@ def test_grouped_entry_points_reject_bad_head_counts():
     st = lib.gdr_decode_step_grouped(P, P, P, P, P, P, 2, 2, 2, P, P, 2, 3, 4, 128, 128, 0,
                                      None, None)
     assert st == _lib.GDR_ERR_INVALID_ARG
+
+
+def bwd(**kw):
+    a = dict(q=P, k=P, v=P, alpha=P, b=P, w=NULL, ak=1, bk=1, wk=3, S0=NULL, dO=P, dST=NULL, dq=P,
+             dk_=P, dv_=P, dal=P, db=P, dw=NULL, dS0=P, ws=P, ws_bytes=1 << 30, B=1, T=64, H=1,
+             dk=128, dv=128, chunk=64, dtype=0)
+    a.update(kw)
+    return _lib.load().gdr_chunk_bwd(a["q"], a["k"], a["v"], a["alpha"], a["b"], a["w"], a["ak"],
+                                     a["bk"], a["wk"], a["S0"], a["dO"], a["dST"], a["dq"],
+                                     a["dk_"], a["dv_"], a["dal"], a["db"], a["dw"], a["dS0"],
+                                     a["ws"], a["ws_bytes"], a["B"], a["T"], a["H"], a["dk"],
+                                     a["dv"], a["chunk"], a["dtype"], None, None)
+
+
+# every case fails on the host, before any launch
+@pytest.mark.parametrize("kw,expect", [
+    (dict(B=0), _lib.GDR_ERR_INVALID_ARG),
+    (dict(T=-1), _lib.GDR_ERR_INVALID_ARG),
+    (dict(dtype=3), _lib.GDR_ERR_INVALID_ARG),
+    (dict(dO=NULL), _lib.GDR_ERR_INVALID_ARG),
+    (dict(dq=NULL), _lib.GDR_ERR_INVALID_ARG),
+    (dict(dal=NULL), _lib.GDR_ERR_INVALID_ARG),          # scalar alpha needs its gradient
+    (dict(dw=P), _lib.GDR_ERR_INVALID_ARG),              # tied w has no gradient of its own
+    (dict(ak=0, alpha=NULL), _lib.GDR_ERR_INVALID_ARG),  # absent alpha: dalpha must be NULL
+    (dict(ws=NULL), _lib.GDR_ERR_INVALID_ARG),
+    (dict(ws_bytes=1024), _lib.GDR_ERR_INVALID_ARG),     # workspace too small
+    (dict(chunk=32), _lib.GDR_ERR_UNSUPPORTED),
+    (dict(dk=256), _lib.GDR_ERR_UNSUPPORTED),
+    (dict(dv=144), _lib.GDR_ERR_UNSUPPORTED),
+    (dict(dv=40), _lib.GDR_ERR_UNSUPPORTED),
+    (dict(dO=P + 8), _lib.GDR_ERR_MISALIGNED),
+    (dict(dS0=P + 4), _lib.GDR_ERR_MISALIGNED),
+    (dict(ws=P + 16), _lib.GDR_ERR_MISALIGNED),
+])
+def test_chunk_bwd_rejects_bad_arguments(kw, expect):
+    assert bwd(**kw) == expect
+
+
+@pytest.mark.parametrize("shape,expect", [
+    ((4, 4096, 16, 128, 128), 4 * 16 * 64 * 128 * 128 * 4),
+    ((1, 65, 2, 64, 32), 1 * 2 * 2 * 64 * 32 * 4),
+    ((1, 0, 2, 64, 32), 0),
+])
+def test_bwd_workspace_size(shape, expect):
+    assert _lib.gdr_chunk_bwd_workspace_size(*shape) == expect
