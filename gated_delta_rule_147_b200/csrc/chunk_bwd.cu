@@ -1,52 +1,53 @@
-// Backward pass of the gated delta rule: fp32 arithmetic on CUDA cores, one
-// thread-block cluster per head.
+// Backward pass of the gated delta rule: fp32 arithmetic on CUDA cores.
 //
 // The pages ask for a gate-aware backward pass ("Erase-then-Delta Attention"
 // (Gated DeltaNet-2), abstract) without printing one. This is reverse-mode
 // differentiation of the token recurrence
 //   S' = Diag(alpha_t) S_{t-1},  r_t = (b_t . k_t) S',
 //   S_t = S' - k_t^T r_t + (w_t . k_t)^T v_t,  o_t = q_t S_t
-// ("Recurrent Memory: Write, Erase, Decay, Read", sections 01-05), run from the
+// ("Recurrent Memory: Write, Erase, Decay, Read", sections 01-05), from the
 // last token to the first with G = dL/dS_t (e = b.k, u = w.k):
 //   dq_t = dO_t S_t^T,   G += q_t^T dO_t,
-//   dv_t = u G,  du = G v_t^T,  dk = -G r_t^T,  dr = -k G,
-//   de = S' dr^T,  dS' = G + e^T dr,  dalpha = rowsum(dS' . S_{t-1}),
+//   dv_t = u G,  dr_t = -k G,  du = G v_t^T,  dk = -G r_t^T,
+//   de = S' dr_t^T,  dS' = G + e^T dr_t,  dalpha = rowsum(dS' . S_{t-1}),
 //   G <- Diag(alpha_t) dS',  dk += b.de + w.du,  db = k.de,  dw = k.du.
 //
-// Launches:
-//  1. bwd_ckpt_kernel: the forward recurrence, storing the state at the start
-//     of every 64-token chunk in the caller's workspace.
-//  2. bwd_main_kernel: chunks last to first. Per chunk the forward is
-//     recomputed from its checkpoint, keeping r_t of every token and the state
-//     at every 8-token sub-chunk start in shared memory; then, per sub-chunk
-//     last to first, its 8 states are rebuilt in registers (no reduction
-//     needed once r_t is known) and the reverse step runs token by token.
-// Layout: the cluster's CTA x owns state columns [16x, 16x + 16) of one head;
-// warp w of its 8 holds rows 32 (w % 4) + lane and columns 8 (w / 4) .. + 8 of
-// that slice, so S and G are 8 + 8 fp32 registers per thread. Sums over rows
-// (r, dr, dv) stay inside the CTA (warp shuffles, then four warps through
-// shared memory); sums over columns (the dq, dk, du, de, dalpha rows) are
-// partial per CTA and are added across the cluster through distributed shared
-// memory once per sub-chunk.
+// Structure. The state gradient obeys its own recurrence,
+//   G_{t-1} = Diag(alpha_t) (I - e_t^T k_t) G_t + q_{t-1}^T dO_{t-1},
+// which never reads S, so the two sequential parts are independent scans:
+//  1. bwd_scan_kernel, one warp per 8 state columns of a head (the column
+//     sums over d_k are in-thread plus warp shuffles, no block barrier):
+//     forward over the tokens: the state at every 64-token chunk start and
+//     r_t of every token; backward over the tokens: G at every chunk end,
+//     dr_t and dv_t of every token, and dS0. Both directions run at once.
+//  2. bwd_chunk_kernel, parallel over (row block, chunk, head): from the
+//     chunk's start state and end gradient it rebuilds S_{t-1} (elementwise,
+//     with r_t known; two levels: states at 8-token sub-chunk starts in
+//     shared memory, then 8 states in registers) and G_t (elementwise, with
+//     dr_t known), and forms dq, dk and the gate gradients. A CTA holds
+//     whole rows of the state, so the sums over columns stay inside it.
+//  3. bwd_gate_sum_kernel (scalar gates only): the sum over key channels of a
+//     scalar gate's gradient, from the per-row-block partial sums of pass 2.
 #include "common.cuh"
 
 namespace gdr {
 namespace bwd {
 
-constexpr int kC = 64;               // checkpoint interval (the chunk)
-constexpr int kSub = 8;              // sub-chunk: states rebuilt in registers
+constexpr int kC = 64;           // chunk: checkpoint interval of the scans
+constexpr int kSub = 8;          // sub-chunk: states rebuilt in registers
 constexpr int kNSub = kC / kSub;
-constexpr int kNC = 16;              // state columns per CTA
-constexpr int kThreads = 256;
-constexpr int kRows = 128;           // d_k limit (one thread per row and column half)
-constexpr int kMaxNB = 8;            // portable cluster size: d_v <= 128
-constexpr int kQty = 5;              // per-row partials: dq, dk (from r), du, de, dalpha
+constexpr int kMaxDK = 128;      // 4 rows per lane in the scans
+constexpr int kMaxDV = 256;      // 8 columns per thread, up to 32 threads per row in pass 2
+constexpr int kScanWarps = 4;    // scan CTA: 4 warps
+constexpr int kScanCols = 8;     // state columns per scan warp
+constexpr int kChunkThreads = 128;
 
 struct Params {
     const void *q, *k, *v, *alpha, *b, *w, *dO;
     const float *S0, *dST;
-    float *dq, *dk, *dv, *dalpha, *db, *dw, *dS0, *ckpt;
-    int T, H, dk_, dv_, akind, bkind, wkind, nchunks;
+    float *dq, *dk, *dv, *dalpha, *db, *dw, *dS0;
+    float *ckS, *ckG, *R, *DR, *GP;  // workspace
+    int B, T, H, dk_, dv_, akind, bkind, wkind, nchunks, tpr, nrb;
 };
 
 template <typename TI>
@@ -54,25 +55,31 @@ __device__ __forceinline__ float ld1(const void* p, size_t i) {
     return to_f32(static_cast<const TI*>(p)[i]);
 }
 
-// Eight consecutive elements (16- or 32-byte aligned) widened to fp32.
 template <typename TI>
-__device__ __forceinline__ void load8(const void* p, size_t off, float (&x)[8]);
+__device__ __forceinline__ void load4(const void* p, size_t off, float (&x)[4]);
 template <>
-__device__ __forceinline__ void load8<float>(const void* p, size_t off, float (&x)[8]) {
-    const float4* s = reinterpret_cast<const float4*>(static_cast<const float*>(p) + off);
-    const float4 a = s[0], b = s[1];
+__device__ __forceinline__ void load4<float>(const void* p, size_t off, float (&x)[4]) {
+    const float4 a = *reinterpret_cast<const float4*>(static_cast<const float*>(p) + off);
     x[0] = a.x; x[1] = a.y; x[2] = a.z; x[3] = a.w;
-    x[4] = b.x; x[5] = b.y; x[6] = b.z; x[7] = b.w;
 }
 template <>
-__device__ __forceinline__ void load8<__nv_bfloat16>(const void* p, size_t off, float (&x)[8]) {
-    const uint4 u = *reinterpret_cast<const uint4*>(static_cast<const __nv_bfloat16*>(p) + off);
-    const uint32_t w[4] = {u.x, u.y, u.z, u.w};
+__device__ __forceinline__ void load4<__nv_bfloat16>(const void* p, size_t off, float (&x)[4]) {
+    const uint2 u = *reinterpret_cast<const uint2*>(static_cast<const __nv_bfloat16*>(p) + off);
+    x[0] = __uint_as_float(u.x << 16); x[1] = __uint_as_float(u.x & 0xffff0000u);
+    x[2] = __uint_as_float(u.y << 16); x[3] = __uint_as_float(u.y & 0xffff0000u);
+}
+
+template <typename TI>
+__device__ __forceinline__ void load8(const void* p, size_t off, float (&x)[8]) {
+    float a[4], b[4];
+    load4<TI>(p, off, a);
+    load4<TI>(p, off + 4, b);
 #pragma unroll
-    for (int c = 0; c < 4; ++c) {
-        x[2 * c] = __uint_as_float(w[c] << 16);
-        x[2 * c + 1] = __uint_as_float(w[c] & 0xffff0000u);
-    }
+    for (int c = 0; c < 4; ++c) { x[c] = a[c]; x[4 + c] = b[c]; }
+}
+
+__device__ __forceinline__ void store4(float* dst, const float (&x)[4]) {
+    *reinterpret_cast<float4*>(dst) = make_float4(x[0], x[1], x[2], x[3]);
 }
 
 // Per-row scalars of one token for key channel i (neutral beyond d_k).
@@ -99,371 +106,471 @@ __device__ __forceinline__ Row load_row(const Params& p, size_t tok, int i) {
     return r;
 }
 
-// Sum over the warp's 32 lanes of NV values per lane, scattered: on return
-// the lane holds the total of value (lane / (32 / NV)). Each halving step
-// sends the half of the values the partner keeps.
+// Warp sum of NV values per lane, all lanes receiving all NV totals:
+// halving exchanges (each lane keeps the half its partner does not), plain
+// sums over the remaining lanes, then a broadcast of each total.
 template <int NV>
-__device__ __forceinline__ float warp_reduce_scatter(float* x, int lane) {
+__device__ __forceinline__ void warp_allsum(float (&x)[NV], int lane) {
+    float y[NV];
+#pragma unroll
+    for (int v = 0; v < NV; ++v) y[v] = x[v];
     int off = 16;
 #pragma unroll
     for (int half = NV / 2; half >= 1; half >>= 1, off >>= 1) {
         const bool hi = (lane & off) != 0;
 #pragma unroll
         for (int v = 0; v < half; ++v) {
-            const float send = hi ? x[v] : x[v + half];
-            const float keep = hi ? x[v + half] : x[v];
-            x[v] = keep + __shfl_xor_sync(0xffffffffu, send, off);
+            const float send = hi ? y[v] : y[v + half];
+            const float keep = hi ? y[v + half] : y[v];
+            y[v] = keep + __shfl_xor_sync(0xffffffffu, send, off);
         }
     }
-    float s = x[0];
+    float s = y[0];
 #pragma unroll
     for (; off >= 1; off >>= 1) s += __shfl_xor_sync(0xffffffffu, s, off);
-    return s;
-}
-
-// Row-group partial sums: red[parity][column half][row group][16].
-__device__ __forceinline__ float* red_at(float* red, int par, int cg, int rg) {
-    return red + ((par * 2 + cg) * 4 + rg) * 16;
-}
-
-// Column sums over the CTA's 128 rows of x[0..NV): warp shuffles, then one
-// barrier; the four row-group totals are read back with red_sum8.
-template <int NV>
-__device__ __forceinline__ void colsum_publish(float* x, float* red, int par, int cg, int rg,
-                                               int lane) {
-    const float s = warp_reduce_scatter<NV>(x, lane);
-    constexpr int G = 32 / NV;
-    if ((lane & (G - 1)) == 0) red_at(red, par, cg, rg)[lane / G] = s;
-    __syncthreads();
-}
-
-__device__ __forceinline__ void red_sum8(const float* red, int par, int cg, int c0, float (&out)[8]) {
+    // lane l now holds the total of value (l / (32 / NV))
 #pragma unroll
-    for (int c = 0; c < 8; ++c) out[c] = 0.f;
+    for (int v = 0; v < NV; ++v) x[v] = __shfl_sync(0xffffffffu, s, v * (32 / NV));
+}
+
+// Per-row scalars of rows i0 .. i0 + 3 of one token (neutral beyond d_k). With
+// d_k a multiple of 4 the four rows are one vector load per input.
+struct Rows4 {
+    float q[4], k[4], a[4], bg[4], wg[4];
+};
+
+template <typename TI>
+__device__ __forceinline__ void load_rows4(const Params& p, size_t tok, int i0, Rows4& r) {
+    if ((p.dk_ & 3) == 0) {
+        if (i0 < p.dk_) {
+            const size_t gi = tok * p.dk_ + i0;
+            load4<TI>(p.q, gi, r.q);
+            load4<TI>(p.k, gi, r.k);
+            if (p.akind == GDR_GATE_CHANNEL) load4<TI>(p.alpha, gi, r.a);
+            else {
+                const float a = p.akind == GDR_GATE_SCALAR ? ld1<TI>(p.alpha, tok) : 1.f;
+                r.a[0] = r.a[1] = r.a[2] = r.a[3] = a;
+            }
+            if (p.bkind == GDR_GATE_CHANNEL) load4<TI>(p.b, gi, r.bg);
+            else {
+                const float bb = p.bkind == GDR_GATE_SCALAR ? ld1<TI>(p.b, tok) : 0.f;
+                r.bg[0] = r.bg[1] = r.bg[2] = r.bg[3] = bb;
+            }
+            if (p.wkind == GDR_GATE_CHANNEL) load4<TI>(p.w, gi, r.wg);
+            else if (p.wkind == GDR_GATE_TIED) {
 #pragma unroll
-    for (int rg = 0; rg < 4; ++rg) {
-        const float4* s = reinterpret_cast<const float4*>(red_at(const_cast<float*>(red), par, cg, rg) + c0);
-        const float4 a = s[0], b = s[1];
-        out[0] += a.x; out[1] += a.y; out[2] += a.z; out[3] += a.w;
-        out[4] += b.x; out[5] += b.y; out[6] += b.z; out[7] += b.w;
+                for (int rr = 0; rr < 4; ++rr) r.wg[rr] = r.bg[rr];
+            } else {
+                const float ww = p.wkind == GDR_GATE_SCALAR ? ld1<TI>(p.w, tok) : 1.f;
+                r.wg[0] = r.wg[1] = r.wg[2] = r.wg[3] = ww;
+            }
+            return;
+        }
+#pragma unroll
+        for (int rr = 0; rr < 4; ++rr) {
+            r.q[rr] = r.k[rr] = r.bg[rr] = r.wg[rr] = 0.f;
+            r.a[rr] = 1.f;
+        }
+        return;
     }
-}
-
-// One forward token: S <- Diag(a) S; r = (b.k) S (column sums); S <- S - k^T r + (w.k)^T v.
-__device__ __forceinline__ void fwd_step(float (&S)[8], const Row& rw, const float (&v)[8], float* red,
-                                         int par, int cg, int rg, int lane, float (&r)[8]) {
-    const float e = rw.bg * rw.k, u = rw.wg * rw.k;
-    float x[8];
 #pragma unroll
-    for (int c = 0; c < 8; ++c) {
-        S[c] *= rw.a;
-        x[c] = e * S[c];
+    for (int rr = 0; rr < 4; ++rr) {
+        const Row w1 = load_row<TI>(p, tok, i0 + rr);
+        r.q[rr] = w1.q; r.k[rr] = w1.k; r.a[rr] = w1.a; r.bg[rr] = w1.bg; r.wg[rr] = w1.wg;
     }
-    colsum_publish<8>(x, red, par, cg, rg, lane);
-    red_sum8(red, par, cg, 0, r);
-#pragma unroll
-    for (int c = 0; c < 8; ++c) S[c] = fmaf(-rw.k, r[c], fmaf(u, v[c], S[c]));
-}
-
-__device__ __forceinline__ void store8(float* dst, const float (&x)[8]) {
-    reinterpret_cast<float4*>(dst)[0] = make_float4(x[0], x[1], x[2], x[3]);
-    reinterpret_cast<float4*>(dst)[1] = make_float4(x[4], x[5], x[6], x[7]);
-}
-__device__ __forceinline__ void load8f(const float* src, float (&x)[8]) {
-    const float4 a = reinterpret_cast<const float4*>(src)[0];
-    const float4 b = reinterpret_cast<const float4*>(src)[1];
-    x[0] = a.x; x[1] = a.y; x[2] = a.z; x[3] = a.w;
-    x[4] = b.x; x[5] = b.y; x[6] = b.z; x[7] = b.w;
 }
 
 // ----------------------------------------------------------------- pass 1 --
+// blockIdx.z = 2 b + direction; warp w of CTA x owns columns
+// 8 (kScanWarps x + w) .. + 8 (those below d_v), lane l owns rows 4 l .. 4 l + 3.
 template <typename TI>
-__global__ void __launch_bounds__(kThreads) bwd_ckpt_kernel(Params p) {
-    __shared__ __align__(16) float red[2 * 2 * 4 * 16];
-    const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5, rg = warp & 3, cg = warp >> 2;
-    const int i = 32 * rg + lane;
-    const int b = blockIdx.z, h = blockIdx.y;
-    const int col = kNC * blockIdx.x + 8 * cg;
+__global__ void __launch_bounds__(kScanWarps * 32) bwd_scan_kernel(Params p) {
+    constexpr int NC = kScanCols;
+    const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
+    const int c0 = NC * (kScanWarps * blockIdx.x + warp);
+    if (c0 >= p.dv_) return;  // no block-wide barriers in this kernel
+    const int b = blockIdx.z >> 1, dir = blockIdx.z & 1, h = blockIdx.y;
     const size_t head = (size_t)b * p.H + h;
-    const bool row_ok = i < p.dk_;
-    float S[8];
-    if (p.S0 && row_ok) load8f(p.S0 + (head * p.dk_ + i) * p.dv_ + col, S);
-    else
-        for (int c = 0; c < 8; ++c) S[c] = 0.f;
+    const int i0 = 4 * lane;
     auto tok_of = [&](int t) { return ((size_t)b * p.T + t) * p.H + h; };
-    Row nr = load_row<TI>(p, tok_of(0), i);
-    float nv[8];
-    load8<TI>(p.v, tok_of(0) * p.dv_ + col, nv);
-    int par = 0;
-    for (int t = 0; t < p.T; ++t) {
-        const Row rw = nr;
-        float v[8];
+    auto ck_at = [&](float* base, int chunk, int i) {
+        return base + ((head * p.nchunks + chunk) * p.dk_ + i) * p.dv_ + c0;
+    };
+    float X[4][NC];  // S (forward) or G (backward): rows i0 + rr, columns c0 + c
+    const float* init = dir == 0 ? p.S0 : p.dST;
 #pragma unroll
-        for (int c = 0; c < 8; ++c) v[c] = nv[c];
-        if (t + 1 < p.T) {  // next token's inputs are in flight during this step
-            nr = load_row<TI>(p, tok_of(t + 1), i);
-            load8<TI>(p.v, tok_of(t + 1) * p.dv_ + col, nv);
-        }
-        if (t % kC == 0 && row_ok)
-            store8(p.ckpt + (((head * p.nchunks + t / kC) * p.dk_) + i) * p.dv_ + col, S);
-        float r[8];
-        fwd_step(S, rw, v, red, par, cg, rg, lane, r);
-        par ^= 1;
+    for (int rr = 0; rr < 4; ++rr) {
+        if (init && i0 + rr < p.dk_) load8<float>(init, (head * p.dk_ + i0 + rr) * p.dv_ + c0, X[rr]);
+        else
+            for (int c = 0; c < NC; ++c) X[rr][c] = 0.f;
     }
+    // the next token's inputs are loaded while the current one is computed
+    const void* colsrc = dir == 0 ? p.v : p.dO;
+    Rows4 nrw;
+    float nvec[NC];
+    const int tfirst = dir == 0 ? 0 : p.T - 1;
+    load_rows4<TI>(p, tok_of(tfirst), i0, nrw);
+    load8<TI>(colsrc, tok_of(tfirst) * p.dv_ + c0, nvec);
+    for (int n = 0; n < p.T; ++n) {
+        const int t = dir == 0 ? n : p.T - 1 - n;
+        const size_t tok = tok_of(t);
+        const bool store_ck = dir == 0 ? (t % kC == 0) : (t == p.T - 1 || (t + 1) % kC == 0);
+        if (store_ck)  // forward: chunk start; backward: before the chunk's last token
+#pragma unroll
+            for (int rr = 0; rr < 4; ++rr)
+                if (i0 + rr < p.dk_) {
+                    float* dst = ck_at(dir == 0 ? p.ckS : p.ckG, t / kC, i0 + rr);
+                    reinterpret_cast<float4*>(dst)[0] = make_float4(X[rr][0], X[rr][1], X[rr][2], X[rr][3]);
+                    reinterpret_cast<float4*>(dst)[1] = make_float4(X[rr][4], X[rr][5], X[rr][6], X[rr][7]);
+                }
+        const Rows4 rw = nrw;
+        float cv[NC];
+#pragma unroll
+        for (int c = 0; c < NC; ++c) cv[c] = nvec[c];
+        if (n + 1 < p.T) {
+            const size_t tn = tok_of(dir == 0 ? t + 1 : t - 1);
+            load_rows4<TI>(p, tn, i0, nrw);
+            load8<TI>(colsrc, tn * p.dv_ + c0, nvec);
+        }
+        if (dir == 0) {
+            // S' = Diag(a) S; r = e S' (sum over rows); S = S' - k^T r + u^T v
+            float r[NC];
+#pragma unroll
+            for (int c = 0; c < NC; ++c) r[c] = 0.f;
+#pragma unroll
+            for (int rr = 0; rr < 4; ++rr) {
+                const float e = rw.bg[rr] * rw.k[rr];
+#pragma unroll
+                for (int c = 0; c < NC; ++c) {
+                    X[rr][c] *= rw.a[rr];
+                    r[c] = fmaf(e, X[rr][c], r[c]);
+                }
+            }
+            warp_allsum<NC>(r, lane);
+#pragma unroll
+            for (int rr = 0; rr < 4; ++rr) {
+                const float u = rw.wg[rr] * rw.k[rr];
+#pragma unroll
+                for (int c = 0; c < NC; ++c)
+                    X[rr][c] = fmaf(-rw.k[rr], r[c], fmaf(u, cv[c], X[rr][c]));
+            }
+            if (lane == 0) {
+                float* dst = p.R + tok * p.dv_ + c0;
+                reinterpret_cast<float4*>(dst)[0] = make_float4(r[0], r[1], r[2], r[3]);
+                reinterpret_cast<float4*>(dst)[1] = make_float4(r[4], r[5], r[6], r[7]);
+            }
+        } else {
+            // G += q^T dO; dr = -k G, dv = u G (sums over rows); G = Diag(a) (G + e^T dr)
+            float z[2 * NC];  // k G | u G
+#pragma unroll
+            for (int c = 0; c < 2 * NC; ++c) z[c] = 0.f;
+#pragma unroll
+            for (int rr = 0; rr < 4; ++rr) {
+                const float u = rw.wg[rr] * rw.k[rr];
+#pragma unroll
+                for (int c = 0; c < NC; ++c) {
+                    X[rr][c] = fmaf(rw.q[rr], cv[c], X[rr][c]);
+                    z[c] = fmaf(rw.k[rr], X[rr][c], z[c]);
+                    z[NC + c] = fmaf(u, X[rr][c], z[NC + c]);
+                }
+            }
+            warp_allsum<2 * NC>(z, lane);
+#pragma unroll
+            for (int rr = 0; rr < 4; ++rr) {
+                const float e = rw.bg[rr] * rw.k[rr];
+#pragma unroll
+                for (int c = 0; c < NC; ++c) X[rr][c] = rw.a[rr] * fmaf(-e, z[c], X[rr][c]);
+            }
+            if (lane == 0) {
+                float* dst = p.DR + tok * p.dv_ + c0;
+                reinterpret_cast<float4*>(dst)[0] = make_float4(-z[0], -z[1], -z[2], -z[3]);
+                reinterpret_cast<float4*>(dst)[1] = make_float4(-z[4], -z[5], -z[6], -z[7]);
+                float* dvp = p.dv + tok * p.dv_ + c0;
+                reinterpret_cast<float4*>(dvp)[0] = make_float4(z[8], z[9], z[10], z[11]);
+                reinterpret_cast<float4*>(dvp)[1] = make_float4(z[12], z[13], z[14], z[15]);
+            }
+        }
+    }
+    if (dir == 1 && p.dS0)
+#pragma unroll
+        for (int rr = 0; rr < 4; ++rr)
+            if (i0 + rr < p.dk_) {
+                float* dst = p.dS0 + (head * p.dk_ + i0 + rr) * p.dv_ + c0;
+                reinterpret_cast<float4*>(dst)[0] = make_float4(X[rr][0], X[rr][1], X[rr][2], X[rr][3]);
+                reinterpret_cast<float4*>(dst)[1] = make_float4(X[rr][4], X[rr][5], X[rr][6], X[rr][7]);
+            }
 }
 
 // ----------------------------------------------------------------- pass 2 --
-struct __align__(16) MainSmem {
-    float4 subck[kNSub][2][2][kRows];     // state at sub-chunk starts: [sub][col half][float4][row]
-    float rch[kC][kNC];                   // r_t of every token of the chunk
-    float red[2 * 2 * 4 * 16];            // row-group partial sums
-    float part[2][kSub][kQty][2][kRows];  // per-row partials: [buffer][token][qty][col half][row]
-    float sred[kSub][3][4];               // scalar-gate totals: [token][gate][warp]
+// CTA (row block, chunk, head). Thread t: row rb * RB + t / tpr, columns
+// 8 (t % tpr) .. + 8, with tpr threads per row (a power of two <= 32, so a
+// row's threads share a warp) and RB = 128 / tpr rows per CTA. A sub-chunk's
+// inputs (row scalars of the CTA's rows, v, dO, r, dr over all columns) are
+// staged in shared memory as fp32 by the whole CTA before it is used.
+struct ChunkSmem {
+    // byte offsets into the dynamic shared memory
+    uint32_t subck, col, row, sred, total;
+    int dvp, RB;
 };
 
-__device__ __forceinline__ void cluster_sync_all() {
-    asm volatile(
-        "barrier.cluster.arrive.release.aligned;\n\t"
-        "barrier.cluster.wait.acquire.aligned;" ::: "memory");
+__host__ __device__ inline ChunkSmem chunk_smem(int tpr) {
+    ChunkSmem m;
+    m.dvp = 8 * tpr;
+    m.RB = kChunkThreads / tpr;
+    m.subck = 0;                                                    // [kNSub][2][128] float4
+    m.col = m.subck + kNSub * 2 * kChunkThreads * 16;               // [4][kSub][dvp] fp32
+    m.row = m.col + 4 * kSub * m.dvp * 4;                           // [kSub][5][RB] fp32
+    m.sred = m.row + kSub * 5 * m.RB * 4;                           // [kSub][3][4] fp32
+    m.total = m.sred + kSub * 3 * (kChunkThreads / 32) * 4;
+    return m;
 }
 
-__device__ __forceinline__ uint32_t map_to_rank(uint32_t local_smem, int rank) {
-    uint32_t r;
-    asm volatile("mapa.shared::cluster.u32 %0, %1, %2;" : "=r"(r) : "r"(local_smem), "r"(rank));
-    return r;
-}
-
-__device__ __forceinline__ float ld_cluster(uint32_t addr) {
-    float v;
-    asm volatile("ld.shared::cluster.f32 %0, [%1];" : "=f"(v) : "r"(addr) : "memory");
-    return v;
-}
+enum { kV = 0, kDO = 1, kR = 2, kDR = 3 };
 
 template <typename TI>
-__global__ void __launch_bounds__(kThreads, 1) bwd_main_kernel(Params p) {
+__global__ void __launch_bounds__(kChunkThreads, 4) bwd_chunk_kernel(Params p) {
     extern __shared__ __align__(16) unsigned char smem_raw[];
-    MainSmem& sm = *reinterpret_cast<MainSmem*>(smem_raw);
-    const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5, rg = warp & 3, cg = warp >> 2;
-    const int i = 32 * rg + lane;
-    const int rank = blockIdx.x, NB = gridDim.x;  // the cluster spans gridDim.x
-    const int b = blockIdx.z, h = blockIdx.y;
-    const int col = kNC * rank + 8 * cg;
-    const size_t head = (size_t)b * p.H + h;
-    const bool row_ok = i < p.dk_;
+    const int tpr = p.tpr;
+    const ChunkSmem L = chunk_smem(tpr);
+    float4* subck = reinterpret_cast<float4*>(smem_raw + L.subck);
+    float* colb = reinterpret_cast<float*>(smem_raw + L.col);
+    float* rowb = reinterpret_cast<float*>(smem_raw + L.row);
+    float* sred = reinterpret_cast<float*>(smem_raw + L.sred);
+    const int dvp = L.dvp, RB = L.RB;
+    auto col_at = [&](int a, int u) { return colb + (a * kSub + u) * dvp; };
+    auto row_at = [&](int u, int qy) { return rowb + (u * 5 + qy) * RB; };
+
+    const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
+    const int g = tid & (tpr - 1), lr = tid / tpr;
+    const int rb = blockIdx.x, c = blockIdx.y;
+    const int bh = blockIdx.z, b = bh / p.H, h = bh % p.H;
+    const size_t head = (size_t)bh;
+    const int i = rb * RB + lr;
+    const int j0 = 8 * g;
+    const bool ok = i < p.dk_ && j0 < p.dv_;
+    const int t0 = c * kC, Lc = min(kC, p.T - t0);
     auto tok_of = [&](int t) { return ((size_t)b * p.T + t) * p.H + h; };
 
-    float G[8];
-    if (p.dST && row_ok) load8f(p.dST + (head * p.dk_ + i) * p.dv_ + col, G);
-    else
-        for (int c = 0; c < 8; ++c) G[c] = 0.f;
-
-    const uint32_t part_local = smem_u32(&sm.part[0][0][0][0][0]);
-    int par = 0, sbuf = 0;
-    for (int c = p.nchunks - 1; c >= 0; --c) {
-        const int t0 = c * kC;
-        const int L = min(kC, p.T - t0);
-        // ---- forward over the chunk from its checkpoint: r_t, sub-chunk states
-        float S[8];
-        if (row_ok) load8f(p.ckpt + (((head * p.nchunks + c) * p.dk_) + i) * p.dv_ + col, S);
-        else
-            for (int cc = 0; cc < 8; ++cc) S[cc] = 0.f;
-        Row nr = load_row<TI>(p, tok_of(t0), i);
-        float nv[8];
-        load8<TI>(p.v, tok_of(t0) * p.dv_ + col, nv);
-        for (int tau = 0; tau < L; ++tau) {
-            const Row rw = nr;
-            float v[8];
-#pragma unroll
-            for (int cc = 0; cc < 8; ++cc) v[cc] = nv[cc];
-            if (tau + 1 < L) {
-                nr = load_row<TI>(p, tok_of(t0 + tau + 1), i);
-                load8<TI>(p.v, tok_of(t0 + tau + 1) * p.dv_ + col, nv);
+    // Stage tokens tau0 .. tau0 + ns - 1 of the chunk: the listed column
+    // arrays (zero beyond d_v) and the row scalars.
+    auto stage = [&](int tau0, int ns, bool bwd) {
+        __syncthreads();  // previous contents fully read
+        const int n4 = dvp / 4;
+        const int narr = bwd ? 4 : 2;
+        for (int idx = tid; idx < narr * kSub * n4; idx += kChunkThreads) {
+            const int ai = idx / (kSub * n4), rem = idx % (kSub * n4);
+            const int u = rem / n4, c4 = 4 * (rem % n4);
+            const int a = bwd ? ai : (ai == 0 ? kV : kR);
+            float x[4] = {0.f, 0.f, 0.f, 0.f};
+            if (u < ns && c4 < p.dv_) {
+                const size_t off = tok_of(t0 + tau0 + u) * p.dv_ + c4;
+                if (a == kV) load4<TI>(p.v, off, x);
+                else if (a == kDO) load4<TI>(p.dO, off, x);
+                else load4<float>(a == kR ? p.R : p.DR, off, x);
             }
-            if (tau % kSub == 0) {
-                sm.subck[tau / kSub][cg][0][i] = make_float4(S[0], S[1], S[2], S[3]);
-                sm.subck[tau / kSub][cg][1][i] = make_float4(S[4], S[5], S[6], S[7]);
-            }
-            float r[8];
-            fwd_step(S, rw, v, sm.red, par, cg, rg, lane, r);
-            par ^= 1;
-            if (rg == 0 && lane == 0) store8(&sm.rch[tau][8 * cg], r);
+            *reinterpret_cast<float4*>(col_at(a, u) + c4) = make_float4(x[0], x[1], x[2], x[3]);
         }
-        __syncthreads();  // rch complete
+        for (int idx = tid; idx < kSub * RB; idx += kChunkThreads) {
+            const int u = idx / RB, r = idx % RB;
+            Row rw{0.f, 0.f, 1.f, 0.f, 0.f};
+            if (u < ns) rw = load_row<TI>(p, tok_of(t0 + tau0 + u), rb * RB + r);
+            row_at(u, 0)[r] = rw.q;
+            row_at(u, 1)[r] = rw.k;
+            row_at(u, 2)[r] = rw.a;
+            row_at(u, 3)[r] = rw.bg;
+            row_at(u, 4)[r] = rw.wg;
+        }
+        __syncthreads();
+    };
+    auto ld8s = [&](const float* src, float (&x)[8]) {
+        const float4 a = reinterpret_cast<const float4*>(src)[0];
+        const float4 bq = reinterpret_cast<const float4*>(src)[1];
+        x[0] = a.x; x[1] = a.y; x[2] = a.z; x[3] = a.w;
+        x[4] = bq.x; x[5] = bq.y; x[6] = bq.z; x[7] = bq.w;
+    };
 
-        // ---- reverse, one sub-chunk at a time
-        const int nsub = (L + kSub - 1) / kSub;
-        for (int s = nsub - 1; s >= 0; --s) {
-            const int tau0 = s * kSub;
-            const int ns = min(kSub, L - tau0);
-            float Sst[kSub][8];  // S_{t-1} of each token of the sub-chunk
-            {
-                const float4 a0 = sm.subck[s][cg][0][i], a1 = sm.subck[s][cg][1][i];
-                S[0] = a0.x; S[1] = a0.y; S[2] = a0.z; S[3] = a0.w;
-                S[4] = a1.x; S[5] = a1.y; S[6] = a1.z; S[7] = a1.w;
-            }
+    float S[8], G[8];
+    {
+        const size_t off = ((head * p.nchunks + c) * p.dk_ + i) * p.dv_ + j0;
+        if (ok) {
+            load8<float>(p.ckS, off, S);
+            load8<float>(p.ckG, off, G);
+        } else {
 #pragma unroll
-            for (int u = 0; u < kSub; ++u) {
-                if (u < ns) {
-#pragma unroll
-                    for (int cc = 0; cc < 8; ++cc) Sst[u][cc] = S[cc];
-                    if (u + 1 < ns) {
-                        const size_t tok = tok_of(t0 + tau0 + u);
-                        const Row rw = load_row<TI>(p, tok, i);
-                        float v[8], r[8];
-                        load8<TI>(p.v, tok * p.dv_ + col, v);
-                        load8f(&sm.rch[tau0 + u][8 * cg], r);
-                        const float uu = rw.wg * rw.k;
-#pragma unroll
-                        for (int cc = 0; cc < 8; ++cc)
-                            S[cc] = fmaf(-rw.k, r[cc], fmaf(uu, v[cc], rw.a * S[cc]));
-                    }
-                }
-            }
-#pragma unroll
-            for (int u = kSub - 1; u >= 0; --u) {
-                if (u < ns) {
-                    const size_t tok = tok_of(t0 + tau0 + u);
-                    const Row rw = load_row<TI>(p, tok, i);
-                    float v[8], d[8], r[8];
-                    load8<TI>(p.v, tok * p.dv_ + col, v);
-                    load8<TI>(p.dO, tok * p.dv_ + col, d);
-                    load8f(&sm.rch[tau0 + u][8 * cg], r);
-                    const float e = rw.bg * rw.k, uu = rw.wg * rw.k;
-                    // o_t = q_t S_t
-                    float pdq = 0.f;
-#pragma unroll
-                    for (int cc = 0; cc < 8; ++cc) {
-                        const float st = fmaf(-rw.k, r[cc], fmaf(uu, v[cc], rw.a * Sst[u][cc]));
-                        pdq = fmaf(st, d[cc], pdq);
-                        G[cc] = fmaf(rw.q, d[cc], G[cc]);
-                    }
-                    // S_t = S' - k^T r + u^T v
-                    float x[16], pdu = 0.f, pdkd = 0.f;
-#pragma unroll
-                    for (int cc = 0; cc < 8; ++cc) {
-                        x[cc] = uu * G[cc];
-                        x[8 + cc] = rw.k * G[cc];
-                        pdu = fmaf(G[cc], v[cc], pdu);
-                        pdkd = fmaf(-G[cc], r[cc], pdkd);
-                    }
-                    colsum_publish<16>(x, sm.red, par, cg, rg, lane);
-                    if (rg == 0 && lane < 8) {
-                        float sv = 0.f;
-#pragma unroll
-                        for (int g = 0; g < 4; ++g) sv += red_at(sm.red, par, cg, g)[lane];
-                        p.dv[tok * p.dv_ + col + lane] = sv;
-                    }
-                    float dr[8];
-                    red_sum8(sm.red, par, cg, 8, dr);
-                    par ^= 1;
-                    // r = e S';  S' = Diag(a) S_{t-1}
-                    float pde = 0.f, pdal = 0.f;
-#pragma unroll
-                    for (int cc = 0; cc < 8; ++cc) {
-                        const float drc = -dr[cc];
-                        pde = fmaf(rw.a * Sst[u][cc], drc, pde);
-                        const float dsd = fmaf(e, drc, G[cc]);
-                        pdal = fmaf(dsd, Sst[u][cc], pdal);
-                        G[cc] = rw.a * dsd;
-                    }
-                    float* pp = &sm.part[sbuf][u][0][cg][i];
-                    pp[0] = pdq;
-                    pp[2 * kRows] = pdkd;
-                    pp[4 * kRows] = pdu;
-                    pp[6 * kRows] = pde;
-                    pp[8 * kRows] = pdal;
-                }
-            }
-            cluster_sync_all();  // this sub-chunk's partials are visible cluster-wide
+            for (int cc = 0; cc < 8; ++cc) S[cc] = G[cc] = 0.f;
+        }
+    }
 
-            // ---- totals over the cluster: CTA `rank` finishes tokens rank, rank + NB, ...
-            if (tid < kRows) {
-                for (int u = rank; u < ns; u += NB) {
-                    float tot[kQty] = {0.f, 0.f, 0.f, 0.f, 0.f};
-                    for (int rk = 0; rk < NB; ++rk) {
-                        const uint32_t base = map_to_rank(part_local, rk);
+    // forward over the chunk: the state at every sub-chunk start
+    const int nsub = (Lc + kSub - 1) / kSub;
+    for (int s = 0; s < nsub; ++s) {
+        const int tau0 = s * kSub, ns = min(kSub, Lc - tau0);
+        subck[(s * 2 + 0) * kChunkThreads + tid] = make_float4(S[0], S[1], S[2], S[3]);
+        subck[(s * 2 + 1) * kChunkThreads + tid] = make_float4(S[4], S[5], S[6], S[7]);
+        if (s == nsub - 1) break;  // the last sub-chunk's start is all the reverse pass needs
+        stage(tau0, ns, false);
 #pragma unroll
-                        for (int qy = 0; qy < kQty; ++qy)
+        for (int u = 0; u < kSub; ++u) {
+            float v[8], r[8];
+            ld8s(col_at(kV, u) + j0, v);
+            ld8s(col_at(kR, u) + j0, r);
+            const float a = row_at(u, 2)[lr], kk = row_at(u, 1)[lr], uu = row_at(u, 4)[lr] * kk;
 #pragma unroll
-                            for (int hc = 0; hc < 2; ++hc) {
-                                const uint32_t off =
-                                    ((((sbuf * kSub + u) * kQty + qy) * 2 + hc) * kRows + tid) * 4u;
-                                tot[qy] += ld_cluster(base + off);
-                            }
-                    }
-                    const size_t tok = tok_of(t0 + tau0 + u);
-                    const Row rw = load_row<TI>(p, tok, tid);
-                    const bool tied = p.wkind == GDR_GATE_TIED;
-                    const float de_b = tot[3] + (tied ? tot[2] : 0.f);  // dL/db through e (and u if tied)
-                    const float g_a = tot[4], g_b = rw.k * de_b, g_w = rw.k * tot[2];
-                    if (tid < p.dk_) {
-                        const size_t gi = tok * p.dk_ + tid;
-                        p.dq[gi] = tot[0];
-                        p.dk[gi] = tot[1] + rw.bg * tot[3] + rw.wg * tot[2];
-                        if (p.akind == GDR_GATE_CHANNEL) p.dalpha[gi] = g_a;
-                        if (p.bkind == GDR_GATE_CHANNEL) p.db[gi] = g_b;
-                        if (p.wkind == GDR_GATE_CHANNEL) p.dw[gi] = g_w;
-                    }
-                    // scalar gates: sum over the key channels (rows beyond d_k hold zeros)
-                    float sc[3] = {g_a, g_b, g_w};
+            for (int cc = 0; cc < 8; ++cc) S[cc] = fmaf(-kk, r[cc], fmaf(uu, v[cc], a * S[cc]));
+        }
+    }
+
+    for (int s = nsub - 1; s >= 0; --s) {
+        const int tau0 = s * kSub, ns = min(kSub, Lc - tau0);
+        stage(tau0, ns, true);
+        float Sst[kSub + 1][8];  // S_{t-1} of each token, then the state after the last one
+        {
+            const float4 a0 = subck[(s * 2 + 0) * kChunkThreads + tid];
+            const float4 a1 = subck[(s * 2 + 1) * kChunkThreads + tid];
+            Sst[0][0] = a0.x; Sst[0][1] = a0.y; Sst[0][2] = a0.z; Sst[0][3] = a0.w;
+            Sst[0][4] = a1.x; Sst[0][5] = a1.y; Sst[0][6] = a1.z; Sst[0][7] = a1.w;
+        }
 #pragma unroll
-                    for (int g = 0; g < 3; ++g)
+        for (int u = 0; u < kSub; ++u) {
+            float v[8], r[8];
+            ld8s(col_at(kV, u) + j0, v);
+            ld8s(col_at(kR, u) + j0, r);
+            const float a = row_at(u, 2)[lr], kk = row_at(u, 1)[lr], uu = row_at(u, 4)[lr] * kk;
 #pragma unroll
-                        for (int o = 16; o >= 1; o >>= 1)
-                            sc[g] += __shfl_xor_sync(0xffffffffu, sc[g], o);
+            for (int cc = 0; cc < 8; ++cc)
+                Sst[u + 1][cc] = fmaf(-kk, r[cc], fmaf(uu, v[cc], a * Sst[u][cc]));
+        }
+#pragma unroll
+        for (int u = kSub - 1; u >= 0; --u) {
+            if (u < ns) {
+                float v[8], d[8], r[8], dr[8];
+                ld8s(col_at(kV, u) + j0, v);
+                ld8s(col_at(kDO, u) + j0, d);
+                ld8s(col_at(kR, u) + j0, r);
+                ld8s(col_at(kDR, u) + j0, dr);
+                const float q = row_at(u, 0)[lr], kk = row_at(u, 1)[lr], a = row_at(u, 2)[lr];
+                const float bg = row_at(u, 3)[lr], wg = row_at(u, 4)[lr];
+                const float e = bg * kk;
+                // partial sums over this thread's 8 columns:
+                // dq (S_t dO^T), dk from r (-G r^T), du (G v^T), de (S' dr^T), dalpha
+                float acc[5] = {0.f, 0.f, 0.f, 0.f, 0.f};
+#pragma unroll
+                for (int cc = 0; cc < 8; ++cc) {
+                    acc[0] = fmaf(Sst[u + 1][cc], d[cc], acc[0]);
+                    G[cc] = fmaf(q, d[cc], G[cc]);
+                    acc[1] = fmaf(-G[cc], r[cc], acc[1]);
+                    acc[2] = fmaf(G[cc], v[cc], acc[2]);
+                    acc[3] = fmaf(a * Sst[u][cc], dr[cc], acc[3]);
+                    const float dsd = fmaf(e, dr[cc], G[cc]);
+                    acc[4] = fmaf(dsd, Sst[u][cc], acc[4]);
+                    G[cc] = a * dsd;
+                }
+                if (!ok)
+#pragma unroll
+                    for (int qy = 0; qy < 5; ++qy) acc[qy] = 0.f;
+                for (int o = 1; o < tpr; o <<= 1)
+#pragma unroll
+                    for (int qy = 0; qy < 5; ++qy) acc[qy] += __shfl_xor_sync(0xffffffffu, acc[qy], o);
+                const bool tied = p.wkind == GDR_GATE_TIED;
+                const float de_b = acc[3] + (tied ? acc[2] : 0.f);
+                float gsc[3] = {acc[4], kk * de_b, kk * acc[2]};  // dalpha, db, dw for row i
+                if (g == 0 && i < p.dk_) {
+                    const size_t gi = tok_of(t0 + tau0 + u) * p.dk_ + i;
+                    p.dq[gi] = acc[0];
+                    p.dk[gi] = acc[1] + bg * acc[3] + wg * acc[2];
+                    if (p.akind == GDR_GATE_CHANNEL) p.dalpha[gi] = gsc[0];
+                    if (p.bkind == GDR_GATE_CHANNEL) p.db[gi] = gsc[1];
+                    if (p.wkind == GDR_GATE_CHANNEL) p.dw[gi] = gsc[2];
+                }
+                if (p.GP) {  // scalar gates: this warp's rows, summed
+                    if (g != 0 || i >= p.dk_)
+#pragma unroll
+                        for (int qy = 0; qy < 3; ++qy) gsc[qy] = 0.f;
+                    for (int o = tpr; o < 32; o <<= 1)
+#pragma unroll
+                        for (int qy = 0; qy < 3; ++qy) gsc[qy] += __shfl_xor_sync(0xffffffffu, gsc[qy], o);
                     if (lane == 0)
 #pragma unroll
-                        for (int g = 0; g < 3; ++g) sm.sred[u][g][warp] = sc[g];
+                        for (int qy = 0; qy < 3; ++qy) sred[(u * 3 + qy) * (kChunkThreads / 32) + warp] = gsc[qy];
                 }
             }
+        }
+        if (p.GP) {  // the CTA's partial sum per token and scalar gate
             __syncthreads();
             if (tid < kSub * 3) {
-                const int u = tid / 3, g = tid % 3;
-                const int kind = g == 0 ? p.akind : g == 1 ? p.bkind : p.wkind;
-                if (u < ns && u % NB == rank && kind == GDR_GATE_SCALAR) {
-                    const float sv = sm.sred[u][g][0] + sm.sred[u][g][1] + sm.sred[u][g][2] +
-                                     sm.sred[u][g][3];
-                    float* dst = g == 0 ? p.dalpha : g == 1 ? p.db : p.dw;
-                    dst[tok_of(t0 + tau0 + u)] = sv;
+                const int u = tid / 3, qy = tid % 3;
+                if (u < ns) {
+                    float sv = 0.f;
+#pragma unroll
+                    for (int w = 0; w < kChunkThreads / 32; ++w) sv += sred[(u * 3 + qy) * (kChunkThreads / 32) + w];
+                    const size_t BTH = (size_t)p.B * p.T * p.H;
+                    p.GP[((size_t)qy * p.nrb + rb) * BTH + tok_of(t0 + tau0 + u)] = sv;
                 }
             }
-            sbuf ^= 1;
         }
-        __syncthreads();  // rch and subck are rewritten by the next chunk
     }
-    if (p.dS0 && row_ok) store8(p.dS0 + (head * p.dk_ + i) * p.dv_ + col, G);
-    cluster_sync_all();  // no CTA leaves while a peer may still read its partials
 }
 
-size_t ckpt_bytes(int B, int T, int H, int dk, int dv) {
-    if (T <= 0) return 0;
+// ----------------------------------------------------------------- pass 3 --
+__global__ void bwd_gate_sum_kernel(Params p) {
+    const size_t BTH = (size_t)p.B * p.T * p.H;
+    const size_t n = blockIdx.x * (size_t)blockDim.x + threadIdx.x;
+    if (n >= BTH) return;
+    const int kinds[3] = {p.akind, p.bkind, p.wkind};
+    float* dst[3] = {p.dalpha, p.db, p.dw};
+#pragma unroll
+    for (int qy = 0; qy < 3; ++qy) {
+        if (kinds[qy] != GDR_GATE_SCALAR) continue;
+        float s = 0.f;
+        for (int rb = 0; rb < p.nrb; ++rb) s += p.GP[((size_t)qy * p.nrb + rb) * BTH + n];
+        dst[qy][n] = s;
+    }
+}
+
+int threads_per_row(int dv) {
+    int t = 1;
+    while (8 * t < dv) t <<= 1;
+    return t;
+}
+
+size_t round256(size_t x) { return (x + 255) & ~size_t(255); }
+
+struct WsLayout {
+    size_t ckS, ckG, R, DR, GP, total;
+};
+
+WsLayout ws_layout(int B, int T, int H, int dk, int dv) {
+    WsLayout l{};
     const size_t nch = (size_t)(T + kC - 1) / kC;
-    return (size_t)B * H * nch * dk * dv * sizeof(float);
+    const size_t ck = round256((size_t)B * H * nch * dk * dv * sizeof(float));
+    const size_t rr = round256((size_t)B * T * H * dv * sizeof(float));
+    const int nrb = (dk + kChunkThreads / threads_per_row(dv) - 1) / (kChunkThreads / threads_per_row(dv));
+    const size_t gp = round256((size_t)3 * nrb * B * T * H * sizeof(float));
+    l.ckS = 0;
+    l.ckG = l.ckS + ck;
+    l.R = l.ckG + ck;
+    l.DR = l.R + rr;
+    l.GP = l.DR + rr;
+    l.total = l.GP + gp;
+    return l;
 }
 
 template <typename TI>
-cudaError_t launch_typed(const Params& p, int B, int H, cudaStream_t st) {
-    const int NB = p.dv_ / kNC;
-    bwd_ckpt_kernel<TI><<<dim3(NB, H, B), kThreads, 0, st>>>(p);
+cudaError_t launch_typed(Params p, cudaStream_t st) {
+    bwd_scan_kernel<TI><<<dim3((p.dv_ + kScanCols * kScanWarps - 1) / (kScanCols * kScanWarps), p.H, 2 * p.B),
+                          kScanWarps * 32, 0, st>>>(p);
     cudaError_t e = cudaGetLastError();
     if (e != cudaSuccess) return e;
-    const size_t smem = sizeof(MainSmem);
-    e = cudaFuncSetAttribute(bwd_main_kernel<TI>, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                             (int)smem);
+    const uint32_t smem = chunk_smem(p.tpr).total;
+    void (*kern)(Params) = bwd_chunk_kernel<TI>;
+    e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
     if (e != cudaSuccess) return e;
-    cudaLaunchConfig_t cfg = {};
-    cfg.gridDim = dim3(NB, H, B);
-    cfg.blockDim = dim3(kThreads, 1, 1);
-    cfg.dynamicSmemBytes = smem;
-    cfg.stream = st;
-    cudaLaunchAttribute attr[1];
-    attr[0].id = cudaLaunchAttributeClusterDimension;
-    attr[0].val.clusterDim.x = NB;
-    attr[0].val.clusterDim.y = 1;
-    attr[0].val.clusterDim.z = 1;
-    cfg.attrs = attr;
-    cfg.numAttrs = 1;
-    return cudaLaunchKernelEx(&cfg, bwd_main_kernel<TI>, p);
+    kern<<<dim3(p.nrb, p.nchunks, p.B * p.H), kChunkThreads, smem, st>>>(p);
+    e = cudaGetLastError();
+    if (e != cudaSuccess || !p.GP) return e;
+    const size_t BTH = (size_t)p.B * p.T * p.H;
+    bwd_gate_sum_kernel<<<(unsigned)((BTH + 255) / 256), 256, 0, st>>>(p);
+    return cudaGetLastError();
 }
 
 }  // namespace bwd
@@ -484,7 +591,7 @@ extern "C" {
 
 size_t gdr_chunk_bwd_workspace_size(int B, int T, int H, int d_k, int d_v) {
     if (B < 1 || H < 1 || T < 1 || d_k < 1 || d_v < 1) return 0;
-    return gdr::bwd::ckpt_bytes(B, T, H, d_k, d_v);
+    return gdr::bwd::ws_layout(B, T, H, d_k, d_v).total;
 }
 
 gdr_status gdr_chunk_bwd(const void* q, const void* k, const void* v, const void* alpha,
@@ -507,8 +614,7 @@ gdr_status gdr_chunk_bwd(const void* q, const void* k, const void* v, const void
         return GDR_ERR_INVALID_ARG;
     if (T > 0 && (!q || !k || !v || !dO || !dq || !dk || !dv)) return GDR_ERR_INVALID_ARG;
     if (chunk != 64) return GDR_ERR_UNSUPPORTED;
-    if (d_k > gdr::bwd::kRows || d_v % gdr::bwd::kNC != 0 ||
-        d_v > gdr::bwd::kNC * gdr::bwd::kMaxNB)
+    if (d_k > gdr::bwd::kMaxDK || d_v % 8 != 0 || d_v > gdr::bwd::kMaxDV)
         return GDR_ERR_UNSUPPORTED;
     cudaStream_t st = reinterpret_cast<cudaStream_t>(stream);
     const size_t state_bytes = (size_t)B * H * d_k * d_v * sizeof(float);
@@ -518,23 +624,35 @@ gdr_status gdr_chunk_bwd(const void* q, const void* k, const void* v, const void
                              : cudaMemsetAsync(dS0, 0, state_bytes, st);
         return e == cudaSuccess ? GDR_OK : GDR_ERR_LAUNCH;
     }
+    const int nch = (T + gdr::bwd::kC - 1) / gdr::bwd::kC;
+    if (nch > 65535 || (size_t)B * H > 65535u) return GDR_ERR_UNSUPPORTED;  // grid limits
     const void* ptrs[] = {q, k, v, dO, dq, dk, dv, S0, dS_T, dS0, dalpha, db, dw, alpha, b, w};
     for (const void* p : ptrs)
         if (p && !a16(p)) return GDR_ERR_MISALIGNED;
-    if (!workspace || workspace_bytes < gdr_chunk_bwd_workspace_size(B, T, H, d_k, d_v))
-        return GDR_ERR_INVALID_ARG;
+    const gdr::bwd::WsLayout wl = gdr::bwd::ws_layout(B, T, H, d_k, d_v);
+    if (!workspace || workspace_bytes < wl.total) return GDR_ERR_INVALID_ARG;
     if ((reinterpret_cast<uintptr_t>(workspace) & 255u) != 0) return GDR_ERR_MISALIGNED;
 
+    unsigned char* ws = static_cast<unsigned char*>(workspace);
     gdr::bwd::Params p;
     p.q = q; p.k = k; p.v = v; p.alpha = alpha; p.b = b; p.w = w; p.dO = dO;
     p.S0 = S0; p.dST = dS_T;
     p.dq = dq; p.dk = dk; p.dv = dv; p.dalpha = dalpha; p.db = db; p.dw = dw; p.dS0 = dS0;
-    p.ckpt = static_cast<float*>(workspace);
-    p.T = T; p.H = H; p.dk_ = d_k; p.dv_ = d_v;
+    p.ckS = reinterpret_cast<float*>(ws + wl.ckS);
+    p.ckG = reinterpret_cast<float*>(ws + wl.ckG);
+    p.R = reinterpret_cast<float*>(ws + wl.R);
+    p.DR = reinterpret_cast<float*>(ws + wl.DR);
+    const bool any_scalar = alpha_kind == GDR_GATE_SCALAR || b_kind == GDR_GATE_SCALAR ||
+                            w_kind == GDR_GATE_SCALAR;
+    p.GP = any_scalar ? reinterpret_cast<float*>(ws + wl.GP) : nullptr;
+    p.B = B; p.T = T; p.H = H; p.dk_ = d_k; p.dv_ = d_v;
     p.akind = alpha_kind; p.bkind = b_kind; p.wkind = w_kind;
-    p.nchunks = (T + gdr::bwd::kC - 1) / gdr::bwd::kC;
-    const cudaError_t e = dtype == GDR_BF16 ? gdr::bwd::launch_typed<__nv_bfloat16>(p, B, H, st)
-                                            : gdr::bwd::launch_typed<float>(p, B, H, st);
+    p.nchunks = nch;
+    p.tpr = gdr::bwd::threads_per_row(d_v);
+    const int RB = gdr::bwd::kChunkThreads / p.tpr;
+    p.nrb = (d_k + RB - 1) / RB;
+    const cudaError_t e = dtype == GDR_BF16 ? gdr::bwd::launch_typed<__nv_bfloat16>(p, st)
+                                            : gdr::bwd::launch_typed<float>(p, st);
     return e == cudaSuccess ? GDR_OK : GDR_ERR_LAUNCH;
 }
 

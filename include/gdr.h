@@ -225,16 +225,20 @@ size_t gdr_chunk_fwd_static_capacity(void);
  *   the gate has no data of its own (kind NONE, or w TIED); dS0
  *   [B, H, d_k, d_v] or NULL (not written).
  * workspace: caller-owned device scratch of at least
- *   gdr_chunk_bwd_workspace_size() bytes, 256-byte aligned (the forward
- *   state at the start of every 64-token chunk, fp32).
- * Method: fp32 arithmetic for both dtypes. A first kernel runs the forward
- *   and stores the chunk-start states; a second walks the chunks backwards,
- *   recomputing each chunk's states from its checkpoint, with one
- *   thread-block cluster of d_v / 16 CTAs per head (16 state columns each)
- *   adding the per-row partial sums over columns through distributed shared
- *   memory. d_status is not used (no bounded waits on this path).
- * Supported: chunk = 64, 1 <= d_k <= 128, d_v a multiple of 16 up to 128.
- *   Every pointer 16-byte aligned.
+ *   gdr_chunk_bwd_workspace_size() bytes, 256-byte aligned; contents on
+ *   entry ignored, on exit undefined.
+ * Method: fp32 arithmetic for both dtypes. The state gradient G follows its
+ *   own backward recurrence G_{t-1} = Diag(alpha_t)(I - e^T k) G_t +
+ *   q_{t-1}^T dO_{t-1}, which does not involve S, so a first kernel scans the
+ *   tokens forward (S at every 64-token chunk start, r_t) and backward (G at
+ *   every chunk end, dr_t = -k G, dv_t, dS0) at the same time, one warp per
+ *   4 state columns; a second kernel, parallel over chunks, heads and blocks
+ *   of state rows, rebuilds each chunk's states from those and forms dq, dk
+ *   and the gate gradients; a third sums scalar gates' gradients over the
+ *   key channels. Deterministic (no atomics). d_status is not used (no
+ *   bounded waits on this path).
+ * Supported: chunk = 64, 1 <= d_k <= 128, d_v a multiple of 8 up to 256,
+ *   ceil(T / 64) <= 65535 and B * H <= 65535. Every pointer 16-byte aligned.
  * Returns GDR_OK, GDR_ERR_INVALID_ARG (bad sizes or kinds, a NULL array that
  * is required, a gradient pointer that does not match its gate, workspace
  * missing or too small), GDR_ERR_UNSUPPORTED, GDR_ERR_MISALIGNED or
@@ -251,8 +255,11 @@ gdr_status gdr_chunk_bwd(const void* q, const void* k, const void* v,
                          int B, int T, int H, int d_k, int d_v, int chunk,
                          int dtype, int* d_status, void* stream);
 
-/* Bytes of workspace gdr_chunk_bwd needs: B * H * ceil(T / 64) * d_k * d_v *
- * 4 (0 for T < 1 or bad sizes). Host-only; launches nothing. */
+/* Bytes of workspace gdr_chunk_bwd needs (0 for T < 1 or bad sizes): fp32
+ * chunk-start states and chunk-end state gradients (2 x B H ceil(T/64) d_k
+ * d_v), r_t and dr_t of every token (2 x B T H d_v), and scalar-gate partial
+ * sums (3 x ceil(d_k / RB) x B T H, RB = 128 / (d_v / 8 rounded up to a power
+ * of two)), each rounded up to 256 bytes. Host-only; launches nothing. */
 size_t gdr_chunk_bwd_workspace_size(int B, int T, int H, int d_k, int d_v);
 
 /*

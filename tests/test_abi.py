@@ -159,8 +159,8 @@ def bwd(**kw):
     (dict(ws_bytes=1024), _lib.GDR_ERR_INVALID_ARG),     # workspace too small
     (dict(chunk=32), _lib.GDR_ERR_UNSUPPORTED),
     (dict(dk=256), _lib.GDR_ERR_UNSUPPORTED),
-    (dict(dv=144), _lib.GDR_ERR_UNSUPPORTED),
-    (dict(dv=40), _lib.GDR_ERR_UNSUPPORTED),
+    (dict(dv=264), _lib.GDR_ERR_UNSUPPORTED),
+    (dict(dv=44), _lib.GDR_ERR_UNSUPPORTED),
     (dict(dO=P + 8), _lib.GDR_ERR_MISALIGNED),
     (dict(dS0=P + 4), _lib.GDR_ERR_MISALIGNED),
     (dict(ws=P + 16), _lib.GDR_ERR_MISALIGNED),
@@ -169,9 +169,16 @@ def test_chunk_bwd_rejects_bad_arguments(kw, expect):
     assert bwd(**kw) == expect
 
 
+def r256(x):
+    return (x + 255) // 256 * 256
+
+
 @pytest.mark.parametrize("shape,expect", [
-    ((4, 4096, 16, 128, 128), 4 * 16 * 64 * 128 * 128 * 4),
-    ((1, 65, 2, 64, 32), 1 * 2 * 2 * 64 * 32 * 4),
+    # checkpoints of S and G, r and dr per token, scalar-gate partials (16 row blocks of 8)
+    ((4, 4096, 16, 128, 128), 2 * 4 * 16 * 64 * 128 * 128 * 4 + 2 * 4 * 4096 * 16 * 128 * 4
+     + 3 * 16 * 4 * 4096 * 16 * 4),
+    # d_v = 32: 4 threads per row, 32 rows per block, 2 blocks
+    ((1, 65, 2, 64, 32), 2 * 2 * 2 * 64 * 32 * 4 + 2 * r256(65 * 2 * 32 * 4) + r256(3 * 2 * 65 * 2 * 4)),
     ((1, 0, 2, 64, 32), 0),
 ])
 def test_bwd_workspace_size(shape, expect):

@@ -79,9 +79,11 @@ def test_ragged_lengths(cuda_device, T):
     check(run_bwd(inp, cot, cuda_device), run_oracle_bwd(inp, cot), f"T={T} ")
 
 
-@pytest.mark.parametrize("dk,dv", [(128, 64), (64, 128), (40, 48), (16, 16), (100, 112), (128, 16)])
+@pytest.mark.parametrize("dk,dv", [(128, 64), (64, 128), (40, 48), (16, 16), (100, 112), (128, 8),
+                                   (128, 256), (7, 24)])
 def test_head_shapes(cuda_device, dk, dv):
-    """Cluster sizes 1 to 8 (d_v / 16) and rows beyond d_k left idle."""
+    """1 to 32 threads per state row (d_v / 8), some of them idle, and row
+    blocks that run past d_k."""
     wl = WORKLOADS["kda"].with_(B=1, H=3, T=90, dk=dk, dv=dv, dtype="fp32", s0=True, seed=dk + dv)
     inp = make_chunk_inputs(wl)
     cot = make_cotangents(wl)
