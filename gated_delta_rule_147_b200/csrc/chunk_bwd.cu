@@ -355,25 +355,28 @@ __global__ void __launch_bounds__(kChunkThreads, 4) bwd_chunk_kernel(Params p) {
     // arrays (zero beyond d_v) and the row scalars.
     auto stage = [&](int tau0, int ns, bool bwd) {
         __syncthreads();  // previous contents fully read
-        const int n4 = dvp / 4;
+        const int n4 = dvp / 4;  // float4 per token row (a power of two, as is RB)
+        const int lg_n4 = __ffs(n4) - 1, lg_rb = __ffs(RB) - 1;
+        const size_t tok0 = tok_of(t0 + tau0);  // token u of the sub-chunk: tok0 + u H
         const int narr = bwd ? 4 : 2;
-        for (int idx = tid; idx < narr * kSub * n4; idx += kChunkThreads) {
-            const int ai = idx / (kSub * n4), rem = idx % (kSub * n4);
-            const int u = rem / n4, c4 = 4 * (rem % n4);
+        for (int ai = 0; ai < narr; ++ai) {
             const int a = bwd ? ai : (ai == 0 ? kV : kR);
-            float x[4] = {0.f, 0.f, 0.f, 0.f};
-            if (u < ns && c4 < p.dv_) {
-                const size_t off = tok_of(t0 + tau0 + u) * p.dv_ + c4;
-                if (a == kV) load4<TI>(p.v, off, x);
-                else if (a == kDO) load4<TI>(p.dO, off, x);
-                else load4<float>(a == kR ? p.R : p.DR, off, x);
+            for (int idx = tid; idx < (kSub << lg_n4); idx += kChunkThreads) {
+                const int u = idx >> lg_n4, c4 = (idx & (n4 - 1)) << 2;
+                float x[4] = {0.f, 0.f, 0.f, 0.f};
+                if (u < ns && c4 < p.dv_) {
+                    const size_t off = (tok0 + (size_t)u * p.H) * p.dv_ + c4;
+                    if (a == kV) load4<TI>(p.v, off, x);
+                    else if (a == kDO) load4<TI>(p.dO, off, x);
+                    else load4<float>(a == kR ? p.R : p.DR, off, x);
+                }
+                *reinterpret_cast<float4*>(col_at(a, u) + c4) = make_float4(x[0], x[1], x[2], x[3]);
             }
-            *reinterpret_cast<float4*>(col_at(a, u) + c4) = make_float4(x[0], x[1], x[2], x[3]);
         }
-        for (int idx = tid; idx < kSub * RB; idx += kChunkThreads) {
-            const int u = idx / RB, r = idx % RB;
+        for (int idx = tid; idx < (kSub << lg_rb); idx += kChunkThreads) {
+            const int u = idx >> lg_rb, r = idx & (RB - 1);
             Row rw{0.f, 0.f, 1.f, 0.f, 0.f};
-            if (u < ns) rw = load_row<TI>(p, tok_of(t0 + tau0 + u), rb * RB + r);
+            if (u < ns) rw = load_row<TI>(p, tok0 + (size_t)u * p.H, rb * RB + r);
             row_at(u, 0)[r] = rw.q;
             row_at(u, 1)[r] = rw.k;
             row_at(u, 2)[r] = rw.a;
@@ -468,9 +471,30 @@ __global__ void __launch_bounds__(kChunkThreads, 4) bwd_chunk_kernel(Params p) {
                 if (!ok)
 #pragma unroll
                     for (int qy = 0; qy < 5; ++qy) acc[qy] = 0.f;
-                for (int o = 1; o < tpr; o <<= 1)
+                if (tpr == 16) {
+                    // reduce-scatter over the row's 16 lanes (8 slots, 5 used):
+                    // lane g ends with the total of slot (g >> 1), then each
+                    // total is fetched from its owner
+                    float y[8] = {acc[0], acc[1], acc[2], acc[3], acc[4], 0.f, 0.f, 0.f};
 #pragma unroll
-                    for (int qy = 0; qy < 5; ++qy) acc[qy] += __shfl_xor_sync(0xffffffffu, acc[qy], o);
+                    for (int o = 8, half = 4; half >= 1; o >>= 1, half >>= 1) {
+                        const bool hi = (g & o) != 0;
+#pragma unroll
+                        for (int v = 0; v < half; ++v) {
+                            const float send = hi ? y[v] : y[v + half];
+                            const float keep = hi ? y[v + half] : y[v];
+                            y[v] = keep + __shfl_xor_sync(0xffffffffu, send, o);
+                        }
+                    }
+                    const float tot = y[0] + __shfl_xor_sync(0xffffffffu, y[0], 1);
+                    const int base = lane & ~15;
+#pragma unroll
+                    for (int qy = 0; qy < 5; ++qy) acc[qy] = __shfl_sync(0xffffffffu, tot, base + 2 * qy);
+                } else {
+                    for (int o = 1; o < tpr; o <<= 1)
+#pragma unroll
+                        for (int qy = 0; qy < 5; ++qy) acc[qy] += __shfl_xor_sync(0xffffffffu, acc[qy], o);
+                }
                 const bool tied = p.wkind == GDR_GATE_TIED;
                 const float de_b = acc[3] + (tied ? acc[2] : 0.f);
                 float gsc[3] = {acc[4], kk * de_b, kk * acc[2]};  // dalpha, db, dw for row i
