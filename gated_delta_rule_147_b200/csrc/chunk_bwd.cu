@@ -301,6 +301,244 @@ __global__ void __launch_bounds__(kScanWarps * 32) bwd_scan_kernel(Params p) {
             }
 }
 
+// Staged form of pass 1, used when a token's d_k-row of q / k / channel gate
+// is a whole number of 16-byte pieces: the CTA's four warps (one head, 32
+// columns) share the row scalars, so the CTA copies blocks of kNT tokens
+// into shared memory with cp.async, one block ahead of the one it computes
+// (double buffer), instead of every lane loading its rows per token.
+constexpr int kNT = 8;
+
+template <typename TI>
+struct ScanStage {
+    TI rows[5][kNT][kMaxDK];                  // q, k, alpha, b, w (channel kinds)
+    TI cols[kNT][kScanWarps * kScanCols];     // v (forward) or dO (backward)
+    float scal[3][kNT];                       // scalar alpha, b, w
+};
+
+__device__ __forceinline__ void cp_async16(void* smem, const void* gmem) {
+    asm volatile("cp.async.cg.shared.global [%0], [%1], 16;" ::"r"(smem_u32(smem)), "l"(gmem)
+                 : "memory");
+}
+__device__ __forceinline__ void cp_async_commit() { asm volatile("cp.async.commit_group;" ::: "memory"); }
+__device__ __forceinline__ void cp_async_wait_prev() {  // all but the most recent group landed
+    asm volatile("cp.async.wait_group 1;" ::: "memory");
+}
+
+template <typename TI>
+__device__ __forceinline__ void lds4(const TI* src, float (&x)[4]);
+template <>
+__device__ __forceinline__ void lds4<float>(const float* src, float (&x)[4]) {
+    const float4 a = *reinterpret_cast<const float4*>(src);
+    x[0] = a.x; x[1] = a.y; x[2] = a.z; x[3] = a.w;
+}
+template <>
+__device__ __forceinline__ void lds4<__nv_bfloat16>(const __nv_bfloat16* src, float (&x)[4]) {
+    const uint2 u = *reinterpret_cast<const uint2*>(src);
+    x[0] = __uint_as_float(u.x << 16); x[1] = __uint_as_float(u.x & 0xffff0000u);
+    x[2] = __uint_as_float(u.y << 16); x[3] = __uint_as_float(u.y & 0xffff0000u);
+}
+
+template <typename TI>
+__global__ void __launch_bounds__(kScanWarps * 32) bwd_scan_staged_kernel(Params p) {
+    constexpr int NC = kScanCols, CTA_COLS = kScanWarps * kScanCols;
+    __shared__ __align__(16) ScanStage<TI> stg[2];
+    const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
+    const int cb = CTA_COLS * blockIdx.x;  // the CTA's first column
+    const int c0 = cb + NC * warp;
+    const bool active = c0 < p.dv_;       // idle warps still copy and meet the barriers
+    const int ncols = min(CTA_COLS, p.dv_ - cb);
+    const int b = blockIdx.z >> 1, dir = blockIdx.z & 1, h = blockIdx.y;
+    const size_t head = (size_t)b * p.H + h;
+    const int i0 = 4 * lane;
+    const bool rows_ok = i0 < p.dk_;       // d_k is a multiple of 4 here
+    auto tok_of = [&](int t) { return ((size_t)b * p.T + t) * p.H + h; };
+    auto tok_n = [&](int n) { return tok_of(dir == 0 ? n : p.T - 1 - n); };
+    const void* colsrc = dir == 0 ? p.v : p.dO;
+    // vectors copied per token: q (backward only), k, and the channel gates
+    const void* vsrc[5] = {p.q, p.k, p.alpha, p.b, p.w};
+    bool vneed[5] = {dir == 1, true, p.akind == GDR_GATE_CHANNEL, p.bkind == GDR_GATE_CHANNEL,
+                     p.wkind == GDR_GATE_CHANNEL};
+    constexpr int EPC = 16 / sizeof(TI);  // elements per 16-byte piece
+    const int row_pieces = p.dk_ / EPC, col_pieces = ncols / EPC;
+
+    auto issue = [&](int blk, int buf) {
+        const int n0 = blk * kNT, nt = min(kNT, p.T - n0);
+        for (int vi = 0; vi < 5; ++vi) {
+            if (!vneed[vi]) continue;
+            for (int idx = tid; idx < nt * row_pieces; idx += kScanWarps * 32) {
+                const int tt = idx / row_pieces, pc = idx % row_pieces;
+                cp_async16(&stg[buf].rows[vi][tt][pc * EPC],
+                           static_cast<const TI*>(vsrc[vi]) + tok_n(n0 + tt) * p.dk_ + pc * EPC);
+            }
+        }
+        for (int idx = tid; idx < nt * col_pieces; idx += kScanWarps * 32) {
+            const int tt = idx / col_pieces, pc = idx % col_pieces;
+            cp_async16(&stg[buf].cols[tt][pc * EPC],
+                       static_cast<const TI*>(colsrc) + tok_n(n0 + tt) * p.dv_ + cb + pc * EPC);
+        }
+        cp_async_commit();
+    };
+    // scalar gates: thread tt < kNT loads token tt of a block into registers
+    auto load_scal = [&](int blk, float (&sc)[3]) {
+        const int n = blk * kNT + tid;
+        sc[0] = 1.f; sc[1] = 0.f; sc[2] = 1.f;
+        if (tid < kNT && n < p.T) {
+            const size_t tok = tok_n(n);
+            if (p.akind == GDR_GATE_SCALAR) sc[0] = ld1<TI>(p.alpha, tok);
+            if (p.bkind == GDR_GATE_SCALAR) sc[1] = ld1<TI>(p.b, tok);
+            if (p.wkind == GDR_GATE_SCALAR) sc[2] = ld1<TI>(p.w, tok);
+        }
+    };
+    auto store_scal = [&](int buf, const float (&sc)[3]) {
+        if (tid < kNT)
+#pragma unroll
+            for (int g = 0; g < 3; ++g) stg[buf].scal[g][tid] = sc[g];
+    };
+
+    float X[4][NC];
+    const float* init = dir == 0 ? p.S0 : p.dST;
+#pragma unroll
+    for (int rr = 0; rr < 4; ++rr) {
+        if (active && init && i0 + rr < p.dk_)
+            load8<float>(init, (head * p.dk_ + i0 + rr) * p.dv_ + c0, X[rr]);
+        else
+            for (int c = 0; c < NC; ++c) X[rr][c] = 0.f;
+    }
+
+    const int nblk = (p.T + kNT - 1) / kNT;
+    {
+        float sc[3];
+        load_scal(0, sc);
+        store_scal(0, sc);
+    }
+    issue(0, 0);
+    for (int blk = 0; blk < nblk; ++blk) {
+        const int buf = blk & 1;
+        float scn[3];
+        if (blk + 1 < nblk) {
+            issue(blk + 1, buf ^ 1);
+            load_scal(blk + 1, scn);
+        } else {
+            cp_async_commit();  // empty group keeps the wait count uniform
+        }
+        cp_async_wait_prev();
+        __syncthreads();  // block blk visible to every thread
+        const ScanStage<TI>& S_ = stg[buf];
+        const int n0 = blk * kNT, nt = min(kNT, p.T - n0);
+        if (active) {
+            for (int tt = 0; tt < nt; ++tt) {
+                const int t = dir == 0 ? n0 + tt : p.T - 1 - (n0 + tt);
+                const size_t tok = tok_of(t);
+                const bool store_ck = dir == 0 ? (t % kC == 0) : (t == p.T - 1 || (t + 1) % kC == 0);
+                if (store_ck)
+#pragma unroll
+                    for (int rr = 0; rr < 4; ++rr)
+                        if (i0 + rr < p.dk_) {
+                            float* dst = (dir == 0 ? p.ckS : p.ckG) +
+                                  ((head * p.nchunks + t / kC) * p.dk_ + i0 + rr) * p.dv_ + c0;
+                            reinterpret_cast<float4*>(dst)[0] = make_float4(X[rr][0], X[rr][1], X[rr][2], X[rr][3]);
+                            reinterpret_cast<float4*>(dst)[1] = make_float4(X[rr][4], X[rr][5], X[rr][6], X[rr][7]);
+                        }
+                Rows4 rw;
+                if (rows_ok) {
+                    if (dir == 1) lds4<TI>(&S_.rows[0][tt][i0], rw.q);
+                    lds4<TI>(&S_.rows[1][tt][i0], rw.k);
+                    if (vneed[2]) lds4<TI>(&S_.rows[2][tt][i0], rw.a);
+                    else rw.a[0] = rw.a[1] = rw.a[2] = rw.a[3] = S_.scal[0][tt];
+                    if (vneed[3]) lds4<TI>(&S_.rows[3][tt][i0], rw.bg);
+                    else rw.bg[0] = rw.bg[1] = rw.bg[2] = rw.bg[3] = S_.scal[1][tt];
+                    if (p.wkind == GDR_GATE_TIED) {
+#pragma unroll
+                        for (int rr = 0; rr < 4; ++rr) rw.wg[rr] = rw.bg[rr];
+                    } else if (vneed[4]) lds4<TI>(&S_.rows[4][tt][i0], rw.wg);
+                    else rw.wg[0] = rw.wg[1] = rw.wg[2] = rw.wg[3] = S_.scal[2][tt];
+                    if (dir == 0) rw.q[0] = rw.q[1] = rw.q[2] = rw.q[3] = 0.f;
+                } else {
+#pragma unroll
+                    for (int rr = 0; rr < 4; ++rr) {
+                        rw.q[rr] = rw.k[rr] = rw.bg[rr] = rw.wg[rr] = 0.f;
+                        rw.a[rr] = 1.f;
+                    }
+                }
+                float cv[NC];
+                {
+                    float a4[4], b4[4];
+                    lds4<TI>(&S_.cols[tt][NC * warp], a4);
+                    lds4<TI>(&S_.cols[tt][NC * warp + 4], b4);
+#pragma unroll
+                    for (int c = 0; c < 4; ++c) { cv[c] = a4[c]; cv[4 + c] = b4[c]; }
+                }
+                if (dir == 0) {
+                    float r[NC];
+#pragma unroll
+                    for (int c = 0; c < NC; ++c) r[c] = 0.f;
+#pragma unroll
+                    for (int rr = 0; rr < 4; ++rr) {
+                        const float e = rw.bg[rr] * rw.k[rr];
+#pragma unroll
+                        for (int c = 0; c < NC; ++c) {
+                            X[rr][c] *= rw.a[rr];
+                            r[c] = fmaf(e, X[rr][c], r[c]);
+                        }
+                    }
+                    warp_allsum<NC>(r, lane);
+#pragma unroll
+                    for (int rr = 0; rr < 4; ++rr) {
+                        const float u = rw.wg[rr] * rw.k[rr];
+#pragma unroll
+                        for (int c = 0; c < NC; ++c)
+                            X[rr][c] = fmaf(-rw.k[rr], r[c], fmaf(u, cv[c], X[rr][c]));
+                    }
+                    if (lane == 0) {
+                        float* dst = p.R + tok * p.dv_ + c0;
+                        reinterpret_cast<float4*>(dst)[0] = make_float4(r[0], r[1], r[2], r[3]);
+                        reinterpret_cast<float4*>(dst)[1] = make_float4(r[4], r[5], r[6], r[7]);
+                    }
+                } else {
+                    float z[2 * NC];
+#pragma unroll
+                    for (int c = 0; c < 2 * NC; ++c) z[c] = 0.f;
+#pragma unroll
+                    for (int rr = 0; rr < 4; ++rr) {
+                        const float u = rw.wg[rr] * rw.k[rr];
+#pragma unroll
+                        for (int c = 0; c < NC; ++c) {
+                            X[rr][c] = fmaf(rw.q[rr], cv[c], X[rr][c]);
+                            z[c] = fmaf(rw.k[rr], X[rr][c], z[c]);
+                            z[NC + c] = fmaf(u, X[rr][c], z[NC + c]);
+                        }
+                    }
+                    warp_allsum<2 * NC>(z, lane);
+#pragma unroll
+                    for (int rr = 0; rr < 4; ++rr) {
+                        const float e = rw.bg[rr] * rw.k[rr];
+#pragma unroll
+                        for (int c = 0; c < NC; ++c) X[rr][c] = rw.a[rr] * fmaf(-e, z[c], X[rr][c]);
+                    }
+                    if (lane == 0) {
+                        float* dst = p.DR + tok * p.dv_ + c0;
+                        reinterpret_cast<float4*>(dst)[0] = make_float4(-z[0], -z[1], -z[2], -z[3]);
+                        reinterpret_cast<float4*>(dst)[1] = make_float4(-z[4], -z[5], -z[6], -z[7]);
+                        float* dvp = p.dv + tok * p.dv_ + c0;
+                        reinterpret_cast<float4*>(dvp)[0] = make_float4(z[8], z[9], z[10], z[11]);
+                        reinterpret_cast<float4*>(dvp)[1] = make_float4(z[12], z[13], z[14], z[15]);
+                    }
+                }
+            }
+        }
+        if (blk + 1 < nblk) store_scal(buf ^ 1, scn);
+        __syncthreads();  // buffer blk is reused by the copies issued next
+    }
+    if (active && dir == 1 && p.dS0)
+#pragma unroll
+        for (int rr = 0; rr < 4; ++rr)
+            if (i0 + rr < p.dk_) {
+                float* dst = p.dS0 + (head * p.dk_ + i0 + rr) * p.dv_ + c0;
+                reinterpret_cast<float4*>(dst)[0] = make_float4(X[rr][0], X[rr][1], X[rr][2], X[rr][3]);
+                reinterpret_cast<float4*>(dst)[1] = make_float4(X[rr][4], X[rr][5], X[rr][6], X[rr][7]);
+            }
+}
+
 // ----------------------------------------------------------------- pass 2 --
 // CTA (row block, chunk, head). Thread t: row rb * RB + t / tpr, columns
 // 8 (t % tpr) .. + 8, with tpr threads per row (a power of two <= 32, so a
@@ -346,8 +584,10 @@ __global__ void __launch_bounds__(kChunkThreads, 4) bwd_chunk_kernel(Params p) {
     const int bh = blockIdx.z, b = bh / p.H, h = bh % p.H;
     const size_t head = (size_t)bh;
     const int i = rb * RB + lr;
-    const int j0 = 8 * g;
-    const bool ok = i < p.dk_ && j0 < p.dv_;
+    // columns 4 g .. 4 g + 3 and 4 (g + tpr) .. + 3: a row's threads read
+    // consecutive 16-byte pieces of a staged row (no bank conflicts)
+    const int ja = 4 * g, jb = 4 * (g + tpr);
+    const bool row_ok = i < p.dk_;
     const int t0 = c * kC, Lc = min(kC, p.T - t0);
     auto tok_of = [&](int t) { return ((size_t)b * p.T + t) * p.H + h; };
 
@@ -385,23 +625,31 @@ __global__ void __launch_bounds__(kChunkThreads, 4) bwd_chunk_kernel(Params p) {
         }
         __syncthreads();
     };
-    auto ld8s = [&](const float* src, float (&x)[8]) {
-        const float4 a = reinterpret_cast<const float4*>(src)[0];
-        const float4 bq = reinterpret_cast<const float4*>(src)[1];
+    auto ld8s = [&](const float* src, float (&x)[8]) {  // this thread's 8 columns of a staged row
+        const float4 a = *reinterpret_cast<const float4*>(src + ja);
+        const float4 bq = *reinterpret_cast<const float4*>(src + jb);
         x[0] = a.x; x[1] = a.y; x[2] = a.z; x[3] = a.w;
         x[4] = bq.x; x[5] = bq.y; x[6] = bq.z; x[7] = bq.w;
     };
 
     float S[8], G[8];
     {
-        const size_t off = ((head * p.nchunks + c) * p.dk_ + i) * p.dv_ + j0;
-        if (ok) {
-            load8<float>(p.ckS, off, S);
-            load8<float>(p.ckG, off, G);
-        } else {
+        // columns at or beyond d_v (and rows beyond d_k) hold zeros and stay zero:
+        // their staged inputs are zero and their row scalars neutral
+        const size_t off = ((head * p.nchunks + c) * p.dk_ + i) * p.dv_;
+        float a4[4], b4[4];
 #pragma unroll
-            for (int cc = 0; cc < 8; ++cc) S[cc] = G[cc] = 0.f;
-        }
+        for (int cc = 0; cc < 4; ++cc) a4[cc] = b4[cc] = 0.f;
+        if (row_ok && ja < p.dv_) load4<float>(p.ckS, off + ja, a4);
+        if (row_ok && jb < p.dv_) load4<float>(p.ckS, off + jb, b4);
+#pragma unroll
+        for (int cc = 0; cc < 4; ++cc) { S[cc] = a4[cc]; S[4 + cc] = b4[cc]; }
+#pragma unroll
+        for (int cc = 0; cc < 4; ++cc) a4[cc] = b4[cc] = 0.f;
+        if (row_ok && ja < p.dv_) load4<float>(p.ckG, off + ja, a4);
+        if (row_ok && jb < p.dv_) load4<float>(p.ckG, off + jb, b4);
+#pragma unroll
+        for (int cc = 0; cc < 4; ++cc) { G[cc] = a4[cc]; G[4 + cc] = b4[cc]; }
     }
 
     // forward over the chunk: the state at every sub-chunk start
@@ -415,8 +663,8 @@ __global__ void __launch_bounds__(kChunkThreads, 4) bwd_chunk_kernel(Params p) {
 #pragma unroll
         for (int u = 0; u < kSub; ++u) {
             float v[8], r[8];
-            ld8s(col_at(kV, u) + j0, v);
-            ld8s(col_at(kR, u) + j0, r);
+            ld8s(col_at(kV, u), v);
+            ld8s(col_at(kR, u), r);
             const float a = row_at(u, 2)[lr], kk = row_at(u, 1)[lr], uu = row_at(u, 4)[lr] * kk;
 #pragma unroll
             for (int cc = 0; cc < 8; ++cc) S[cc] = fmaf(-kk, r[cc], fmaf(uu, v[cc], a * S[cc]));
@@ -436,8 +684,8 @@ __global__ void __launch_bounds__(kChunkThreads, 4) bwd_chunk_kernel(Params p) {
 #pragma unroll
         for (int u = 0; u < kSub; ++u) {
             float v[8], r[8];
-            ld8s(col_at(kV, u) + j0, v);
-            ld8s(col_at(kR, u) + j0, r);
+            ld8s(col_at(kV, u), v);
+            ld8s(col_at(kR, u), r);
             const float a = row_at(u, 2)[lr], kk = row_at(u, 1)[lr], uu = row_at(u, 4)[lr] * kk;
 #pragma unroll
             for (int cc = 0; cc < 8; ++cc)
@@ -447,10 +695,10 @@ __global__ void __launch_bounds__(kChunkThreads, 4) bwd_chunk_kernel(Params p) {
         for (int u = kSub - 1; u >= 0; --u) {
             if (u < ns) {
                 float v[8], d[8], r[8], dr[8];
-                ld8s(col_at(kV, u) + j0, v);
-                ld8s(col_at(kDO, u) + j0, d);
-                ld8s(col_at(kR, u) + j0, r);
-                ld8s(col_at(kDR, u) + j0, dr);
+                ld8s(col_at(kV, u), v);
+                ld8s(col_at(kDO, u), d);
+                ld8s(col_at(kR, u), r);
+                ld8s(col_at(kDR, u), dr);
                 const float q = row_at(u, 0)[lr], kk = row_at(u, 1)[lr], a = row_at(u, 2)[lr];
                 const float bg = row_at(u, 3)[lr], wg = row_at(u, 4)[lr];
                 const float e = bg * kk;
@@ -468,9 +716,6 @@ __global__ void __launch_bounds__(kChunkThreads, 4) bwd_chunk_kernel(Params p) {
                     acc[4] = fmaf(dsd, Sst[u][cc], acc[4]);
                     G[cc] = a * dsd;
                 }
-                if (!ok)
-#pragma unroll
-                    for (int qy = 0; qy < 5; ++qy) acc[qy] = 0.f;
                 if (tpr == 16) {
                     // reduce-scatter over the row's 16 lanes (8 slots, 5 used):
                     // lane g ends with the total of slot (g >> 1), then each
@@ -498,7 +743,7 @@ __global__ void __launch_bounds__(kChunkThreads, 4) bwd_chunk_kernel(Params p) {
                 const bool tied = p.wkind == GDR_GATE_TIED;
                 const float de_b = acc[3] + (tied ? acc[2] : 0.f);
                 float gsc[3] = {acc[4], kk * de_b, kk * acc[2]};  // dalpha, db, dw for row i
-                if (g == 0 && i < p.dk_) {
+                if (g == 0 && row_ok) {
                     const size_t gi = tok_of(t0 + tau0 + u) * p.dk_ + i;
                     p.dq[gi] = acc[0];
                     p.dk[gi] = acc[1] + bg * acc[3] + wg * acc[2];
@@ -507,7 +752,7 @@ __global__ void __launch_bounds__(kChunkThreads, 4) bwd_chunk_kernel(Params p) {
                     if (p.wkind == GDR_GATE_CHANNEL) p.dw[gi] = gsc[2];
                 }
                 if (p.GP) {  // scalar gates: this warp's rows, summed
-                    if (g != 0 || i >= p.dk_)
+                    if (g != 0 || !row_ok)
 #pragma unroll
                         for (int qy = 0; qy < 3; ++qy) gsc[qy] = 0.f;
                     for (int o = tpr; o < 32; o <<= 1)
@@ -581,8 +826,11 @@ WsLayout ws_layout(int B, int T, int H, int dk, int dv) {
 
 template <typename TI>
 cudaError_t launch_typed(Params p, cudaStream_t st) {
-    bwd_scan_kernel<TI><<<dim3((p.dv_ + kScanCols * kScanWarps - 1) / (kScanCols * kScanWarps), p.H, 2 * p.B),
-                          kScanWarps * 32, 0, st>>>(p);
+    const dim3 sgrid((p.dv_ + kScanCols * kScanWarps - 1) / (kScanCols * kScanWarps), p.H, 2 * p.B);
+    if ((p.dk_ * sizeof(TI)) % 16 == 0)
+        bwd_scan_staged_kernel<TI><<<sgrid, kScanWarps * 32, 0, st>>>(p);
+    else
+        bwd_scan_kernel<TI><<<sgrid, kScanWarps * 32, 0, st>>>(p);
     cudaError_t e = cudaGetLastError();
     if (e != cudaSuccess) return e;
     const uint32_t smem = chunk_smem(p.tpr).total;
