@@ -16,6 +16,7 @@ from __future__ import annotations
 
 from ._lib import (GATE_CHANNEL, GATE_NONE, GATE_SCALAR, GATE_TIED, GDR_BF16, GDR_FP32,
                    GDR_DEVICE_DECAY_RANGE, GDR_DEVICE_TIMEOUT, GdrError, gdr_chunk_bwd,
+                   gdr_chunk_bwd_grouped, gdr_chunk_bwd_grouped_workspace_size,
                    gdr_chunk_bwd_workspace_size, gdr_chunk_fwd, gdr_chunk_fwd_grouped, gdr_chunk_fwd_static, gdr_chunk_fwd_workspace_size,
                    gdr_decode_step, gdr_decode_step_grouped, load)
 
@@ -100,31 +101,31 @@ def chunk_bwd(q, k, v, alpha=None, b=None, w=None, S0=None, *, dO, dS_T=None, ch
               workspace=None, need_dS0: bool = True, stream=None):
     """Backward of chunk_fwd for the same inputs: returns a dict with dq, dk,
     dv, dalpha, db, dw (None for an absent or tied gate) and dS0 (None when
-    need_dS0 is False), all fp32. dO has v's shape and dtype; dS_T is the
+    need_dS0 is False), all fp32. q and k may have fewer heads than v
+    (grouped heads, as in chunk_fwd; dq and dk then sum over each group). dO has v's shape and dtype; dS_T is the
     gradient of the final state (None = 0). workspace: None allocates the
     chunk-checkpoint scratch with torch, or a uint8 device tensor of at least
-    gdr_chunk_bwd_workspace_size bytes."""
+    gdr_chunk_bwd_grouped_workspace_size bytes."""
     import torch
     _check(q, k, v, alpha, b, w, S0, dO, dS_T)
-    B, T, H, dk = q.shape
-    dv = v.shape[-1]
-    if k.shape[2] != H or v.shape[2] != H:
-        raise ValueError("the backward pass takes ungrouped heads")
+    B, T, Hq, dk = q.shape
+    H, dv = v.shape[2], v.shape[-1]
     dev = v.device
     f32 = dict(dtype=torch.float32, device=dev)
-    grads = {"dq": torch.empty((B, T, H, dk), **f32), "dk": torch.empty((B, T, H, dk), **f32),
+    grads = {"dq": torch.empty((B, T, Hq, dk), **f32), "dk": torch.empty((B, T, Hq, dk), **f32),
              "dv": torch.empty((B, T, H, dv), **f32),
              "dS0": torch.empty((B, H, dk, dv), **f32) if need_dS0 else None}
     for name, g in (("dalpha", alpha), ("db", b), ("dw", w)):
         grads[name] = None if g is None or isinstance(g, str) else torch.empty(g.shape, **f32)
     if workspace is None:
-        nbytes = gdr_chunk_bwd_workspace_size(B, T, H, dk, dv)
+        nbytes = gdr_chunk_bwd_grouped_workspace_size(B, T, Hq, H, dk, dv)
         workspace = torch.empty(max(nbytes, 1), dtype=torch.uint8, device=dev)
     ws_bytes = workspace.numel() * workspace.element_size()
-    gdr_chunk_bwd(q, k, v, alpha, b, None if isinstance(w, str) else w, _gate_kind(alpha, 3),
-                  _gate_kind(b, 3), _gate_kind(w, 3), S0, dO, dS_T, grads["dq"], grads["dk"],
-                  grads["dv"], grads["dalpha"], grads["db"], grads["dw"], grads["dS0"], workspace,
-                  ws_bytes, B, T, H, dk, dv, chunk, _dtype_code(q), None, stream)
+    gdr_chunk_bwd_grouped(q, k, v, alpha, b, None if isinstance(w, str) else w,
+                          _gate_kind(alpha, 3), _gate_kind(b, 3), _gate_kind(w, 3), S0, dO, dS_T,
+                          grads["dq"], grads["dk"], grads["dv"], grads["dalpha"], grads["db"],
+                          grads["dw"], grads["dS0"], workspace, ws_bytes, B, T, Hq, H, dk, dv, chunk,
+                          _dtype_code(q), None, stream)
     return grads
 
 

@@ -19,7 +19,8 @@ GATE_NONE, GATE_SCALAR, GATE_CHANNEL, GATE_TIED = 0, 1, 2, 3
 
 EXPORTS = ("gdr_chunk_fwd", "gdr_chunk_fwd_grouped", "gdr_chunk_fwd_workspace_size",
            "gdr_chunk_fwd_static", "gdr_chunk_fwd_static_capacity", "gdr_chunk_bwd",
-           "gdr_chunk_bwd_workspace_size", "gdr_decode_step",
+           "gdr_chunk_bwd_workspace_size", "gdr_chunk_bwd_grouped",
+           "gdr_chunk_bwd_grouped_workspace_size", "gdr_decode_step",
            "gdr_decode_step_grouped", "gdr_selftest_bounded_wait", "gdr_status_string",
            "gdr_version")
 
@@ -66,6 +67,10 @@ def load(build_if_missing: bool = True) -> ctypes.CDLL:
         lib.gdr_chunk_bwd.restype = ip
         lib.gdr_chunk_bwd_workspace_size.argtypes = [ip] * 5
         lib.gdr_chunk_bwd_workspace_size.restype = sz
+        lib.gdr_chunk_bwd_grouped.argtypes = [vp] * 6 + [ip] * 3 + [vp] * 11 + [sz] + [ip] * 8 + [vp, vp]
+        lib.gdr_chunk_bwd_grouped.restype = ip
+        lib.gdr_chunk_bwd_grouped_workspace_size.argtypes = [ip] * 6
+        lib.gdr_chunk_bwd_grouped_workspace_size.restype = sz
         lib.gdr_decode_step.argtypes = [vp] * 6 + [ip] * 3 + [vp, vp] + [ip] * 5 + [vp, vp]
         lib.gdr_decode_step.restype = ip
         lib.gdr_status_string.argtypes = [ip]
@@ -160,6 +165,22 @@ def gdr_chunk_bwd(q, k, v, alpha, b, w, alpha_kind, b_kind, w_kind, S0, dO, dS_T
 
 def gdr_chunk_bwd_workspace_size(B, T, H, d_k, d_v) -> int:
     return int(load().gdr_chunk_bwd_workspace_size(B, T, H, d_k, d_v))
+
+
+def gdr_chunk_bwd_grouped(q, k, v, alpha, b, w, alpha_kind, b_kind, w_kind, S0, dO, dS_T, dq, dk, dv,
+                          dalpha, db, dw, dS0, workspace, workspace_bytes, B, T, H_qk, H, d_k, d_v,
+                          chunk, dtype, d_status=None, stream=None) -> None:
+    st = load().gdr_chunk_bwd_grouped(_p(q), _p(k), _p(v), _p(alpha), _p(b), _p(w), alpha_kind,
+                                      b_kind, w_kind, _p(S0), _p(dO), _p(dS_T), _p(dq), _p(dk),
+                                      _p(dv), _p(dalpha), _p(db), _p(dw), _p(dS0), _p(workspace),
+                                      int(workspace_bytes), B, T, H_qk, H, d_k, d_v, chunk, dtype,
+                                      _p(d_status), _stream(stream))
+    if st != GDR_OK:
+        raise GdrError("gdr_chunk_bwd_grouped", st)
+
+
+def gdr_chunk_bwd_grouped_workspace_size(B, T, H_qk, H, d_k, d_v) -> int:
+    return int(load().gdr_chunk_bwd_grouped_workspace_size(B, T, H_qk, H, d_k, d_v))
 
 
 def gdr_decode_step(q, k, v, alpha, b, w, alpha_kind, b_kind, w_kind, S, o, B, H, d_k, d_v, dtype,

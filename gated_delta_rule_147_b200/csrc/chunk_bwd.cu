@@ -47,7 +47,8 @@ struct Params {
     const float *S0, *dST;
     float *dq, *dk, *dv, *dalpha, *db, *dw, *dS0;
     float *ckS, *ckG, *R, *DR, *GP;  // workspace
-    int B, T, H, dk_, dv_, akind, bkind, wkind, nchunks, tpr, nrb;
+    float *dq_out, *dk_out;          // grouped heads: the caller's dq, dk (dq, dk are then workspace)
+    int B, T, H, Hq, group, dk_, dv_, akind, bkind, wkind, nchunks, tpr, nrb;
 };
 
 template <typename TI>
@@ -87,13 +88,14 @@ struct Row {
     float q, k, a, bg, wg;
 };
 
+// tok indexes the value head's [B, T, H] token, tokq the q/k head's [B, T, H_qk] one.
 template <typename TI>
-__device__ __forceinline__ Row load_row(const Params& p, size_t tok, int i) {
+__device__ __forceinline__ Row load_row(const Params& p, size_t tok, size_t tokq, int i) {
     Row r{0.f, 0.f, 1.f, 0.f, 0.f};
     if (i < p.dk_) {
         const size_t gi = tok * p.dk_ + i;
-        r.q = ld1<TI>(p.q, gi);
-        r.k = ld1<TI>(p.k, gi);
+        r.q = ld1<TI>(p.q, tokq * p.dk_ + i);
+        r.k = ld1<TI>(p.k, tokq * p.dk_ + i);
         if (p.akind == GDR_GATE_SCALAR) r.a = ld1<TI>(p.alpha, tok);
         else if (p.akind == GDR_GATE_CHANNEL) r.a = ld1<TI>(p.alpha, gi);
         if (p.bkind == GDR_GATE_SCALAR) r.bg = ld1<TI>(p.b, tok);
@@ -140,12 +142,12 @@ struct Rows4 {
 };
 
 template <typename TI>
-__device__ __forceinline__ void load_rows4(const Params& p, size_t tok, int i0, Rows4& r) {
+__device__ __forceinline__ void load_rows4(const Params& p, size_t tok, size_t tokq, int i0, Rows4& r) {
     if ((p.dk_ & 3) == 0) {
         if (i0 < p.dk_) {
             const size_t gi = tok * p.dk_ + i0;
-            load4<TI>(p.q, gi, r.q);
-            load4<TI>(p.k, gi, r.k);
+            load4<TI>(p.q, tokq * p.dk_ + i0, r.q);
+            load4<TI>(p.k, tokq * p.dk_ + i0, r.k);
             if (p.akind == GDR_GATE_CHANNEL) load4<TI>(p.alpha, gi, r.a);
             else {
                 const float a = p.akind == GDR_GATE_SCALAR ? ld1<TI>(p.alpha, tok) : 1.f;
@@ -175,7 +177,7 @@ __device__ __forceinline__ void load_rows4(const Params& p, size_t tok, int i0, 
     }
 #pragma unroll
     for (int rr = 0; rr < 4; ++rr) {
-        const Row w1 = load_row<TI>(p, tok, i0 + rr);
+        const Row w1 = load_row<TI>(p, tok, tokq, i0 + rr);
         r.q[rr] = w1.q; r.k[rr] = w1.k; r.a[rr] = w1.a; r.bg[rr] = w1.bg; r.wg[rr] = w1.wg;
     }
 }
@@ -193,6 +195,8 @@ __global__ void __launch_bounds__(kScanWarps * 32) bwd_scan_kernel(Params p) {
     const size_t head = (size_t)b * p.H + h;
     const int i0 = 4 * lane;
     auto tok_of = [&](int t) { return ((size_t)b * p.T + t) * p.H + h; };
+    const int hq = h / p.group;
+    auto tokq_of = [&](int t) { return ((size_t)b * p.T + t) * p.Hq + hq; };
     auto ck_at = [&](float* base, int chunk, int i) {
         return base + ((head * p.nchunks + chunk) * p.dk_ + i) * p.dv_ + c0;
     };
@@ -209,7 +213,7 @@ __global__ void __launch_bounds__(kScanWarps * 32) bwd_scan_kernel(Params p) {
     Rows4 nrw;
     float nvec[NC];
     const int tfirst = dir == 0 ? 0 : p.T - 1;
-    load_rows4<TI>(p, tok_of(tfirst), i0, nrw);
+    load_rows4<TI>(p, tok_of(tfirst), tokq_of(tfirst), i0, nrw);
     load8<TI>(colsrc, tok_of(tfirst) * p.dv_ + c0, nvec);
     for (int n = 0; n < p.T; ++n) {
         const int t = dir == 0 ? n : p.T - 1 - n;
@@ -228,8 +232,9 @@ __global__ void __launch_bounds__(kScanWarps * 32) bwd_scan_kernel(Params p) {
 #pragma unroll
         for (int c = 0; c < NC; ++c) cv[c] = nvec[c];
         if (n + 1 < p.T) {
-            const size_t tn = tok_of(dir == 0 ? t + 1 : t - 1);
-            load_rows4<TI>(p, tn, i0, nrw);
+            const int tnext = dir == 0 ? t + 1 : t - 1;
+            const size_t tn = tok_of(tnext);
+            load_rows4<TI>(p, tn, tokq_of(tnext), i0, nrw);
             load8<TI>(colsrc, tn * p.dv_ + c0, nvec);
         }
         if (dir == 0) {
@@ -353,6 +358,8 @@ __global__ void __launch_bounds__(kScanWarps * 32) bwd_scan_staged_kernel(Params
     const bool rows_ok = i0 < p.dk_;       // d_k is a multiple of 4 here
     auto tok_of = [&](int t) { return ((size_t)b * p.T + t) * p.H + h; };
     auto tok_n = [&](int n) { return tok_of(dir == 0 ? n : p.T - 1 - n); };
+    const int hq = h / p.group;
+    auto tokq_n = [&](int n) { return ((size_t)b * p.T + (dir == 0 ? n : p.T - 1 - n)) * p.Hq + hq; };
     const void* colsrc = dir == 0 ? p.v : p.dO;
     // vectors copied per token: q (backward only), k, and the channel gates
     const void* vsrc[5] = {p.q, p.k, p.alpha, p.b, p.w};
@@ -367,8 +374,9 @@ __global__ void __launch_bounds__(kScanWarps * 32) bwd_scan_staged_kernel(Params
             if (!vneed[vi]) continue;
             for (int idx = tid; idx < nt * row_pieces; idx += kScanWarps * 32) {
                 const int tt = idx / row_pieces, pc = idx % row_pieces;
+                const size_t tk = vi < 2 ? tokq_n(n0 + tt) : tok_n(n0 + tt);  // q, k: q/k head
                 cp_async16(&stg[buf].rows[vi][tt][pc * EPC],
-                           static_cast<const TI*>(vsrc[vi]) + tok_n(n0 + tt) * p.dk_ + pc * EPC);
+                           static_cast<const TI*>(vsrc[vi]) + tk * p.dk_ + pc * EPC);
             }
         }
         for (int idx = tid; idx < nt * col_pieces; idx += kScanWarps * 32) {
@@ -598,6 +606,7 @@ __global__ void __launch_bounds__(kChunkThreads, 4) bwd_chunk_kernel(Params p) {
         const int n4 = dvp / 4;  // float4 per token row (a power of two, as is RB)
         const int lg_n4 = __ffs(n4) - 1, lg_rb = __ffs(RB) - 1;
         const size_t tok0 = tok_of(t0 + tau0);  // token u of the sub-chunk: tok0 + u H
+        const size_t tokq0 = ((size_t)b * p.T + t0 + tau0) * p.Hq + h / p.group;
         const int narr = bwd ? 4 : 2;
         for (int ai = 0; ai < narr; ++ai) {
             const int a = bwd ? ai : (ai == 0 ? kV : kR);
@@ -616,7 +625,7 @@ __global__ void __launch_bounds__(kChunkThreads, 4) bwd_chunk_kernel(Params p) {
         for (int idx = tid; idx < (kSub << lg_rb); idx += kChunkThreads) {
             const int u = idx >> lg_rb, r = idx & (RB - 1);
             Row rw{0.f, 0.f, 1.f, 0.f, 0.f};
-            if (u < ns) rw = load_row<TI>(p, tok0 + (size_t)u * p.H, rb * RB + r);
+            if (u < ns) rw = load_row<TI>(p, tok0 + (size_t)u * p.H, tokq0 + (size_t)u * p.Hq, rb * RB + r);
             row_at(u, 0)[r] = rw.q;
             row_at(u, 1)[r] = rw.k;
             row_at(u, 2)[r] = rw.a;
@@ -796,6 +805,26 @@ __global__ void bwd_gate_sum_kernel(Params p) {
     }
 }
 
+// Grouped heads: dq, dk of a q/k head are the sums over the value heads that
+// share it (value heads hq G .. hq G + G - 1), added in that order.
+__global__ void bwd_group_sum_kernel(Params p) {
+    const size_t n = blockIdx.x * (size_t)blockDim.x + threadIdx.x;  // over [B, T, H_qk, d_k]
+    const size_t total = (size_t)p.B * p.T * p.Hq * p.dk_;
+    if (n >= total) return;
+    const int i = (int)(n % p.dk_);
+    const size_t tq = n / p.dk_;  // (b t) H_qk + hq
+    const size_t bt = tq / p.Hq;
+    const int hq = (int)(tq % p.Hq);
+    float sq = 0.f, sk = 0.f;
+    for (int g = 0; g < p.group; ++g) {
+        const size_t src = (bt * p.H + (size_t)hq * p.group + g) * p.dk_ + i;
+        sq += p.dq[src];
+        sk += p.dk[src];
+    }
+    p.dq_out[n] = sq;
+    p.dk_out[n] = sk;
+}
+
 int threads_per_row(int dv) {
     int t = 1;
     while (8 * t < dv) t <<= 1;
@@ -805,10 +834,10 @@ int threads_per_row(int dv) {
 size_t round256(size_t x) { return (x + 255) & ~size_t(255); }
 
 struct WsLayout {
-    size_t ckS, ckG, R, DR, GP, total;
+    size_t ckS, ckG, R, DR, GP, DQ, DK, total;
 };
 
-WsLayout ws_layout(int B, int T, int H, int dk, int dv) {
+WsLayout ws_layout(int B, int T, int H, int dk, int dv, bool grouped) {
     WsLayout l{};
     const size_t nch = (size_t)(T + kC - 1) / kC;
     const size_t ck = round256((size_t)B * H * nch * dk * dv * sizeof(float));
@@ -820,7 +849,10 @@ WsLayout ws_layout(int B, int T, int H, int dk, int dv) {
     l.R = l.ckG + ck;
     l.DR = l.R + rr;
     l.GP = l.DR + rr;
-    l.total = l.GP + gp;
+    const size_t gq = grouped ? round256((size_t)B * T * H * dk * sizeof(float)) : 0;
+    l.DQ = l.GP + gp;
+    l.DK = l.DQ + gq;
+    l.total = l.DK + gq;
     return l;
 }
 
@@ -839,10 +871,19 @@ cudaError_t launch_typed(Params p, cudaStream_t st) {
     if (e != cudaSuccess) return e;
     kern<<<dim3(p.nrb, p.nchunks, p.B * p.H), kChunkThreads, smem, st>>>(p);
     e = cudaGetLastError();
-    if (e != cudaSuccess || !p.GP) return e;
-    const size_t BTH = (size_t)p.B * p.T * p.H;
-    bwd_gate_sum_kernel<<<(unsigned)((BTH + 255) / 256), 256, 0, st>>>(p);
-    return cudaGetLastError();
+    if (e != cudaSuccess) return e;
+    if (p.GP) {
+        const size_t BTH = (size_t)p.B * p.T * p.H;
+        bwd_gate_sum_kernel<<<(unsigned)((BTH + 255) / 256), 256, 0, st>>>(p);
+        e = cudaGetLastError();
+        if (e != cudaSuccess) return e;
+    }
+    if (p.group > 1) {
+        const size_t n = (size_t)p.B * p.T * p.Hq * p.dk_;
+        bwd_group_sum_kernel<<<(unsigned)((n + 255) / 256), 256, 0, st>>>(p);
+        e = cudaGetLastError();
+    }
+    return e;
 }
 
 }  // namespace bwd
@@ -861,19 +902,25 @@ bool ptr_matches(int kind, const void* ptr) { return has_data(kind) ? ptr != nul
 
 extern "C" {
 
-size_t gdr_chunk_bwd_workspace_size(int B, int T, int H, int d_k, int d_v) {
-    if (B < 1 || H < 1 || T < 1 || d_k < 1 || d_v < 1) return 0;
-    return gdr::bwd::ws_layout(B, T, H, d_k, d_v).total;
+size_t gdr_chunk_bwd_grouped_workspace_size(int B, int T, int H_qk, int H, int d_k, int d_v) {
+    if (B < 1 || H < 1 || T < 1 || d_k < 1 || d_v < 1 || H_qk < 1 || H % H_qk != 0) return 0;
+    return gdr::bwd::ws_layout(B, T, H, d_k, d_v, H_qk != H).total;
 }
 
-gdr_status gdr_chunk_bwd(const void* q, const void* k, const void* v, const void* alpha,
-                         const void* b, const void* w, int alpha_kind, int b_kind, int w_kind,
-                         const float* S0, const void* dO, const float* dS_T, float* dq, float* dk,
-                         float* dv, float* dalpha, float* db, float* dw, float* dS0,
-                         void* workspace, size_t workspace_bytes, int B, int T, int H, int d_k,
-                         int d_v, int chunk, int dtype, int* d_status, void* stream) {
+size_t gdr_chunk_bwd_workspace_size(int B, int T, int H, int d_k, int d_v) {
+    return gdr_chunk_bwd_grouped_workspace_size(B, T, H, H, d_k, d_v);
+}
+
+gdr_status gdr_chunk_bwd_grouped(const void* q, const void* k, const void* v, const void* alpha,
+                                 const void* b, const void* w, int alpha_kind, int b_kind,
+                                 int w_kind, const float* S0, const void* dO, const float* dS_T,
+                                 float* dq, float* dk, float* dv, float* dalpha, float* db,
+                                 float* dw, float* dS0, void* workspace, size_t workspace_bytes,
+                                 int B, int T, int H_qk, int H, int d_k, int d_v, int chunk,
+                                 int dtype, int* d_status, void* stream) {
     (void)d_status;  // this path has no bounded waits to report
     if (B < 1 || H < 1 || T < 0 || d_k < 1 || d_v < 1) return GDR_ERR_INVALID_ARG;
+    if (H_qk < 1 || H % H_qk != 0) return GDR_ERR_INVALID_ARG;
     if (dtype != GDR_BF16 && dtype != GDR_FP32) return GDR_ERR_INVALID_ARG;
     if (!kind_valid(alpha_kind, false) || !kind_valid(b_kind, false) || !kind_valid(w_kind, true))
         return GDR_ERR_INVALID_ARG;
@@ -899,9 +946,10 @@ gdr_status gdr_chunk_bwd(const void* q, const void* k, const void* v, const void
     const int nch = (T + gdr::bwd::kC - 1) / gdr::bwd::kC;
     if (nch > 65535 || (size_t)B * H > 65535u) return GDR_ERR_UNSUPPORTED;  // grid limits
     const void* ptrs[] = {q, k, v, dO, dq, dk, dv, S0, dS_T, dS0, dalpha, db, dw, alpha, b, w};
-    for (const void* p : ptrs)
-        if (p && !a16(p)) return GDR_ERR_MISALIGNED;
-    const gdr::bwd::WsLayout wl = gdr::bwd::ws_layout(B, T, H, d_k, d_v);
+    for (const void* ptr : ptrs)
+        if (ptr && !a16(ptr)) return GDR_ERR_MISALIGNED;
+    const bool grouped = H_qk != H;
+    const gdr::bwd::WsLayout wl = gdr::bwd::ws_layout(B, T, H, d_k, d_v, grouped);
     if (!workspace || workspace_bytes < wl.total) return GDR_ERR_INVALID_ARG;
     if ((reinterpret_cast<uintptr_t>(workspace) & 255u) != 0) return GDR_ERR_MISALIGNED;
 
@@ -909,7 +957,17 @@ gdr_status gdr_chunk_bwd(const void* q, const void* k, const void* v, const void
     gdr::bwd::Params p;
     p.q = q; p.k = k; p.v = v; p.alpha = alpha; p.b = b; p.w = w; p.dO = dO;
     p.S0 = S0; p.dST = dS_T;
-    p.dq = dq; p.dk = dk; p.dv = dv; p.dalpha = dalpha; p.db = db; p.dw = dw; p.dS0 = dS0;
+    p.dv = dv; p.dalpha = dalpha; p.db = db; p.dw = dw; p.dS0 = dS0;
+    if (grouped) {  // per-value-head dq, dk in the workspace, summed over each group at the end
+        p.dq = reinterpret_cast<float*>(ws + wl.DQ);
+        p.dk = reinterpret_cast<float*>(ws + wl.DK);
+        p.dq_out = dq;
+        p.dk_out = dk;
+    } else {
+        p.dq = dq;
+        p.dk = dk;
+        p.dq_out = p.dk_out = nullptr;
+    }
     p.ckS = reinterpret_cast<float*>(ws + wl.ckS);
     p.ckG = reinterpret_cast<float*>(ws + wl.ckG);
     p.R = reinterpret_cast<float*>(ws + wl.R);
@@ -917,7 +975,7 @@ gdr_status gdr_chunk_bwd(const void* q, const void* k, const void* v, const void
     const bool any_scalar = alpha_kind == GDR_GATE_SCALAR || b_kind == GDR_GATE_SCALAR ||
                             w_kind == GDR_GATE_SCALAR;
     p.GP = any_scalar ? reinterpret_cast<float*>(ws + wl.GP) : nullptr;
-    p.B = B; p.T = T; p.H = H; p.dk_ = d_k; p.dv_ = d_v;
+    p.B = B; p.T = T; p.H = H; p.Hq = H_qk; p.group = H / H_qk; p.dk_ = d_k; p.dv_ = d_v;
     p.akind = alpha_kind; p.bkind = b_kind; p.wkind = w_kind;
     p.nchunks = nch;
     p.tpr = gdr::bwd::threads_per_row(d_v);
@@ -926,6 +984,17 @@ gdr_status gdr_chunk_bwd(const void* q, const void* k, const void* v, const void
     const cudaError_t e = dtype == GDR_BF16 ? gdr::bwd::launch_typed<__nv_bfloat16>(p, st)
                                             : gdr::bwd::launch_typed<float>(p, st);
     return e == cudaSuccess ? GDR_OK : GDR_ERR_LAUNCH;
+}
+
+gdr_status gdr_chunk_bwd(const void* q, const void* k, const void* v, const void* alpha,
+                         const void* b, const void* w, int alpha_kind, int b_kind, int w_kind,
+                         const float* S0, const void* dO, const float* dS_T, float* dq, float* dk,
+                         float* dv, float* dalpha, float* db, float* dw, float* dS0,
+                         void* workspace, size_t workspace_bytes, int B, int T, int H, int d_k,
+                         int d_v, int chunk, int dtype, int* d_status, void* stream) {
+    return gdr_chunk_bwd_grouped(q, k, v, alpha, b, w, alpha_kind, b_kind, w_kind, S0, dO, dS_T,
+                                 dq, dk, dv, dalpha, db, dw, dS0, workspace, workspace_bytes, B, T,
+                                 H, H, d_k, d_v, chunk, dtype, d_status, stream);
 }
 
 }  // extern "C"

@@ -255,6 +255,30 @@ gdr_status gdr_chunk_bwd(const void* q, const void* k, const void* v,
                          int B, int T, int H, int d_k, int d_v, int chunk,
                          int dtype, int* d_status, void* stream);
 
+/*
+ * gdr_chunk_bwd_grouped -- gdr_chunk_bwd with grouped query/key heads, as in
+ * gdr_chunk_fwd_grouped: q, k and their gradients dq, dk are [B, T, H_qk,
+ * d_k]; value head h reads q/k head h / (H / H_qk). dq and dk of a q/k head
+ * are the sums over the value heads that share it (added in head order).
+ * The workspace is gdr_chunk_bwd_grouped_workspace_size() bytes; everything
+ * else is as gdr_chunk_bwd, which is this call with H_qk = H. Returns
+ * GDR_ERR_INVALID_ARG also when H_qk < 1 or H is not a multiple of H_qk.
+ */
+gdr_status gdr_chunk_bwd_grouped(const void* q, const void* k, const void* v,
+                                 const void* alpha, const void* b, const void* w,
+                                 int alpha_kind, int b_kind, int w_kind,
+                                 const float* S0, const void* dO, const float* dS_T,
+                                 float* dq, float* dk, float* dv,
+                                 float* dalpha, float* db, float* dw, float* dS0,
+                                 void* workspace, size_t workspace_bytes,
+                                 int B, int T, int H_qk, int H, int d_k, int d_v,
+                                 int chunk, int dtype, int* d_status, void* stream);
+
+/* Bytes of workspace gdr_chunk_bwd_grouped needs: gdr_chunk_bwd_workspace_size
+ * plus, when H_qk < H, per-value-head dq and dk (2 x B T H d_k fp32, each
+ * rounded up to 256 bytes). 0 for bad sizes. Host-only. */
+size_t gdr_chunk_bwd_grouped_workspace_size(int B, int T, int H_qk, int H, int d_k, int d_v);
+
 /* Bytes of workspace gdr_chunk_bwd needs (0 for T < 1 or bad sizes): fp32
  * chunk-start states and chunk-end state gradients (2 x B H ceil(T/64) d_k
  * d_v), r_t and dr_t of every token (2 x B T H d_v), and scalar-gate partial

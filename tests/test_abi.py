@@ -183,3 +183,17 @@ def r256(x):
 ])
 def test_bwd_workspace_size(shape, expect):
     assert _lib.gdr_chunk_bwd_workspace_size(*shape) == expect
+
+
+def test_grouped_backward_rejects_bad_head_counts_and_sizes_its_workspace():
+    lib = _lib.load()
+    args = [P, P, P, P, P, None, 1, 1, 3, None, P, None, P, P, P, P, P, None, P, P, 1 << 30]
+    st = lib.gdr_chunk_bwd_grouped(*args, 1, 64, 3, 4, 128, 128, 64, 0, None, None)  # 4 % 3 != 0
+    assert st == _lib.GDR_ERR_INVALID_ARG
+    st = lib.gdr_chunk_bwd_grouped(*args, 1, 64, 0, 4, 128, 128, 64, 0, None, None)  # H_qk = 0
+    assert st == _lib.GDR_ERR_INVALID_ARG
+    base = _lib.gdr_chunk_bwd_grouped_workspace_size(1, 64, 4, 4, 128, 128)
+    assert base == _lib.gdr_chunk_bwd_workspace_size(1, 64, 4, 128, 128)
+    # grouped: per-value-head dq and dk in the workspace
+    assert _lib.gdr_chunk_bwd_grouped_workspace_size(1, 64, 2, 4, 128, 128) == base + 2 * 64 * 4 * 128 * 4
+    assert _lib.gdr_chunk_bwd_grouped_workspace_size(1, 64, 3, 4, 128, 128) == 0

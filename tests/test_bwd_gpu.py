@@ -138,3 +138,20 @@ def test_full_size_sampled_heads(cuda_device):
         else:
             g = np.stack([got[n][bi][:, hi] for bi, hi in heads])[:, :, None]
         assert_close(g, ref[n], TOL, n)
+
+
+@pytest.mark.parametrize("form", ["gdn", "gdn2"])
+def test_grouped_heads(cuda_device, form):
+    """q/k heads shared by pairs of value heads: dq, dk of a q/k head are the
+    sums over its value heads of the oracle's gradients with q, k repeated."""
+    wl = WORKLOADS["kda"].with_(B=2, H=4, hq=2, T=150, s0=True, seed=330, **FORMS[form])
+    inp = make_chunk_inputs(wl)
+    cot = make_cotangents(wl)
+    got = run_bwd(inp, cot, cuda_device)
+    G = wl.H // wl.hq
+    rep = dict(inp, q=inp["q"].repeat_interleave(G, dim=2), k=inp["k"].repeat_interleave(G, dim=2))
+    ref = run_oracle_bwd(rep, cot)
+    for n in ("dq", "dk"):
+        B, T, H, dk = ref[n].shape
+        ref[n] = ref[n].reshape(B, T, H // G, G, dk).sum(axis=3)
+    check(got, ref, f"grouped {form} ")
