@@ -378,7 +378,10 @@ def cpu_baseline(wl, budget_s=15.0):
     return {"value": token_heads / wl.H / dt, "unit": "tokens/s", "cores": min(cores, heads),
             "kind": "oracle",
             "sample": f"{heads} of {wl.B * wl.H} heads of the same workload, full T={wl.T}, "
-                      f"fp64 token loop, {dt:.1f} s"}
+                      f"fp64 token loop, {dt:.1f} s",
+            # the same oracle on one thread (the calibration run): tokens/s of the workload per core
+            "single_core": {"value": 1.0 / (per_head_token * wl.H), "unit": "tokens/s",
+                            "sample": f"1 head, T={small.T}, 1 thread"}}
 
 
 def run_ours(args):
