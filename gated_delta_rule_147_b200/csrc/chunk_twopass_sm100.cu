@@ -133,6 +133,9 @@ __global__ void __launch_bounds__(NT, 2) prep_gdn_kernel(const __grid_constant__
     };
     auto bits_to_f32 = [](unsigned short u) { return __uint_as_float((uint32_t)u << 16); };
 
+    // the state pass may be scheduled now: its CTAs take SMs as this grid's
+    // CTAs leave them, and wait for this grid's completion before reading
+    asm volatile("griddepcontrol.launch_dependents;");
     if (tid == 0) {
         mbar_init(&bar_tma[0], 1);
         mbar_init(&bar_tma[1], 1);
@@ -496,6 +499,10 @@ __global__ void __launch_bounds__(NT, 1) state_gdn_kernel(
     auto stage_alpha = [&](int ci) {
         if (tid < C) s_alpha[tid] = ci * C + tid < T ? bits_to_f32(g_a) : 1.f;
     };
+    // Everything above overlaps the first pass's tail (this grid may be
+    // launched before that one completes: programmatic dependent launch);
+    // the first pass's factors are read only after it has completed.
+    asm volatile("griddepcontrol.wait;" ::: "memory");
     if (tid == 0) {
         if (nchunks > 0) issue_loads(0);
         if (nchunks > 1) issue_loads(1);
@@ -745,8 +752,17 @@ cudaError_t launch_chunk_twopass_gdn(const CUtensorMap* maps, const CUtensorMap*
     p.group = group;
     e = cudaFuncSetAttribute(state_gdn_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, S_SMEM_BYTES);
     if (e != cudaSuccess) return e;
-    state_gdn_kernel<<<dim3(dv / NV, H, B), NT, S_SMEM_BYTES, st>>>(maps[0], maps[1], ws_maps[0], ws_maps[1], p);
-    return cudaGetLastError();
+    cudaLaunchConfig_t cfg = {};
+    cfg.gridDim = dim3(dv / NV, H, B);
+    cfg.blockDim = dim3(NT, 1, 1);
+    cfg.dynamicSmemBytes = S_SMEM_BYTES;
+    cfg.stream = st;
+    cudaLaunchAttribute attr[1];
+    attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;  // overlap the prep tail
+    attr[0].val.programmaticStreamSerializationAllowed = 1;
+    cfg.attrs = attr;
+    cfg.numAttrs = 1;
+    return cudaLaunchKernelEx(&cfg, state_gdn_kernel, maps[0], maps[1], ws_maps[0], ws_maps[1], p);
 }
 
 }  // namespace gdr
