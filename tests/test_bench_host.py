@@ -1,0 +1,59 @@
+"""bench.py's host-side accounting (no GPU): the algorithmic bytes and flops
+the roofline divides by, the kernel family each workload runs, the keying of
+recorded DRAM traffic to the kernel sources, and the CPU-baseline record."""
+import json
+import os
+
+import pytest
+
+import bench
+from gated_delta_rule_147_b200.inputs import WORKLOADS
+
+
+@pytest.mark.parametrize("name,mb,gf", [
+    ("gdn", 273.7, 47.96),    # 1028 B per token-head + S_T; 182,955 flop per token-head
+    ("kda", 680.5, 95.92),    # + channel alpha, random S0 read
+    ("gdn2", 940.6, 147.46),  # + channel b, w; 281,259 flop per token-head
+])
+def test_algorithmic_work(name, mb, gf):
+    wl = WORKLOADS[name]
+    assert bench.workload_bytes(wl) / 1e6 == pytest.approx(mb, abs=0.05)
+    assert bench.workload_flops(wl) / 1e9 == pytest.approx(gf, abs=0.005)
+
+
+def test_kernel_families():
+    fam = {n: bench.kernel_family(w) for n, w in WORKLOADS.items()}
+    assert fam == {"tiny": "general", "gdn": "twopass", "kda": "twopass_general",
+                   "gdn2": "twopass_general", "gla": "erasefree", "gdn_gqa": "twopass"}
+    assert set(bench.LAUNCHES_PER_CALL) == set(bench.KERNEL_SOURCES) == set(bench.KERNEL_NAMES)
+
+
+def test_recorded_traffic_is_keyed_to_the_kernel_sources(monkeypatch, tmp_path):
+    rec = {"workloads": {"gla": {"source_sha256": bench.kernel_source_hash("erasefree"),
+                                 "dram_bytes_per_launch": 123}}}
+    (tmp_path / "profiles").mkdir()
+    (tmp_path / "profiles" / "chunk_fwd_traffic.json").write_text(json.dumps(rec))
+    monkeypatch.setattr(bench, "ROOT", str(tmp_path))
+    # the recorded figure needs the sources it was taken on: here they are absent
+    with pytest.raises(OSError):
+        bench.kernel_source_hash("erasefree")
+    monkeypatch.setattr(bench, "kernel_source_hash", lambda fam: rec["workloads"]["gla"]["source_sha256"])
+    assert bench.measured_traffic("gla") == 123
+    monkeypatch.setattr(bench, "kernel_source_hash", lambda fam: "0" * 64)
+    assert bench.measured_traffic("gla") is None
+    assert bench.measured_traffic("kda") is None
+
+
+def test_backward_flops_per_element():
+    # forward step 4 multiply-adds, reverse step 9, per state element and token
+    assert bench.BWD_FLOPS_PER_ELEMENT == 26
+    assert bench.ALU_FP32_TFLOPS == pytest.approx(74.45, abs=0.01)
+
+
+def test_cpu_baseline_record():
+    wl = WORKLOADS["gdn"].with_(B=1, H=2, T=64)
+    rec = bench.cpu_baseline(wl, budget_s=0.2)
+    assert rec["kind"] == "oracle" and rec["unit"] == "tokens/s"
+    assert rec["value"] > 0 and rec["cores"] >= 1
+    assert rec["single_core"]["value"] > 0
+    assert "heads" in rec["sample"]
