@@ -39,6 +39,26 @@ def _check(*ts):
             raise ValueError("tensors passed to the library must be contiguous")
 
 
+def _check_types(ref, same=(), fp32=()):
+    """The library reads raw device pointers with one element type: `ref` (q)
+    and every (name, tensor) in `same` share q's dtype, every one in `fp32` is
+    float32, and all live on one CUDA device. Raised before any call."""
+    import torch
+    _dtype_code(ref)
+    tensors = [(n, t) for n, t in list(same) + list(fp32) if t is not None and not isinstance(t, str)]
+    for name, t in same:
+        if t is not None and not isinstance(t, str) and t.dtype != ref.dtype:
+            raise TypeError(f"{name} has dtype {t.dtype}; expected {ref.dtype} like q")
+    for name, t in fp32:
+        if t is not None and t.dtype != torch.float32:
+            raise TypeError(f"{name} has dtype {t.dtype}; the state is float32")
+    if ref.device.type != "cuda":
+        raise ValueError(f"q is on {ref.device}; the library takes CUDA tensors")
+    for name, t in tensors:
+        if t.device != ref.device:
+            raise ValueError(f"{name} is on {t.device}; expected {ref.device} like q")
+
+
 def _gate_kind(g, ndim_scalar: int):
     if g is None:
         return GATE_NONE
@@ -71,6 +91,8 @@ def chunk_fwd(q, k, v, alpha=None, b=None, w=None, S0=None, *, out=None, final_s
     is False."""
     import torch
     _check(q, k, v, alpha, b, w, S0, out, S_T)
+    _check_types(q, [("k", k), ("v", v), ("alpha", alpha), ("b", b), ("w", w), ("out", out)],
+                 [("S0", S0), ("S_T", S_T)])
     B, T, Hq, dk = q.shape
     H, dv = v.shape[2], v.shape[-1]
     o = out if out is not None else torch.empty((B, T, H, dv), dtype=v.dtype, device=v.device)
@@ -89,6 +111,8 @@ def chunk_fwd(q, k, v, alpha=None, b=None, w=None, S0=None, *, out=None, final_s
             raise ValueError(workspace)
         nbytes = workspace_bytes(q, v, alpha, b, w)
         workspace = torch.empty(nbytes, dtype=torch.uint8, device=v.device) if nbytes else None
+    if workspace is not None and workspace.device != q.device:
+        raise ValueError(f"workspace is on {workspace.device}; expected {q.device} like q")
     ws_bytes = 0 if workspace is None else workspace.numel() * workspace.element_size()
     gdr_chunk_fwd_grouped(q, k, v, alpha, b, None if isinstance(w, str) else w,
                           _gate_kind(alpha, 3), _gate_kind(b, 3), _gate_kind(w, 3), S0, o,
@@ -108,6 +132,8 @@ def chunk_bwd(q, k, v, alpha=None, b=None, w=None, S0=None, *, dO, dS_T=None, ch
     gdr_chunk_bwd_grouped_workspace_size bytes."""
     import torch
     _check(q, k, v, alpha, b, w, S0, dO, dS_T)
+    _check_types(q, [("k", k), ("v", v), ("alpha", alpha), ("b", b), ("w", w), ("dO", dO)],
+                 [("S0", S0), ("dS_T", dS_T)])
     B, T, Hq, dk = q.shape
     H, dv = v.shape[2], v.shape[-1]
     dev = v.device
@@ -120,6 +146,8 @@ def chunk_bwd(q, k, v, alpha=None, b=None, w=None, S0=None, *, dO, dS_T=None, ch
     if workspace is None:
         nbytes = gdr_chunk_bwd_grouped_workspace_size(B, T, Hq, H, dk, dv)
         workspace = torch.empty(max(nbytes, 1), dtype=torch.uint8, device=dev)
+    if workspace.device != q.device:
+        raise ValueError(f"workspace is on {workspace.device}; expected {q.device} like q")
     ws_bytes = workspace.numel() * workspace.element_size()
     gdr_chunk_bwd_grouped(q, k, v, alpha, b, None if isinstance(w, str) else w,
                           _gate_kind(alpha, 3), _gate_kind(b, 3), _gate_kind(w, 3), S0, dO, dS_T,
@@ -135,6 +163,8 @@ def decode_step(q, k, v, alpha, b, w, S, *, out=None, d_status=None, stream=None
     Returns o [B,H,d_v]."""
     import torch
     _check(q, k, v, alpha, b, w, S, out)
+    _check_types(q, [("k", k), ("v", v), ("alpha", alpha), ("b", b), ("w", w), ("out", out)],
+                 [("S", S)])
     B, Hq, dk = q.shape
     H, dv = v.shape[1], v.shape[-1]
     o = out if out is not None else torch.empty((B, H, dv), dtype=v.dtype, device=v.device)
