@@ -15,11 +15,12 @@
 // Structure. The state gradient obeys its own recurrence,
 //   G_{t-1} = Diag(alpha_t) (I - e_t^T k_t) G_t + q_{t-1}^T dO_{t-1},
 // which never reads S, so the two sequential parts are independent scans:
-//  1. bwd_scan_kernel, one warp per 8 state columns of a head (the column
-//     sums over d_k are in-thread plus warp shuffles, no block barrier):
-//     forward over the tokens: the state at every 64-token chunk start and
-//     r_t of every token; backward over the tokens: G at every chunk end,
-//     dr_t and dv_t of every token, and dS0. Both directions run at once.
+//  1. bwd_scan_staged_kernel (bwd_scan_kernel when a d_k row is not a whole
+//     number of 16-byte pieces), one warp per 8 state columns of a head (the
+//     column sums over d_k are in-thread plus warp shuffles): forward over
+//     the tokens: the state at every 64-token chunk start and r_t of every
+//     token; backward over the tokens: G at every chunk end, dr_t and dv_t
+//     of every token, and dS0. Both directions run in one launch.
 //  2. bwd_chunk_kernel, parallel over (row block, chunk, head): from the
 //     chunk's start state and end gradient it rebuilds S_{t-1} (elementwise,
 //     with r_t known; two levels: states at 8-token sub-chunk starts in
@@ -27,7 +28,9 @@
 //     dr_t known), and forms dq, dk and the gate gradients. A CTA holds
 //     whole rows of the state, so the sums over columns stay inside it.
 //  3. bwd_gate_sum_kernel (scalar gates only): the sum over key channels of a
-//     scalar gate's gradient, from the per-row-block partial sums of pass 2.
+//     scalar gate's gradient, from the per-row-block partial sums of pass 2;
+//     bwd_group_sum_kernel (grouped heads only): dq, dk of each q/k head
+//     summed over the value heads that share it.
 #include "common.cuh"
 
 namespace gdr {
