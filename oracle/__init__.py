@@ -17,6 +17,9 @@ Routes (each follows a different passage, so they pin each other):
   recurrence_bwd        its reverse-mode gradient (C, all states kept),
                         pinned by finite differences of `recurrence` and by
                         the linear-attention closed form.
+  chunkwise_bwd         the same gradients per chunk as masked matrix
+                        products (numpy, small cases), from the per-token
+                        erase reads r_t and their gradients dr_t.
   recurrence_py         the same definition as a numpy token loop (small cases).
   unrolled_contributions  S_t = sum_i C_i^(t) with explicit d_k x d_k
                         transition matrices ("How Linear Attention Remembers",
@@ -338,3 +341,96 @@ def unified_decay_after_erase(q, k, v, alpha, beta, S0=None):
                     + beta[bi, t, h] * np.outer(kt, v[bi, t, h])
                 o[bi, t, h] = q[bi, t, h] @ S
     return o
+
+
+def chunkwise_bwd(q, k, v, alpha=None, b=None, w=None, S0=None, gates=None, dO=None, dS_T=None,
+                  chunk: int = 8):
+    """Gradients of L = sum(o * dO) + sum(S_T * dS_T), chunk by chunk.
+
+    Two token scans give, per token, the erase read r_t = (b.k) Diag(alpha) S_{t-1}
+    and its gradient dr_t = -k_t Ghat_t (Ghat_t = dL/dS_t after adding q_t^T dO_t),
+    plus the state at every chunk start and the state gradient at every chunk
+    end. With r and dr known, a chunk is a diagonal-decay (erase-free) system
+    ("The Eraser Trilogy", "The Rosetta Stone": the masked-matrix form), so
+    with gamma the running product of alpha inside the chunk (rows of Gam):
+      dq  = Gam (dO S0^T) + Gam [(M o dO V^T)(U/Gam) - (M o dO R^T)(K/Gam)]
+      de  = Gam (DR S0^T) + Gam [(M1 o DR V^T)(U/Gam) - (M1 o DR R^T)(K/Gam)]
+      du  = [(M^T o V dO^T)(Q Gam) + (M1^T o V DR^T)(E Gam) + gamma_C (V Ge^T)] / Gam
+      dkr = -[(M^T o R dO^T)(Q Gam) + (M1^T o R DR^T)(E Gam) + gamma_C (R Ge^T)] / Gam
+    (M causal with the diagonal, M1 without; U = w.k, E = b.k, S0 / Ge the
+    chunk's start state / end gradient), dk = dkr + b.de + w.du, db = k.de,
+    dw = k.du, and the decay through the log of the running product: readers
+    minus writers, q.dq + e.de - u.du - k.dkr, plus rowsum(Ge . S_end) on the
+    chunk's last token, summed from each token to the chunk end, divided by
+    alpha. Returns the dict of `recurrence_bwd` (per-channel gates only
+    materialised: scalar and tied forms are summed / merged as there)."""
+    q, k, v = f64(q), f64(k), f64(v)
+    B, T, H, dk = q.shape
+    dv = v.shape[-1]
+    g = dict(gates or {})
+    tied = g.get("w") == "tied"
+    A, Bg, W = _full_gates(alpha, b, w, gates, B, T, H, dk)
+    S0 = f64(S0)
+    dO = f64(dO)
+    dS_T = f64(dS_T)
+    out = {n: np.zeros((B, T, H, dk)) for n in ("dq", "dk", "da", "db", "dw")}
+    out["dv"] = np.zeros((B, T, H, dv))
+    out["dS0"] = np.zeros((B, H, dk, dv))
+    for bi in range(B):
+        for h in range(H):
+            qq, kk, vv, aa = q[bi, :, h], k[bi, :, h], v[bi, :, h], A[bi, :, h]
+            e, u = Bg[bi, :, h] * kk, W[bi, :, h] * kk
+            do = dO[bi, :, h]
+            # forward scan: states and erase reads
+            S = np.zeros((dk, dv)) if S0 is None else S0[bi, h].copy()
+            states = [S.copy()]
+            r = np.zeros((T, dv))
+            for t in range(T):
+                Sd = aa[t][:, None] * S
+                r[t] = e[t] @ Sd
+                S = Sd - np.outer(kk[t], r[t]) + np.outer(u[t], vv[t])
+                states.append(S.copy())
+            # backward scan: state-gradient at chunk ends, dr and dv per token
+            G = np.zeros((dk, dv)) if dS_T is None else dS_T[bi, h].copy()
+            g_end = {}
+            dr = np.zeros((T, dv))
+            for t in range(T - 1, -1, -1):
+                if t == T - 1 or (t + 1) % chunk == 0:
+                    g_end[t // chunk] = G.copy()
+                G = G + np.outer(qq[t], do[t])
+                dr[t] = -(kk[t] @ G)
+                out["dv"][bi, t, h] = u[t] @ G
+                G = aa[t][:, None] * (G + np.outer(e[t], dr[t]))
+            out["dS0"][bi, h] = G
+            for c in range((T + chunk - 1) // chunk):
+                t0, t1 = c * chunk, min(T, c * chunk + chunk)
+                n = t1 - t0
+                sl = slice(t0, t1)
+                Q, K, V, E, U, R, DR, DO = qq[sl], kk[sl], vv[sl], e[sl], u[sl], r[sl], dr[sl], do[sl]
+                Gam = np.cumprod(aa[sl], axis=0)
+                S_0, Ge, S_end = states[t0], g_end[c], states[t1]
+                M = np.tril(np.ones((n, n)))
+                M1 = np.tril(np.ones((n, n)), -1)
+                DQ = Gam * (DO @ S_0.T) + Gam * ((M * (DO @ V.T)) @ (U / Gam) - (M * (DO @ R.T)) @ (K / Gam))
+                DE = Gam * (DR @ S_0.T) + Gam * ((M1 * (DR @ V.T)) @ (U / Gam) - (M1 * (DR @ R.T)) @ (K / Gam))
+                QG, EG = Q * Gam, E * Gam
+                DU = ((M.T * (V @ DO.T)) @ QG + (M1.T * (V @ DR.T)) @ EG + (V @ Ge.T) * Gam[-1]) / Gam
+                DKR = -((M.T * (R @ DO.T)) @ QG + (M1.T * (R @ DR.T)) @ EG + (R @ Ge.T) * Gam[-1]) / Gam
+                dlam = Q * DQ + E * DE - U * DU - K * DKR
+                dlam[-1] += np.sum(Ge * S_end, axis=1)
+                dlam = np.cumsum(dlam[::-1], axis=0)[::-1]
+                out["dq"][bi, sl, h] = DQ
+                out["dk"][bi, sl, h] = DKR + Bg[bi, sl, h] * DE + W[bi, sl, h] * DU
+                out["da"][bi, sl, h] = dlam / aa[sl]
+                out["db"][bi, sl, h] = K * DE
+                out["dw"][bi, sl, h] = K * DU
+
+    def shape_like(kind, full):
+        if kind in (None, "none", "tied"):
+            return None
+        return full if kind == "channel" else full.sum(axis=-1)
+    ka, kb, kw = g.get("alpha", "none"), g.get("b", "none"), g.get("w", "none")
+    db_full = out["db"] + (out["dw"] if tied else 0.0)
+    return {"dq": out["dq"], "dk": out["dk"], "dv": out["dv"], "dS0": out["dS0"],
+            "dalpha": shape_like(ka, out["da"]), "db": shape_like(kb, db_full),
+            "dw": shape_like(kw, out["dw"])}

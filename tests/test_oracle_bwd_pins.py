@@ -111,3 +111,27 @@ def test_zero_length_gradient_is_dS_T():
     g = oracle.recurrence_bwd(z(2, 0, 3, 4), z(2, 0, 3, 4), z(2, 0, 3, 5), gates={},
                               S0=z(2, 3, 4, 5), dO=z(2, 0, 3, 5), dS_T=dS_T)
     np.testing.assert_array_equal(g["dS0"], dS_T)
+
+
+@pytest.mark.parametrize("gates", [
+    {"alpha": "channel", "b": "channel", "w": "channel"},
+    {"alpha": "scalar", "b": "scalar", "w": "tied"},
+    {"alpha": "channel", "b": "none", "w": "none"},
+    {"alpha": "none", "b": "scalar", "w": "tied"},
+])
+@pytest.mark.parametrize("T", [1, 8, 21])
+def test_chunkwise_route_agrees(gates, T):
+    """The chunkwise route (masked products per chunk from the scans' r and
+    dr, decay gradient through the running product's logarithm) equals the
+    reverse token loop, including ragged final chunks."""
+    rng = np.random.default_rng(100 + T)
+    q, k, v, a, b, w, S0 = rand_inputs(rng, 2, T, 2, 5, 4, gates, s0=True, k_unit=False)
+    dO = rng.standard_normal(v.shape)
+    dS_T = rng.standard_normal(S0.shape)
+    ref = oracle.recurrence_bwd(q, k, v, a, b, w, S0, gates, dO, dS_T)
+    got = oracle.chunkwise_bwd(q, k, v, a, b, w, S0, gates, dO, dS_T, chunk=8)
+    for n, x in ref.items():
+        if x is None:
+            assert got[n] is None, n
+        else:
+            np.testing.assert_allclose(got[n], x, atol=1e-10 * max(1.0, np.abs(x).max()), err_msg=n)
