@@ -310,7 +310,7 @@ def time_backward(dev, steps, warmup, pk):
     return {"workload": f"Gated DeltaNet backward B={wl.B} H={wl.H} T={wl.T} d_k=d_v={wl.dk} bf16 "
                         f"inputs, fp32 gradients, dO and dS_T ~ N(0, 1)",
             "ms_per_call": ms, "tokens_per_s": wl.B * wl.T / (ms * 1e-3), "launches_per_call": 3,
-            "kernel": "gdr::bwd::bwd_scan_kernel + gdr::bwd::bwd_chunk_kernel + gdr::bwd::bwd_gate_sum_kernel",
+            "kernel": "gdr::bwd::bwd_scan_staged_kernel + gdr::bwd::bwd_chunk_kernel + gdr::bwd::bwd_gate_sum_kernel",
             "roofline": {"bound": "alu", "achieved": achieved, "peak": ALU_FP32_TFLOPS,
                          "unit": "TFLOP/s", "frac": achieved / ALU_FP32_TFLOPS,
                          "peak_source": "derived: 148 SMs x 128 fp32 lanes x 2 x 1965 MHz",

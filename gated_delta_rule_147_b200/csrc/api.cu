@@ -32,7 +32,7 @@ cudaError_t launch_chunk_twopass_general(const CUtensorMap* maps,
                                          const void* b, const void* w, int akind, int bkind,
                                          int wkind, const float* S0, void* o, float* ST,
                                          int* d_status, int B, int T, int H, int dv, int group,
-                                         cudaStream_t st);
+                                         bool allow_segments, cudaStream_t st);
 cudaError_t launch_chunk_sm100(const CUtensorMap* maps, const void* alpha, const void* b,
                                const void* w, int akind, int bkind, int wkind, bool tied,
                                const float* S0, void* o, float* ST, int* d_status, int B, int T,
@@ -130,11 +130,18 @@ const char* gdr_status_string(int s) {
 
 int gdr_version(void) { return (1 << 16) | 0; }
 
-gdr_status gdr_chunk_fwd_grouped(const void* q, const void* k, const void* v, const void* alpha,
-                                 const void* b, const void* w, int alpha_kind, int b_kind,
-                                 int w_kind, const float* S0, void* o, float* S_T, void* workspace,
-                                 size_t workspace_bytes, int B, int T, int H_qk, int H, int d_k,
-                                 int d_v, int chunk, int dtype, int* d_status, void* stream) {
+}  // extern "C"
+
+namespace gdr {
+
+// gdr_chunk_fwd_grouped with one more switch: allow_segments = false keeps the
+// general two-pass path on the caller's stream alone (no auxiliary stream or
+// events are created or used).
+gdr_status chunk_fwd_impl(const void* q, const void* k, const void* v, const void* alpha,
+                          const void* b, const void* w, int alpha_kind, int b_kind, int w_kind,
+                          const float* S0, void* o, float* S_T, void* workspace,
+                          size_t workspace_bytes, int B, int T, int H_qk, int H, int d_k, int d_v,
+                          int chunk, int dtype, int* d_status, bool allow_segments, void* stream) {
     if (B < 1 || H < 1 || T < 0 || d_k < 1 || d_v < 1) return GDR_ERR_INVALID_ARG;
     if (H_qk < 1 || H % H_qk != 0) return GDR_ERR_INVALID_ARG;
     const int group = H / H_qk;
@@ -192,7 +199,7 @@ gdr_status gdr_chunk_fwd_grouped(const void* q, const void* k, const void* v, co
         if (tp == TP_GENERAL) {
             e = gdr::launch_chunk_twopass_general(maps, make_map, workspace, q, k, alpha, b, w,
                                                   alpha_kind, b_kind, w_kind, S0, o, S_T, d_status,
-                                                  B, T, H, d_v, group, st);
+                                                  B, T, H, d_v, group, allow_segments, st);
         } else if (tp == TP_GDN) {
             CUtensorMap ws_maps[2];
             const uint8_t* pbase = reinterpret_cast<const uint8_t*>(workspace) +
@@ -213,6 +220,20 @@ gdr_status gdr_chunk_fwd_grouped(const void* q, const void* k, const void* v, co
                                   T, H, d_k, d_v, dtype, group, st);
     }
     return e == cudaSuccess ? GDR_OK : GDR_ERR_LAUNCH;
+}
+
+}  // namespace gdr
+
+extern "C" {
+
+gdr_status gdr_chunk_fwd_grouped(const void* q, const void* k, const void* v, const void* alpha,
+                                 const void* b, const void* w, int alpha_kind, int b_kind,
+                                 int w_kind, const float* S0, void* o, float* S_T, void* workspace,
+                                 size_t workspace_bytes, int B, int T, int H_qk, int H, int d_k,
+                                 int d_v, int chunk, int dtype, int* d_status, void* stream) {
+    return gdr::chunk_fwd_impl(q, k, v, alpha, b, w, alpha_kind, b_kind, w_kind, S0, o, S_T,
+                               workspace, workspace_bytes, B, T, H_qk, H, d_k, d_v, chunk, dtype,
+                               d_status, true, stream);
 }
 
 gdr_status gdr_chunk_fwd(const void* q, const void* k, const void* v, const void* alpha,

@@ -948,9 +948,17 @@ gdr_status gdr_chunk_bwd_grouped(const void* q, const void* k, const void* v, co
     }
     const int nch = (T + gdr::bwd::kC - 1) / gdr::bwd::kC;
     if (nch > 65535 || (size_t)B * H > 65535u) return GDR_ERR_UNSUPPORTED;  // grid limits
-    const void* ptrs[] = {q, k, v, dO, dq, dk, dv, S0, dS_T, dS0, dalpha, db, dw, alpha, b, w};
+    // vector rows move in 16-byte pieces; scalar gates and their gradients are
+    // read and written one element at a time and need only element alignment
+    const void* ptrs[] = {q, k, v, dO, dq, dk, dv, S0, dS_T, dS0};
     for (const void* ptr : ptrs)
         if (ptr && !a16(ptr)) return GDR_ERR_MISALIGNED;
+    const int kinds[3] = {alpha_kind, b_kind, w_kind};
+    const void* gates[3] = {alpha, b, w};
+    const void* grads[3] = {dalpha, db, dw};
+    for (int i = 0; i < 3; ++i)
+        if (kinds[i] == GDR_GATE_CHANNEL && (!a16(gates[i]) || (grads[i] && !a16(grads[i]))))
+            return GDR_ERR_MISALIGNED;
     const bool grouped = H_qk != H;
     const gdr::bwd::WsLayout wl = gdr::bwd::ws_layout(B, T, H, d_k, d_v, grouped);
     if (!workspace || workspace_bytes < wl.total) return GDR_ERR_INVALID_ARG;

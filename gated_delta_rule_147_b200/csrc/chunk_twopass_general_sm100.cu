@@ -911,26 +911,41 @@ using MapFn = bool (*)(CUtensorMap*, const void*, int, int, int, int);
 
 // Segmented state pass: segments of at least kSegMin chunks, at most
 // kMaxSegments. The auxiliary stream and events are created on the first
-// segmented call on a device and kept for the process.
+// segmented call on a device and kept for the process. They are shared by
+// every call on that device, so a call holds the device's lock from its first
+// event record to its last stream wait: another call's records can then never
+// be the ones this call waits on. A call that finds the lock taken, or whose
+// stream is being captured into a graph, does not segment (one prep launch,
+// one state launch on the caller's stream).
 constexpr int kSegMin = 32;
 constexpr int kMaxSegments = 8;
 
-static bool aux_resources(int dev, cudaStream_t* aux, cudaEvent_t** evs) {
-    static std::mutex mu;
-    static cudaStream_t streams[64] = {};
-    static cudaEvent_t events[64][kMaxSegments + 1] = {};
-    if (dev < 0 || dev >= 64) return false;
-    std::lock_guard<std::mutex> lock(mu);
-    if (!streams[dev]) {
+struct AuxResources {
+    std::mutex mu;  // held for a whole segmented enqueue sequence
+    cudaStream_t stream = nullptr;
+    cudaEvent_t events[kMaxSegments + 1] = {};
+    bool ready = false;
+};
+
+static AuxResources* aux_resources(int dev) {
+    static std::mutex create_mu;
+    static AuxResources res[64];
+    if (dev < 0 || dev >= 64) return nullptr;
+    std::lock_guard<std::mutex> lock(create_mu);
+    AuxResources& r = res[dev];
+    if (!r.ready) {
         cudaStream_t s = nullptr;
-        if (cudaStreamCreateWithFlags(&s, cudaStreamNonBlocking) != cudaSuccess) return false;
+        if (cudaStreamCreateWithFlags(&s, cudaStreamNonBlocking) != cudaSuccess) return nullptr;
         for (int i = 0; i <= kMaxSegments; ++i)
-            if (cudaEventCreateWithFlags(&events[dev][i], cudaEventDisableTiming) != cudaSuccess) return false;
-        streams[dev] = s;
+            if (cudaEventCreateWithFlags(&r.events[i], cudaEventDisableTiming) != cudaSuccess) {
+                for (int j = 0; j < i; ++j) cudaEventDestroy(r.events[j]);
+                cudaStreamDestroy(s);
+                return nullptr;
+            }
+        r.stream = s;
+        r.ready = true;
     }
-    *aux = streams[dev];
-    *evs = events[dev];
-    return true;
+    return &r;
 }
 
 // maps: q, k, v (of the call). alpha/b/w kinds as in the C ABI.
@@ -939,7 +954,7 @@ cudaError_t launch_chunk_twopass_general(const CUtensorMap* maps, MapFn make_map
                                          const void* b, const void* w, int akind, int bkind,
                                          int wkind, const float* S0, void* o, float* ST,
                                          int* d_status, int B, int T, int H, int dv, int group,
-                                         cudaStream_t st) {
+                                         bool allow_segments, cudaStream_t st) {
     using namespace twopass_g;
     const bool tied = wkind == GDR_GATE_TIED && bkind == GDR_GATE_SCALAR;
     const bool ach = akind == GDR_GATE_CHANNEL;
@@ -1008,27 +1023,31 @@ cudaError_t launch_chunk_twopass_general(const CUtensorMap* maps, MapFn make_map
     // segments run on an auxiliary stream while the state pass works through
     // earlier ones (ordered by events only).
     int nseg = 1;
-    cudaStream_t aux = nullptr;
-    cudaEvent_t* evs = nullptr;
+    AuxResources* aux = nullptr;
+    std::unique_lock<std::mutex> aux_lock;
     int dev = 0, nsm = 0;
-    if (cudaGetDevice(&dev) == cudaSuccess &&
+    cudaStreamCaptureStatus cap = cudaStreamCaptureStatusNone;
+    if (allow_segments && cudaGetDevice(&dev) == cudaSuccess &&
         cudaDeviceGetAttribute(&nsm, cudaDevAttrMultiProcessorCount, dev) == cudaSuccess &&
-        (int)(sgrid.x * sgrid.y * sgrid.z) * 2 <= nsm && nchunks >= 2 * kSegMin) {
-        nseg = min(kMaxSegments, nchunks / kSegMin);
-        if (!aux_resources(dev, &aux, &evs)) nseg = 1;
+        (int)(sgrid.x * sgrid.y * sgrid.z) * 2 <= nsm && nchunks >= 2 * kSegMin &&
+        cudaStreamIsCapturing(st, &cap) == cudaSuccess && cap == cudaStreamCaptureStatusNone &&
+        (aux = aux_resources(dev)) != nullptr) {
+        aux_lock = std::unique_lock<std::mutex>(aux->mu, std::try_to_lock);
+        if (aux_lock.owns_lock()) nseg = min(kMaxSegments, nchunks / kSegMin);
     }
     if (nseg == 1) {
         cudaError_t e = prep_range(0, nchunks, st);
         if (e != cudaSuccess) return e;
         return state_range(0, nchunks, S0, ST);
     }
+    cudaEvent_t* evs = aux->events;
     float* carry = reinterpret_cast<float*>(base + lay.off[8]);
     cudaError_t e = cudaEventRecord(evs[kMaxSegments], st);
-    if (e == cudaSuccess) e = cudaStreamWaitEvent(aux, evs[kMaxSegments], 0);
+    if (e == cudaSuccess) e = cudaStreamWaitEvent(aux->stream, evs[kMaxSegments], 0);
     for (int sgi = 0; sgi < nseg && e == cudaSuccess; ++sgi) {
         const int c0 = (int)((long long)nchunks * sgi / nseg), c1 = (int)((long long)nchunks * (sgi + 1) / nseg);
-        e = prep_range(c0, c1, sgi == 0 ? st : aux);
-        if (e == cudaSuccess && sgi > 0) e = cudaEventRecord(evs[sgi], aux);
+        e = prep_range(c0, c1, sgi == 0 ? st : aux->stream);
+        if (e == cudaSuccess && sgi > 0) e = cudaEventRecord(evs[sgi], aux->stream);
     }
     for (int sgi = 0; sgi < nseg && e == cudaSuccess; ++sgi) {
         const int c0 = (int)((long long)nchunks * sgi / nseg), c1 = (int)((long long)nchunks * (sgi + 1) / nseg);
@@ -1036,6 +1055,7 @@ cudaError_t launch_chunk_twopass_general(const CUtensorMap* maps, MapFn make_map
         if (e == cudaSuccess)
             e = state_range(c0, c1, sgi == 0 ? S0 : carry, sgi == nseg - 1 ? ST : carry);
     }
+    // every wait of this call is enqueued: later records cannot affect them
     return e;
 }
 

@@ -9,6 +9,7 @@
 #include <stdint.h>
 
 #include "../../include/gdr.h"
+#include "rcp_seed.h"
 
 namespace gdr {
 
@@ -48,16 +49,9 @@ __device__ __forceinline__ float lg2_approx(float x) {
     return y;
 }
 
-// 1/a for positive normal a by Newton-Raphson, x <- x (2 - a x), from a seed
-// that flips the exponent bits (relative error of the seed below 1/8, so
-// three steps reach fp32 precision). Runs on the FMA pipe.
-__device__ __forceinline__ float rcp_newton(float a) {
-    float x = __int_as_float(0x7EF311C7 - __float_as_int(a));
-    x = x * fmaf(-a, x, 2.f);
-    x = x * fmaf(-a, x, 2.f);
-    x = x * fmaf(-a, x, 2.f);
-    return x;
-}
+// 1/a for positive normal a by Newton-Raphson from a bit-pattern seed
+// (derivation of the seed and the error per step in rcp_seed.h).
+__device__ __forceinline__ float rcp_newton(float a) { return gdr_rcp_newton3(a); }
 
 __device__ __forceinline__ uint32_t pack_bf16x2(float lo, float hi) {
     __nv_bfloat162 h = __floats2bfloat162_rn(lo, hi);

@@ -10,6 +10,14 @@
 
 #include "gdr.h"
 
+namespace gdr {
+gdr_status chunk_fwd_impl(const void* q, const void* k, const void* v, const void* alpha,
+                          const void* b, const void* w, int alpha_kind, int b_kind, int w_kind,
+                          const float* S0, void* o, float* S_T, void* workspace,
+                          size_t workspace_bytes, int B, int T, int H_qk, int H, int d_k, int d_v,
+                          int chunk, int dtype, int* d_status, bool allow_segments, void* stream);
+}  // namespace gdr
+
 namespace {
 
 constexpr size_t kStaticScratchBytes = size_t(64) << 20;  // 64 MiB
@@ -47,8 +55,9 @@ gdr_status gdr_chunk_fwd_static(const void* q, const void* k, const void* v, con
         }
         ws = g_scratch_addr[dev];
     }
-    return gdr_chunk_fwd(q, k, v, alpha, b, w, alpha_kind, b_kind, w_kind, S0, o, S_T, ws, need, B,
-                         T, H, d_k, d_v, chunk, dtype, d_status, stream);
+    // no auxiliary stream or events: this call creates no CUDA objects either
+    return gdr::chunk_fwd_impl(q, k, v, alpha, b, w, alpha_kind, b_kind, w_kind, S0, o, S_T, ws,
+                               need, B, T, H, H, d_k, d_v, chunk, dtype, d_status, false, stream);
 }
 
 }  // extern "C"

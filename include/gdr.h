@@ -27,7 +27,11 @@
  * ---------------------------------------
  * Pointers: every array argument is a DEVICE pointer (memory the CUDA device
  *   can read/write). The caller owns every buffer; the library allocates no
- *   memory, keeps no state between calls and never frees caller memory.
+ *   device memory, keeps no data between calls and never frees caller
+ *   memory. The one CUDA object it keeps is described at
+ *   gdr_chunk_fwd_workspace_size: an auxiliary stream and a few events per
+ *   device, created by the first call that splits a general-form state pass
+ *   into segments.
  * Layouts (contiguous, row-major, innermost last):
  *   q, k        [B, T, H, d_k]       chunk forward;  [B, H, d_k] decode
  *   v, o        [B, T, H, d_v]                       [B, H, d_v]
@@ -163,7 +167,13 @@ gdr_status gdr_chunk_fwd_grouped(const void* q, const void* k, const void* v,
  * general form splits the state pass into segments and runs the first pass of
  * later segments on an auxiliary stream while the state pass works through
  * earlier ones; the library then keeps that stream and a few events per
- * device for the rest of the process.
+ * device for the rest of the process. Those are shared by every call on the
+ * device: a call holds a per-device lock from its first event record to its
+ * last stream wait, so concurrent calls from several host threads never wait
+ * on each other's events. A call that finds the lock held by another thread,
+ * or whose stream is being captured into a CUDA graph, does not split (it
+ * launches one first pass and one state pass on its own stream), and so
+ * neither touches the auxiliary stream nor serialises behind another caller.
  * Host-only; launches nothing.
  */
 size_t gdr_chunk_fwd_workspace_size(int B, int T, int H, int d_k, int d_v,
@@ -187,7 +197,9 @@ size_t gdr_chunk_fwd_workspace_size(int B, int T, int H, int d_k, int d_v,
  * running concurrently) race on it and corrupt each other's results;
  * serialise them. The first call on each device looks the array up
  * (cudaGetSymbolAddress, which may load the module): make it before any
- * stream capture that records later calls.
+ * stream capture that records later calls. This call never splits the
+ * general-form state pass into segments, so it creates no stream or event:
+ * everything it launches goes to `stream`.
  */
 gdr_status gdr_chunk_fwd_static(const void* q, const void* k, const void* v,
                                 const void* alpha, const void* b, const void* w,
@@ -238,7 +250,8 @@ size_t gdr_chunk_fwd_static_capacity(void);
  *   key channels. Deterministic (no atomics). d_status is not used (no
  *   bounded waits on this path).
  * Supported: chunk = 64, 1 <= d_k <= 128, d_v a multiple of 8 up to 256,
- *   ceil(T / 64) <= 65535 and B * H <= 65535. Every pointer 16-byte aligned.
+ *   ceil(T / 64) <= 65535 and B * H <= 65535. Every pointer 16-byte
+ *   aligned, except scalar gates and their gradients (element aligned).
  * Returns GDR_OK, GDR_ERR_INVALID_ARG (bad sizes or kinds, a NULL array that
  * is required, a gradient pointer that does not match its gate, workspace
  * missing or too small), GDR_ERR_UNSUPPORTED, GDR_ERR_MISALIGNED or

@@ -363,7 +363,13 @@ def chunkwise_bwd(q, k, v, alpha=None, b=None, w=None, S0=None, gates=None, dO=N
     minus writers, q.dq + e.de - u.du - k.dkr, plus rowsum(Ge . S_end) on the
     chunk's last token, summed from each token to the chunk end, divided by
     alpha. Returns the dict of `recurrence_bwd` (per-channel gates only
-    materialised: scalar and tied forms are summed / merged as there)."""
+    materialised: scalar and tied forms are summed / merged as there).
+
+    Validity domain: alpha > 0 and short chunks (default 8 tokens). The route
+    divides by running products of alpha inside a chunk (U/Gam, K/Gam, /Gam)
+    and by alpha itself; it refuses (AssertionError) a chunk whose running
+    product falls below 1e-200, where those quotients lose their precision.
+    Outside that domain use `recurrence_bwd`, the reverse token loop."""
     q, k, v = f64(q), f64(k), f64(v)
     B, T, H, dk = q.shape
     dv = v.shape[-1]
@@ -408,6 +414,8 @@ def chunkwise_bwd(q, k, v, alpha=None, b=None, w=None, S0=None, gates=None, dO=N
                 sl = slice(t0, t1)
                 Q, K, V, E, U, R, DR, DO = qq[sl], kk[sl], vv[sl], e[sl], u[sl], r[sl], dr[sl], do[sl]
                 Gam = np.cumprod(aa[sl], axis=0)
+                assert Gam.min() > 1e-200, "chunkwise_bwd: running decay product underflows; " \
+                    "use a shorter chunk or recurrence_bwd"
                 S_0, Ge, S_end = states[t0], g_end[c], states[t1]
                 M = np.tril(np.ones((n, n)))
                 M1 = np.tril(np.ones((n, n)), -1)

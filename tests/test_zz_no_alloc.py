@@ -64,3 +64,20 @@ def test_static_scratch_matches_caller_workspace_twice(cuda_device, family):
         assert torch.equal(o_ref.view(torch.int16), o_st.view(torch.int16))
         assert torch.equal(S_ref, S_st)
         assert np.isfinite(o_st.float().numpy()).all()
+
+
+@pytest.mark.gpu
+def test_static_scratch_long_sequence_few_heads(cuda_device):
+    """A shape whose caller-workspace call splits the general state pass into
+    segments (few heads, long sequence) and still fits the static array: the
+    static call keeps one stream and gives the same bits."""
+    wl = WORKLOADS["gdn2"].with_(B=1, H=2, T=9000, s0=True, seed=503)
+    need = _lib.gdr_chunk_fwd_workspace_size(1, 9000, 2, 128, 128, KIND["channel"], KIND["channel"],
+                                             KIND["channel"], GDR_BF16)
+    assert 0 < need <= _lib.gdr_chunk_fwd_static_capacity()
+    inp = make_chunk_inputs(wl)
+    for _ in range(2):
+        o_ref, S_ref = _run(inp, cuda_device, static=False)
+        o_st, S_st = _run(inp, cuda_device, static=True)
+        assert torch.equal(o_ref.view(torch.int16), o_st.view(torch.int16))
+        assert torch.equal(S_ref, S_st)
