@@ -16,7 +16,8 @@ cudaError_t launch_recurrent(const void* q, const void* k, const void* v, const 
                              const void* b, const void* w, int ak, int bk, int wk, const float* S0,
                              void* o, float* ST, int B, int T, int H, int dk, int dv, int dtype,
                              int group, cudaStream_t st);
-cudaError_t launch_chunk_erasefree_sm100(const CUtensorMap* maps, const void* alpha, const void* w,
+cudaError_t launch_chunk_erasefree_sm100(const CUtensorMap* maps, const void* q, const void* k,
+                                         const void* v, const void* alpha, const void* w,
                                          int akind, int wkind, const float* S0, void* o, float* ST,
                                          int* d_status, int B, int T, int H, int dv, int group,
                                          cudaStream_t st);
@@ -28,12 +29,14 @@ cudaError_t launch_chunk_twopass_gdn(const CUtensorMap* maps, const CUtensorMap*
 size_t twopass_general_workspace_bytes(int B, int T, int H, int dv, bool untied);
 cudaError_t launch_chunk_twopass_general(const CUtensorMap* maps,
                                          bool (*make_map)(CUtensorMap*, const void*, int, int, int, int),
-                                         void* ws, const void* q, const void* k, const void* alpha,
+                                         void* ws, const void* q, const void* k, const void* v,
+                                         const void* alpha,
                                          const void* b, const void* w, int akind, int bkind,
                                          int wkind, const float* S0, void* o, float* ST,
                                          int* d_status, int B, int T, int H, int dv, int group,
                                          bool allow_segments, cudaStream_t st);
-cudaError_t launch_chunk_sm100(const CUtensorMap* maps, const void* alpha, const void* b,
+cudaError_t launch_chunk_sm100(const CUtensorMap* maps, const void* q, const void* k, const void* v,
+                               const void* alpha, const void* b,
                                const void* w, int akind, int bkind, int wkind, bool tied,
                                const float* S0, void* o, float* ST, int* d_status, int B, int T,
                                int H, int dv, int group, cudaStream_t st);
@@ -197,7 +200,7 @@ gdr_status chunk_fwd_impl(const void* q, const void* k, const void* v, const voi
             return GDR_ERR_INVALID_ARG;
         const bool tied = w_kind == GDR_GATE_TIED && b_kind == GDR_GATE_SCALAR;
         if (tp == TP_GENERAL) {
-            e = gdr::launch_chunk_twopass_general(maps, make_map, workspace, q, k, alpha, b, w,
+            e = gdr::launch_chunk_twopass_general(maps, make_map, workspace, q, k, v, alpha, b, w,
                                                   alpha_kind, b_kind, w_kind, S0, o, S_T, d_status,
                                                   B, T, H, d_v, group, allow_segments, st);
         } else if (tp == TP_GDN) {
@@ -210,10 +213,10 @@ gdr_status chunk_fwd_impl(const void* q, const void* k, const void* v, const voi
             e = gdr::launch_chunk_twopass_gdn(maps, ws_maps, workspace, alpha, b, S0, o, S_T,
                                               d_status, B, T, H, d_v, group, st);
         } else if (b_kind == GDR_GATE_NONE)  // no erase: no triangular solve
-            e = gdr::launch_chunk_erasefree_sm100(maps, alpha, w, alpha_kind, w_kind, S0, o, S_T,
+            e = gdr::launch_chunk_erasefree_sm100(maps, q, k, v, alpha, w, alpha_kind, w_kind, S0, o, S_T,
                                                   d_status, B, T, H, d_v, group, st);
         else
-            e = gdr::launch_chunk_sm100(maps, alpha, b, w, alpha_kind, b_kind, w_kind, tied, S0, o,
+            e = gdr::launch_chunk_sm100(maps, q, k, v, alpha, b, w, alpha_kind, b_kind, w_kind, tied, S0, o,
                                         S_T, d_status, B, T, H, d_v, group, st);
     } else {
         e = gdr::launch_recurrent(q, k, v, alpha, b, w, alpha_kind, b_kind, w_kind, S0, o, S_T, B,

@@ -13,6 +13,7 @@ constexpr int NV = 64;    // value columns per CTA
 constexpr int NT = 256;   // threads per CTA (two warpgroups)
 
 struct Params {
+    const void *q, *k, *v;  // raw inputs (for chunks that take the exact path)
     const void* alpha;  // scalar gates are read with plain loads
     const void* bg;
     const void* wg;
@@ -184,6 +185,131 @@ __device__ __forceinline__ void solve_unit_lower(float* A32, float* T32, float* 
         *f32_at(T32, 32 + 16 * mt + gq + 8, 8 * nt + 2 * tq + 1) = -acc[3];
     }
     __syncthreads();
+}
+
+}  // namespace chunkc
+}  // namespace gdr
+
+namespace gdr {
+namespace chunkc {
+
+// Raw inputs of a head for the exact token-by-token fallback.
+struct ExactArgs {
+    const __nv_bfloat16 *q, *k, *v, *alpha, *b, *w;
+    int akind, bkind, wkind;
+    __nv_bfloat16* o;
+    int T, H, Hq, dv;
+};
+
+// Barrier over threads 0..255 only (named barrier 1): the whole block in the
+// 256-thread kernels, the compute warps where a further warp issues MMAs.
+__device__ __forceinline__ void compute_bar() {
+    asm volatile("bar.sync 1, 256;" ::: "memory");
+}
+
+// In lane l, the sum over the warp's 32 lanes of x[l] (a reduce-scatter by
+// recursive halving: 31 shuffles for 32 columns). x is destroyed.
+__device__ __forceinline__ float warp_colsum32(float* x, int lane) {
+#pragma unroll
+    for (int off = 16; off >= 1; off >>= 1) {
+        const bool up = (lane & off) != 0;
+#pragma unroll
+        for (int i = 0; i < off; ++i) {
+            const float send = up ? x[i] : x[i + off];
+            const float keep = up ? x[i + off] : x[i];
+            x[i] = keep + __shfl_xor_sync(0xffffffffu, send, off);
+        }
+    }
+    return x[0];
+}
+
+// Tokens [t0, t0 + n) of head (bb, h) applied exactly in fp32 to the block's
+// 128 x (2 NPT) state slice (thread: state row `row` = tid & 127, columns
+// v0 + wg * NPT + 0..NPT-1 in S[NPT], wg = tid >> 7), token by token as the
+// recurrence defines it: S <- Diag(alpha) S; r = (b.k) S; S <- S - k^T r +
+// (w.k)^T v; o = q S. Writes o of those tokens and columns. Used for a chunk
+// whose decay span is outside what the tensor-core factorisation can hold.
+// Threads 0..255; red is shared scratch of 18 NPT floats; ends with a barrier.
+template <int NPT>
+__device__ __forceinline__ void exact_tokens(const ExactArgs& a, float (&S)[NPT], float* red, int bb,
+                                             int h, int hq, int v0, int t0, int n, int tid) {
+    static_assert(NPT % 32 == 0, "columns per thread: a multiple of 32");
+    const int row = tid & 127, wg = tid >> 7, w4 = (tid >> 5) & 3, lane = tid & 31;
+    float* redR = red;                 // [2][4][NPT] per-warp partial sums
+    float* redO = red + 8 * NPT;       // [2][4][NPT]
+    float* r2 = red + 16 * NPT;        // [2][NPT] erase reads r
+    auto bf = [](__nv_bfloat16 x) { return __bfloat162float(x); };
+    for (int tt = 0; tt < n; ++tt) {
+        const int t = t0 + tt;
+        const size_t tk = ((size_t)bb * a.T + t) * a.H + h;
+        const size_t tq = ((size_t)bb * a.T + t) * a.Hq + hq;
+        const float kr = bf(a.k[tq * DK + row]), qr = bf(a.q[tq * DK + row]);
+        const float ar = a.akind == GDR_GATE_CHANNEL ? bf(a.alpha[tk * DK + row])
+                         : a.akind == GDR_GATE_SCALAR ? bf(a.alpha[tk]) : 1.f;
+        const float br = a.bkind == GDR_GATE_CHANNEL ? bf(a.b[tk * DK + row])
+                         : a.bkind == GDR_GATE_SCALAR ? bf(a.b[tk]) : 0.f;
+        const float wr = a.wkind == GDR_GATE_TIED ? br
+                         : a.wkind == GDR_GATE_CHANNEL ? bf(a.w[tk * DK + row])
+                         : a.wkind == GDR_GATE_SCALAR ? bf(a.w[tk]) : 1.f;
+        const uint4* vp = reinterpret_cast<const uint4*>(a.v + tk * a.dv + v0 + wg * NPT);
+        // decay, then the erase read r = (b.k) S over the 128 rows
+        const float er = br * kr;
+#pragma unroll
+        for (int g = 0; g < NPT / 32; ++g) {
+            float x[32];
+#pragma unroll
+            for (int j = 0; j < 32; ++j) {
+                S[g * 32 + j] *= ar;
+                x[j] = er * S[g * 32 + j];
+            }
+            redR[(wg * 4 + w4) * NPT + g * 32 + lane] = warp_colsum32(x, lane);
+        }
+        compute_bar();
+        if (w4 == 0) {
+#pragma unroll
+            for (int g = 0; g < NPT / 32; ++g) {
+                const int c = g * 32 + lane;
+                r2[wg * NPT + c] = redR[(wg * 4) * NPT + c] + redR[(wg * 4 + 1) * NPT + c] +
+                                   redR[(wg * 4 + 2) * NPT + c] + redR[(wg * 4 + 3) * NPT + c];
+            }
+        }
+        compute_bar();
+        // erase along k, write with key w.k, then the read o = q S
+        const float ur = wr * kr;
+#pragma unroll
+        for (int g = 0; g < NPT / 32; ++g) {
+            float v[32], x[32];  // 32 columns of v at a time
+#pragma unroll
+            for (int c = 0; c < 4; ++c) {
+                const uint4 u = vp[g * 4 + c];
+                const __nv_bfloat162* hh = reinterpret_cast<const __nv_bfloat162*>(&u);
+#pragma unroll
+                for (int e = 0; e < 4; ++e) {
+                    const float2 f = __bfloat1622float2(hh[e]);
+                    v[c * 8 + 2 * e] = f.x;
+                    v[c * 8 + 2 * e + 1] = f.y;
+                }
+            }
+#pragma unroll
+            for (int j = 0; j < 32; ++j) {
+                const int c = g * 32 + j;
+                S[c] = fmaf(-kr, r2[wg * NPT + c], fmaf(ur, v[j], S[c]));
+                x[j] = qr * S[c];
+            }
+            redO[(wg * 4 + w4) * NPT + g * 32 + lane] = warp_colsum32(x, lane);
+        }
+        compute_bar();
+        if (w4 == 0) {
+#pragma unroll
+            for (int g = 0; g < NPT / 32; ++g) {
+                const int c = g * 32 + lane;
+                const float ov = redO[(wg * 4) * NPT + c] + redO[(wg * 4 + 1) * NPT + c] +
+                                 redO[(wg * 4 + 2) * NPT + c] + redO[(wg * 4 + 3) * NPT + c];
+                a.o[tk * a.dv + v0 + wg * NPT + c] = __float2bfloat16_rn(ov);
+            }
+        }
+    }
+    compute_bar();
 }
 
 }  // namespace chunkc

@@ -169,6 +169,7 @@ __global__ void __launch_bounds__(NT, 1) chunk_fwd_erasefree_kernel(
             const int cg = tid & 31, rg = warp;  // 8 tokens x 4 channels per thread
             const int ch0 = cg * 4;
             float* scan = reinterpret_cast<float*>(sm + OFF_SCAN);
+            bool chunk_bad = false;  // decay span beyond the factorisation's range
             float lrow[8][4], aval[8][4];
             if (!ACH) {
                 if (warp == 0) {
@@ -193,10 +194,11 @@ __global__ void __launch_bounds__(NT, 1) chunk_fwd_erasefree_kernel(
                         scan[0] = ex2_approx(ref);
                         scan[1] = ex2_approx(last);
                         scan[2] = ex2_approx(last - ref);
-                        if (first - last > 230.f) flag_status(p.d_status, GDR_DEVICE_DECAY_RANGE);
+                        scan[3] = first - last > 230.f ? 1.f : 0.f;
                     }
                 }
                 __syncthreads();
+                chunk_bad = scan[3] != 0.f;
                 if (tid < 128) {
                     s_eref[tid] = scan[0];
                     s_gC[tid] = scan[1];
@@ -242,7 +244,7 @@ __global__ void __launch_bounds__(NT, 1) chunk_fwd_erasefree_kernel(
 #pragma unroll
                     for (int i = 0; i < 8; ++i) lrow[i][e] += pre[e] - ref[e];
                 }
-                if (bad) flag_status(p.d_status, GDR_DEVICE_DECAY_RANGE);
+                chunk_bad = bad;
                 if (rg == 0) {
 #pragma unroll
                     for (int e = 0; e < 4; ++e) {
@@ -252,6 +254,24 @@ __global__ void __launch_bounds__(NT, 1) chunk_fwd_erasefree_kernel(
                     }
                 }
                 __syncthreads();  // s_eref of every channel is needed below
+            }
+            if (__syncthreads_or(chunk_bad)) {
+                // the chunk's decay ratios do not fit two bounded factors: apply
+                // its tokens one by one (fp32, raw inputs), then go on
+                if (tid == 0) flag_status(p.d_status, GDR_DEVICE_DECAY_RANGE);
+                if (tid == 0 && ci + 1 < nchunks) issue_loads(ci + 1);
+                const ExactArgs ex{(const __nv_bfloat16*)p.q, (const __nv_bfloat16*)p.k,
+                                   (const __nv_bfloat16*)p.v, (const __nv_bfloat16*)p.alpha,
+                                   nullptr, (const __nv_bfloat16*)p.wg,
+                                   p.akind, GDR_GATE_NONE, p.wkind, p.o, T, H, H / p.group, p.dv};
+                exact_tokens(ex, S, scan, bb, h, hq, v0, t0, n, tid);
+#pragma unroll
+                for (int ch = 0; ch < NH / 8; ++ch)
+                    st_chunk(sm + OFF_SBF, sw128_chunk(row, wg * (NH / 8) + ch, DK), &S[8 * ch]);
+                fence_proxy_async();
+                tc_fence_before();
+                __syncthreads();
+                continue;
             }
             float er[4];
             if (ACH) {
@@ -405,11 +425,13 @@ finish:
 }  // namespace erasefree
 
 // maps: q, k, v, alpha (channel) or q, w (channel) or q
-cudaError_t launch_chunk_erasefree_sm100(const CUtensorMap* maps, const void* alpha, const void* w,
+cudaError_t launch_chunk_erasefree_sm100(const CUtensorMap* maps, const void* q, const void* k,
+                                         const void* v, const void* alpha, const void* w,
                                          int akind, int wkind, const float* S0, void* o, float* ST,
                                          int* d_status, int B, int T, int H, int dv, int group,
                                          cudaStream_t st) {
     chunkc::Params p;
+    p.q = q; p.k = k; p.v = v;
     p.alpha = alpha; p.bg = nullptr; p.wg = w;
     p.S0 = S0; p.o = (__nv_bfloat16*)o; p.ST = ST; p.d_status = d_status;
     p.B = B; p.T = T; p.H = H; p.dv = dv;

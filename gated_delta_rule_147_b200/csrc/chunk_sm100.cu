@@ -246,6 +246,7 @@ __global__ void __launch_bounds__(NT, 1) chunk_fwd_kernel(
                 *reinterpret_cast<uint2*>(sm + base + piece(r, rows)) = u;
             };
             float* scan = reinterpret_cast<float*>(sm + OFF_SCAN);  // [8 rg][128 ch] + [128]
+            bool chunk_bad = false;  // decay span beyond the factorisation's range
             float lrow[8][4];  // channel decay: l_r - ref
             float aval[8][4];  // channel decay: alpha of this thread's tokens
             if (!ach) {
@@ -272,10 +273,11 @@ __global__ void __launch_bounds__(NT, 1) chunk_fwd_kernel(
                         scan[0] = ex2_approx(ref);
                         scan[1] = ex2_approx(last);
                         scan[2] = ex2_approx(last - ref);
-                        if (first - last > 230.f) flag_status(p.d_status, GDR_DEVICE_DECAY_RANGE);
+                        scan[3] = first - last > 230.f ? 1.f : 0.f;
                     }
                 }
                 __syncthreads();
+                chunk_bad = scan[3] != 0.f;
                 if (tid < 128) {
                     s_eref[tid] = scan[0];
                     s_gC[tid] = scan[1];
@@ -321,7 +323,7 @@ __global__ void __launch_bounds__(NT, 1) chunk_fwd_kernel(
 #pragma unroll
                     for (int i = 0; i < 8; ++i) lrow[i][e] += pre[e] - ref[e];
                 }
-                if (bad) flag_status(p.d_status, GDR_DEVICE_DECAY_RANGE);
+                chunk_bad = bad;
                 if (rg == 0) {
 #pragma unroll
                     for (int e = 0; e < 4; ++e) {
@@ -330,6 +332,24 @@ __global__ void __launch_bounds__(NT, 1) chunk_fwd_kernel(
                         s_fS[ch0 + e] = ex2_approx(tot[e] - ref[e]);
                     }
                 }
+            }
+            if (__syncthreads_or(chunk_bad)) {
+                // the chunk's decay ratios do not fit two bounded factors: apply
+                // its tokens one by one (fp32, raw inputs), then go on
+                if (tid == 0) flag_status(p.d_status, GDR_DEVICE_DECAY_RANGE);
+                if (tid == 0 && ci + 1 < nchunks) issue_loads(ci + 1);
+                if (ci + 1 < nchunks) load_scalar_gates(ci + 1);
+                const ExactArgs ex{(const __nv_bfloat16*)p.q, (const __nv_bfloat16*)p.k,
+                                   (const __nv_bfloat16*)p.v, (const __nv_bfloat16*)p.alpha,
+                                   (const __nv_bfloat16*)p.bg, (const __nv_bfloat16*)p.wg,
+                                   p.akind, p.bkind, p.wkind, p.o, T, H, H / p.group, p.dv};
+                exact_tokens(ex, S, reinterpret_cast<float*>(sm + OFF_U), bb, h, hq, v0, t0, n, tid);
+#pragma unroll
+                for (int ch = 0; ch < 4; ++ch) st_chunk(sm + OFF_SBF, sw128_chunk(row, wg * 4 + ch, DK), &S[8 * ch]);
+                fence_proxy_async();
+                tc_fence_before();
+                __syncthreads();
+                continue;
             }
             float rowf_c[4];
 #pragma unroll
@@ -688,13 +708,14 @@ finish:
 // Every scale factor is per token, so it folds into MMA outputs or into the
 // small T-derived operands and the raw q / k tiles from TMA are the MMA
 // operands (no operand build):
-//   A  = Diag(beta rowf) (K K^T) Diag(colf)  (strict lower)     [D1 unload]
-//   Aq = Diag(rowf) (Q K^T) Diag(colf)       (lower)            [D1 unload]
+//   A  = Diag(beta) ((K K^T) . G)            (strict lower)     [D1 unload]
+//   Aq = (Q K^T) . G                         (lower)            [D1 unload]
 //   W  = T Diag(beta g) K                     (P2, A = [T Diag(beta g) ; 0])
 //   U  = T Diag(beta) V - W S                 (P3 pre-load + S1)
 //   O  = Diag(g) (Q S) + Aq U                 (S1 gives Q S, S2 gives Aq U)
 //   S' = g_{n-1} S + (Diag(g_{n-1}/g) K)^T U  (K copy scaled per token, S2)
-// with g_r = 2^l_r and rowf_r colf_j = g_r / g_j around the chunk's reference.
+// with g_r = 2^l_r and G_rj = g_r / g_j = 2^(l_r - l_j), formed per element on
+// the unload (at most 1 wherever it is used, so every alpha in (0, 1] is in range).
 // Inputs are double-buffered: the next chunk's TMA is issued as a chunk starts.
 namespace gdn {
 constexpr uint32_t OFF_QK = 0;          // [K ; Q] bf16 [128 x 128], 2 buffers; rows 0..63 become -W
@@ -731,8 +752,7 @@ __global__ void __launch_bounds__(NT, 1) chunk_fwd_gdn_kernel(
     // per-token factors, double-buffered by chunk parity (the next chunk's are
     // computed while the current chunk's last MMA runs): [2][64] each
     float* s_beta2 = reinterpret_cast<float*>(sm + gdn::OFF_SMALL);
-    float* s_rowf2 = s_beta2 + 128;
-    float* s_colf2 = s_beta2 + 256;
+    float* s_l2 = s_beta2 + 128;   // [2][64] log2 prefix of alpha over the chunk
     float* s_g2 = s_beta2 + 384;
     float* s_gcr2 = s_beta2 + 512;
     float* s_misc2 = s_beta2 + 640;   // [2][4]: g_{n-1}
@@ -819,25 +839,17 @@ __global__ void __launch_bounds__(NT, 1) chunk_fwd_gdn_kernel(
             if (lane >= off) x += y;
         }
         const float l1 = x, l0v = x - la1;
-        const float first = __shfl_sync(0xffffffffu, l0v, 0);
         const float last = __shfl_sync(0xffffffffu, l1, 31);
-        const float ref = 0.5f * (first + last);
-        float* rf = s_rowf2 + par * 64;
-        float* cf = s_colf2 + par * 64;
+        float* l = s_l2 + par * 64;
         float* g = s_g2 + par * 64;
         float* gcr = s_gcr2 + par * 64;
-        rf[2 * lane] = ex2_approx(l0v - ref);
-        rf[2 * lane + 1] = ex2_approx(l1 - ref);
-        cf[2 * lane] = ex2_approx(ref - l0v);
-        cf[2 * lane + 1] = ex2_approx(ref - l1);
+        l[2 * lane] = l0v;
+        l[2 * lane + 1] = l1;
         g[2 * lane] = ex2_approx(l0v);
         g[2 * lane + 1] = ex2_approx(l1);
         gcr[2 * lane] = ex2_approx(last - l0v);
         gcr[2 * lane + 1] = ex2_approx(last - l1);
-        if (lane == 0) {
-            s_misc2[par * 4] = ex2_approx(last);
-            if (first - last > 230.f) flag_status(p.d_status, GDR_DEVICE_DECAY_RANGE);
-        }
+        if (lane == 0) s_misc2[par * 4] = ex2_approx(last);
     };
     // stage chunk ci's gates (threads 0..63 hold them in g_a, g_b)
     auto stage_gates = [&](int ci) {
@@ -881,8 +893,7 @@ __global__ void __launch_bounds__(NT, 1) chunk_fwd_gdn_kernel(
         if (ci + 1 < nchunks) load_scalar_gates(ci + 1);         // consumed before S2 of this chunk
         const int par = ci & 1;
         const float* s_beta = s_beta2 + par * 64;
-        const float* s_rowf = s_rowf2 + par * 64;
-        const float* s_colf = s_colf2 + par * 64;
+        const float* s_l = s_l2 + par * 64;
         const float* s_g = s_g2 + par * 64;
         const float* s_gcr = s_gcr2 + par * 64;
         const float* s_misc = s_misc2 + par * 4;
@@ -926,12 +937,16 @@ __global__ void __launch_bounds__(NT, 1) chunk_fwd_gdn_kernel(
             const int r = row & 63;
             float d[32];
             tmem_ld32(tmem + lane_base + gdn::TM_D1 + wg * 32, d);
-            const float rf = s_rowf[r] * (row < 64 ? s_beta[r] : 1.f);
+            // decay ratio g_r / g_j = 2^(l_r - l_j) per element (at most 1 where used)
+            const float rf = row < 64 ? s_beta[r] : 1.f, lr = s_l[r];
             float cf[32];
 #pragma unroll
             for (int j4 = 0; j4 < 32; j4 += 4) {
-                const float4 c4v = *reinterpret_cast<const float4*>(s_colf + wg * 32 + j4);
-                cf[j4] = c4v.x; cf[j4 + 1] = c4v.y; cf[j4 + 2] = c4v.z; cf[j4 + 3] = c4v.w;
+                const float4 l4 = *reinterpret_cast<const float4*>(s_l + wg * 32 + j4);
+                cf[j4] = ex2_approx(fminf(lr - l4.x, 0.f));
+                cf[j4 + 1] = ex2_approx(fminf(lr - l4.y, 0.f));
+                cf[j4 + 2] = ex2_approx(fminf(lr - l4.z, 0.f));
+                cf[j4 + 3] = ex2_approx(fminf(lr - l4.w, 0.f));
             }
             if (row < 64) {
                 float* A32 = reinterpret_cast<float*>(sm + gdn::OFF_A32);
@@ -1144,11 +1159,13 @@ finish:
 }  // namespace chunk
 
 // Host-side launch (tensor maps are built by the caller).
-cudaError_t launch_chunk_sm100(const CUtensorMap* maps, const void* alpha, const void* b,
+cudaError_t launch_chunk_sm100(const CUtensorMap* maps, const void* q, const void* k, const void* v,
+                               const void* alpha, const void* b,
                                const void* w, int akind, int bkind, int wkind, bool tied,
                                const float* S0, void* o, float* ST, int* d_status, int B, int T,
                                int H, int dv, int group, cudaStream_t st) {
     chunk::Params p;
+    p.q = q; p.k = k; p.v = v;
     p.alpha = alpha; p.bg = b; p.wg = w;
     p.S0 = S0; p.o = (__nv_bfloat16*)o; p.ST = ST; p.d_status = d_status;
     p.B = B; p.T = T; p.H = H; p.dv = dv;

@@ -214,6 +214,7 @@ __global__ void __launch_bounds__(NT, 2) prep_general_kernel(
     {
         float* scan = reinterpret_cast<float*>(sm + G_OFF_SCR);  // [8 rg][128 ch] + [128]
         float lrow0[4];   // channel decay: l at this thread's first token - ref
+        bool out_of_range;  // the chunk's decay span exceeds the factorisation's range
         if (!ACH) {
             if (warp == 0) {
                 const int lane = tid;
@@ -237,10 +238,11 @@ __global__ void __launch_bounds__(NT, 2) prep_general_kernel(
                     scan[0] = ex2_approx(ref);
                     scan[1] = ex2_approx(last);
                     scan[2] = ex2_approx(last - ref);
-                    if (first - last > 230.f) flag_status(pp.d_status, GDR_DEVICE_DECAY_RANGE);
+                    scan[3] = first - last > 230.f ? 1.f : 0.f;
                 }
             }
             __syncthreads();
+            out_of_range = scan[3] != 0.f;
             if (tid < 128) {
                 s_eref[tid] = scan[0];
                 s_gC[tid] = scan[1];
@@ -289,9 +291,10 @@ __global__ void __launch_bounds__(NT, 2) prep_general_kernel(
                     s_fS[ch0 + e] = ex2_approx(tot[e] - ref);
                 }
             }
-            if (bad) flag_status(pp.d_status, GDR_DEVICE_DECAY_RANGE);
-            __syncthreads();  // every channel's eref / fS is needed below
+            // every channel's eref / fS is needed below
+            out_of_range = __syncthreads_or(bad) != 0;
         }
+        if (out_of_range && tid == 0) flag_status(pp.d_status, GDR_DEVICE_DECAY_RANGE);
         GDR_TRACE_G(2);
         float er[4], fs[4];
         {
@@ -301,7 +304,10 @@ __global__ void __launch_bounds__(NT, 2) prep_general_kernel(
             fs[0] = f4.x; fs[1] = f4.y; fs[2] = f4.z; fs[3] = f4.w;
         }
         if (rg == 0) {
-            const float4 g4 = *reinterpret_cast<const float4*>(s_gC + ch0);
+            // a negative g_{n-1} in every channel sends the chunk down the state
+            // pass's exact path (this pass's other outputs for it are then unused)
+            const float4 g4 = out_of_range ? make_float4(-1.f, -1.f, -1.f, -1.f)
+                                           : *reinterpret_cast<const float4*>(s_gC + ch0);
             *reinterpret_cast<float4*>(pp.gc + (((size_t)bb * H + h) * nchunks + ci) * DK + ch0) = g4;
         }
         float rowf_c[4];
@@ -616,26 +622,31 @@ struct StateLayout {
     // inputs are triple-buffered with tied gates (chunk ci + 2 loads while chunk
     // ci runs), double-buffered with independent gates (more inputs per chunk)
     static constexpr int NBUF = UNTIED ? 2 : 3;
-    static constexpr uint32_t WQ = 0;                          // [WN ; QG] bf16 [128 x 128], 32 KB each
-    static constexpr uint32_t K2 = WQ + NBUF * 32768;          // K2 bf16 [64 x 128], 16 KB each
+    static constexpr uint32_t QW = 0;                          // [QG ; WN] bf16 [128 x 128], 32 KB each
+    static constexpr uint32_t K2 = QW + NBUF * 32768;          // K2 bf16 [64 x 128], 16 KB each
     static constexpr uint32_t P = K2 + NBUF * 16384;           // P slice bf16 [64 x 64], 8 KB each
     static constexpr uint32_t AQ = P + NBUF * 8192;            // AQ bf16 [64 x 64], 8 KB each: rows
-                                                               // 64..127 of an M = 128 operand whose
-                                                               // rows 0..63 (the 8 KB before) are unused
+                                                               // 0..63 of an M = 128 operand whose
+                                                               // rows 64..127 (the 8 KB after) are unused
     static constexpr uint32_t KW2 = AQ + NBUF * 8192;          // KW2 bf16 [64 x 128], 16 KB each (untied)
     static constexpr uint32_t BQ = KW2 + (UNTIED ? NBUF * 16384 : 0);  // BQ bf16 [64 x 64] (untied)
     static constexpr uint32_t V = BQ + (UNTIED ? NBUF * 8192 : 0);     // V slice bf16 [64 x 64] (untied)
     static constexpr uint32_t U = V + (UNTIED ? NBUF * 8192 : 0);      // U bf16 [64 x 64]
     static constexpr uint32_t SBF = U + 8192;                          // S bf16 [128 x 64]
-    static constexpr uint32_t SMALL = SBF + 16384;                     // barriers, TMEM slot (1 KB)
+    static constexpr uint32_t EXR = SBF + 16384;                       // exact-path scratch (2.5 KB)
+    static constexpr uint32_t SMALL = EXR + 2560;                      // barriers, TMEM slot (1 KB)
     static constexpr uint32_t BYTES = SMALL + 1024 + 1024;
 };
-// D3 (U, QG S) and D5 (AQ U, BQ V) alternate between two column sets by chunk parity.
+// D3 ([QG S ; U - P]) and D5 (AQ U (+ BQ V), lanes 0..63) alternate between two
+// column sets by chunk parity; D4 = K2^T U (+ KW2^T V).
 constexpr uint32_t GS_TM_D3 = 0, GS_TM_D5 = 128, GS_TM_D4 = 256, GS_TM_COLS = 512;
+constexpr int GS_BAR_U = 2;  // named barrier: U written (warps 2, 3, 6, 7); 1 is the fallback's
 
 struct GStateParams {
     const float* S0;  // state at chunk c_begin (NULL: zero)
-    const float* gc;
+    const float* gc;  // g_{n-1} per chunk and channel; negative: take the exact path
+    ExactArgs ex;     // raw inputs for chunks that take the exact path
+    int group;        // value heads per q/k head
     __nv_bfloat16* o;
     float* ST;        // state after chunk c_end - 1 (NULL: not written); may alias S0
     int* d_status;
@@ -643,6 +654,19 @@ struct GStateParams {
     int c_begin, c_end;  // chunk range of this launch
 };
 
+__device__ __forceinline__ void gs_named_bar_sync(int id, int n) {
+    asm volatile("bar.sync %0, %1;" ::"r"(id), "r"(n) : "memory");
+}
+
+// Chunk step. The chain from one chunk to the next holds only the products
+// that depend on the state:
+//   D3 = [QG ; WN] S          (U = P + WN S in lanes 64..127, by warps 2, 3, 6, 7)
+//   D4 (+)= K2^T U            (S <- Diag(g_{n-1}) S + D4, all warps)
+// and beside it, on the same issuing thread (thread 64) so products into one
+// accumulator keep their order: untied D4 = KW2^T V and D5 = [BQ ; .] V
+// (queued after D3, before U exists), and D5 (+)= [AQ ; .] U after D4's
+// product; O = QG S + AQ U (+ BQ V), lanes 0..63, is written by warps 0, 1,
+// 4, 5 during the next chunk's first product.
 template <bool UNTIED>
 __global__ void __launch_bounds__(NT, 1) state_general_kernel(
     const __grid_constant__ CUtensorMap tm_wn, const __grid_constant__ CUtensorMap tm_qg,
@@ -655,20 +679,26 @@ __global__ void __launch_bounds__(NT, 1) state_general_kernel(
     uint8_t* sm = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) &
                                              ~uintptr_t(1023));
     const int tid = threadIdx.x, warp = tid >> 5, wg = warp >> 2, row = tid & 127;
+    const bool lo = row < 64;
     const int vt = blockIdx.x, h = blockIdx.y, bb = blockIdx.z;
     const int v0 = vt * NV;
     const int T = p.T, H = p.H;
     const int nchunks = (T + C - 1) / C;
+    constexpr int ISSUER = 64;  // thread that issues every MMA (warp 2)
 
     constexpr int NBUF = Lay::NBUF;
-    uint64_t* bar_tma = reinterpret_cast<uint64_t*>(sm + Lay::SMALL);  // [NBUF]
-    uint64_t* bar_mma = bar_tma + 3;
-    uint32_t* s_tmem = reinterpret_cast<uint32_t*>(sm + Lay::SMALL + 32);
+    uint64_t* bar_tma = reinterpret_cast<uint64_t*>(sm + Lay::SMALL);  // [3]
+    uint64_t* bar_w = bar_tma + 3;
+    uint64_t* bar_k = bar_tma + 4;
+    uint64_t* bar_a = bar_tma + 5;
+    uint64_t* bar_drain = bar_tma + 6;
+    uint32_t* s_tmem = reinterpret_cast<uint32_t*>(sm + Lay::SMALL + 64);
     if (tid == 0) {
-        mbar_init(&bar_tma[0], 1);
-        mbar_init(&bar_tma[1], 1);
-        mbar_init(&bar_tma[2], 1);
-        mbar_init(bar_mma, 1);
+        for (int i = 0; i < 3; ++i) mbar_init(&bar_tma[i], 1);
+        mbar_init(bar_w, 1);
+        mbar_init(bar_k, 1);
+        mbar_init(bar_a, 1);
+        mbar_init(bar_drain, 1);
         fence_barrier_init();
     }
     if (warp == 0) tmem_alloc(s_tmem, GS_TM_COLS);
@@ -677,19 +707,22 @@ __global__ void __launch_bounds__(NT, 1) state_general_kernel(
     tc_fence_after();
     const uint32_t tmem = *s_tmem;
     const uint32_t lane_base = (uint32_t)((warp & 3) * 32) << 16;
-    uint32_t ph_tma0 = 0u, ph_tma1 = 0u, ph_tma2 = 0u, ph_mma = 0;
+    uint32_t ph_tma = 0u;  // bit i: phase parity of stage i
     bool ok = true;
     const uint32_t sbase = smem_u32(sm);
+    const int c_begin = p.c_begin, c_end = p.c_end;
+    int loads_issued = c_begin;  // chunks [c_begin, loads_issued) have been requested
 
     auto issue_loads = [&](int ci) {
         const int t0 = ci * C, buf = ci % NBUF;
         uint64_t* bar = &bar_tma[buf];
-        uint8_t* wq = sm + Lay::WQ + buf * 32768;
+        uint8_t* qw = sm + Lay::QW + buf * 32768;
         mbar_expect_tx(bar, (UNTIED ? 12u : 8u) * 8192u);
-        tma_load_4d(wq, &tm_wn, bar, 0, h, t0, bb);
-        tma_load_4d(wq + 16384, &tm_wn, bar, 64, h, t0, bb);
-        tma_load_4d(wq + 8192, &tm_qg, bar, 0, h, t0, bb);
-        tma_load_4d(wq + 16384 + 8192, &tm_qg, bar, 64, h, t0, bb);
+        // [QG ; WN]: each 64-column block holds 128 rows (QG rows 0..63, WN rows 64..127)
+        tma_load_4d(qw, &tm_qg, bar, 0, h, t0, bb);
+        tma_load_4d(qw + 16384, &tm_qg, bar, 64, h, t0, bb);
+        tma_load_4d(qw + 8192, &tm_wn, bar, 0, h, t0, bb);
+        tma_load_4d(qw + 16384 + 8192, &tm_wn, bar, 64, h, t0, bb);
         tma_load_4d(sm + Lay::K2 + buf * 16384, &tm_k2, bar, 0, h, t0, bb);
         tma_load_4d(sm + Lay::K2 + buf * 16384 + 8192, &tm_k2, bar, 64, h, t0, bb);
         tma_load_4d(sm + Lay::AQ + buf * 8192, &tm_aq, bar, 0, h, t0, bb);
@@ -718,17 +751,15 @@ __global__ void __launch_bounds__(NT, 1) state_general_kernel(
     fence_proxy_async();
     tc_fence_before();
     __syncthreads();
-    const int c_begin = p.c_begin, c_end = p.c_end;
     const float* gcp = p.gc + ((size_t)bb * H + h) * nchunks * DK + row;
     float gC_next = c_begin < c_end ? gcp[(size_t)c_begin * DK] : 0.f;
-    if (tid == 0) {
-        if (c_begin < c_end) issue_loads(c_begin);
-        if (NBUF == 3 && c_begin + 1 < c_end) issue_loads(c_begin + 1);
+    if (tid == 32) {
+        for (int ci = c_begin; ci < c_end && ci < c_begin + NBUF - 1; ++ci) issue_loads(ci);
     }
+    loads_issued = min(c_end, c_begin + NBUF - 1);
 
-    auto store_o = [&](int cj) {
-        const int pj = cj & 1;
-        const int t = cj * C + row - 64;
+    auto store_o = [&](int cj, int pj) {
+        const int t = cj * C + row;
         float d[32], d5[32];
         tmem_ld32_async(tmem + lane_base + GS_TM_D3 + pj * 64 + wg * 32, d);
         tmem_ld32_async(tmem + lane_base + GS_TM_D5 + pj * 64 + wg * 32, d5);
@@ -740,58 +771,55 @@ __global__ void __launch_bounds__(NT, 1) state_general_kernel(
         }
     };
 
-#define GDR_WAIT(bar, ph)                                                   \
-    do {                                                                    \
-        bool w_ok = mbar_wait(bar, ph);                                     \
-        ph ^= 1u;                                                           \
-        if (!__syncthreads_and(w_ok)) { ok = false; goto finish; }          \
-    } while (0)
-#define GDR_BEFORE_MMA()    \
-    do {                    \
-        fence_proxy_async(); \
-        tc_fence_before();  \
-        __syncthreads();    \
-    } while (0)
     // Waits inside the chunk loop are per thread; a timed-out wait is carried in
-    // w_ok to the next block barrier, where the block leaves together.
+    // w_ok to the block barrier that ends the chunk, where the block leaves together.
     bool w_ok = true;
 #define GDR_WAIT_SOLO(bar, ph)              \
     do {                                    \
         w_ok = mbar_wait(bar, ph) && w_ok;  \
-        ph ^= 1u;                           \
     } while (0)
 #define GDR_SYNC_CHECK()                                            \
     do {                                                            \
         if (!__syncthreads_and(w_ok)) { ok = false; goto finish; }  \
     } while (0)
 
+    // nm counts the chunks taken on the tensor cores: their barriers' phases
+    // and TMEM column sets follow it. A chunk whose g_{n-1} is marked negative
+    // by the first pass (decay span outside the factorisation's range) is
+    // applied token by token instead, from the raw inputs.
+    int nm = 0;
+    int pend = -1;  // chunk whose O still sits in TMEM (column set pend_set), or -1
+    int pend_set = 0;
+    uint32_t pend_ph = 0;
     for (int ci = c_begin; ci < c_end; ++ci) {
-        const int buf = ci % NBUF, par = ci & 1;
-        const uint32_t wqb = sbase + Lay::WQ + buf * 32768u;
+        const int buf = ci % NBUF, par = nm & 1;
+        const uint32_t ph = (uint32_t)(nm & 1);
+        const uint32_t qwb = sbase + Lay::QW + buf * 32768u;
         const uint32_t k2b = sbase + Lay::K2 + buf * 16384u;
-        const uint32_t aqa = sbase + Lay::AQ + buf * 8192u - 8192u;  // AQ = rows 64..127
+        const uint32_t aqa = sbase + Lay::AQ + buf * 8192u;  // AQ = rows 0..63
         const uint32_t ub = sbase + Lay::U;
         const uint32_t d3 = GS_TM_D3 + (uint32_t)par * 64u, d5 = GS_TM_D5 + (uint32_t)par * 64u;
         const float gC = gC_next;
         if (ci + 1 < c_end) gC_next = gcp[(size_t)(ci + 1) * DK];
-        if (buf == 0) GDR_WAIT_SOLO(&bar_tma[0], ph_tma0);
-        else if (buf == 1) GDR_WAIT_SOLO(&bar_tma[1], ph_tma1);
-        else GDR_WAIT_SOLO(&bar_tma[2], ph_tma2);
+        const bool exact = gC < 0.f;  // the same mark in every channel: uniform
+        GDR_WAIT_SOLO(&bar_tma[buf], (ph_tma >> buf) & 1u);
+        ph_tma ^= 1u << buf;
 
-        // ---- batch 1: D3 = [WN ; QG] S;  untied: D4 = KW2^T V, D5 = [. ; BQ] V --------
-        if (tid == 0) {
+        // ---- D3 = [QG ; WN] S;  untied: D4 = KW2^T V, D5 = [BQ ; .] V --------------------
+        if (tid == ISSUER && !exact) {
             tc_fence_after();
             const uint32_t idS = idesc_bf16(128, NV, 0, 1);
-            const uint32_t idM = idesc_bf16(128, NV, 1, 1);
 #pragma unroll
             for (int ks = 0; ks < 8; ++ks) {
                 const uint32_t koff = (ks >> 2) * 16384u + (ks & 3) * 32u;
-                mma_bf16(tmem + d3, sdesc_sw128(wqb + koff, 16, 1024),
+                mma_bf16(tmem + d3, sdesc_sw128(qwb + koff, 16, 1024),
                          sdesc_sw128(sbase + Lay::SBF + ks * 2048u, 8192, 1024), idS, ks > 0);
             }
+            mma_commit(bar_w);
             if (UNTIED) {
+                const uint32_t idM = idesc_bf16(128, NV, 1, 1);
                 const uint32_t vb = sbase + Lay::V + buf * 8192u;
-                const uint32_t bqa = sbase + Lay::BQ + buf * 8192u - 8192u;  // BQ = rows 64..127
+                const uint32_t bqa = sbase + Lay::BQ + buf * 8192u;  // BQ = rows 0..63
 #pragma unroll
                 for (int ks = 0; ks < 4; ++ks) {
                     mma_bf16(tmem + GS_TM_D4, sdesc_sw128(sbase + Lay::KW2 + buf * 16384u + ks * 2048u, 8192, 1024),
@@ -800,78 +828,110 @@ __global__ void __launch_bounds__(NT, 1) state_general_kernel(
                              sdesc_sw128(vb + ks * 2048u, 8192, 1024), idS, ks > 0);
                 }
             }
-            mma_commit(bar_mma);
         }
-        // chunk ci + NBUF - 1's inputs go to the buffers chunk ci - 1 has released
-        if (tid == 32 && ci + NBUF - 1 < c_end) issue_loads(ci + NBUF - 1);
-        // the previous chunk's outputs, while batch 1 runs
-        if (row >= 64 && ci > c_begin) store_o(ci - 1);
-        GDR_WAIT_SOLO(bar_mma, ph_mma);
-        tc_fence_after();
-
-        // ---- U = P + WN S (rows 0..63) -> rows 0..63 of [U ; AQ] ------------------------
-        if (row < 64) {
-            float d[32];
-            tmem_ld32(tmem + lane_base + d3 + wg * 32, d);
-#pragma unroll
-            for (int c8 = 0; c8 < 4; ++c8) {
-                float x[8];
-                ld_chunk(sm + Lay::P + buf * 8192, sw128_chunk(row, wg * 4 + c8, 64), x);
-#pragma unroll
-                for (int e = 0; e < 8; ++e) x[e] += d[c8 * 8 + e];
-                st_chunk(sm + Lay::U, sw128_chunk(row, wg * 4 + c8, 64), x);
-            }
-        }
-        fence_proxy_async();
-        tc_fence_before();
-        GDR_SYNC_CHECK();
-
-        // ---- batch 2: D5 (+)= [U ; AQ] U (rows 64..127: AQ U);  D4 (+)= K2^T U ----------
-        if (tid == 0) {
+        // the previous chunk's outputs (lanes 0..63), while the first product runs
+        if (lo && pend >= 0) {
+            GDR_WAIT_SOLO(bar_a, pend_ph);
             tc_fence_after();
-            const uint32_t idK = idesc_bf16(128, NV, 0, 1);
-            const uint32_t idM = idesc_bf16(128, NV, 1, 1);
+            store_o(pend, pend_set);
+        }
+        pend = -1;
+        // chunk ci + NBUF - 1's inputs go to the buffers of chunk ci - 1, whose last
+        // reader (its AQ U product) the wait above has seen complete (thread 32 is
+        // one of the waiting warps)
+        if (tid == 32 && ci + NBUF - 1 < c_end) issue_loads(ci + NBUF - 1);
+        if (ci + NBUF - 1 < c_end) loads_issued = ci + NBUF;
+        if (exact) {
+            exact_tokens(p.ex, S, reinterpret_cast<float*>(sm + Lay::EXR), bb, h, h / p.group, v0,
+                         ci * C, min(C, T - ci * C), tid);
+        } else {
+            if (!lo) {
+                // ---- U = P + WN S (lanes 64..127 of D3) -> U -------------------------------
+                GDR_WAIT_SOLO(bar_w, ph);
+                tc_fence_after();
+                {
+                    const int j = row - 64;
+                    float d[32];
+                    tmem_ld32(tmem + lane_base + d3 + wg * 32, d);
 #pragma unroll
-            for (int ks = 0; ks < 4; ++ks) {
-                const uint32_t acc = UNTIED ? 1u : (uint32_t)(ks > 0);
-                mma_bf16(tmem + d5, sdesc_sw128(aqa + ks * 32u, 16, 1024),
-                         sdesc_sw128(ub + ks * 2048u, 8192, 1024), idK, acc);
-                mma_bf16(tmem + GS_TM_D4, sdesc_sw128(k2b + ks * 2048u, 8192, 1024),
-                         sdesc_sw128(ub + ks * 2048u, 8192, 1024), idM, acc);
+                    for (int c8 = 0; c8 < 4; ++c8) {
+                        float x[8];
+                        const uint32_t off = sw128_chunk(j, wg * 4 + c8, 64);
+                        ld_chunk(sm + Lay::P + buf * 8192, off, x);
+#pragma unroll
+                        for (int e = 0; e < 8; ++e) x[e] += d[c8 * 8 + e];
+                        st_chunk(sm + Lay::U, off, x);
+                    }
+                }
+                fence_proxy_async();
+                tc_fence_before();
+                gs_named_bar_sync(GS_BAR_U, 128);
+                if (tid == ISSUER) {
+                    // ---- D4 (+)= K2^T U, then D5 (+)= [AQ ; .] U ------------------------------
+                    tc_fence_after();
+                    const uint32_t idK = idesc_bf16(128, NV, 0, 1);
+                    const uint32_t idM = idesc_bf16(128, NV, 1, 1);
+#pragma unroll
+                    for (int ks = 0; ks < 4; ++ks)
+                        mma_bf16(tmem + GS_TM_D4, sdesc_sw128(k2b + ks * 2048u, 8192, 1024),
+                                 sdesc_sw128(ub + ks * 2048u, 8192, 1024), idM, UNTIED ? 1u : (uint32_t)(ks > 0));
+                    mma_commit(bar_k);
+#pragma unroll
+                    for (int ks = 0; ks < 4; ++ks)
+                        mma_bf16(tmem + d5, sdesc_sw128(aqa + ks * 32u, 16, 1024),
+                                 sdesc_sw128(ub + ks * 2048u, 8192, 1024), idK, UNTIED ? 1u : (uint32_t)(ks > 0));
+                    mma_commit(bar_a);
+                }
             }
-            mma_commit(bar_mma);
-        }
-        GDR_WAIT_SOLO(bar_mma, ph_mma);
-        tc_fence_after();
-
-        // ---- S = Diag(GC) S + D4 ---------------------------------------------------------
-        {
-            float dS[32];
-            tmem_ld32(tmem + lane_base + GS_TM_D4 + wg * 32, dS);
+            // ---- S = Diag(GC) S + D4 -----------------------------------------------------
+            GDR_WAIT_SOLO(bar_k, ph);
+            tc_fence_after();
+            {
+                float dS[32];
+                tmem_ld32(tmem + lane_base + GS_TM_D4 + wg * 32, dS);
 #pragma unroll
-            for (int j = 0; j < NH; ++j) S[j] = fmaf(gC, S[j], dS[j]);
-#pragma unroll
-            for (int ch = 0; ch < 4; ++ch) st_chunk(sm + Lay::SBF, sw128_chunk(row, wg * 4 + ch, DK), &S[8 * ch]);
+                for (int j = 0; j < NH; ++j) S[j] = fmaf(gC, S[j], dS[j]);
+            }
+            pend = ci;
+            pend_set = par;
+            pend_ph = ph;
+            ++nm;
         }
+#pragma unroll
+        for (int ch = 0; ch < 4; ++ch) st_chunk(sm + Lay::SBF, sw128_chunk(row, wg * 4 + ch, DK), &S[8 * ch]);
         fence_proxy_async();  // the state copy feeds the next chunk's MMAs
         tc_fence_before();
         GDR_SYNC_CHECK();
     }
-    if (row >= 64 && c_begin < c_end) store_o(c_end - 1);
+    if (lo && pend >= 0) {
+        GDR_WAIT_SOLO(bar_a, pend_ph);
+        tc_fence_after();
+        store_o(pend, pend_set);
+    }
+    if (!__syncthreads_and(w_ok)) ok = false;
 
-    if (p.ST) {
+    if (ok && p.ST) {
         float* st = p.ST + (((size_t)bb * H + h) * DK + row) * p.dv + v0 + wg * NH;
 #pragma unroll
         for (int j = 0; j < NH; j += 4) *reinterpret_cast<float4*>(st + j) = make_float4(S[j], S[j + 1], S[j + 2], S[j + 3]);
     }
 
 finish:
-    if (!ok && tid == 0) flag_status(p.d_status, GDR_DEVICE_TIMEOUT);
+    if (!ok) {
+        if (tid == 0) flag_status(p.d_status, GDR_DEVICE_TIMEOUT);
+        // before the block leaves (each wait bounded): the input copies it
+        // requested have landed and the issued MMAs are done
+        if (tid == 32)
+            for (int ci = max(c_begin, loads_issued - NBUF); ci < loads_issued; ++ci)
+                (void)mbar_wait(&bar_tma[ci % NBUF], (uint32_t)(((ci - c_begin) / NBUF) & 1));
+        if (tid == ISSUER) {
+            mma_commit(bar_drain);
+            (void)mbar_wait(bar_drain, 0);
+        }
+    }
     tc_fence_before();
     __syncthreads();
     if (warp == 0) tmem_dealloc(tmem, GS_TM_COLS);
-#undef GDR_WAIT
-#undef GDR_BEFORE_MMA
 #undef GDR_WAIT_SOLO
 #undef GDR_SYNC_CHECK
 }
@@ -950,7 +1010,7 @@ static AuxResources* aux_resources(int dev) {
 
 // maps: q, k, v (of the call). alpha/b/w kinds as in the C ABI.
 cudaError_t launch_chunk_twopass_general(const CUtensorMap* maps, MapFn make_map, void* ws,
-                                         const void* q, const void* k, const void* alpha,
+                                         const void* q, const void* k, const void* v, const void* alpha,
                                          const void* b, const void* w, int akind, int bkind,
                                          int wkind, const float* S0, void* o, float* ST,
                                          int* d_status, int B, int T, int H, int dv, int group,
@@ -1002,6 +1062,11 @@ cudaError_t launch_chunk_twopass_general(const CUtensorMap* maps, MapFn make_map
     };
     GStateParams sp;
     sp.gc = pp.gc; sp.o = reinterpret_cast<__nv_bfloat16*>(o);
+    sp.ex.q = pp.q; sp.ex.k = pp.k; sp.ex.v = reinterpret_cast<const __nv_bfloat16*>(v);
+    sp.ex.alpha = pp.alpha; sp.ex.b = pp.bg; sp.ex.w = pp.wg;
+    sp.ex.akind = akind; sp.ex.bkind = bkind; sp.ex.wkind = wkind;
+    sp.ex.o = sp.o; sp.ex.T = T; sp.ex.H = H; sp.ex.Hq = H / group; sp.ex.dv = dv;
+    sp.group = group;
     sp.d_status = d_status; sp.T = T; sp.H = H; sp.dv = dv;
     const dim3 sgrid(dv / NV, H, B);
     auto state_range = [&](int c0, int c1, const float* s_in, float* s_out) -> cudaError_t {

@@ -7,19 +7,20 @@
 // Write, Erase, Decay, Read" section 03 for the chunk reassociation). So the
 // forward runs in two passes:
 //
-//   pass 1 (prep, one CTA per chunk, all chunks of all heads in parallel):
-//     A  = Diag(beta rowf) (K K^T) Diag(colf)       strict lower
+//   pass 1 (prep, persistent CTAs over all chunks of all heads):
+//     A  = Diag(beta) ((K K^T) . G) strict lower, G_rj = g_r / g_j
 //     T  = (I + A)^-1
 //     -W = -T Diag(beta g) K                        -> workspace [B,T,H,128] bf16
 //     P  =  T Diag(beta) V                          -> workspace [B,T,H,d_v] bf16
 //   pass 2 (state, one CTA per (batch, head, 64 columns of d_v), chunks in order):
-//     U  = P - W S                                  (MMA [-W ; Q] S, plus P)
-//     Aq = Diag(rowf) (Q K^T) Diag(colf)            lower   (same MMA batch)
+//     U  = P - W S                                  (MMA [Q ; -W] S, plus P)
+//     Aq = (Q K^T) . G                              lower, incl. the diagonal
 //     O  = Diag(g) (Q S) + Aq U
 //     S' = g_{n-1} S + (Diag(g_{n-1}/g) K)^T U
-// with l_r the prefix sum of log2 alpha over the chunk, g_r = 2^l_r, and the
-// bounded factors rowf_r = 2^(l_r - ref), colf_r = 2^(ref - l_r) around the
-// chunk's reference ref = (l_0 + l_{n-1}) / 2.
+// with l_r the prefix sum of log2 alpha over the chunk and g_r = 2^l_r. The
+// scalar decay factors out of every product, so each ratio g_r / g_j =
+// 2^(l_r - l_j) (r >= j) is formed per element on the accumulator unload:
+// every factor is at most 1 and no alpha in (0, 1] leaves the range.
 //
 // Pass 2's per-chunk chain is two MMA round trips; the triangular solve and
 // the W / P products (most of the single-pass kernel's chain) run in pass 1
@@ -42,9 +43,9 @@ __device__ unsigned long long g_trace2[64 * 16];
         if (blockIdx.x == 0 && threadIdx.x == 0 && it < 64)                               \
             g_trace2[it * 16 + (k)] = clock64();                                          \
     } while (0)
-#define GDR_TRACE_S(k)                                                                     \
+#define GDR_TRACE_S(k, thr)                                                                \
     do {                                                                                  \
-        if (blockIdx.x == 0 && blockIdx.y == 0 && blockIdx.z == 0 && threadIdx.x == 0 &&  \
+        if (blockIdx.x == 0 && blockIdx.y == 0 && blockIdx.z == 0 && threadIdx.x == (thr) && \
             ci < 64)                                                                      \
             g_trace2[ci * 16 + 8 + (k)] = clock64();                                      \
     } while (0)
@@ -52,8 +53,8 @@ __device__ unsigned long long g_trace2[64 * 16];
 #define GDR_TRACE_P(k) \
     do {              \
     } while (0)
-#define GDR_TRACE_S(k) \
-    do {              \
+#define GDR_TRACE_S(k, thr) \
+    do {                   \
     } while (0)
 #endif
 
@@ -94,8 +95,7 @@ __global__ void __launch_bounds__(NT, 2) prep_gdn_kernel(const __grid_constant__
     const int nvt = dv / 64;
 
     float* s_beta = reinterpret_cast<float*>(sm + P_OFF_SMALL);
-    float* s_rowf = s_beta + 64;
-    float* s_colf = s_beta + 128;
+    float* s_l = s_beta + 64;   // log2 prefix of alpha over the chunk
     float* s_g = s_beta + 192;
     float* s_alpha = s_beta + 256;
     uint64_t* bar_tma = reinterpret_cast<uint64_t*>(sm + P_OFF_SMALL + 1280);  // [2]
@@ -197,16 +197,10 @@ __global__ void __launch_bounds__(NT, 2) prep_gdn_kernel(const __grid_constant__
                 if (lane >= off) x += y;
             }
             const float l1 = x, l0v = x - la1;
-            const float first = __shfl_sync(0xffffffffu, l0v, 0);
-            const float last = __shfl_sync(0xffffffffu, l1, 31);
-            const float ref = 0.5f * (first + last);
-            s_rowf[2 * lane] = ex2_approx(l0v - ref);
-            s_rowf[2 * lane + 1] = ex2_approx(l1 - ref);
-            s_colf[2 * lane] = ex2_approx(ref - l0v);
-            s_colf[2 * lane + 1] = ex2_approx(ref - l1);
+            s_l[2 * lane] = l0v;
+            s_l[2 * lane + 1] = l1;
             s_g[2 * lane] = ex2_approx(l0v);
             s_g[2 * lane + 1] = ex2_approx(l1);
-            if (lane == 0 && first - last > 230.f) flag_status(pp.d_status, GDR_DEVICE_DECAY_RANGE);
         }
         if (buf == 0) GDR_WAIT(&bar_tma[0], ph_tma0);  // also publishes the scan
         else GDR_WAIT(&bar_tma[1], ph_tma1);
@@ -235,17 +229,18 @@ __global__ void __launch_bounds__(NT, 2) prep_gdn_kernel(const __grid_constant__
             const int r = row;  // 0..63
             float d[32];
             tmem_ld32(tmem + lane_base + P_TM_D1 + wg * 32, d);
-            const float rf = s_rowf[r] * s_beta[r];
+            // A_rj = beta_r (k_r . k_j) 2^(l_r - l_j), j < r: every ratio at most 1
+            const float rf = s_beta[r], lr = s_l[r];
             float* A32 = reinterpret_cast<float*>(sm + P_OFF_A32);
 #pragma unroll
             for (int j4 = 0; j4 < 32; j4 += 4) {
                 const int j = wg * 32 + j4;
-                const float4 c4v = *reinterpret_cast<const float4*>(s_colf + j);
+                const float4 l4 = *reinterpret_cast<const float4*>(s_l + j);
                 float4 x;
-                x.x = j < r ? rf * c4v.x * d[j4] : 0.f;
-                x.y = j + 1 < r ? rf * c4v.y * d[j4 + 1] : 0.f;
-                x.z = j + 2 < r ? rf * c4v.z * d[j4 + 2] : 0.f;
-                x.w = j + 3 < r ? rf * c4v.w * d[j4 + 3] : 0.f;
+                x.x = j < r ? rf * ex2_approx(fminf(lr - l4.x, 0.f)) * d[j4] : 0.f;
+                x.y = j + 1 < r ? rf * ex2_approx(fminf(lr - l4.y, 0.f)) * d[j4 + 1] : 0.f;
+                x.z = j + 2 < r ? rf * ex2_approx(fminf(lr - l4.z, 0.f)) * d[j4 + 2] : 0.f;
+                x.w = j + 3 < r ? rf * ex2_approx(fminf(lr - l4.w, 0.f)) * d[j4 + 3] : 0.f;
                 d[j4] = x.x; d[j4 + 1] = x.y; d[j4 + 2] = x.z; d[j4 + 3] = x.w;
                 *reinterpret_cast<float4*>(f32_at(A32, r, j)) = x;
             }
@@ -363,21 +358,48 @@ finish:
 }
 
 // ---- pass 2 shared memory ---------------------------------------------------
-// Inputs are triple-buffered (chunk ci + 2 loads while chunk ci runs).
+// Inputs are triple-buffered (chunk ci + 2 loads while chunk ci runs); a stage
+// holds [Q ; -W] (Q in rows 0..63, -W in rows 64..127, two 64-column blocks
+// of 16 KB), K and this CTA's 64 columns of P.
 constexpr int S_NBUF = 3;
-constexpr uint32_t S_OFF_WQ = 0;        // [-W ; Q] bf16 [128 x 128], 32 KB per buffer
-constexpr uint32_t S_OFF_K = 98304;     // K bf16 [64 x 128], 16 KB per buffer (B operand of Q K^T)
-constexpr uint32_t S_OFF_P = 147456;    // P slice bf16 [64 x 64], 8 KB per buffer
-constexpr uint32_t S_OFF_K2 = 172032;   // K scaled by g_{n-1}/g per token, bf16 [64 x 128]
-constexpr uint32_t S_OFF_AQU = 188416;  // [U ; Aq] bf16 [128 x 64]: U (rows 0..63) is also the
-                                        // B operand; Aq U lands in rows 64..127 of the product
-constexpr uint32_t S_OFF_SBF = 204800;  // S bf16 [128 x 64]
-constexpr uint32_t S_OFF_SMALL = 221184;
+constexpr uint32_t S_STAGE = 57344;
+constexpr uint32_t S_ST_QW = 0;         // [Q ; -W] bf16 [128 x 128]
+constexpr uint32_t S_ST_K = 32768;      // K bf16 [64 x 128]
+constexpr uint32_t S_ST_P = 49152;      // P slice bf16 [64 x 64]
+constexpr uint32_t S_OFF_SBF = S_NBUF * S_STAGE;     // S bf16 [128 x 64] (B operand, MN-major)
+constexpr uint32_t S_OFF_AQ = S_OFF_SBF + 16384;     // Aq bf16 [64 x 64] (rows 0..63 of the
+                                                     // Aq U A operand; U below are its rows 64..127)
+constexpr uint32_t S_OFF_U = S_OFF_AQ + 8192;        // U bf16 [64 x 64] (B operand of Aq U)
+constexpr uint32_t S_OFF_U2 = S_OFF_U + 8192;        // Diag(g_{n-1}/g) U (B operand of K^T U)
+constexpr uint32_t S_OFF_SMALL = S_OFF_U2 + 8192;
 constexpr uint32_t S_SMEM_BYTES = S_OFF_SMALL + 3072 + 1024;
-// D3 (U and Q S) and D5 (Aq U) alternate between two column sets by chunk
-// parity, so chunk ci's outputs are written while chunk ci + 1's first batch runs.
-constexpr uint32_t S_TM_D1 = 0, S_TM_D3 = 64, S_TM_D4 = 192, S_TM_D5 = 256, S_TM_COLS = 512;
+// TMEM columns: D3 [Q S ; -W S] and D5 (Aq U, lanes 0..63) alternate between
+// two column sets by chunk parity, so chunk ci's outputs are written while
+// chunk ci + 1 runs; D1 = [Q ; -W] K^T (lanes 0..63: Q K^T); D4 = K^T U'.
+constexpr uint32_t S_TM_D3 = 0, S_TM_D1 = 128, S_TM_D4 = 192, S_TM_D5 = 256, S_TM_COLS = 512;
+// Named barriers (0 is __syncthreads): U ready for K^T U (warps 2, 3, 6, 7);
+// U and Aq ready for Aq U (warps 2, 3, 6, 7 arrive, warps 0, 1, 4, 5 wait).
+constexpr int S_BAR_U = 1, S_BAR_AQ = 2;
 
+__device__ __forceinline__ void named_bar_sync(int id, int n) {
+    asm volatile("bar.sync %0, %1;" ::"r"(id), "r"(n) : "memory");
+}
+__device__ __forceinline__ void named_bar_arrive(int id, int n) {
+    asm volatile("bar.arrive %0, %1;" ::"r"(id), "r"(n) : "memory");
+}
+
+// Chunk step of the state pass. Only the two products that depend on the
+// state are on the chain from one chunk to the next:
+//   D3 = [Q ; -W] S           (then U = P - W S, rows 64..127 of D3, by warps 2, 3, 6, 7)
+//   D4 = K^T Diag(g_{n-1}/g) U  (then S <- g_{n-1} S + D4, all warps)
+// The output's products run beside them on their own barriers:
+//   D1 = [Q ; -W] K^T          (queued right after D3; Aq = masked
+//                               (Q K^T) . 2^(l_r - l_j) by warps 0, 1, 4, 5
+//                               while warps 2, 3, 6, 7 form U)
+//   D5 = [Aq ; .] U            (queued after D4; read with Q S for O of this
+//                               chunk during the next chunk's first product)
+// Decay ratios are formed per element from the log2 prefix l (exact for any
+// alpha in (0, 1]: every factor used is at most 1).
 __global__ void __launch_bounds__(NT, 1) state_gdn_kernel(
     const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ CUtensorMap tm_k,
     const __grid_constant__ CUtensorMap tm_w, const __grid_constant__ CUtensorMap tm_p,
@@ -387,28 +409,35 @@ __global__ void __launch_bounds__(NT, 1) state_gdn_kernel(
                                              ~uintptr_t(1023));
     const int tid = threadIdx.x, warp = tid >> 5;
     const int wg = warp >> 2;
-    const int row = tid & 127;
+    const int row = tid & 127;             // TMEM lane / state row
+    const bool lo = row < 64;              // warps 0, 1, 4, 5: lanes 0..63
     const int vt = blockIdx.x, h = blockIdx.y, bb = blockIdx.z;
     const int hq = h / p.group;  // q / k head of this value head
     const int v0 = vt * NV;
     const int T = p.T, H = p.H;
     const int nchunks = (T + C - 1) / C;
 
-    // per-token factors, double-buffered by chunk parity: [2][64] each
-    float* s_rowf2 = reinterpret_cast<float*>(sm + S_OFF_SMALL);
-    float* s_colf2 = s_rowf2 + 128;
-    float* s_g2 = s_rowf2 + 256;
-    float* s_gcr2 = s_rowf2 + 384;
-    float* s_misc2 = s_rowf2 + 512;   // [2][4]: g_{n-1}
-    float* s_alpha = s_rowf2 + 520;   // [64] staging of the next chunk's decays
-    uint64_t* bar_tma = reinterpret_cast<uint64_t*>(sm + S_OFF_SMALL + 2880);  // [3]
-    uint64_t* bar_mma = bar_tma + 3;
-    uint32_t* s_tmem = reinterpret_cast<uint32_t*>(sm + S_OFF_SMALL + 2912);
+    // per-chunk factors, three sets by chunk % 3 (written one chunk ahead,
+    // read up to one chunk behind): l (log2 prefix), g = 2^l,
+    // gcr = 2^(l_{n-1} - l), and g_{n-1}
+    float* s_l3 = reinterpret_cast<float*>(sm + S_OFF_SMALL);   // [3][64]
+    float* s_g3 = s_l3 + 192;                                    // [3][64]
+    float* s_gcr3 = s_l3 + 384;                                  // [3][64]
+    float* s_gC3 = s_l3 + 576;                                   // [3][4]
+    uint64_t* bar_tma = reinterpret_cast<uint64_t*>(sm + S_OFF_SMALL + 2816);  // [3]
+    uint64_t* bar_w = bar_tma + 3;
+    uint64_t* bar_q = bar_tma + 4;
+    uint64_t* bar_k = bar_tma + 5;
+    uint64_t* bar_a = bar_tma + 6;
+    uint64_t* bar_drain = bar_tma + 7;  // timeout path: both MMA issuers' work has finished
+    uint32_t* s_tmem = reinterpret_cast<uint32_t*>(sm + S_OFF_SMALL + 2880);
     if (tid == 0) {
-        mbar_init(&bar_tma[0], 1);
-        mbar_init(&bar_tma[1], 1);
-        mbar_init(&bar_tma[2], 1);
-        mbar_init(bar_mma, 1);
+        for (int i = 0; i < 3; ++i) mbar_init(&bar_tma[i], 1);
+        mbar_init(bar_w, 1);
+        mbar_init(bar_q, 1);
+        mbar_init(bar_k, 1);
+        mbar_init(bar_a, 1);
+        mbar_init(bar_drain, 2);
         fence_barrier_init();
         prefetch_tmap(&tm_q);
         prefetch_tmap(&tm_k);
@@ -421,23 +450,22 @@ __global__ void __launch_bounds__(NT, 1) state_gdn_kernel(
     tc_fence_after();
     const uint32_t tmem = *s_tmem;
     const uint32_t lane_base = (uint32_t)((warp & 3) * 32) << 16;
-    uint32_t ph_tma0 = 0u, ph_tma1 = 0u, ph_tma2 = 0u, ph_mma = 0;
-    bool ok = true;
     const uint32_t sbase = smem_u32(sm);
+    bool ok = true;
+    int loads_issued = 0;  // chunks whose inputs were requested (tid 0 / 32 bookkeeping)
 
     auto issue_loads = [&](int ci) {
         const int t0 = ci * C, buf = ci % S_NBUF;
-        uint8_t* wq = sm + S_OFF_WQ + buf * 32768;
-        uint8_t* kk = sm + S_OFF_K + buf * 16384;
+        uint8_t* st = sm + buf * S_STAGE;
         mbar_expect_tx(&bar_tma[buf], 7u * 8192u);
-        // [-W ; Q]: each 64-column block holds 128 rows (-W rows 0..63, q rows 64..127)
-        tma_load_4d(wq, &tm_w, &bar_tma[buf], 0, h, t0, bb);
-        tma_load_4d(wq + 16384, &tm_w, &bar_tma[buf], 64, h, t0, bb);
-        tma_load_4d(wq + 8192, &tm_q, &bar_tma[buf], 0, hq, t0, bb);
-        tma_load_4d(wq + 16384 + 8192, &tm_q, &bar_tma[buf], 64, hq, t0, bb);
-        tma_load_4d(kk, &tm_k, &bar_tma[buf], 0, hq, t0, bb);
-        tma_load_4d(kk + 8192, &tm_k, &bar_tma[buf], 64, hq, t0, bb);
-        tma_load_4d(sm + S_OFF_P + buf * 8192, &tm_p, &bar_tma[buf], v0, h, t0, bb);
+        // [Q ; -W]: each 64-column block holds 128 rows (q rows 0..63, -W rows 64..127)
+        tma_load_4d(st + S_ST_QW, &tm_q, &bar_tma[buf], 0, hq, t0, bb);
+        tma_load_4d(st + S_ST_QW + 16384, &tm_q, &bar_tma[buf], 64, hq, t0, bb);
+        tma_load_4d(st + S_ST_QW + 8192, &tm_w, &bar_tma[buf], 0, h, t0, bb);
+        tma_load_4d(st + S_ST_QW + 16384 + 8192, &tm_w, &bar_tma[buf], 64, h, t0, bb);
+        tma_load_4d(st + S_ST_K, &tm_k, &bar_tma[buf], 0, hq, t0, bb);
+        tma_load_4d(st + S_ST_K + 8192, &tm_k, &bar_tma[buf], 64, hq, t0, bb);
+        tma_load_4d(st + S_ST_P, &tm_p, &bar_tma[buf], v0, h, t0, bb);
     };
 
     constexpr int NH = NV / 2;
@@ -452,23 +480,22 @@ __global__ void __launch_bounds__(NT, 1) state_gdn_kernel(
 #pragma unroll
         for (int ch = 0; ch < 4; ++ch) st_chunk(sm + S_OFF_SBF, sw128_chunk(row, wg * 4 + ch, DK), &S[8 * ch]);
     }
-    // the state's bf16 copy is read by the first MMA batch (async proxy)
-    fence_proxy_async();
-    tc_fence_before();
-    __syncthreads();
-    unsigned short g_a = 0;
-    auto load_alpha = [&](int ci) {
-        if (tid < C) {
-            const int t = min(ci * C + tid, T - 1);
-            g_a = ((const unsigned short*)p.alpha)[((size_t)bb * T + t) * H + h];
-        }
-    };
+
+    // decay scan of one chunk by warp 1 (two tokens per lane, log2 alpha in
+    // registers): factors set ci % 3
+    const int lane = tid & 31;
     auto bits_to_f32 = [](unsigned short u) { return __uint_as_float((uint32_t)u << 16); };
-    auto decay_scan = [&](int ci, int lane) {
-        const int par = ci & 1;
-        const int n = min(C, T - ci * C);
-        const float la0 = (2 * lane < n) ? lg2_approx(s_alpha[2 * lane]) : 0.f;
-        const float la1 = (2 * lane + 1 < n) ? lg2_approx(s_alpha[2 * lane + 1]) : 0.f;
+    unsigned short a_nx0 = 0x3F80, a_nx1 = 0x3F80;  // alpha of the next chunk to scan (bf16 1.0)
+    auto load_alpha = [&](int ci) {
+        const int t = ci * C + 2 * lane;
+        const unsigned short* ap = (const unsigned short*)p.alpha;
+        a_nx0 = t < T ? ap[((size_t)bb * T + t) * H + h] : (unsigned short)0x3F80;
+        a_nx1 = t + 1 < T ? ap[((size_t)bb * T + t + 1) * H + h] : (unsigned short)0x3F80;
+    };
+    auto decay_scan = [&](int ci) {
+        const int s3 = ci % 3;
+        const float la0 = lg2_approx(bits_to_f32(a_nx0));
+        const float la1 = lg2_approx(bits_to_f32(a_nx1));
         float x = la0 + la1;
 #pragma unroll
         for (int off = 1; off < 32; off <<= 1) {
@@ -476,80 +503,58 @@ __global__ void __launch_bounds__(NT, 1) state_gdn_kernel(
             if (lane >= off) x += y;
         }
         const float l1 = x, l0v = x - la1;
-        const float first = __shfl_sync(0xffffffffu, l0v, 0);
         const float last = __shfl_sync(0xffffffffu, l1, 31);
-        const float ref = 0.5f * (first + last);
-        float* rf = s_rowf2 + par * 64;
-        float* cf = s_colf2 + par * 64;
-        float* g = s_g2 + par * 64;
-        float* gcr = s_gcr2 + par * 64;
-        rf[2 * lane] = ex2_approx(l0v - ref);
-        rf[2 * lane + 1] = ex2_approx(l1 - ref);
-        cf[2 * lane] = ex2_approx(ref - l0v);
-        cf[2 * lane + 1] = ex2_approx(ref - l1);
+        float* l = s_l3 + s3 * 64;
+        float* g = s_g3 + s3 * 64;
+        float* gcr = s_gcr3 + s3 * 64;
+        l[2 * lane] = l0v;
+        l[2 * lane + 1] = l1;
         g[2 * lane] = ex2_approx(l0v);
         g[2 * lane + 1] = ex2_approx(l1);
         gcr[2 * lane] = ex2_approx(last - l0v);
         gcr[2 * lane + 1] = ex2_approx(last - l1);
-        if (lane == 0) {
-            s_misc2[par * 4] = ex2_approx(last);
-            if (first - last > 230.f) flag_status(p.d_status, GDR_DEVICE_DECAY_RANGE);
-        }
+        if (lane == 0) s_gC3[s3 * 4] = ex2_approx(last);
     };
-    auto stage_alpha = [&](int ci) {
-        if (tid < C) s_alpha[tid] = ci * C + tid < T ? bits_to_f32(g_a) : 1.f;
-    };
+
+    // the state's bf16 copy is read by the first MMA (async proxy)
+    fence_proxy_async();
+    tc_fence_before();
     // Everything above overlaps the first pass's tail (this grid may be
     // launched before that one completes: programmatic dependent launch);
     // the first pass's factors are read only after it has completed.
     asm volatile("griddepcontrol.wait;" ::: "memory");
-    if (tid == 0) {
-        if (nchunks > 0) issue_loads(0);
-        if (nchunks > 1) issue_loads(1);
+    if (tid == 32) {
+        for (int ci = 0; ci < 2 && ci < nchunks; ++ci) issue_loads(ci);
     }
-    if (nchunks > 0) {
+    loads_issued = min(2, nchunks);
+    if (warp == 1 && nchunks > 0) {
         load_alpha(0);
-        stage_alpha(0);
-        __syncthreads();
-        if (warp == 7) decay_scan(0, tid & 31);
-        __syncthreads();
+        decay_scan(0);
+        if (nchunks > 1) load_alpha(1);
     }
+    __syncthreads();
 
-#define GDR_WAIT(bar, ph)                                                   \
-    do {                                                                    \
-        bool w_ok = mbar_wait(bar, ph);                                     \
-        ph ^= 1u;                                                           \
-        if (!__syncthreads_and(w_ok)) { ok = false; goto finish; }          \
-    } while (0)
-#define GDR_BEFORE_MMA()    \
-    do {                    \
-        fence_proxy_async(); \
-        tc_fence_before();  \
-        __syncthreads();    \
-    } while (0)
-    // Waits inside the chunk loop are per thread; a timed-out wait is carried in
-    // w_ok to the next block barrier, where the block leaves together.
     bool w_ok = true;
+    uint32_t ph_tma = 0u;  // bit i: phase parity of stage i
 #define GDR_WAIT_SOLO(bar, ph)              \
     do {                                    \
         w_ok = mbar_wait(bar, ph) && w_ok;  \
-        ph ^= 1u;                           \
     } while (0)
 #define GDR_SYNC_CHECK()                                            \
     do {                                                            \
         if (!__syncthreads_and(w_ok)) { ok = false; goto finish; }  \
     } while (0)
 
-    // O rows (64..127 of D3 / D5 in the column set of chunk cj) -> global
+    // O rows of chunk cj (lanes 0..63 of D3 and D5 in the column set of cj) -> global
     auto store_o = [&](int cj) {
         const int pj = cj & 1;
-        const int t = cj * C + row - 64;
+        const int t = cj * C + row;
         float d[32], d5[32];
         tmem_ld32_async(tmem + lane_base + S_TM_D3 + pj * 64 + wg * 32, d);
         tmem_ld32_async(tmem + lane_base + S_TM_D5 + pj * 64 + wg * 32, d5);
         tmem_wait_ld();
         if (t < T) {
-            const float gr = s_g2[pj * 64 + row - 64];
+            const float gr = s_g3[(cj % 3) * 64 + row];
             __nv_bfloat16* op = p.o + (((size_t)bb * T + t) * H + h) * p.dv + v0 + wg * 32;
 #pragma unroll
             for (int c8 = 0; c8 < 4; ++c8) {
@@ -567,150 +572,184 @@ __global__ void __launch_bounds__(NT, 1) state_gdn_kernel(
     };
 
     for (int ci = 0; ci < nchunks; ++ci) {
-        GDR_TRACE_S(7);
         const int buf = ci % S_NBUF;
-        const uint32_t wqb = sbase + S_OFF_WQ + buf * 32768u;
-        const uint32_t kb = sbase + S_OFF_K + buf * 16384u;
-        const uint32_t k2b = sbase + S_OFF_K2;
-        GDR_TRACE_S(0);
-        if (ci + 1 < nchunks) load_alpha(ci + 1);
         const int par = ci & 1;
-        const float* s_rowf = s_rowf2 + par * 64;
-        const float* s_colf = s_colf2 + par * 64;
-        const float* s_gcr = s_gcr2 + par * 64;
-        const float* s_misc = s_misc2 + par * 4;
-        if (buf == 0) GDR_WAIT_SOLO(&bar_tma[0], ph_tma0);
-        else if (buf == 1) GDR_WAIT_SOLO(&bar_tma[1], ph_tma1);
-        else GDR_WAIT_SOLO(&bar_tma[2], ph_tma2);
-        GDR_TRACE_S(1);
+        const uint32_t ph = (uint32_t)(ci & 1);
+        const uint32_t stb = sbase + buf * S_STAGE;
+        const uint32_t qwb = stb + S_ST_QW, kb = stb + S_ST_K;
+        const int s3 = ci % 3;
+        GDR_TRACE_S(0, 0);
+        GDR_WAIT_SOLO(&bar_tma[buf], (ph_tma >> buf) & 1u);
+        ph_tma ^= 1u << buf;
+        GDR_TRACE_S(1, 0);
 
-        // ---- batch 1: D3 = [-W ; Q] S;  D1 = [-W ; Q] K^T (rows 64..127: Q K^T) ------
-        const uint32_t d3 = S_TM_D3 + (uint32_t)par * 64u, d5 = S_TM_D5 + (uint32_t)par * 64u;
+        // ---- D3 = [Q ; -W] S, then D1 = [Q ; -W] K^T ----------------------------
         if (tid == 0) {
             tc_fence_after();
             const uint32_t idS = idesc_bf16(128, NV, 0, 1);
             const uint32_t idK = idesc_bf16(128, 64, 0, 0);
+            const uint32_t d3 = S_TM_D3 + (uint32_t)par * 64u;
+#pragma unroll
+            for (int ks = 0; ks < 8; ++ks) {
+                const uint32_t koff = (ks >> 2) * 16384u + (ks & 3) * 32u;
+                mma_bf16(tmem + d3, sdesc_sw128(qwb + koff, 16, 1024),
+                         sdesc_sw128(sbase + S_OFF_SBF + ks * 2048u, 8192, 1024), idS, ks > 0);
+            }
+            mma_commit(bar_w);
 #pragma unroll
             for (int ks = 0; ks < 8; ++ks) {
                 const uint32_t koff = (ks >> 2) * 16384u + (ks & 3) * 32u;
                 const uint32_t kkoff = (ks >> 2) * 8192u + (ks & 3) * 32u;
-                mma_bf16(tmem + d3, sdesc_sw128(wqb + koff, 16, 1024),
-                         sdesc_sw128(sbase + S_OFF_SBF + ks * 2048u, 8192, 1024), idS, ks > 0);
-                mma_bf16(tmem + S_TM_D1, sdesc_sw128(wqb + koff, 16, 1024),
+                mma_bf16(tmem + S_TM_D1, sdesc_sw128(qwb + koff, 16, 1024),
                          sdesc_sw128(kb + kkoff, 16, 1024), idK, ks > 0);
             }
-            mma_commit(bar_mma);
+            mma_commit(bar_q);
         }
         // chunk ci + 2's inputs go to the buffers chunk ci - 1 has released
         if (tid == 32 && ci + 2 < nchunks) issue_loads(ci + 2);
-        // the previous chunk's outputs, while batch 1 runs
-        if (row >= 64 && ci > 0) store_o(ci - 1);
-        // while batch 1 runs: K2 = K with rows scaled by g_{n-1} / g_r (batch 2 of
-        // the previous chunk, the last reader of K2, has completed)
-        {
-            const int r = tid >> 2, c4 = (tid & 3) * 4;  // 64 rows x 4 threads x 4 chunks
-            const float f = s_gcr[r];
-#pragma unroll
-            for (int cc = 0; cc < 4; ++cc) {
-                float x[8];
-                const uint32_t off = sw128_chunk(r, c4 + cc, 64);
-                ld_chunk(sm + S_OFF_K + buf * 16384, off, x);
-#pragma unroll
-                for (int e = 0; e < 8; ++e) x[e] *= f;
-                st_chunk(sm + S_OFF_K2, off, x);
-            }
-        }
-        GDR_WAIT_SOLO(bar_mma, ph_mma);
-        tc_fence_after();
-        GDR_TRACE_S(2);
+        if (ci + 2 < nchunks) loads_issued = ci + 3;
 
-        // ---- U = P - W S (rows 0..63) and Aq (rows 64..127) -> [U ; Aq] (bf16) ---------
-        if (row < 64) {
-            float d[32];
-            tmem_ld32(tmem + lane_base + d3 + wg * 32, d);
+        if (lo) {
+            // ---- warps 0, 1, 4, 5: O of the previous chunk, the next decay scan, Aq ----
+            if (ci > 0) {
+                GDR_WAIT_SOLO(bar_a, (uint32_t)((ci - 1) & 1));
+                tc_fence_after();
+                store_o(ci - 1);
+            }
+            GDR_TRACE_S(2, 0);
+            if (warp == 1 && ci + 1 < nchunks) {
+                decay_scan(ci + 1);
+                if (ci + 2 < nchunks) load_alpha(ci + 2);
+            }
+            GDR_WAIT_SOLO(bar_q, ph);
+            tc_fence_after();
+            GDR_TRACE_S(3, 0);
+            {
+                const int r = row;
+                float d[32];
+                tmem_ld32(tmem + lane_base + S_TM_D1 + wg * 32, d);
+                const float* l = s_l3 + s3 * 64;
+                const float lr = l[r];
 #pragma unroll
-            for (int c8 = 0; c8 < 4; ++c8) {
-                float x[8];
-                ld_chunk(sm + S_OFF_P + buf * 8192, sw128_chunk(row, wg * 4 + c8, 64), x);
+                for (int c8 = 0; c8 < 4; ++c8) {
+                    const int j0 = wg * 32 + c8 * 8;
+                    float x[8];
+                    if (j0 > r) {
 #pragma unroll
-                for (int e = 0; e < 8; ++e) x[e] += d[c8 * 8 + e];
-                st_chunk(sm + S_OFF_AQU, sw128_chunk(row, wg * 4 + c8, 128), x);
+                        for (int e = 0; e < 8; ++e) x[e] = 0.f;
+                    } else {
+                        const float4 la = *reinterpret_cast<const float4*>(l + j0);
+                        const float4 lb = *reinterpret_cast<const float4*>(l + j0 + 4);
+                        const float lj[8] = {la.x, la.y, la.z, la.w, lb.x, lb.y, lb.z, lb.w};
+#pragma unroll
+                        for (int e = 0; e < 8; ++e)
+                            x[e] = j0 + e <= r ? d[c8 * 8 + e] * ex2_approx(lr - lj[e]) : 0.f;
+                    }
+                    st_chunk(sm + S_OFF_AQ, sw128_chunk(r, wg * 4 + c8, 128), x);
+                }
+            }
+            fence_proxy_async();
+            tc_fence_before();
+            named_bar_sync(S_BAR_AQ, NT);  // U (warps 2, 3, 6, 7) and Aq ready
+            GDR_TRACE_S(4, 0);
+            if (tid == 0) {
+                // ---- D5 = [Aq ; U] U (lanes 0..63: Aq U) ----------------------------------
+                tc_fence_after();
+                const uint32_t idA = idesc_bf16(128, NV, 0, 1);
+                const uint32_t d5 = S_TM_D5 + (uint32_t)par * 64u;
+#pragma unroll
+                for (int ks = 0; ks < 4; ++ks)
+                    mma_bf16(tmem + d5, sdesc_sw128(sbase + S_OFF_AQ + ks * 32u, 16, 1024),
+                             sdesc_sw128(sbase + S_OFF_U + ks * 2048u, 8192, 1024), idA, ks > 0);
+                mma_commit(bar_a);
             }
         } else {
-            const int r = row - 64;
-            float d[32];
-            tmem_ld32(tmem + lane_base + S_TM_D1 + wg * 32, d);
-            const float rf = s_rowf[r];
-#pragma unroll
-            for (int c8 = 0; c8 < 4; ++c8) {
-                float x[8];
-                const float4 ca = *reinterpret_cast<const float4*>(s_colf + wg * 32 + c8 * 8);
-                const float4 cb = *reinterpret_cast<const float4*>(s_colf + wg * 32 + c8 * 8 + 4);
-                const float cf[8] = {ca.x, ca.y, ca.z, ca.w, cb.x, cb.y, cb.z, cb.w};
-#pragma unroll
-                for (int e = 0; e < 8; ++e) {
-                    const int j = wg * 32 + c8 * 8 + e;
-                    x[e] = j <= r ? rf * cf[e] * d[c8 * 8 + e] : 0.f;
-                }
-                st_chunk(sm + S_OFF_AQU, sw128_chunk(row, wg * 4 + c8, 128), x);
-            }
-        }
-        if (ci + 1 < nchunks) stage_alpha(ci + 1);
-        fence_proxy_async();
-        tc_fence_before();
-        GDR_SYNC_CHECK();
-        GDR_TRACE_S(3);
-
-        // ---- batch 2: D5 = [U ; Aq] U (rows 64..127: Aq U);  D4 = (Diag(g_{n-1}/g) K)^T U --
-        if (tid == 0) {
+            // ---- warps 2, 3, 6, 7: U = P - W S (lanes 64..127 of D3) -> U and U' ------
+            GDR_WAIT_SOLO(bar_w, ph);
             tc_fence_after();
-            const uint32_t idK = idesc_bf16(128, NV, 0, 1);
-            const uint32_t idM = idesc_bf16(128, NV, 1, 1);
+            GDR_TRACE_S(7, 64);
+            {
+                const int j = row - 64;  // token
+                float d[32];
+                tmem_ld32(tmem + lane_base + S_TM_D3 + (uint32_t)par * 64u + wg * 32, d);
+                const float f = s_gcr3[s3 * 64 + j];
 #pragma unroll
-            for (int ks = 0; ks < 4; ++ks) {
-                mma_bf16(tmem + d5, sdesc_sw128(sbase + S_OFF_AQU + ks * 32u, 16, 1024),
-                         sdesc_sw128(sbase + S_OFF_AQU + ks * 2048u, 8192, 1024), idK, ks > 0);
-                mma_bf16(tmem + S_TM_D4, sdesc_sw128(k2b + ks * 2048u, 8192, 1024),
-                         sdesc_sw128(sbase + S_OFF_AQU + ks * 2048u, 8192, 1024), idM, ks > 0);
+                for (int c8 = 0; c8 < 4; ++c8) {
+                    float x[8];
+                    const uint32_t off = sw128_chunk(j, wg * 4 + c8, 64);
+                    ld_chunk(sm + buf * S_STAGE + S_ST_P, off, x);
+#pragma unroll
+                    for (int e = 0; e < 8; ++e) x[e] += d[c8 * 8 + e];
+                    st_chunk(sm + S_OFF_U, off, x);
+#pragma unroll
+                    for (int e = 0; e < 8; ++e) x[e] *= f;
+                    st_chunk(sm + S_OFF_U2, off, x);
+                }
             }
-            mma_commit(bar_mma);
+            fence_proxy_async();
+            tc_fence_before();
+            named_bar_sync(S_BAR_U, 128);
+            if (tid == 64) {
+                // ---- D4 = K^T U' (state increment) ---------------------------------------
+                tc_fence_after();
+                const uint32_t idM = idesc_bf16(128, NV, 1, 1);
+#pragma unroll
+                for (int ks = 0; ks < 4; ++ks)
+                    mma_bf16(tmem + S_TM_D4, sdesc_sw128(kb + ks * 2048u, 8192, 1024),
+                             sdesc_sw128(sbase + S_OFF_U2 + ks * 2048u, 8192, 1024), idM, ks > 0);
+                mma_commit(bar_k);
+            }
+            named_bar_arrive(S_BAR_AQ, NT);
         }
-        if (warp == 7 && ci + 1 < nchunks) decay_scan(ci + 1, tid & 31);  // overlaps batch 2
-        GDR_WAIT_SOLO(bar_mma, ph_mma);
-        tc_fence_after();
-        GDR_TRACE_S(4);
 
-        // ---- S = g_{n-1} S + D4 (the outputs are written during the next batch 1) -----
+        // ---- S = g_{n-1} S + D4 (every warp: its lanes, half the columns) -----------
+        GDR_WAIT_SOLO(bar_k, ph);
+        tc_fence_after();
+        GDR_TRACE_S(5, 0);
         {
             float dS[32];
             tmem_ld32(tmem + lane_base + S_TM_D4 + wg * 32, dS);
-            const float gC = s_misc[0];
+            const float gC = s_gC3[s3 * 4];
 #pragma unroll
-            for (int j = 0; j < NH; ++j) S[j] = fmaf(gC, S[j], dS[j]);
+            for (int jj = 0; jj < NH; ++jj) S[jj] = fmaf(gC, S[jj], dS[jj]);
 #pragma unroll
             for (int ch = 0; ch < 4; ++ch) st_chunk(sm + S_OFF_SBF, sw128_chunk(row, wg * 4 + ch, DK), &S[8 * ch]);
         }
-        GDR_TRACE_S(6);
         fence_proxy_async();  // the state copy feeds the next chunk's MMAs
         tc_fence_before();
         GDR_SYNC_CHECK();
-        GDR_TRACE_S(5);
+        GDR_TRACE_S(6, 0);
     }
-    if (row >= 64 && nchunks > 0) store_o(nchunks - 1);
+    if (lo && nchunks > 0) {
+        GDR_WAIT_SOLO(bar_a, (uint32_t)((nchunks - 1) & 1));
+        tc_fence_after();
+        store_o(nchunks - 1);
+    }
+    if (!__syncthreads_and(w_ok)) ok = false;
 
-    if (p.ST) {
+    if (ok && p.ST) {
         float* st = p.ST + (((size_t)bb * H + h) * DK + row) * p.dv + v0 + wg * NH;
 #pragma unroll
-        for (int j = 0; j < NH; j += 4) *reinterpret_cast<float4*>(st + j) = make_float4(S[j], S[j + 1], S[j + 2], S[j + 3]);
+        for (int jj = 0; jj < NH; jj += 4)
+            *reinterpret_cast<float4*>(st + jj) = make_float4(S[jj], S[jj + 1], S[jj + 2], S[jj + 3]);
     }
 
 finish:
-    if (!ok && tid == 0) flag_status(p.d_status, GDR_DEVICE_TIMEOUT);
+    if (!ok) {
+        if (tid == 0) flag_status(p.d_status, GDR_DEVICE_TIMEOUT);
+        // before the block leaves (each wait bounded): the input copies it
+        // requested have landed and the MMAs of both issuing threads are done
+        if (tid == 32)
+            for (int ci = max(0, loads_issued - S_NBUF); ci < loads_issued; ++ci)
+                (void)mbar_wait(&bar_tma[ci % S_NBUF], (uint32_t)((ci / S_NBUF) & 1));
+        if (tid == 0 || tid == 64) {
+            mma_commit(bar_drain);
+            (void)mbar_wait(bar_drain, 0);
+        }
+    }
     tc_fence_before();
     __syncthreads();
     if (warp == 0) tmem_dealloc(tmem, S_TM_COLS);
-#undef GDR_WAIT
-#undef GDR_BEFORE_MMA
 #undef GDR_WAIT_SOLO
 #undef GDR_SYNC_CHECK
 }

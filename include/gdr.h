@@ -78,7 +78,7 @@ typedef enum {
 
 /* Flags ORed into *d_status by the kernels. */
 #define GDR_DEVICE_TIMEOUT 1       /* a bounded pipeline wait expired; results invalid */
-#define GDR_DEVICE_DECAY_RANGE 2   /* chunk decay span outside the tensor-core path's range */
+#define GDR_DEVICE_DECAY_RANGE 2   /* a chunk took the exact fallback (see gdr_chunk_fwd); informational */
 
 typedef enum { GDR_BF16 = 0, GDR_FP32 = 1 } gdr_dtype;
 
@@ -102,11 +102,16 @@ typedef enum {
  * value. The result does not depend on it beyond rounding.
  * Paths: dtype GDR_BF16 with d_k = 128 and d_v a multiple of 64 runs the
  * tcgen05 tensor-core chunk kernel (bf16 operands, fp32 accumulation, fp32
- * state on chip). Its decay range: within every chunk and channel the
- * summed -log(alpha) over the chunk's tokens after the first must not exceed
- * 160 (outside it the kernel sets GDR_DEVICE_DECAY_RANGE). Every other
- * supported shape (fp32, or 1 <= d_k <= 256 and 1 <= d_v <= 1024 otherwise)
- * runs an exact fp32 token-by-token CUDA kernel.
+ * state on chip). Every other supported shape (fp32, or 1 <= d_k <= 256 and
+ * 1 <= d_v <= 1024 otherwise) runs an exact fp32 token-by-token CUDA kernel.
+ * Decay: any alpha in (0, 1] is in range. With one decay per token (scalar
+ * alpha) the tensor-core kernels form every ratio of decay products inside a
+ * chunk per element, where it is at most 1. With channel-wise decay they
+ * split each ratio into two factors around a per-chunk reference; a chunk
+ * whose summed -log(alpha) in some channel exceeds about 160 cannot be split
+ * that way, so that chunk alone is applied token by token in fp32 on CUDA
+ * cores (exact, slower), and GDR_DEVICE_DECAY_RANGE is ORed into d_status to
+ * say that the fallback ran.
  * Alignment: q, k, v, o and channel gates must be 16-byte aligned and, on
  * the tensor-core path, d_k and d_v rows 16-byte multiples (given by the
  * shape rules above).

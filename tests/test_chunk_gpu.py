@@ -128,16 +128,20 @@ def test_final_state_in_place(cuda_device):
 
 
 def test_decay_range_flag(cuda_device):
-    """A chunk whose decay span exceeds the tensor-core path's range is
-    reported through d_status; in-range inputs leave it zero."""
+    """A channel-decay chunk whose decay span exceeds the two-factor range is
+    applied token by token (the result still matches the oracle) and reported
+    through d_status; in-range inputs leave the status zero."""
     wl = small("kda", T=64, H=1, B=1, seed=13)
     inp = make_chunk_inputs(wl)
     st = torch.zeros(1, dtype=torch.int32, device=cuda_device)
     run_chunk(inp, cuda_device, d_status=st)
     assert int(st.item()) == 0
     inp["alpha"] = torch.full_like(inp["alpha"], 0.01)   # 63 x 4.6 nats > 160
-    run_chunk(inp, cuda_device, d_status=st)
+    o, ST = run_chunk(inp, cuda_device, d_status=st)
     assert int(st.item()) & GDR_DEVICE_DECAY_RANGE
+    o_ref, ST_ref = run_oracle(inp)
+    assert_close(o, o_ref, TOL["bf16"], "o (fallback chunk)")
+    assert_close(ST, ST_ref, TOL["bf16"], "S_T (fallback chunk)")
 
 
 @pytest.mark.parametrize("family", FAMILIES)
