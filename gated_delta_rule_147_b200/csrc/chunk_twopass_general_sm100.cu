@@ -638,9 +638,9 @@ struct StateLayout {
     static constexpr uint32_t BYTES = SMALL + 1024 + 1024;
 };
 // D3 ([QG S ; U - P]) and D5 (AQ U (+ BQ V), lanes 0..63) alternate between two
-// column sets by chunk parity; D4 = K2^T U (+ KW2^T V).
+// column sets; D4 = K2^T U (+ KW2^T V).
 constexpr uint32_t GS_TM_D3 = 0, GS_TM_D5 = 128, GS_TM_D4 = 256, GS_TM_COLS = 512;
-constexpr int GS_BAR_U = 2;  // named barrier: U written (warps 2, 3, 6, 7); 1 is the fallback's
+constexpr int GS_NT = 288;  // warps 0..7 compute, warp 8 issues MMAs and TMA loads
 
 struct GStateParams {
     const float* S0;  // state at chunk c_begin (NULL: zero)
@@ -654,21 +654,35 @@ struct GStateParams {
     int c_begin, c_end;  // chunk range of this launch
 };
 
-__device__ __forceinline__ void gs_named_bar_sync(int id, int n) {
-    asm volatile("bar.sync %0, %1;" ::"r"(id), "r"(n) : "memory");
+__device__ __forceinline__ bool gs_compute_bar_and(bool pred) {
+    uint32_t r;
+    asm volatile(
+        "{\n\t.reg .pred p, q;\n\t"
+        "setp.ne.u32 p, %1, 0;\n\t"
+        "barrier.red.and.pred q, 1, 256, p;\n\t"
+        "selp.u32 %0, 1, 0, q;\n\t}"
+        : "=r"(r)
+        : "r"((uint32_t)pred)
+        : "memory");
+    return r != 0;
+}
+
+__device__ __forceinline__ void gs_mbar_arrive(uint64_t* bar) {
+    asm volatile("mbarrier.arrive.shared::cta.b64 _, [%0];" ::"r"(smem_u32(bar)) : "memory");
 }
 
 // Chunk step. The chain from one chunk to the next holds only the products
 // that depend on the state:
 //   D3 = [QG ; WN] S          (U = P + WN S in lanes 64..127, by warps 2, 3, 6, 7)
-//   D4 (+)= K2^T U            (S <- Diag(g_{n-1}) S + D4, all warps)
-// and beside it, on the same issuing thread (thread 64) so products into one
-// accumulator keep their order: untied D4 = KW2^T V and D5 = [BQ ; .] V
-// (queued after D3, before U exists), and D5 (+)= [AQ ; .] U after D4's
-// product; O = QG S + AQ U (+ BQ V), lanes 0..63, is written by warps 0, 1,
-// 4, 5 during the next chunk's first product.
+//   D4 = K2^T U (+ KW2^T V)   (S <- Diag(g_{n-1}) S + D4, warps 0..7)
+// and after it, from the same issuing warp (warp 8), D5 = [AQ ; .] U (+ [BQ ; .]
+// V); O = QG S + AQ U (+ BQ V), lanes 0..63, is written by warps 0, 1, 4, 5
+// during the next chunk. No product is in flight while U is written: their
+// operand reads would take the shared-memory bandwidth the unload needs. A chunk marked by the first pass
+// (negative g_{n-1}: its decay span does not fit two bounded factors) is
+// applied token by token from the raw inputs instead, with no MMA.
 template <bool UNTIED>
-__global__ void __launch_bounds__(NT, 1) state_general_kernel(
+__global__ void __launch_bounds__(GS_NT, 1) state_general_kernel(
     const __grid_constant__ CUtensorMap tm_wn, const __grid_constant__ CUtensorMap tm_qg,
     const __grid_constant__ CUtensorMap tm_k2, const __grid_constant__ CUtensorMap tm_aq,
     const __grid_constant__ CUtensorMap tm_p, const __grid_constant__ CUtensorMap tm_kw2,
@@ -678,13 +692,13 @@ __global__ void __launch_bounds__(NT, 1) state_general_kernel(
     extern __shared__ uint8_t smem_raw[];
     uint8_t* sm = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) &
                                              ~uintptr_t(1023));
-    const int tid = threadIdx.x, warp = tid >> 5, wg = warp >> 2, row = tid & 127;
+    const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
+    const int wg = (warp >> 2) & 1, row = tid & 127;
     const bool lo = row < 64;
     const int vt = blockIdx.x, h = blockIdx.y, bb = blockIdx.z;
     const int v0 = vt * NV;
     const int T = p.T, H = p.H;
     const int nchunks = (T + C - 1) / C;
-    constexpr int ISSUER = 64;  // thread that issues every MMA (warp 2)
 
     constexpr int NBUF = Lay::NBUF;
     uint64_t* bar_tma = reinterpret_cast<uint64_t*>(sm + Lay::SMALL);  // [3]
@@ -692,13 +706,17 @@ __global__ void __launch_bounds__(NT, 1) state_general_kernel(
     uint64_t* bar_k = bar_tma + 4;
     uint64_t* bar_a = bar_tma + 5;
     uint64_t* bar_drain = bar_tma + 6;
-    uint32_t* s_tmem = reinterpret_cast<uint32_t*>(sm + Lay::SMALL + 64);
+    uint64_t* u_ready = bar_tma + 7;
+    uint64_t* s_ready = bar_tma + 8;
+    uint32_t* s_tmem = reinterpret_cast<uint32_t*>(sm + Lay::SMALL + 128);
     if (tid == 0) {
         for (int i = 0; i < 3; ++i) mbar_init(&bar_tma[i], 1);
         mbar_init(bar_w, 1);
         mbar_init(bar_k, 1);
         mbar_init(bar_a, 1);
         mbar_init(bar_drain, 1);
+        mbar_init(u_ready, 128);
+        mbar_init(s_ready, 1);
         fence_barrier_init();
     }
     if (warp == 0) tmem_alloc(s_tmem, GS_TM_COLS);
@@ -707,11 +725,10 @@ __global__ void __launch_bounds__(NT, 1) state_general_kernel(
     tc_fence_after();
     const uint32_t tmem = *s_tmem;
     const uint32_t lane_base = (uint32_t)((warp & 3) * 32) << 16;
-    uint32_t ph_tma = 0u;  // bit i: phase parity of stage i
     bool ok = true;
     const uint32_t sbase = smem_u32(sm);
     const int c_begin = p.c_begin, c_end = p.c_end;
-    int loads_issued = c_begin;  // chunks [c_begin, loads_issued) have been requested
+    const float* gch = p.gc + ((size_t)bb * H + h) * nchunks * DK;  // [nchunks][128]
 
     auto issue_loads = [&](int ci) {
         const int t0 = ci * C, buf = ci % NBUF;
@@ -737,7 +754,7 @@ __global__ void __launch_bounds__(NT, 1) state_general_kernel(
 
     constexpr int NH = NV / 2;
     float S[NH];
-    {
+    if (warp < 8) {
         const float* s0 = p.S0 ? p.S0 + (((size_t)bb * H + h) * DK + row) * p.dv + v0 + wg * NH : nullptr;
 #pragma unroll
         for (int j = 0; j < NH; j += 4) {
@@ -750,190 +767,196 @@ __global__ void __launch_bounds__(NT, 1) state_general_kernel(
     // the state's bf16 copy is read by the first MMA batch (async proxy)
     fence_proxy_async();
     tc_fence_before();
-    __syncthreads();
-    const float* gcp = p.gc + ((size_t)bb * H + h) * nchunks * DK + row;
-    float gC_next = c_begin < c_end ? gcp[(size_t)c_begin * DK] : 0.f;
-    if (tid == 32) {
+    if (warp == 8 && lane == 0)
         for (int ci = c_begin; ci < c_end && ci < c_begin + NBUF - 1; ++ci) issue_loads(ci);
-    }
-    loads_issued = min(c_end, c_begin + NBUF - 1);
+    __syncthreads();
 
-    auto store_o = [&](int cj, int pj) {
-        const int t = cj * C + row;
-        float d[32], d5[32];
-        tmem_ld32_async(tmem + lane_base + GS_TM_D3 + pj * 64 + wg * 32, d);
-        tmem_ld32_async(tmem + lane_base + GS_TM_D5 + pj * 64 + wg * 32, d5);
-        tmem_wait_ld();
-        if (t < T) {
-#pragma unroll
-            for (int j = 0; j < 32; ++j) d[j] += d5[j];
-            st32_bf16(p.o + (((size_t)bb * T + t) * H + h) * p.dv + v0 + wg * 32, d, 1.f);
-        }
-    };
-
-    // Waits inside the chunk loop are per thread; a timed-out wait is carried in
-    // w_ok to the block barrier that ends the chunk, where the block leaves together.
-    bool w_ok = true;
-#define GDR_WAIT_SOLO(bar, ph)              \
-    do {                                    \
-        w_ok = mbar_wait(bar, ph) && w_ok;  \
-    } while (0)
-#define GDR_SYNC_CHECK()                                            \
-    do {                                                            \
-        if (!__syncthreads_and(w_ok)) { ok = false; goto finish; }  \
-    } while (0)
-
-    // nm counts the chunks taken on the tensor cores: their barriers' phases
-    // and TMEM column sets follow it. A chunk whose g_{n-1} is marked negative
-    // by the first pass (decay span outside the factorisation's range) is
-    // applied token by token instead, from the raw inputs.
-    int nm = 0;
-    int pend = -1;  // chunk whose O still sits in TMEM (column set pend_set), or -1
-    int pend_set = 0;
-    uint32_t pend_ph = 0;
-    for (int ci = c_begin; ci < c_end; ++ci) {
-        const int buf = ci % NBUF, par = nm & 1;
-        const uint32_t ph = (uint32_t)(nm & 1);
-        const uint32_t qwb = sbase + Lay::QW + buf * 32768u;
-        const uint32_t k2b = sbase + Lay::K2 + buf * 16384u;
-        const uint32_t aqa = sbase + Lay::AQ + buf * 8192u;  // AQ = rows 0..63
-        const uint32_t ub = sbase + Lay::U;
-        const uint32_t d3 = GS_TM_D3 + (uint32_t)par * 64u, d5 = GS_TM_D5 + (uint32_t)par * 64u;
-        const float gC = gC_next;
-        if (ci + 1 < c_end) gC_next = gcp[(size_t)(ci + 1) * DK];
-        const bool exact = gC < 0.f;  // the same mark in every channel: uniform
-        GDR_WAIT_SOLO(&bar_tma[buf], (ph_tma >> buf) & 1u);
-        ph_tma ^= 1u << buf;
-
-        // ---- D3 = [QG ; WN] S;  untied: D4 = KW2^T V, D5 = [BQ ; .] V --------------------
-        if (tid == ISSUER && !exact) {
+    if (warp == 8) {
+        // ---------------- issuer warp ------------------------------------------------
+        bool iok = true;
+        int nm = 0;            // chunks taken on the tensor cores so far
+        int loads_issued = min(c_end, c_begin + NBUF - 1);
+        bool prev_mma = false;  // chunk ci - 1 ran on the tensor cores (its AQ U may be in flight)
+        for (int ci = c_begin; ci < c_end; ++ci) {
+            const int buf = ci % NBUF, par = nm & 1;
+            const uint32_t qwb = sbase + Lay::QW + buf * 32768u;
+            const uint32_t k2b = sbase + Lay::K2 + buf * 16384u;
+            const uint32_t aqa = sbase + Lay::AQ + buf * 8192u;  // AQ = rows 0..63
+            const uint32_t ub = sbase + Lay::U;
+            const uint32_t d3 = GS_TM_D3 + (uint32_t)par * 64u, d5 = GS_TM_D5 + (uint32_t)par * 64u;
+            const bool exact = gch[(size_t)ci * DK] < 0.f;
+            iok = mbar_wait(&bar_tma[buf], (uint32_t)(((ci - c_begin) / NBUF) & 1)) && iok;
+            if (ci > c_begin) iok = mbar_wait(s_ready, (uint32_t)((ci - 1 - c_begin) & 1)) && iok;
+            // the stage of chunk ci - 1 is refilled below: its AQ tile's last reader done
+            if (prev_mma) iok = mbar_wait(bar_a, (uint32_t)((nm - 1) & 1)) && iok;
+            iok = __all_sync(0xffffffffu, iok);
+            if (!iok) break;
             tc_fence_after();
-            const uint32_t idS = idesc_bf16(128, NV, 0, 1);
+            if (lane == 0) {
+                if (!exact) {
+                    const uint32_t idS = idesc_bf16(128, NV, 0, 1);
 #pragma unroll
-            for (int ks = 0; ks < 8; ++ks) {
-                const uint32_t koff = (ks >> 2) * 16384u + (ks & 3) * 32u;
-                mma_bf16(tmem + d3, sdesc_sw128(qwb + koff, 16, 1024),
-                         sdesc_sw128(sbase + Lay::SBF + ks * 2048u, 8192, 1024), idS, ks > 0);
-            }
-            mma_commit(bar_w);
-            if (UNTIED) {
-                const uint32_t idM = idesc_bf16(128, NV, 1, 1);
-                const uint32_t vb = sbase + Lay::V + buf * 8192u;
-                const uint32_t bqa = sbase + Lay::BQ + buf * 8192u;  // BQ = rows 0..63
-#pragma unroll
-                for (int ks = 0; ks < 4; ++ks) {
-                    mma_bf16(tmem + GS_TM_D4, sdesc_sw128(sbase + Lay::KW2 + buf * 16384u + ks * 2048u, 8192, 1024),
-                             sdesc_sw128(vb + ks * 2048u, 8192, 1024), idM, ks > 0);
-                    mma_bf16(tmem + d5, sdesc_sw128(bqa + ks * 32u, 16, 1024),
-                             sdesc_sw128(vb + ks * 2048u, 8192, 1024), idS, ks > 0);
-                }
-            }
-        }
-        // the previous chunk's outputs (lanes 0..63), while the first product runs
-        if (lo && pend >= 0) {
-            GDR_WAIT_SOLO(bar_a, pend_ph);
-            tc_fence_after();
-            store_o(pend, pend_set);
-        }
-        pend = -1;
-        // chunk ci + NBUF - 1's inputs go to the buffers of chunk ci - 1, whose last
-        // reader (its AQ U product) the wait above has seen complete (thread 32 is
-        // one of the waiting warps)
-        if (tid == 32 && ci + NBUF - 1 < c_end) issue_loads(ci + NBUF - 1);
-        if (ci + NBUF - 1 < c_end) loads_issued = ci + NBUF;
-        if (exact) {
-            exact_tokens(p.ex, S, reinterpret_cast<float*>(sm + Lay::EXR), bb, h, h / p.group, v0,
-                         ci * C, min(C, T - ci * C), tid);
-        } else {
-            if (!lo) {
-                // ---- U = P + WN S (lanes 64..127 of D3) -> U -------------------------------
-                GDR_WAIT_SOLO(bar_w, ph);
-                tc_fence_after();
-                {
-                    const int j = row - 64;
-                    float d[32];
-                    tmem_ld32(tmem + lane_base + d3 + wg * 32, d);
-#pragma unroll
-                    for (int c8 = 0; c8 < 4; ++c8) {
-                        float x[8];
-                        const uint32_t off = sw128_chunk(j, wg * 4 + c8, 64);
-                        ld_chunk(sm + Lay::P + buf * 8192, off, x);
-#pragma unroll
-                        for (int e = 0; e < 8; ++e) x[e] += d[c8 * 8 + e];
-                        st_chunk(sm + Lay::U, off, x);
+                    for (int ks = 0; ks < 8; ++ks) {
+                        const uint32_t koff = (ks >> 2) * 16384u + (ks & 3) * 32u;
+                        mma_bf16(tmem + d3, sdesc_sw128(qwb + koff, 16, 1024),
+                                 sdesc_sw128(sbase + Lay::SBF + ks * 2048u, 8192, 1024), idS, ks > 0);
                     }
+                    mma_commit(bar_w);
                 }
-                fence_proxy_async();
-                tc_fence_before();
-                gs_named_bar_sync(GS_BAR_U, 128);
-                if (tid == ISSUER) {
-                    // ---- D4 (+)= K2^T U, then D5 (+)= [AQ ; .] U ------------------------------
-                    tc_fence_after();
+                // chunk ci + NBUF - 1's inputs go to the buffers of chunk ci - 1
+                if (ci + NBUF - 1 < c_end) issue_loads(ci + NBUF - 1);
+            }
+            if (ci + NBUF - 1 < c_end) loads_issued = ci + NBUF;
+            __syncwarp();
+            if (!exact) {
+                iok = __all_sync(0xffffffffu, mbar_wait(u_ready, (uint32_t)(nm & 1)) && iok);
+                if (!iok) break;
+                tc_fence_after();
+                if (lane == 0) {
+                    // ---- D4 = K2^T U (+ KW2^T V), then D5 = [AQ ; .] U (+ [BQ ; .] V): the
+                    //      products with V come after the state's, and no product runs
+                    //      while U is being written (its shared-memory reads would slow it)
                     const uint32_t idK = idesc_bf16(128, NV, 0, 1);
                     const uint32_t idM = idesc_bf16(128, NV, 1, 1);
+                    const uint32_t vb = sbase + Lay::V + buf * 8192u;
+                    const uint32_t bqa = sbase + Lay::BQ + buf * 8192u;  // BQ = rows 0..63
 #pragma unroll
                     for (int ks = 0; ks < 4; ++ks)
                         mma_bf16(tmem + GS_TM_D4, sdesc_sw128(k2b + ks * 2048u, 8192, 1024),
-                                 sdesc_sw128(ub + ks * 2048u, 8192, 1024), idM, UNTIED ? 1u : (uint32_t)(ks > 0));
+                                 sdesc_sw128(ub + ks * 2048u, 8192, 1024), idM, ks > 0);
+                    if (UNTIED)
+#pragma unroll
+                        for (int ks = 0; ks < 4; ++ks)
+                            mma_bf16(tmem + GS_TM_D4, sdesc_sw128(sbase + Lay::KW2 + buf * 16384u + ks * 2048u, 8192, 1024),
+                                     sdesc_sw128(vb + ks * 2048u, 8192, 1024), idM, 1u);
                     mma_commit(bar_k);
 #pragma unroll
                     for (int ks = 0; ks < 4; ++ks)
                         mma_bf16(tmem + d5, sdesc_sw128(aqa + ks * 32u, 16, 1024),
-                                 sdesc_sw128(ub + ks * 2048u, 8192, 1024), idK, UNTIED ? 1u : (uint32_t)(ks > 0));
+                                 sdesc_sw128(ub + ks * 2048u, 8192, 1024), idK, ks > 0);
+                    if (UNTIED)
+#pragma unroll
+                        for (int ks = 0; ks < 4; ++ks)
+                            mma_bf16(tmem + d5, sdesc_sw128(bqa + ks * 32u, 16, 1024),
+                                     sdesc_sw128(vb + ks * 2048u, 8192, 1024), idK, 1u);
                     mma_commit(bar_a);
                 }
+                __syncwarp();
+                ++nm;
             }
-            // ---- S = Diag(GC) S + D4 -----------------------------------------------------
-            GDR_WAIT_SOLO(bar_k, ph);
+            prev_mma = !exact;
+        }
+        if (!iok) {
+            ok = false;
+            if (lane == 0) {
+                // before the block leaves (each wait bounded): the requested input
+                // copies have landed and the issued MMAs have finished
+                for (int ci = max(c_begin, loads_issued - NBUF); ci < loads_issued; ++ci)
+                    (void)mbar_wait(&bar_tma[ci % NBUF], (uint32_t)(((ci - c_begin) / NBUF) & 1));
+                mma_commit(bar_drain);
+                (void)mbar_wait(bar_drain, 0);
+            }
+            __syncwarp();
+        }
+    } else {
+        // ---------------- compute warps ------------------------------------------------
+        const float* gcp = gch + row;
+        float gC_next = c_begin < c_end ? gcp[(size_t)c_begin * DK] : 0.f;
+        auto store_o = [&](int cj, int pj) {
+            const int t = cj * C + row;
+            float d[32], d5[32];
+            tmem_ld32_async(tmem + lane_base + GS_TM_D3 + pj * 64 + wg * 32, d);
+            tmem_ld32_async(tmem + lane_base + GS_TM_D5 + pj * 64 + wg * 32, d5);
+            tmem_wait_ld();
+            if (t < T) {
+#pragma unroll
+                for (int j = 0; j < 32; ++j) d[j] += d5[j];
+                st32_bf16(p.o + (((size_t)bb * T + t) * H + h) * p.dv + v0 + wg * 32, d, 1.f);
+            }
+        };
+        bool w_ok = true;
+        int nm = 0;
+        int pend = -1, pend_set = 0;  // chunk whose O still sits in TMEM
+        uint32_t pend_ph = 0;
+        int ci = c_begin;
+        for (; ci < c_end; ++ci) {
+            const int buf = ci % NBUF, par = nm & 1;
+            const uint32_t ph = (uint32_t)(nm & 1);
+            const uint32_t d3 = GS_TM_D3 + (uint32_t)par * 64u;
+            const float gC = gC_next;
+            if (ci + 1 < c_end) gC_next = gcp[(size_t)(ci + 1) * DK];
+            const bool exact = gC < 0.f;  // the same mark in every channel: uniform
+            if (lo && pend >= 0) {
+                w_ok = mbar_wait(bar_a, pend_ph) && w_ok;
+                tc_fence_after();
+                store_o(pend, pend_set);
+            }
+            pend = -1;
+            if (exact) {
+                exact_tokens(p.ex, S, reinterpret_cast<float*>(sm + Lay::EXR), bb, h, h / p.group, v0,
+                             ci * C, min(C, T - ci * C), tid);
+            } else {
+                if (!lo) {
+                    // ---- U = P + WN S (lanes 64..127 of D3) -> U --------------------------
+                    w_ok = mbar_wait(&bar_tma[buf], (uint32_t)(((ci - c_begin) / NBUF) & 1)) && w_ok;
+                    w_ok = mbar_wait(bar_w, ph) && w_ok;
+                    tc_fence_after();
+                    {
+                        const int j = row - 64;
+                        float d[32];
+                        tmem_ld32(tmem + lane_base + d3 + wg * 32, d);
+#pragma unroll
+                        for (int c8 = 0; c8 < 4; ++c8) {
+                            float x[8];
+                            const uint32_t off = sw128_chunk(j, wg * 4 + c8, 64);
+                            ld_chunk(sm + Lay::P + buf * 8192, off, x);
+#pragma unroll
+                            for (int e = 0; e < 8; ++e) x[e] += d[c8 * 8 + e];
+                            st_chunk(sm + Lay::U, off, x);
+                        }
+                    }
+                    fence_proxy_async();
+                    tc_fence_before();
+                    gs_mbar_arrive(u_ready);
+                }
+                // ---- S = Diag(GC) S + D4 -------------------------------------------------
+                w_ok = mbar_wait(bar_k, ph) && w_ok;
+                tc_fence_after();
+                {
+                    float dS[32];
+                    tmem_ld32(tmem + lane_base + GS_TM_D4 + wg * 32, dS);
+#pragma unroll
+                    for (int j = 0; j < NH; ++j) S[j] = fmaf(gC, S[j], dS[j]);
+                }
+                pend = ci;
+                pend_set = par;
+                pend_ph = ph;
+                ++nm;
+            }
+#pragma unroll
+            for (int ch = 0; ch < 4; ++ch) st_chunk(sm + Lay::SBF, sw128_chunk(row, wg * 4 + ch, DK), &S[8 * ch]);
+            fence_proxy_async();  // the state copy feeds the next chunk's MMAs
+            tc_fence_before();
+            if (!gs_compute_bar_and(w_ok)) break;
+            if (tid == 0) gs_mbar_arrive(s_ready);
+        }
+        if (ci < c_end) ok = false;  // a wait gave up
+        if (ok && lo && pend >= 0) {
+            ok = mbar_wait(bar_a, pend_ph);
             tc_fence_after();
-            {
-                float dS[32];
-                tmem_ld32(tmem + lane_base + GS_TM_D4 + wg * 32, dS);
-#pragma unroll
-                for (int j = 0; j < NH; ++j) S[j] = fmaf(gC, S[j], dS[j]);
-            }
-            pend = ci;
-            pend_set = par;
-            pend_ph = ph;
-            ++nm;
+            if (ok) store_o(pend, pend_set);
         }
+        if (!gs_compute_bar_and(ok)) ok = false;
+        if (ok && p.ST) {
+            float* st = p.ST + (((size_t)bb * H + h) * DK + row) * p.dv + v0 + wg * NH;
 #pragma unroll
-        for (int ch = 0; ch < 4; ++ch) st_chunk(sm + Lay::SBF, sw128_chunk(row, wg * 4 + ch, DK), &S[8 * ch]);
-        fence_proxy_async();  // the state copy feeds the next chunk's MMAs
-        tc_fence_before();
-        GDR_SYNC_CHECK();
-    }
-    if (lo && pend >= 0) {
-        GDR_WAIT_SOLO(bar_a, pend_ph);
-        tc_fence_after();
-        store_o(pend, pend_set);
-    }
-    if (!__syncthreads_and(w_ok)) ok = false;
-
-    if (ok && p.ST) {
-        float* st = p.ST + (((size_t)bb * H + h) * DK + row) * p.dv + v0 + wg * NH;
-#pragma unroll
-        for (int j = 0; j < NH; j += 4) *reinterpret_cast<float4*>(st + j) = make_float4(S[j], S[j + 1], S[j + 2], S[j + 3]);
-    }
-
-finish:
-    if (!ok) {
-        if (tid == 0) flag_status(p.d_status, GDR_DEVICE_TIMEOUT);
-        // before the block leaves (each wait bounded): the input copies it
-        // requested have landed and the issued MMAs are done
-        if (tid == 32)
-            for (int ci = max(c_begin, loads_issued - NBUF); ci < loads_issued; ++ci)
-                (void)mbar_wait(&bar_tma[ci % NBUF], (uint32_t)(((ci - c_begin) / NBUF) & 1));
-        if (tid == ISSUER) {
-            mma_commit(bar_drain);
-            (void)mbar_wait(bar_drain, 0);
+            for (int j = 0; j < NH; j += 4) *reinterpret_cast<float4*>(st + j) = make_float4(S[j], S[j + 1], S[j + 2], S[j + 3]);
         }
     }
+    if (!ok && (tid == 0 || tid == 256)) flag_status(p.d_status, GDR_DEVICE_TIMEOUT);
     tc_fence_before();
     __syncthreads();
     if (warp == 0) tmem_dealloc(tmem, GS_TM_COLS);
-#undef GDR_WAIT_SOLO
-#undef GDR_SYNC_CHECK
 }
 
 }  // namespace twopass_g
@@ -1075,7 +1098,7 @@ cudaError_t launch_chunk_twopass_general(const CUtensorMap* maps, MapFn make_map
         auto go = [&](auto kern, uint32_t bytes) -> cudaError_t {
             cudaError_t e2 = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, bytes);
             if (e2 != cudaSuccess) return e2;
-            kern<<<sgrid, NT, bytes, st>>>(sm_maps[0], sm_maps[1], sm_maps[2], sm_maps[3], sm_maps[4],
+            kern<<<sgrid, GS_NT, bytes, st>>>(sm_maps[0], sm_maps[1], sm_maps[2], sm_maps[3], sm_maps[4],
                                            sm_maps[5], sm_maps[6], sm_maps[7], sr);
             return cudaGetLastError();
         };

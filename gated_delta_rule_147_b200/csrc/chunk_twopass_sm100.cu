@@ -377,39 +377,51 @@ constexpr uint32_t S_SMEM_BYTES = S_OFF_SMALL + 3072 + 1024;
 // two column sets by chunk parity, so chunk ci's outputs are written while
 // chunk ci + 1 runs; D1 = [Q ; -W] K^T (lanes 0..63: Q K^T); D4 = K^T U'.
 constexpr uint32_t S_TM_D3 = 0, S_TM_D1 = 128, S_TM_D4 = 192, S_TM_D5 = 256, S_TM_COLS = 512;
-// Named barriers (0 is __syncthreads): U ready for K^T U (warps 2, 3, 6, 7);
-// U and Aq ready for Aq U (warps 2, 3, 6, 7 arrive, warps 0, 1, 4, 5 wait).
-constexpr int S_BAR_U = 1, S_BAR_AQ = 2;
+// Threads: warps 0..7 compute (thread t < 256: state row t & 127, columns
+// 32 (t >> 7) .. + 31 of the CTA's 64); warp 8 issues every MMA and TMA load.
+constexpr int S_NT = 288;
+constexpr int S_BAR_CHUNK = 1;  // named barrier over the 256 compute threads
 
-__device__ __forceinline__ void named_bar_sync(int id, int n) {
-    asm volatile("bar.sync %0, %1;" ::"r"(id), "r"(n) : "memory");
+__device__ __forceinline__ bool named_bar_and(int id, int n, bool pred) {
+    uint32_t r;
+    asm volatile(
+        "{\n\t.reg .pred p, q;\n\t"
+        "setp.ne.u32 p, %1, 0;\n\t"
+        "barrier.red.and.pred q, %2, %3, p;\n\t"
+        "selp.u32 %0, 1, 0, q;\n\t}"
+        : "=r"(r)
+        : "r"((uint32_t)pred), "r"(id), "r"(n)
+        : "memory");
+    return r != 0;
 }
-__device__ __forceinline__ void named_bar_arrive(int id, int n) {
-    asm volatile("bar.arrive %0, %1;" ::"r"(id), "r"(n) : "memory");
+
+__device__ __forceinline__ void mbar_arrive(uint64_t* bar) {
+    asm volatile("mbarrier.arrive.shared::cta.b64 _, [%0];" ::"r"(smem_u32(bar)) : "memory");
 }
 
 // Chunk step of the state pass. Only the two products that depend on the
 // state are on the chain from one chunk to the next:
-//   D3 = [Q ; -W] S           (then U = P - W S, rows 64..127 of D3, by warps 2, 3, 6, 7)
-//   D4 = K^T Diag(g_{n-1}/g) U  (then S <- g_{n-1} S + D4, all warps)
-// The output's products run beside them on their own barriers:
-//   D1 = [Q ; -W] K^T          (queued right after D3; Aq = masked
-//                               (Q K^T) . 2^(l_r - l_j) by warps 0, 1, 4, 5
-//                               while warps 2, 3, 6, 7 form U)
-//   D5 = [Aq ; .] U            (queued after D4; read with Q S for O of this
-//                               chunk during the next chunk's first product)
-// Decay ratios are formed per element from the log2 prefix l (exact for any
-// alpha in (0, 1]: every factor used is at most 1).
-__global__ void __launch_bounds__(NT, 1) state_gdn_kernel(
+//   D3 = [Q ; -W] S             (U = P - W S, lanes 64..127, by warps 2, 3, 6, 7)
+//   D4 = K^T Diag(g_{n-1}/g) U  (S <- g_{n-1} S + D4, all compute warps)
+// The output's products are queued between them and after them:
+//   D1 = [Q ; -W] K^T           (Aq = masked (Q K^T) . 2^(l_r - l_j), lanes 0..63,
+//                                by warps 0, 1, 4, 5 while warps 2, 3, 6, 7 form U)
+//   D5 = [Aq ; U] U             (lanes 0..63: Aq U; with Q S it gives O of the
+//                                chunk, written during the next chunk)
+// Warp 8 issues them in that order, each when its operands are in shared
+// memory (mbarriers u_ready, aq_ready, s_ready), so no compute warp waits on
+// MMA issue. Decay ratios are formed per element from the log2 prefix l
+// (exact for any alpha in (0, 1]: every factor used is at most 1).
+__global__ void __launch_bounds__(S_NT, 1) state_gdn_kernel(
     const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ CUtensorMap tm_k,
     const __grid_constant__ CUtensorMap tm_w, const __grid_constant__ CUtensorMap tm_p,
     const Params p) {
     extern __shared__ uint8_t smem_raw[];
     uint8_t* sm = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) &
                                              ~uintptr_t(1023));
-    const int tid = threadIdx.x, warp = tid >> 5;
-    const int wg = warp >> 2;
-    const int row = tid & 127;             // TMEM lane / state row
+    const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
+    const int wg = (warp >> 2) & 1;
+    const int row = tid & 127;             // TMEM lane / state row (compute threads)
     const bool lo = row < 64;              // warps 0, 1, 4, 5: lanes 0..63
     const int vt = blockIdx.x, h = blockIdx.y, bb = blockIdx.z;
     const int hq = h / p.group;  // q / k head of this value head
@@ -424,12 +436,15 @@ __global__ void __launch_bounds__(NT, 1) state_gdn_kernel(
     float* s_g3 = s_l3 + 192;                                    // [3][64]
     float* s_gcr3 = s_l3 + 384;                                  // [3][64]
     float* s_gC3 = s_l3 + 576;                                   // [3][4]
-    uint64_t* bar_tma = reinterpret_cast<uint64_t*>(sm + S_OFF_SMALL + 2816);  // [3]
-    uint64_t* bar_w = bar_tma + 3;
+    uint64_t* bar_tma = reinterpret_cast<uint64_t*>(sm + S_OFF_SMALL + 2752);  // [3]
+    uint64_t* bar_w = bar_tma + 3;      // MMA commits
     uint64_t* bar_q = bar_tma + 4;
     uint64_t* bar_k = bar_tma + 5;
     uint64_t* bar_a = bar_tma + 6;
-    uint64_t* bar_drain = bar_tma + 7;  // timeout path: both MMA issuers' work has finished
+    uint64_t* bar_drain = bar_tma + 7;
+    uint64_t* u_ready = bar_tma + 8;    // operands written (compute -> issuer)
+    uint64_t* aq_ready = bar_tma + 9;
+    uint64_t* s_ready = bar_tma + 10;
     uint32_t* s_tmem = reinterpret_cast<uint32_t*>(sm + S_OFF_SMALL + 2880);
     if (tid == 0) {
         for (int i = 0; i < 3; ++i) mbar_init(&bar_tma[i], 1);
@@ -437,7 +452,10 @@ __global__ void __launch_bounds__(NT, 1) state_gdn_kernel(
         mbar_init(bar_q, 1);
         mbar_init(bar_k, 1);
         mbar_init(bar_a, 1);
-        mbar_init(bar_drain, 2);
+        mbar_init(bar_drain, 1);
+        mbar_init(u_ready, 128);
+        mbar_init(aq_ready, 128);
+        mbar_init(s_ready, 1);
         fence_barrier_init();
         prefetch_tmap(&tm_q);
         prefetch_tmap(&tm_k);
@@ -452,25 +470,10 @@ __global__ void __launch_bounds__(NT, 1) state_gdn_kernel(
     const uint32_t lane_base = (uint32_t)((warp & 3) * 32) << 16;
     const uint32_t sbase = smem_u32(sm);
     bool ok = true;
-    int loads_issued = 0;  // chunks whose inputs were requested (tid 0 / 32 bookkeeping)
-
-    auto issue_loads = [&](int ci) {
-        const int t0 = ci * C, buf = ci % S_NBUF;
-        uint8_t* st = sm + buf * S_STAGE;
-        mbar_expect_tx(&bar_tma[buf], 7u * 8192u);
-        // [Q ; -W]: each 64-column block holds 128 rows (q rows 0..63, -W rows 64..127)
-        tma_load_4d(st + S_ST_QW, &tm_q, &bar_tma[buf], 0, hq, t0, bb);
-        tma_load_4d(st + S_ST_QW + 16384, &tm_q, &bar_tma[buf], 64, hq, t0, bb);
-        tma_load_4d(st + S_ST_QW + 8192, &tm_w, &bar_tma[buf], 0, h, t0, bb);
-        tma_load_4d(st + S_ST_QW + 16384 + 8192, &tm_w, &bar_tma[buf], 64, h, t0, bb);
-        tma_load_4d(st + S_ST_K, &tm_k, &bar_tma[buf], 0, hq, t0, bb);
-        tma_load_4d(st + S_ST_K + 8192, &tm_k, &bar_tma[buf], 64, hq, t0, bb);
-        tma_load_4d(st + S_ST_P, &tm_p, &bar_tma[buf], v0, h, t0, bb);
-    };
 
     constexpr int NH = NV / 2;
     float S[NH];
-    {
+    if (warp < 8) {
         const float* s0 = p.S0 ? p.S0 + (((size_t)bb * H + h) * DK + row) * p.dv + v0 + wg * NH : nullptr;
 #pragma unroll
         for (int j = 0; j < NH; j += 4) {
@@ -481,9 +484,8 @@ __global__ void __launch_bounds__(NT, 1) state_gdn_kernel(
         for (int ch = 0; ch < 4; ++ch) st_chunk(sm + S_OFF_SBF, sw128_chunk(row, wg * 4 + ch, DK), &S[8 * ch]);
     }
 
-    // decay scan of one chunk by warp 1 (two tokens per lane, log2 alpha in
+    // decay scan of one chunk by warp 1 (two tokens per lane, alpha in
     // registers): factors set ci % 3
-    const int lane = tid & 31;
     auto bits_to_f32 = [](unsigned short u) { return __uint_as_float((uint32_t)u << 16); };
     unsigned short a_nx0 = 0x3F80, a_nx1 = 0x3F80;  // alpha of the next chunk to scan (bf16 1.0)
     auto load_alpha = [&](int ci) {
@@ -516,6 +518,20 @@ __global__ void __launch_bounds__(NT, 1) state_gdn_kernel(
         if (lane == 0) s_gC3[s3 * 4] = ex2_approx(last);
     };
 
+    auto issue_loads = [&](int ci) {
+        const int t0 = ci * C, buf = ci % S_NBUF;
+        uint8_t* st = sm + buf * S_STAGE;
+        mbar_expect_tx(&bar_tma[buf], 7u * 8192u);
+        // [Q ; -W]: each 64-column block holds 128 rows (q rows 0..63, -W rows 64..127)
+        tma_load_4d(st + S_ST_QW, &tm_q, &bar_tma[buf], 0, hq, t0, bb);
+        tma_load_4d(st + S_ST_QW + 16384, &tm_q, &bar_tma[buf], 64, hq, t0, bb);
+        tma_load_4d(st + S_ST_QW + 8192, &tm_w, &bar_tma[buf], 0, h, t0, bb);
+        tma_load_4d(st + S_ST_QW + 16384 + 8192, &tm_w, &bar_tma[buf], 64, h, t0, bb);
+        tma_load_4d(st + S_ST_K, &tm_k, &bar_tma[buf], 0, hq, t0, bb);
+        tma_load_4d(st + S_ST_K + 8192, &tm_k, &bar_tma[buf], 64, hq, t0, bb);
+        tma_load_4d(st + S_ST_P, &tm_p, &bar_tma[buf], v0, h, t0, bb);
+    };
+
     // the state's bf16 copy is read by the first MMA (async proxy)
     fence_proxy_async();
     tc_fence_before();
@@ -523,10 +539,9 @@ __global__ void __launch_bounds__(NT, 1) state_gdn_kernel(
     // launched before that one completes: programmatic dependent launch);
     // the first pass's factors are read only after it has completed.
     asm volatile("griddepcontrol.wait;" ::: "memory");
-    if (tid == 32) {
+    if (warp == 8 && lane == 0) {
         for (int ci = 0; ci < 2 && ci < nchunks; ++ci) issue_loads(ci);
     }
-    loads_issued = min(2, nchunks);
     if (warp == 1 && nchunks > 0) {
         load_alpha(0);
         decay_scan(0);
@@ -534,127 +549,65 @@ __global__ void __launch_bounds__(NT, 1) state_gdn_kernel(
     }
     __syncthreads();
 
-    bool w_ok = true;
-    uint32_t ph_tma = 0u;  // bit i: phase parity of stage i
-#define GDR_WAIT_SOLO(bar, ph)              \
-    do {                                    \
-        w_ok = mbar_wait(bar, ph) && w_ok;  \
-    } while (0)
-#define GDR_SYNC_CHECK()                                            \
-    do {                                                            \
-        if (!__syncthreads_and(w_ok)) { ok = false; goto finish; }  \
-    } while (0)
-
-    // O rows of chunk cj (lanes 0..63 of D3 and D5 in the column set of cj) -> global
-    auto store_o = [&](int cj) {
-        const int pj = cj & 1;
-        const int t = cj * C + row;
-        float d[32], d5[32];
-        tmem_ld32_async(tmem + lane_base + S_TM_D3 + pj * 64 + wg * 32, d);
-        tmem_ld32_async(tmem + lane_base + S_TM_D5 + pj * 64 + wg * 32, d5);
-        tmem_wait_ld();
-        if (t < T) {
-            const float gr = s_g3[(cj % 3) * 64 + row];
-            __nv_bfloat16* op = p.o + (((size_t)bb * T + t) * H + h) * p.dv + v0 + wg * 32;
-#pragma unroll
-            for (int c8 = 0; c8 < 4; ++c8) {
-                float y[8];
-#pragma unroll
-                for (int e = 0; e < 8; ++e) y[e] = fmaf(gr, d[c8 * 8 + e], d5[c8 * 8 + e]);
-                uint4 u;
-                u.x = pack_bf16x2(y[0], y[1]);
-                u.y = pack_bf16x2(y[2], y[3]);
-                u.z = pack_bf16x2(y[4], y[5]);
-                u.w = pack_bf16x2(y[6], y[7]);
-                *reinterpret_cast<uint4*>(op + c8 * 8) = u;
-            }
-        }
-    };
-
-    for (int ci = 0; ci < nchunks; ++ci) {
-        const int buf = ci % S_NBUF;
-        const int par = ci & 1;
-        const uint32_t ph = (uint32_t)(ci & 1);
-        const uint32_t stb = sbase + buf * S_STAGE;
-        const uint32_t qwb = stb + S_ST_QW, kb = stb + S_ST_K;
-        const int s3 = ci % 3;
-        GDR_TRACE_S(0, 0);
-        GDR_WAIT_SOLO(&bar_tma[buf], (ph_tma >> buf) & 1u);
-        ph_tma ^= 1u << buf;
-        GDR_TRACE_S(1, 0);
-
-        // ---- D3 = [Q ; -W] S, then D1 = [Q ; -W] K^T ----------------------------
-        if (tid == 0) {
+    int loads_issued = min(2, nchunks);  // issuer's bookkeeping
+    if (warp == 8) {
+        // ---------------- issuer warp: MMAs in chain order, TMA two chunks ahead --------
+        bool iok = true;
+        for (int ci = 0; ci < nchunks && iok; ++ci) {
+            const int buf = ci % S_NBUF;
+            const int par = ci & 1;
+            const uint32_t ph = (uint32_t)(ci & 1);
+            const uint32_t stb = sbase + buf * S_STAGE;
+            const uint32_t qwb = stb + S_ST_QW, kb = stb + S_ST_K;
+            // inputs landed, and (after the first chunk) the state copy is written
+            iok = mbar_wait(&bar_tma[buf], (uint32_t)((ci / S_NBUF) & 1)) && iok;
+            if (ci > 0) iok = mbar_wait(s_ready, (uint32_t)((ci - 1) & 1)) && iok;
+            iok = __all_sync(0xffffffffu, iok);
+            if (!iok) break;
+            GDR_TRACE_S(0, 256);
             tc_fence_after();
-            const uint32_t idS = idesc_bf16(128, NV, 0, 1);
-            const uint32_t idK = idesc_bf16(128, 64, 0, 0);
-            const uint32_t d3 = S_TM_D3 + (uint32_t)par * 64u;
+            if (lane == 0) {
+                const uint32_t idS = idesc_bf16(128, NV, 0, 1);
+                const uint32_t idK = idesc_bf16(128, 64, 0, 0);
+                const uint32_t d3 = S_TM_D3 + (uint32_t)par * 64u;
+                // D3 and D1 k-step by k-step: two independent accumulators in flight
 #pragma unroll
-            for (int ks = 0; ks < 8; ++ks) {
-                const uint32_t koff = (ks >> 2) * 16384u + (ks & 3) * 32u;
-                mma_bf16(tmem + d3, sdesc_sw128(qwb + koff, 16, 1024),
-                         sdesc_sw128(sbase + S_OFF_SBF + ks * 2048u, 8192, 1024), idS, ks > 0);
-            }
-            mma_commit(bar_w);
-#pragma unroll
-            for (int ks = 0; ks < 8; ++ks) {
-                const uint32_t koff = (ks >> 2) * 16384u + (ks & 3) * 32u;
-                const uint32_t kkoff = (ks >> 2) * 8192u + (ks & 3) * 32u;
-                mma_bf16(tmem + S_TM_D1, sdesc_sw128(qwb + koff, 16, 1024),
-                         sdesc_sw128(kb + kkoff, 16, 1024), idK, ks > 0);
-            }
-            mma_commit(bar_q);
-        }
-        // chunk ci + 2's inputs go to the buffers chunk ci - 1 has released
-        if (tid == 32 && ci + 2 < nchunks) issue_loads(ci + 2);
-        if (ci + 2 < nchunks) loads_issued = ci + 3;
-
-        if (lo) {
-            // ---- warps 0, 1, 4, 5: O of the previous chunk, the next decay scan, Aq ----
-            if (ci > 0) {
-                GDR_WAIT_SOLO(bar_a, (uint32_t)((ci - 1) & 1));
-                tc_fence_after();
-                store_o(ci - 1);
-            }
-            GDR_TRACE_S(2, 0);
-            if (warp == 1 && ci + 1 < nchunks) {
-                decay_scan(ci + 1);
-                if (ci + 2 < nchunks) load_alpha(ci + 2);
-            }
-            GDR_WAIT_SOLO(bar_q, ph);
-            tc_fence_after();
-            GDR_TRACE_S(3, 0);
-            {
-                const int r = row;
-                float d[32];
-                tmem_ld32(tmem + lane_base + S_TM_D1 + wg * 32, d);
-                const float* l = s_l3 + s3 * 64;
-                const float lr = l[r];
-#pragma unroll
-                for (int c8 = 0; c8 < 4; ++c8) {
-                    const int j0 = wg * 32 + c8 * 8;
-                    float x[8];
-                    if (j0 > r) {
-#pragma unroll
-                        for (int e = 0; e < 8; ++e) x[e] = 0.f;
-                    } else {
-                        const float4 la = *reinterpret_cast<const float4*>(l + j0);
-                        const float4 lb = *reinterpret_cast<const float4*>(l + j0 + 4);
-                        const float lj[8] = {la.x, la.y, la.z, la.w, lb.x, lb.y, lb.z, lb.w};
-#pragma unroll
-                        for (int e = 0; e < 8; ++e)
-                            x[e] = j0 + e <= r ? d[c8 * 8 + e] * ex2_approx(lr - lj[e]) : 0.f;
-                    }
-                    st_chunk(sm + S_OFF_AQ, sw128_chunk(r, wg * 4 + c8, 128), x);
+                for (int ks = 0; ks < 8; ++ks) {
+                    const uint32_t koff = (ks >> 2) * 16384u + (ks & 3) * 32u;
+                    const uint32_t kkoff = (ks >> 2) * 8192u + (ks & 3) * 32u;
+                    mma_bf16(tmem + d3, sdesc_sw128(qwb + koff, 16, 1024),
+                             sdesc_sw128(sbase + S_OFF_SBF + ks * 2048u, 8192, 1024), idS, ks > 0);
+                    if (ks == 7) mma_commit(bar_w);
+                    mma_bf16(tmem + S_TM_D1, sdesc_sw128(qwb + koff, 16, 1024),
+                             sdesc_sw128(kb + kkoff, 16, 1024), idK, ks > 0);
                 }
+                mma_commit(bar_q);
+                // chunk ci + 2's inputs go to the stage of chunk ci - 1, all of whose
+                // readers finished before the state copy of chunk ci was written
+                if (ci + 2 < nchunks) issue_loads(ci + 2);
             }
-            fence_proxy_async();
-            tc_fence_before();
-            named_bar_sync(S_BAR_AQ, NT);  // U (warps 2, 3, 6, 7) and Aq ready
-            GDR_TRACE_S(4, 0);
-            if (tid == 0) {
-                // ---- D5 = [Aq ; U] U (lanes 0..63: Aq U) ----------------------------------
-                tc_fence_after();
+            if (ci + 2 < nchunks) loads_issued = ci + 3;
+            __syncwarp();
+            // ---- D4 = K^T U' once U is written --------------------------------------
+            iok = __all_sync(0xffffffffu, mbar_wait(u_ready, ph) && iok);
+            if (!iok) break;
+            GDR_TRACE_S(1, 256);
+            tc_fence_after();
+            if (lane == 0) {
+                const uint32_t idM = idesc_bf16(128, NV, 1, 1);
+#pragma unroll
+                for (int ks = 0; ks < 4; ++ks)
+                    mma_bf16(tmem + S_TM_D4, sdesc_sw128(kb + ks * 2048u, 8192, 1024),
+                             sdesc_sw128(sbase + S_OFF_U2 + ks * 2048u, 8192, 1024), idM, ks > 0);
+                mma_commit(bar_k);
+            }
+            __syncwarp();
+            // ---- D5 = [Aq ; U] U once Aq is written ---------------------------------
+            iok = __all_sync(0xffffffffu, mbar_wait(aq_ready, ph) && iok);
+            if (!iok) break;
+            GDR_TRACE_S(2, 256);
+            tc_fence_after();
+            if (lane == 0) {
                 const uint32_t idA = idesc_bf16(128, NV, 0, 1);
                 const uint32_t d5 = S_TM_D5 + (uint32_t)par * 64u;
 #pragma unroll
@@ -663,95 +616,156 @@ __global__ void __launch_bounds__(NT, 1) state_gdn_kernel(
                              sdesc_sw128(sbase + S_OFF_U + ks * 2048u, 8192, 1024), idA, ks > 0);
                 mma_commit(bar_a);
             }
-        } else {
-            // ---- warps 2, 3, 6, 7: U = P - W S (lanes 64..127 of D3) -> U and U' ------
-            GDR_WAIT_SOLO(bar_w, ph);
-            tc_fence_after();
-            GDR_TRACE_S(7, 64);
-            {
-                const int j = row - 64;  // token
-                float d[32];
-                tmem_ld32(tmem + lane_base + S_TM_D3 + (uint32_t)par * 64u + wg * 32, d);
-                const float f = s_gcr3[s3 * 64 + j];
+            __syncwarp();
+        }
+        if (!iok) {
+            ok = false;
+            if (lane == 0) {
+                // before the block leaves (each wait bounded): the requested input
+                // copies have landed and the issued MMAs have finished
+                for (int ci = max(0, loads_issued - S_NBUF); ci < loads_issued; ++ci)
+                    (void)mbar_wait(&bar_tma[ci % S_NBUF], (uint32_t)((ci / S_NBUF) & 1));
+                mma_commit(bar_drain);
+                (void)mbar_wait(bar_drain, 0);
+            }
+            __syncwarp();
+        }
+    } else {
+        // ---------------- compute warps ----------------------------------------------
+        bool w_ok = true;
+        // O rows of chunk cj (lanes 0..63 of D3 and D5 in the column set of cj) -> global
+        auto store_o = [&](int cj) {
+            const int pj = cj & 1;
+            const int t = cj * C + row;
+            float d[32], d5[32];
+            tmem_ld32_async(tmem + lane_base + S_TM_D3 + pj * 64 + wg * 32, d);
+            tmem_ld32_async(tmem + lane_base + S_TM_D5 + pj * 64 + wg * 32, d5);
+            tmem_wait_ld();
+            if (t < T) {
+                const float gr = s_g3[(cj % 3) * 64 + row];
+                __nv_bfloat16* op = p.o + (((size_t)bb * T + t) * H + h) * p.dv + v0 + wg * 32;
 #pragma unroll
                 for (int c8 = 0; c8 < 4; ++c8) {
-                    float x[8];
-                    const uint32_t off = sw128_chunk(j, wg * 4 + c8, 64);
-                    ld_chunk(sm + buf * S_STAGE + S_ST_P, off, x);
+                    float y[8];
 #pragma unroll
-                    for (int e = 0; e < 8; ++e) x[e] += d[c8 * 8 + e];
-                    st_chunk(sm + S_OFF_U, off, x);
-#pragma unroll
-                    for (int e = 0; e < 8; ++e) x[e] *= f;
-                    st_chunk(sm + S_OFF_U2, off, x);
+                    for (int e = 0; e < 8; ++e) y[e] = fmaf(gr, d[c8 * 8 + e], d5[c8 * 8 + e]);
+                    uint4 u;
+                    u.x = pack_bf16x2(y[0], y[1]);
+                    u.y = pack_bf16x2(y[2], y[3]);
+                    u.z = pack_bf16x2(y[4], y[5]);
+                    u.w = pack_bf16x2(y[6], y[7]);
+                    *reinterpret_cast<uint4*>(op + c8 * 8) = u;
                 }
             }
-            fence_proxy_async();
-            tc_fence_before();
-            named_bar_sync(S_BAR_U, 128);
-            if (tid == 64) {
-                // ---- D4 = K^T U' (state increment) ---------------------------------------
+        };
+        int ci = 0;
+        for (; ci < nchunks; ++ci) {
+            const int buf = ci % S_NBUF;
+            const int par = ci & 1;
+            const uint32_t ph = (uint32_t)(ci & 1);
+            const int s3 = ci % 3;
+            if (lo) {
+                // ---- O of the previous chunk, the next decay scan, Aq -----------------------
+                if (ci > 0) {
+                    w_ok = mbar_wait(bar_a, (uint32_t)((ci - 1) & 1)) && w_ok;
+                    tc_fence_after();
+                    store_o(ci - 1);
+                }
+                if (warp == 1 && ci + 1 < nchunks) {
+                    decay_scan(ci + 1);
+                    if (ci + 2 < nchunks) load_alpha(ci + 2);
+                }
+                w_ok = mbar_wait(bar_q, ph) && w_ok;
                 tc_fence_after();
-                const uint32_t idM = idesc_bf16(128, NV, 1, 1);
+                GDR_TRACE_S(3, 0);
+                {
+                    const int r = row;
+                    float d[32];
+                    tmem_ld32(tmem + lane_base + S_TM_D1 + wg * 32, d);
+                    const float* l = s_l3 + s3 * 64;
+                    const float lr = l[r];
 #pragma unroll
-                for (int ks = 0; ks < 4; ++ks)
-                    mma_bf16(tmem + S_TM_D4, sdesc_sw128(kb + ks * 2048u, 8192, 1024),
-                             sdesc_sw128(sbase + S_OFF_U2 + ks * 2048u, 8192, 1024), idM, ks > 0);
-                mma_commit(bar_k);
+                    for (int c8 = 0; c8 < 4; ++c8) {
+                        const int j0 = wg * 32 + c8 * 8;
+                        float x[8];
+                        const float4 la = *reinterpret_cast<const float4*>(l + j0);
+                        const float4 lb = *reinterpret_cast<const float4*>(l + j0 + 4);
+                        const float lj[8] = {la.x, la.y, la.z, la.w, lb.x, lb.y, lb.z, lb.w};
+#pragma unroll
+                        for (int e = 0; e < 8; ++e)
+                            x[e] = j0 + e <= r ? d[c8 * 8 + e] * ex2_approx(fminf(lr - lj[e], 0.f)) : 0.f;
+                        st_chunk(sm + S_OFF_AQ, sw128_chunk(r, wg * 4 + c8, 128), x);
+                    }
+                }
+                fence_proxy_async();
+                tc_fence_before();
+                mbar_arrive(aq_ready);
+                GDR_TRACE_S(4, 0);
+            } else {
+                // ---- U = P - W S (lanes 64..127 of D3) -> U and U' -------------------------
+                w_ok = mbar_wait(&bar_tma[buf], (uint32_t)((ci / S_NBUF) & 1)) && w_ok;  // P landed
+                w_ok = mbar_wait(bar_w, ph) && w_ok;
+                tc_fence_after();
+                GDR_TRACE_S(7, 64);
+                {
+                    const int j = row - 64;  // token
+                    float d[32];
+                    tmem_ld32(tmem + lane_base + S_TM_D3 + (uint32_t)par * 64u + wg * 32, d);
+                    const float f = s_gcr3[s3 * 64 + j];
+#pragma unroll
+                    for (int c8 = 0; c8 < 4; ++c8) {
+                        float x[8];
+                        const uint32_t off = sw128_chunk(j, wg * 4 + c8, 64);
+                        ld_chunk(sm + buf * S_STAGE + S_ST_P, off, x);
+#pragma unroll
+                        for (int e = 0; e < 8; ++e) x[e] += d[c8 * 8 + e];
+                        st_chunk(sm + S_OFF_U, off, x);
+#pragma unroll
+                        for (int e = 0; e < 8; ++e) x[e] *= f;
+                        st_chunk(sm + S_OFF_U2, off, x);
+                    }
+                }
+                fence_proxy_async();
+                tc_fence_before();
+                mbar_arrive(u_ready);
             }
-            named_bar_arrive(S_BAR_AQ, NT);
+            // ---- S = g_{n-1} S + D4 (every compute warp: its lanes, half the columns) ----
+            w_ok = mbar_wait(bar_k, ph) && w_ok;
+            tc_fence_after();
+            GDR_TRACE_S(5, 0);
+            {
+                float dS[32];
+                tmem_ld32(tmem + lane_base + S_TM_D4 + wg * 32, dS);
+                const float gC = s_gC3[s3 * 4];
+#pragma unroll
+                for (int jj = 0; jj < NH; ++jj) S[jj] = fmaf(gC, S[jj], dS[jj]);
+#pragma unroll
+                for (int ch = 0; ch < 4; ++ch) st_chunk(sm + S_OFF_SBF, sw128_chunk(row, wg * 4 + ch, DK), &S[8 * ch]);
+            }
+            fence_proxy_async();  // the state copy feeds the next chunk's MMAs
+            tc_fence_before();
+            if (!named_bar_and(S_BAR_CHUNK, 256, w_ok)) break;
+            GDR_TRACE_S(6, 0);
+            if (tid == 0) mbar_arrive(s_ready);
         }
-
-        // ---- S = g_{n-1} S + D4 (every warp: its lanes, half the columns) -----------
-        GDR_WAIT_SOLO(bar_k, ph);
-        tc_fence_after();
-        GDR_TRACE_S(5, 0);
-        {
-            float dS[32];
-            tmem_ld32(tmem + lane_base + S_TM_D4 + wg * 32, dS);
-            const float gC = s_gC3[s3 * 4];
-#pragma unroll
-            for (int jj = 0; jj < NH; ++jj) S[jj] = fmaf(gC, S[jj], dS[jj]);
-#pragma unroll
-            for (int ch = 0; ch < 4; ++ch) st_chunk(sm + S_OFF_SBF, sw128_chunk(row, wg * 4 + ch, DK), &S[8 * ch]);
+        if (ci < nchunks) ok = false;  // a wait gave up
+        if (ok && lo && nchunks > 0) {
+            ok = mbar_wait(bar_a, (uint32_t)((nchunks - 1) & 1));
+            tc_fence_after();
+            if (ok) store_o(nchunks - 1);
         }
-        fence_proxy_async();  // the state copy feeds the next chunk's MMAs
-        tc_fence_before();
-        GDR_SYNC_CHECK();
-        GDR_TRACE_S(6, 0);
-    }
-    if (lo && nchunks > 0) {
-        GDR_WAIT_SOLO(bar_a, (uint32_t)((nchunks - 1) & 1));
-        tc_fence_after();
-        store_o(nchunks - 1);
-    }
-    if (!__syncthreads_and(w_ok)) ok = false;
-
-    if (ok && p.ST) {
-        float* st = p.ST + (((size_t)bb * H + h) * DK + row) * p.dv + v0 + wg * NH;
+        if (!named_bar_and(S_BAR_CHUNK, 256, ok)) ok = false;
+        if (ok && p.ST) {
+            float* st = p.ST + (((size_t)bb * H + h) * DK + row) * p.dv + v0 + wg * NH;
 #pragma unroll
-        for (int jj = 0; jj < NH; jj += 4)
-            *reinterpret_cast<float4*>(st + jj) = make_float4(S[jj], S[jj + 1], S[jj + 2], S[jj + 3]);
-    }
-
-finish:
-    if (!ok) {
-        if (tid == 0) flag_status(p.d_status, GDR_DEVICE_TIMEOUT);
-        // before the block leaves (each wait bounded): the input copies it
-        // requested have landed and the MMAs of both issuing threads are done
-        if (tid == 32)
-            for (int ci = max(0, loads_issued - S_NBUF); ci < loads_issued; ++ci)
-                (void)mbar_wait(&bar_tma[ci % S_NBUF], (uint32_t)((ci / S_NBUF) & 1));
-        if (tid == 0 || tid == 64) {
-            mma_commit(bar_drain);
-            (void)mbar_wait(bar_drain, 0);
+            for (int jj = 0; jj < NH; jj += 4)
+                *reinterpret_cast<float4*>(st + jj) = make_float4(S[jj], S[jj + 1], S[jj + 2], S[jj + 3]);
         }
     }
+    if (!ok && (tid == 0 || tid == 256)) flag_status(p.d_status, GDR_DEVICE_TIMEOUT);
     tc_fence_before();
     __syncthreads();
     if (warp == 0) tmem_dealloc(tmem, S_TM_COLS);
-#undef GDR_WAIT_SOLO
-#undef GDR_SYNC_CHECK
 }
 
 }  // namespace twopass
@@ -793,7 +807,7 @@ cudaError_t launch_chunk_twopass_gdn(const CUtensorMap* maps, const CUtensorMap*
     if (e != cudaSuccess) return e;
     cudaLaunchConfig_t cfg = {};
     cfg.gridDim = dim3(dv / NV, H, B);
-    cfg.blockDim = dim3(NT, 1, 1);
+    cfg.blockDim = dim3(S_NT, 1, 1);
     cfg.dynamicSmemBytes = S_SMEM_BYTES;
     cfg.stream = st;
     cudaLaunchAttribute attr[1];
