@@ -122,14 +122,16 @@ def chunk_fwd(q, k, v, alpha=None, b=None, w=None, S0=None, *, out=None, final_s
 
 
 def chunk_bwd(q, k, v, alpha=None, b=None, w=None, S0=None, *, dO, dS_T=None, chunk: int = 64,
-              workspace=None, need_dS0: bool = True, stream=None):
+              workspace=None, need_dS0: bool = True, d_status=None, stream=None):
     """Backward of chunk_fwd for the same inputs: returns a dict with dq, dk,
     dv, dalpha, db, dw (None for an absent or tied gate) and dS0 (None when
     need_dS0 is False), all fp32. q and k may have fewer heads than v
     (grouped heads, as in chunk_fwd; dq and dk then sum over each group). dO has v's shape and dtype; dS_T is the
     gradient of the final state (None = 0). workspace: None allocates the
     chunk-checkpoint scratch with torch, or a uint8 device tensor of at least
-    gdr_chunk_bwd_grouped_workspace_size bytes."""
+    gdr_chunk_bwd_grouped_workspace_size bytes. d_status: optional int32
+    device tensor the bounded waits of the tensor-core kernel OR their
+    timeout flag into."""
     import torch
     _check(q, k, v, alpha, b, w, S0, dO, dS_T)
     _check_types(q, [("k", k), ("v", v), ("alpha", alpha), ("b", b), ("w", w), ("dO", dO)],
@@ -153,7 +155,7 @@ def chunk_bwd(q, k, v, alpha=None, b=None, w=None, S0=None, *, dO, dS_T=None, ch
                           _gate_kind(alpha, 3), _gate_kind(b, 3), _gate_kind(w, 3), S0, dO, dS_T,
                           grads["dq"], grads["dk"], grads["dv"], grads["dalpha"], grads["db"],
                           grads["dw"], grads["dS0"], workspace, ws_bytes, B, T, Hq, H, dk, dv, chunk,
-                          _dtype_code(q), None, stream)
+                          _dtype_code(q), d_status, stream)
     return grads
 
 

@@ -87,6 +87,16 @@ bool make_map(CUtensorMap* m, const void* base, int B, int T, int H, int d) {
     return r == CUDA_SUCCESS;
 }
 
+}  // namespace
+
+namespace gdr {
+bool make_tma_map_bf16(CUtensorMap* m, const void* base, int B, int T, int H, int d) {
+    return make_map(m, base, B, T, H, d);
+}
+}  // namespace gdr
+
+namespace {
+
 // Two-pass paths (per-chunk factors of all chunks in parallel, then the state
 // pass) exist for the tensor-core shape with an erase gate and d_v <= 128:
 // the Gated DeltaNet form (scalar decay, tied scalar beta) has its own pair of

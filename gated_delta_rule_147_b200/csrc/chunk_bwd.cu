@@ -34,6 +34,13 @@
 #include "common.cuh"
 
 namespace gdr {
+cudaError_t launch_bwd_chunk_tc(const CUtensorMap* maps, const float* ckS, const float* ckG,
+                                const float* R, const float* DR, const void* alpha,
+                                const void* beta, float* dq, float* dk, float* dalpha, float* db,
+                                int* d_status, int B, int T, int H, int group, int nchunks,
+                                cudaStream_t st);
+bool make_tma_map_bf16(CUtensorMap* m, const void* base, int B, int T, int H, int d);
+
 namespace bwd {
 
 constexpr int kC = 64;           // chunk: checkpoint interval of the scans
@@ -50,6 +57,7 @@ struct Params {
     const float *S0, *dST;
     float *dq, *dk, *dv, *dalpha, *db, *dw, *dS0;
     float *ckS, *ckG, *R, *DR, *GP;  // workspace
+    int* d_status;                   // bounded waits of the tensor-core pass 2
     float *dq_out, *dk_out;          // grouped heads: the caller's dq, dk (dq, dk are then workspace)
     int B, T, H, Hq, group, dk_, dv_, akind, bkind, wkind, nchunks, tpr, nrb;
 };
@@ -859,8 +867,10 @@ WsLayout ws_layout(int B, int T, int H, int dk, int dv, bool grouped) {
     return l;
 }
 
+// tc_maps (q, k, v, dO tensor maps) selects the tensor-core pass 2 of the
+// Gated DeltaNet form; it writes the scalar gate gradients itself.
 template <typename TI>
-cudaError_t launch_typed(Params p, cudaStream_t st) {
+cudaError_t launch_typed(Params p, const CUtensorMap* tc_maps, cudaStream_t st) {
     const dim3 sgrid((p.dv_ + kScanCols * kScanWarps - 1) / (kScanCols * kScanWarps), p.H, 2 * p.B);
     if ((p.dk_ * sizeof(TI)) % 16 == 0)
         bwd_scan_staged_kernel<TI><<<sgrid, kScanWarps * 32, 0, st>>>(p);
@@ -868,6 +878,17 @@ cudaError_t launch_typed(Params p, cudaStream_t st) {
         bwd_scan_kernel<TI><<<sgrid, kScanWarps * 32, 0, st>>>(p);
     cudaError_t e = cudaGetLastError();
     if (e != cudaSuccess) return e;
+    if (tc_maps) {
+        e = launch_bwd_chunk_tc(tc_maps, p.ckS, p.ckG, p.R, p.DR, p.alpha, p.b, p.dq, p.dk,
+                                p.dalpha, p.db, p.d_status, p.B, p.T, p.H, p.group, p.nchunks, st);
+        if (e != cudaSuccess) return e;
+        if (p.group > 1) {
+            const size_t n = (size_t)p.B * p.T * p.Hq * p.dk_;
+            bwd_group_sum_kernel<<<(unsigned)((n + 255) / 256), 256, 0, st>>>(p);
+            e = cudaGetLastError();
+        }
+        return e;
+    }
     const uint32_t smem = chunk_smem(p.tpr).total;
     void (*kern)(Params) = bwd_chunk_kernel<TI>;
     e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
@@ -921,7 +942,6 @@ gdr_status gdr_chunk_bwd_grouped(const void* q, const void* k, const void* v, co
                                  float* dw, float* dS0, void* workspace, size_t workspace_bytes,
                                  int B, int T, int H_qk, int H, int d_k, int d_v, int chunk,
                                  int dtype, int* d_status, void* stream) {
-    (void)d_status;  // this path has no bounded waits to report
     if (B < 1 || H < 1 || T < 0 || d_k < 1 || d_v < 1) return GDR_ERR_INVALID_ARG;
     if (H_qk < 1 || H % H_qk != 0) return GDR_ERR_INVALID_ARG;
     if (dtype != GDR_BF16 && dtype != GDR_FP32) return GDR_ERR_INVALID_ARG;
@@ -992,8 +1012,23 @@ gdr_status gdr_chunk_bwd_grouped(const void* q, const void* k, const void* v, co
     p.tpr = gdr::bwd::threads_per_row(d_v);
     const int RB = gdr::bwd::kChunkThreads / p.tpr;
     p.nrb = (d_k + RB - 1) / RB;
-    const cudaError_t e = dtype == GDR_BF16 ? gdr::bwd::launch_typed<__nv_bfloat16>(p, st)
-                                            : gdr::bwd::launch_typed<float>(p, st);
+    p.d_status = d_status;
+    // the Gated DeltaNet form on tensor cores: scalar decay, tied scalar beta,
+    // bf16, d_k = d_v = 128
+    CUtensorMap maps[4];
+    const CUtensorMap* tc_maps = nullptr;
+    if (dtype == GDR_BF16 && d_k == 128 && d_v == 128 && alpha_kind == GDR_GATE_SCALAR &&
+        b_kind == GDR_GATE_SCALAR && w_kind == GDR_GATE_TIED) {
+        if (!gdr::make_tma_map_bf16(&maps[0], q, B, T, H_qk, d_k) ||
+            !gdr::make_tma_map_bf16(&maps[1], k, B, T, H_qk, d_k) ||
+            !gdr::make_tma_map_bf16(&maps[2], v, B, T, H, d_v) ||
+            !gdr::make_tma_map_bf16(&maps[3], dO, B, T, H, d_v))
+            return GDR_ERR_NO_DEVICE;
+        tc_maps = maps;
+        p.GP = nullptr;
+    }
+    const cudaError_t e = dtype == GDR_BF16 ? gdr::bwd::launch_typed<__nv_bfloat16>(p, tc_maps, st)
+                                            : gdr::bwd::launch_typed<float>(p, nullptr, st);
     return e == cudaSuccess ? GDR_OK : GDR_ERR_LAUNCH;
 }
 

@@ -244,16 +244,24 @@ size_t gdr_chunk_fwd_static_capacity(void);
  * workspace: caller-owned device scratch of at least
  *   gdr_chunk_bwd_workspace_size() bytes, 256-byte aligned; contents on
  *   entry ignored, on exit undefined.
- * Method: fp32 arithmetic for both dtypes. The state gradient G follows its
- *   own backward recurrence G_{t-1} = Diag(alpha_t)(I - e^T k) G_t +
- *   q_{t-1}^T dO_{t-1}, which does not involve S, so a first kernel scans the
- *   tokens forward (S at every 64-token chunk start, r_t) and backward (G at
- *   every chunk end, dr_t = -k G, dv_t, dS0) at the same time, one warp per
- *   4 state columns; a second kernel, parallel over chunks, heads and blocks
- *   of state rows, rebuilds each chunk's states from those and forms dq, dk
- *   and the gate gradients; a third sums scalar gates' gradients over the
- *   key channels. Deterministic (no atomics). d_status is not used (no
- *   bounded waits on this path).
+ * Method: the state gradient G follows its own backward recurrence
+ *   G_{t-1} = Diag(alpha_t)(I - e^T k) G_t + q_{t-1}^T dO_{t-1}, which does
+ *   not involve S, so a first kernel scans the tokens forward (S at every
+ *   64-token chunk start, r_t) and backward (G at every
+ *   chunk end, dr_t = -k G, dv_t, dS0) at the same time in fp32, one warp
+ *   per 8 state columns. A second kernel, parallel over chunks and heads,
+ *   forms dq, dk and the gate gradients of each chunk from its start state,
+ *   end gradient, r and dr:
+ *   - the Gated DeltaNet form in bf16 with d_k = d_v = 128 (alpha and b
+ *     scalar, w tied): on tensor cores as masked, decay-scaled products
+ *     (bf16 operands: the fp32 checkpoints, r and dr are rounded to bf16;
+ *     fp32 accumulation), one CTA per (chunk, head) writing dalpha and db
+ *     directly; its bounded waits OR GDR_DEVICE_TIMEOUT into *d_status
+ *     (if not NULL) and end the kernel, leaving the outputs undefined;
+ *   - every other form and dtype: fp32 on CUDA cores, per block of state
+ *     rows, rebuilding the chunk's states elementwise; a third kernel then
+ *     sums scalar gates' gradients over the key channels; d_status unused.
+ *   Deterministic (no atomics) on both paths.
  * Supported: chunk = 64, 1 <= d_k <= 128, d_v a multiple of 8 up to 256,
  *   ceil(T / 64) <= 65535 and B * H <= 65535. Every pointer 16-byte
  *   aligned, except scalar gates and their gradients (element aligned).
