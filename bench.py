@@ -267,15 +267,19 @@ def time_chunk_e2e(inp, wl, dev, steps, warmup):
 
 # fp32 CUDA-core peak: 148 SMs x 128 FP32 lanes x 2 flop (FMA) x 1965 MHz
 ALU_FP32_TFLOPS = 148 * 128 * 2 * 1965e6 / 1e12
-# reverse-mode step per state element and token: forward step (decay, erase
-# read, erase, write: 4 multiply-adds) + reverse step (dq, G += q^T dO, dv, dr,
-# du, dk, de, dS', dalpha: 9 multiply-adds), 2 flop each
-BWD_FLOPS_PER_ELEMENT = 2 * 13
+# the scans of the backward, per state element and token: forward (decay,
+# erase read, erase + write: 4 multiply-adds) and backward (G += q^T dO, k G,
+# u G, G <- alpha (G - e^T (k G)): 5 multiply-adds), 2 flop each
+BWD_SCAN_FLOPS_PER_ELEMENT = 2 * 9
+# tensor-core products of the chunk kernel per (chunk, head), d = 128, C = 64:
+# [dO;DR][S0|V|R]^T (128x256x128), [Q;U]K^T (128x64x128), P[U;K], P^T[Q;E],
+# [V';-R']G_e^T (128x128x128 each)
+BWD_TC_FLOPS_PER_CHUNK = 2 * 128 * (256 * 128 + 64 * 128 + 3 * 128 * 128)
 
 
 def time_backward(dev, steps, warmup, pk):
     """The backward pass (gdr_chunk_bwd) on the Gated DeltaNet workload: CUDA
-    events per call, both launches."""
+    events per call (the fp32 scans, then the tensor-core chunk kernel)."""
     import torch
     from gated_delta_rule_147_b200 import TIED, chunk_bwd, gdr_chunk_bwd_workspace_size
     from gated_delta_rule_147_b200.inputs import WORKLOADS, make_cotangents
@@ -305,17 +309,23 @@ def time_backward(dev, steps, warmup, pk):
     state = wl.B * wl.H * wl.dk * wl.dv * 4
     # read q, k, v, dO (bf16), alpha, beta (bf16), dS_T; write dq, dk, dv (fp32), dalpha, dbeta, dS0
     bytes_ = th * (2 * (2 * wl.dk + 2 * wl.dv) + 2 * 2 + 4 * (2 * wl.dk + wl.dv) + 2 * 4) + 2 * state
-    flops = BWD_FLOPS_PER_ELEMENT * wl.dk * wl.dv * th
-    achieved = flops / (ms * 1e-3) / 1e12
+    scan_flops = BWD_SCAN_FLOPS_PER_ELEMENT * wl.dk * wl.dv * th
+    tc_flops = BWD_TC_FLOPS_PER_CHUNK * wl.B * wl.H * ((wl.T + 63) // 64)
+    achieved = scan_flops / (ms * 1e-3) / 1e12
     return {"workload": f"Gated DeltaNet backward B={wl.B} H={wl.H} T={wl.T} d_k=d_v={wl.dk} bf16 "
                         f"inputs, fp32 gradients, dO and dS_T ~ N(0, 1)",
-            "ms_per_call": ms, "tokens_per_s": wl.B * wl.T / (ms * 1e-3), "launches_per_call": 3,
-            "kernel": "gdr::bwd::bwd_scan_staged_kernel + gdr::bwd::bwd_chunk_kernel + gdr::bwd::bwd_gate_sum_kernel",
+            "ms_per_call": ms, "tokens_per_s": wl.B * wl.T / (ms * 1e-3), "launches_per_call": 2,
+            "kernel": "gdr::bwd::bwd_scan_staged_kernel (fp32 scans) + gdr::bwdtc::bwd_chunk_tc_kernel "
+                      "(tcgen05 chunk products)",
             "roofline": {"bound": "alu", "achieved": achieved, "peak": ALU_FP32_TFLOPS,
                          "unit": "TFLOP/s", "frac": achieved / ALU_FP32_TFLOPS,
                          "peak_source": "derived: 148 SMs x 128 fp32 lanes x 2 x 1965 MHz",
-                         "algorithmic_flops": flops, "algorithmic_bytes": bytes_,
-                         "hbm_frac": bytes_ / (ms * 1e-3) / 1e9 / pk["hbm_gbs"]}}
+                         "note": "the scans' flops over the whole call (the scans take most of it)",
+                         "algorithmic_flops": scan_flops, "algorithmic_bytes": bytes_,
+                         "hbm_frac": bytes_ / (ms * 1e-3) / 1e9 / pk["hbm_gbs"]},
+            "tensor_products": {"kernel": "gdr::bwdtc::bwd_chunk_tc_kernel", "flops_per_call": tc_flops,
+                                "peak_tflops": pk["bf16_tflops"],
+                                "duration": "per launch in the ncu launch list summary of this workload"}}
 
 
 def time_decode(dev, nsteps, warmup):

@@ -708,6 +708,10 @@ __global__ void __launch_bounds__(GS_NT, 1) state_general_kernel(
     uint64_t* bar_drain = bar_tma + 6;
     uint64_t* u_ready = bar_tma + 7;
     uint64_t* s_ready = bar_tma + 8;
+    // D5 commits, one barrier per TMEM column set (chunk parity): a barrier completes
+    // every second chunk, so a wait for one chunk's completion can never see the next
+    // completion of the same barrier first (that needs the state step in between)
+    auto bar_a_set = [&](int set) { return bar_tma + 5 + 4 * set; };  // bar_a, bar_tma + 9
     uint32_t* s_tmem = reinterpret_cast<uint32_t*>(sm + Lay::SMALL + 128);
     if (tid == 0) {
         for (int i = 0; i < 3; ++i) mbar_init(&bar_tma[i], 1);
@@ -717,6 +721,7 @@ __global__ void __launch_bounds__(GS_NT, 1) state_general_kernel(
         mbar_init(bar_drain, 1);
         mbar_init(u_ready, 128);
         mbar_init(s_ready, 1);
+        mbar_init(bar_a_set(1), 1);
         fence_barrier_init();
     }
     if (warp == 0) tmem_alloc(s_tmem, GS_TM_COLS);
@@ -788,7 +793,7 @@ __global__ void __launch_bounds__(GS_NT, 1) state_general_kernel(
             iok = mbar_wait(&bar_tma[buf], (uint32_t)(((ci - c_begin) / NBUF) & 1)) && iok;
             if (ci > c_begin) iok = mbar_wait(s_ready, (uint32_t)((ci - 1 - c_begin) & 1)) && iok;
             // the stage of chunk ci - 1 is refilled below: its AQ tile's last reader done
-            if (prev_mma) iok = mbar_wait(bar_a, (uint32_t)((nm - 1) & 1)) && iok;
+            if (prev_mma) iok = mbar_wait(bar_a_set((nm - 1) & 1), (uint32_t)(((nm - 1) >> 1) & 1)) && iok;
             iok = __all_sync(0xffffffffu, iok);
             if (!iok) break;
             tc_fence_after();
@@ -816,10 +821,8 @@ __global__ void __launch_bounds__(GS_NT, 1) state_general_kernel(
                     // ---- D4 = K2^T U (+ KW2^T V), then D5 = [AQ ; .] U (+ [BQ ; .] V): the
                     //      products with V come after the state's, and no product runs
                     //      while U is being written (its shared-memory reads would slow it)
-                    const uint32_t idK = idesc_bf16(128, NV, 0, 1);
                     const uint32_t idM = idesc_bf16(128, NV, 1, 1);
                     const uint32_t vb = sbase + Lay::V + buf * 8192u;
-                    const uint32_t bqa = sbase + Lay::BQ + buf * 8192u;  // BQ = rows 0..63
 #pragma unroll
                     for (int ks = 0; ks < 4; ++ks)
                         mma_bf16(tmem + GS_TM_D4, sdesc_sw128(k2b + ks * 2048u, 8192, 1024),
@@ -830,6 +833,8 @@ __global__ void __launch_bounds__(GS_NT, 1) state_general_kernel(
                             mma_bf16(tmem + GS_TM_D4, sdesc_sw128(sbase + Lay::KW2 + buf * 16384u + ks * 2048u, 8192, 1024),
                                      sdesc_sw128(vb + ks * 2048u, 8192, 1024), idM, 1u);
                     mma_commit(bar_k);
+                    const uint32_t idK = idesc_bf16(128, NV, 0, 1);
+                    const uint32_t bqa = sbase + Lay::BQ + buf * 8192u;  // BQ = rows 0..63
 #pragma unroll
                     for (int ks = 0; ks < 4; ++ks)
                         mma_bf16(tmem + d5, sdesc_sw128(aqa + ks * 32u, 16, 1024),
@@ -839,7 +844,7 @@ __global__ void __launch_bounds__(GS_NT, 1) state_general_kernel(
                         for (int ks = 0; ks < 4; ++ks)
                             mma_bf16(tmem + d5, sdesc_sw128(bqa + ks * 32u, 16, 1024),
                                      sdesc_sw128(vb + ks * 2048u, 8192, 1024), idK, 1u);
-                    mma_commit(bar_a);
+                    mma_commit(bar_a_set(par));
                 }
                 __syncwarp();
                 ++nm;
@@ -887,7 +892,7 @@ __global__ void __launch_bounds__(GS_NT, 1) state_general_kernel(
             if (ci + 1 < c_end) gC_next = gcp[(size_t)(ci + 1) * DK];
             const bool exact = gC < 0.f;  // the same mark in every channel: uniform
             if (lo && pend >= 0) {
-                w_ok = mbar_wait(bar_a, pend_ph) && w_ok;
+                w_ok = mbar_wait(bar_a_set(pend_set), pend_ph) && w_ok;
                 tc_fence_after();
                 store_o(pend, pend_set);
             }
@@ -930,7 +935,7 @@ __global__ void __launch_bounds__(GS_NT, 1) state_general_kernel(
                 }
                 pend = ci;
                 pend_set = par;
-                pend_ph = ph;
+                pend_ph = (uint32_t)((nm >> 1) & 1);  // the set's own completion count
                 ++nm;
             }
 #pragma unroll
@@ -942,7 +947,7 @@ __global__ void __launch_bounds__(GS_NT, 1) state_general_kernel(
         }
         if (ci < c_end) ok = false;  // a wait gave up
         if (ok && lo && pend >= 0) {
-            ok = mbar_wait(bar_a, pend_ph);
+            ok = mbar_wait(bar_a_set(pend_set), pend_ph);
             tc_fence_after();
             if (ok) store_o(pend, pend_set);
         }

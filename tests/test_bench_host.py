@@ -44,10 +44,12 @@ def test_recorded_traffic_is_keyed_to_the_kernel_sources(monkeypatch, tmp_path):
     assert bench.measured_traffic("kda") is None
 
 
-def test_backward_flops_per_element():
-    # forward step 4 multiply-adds, reverse step 9, per state element and token
-    assert bench.BWD_FLOPS_PER_ELEMENT == 26
+def test_backward_flop_counts():
+    # scans: forward 4 multiply-adds, backward 5, per state element and token
+    assert bench.BWD_SCAN_FLOPS_PER_ELEMENT == 18
     assert bench.ALU_FP32_TFLOPS == pytest.approx(74.45, abs=0.01)
+    # chunk kernel: one 128x256x128, one 128x64x128 and three 128x128x128 products
+    assert bench.BWD_TC_FLOPS_PER_CHUNK == 2 * (128 * 256 * 128 + 128 * 64 * 128 + 3 * 128 ** 3)
 
 
 def test_cpu_baseline_record():

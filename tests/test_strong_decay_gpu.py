@@ -45,3 +45,18 @@ def test_strong_decay(cuda_device, family, alpha, workspace):
     assert np.all(np.isfinite(o)) and np.all(np.isfinite(ST))
     assert_close(o, o_ref, TOL["bf16"], f"o (alpha {alpha})")
     assert_close(ST, ST_ref, TOL["bf16"], f"S_T (alpha {alpha})")
+
+
+@pytest.mark.parametrize("alpha", ["mixed", "bursts", "1e-4"])
+@pytest.mark.parametrize("family", ["kda", "gdn2"])
+def test_strong_decay_segmented(cuda_device, family, alpha):
+    """Few heads and a long sequence: the general form's state pass runs in
+    segments; chunks whose decay span is outside the two-factor range run
+    token by token in the middle of a segment's walk."""
+    wl = WORKLOADS[family].with_(B=1, H=2, T=4200, s0=True, seed=2300)
+    inp = _with_alpha(make_chunk_inputs(wl), ALPHAS[alpha])
+    o, ST = run_chunk(inp, cuda_device)
+    o_ref, ST_ref = run_oracle(inp)
+    assert np.all(np.isfinite(o)) and np.all(np.isfinite(ST))
+    assert_close(o, o_ref, TOL["bf16"], f"o (alpha {alpha})")
+    assert_close(ST, ST_ref, TOL["bf16"], f"S_T (alpha {alpha})")
