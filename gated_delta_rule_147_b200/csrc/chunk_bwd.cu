@@ -36,10 +36,15 @@
 namespace gdr {
 cudaError_t launch_bwd_chunk_tc(const CUtensorMap* maps, const float* ckS, const float* ckG,
                                 const float* R, const float* DR, const void* alpha,
-                                const void* beta, float* dq, float* dk, float* dalpha, float* db,
-                                int* d_status, int B, int T, int H, int group, int nchunks,
-                                cudaStream_t st);
+                                const void* beta, const void* v, bool r_from_u, float* dq, float* dk,
+                                float* dalpha, float* db, int* d_status, int B, int T, int H,
+                                int group, int nchunks, cudaStream_t st);
 bool make_tma_map_bf16(CUtensorMap* m, const void* base, int B, int T, int H, int d);
+size_t twopass_workspace_bytes(int B, int T, int H, int dv);
+cudaError_t launch_chunk_twopass_gdn(const CUtensorMap* maps, const CUtensorMap* ws_maps, void* ws,
+                                     const void* alpha, const void* beta, const float* S0, void* o,
+                                     float* ST, int* d_status, int B, int T, int H, int dv, int group,
+                                     cudaStream_t st, float* ckS, float* up);
 
 namespace bwd {
 
@@ -58,6 +63,8 @@ struct Params {
     float *dq, *dk, *dv, *dalpha, *db, *dw, *dS0;
     float *ckS, *ckG, *R, *DR, *GP;  // workspace
     int* d_status;                   // bounded waits of the tensor-core pass 2
+    int grad_scan_only;              // 1: the scans run only the backward direction (the
+                                     // forward two-pass kernels gave S and U = beta v - r)
     float *dq_out, *dk_out;          // grouped heads: the caller's dq, dk (dq, dk are then workspace)
     int B, T, H, Hq, group, dk_, dv_, akind, bkind, wkind, nchunks, tpr, nrb;
 };
@@ -194,7 +201,8 @@ __device__ __forceinline__ void load_rows4(const Params& p, size_t tok, size_t t
 }
 
 // ----------------------------------------------------------------- pass 1 --
-// blockIdx.z = 2 b + direction; warp w of CTA x owns columns
+// blockIdx.z = 2 b + direction (b alone, backward direction, when
+// grad_scan_only); warp w of CTA x owns columns
 // 8 (kScanWarps x + w) .. + 8 (those below d_v), lane l owns rows 4 l .. 4 l + 3.
 template <typename TI>
 __global__ void __launch_bounds__(kScanWarps * 32) bwd_scan_kernel(Params p) {
@@ -202,7 +210,8 @@ __global__ void __launch_bounds__(kScanWarps * 32) bwd_scan_kernel(Params p) {
     const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
     const int c0 = NC * (kScanWarps * blockIdx.x + warp);
     if (c0 >= p.dv_) return;  // no block-wide barriers in this kernel
-    const int b = blockIdx.z >> 1, dir = blockIdx.z & 1, h = blockIdx.y;
+    const int b = p.grad_scan_only ? (int)blockIdx.z : (int)(blockIdx.z >> 1);
+    const int dir = p.grad_scan_only ? 1 : (int)(blockIdx.z & 1), h = blockIdx.y;
     const size_t head = (size_t)b * p.H + h;
     const int i0 = 4 * lane;
     auto tok_of = [&](int t) { return ((size_t)b * p.T + t) * p.H + h; };
@@ -354,16 +363,26 @@ __device__ __forceinline__ void lds4<__nv_bfloat16>(const __nv_bfloat16* src, fl
     x[2] = __uint_as_float(u.y << 16); x[3] = __uint_as_float(u.y & 0xffff0000u);
 }
 
-template <typename TI>
+// NC state columns per warp: 8, or 4 when only the backward direction runs
+// (half the warps otherwise, and the scan is then bound by latency).
+template <typename TI, int NC>
 __global__ void __launch_bounds__(kScanWarps * 32) bwd_scan_staged_kernel(Params p) {
-    constexpr int NC = kScanCols, CTA_COLS = kScanWarps * kScanCols;
+    static_assert(NC == 4 || NC == 8, "4 or 8 columns per warp");
+    constexpr int CTA_COLS = kScanWarps * NC;
+    auto st_cols = [](float* dst, const float* x, float sign) {  // NC columns, 16-byte stores
+#pragma unroll
+        for (int c = 0; c < NC; c += 4)
+            *reinterpret_cast<float4*>(dst + c) =
+                make_float4(sign * x[c], sign * x[c + 1], sign * x[c + 2], sign * x[c + 3]);
+    };
     __shared__ __align__(16) ScanStage<TI> stg[2];
     const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
     const int cb = CTA_COLS * blockIdx.x;  // the CTA's first column
     const int c0 = cb + NC * warp;
     const bool active = c0 < p.dv_;       // idle warps still copy and meet the barriers
     const int ncols = min(CTA_COLS, p.dv_ - cb);
-    const int b = blockIdx.z >> 1, dir = blockIdx.z & 1, h = blockIdx.y;
+    const int b = p.grad_scan_only ? (int)blockIdx.z : (int)(blockIdx.z >> 1);
+    const int dir = p.grad_scan_only ? 1 : (int)(blockIdx.z & 1), h = blockIdx.y;
     const size_t head = (size_t)b * p.H + h;
     const int i0 = 4 * lane;
     const bool rows_ok = i0 < p.dk_;       // d_k is a multiple of 4 here
@@ -418,9 +437,14 @@ __global__ void __launch_bounds__(kScanWarps * 32) bwd_scan_staged_kernel(Params
     const float* init = dir == 0 ? p.S0 : p.dST;
 #pragma unroll
     for (int rr = 0; rr < 4; ++rr) {
-        if (active && init && i0 + rr < p.dk_)
-            load8<float>(init, (head * p.dk_ + i0 + rr) * p.dv_ + c0, X[rr]);
-        else
+        if (active && init && i0 + rr < p.dk_) {
+#pragma unroll
+            for (int c = 0; c < NC; c += 4) {
+                float x4[4];
+                load4<float>(init, (head * p.dk_ + i0 + rr) * p.dv_ + c0 + c, x4);
+                X[rr][c] = x4[0]; X[rr][c + 1] = x4[1]; X[rr][c + 2] = x4[2]; X[rr][c + 3] = x4[3];
+            }
+        } else
             for (int c = 0; c < NC; ++c) X[rr][c] = 0.f;
     }
 
@@ -455,8 +479,7 @@ __global__ void __launch_bounds__(kScanWarps * 32) bwd_scan_staged_kernel(Params
                         if (i0 + rr < p.dk_) {
                             float* dst = (dir == 0 ? p.ckS : p.ckG) +
                                   ((head * p.nchunks + t / kC) * p.dk_ + i0 + rr) * p.dv_ + c0;
-                            reinterpret_cast<float4*>(dst)[0] = make_float4(X[rr][0], X[rr][1], X[rr][2], X[rr][3]);
-                            reinterpret_cast<float4*>(dst)[1] = make_float4(X[rr][4], X[rr][5], X[rr][6], X[rr][7]);
+                            st_cols(dst, X[rr], 1.f);
                         }
                 Rows4 rw;
                 if (rows_ok) {
@@ -480,12 +503,11 @@ __global__ void __launch_bounds__(kScanWarps * 32) bwd_scan_staged_kernel(Params
                     }
                 }
                 float cv[NC];
-                {
-                    float a4[4], b4[4];
-                    lds4<TI>(&S_.cols[tt][NC * warp], a4);
-                    lds4<TI>(&S_.cols[tt][NC * warp + 4], b4);
 #pragma unroll
-                    for (int c = 0; c < 4; ++c) { cv[c] = a4[c]; cv[4 + c] = b4[c]; }
+                for (int c = 0; c < NC; c += 4) {
+                    float a4[4];
+                    lds4<TI>(&S_.cols[tt][NC * warp + c], a4);
+                    cv[c] = a4[0]; cv[c + 1] = a4[1]; cv[c + 2] = a4[2]; cv[c + 3] = a4[3];
                 }
                 if (dir == 0) {
                     float r[NC];
@@ -509,9 +531,7 @@ __global__ void __launch_bounds__(kScanWarps * 32) bwd_scan_staged_kernel(Params
                             X[rr][c] = fmaf(-rw.k[rr], r[c], fmaf(u, cv[c], X[rr][c]));
                     }
                     if (lane == 0) {
-                        float* dst = p.R + tok * p.dv_ + c0;
-                        reinterpret_cast<float4*>(dst)[0] = make_float4(r[0], r[1], r[2], r[3]);
-                        reinterpret_cast<float4*>(dst)[1] = make_float4(r[4], r[5], r[6], r[7]);
+                        st_cols(p.R + tok * p.dv_ + c0, r, 1.f);
                     }
                 } else {
                     float z[2 * NC];
@@ -535,12 +555,8 @@ __global__ void __launch_bounds__(kScanWarps * 32) bwd_scan_staged_kernel(Params
                         for (int c = 0; c < NC; ++c) X[rr][c] = rw.a[rr] * fmaf(-e, z[c], X[rr][c]);
                     }
                     if (lane == 0) {
-                        float* dst = p.DR + tok * p.dv_ + c0;
-                        reinterpret_cast<float4*>(dst)[0] = make_float4(-z[0], -z[1], -z[2], -z[3]);
-                        reinterpret_cast<float4*>(dst)[1] = make_float4(-z[4], -z[5], -z[6], -z[7]);
-                        float* dvp = p.dv + tok * p.dv_ + c0;
-                        reinterpret_cast<float4*>(dvp)[0] = make_float4(z[8], z[9], z[10], z[11]);
-                        reinterpret_cast<float4*>(dvp)[1] = make_float4(z[12], z[13], z[14], z[15]);
+                        st_cols(p.DR + tok * p.dv_ + c0, z, -1.f);
+                        st_cols(p.dv + tok * p.dv_ + c0, z + NC, 1.f);
                     }
                 }
             }
@@ -552,9 +568,7 @@ __global__ void __launch_bounds__(kScanWarps * 32) bwd_scan_staged_kernel(Params
 #pragma unroll
         for (int rr = 0; rr < 4; ++rr)
             if (i0 + rr < p.dk_) {
-                float* dst = p.dS0 + (head * p.dk_ + i0 + rr) * p.dv_ + c0;
-                reinterpret_cast<float4*>(dst)[0] = make_float4(X[rr][0], X[rr][1], X[rr][2], X[rr][3]);
-                reinterpret_cast<float4*>(dst)[1] = make_float4(X[rr][4], X[rr][5], X[rr][6], X[rr][7]);
+                st_cols(p.dS0 + (head * p.dk_ + i0 + rr) * p.dv_ + c0, X[rr], 1.f);
             }
 }
 
@@ -845,7 +859,7 @@ int threads_per_row(int dv) {
 size_t round256(size_t x) { return (x + 255) & ~size_t(255); }
 
 struct WsLayout {
-    size_t ckS, ckG, R, DR, GP, DQ, DK, total;
+    size_t ckS, ckG, R, DR, GP, DQ, DK, FW, total;
 };
 
 WsLayout ws_layout(int B, int T, int H, int dk, int dv, bool grouped) {
@@ -863,23 +877,45 @@ WsLayout ws_layout(int B, int T, int H, int dk, int dv, bool grouped) {
     const size_t gq = grouped ? round256((size_t)B * T * H * dk * sizeof(float)) : 0;
     l.DQ = l.GP + gp;
     l.DK = l.DQ + gq;
-    l.total = l.DK + gq;
+    // d_k = d_v = 128: the forward's per-chunk factors (-W, P), which the
+    // tensor-core path computes again to checkpoint S and r on tensor cores
+    l.FW = l.DK + gq;
+    l.total = l.FW + (dk == 128 && dv == 128 ? round256(twopass_workspace_bytes(B, T, H, dv)) : 0);
     return l;
 }
 
-// tc_maps (q, k, v, dO tensor maps) selects the tensor-core pass 2 of the
-// Gated DeltaNet form; it writes the scalar gate gradients itself.
+// tc_maps (q, k, v, dO tensor maps) selects the tensor-core path of the Gated
+// DeltaNet form: the forward two-pass kernels (their factors in fw, maps
+// fw_maps) checkpoint the state at every chunk start and U = beta v - r of
+// every token, the scans run only the backward direction, and the tensor-core
+// pass 2 writes the scalar gate gradients itself.
 template <typename TI>
-cudaError_t launch_typed(Params p, const CUtensorMap* tc_maps, cudaStream_t st) {
-    const dim3 sgrid((p.dv_ + kScanCols * kScanWarps - 1) / (kScanCols * kScanWarps), p.H, 2 * p.B);
-    if ((p.dk_ * sizeof(TI)) % 16 == 0)
-        bwd_scan_staged_kernel<TI><<<sgrid, kScanWarps * 32, 0, st>>>(p);
-    else
-        bwd_scan_kernel<TI><<<sgrid, kScanWarps * 32, 0, st>>>(p);
-    cudaError_t e = cudaGetLastError();
+cudaError_t launch_typed(Params p, const CUtensorMap* tc_maps, const CUtensorMap* fw_maps, void* fw,
+                         cudaStream_t st) {
+    cudaError_t e;
+    if (tc_maps) {
+        e = launch_chunk_twopass_gdn(tc_maps, fw_maps, fw, p.alpha, p.b, p.S0, nullptr, nullptr,
+                                     p.d_status, p.B, p.T, p.H, p.dv_, p.group, st, p.ckS, p.R);
+        if (e != cudaSuccess) return e;
+        p.grad_scan_only = 1;
+    }
+    const int ncw = p.grad_scan_only ? 4 : kScanCols;  // state columns per scan warp
+    const dim3 sgrid((p.dv_ + ncw * kScanWarps - 1) / (ncw * kScanWarps), p.H,
+                     p.grad_scan_only ? p.B : 2 * p.B);
+    if ((p.dk_ * sizeof(TI)) % 16 == 0) {
+        if (p.grad_scan_only)
+            bwd_scan_staged_kernel<TI, 4><<<sgrid, kScanWarps * 32, 0, st>>>(p);
+        else
+            bwd_scan_staged_kernel<TI, kScanCols><<<sgrid, kScanWarps * 32, 0, st>>>(p);
+    } else {
+        const dim3 g8((p.dv_ + kScanCols * kScanWarps - 1) / (kScanCols * kScanWarps), p.H,
+                      p.grad_scan_only ? p.B : 2 * p.B);
+        bwd_scan_kernel<TI><<<g8, kScanWarps * 32, 0, st>>>(p);
+    }
+    e = cudaGetLastError();
     if (e != cudaSuccess) return e;
     if (tc_maps) {
-        e = launch_bwd_chunk_tc(tc_maps, p.ckS, p.ckG, p.R, p.DR, p.alpha, p.b, p.dq, p.dk,
+        e = launch_bwd_chunk_tc(tc_maps, p.ckS, p.ckG, p.R, p.DR, p.alpha, p.b, p.v, true, p.dq, p.dk,
                                 p.dalpha, p.db, p.d_status, p.B, p.T, p.H, p.group, p.nchunks, st);
         if (e != cudaSuccess) return e;
         if (p.group > 1) {
@@ -1013,22 +1049,27 @@ gdr_status gdr_chunk_bwd_grouped(const void* q, const void* k, const void* v, co
     const int RB = gdr::bwd::kChunkThreads / p.tpr;
     p.nrb = (d_k + RB - 1) / RB;
     p.d_status = d_status;
+    p.grad_scan_only = 0;
     // the Gated DeltaNet form on tensor cores: scalar decay, tied scalar beta,
     // bf16, d_k = d_v = 128
-    CUtensorMap maps[4];
+    CUtensorMap maps[4], fw_maps[2];
     const CUtensorMap* tc_maps = nullptr;
+    void* fw = ws + wl.FW;
     if (dtype == GDR_BF16 && d_k == 128 && d_v == 128 && alpha_kind == GDR_GATE_SCALAR &&
         b_kind == GDR_GATE_SCALAR && w_kind == GDR_GATE_TIED) {
         if (!gdr::make_tma_map_bf16(&maps[0], q, B, T, H_qk, d_k) ||
             !gdr::make_tma_map_bf16(&maps[1], k, B, T, H_qk, d_k) ||
             !gdr::make_tma_map_bf16(&maps[2], v, B, T, H, d_v) ||
-            !gdr::make_tma_map_bf16(&maps[3], dO, B, T, H, d_v))
+            !gdr::make_tma_map_bf16(&maps[3], dO, B, T, H, d_v) ||
+            !gdr::make_tma_map_bf16(&fw_maps[0], fw, B, T, H, d_k) ||
+            !gdr::make_tma_map_bf16(&fw_maps[1], ws + wl.FW + (size_t)B * T * H * d_k * 2, B, T, H, d_v))
             return GDR_ERR_NO_DEVICE;
         tc_maps = maps;
         p.GP = nullptr;
     }
-    const cudaError_t e = dtype == GDR_BF16 ? gdr::bwd::launch_typed<__nv_bfloat16>(p, tc_maps, st)
-                                            : gdr::bwd::launch_typed<float>(p, nullptr, st);
+    const cudaError_t e = dtype == GDR_BF16
+                              ? gdr::bwd::launch_typed<__nv_bfloat16>(p, tc_maps, fw_maps, fw, st)
+                              : gdr::bwd::launch_typed<float>(p, nullptr, nullptr, nullptr, st);
     return e == cudaSuccess ? GDR_OK : GDR_ERR_LAUNCH;
 }
 

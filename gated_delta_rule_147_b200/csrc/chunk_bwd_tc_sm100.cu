@@ -50,6 +50,9 @@ struct TcParams {
     const float *ckS, *ckG, *R, *DR;       // scans: chunk-start states, chunk-end state
                                            // gradients, r, dr (fp32)
     const __nv_bfloat16 *alpha, *beta;     // scalar gates [B, T, H]
+    const __nv_bfloat16* v;                // [B, T, H, 128]
+    int r_from_u;                          // R holds U = beta v - r (from the forward
+                                           // kernels): r = beta v - U
     float *dq, *dk, *dalpha, *db;          // dq, dk [B, T, H, 128] per value head; gates [B, T, H]
     int* d_status;
     int T, H, group, nchunks;
@@ -144,7 +147,24 @@ __global__ void __launch_bounds__(256, 1) bwd_chunk_tc_kernel(const __grid_const
 #pragma unroll
             for (int e = 0; e < 32; ++e) x[e] = 0.f;
         put32(sm + R0, 64 + t, part * 4, 128, x);
-        if (t < n) ld32f(p.R + tok * 128 + part * 32, x);
+        if (t < n) {
+            ld32f(p.R + tok * 128 + part * 32, x);
+            if (p.r_from_u) {
+                const float bt = __bfloat162float(p.beta[tok]);
+                const uint4* vp = reinterpret_cast<const uint4*>(p.v + tok * 128 + part * 32);
+#pragma unroll
+                for (int c4 = 0; c4 < 4; ++c4) {
+                    const uint4 u = vp[c4];
+                    const __nv_bfloat162* hh = reinterpret_cast<const __nv_bfloat162*>(&u);
+#pragma unroll
+                    for (int e = 0; e < 4; ++e) {
+                        const float2 f = __bfloat1622float2(hh[e]);
+                        x[c4 * 8 + 2 * e] = fmaf(bt, f.x, -x[c4 * 8 + 2 * e]);
+                        x[c4 * 8 + 2 * e + 1] = fmaf(bt, f.y, -x[c4 * 8 + 2 * e + 1]);
+                    }
+                }
+            }
+        }
         put32(sm + R1, 192 + t, part * 4, 256, x);
         const int i = tid >> 1, half = tid & 1;  // key channel, 64 value columns
         const float* s0 = p.ckS + ((head * p.nchunks + c) * 128 + i) * 128 + half * 64;
@@ -468,12 +488,14 @@ finish:
 // maps: q, k (q/k heads), v, dO (value heads), bf16 [B, T, H, 128] each.
 cudaError_t launch_bwd_chunk_tc(const CUtensorMap* maps, const float* ckS, const float* ckG,
                                 const float* R, const float* DR, const void* alpha,
-                                const void* beta, float* dq, float* dk, float* dalpha, float* db,
-                                int* d_status, int B, int T, int H, int group, int nchunks,
-                                cudaStream_t st) {
+                                const void* beta, const void* v, bool r_from_u, float* dq, float* dk,
+                                float* dalpha, float* db, int* d_status, int B, int T, int H,
+                                int group, int nchunks, cudaStream_t st) {
     using namespace bwdtc;
     TcParams p;
     p.ckS = ckS; p.ckG = ckG; p.R = R; p.DR = DR;
+    p.v = reinterpret_cast<const __nv_bfloat16*>(v);
+    p.r_from_u = r_from_u ? 1 : 0;
     p.alpha = reinterpret_cast<const __nv_bfloat16*>(alpha);
     p.beta = reinterpret_cast<const __nv_bfloat16*>(beta);
     p.dq = dq; p.dk = dk; p.dalpha = dalpha; p.db = db; p.d_status = d_status;

@@ -412,10 +412,22 @@ __device__ __forceinline__ void mbar_arrive(uint64_t* bar) {
 // memory (mbarriers u_ready, aq_ready, s_ready), so no compute warp waits on
 // MMA issue. Decay ratios are formed per element from the log2 prefix l
 // (exact for any alpha in (0, 1]: every factor used is at most 1).
+// Optional checkpoints for the backward pass, written off the chunk chain:
+// the fp32 state at every chunk start ([B, H, nchunks, 128, d_v]) and
+// U = P - W S of every token in fp32 ([B, T, H, d_v]; U = beta v - r, with r
+// the token's erase read).
+struct Ckpt {
+    float* ckS;
+    float* up;
+};
+
+// CKPT: the backward pass's instantiation (checkpoints written, o not written);
+// the forward's has none of that code.
+template <bool CKPT>
 __global__ void __launch_bounds__(S_NT, 1) state_gdn_kernel(
     const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ CUtensorMap tm_k,
     const __grid_constant__ CUtensorMap tm_w, const __grid_constant__ CUtensorMap tm_p,
-    const Params p) {
+    const Params p, const Ckpt ck) {
     extern __shared__ uint8_t smem_raw[];
     uint8_t* sm = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) &
                                              ~uintptr_t(1023));
@@ -641,7 +653,7 @@ __global__ void __launch_bounds__(S_NT, 1) state_gdn_kernel(
             tmem_ld32_async(tmem + lane_base + S_TM_D3 + pj * 64 + wg * 32, d);
             tmem_ld32_async(tmem + lane_base + S_TM_D5 + pj * 64 + wg * 32, d5);
             tmem_wait_ld();
-            if (t < T) {
+            if (t < T && !CKPT) {
                 const float gr = s_g3[(cj % 3) * 64 + row];
                 __nv_bfloat16* op = p.o + (((size_t)bb * T + t) * H + h) * p.dv + v0 + wg * 32;
 #pragma unroll
@@ -664,6 +676,12 @@ __global__ void __launch_bounds__(S_NT, 1) state_gdn_kernel(
             const int par = ci & 1;
             const uint32_t ph = (uint32_t)(ci & 1);
             const int s3 = ci % 3;
+            if (CKPT) {  // the state at this chunk's start, for the backward pass
+                float* dst = ck.ckS + ((((size_t)bb * H + h) * nchunks + ci) * DK + row) * p.dv + v0 + wg * NH;
+#pragma unroll
+                for (int jj = 0; jj < NH; jj += 4)
+                    *reinterpret_cast<float4*>(dst + jj) = make_float4(S[jj], S[jj + 1], S[jj + 2], S[jj + 3]);
+            }
             if (lo) {
                 // ---- O of the previous chunk, the next decay scan, Aq -----------------------
                 if (ci > 0) {
@@ -719,6 +737,11 @@ __global__ void __launch_bounds__(S_NT, 1) state_gdn_kernel(
                         ld_chunk(sm + buf * S_STAGE + S_ST_P, off, x);
 #pragma unroll
                         for (int e = 0; e < 8; ++e) x[e] += d[c8 * 8 + e];
+                        if (CKPT && ci * C + j < T) {
+                            float* up = ck.up + (((size_t)bb * T + ci * C + j) * H + h) * p.dv + v0 + wg * 32 + c8 * 8;
+                            *reinterpret_cast<float4*>(up) = make_float4(x[0], x[1], x[2], x[3]);
+                            *reinterpret_cast<float4*>(up + 4) = make_float4(x[4], x[5], x[6], x[7]);
+                        }
                         st_chunk(sm + S_OFF_U, off, x);
 #pragma unroll
                         for (int e = 0; e < 8; ++e) x[e] *= f;
@@ -775,10 +798,12 @@ size_t twopass_workspace_bytes(int B, int T, int H, int dv) {
 }
 
 // maps: q, k, v, then the workspace maps -W ([B,T,H,128]) and P ([B,T,H,d_v]).
+// ckS, up: the backward pass's checkpoints (struct Ckpt; both or neither), or NULL:
+// with them, o is not written.
 cudaError_t launch_chunk_twopass_gdn(const CUtensorMap* maps, const CUtensorMap* ws_maps, void* ws,
                                      const void* alpha, const void* beta, const float* S0, void* o,
                                      float* ST, int* d_status, int B, int T, int H, int dv, int group,
-                                     cudaStream_t st) {
+                                     cudaStream_t st, float* ckS, float* up) {
     using namespace twopass;
     PrepParams pp;
     pp.alpha = alpha; pp.beta = beta;
@@ -803,7 +828,9 @@ cudaError_t launch_chunk_twopass_gdn(const CUtensorMap* maps, const CUtensorMap*
     p.B = B; p.T = T; p.H = H; p.dv = dv;
     p.akind = GDR_GATE_SCALAR; p.bkind = GDR_GATE_SCALAR; p.wkind = GDR_GATE_TIED;
     p.group = group;
-    e = cudaFuncSetAttribute(state_gdn_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, S_SMEM_BYTES);
+    const bool ckpt = ckS != nullptr;
+    e = ckpt ? cudaFuncSetAttribute(state_gdn_kernel<true>, cudaFuncAttributeMaxDynamicSharedMemorySize, S_SMEM_BYTES)
+             : cudaFuncSetAttribute(state_gdn_kernel<false>, cudaFuncAttributeMaxDynamicSharedMemorySize, S_SMEM_BYTES);
     if (e != cudaSuccess) return e;
     cudaLaunchConfig_t cfg = {};
     cfg.gridDim = dim3(dv / NV, H, B);
@@ -815,7 +842,11 @@ cudaError_t launch_chunk_twopass_gdn(const CUtensorMap* maps, const CUtensorMap*
     attr[0].val.programmaticStreamSerializationAllowed = 1;
     cfg.attrs = attr;
     cfg.numAttrs = 1;
-    return cudaLaunchKernelEx(&cfg, state_gdn_kernel, maps[0], maps[1], ws_maps[0], ws_maps[1], p);
+    Ckpt ck;
+    ck.ckS = ckS;
+    ck.up = up;
+    return ckpt ? cudaLaunchKernelEx(&cfg, state_gdn_kernel<true>, maps[0], maps[1], ws_maps[0], ws_maps[1], p, ck)
+                : cudaLaunchKernelEx(&cfg, state_gdn_kernel<false>, maps[0], maps[1], ws_maps[0], ws_maps[1], p, ck);
 }
 
 }  // namespace gdr

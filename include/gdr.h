@@ -253,11 +253,14 @@ size_t gdr_chunk_fwd_static_capacity(void);
  *   forms dq, dk and the gate gradients of each chunk from its start state,
  *   end gradient, r and dr:
  *   - the Gated DeltaNet form in bf16 with d_k = d_v = 128 (alpha and b
- *     scalar, w tied): on tensor cores as masked, decay-scaled products
- *     (bf16 operands: the fp32 checkpoints, r and dr are rounded to bf16;
- *     fp32 accumulation), one CTA per (chunk, head) writing dalpha and db
- *     directly; its bounded waits OR GDR_DEVICE_TIMEOUT into *d_status
- *     (if not NULL) and end the kernel, leaving the outputs undefined;
+ *     scalar, w tied): the forward two-pass tensor-core kernels run first
+ *     and give S at every chunk start and r_t (so the scan runs only the
+ *     backward direction); then the chunk gradients on tensor cores as
+ *     masked, decay-scaled products (bf16 operands: the checkpoints, r and
+ *     dr are rounded to bf16; fp32 accumulation), one CTA per (chunk,
+ *     head) writing dalpha and db directly; the bounded waits of these
+ *     kernels OR GDR_DEVICE_TIMEOUT into *d_status (if not NULL) and end
+ *     the kernel, leaving the outputs undefined;
  *   - every other form and dtype: fp32 on CUDA cores, per block of state
  *     rows, rebuilding the chunk's states elementwise; a third kernel then
  *     sums scalar gates' gradients over the key channels; d_status unused.
@@ -309,7 +312,9 @@ size_t gdr_chunk_bwd_grouped_workspace_size(int B, int T, int H_qk, int H, int d
  * chunk-start states and chunk-end state gradients (2 x B H ceil(T/64) d_k
  * d_v), r_t and dr_t of every token (2 x B T H d_v), and scalar-gate partial
  * sums (3 x ceil(d_k / RB) x B T H, RB = 128 / (d_v / 8 rounded up to a power
- * of two)), each rounded up to 256 bytes. Host-only; launches nothing. */
+ * of two)), and when d_k = d_v = 128 the forward's per-token -W and P rows
+ * (B T H (d_k + d_v) bf16), each rounded up to 256 bytes. Host-only;
+ * launches nothing. */
 size_t gdr_chunk_bwd_workspace_size(int B, int T, int H, int d_k, int d_v);
 
 /*

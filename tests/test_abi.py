@@ -174,9 +174,10 @@ def r256(x):
 
 
 @pytest.mark.parametrize("shape,expect", [
-    # checkpoints of S and G, r and dr per token, scalar-gate partials (16 row blocks of 8)
+    # checkpoints of S and G, r and dr per token, scalar-gate partials (16 row blocks of
+    # 8), and at d_k = d_v = 128 the forward's -W and P rows (bf16)
     ((4, 4096, 16, 128, 128), 2 * 4 * 16 * 64 * 128 * 128 * 4 + 2 * 4 * 4096 * 16 * 128 * 4
-     + 3 * 16 * 4 * 4096 * 16 * 4),
+     + 3 * 16 * 4 * 4096 * 16 * 4 + 4 * 4096 * 16 * (128 + 128) * 2),
     # d_v = 32: 4 threads per row, 32 rows per block, 2 blocks
     ((1, 65, 2, 64, 32), 2 * 2 * 2 * 64 * 32 * 4 + 2 * r256(65 * 2 * 32 * 4) + r256(3 * 2 * 65 * 2 * 4)),
     ((1, 0, 2, 64, 32), 0),
