@@ -214,11 +214,12 @@ gdr_status chunk_fwd_impl(const void* q, const void* k, const void* v, const voi
                                                   alpha_kind, b_kind, w_kind, S0, o, S_T, d_status,
                                                   B, T, H, d_v, group, allow_segments, st);
         } else if (tp == TP_GDN) {
-            CUtensorMap ws_maps[2];
+            CUtensorMap ws_maps[3];
             const uint8_t* pbase = reinterpret_cast<const uint8_t*>(workspace) +
                                    (size_t)B * T * H * d_k * sizeof(uint16_t);
+            const uint8_t* aqbase = pbase + (size_t)B * T * H * d_v * sizeof(uint16_t);
             if (!make_map(&ws_maps[0], workspace, B, T, H, d_k) ||
-                !make_map(&ws_maps[1], pbase, B, T, H, d_v))
+                !make_map(&ws_maps[1], pbase, B, T, H, d_v) || !make_map(&ws_maps[2], aqbase, B, T, H, 64))
                 return GDR_ERR_INVALID_ARG;
             e = gdr::launch_chunk_twopass_gdn(maps, ws_maps, workspace, alpha, b, S0, o, S_T,
                                               d_status, B, T, H, d_v, group, st);

@@ -1052,7 +1052,7 @@ gdr_status gdr_chunk_bwd_grouped(const void* q, const void* k, const void* v, co
     p.grad_scan_only = 0;
     // the Gated DeltaNet form on tensor cores: scalar decay, tied scalar beta,
     // bf16, d_k = d_v = 128
-    CUtensorMap maps[4], fw_maps[2];
+    CUtensorMap maps[4], fw_maps[3];
     const CUtensorMap* tc_maps = nullptr;
     void* fw = ws + wl.FW;
     if (dtype == GDR_BF16 && d_k == 128 && d_v == 128 && alpha_kind == GDR_GATE_SCALAR &&
@@ -1062,7 +1062,8 @@ gdr_status gdr_chunk_bwd_grouped(const void* q, const void* k, const void* v, co
             !gdr::make_tma_map_bf16(&maps[2], v, B, T, H, d_v) ||
             !gdr::make_tma_map_bf16(&maps[3], dO, B, T, H, d_v) ||
             !gdr::make_tma_map_bf16(&fw_maps[0], fw, B, T, H, d_k) ||
-            !gdr::make_tma_map_bf16(&fw_maps[1], ws + wl.FW + (size_t)B * T * H * d_k * 2, B, T, H, d_v))
+            !gdr::make_tma_map_bf16(&fw_maps[1], ws + wl.FW + (size_t)B * T * H * d_k * 2, B, T, H, d_v) ||
+            !gdr::make_tma_map_bf16(&fw_maps[2], ws + wl.FW + (size_t)B * T * H * (d_k + d_v) * 2, B, T, H, 64))
             return GDR_ERR_NO_DEVICE;
         tc_maps = maps;
         p.GP = nullptr;

@@ -65,13 +65,14 @@ __device__ unsigned long long g_trace2[64 * 16];
 // M = 128 MMAs read A rows 64..127 beyond each 64-row operand; those rows
 // land in the next region (garbage rows whose outputs are never read).
 constexpr uint32_t P_OFF_K = 0;        // K [64 x 128] bf16, two 8 KB column halves; 2 buffers
-constexpr uint32_t P_OFF_V = 32768;    // V [64 x d_v] bf16, d_v / 64 tiles of 8 KB; 2 buffers
+constexpr uint32_t P_OFF_Q = 32768;    // Q [64 x 128] bf16 (one buffer); then the Aq staging tile
+constexpr uint32_t P_OFF_V = 49152;    // V [64 x d_v] bf16, d_v / 64 tiles of 8 KB (one buffer)
 constexpr uint32_t P_OFF_A32 = 65536;  // A fp32 [64 x 64]; then L, PRE bf16; then -W staging
 constexpr uint32_t P_OFF_T32 = 81920;  // T fp32 [64 x 64]; then P staging
 constexpr uint32_t P_OFF_SCR = 98304;  // solve scratch fp32 (5 KB)
 constexpr uint32_t P_OFF_SMALL = 103424;
 constexpr uint32_t P_SMEM_BYTES = P_OFF_SMALL + 2048 + 1024;
-constexpr uint32_t P_TM_D1 = 0, P_TM_D3 = 0, P_TM_D2 = 128, P_TM_COLS = 256;
+constexpr uint32_t P_TM_D1 = 0, P_TM_DQ = 64, P_TM_D3 = 0, P_TM_D2 = 128, P_TM_COLS = 256;
 
 struct PrepParams {
     const void* alpha;
@@ -81,10 +82,17 @@ struct PrepParams {
     int group;  // value heads per k head (k read at head h / group)
 };
 
-__global__ void __launch_bounds__(NT, 2) prep_gdn_kernel(const __grid_constant__ CUtensorMap tm_k,
+// Loads: K two items ahead (two buffers), Q once the current item's Q K^T has
+// read it and its Aq store has left the tile, V once the current item's P
+// product has read it. Q K^T rides in the otherwise unused TMEM lanes 64..127
+// of the K K^T batch (its operand starts 8 KB before Q), so the warps that own
+// those lanes form Aq while the others form A.
+__global__ void __launch_bounds__(NT, 2) prep_gdn_kernel(const __grid_constant__ CUtensorMap tm_q,
+                                                         const __grid_constant__ CUtensorMap tm_k,
                                                          const __grid_constant__ CUtensorMap tm_v,
                                                          const __grid_constant__ CUtensorMap tm_wout,
                                                          const __grid_constant__ CUtensorMap tm_pout,
+                                                         const __grid_constant__ CUtensorMap tm_aqout,
                                                          const PrepParams pp) {
     extern __shared__ uint8_t smem_raw[];
     uint8_t* sm = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) &
@@ -98,9 +106,11 @@ __global__ void __launch_bounds__(NT, 2) prep_gdn_kernel(const __grid_constant__
     float* s_l = s_beta + 64;   // log2 prefix of alpha over the chunk
     float* s_g = s_beta + 192;
     float* s_alpha = s_beta + 256;
-    uint64_t* bar_tma = reinterpret_cast<uint64_t*>(sm + P_OFF_SMALL + 1280);  // [2]
+    uint64_t* bar_tma = reinterpret_cast<uint64_t*>(sm + P_OFF_SMALL + 1280);  // [2]: K
     uint64_t* bar_mma = bar_tma + 2;
-    uint32_t* s_tmem = reinterpret_cast<uint32_t*>(sm + P_OFF_SMALL + 1312);
+    uint64_t* bar_q = bar_tma + 3;
+    uint64_t* bar_v = bar_tma + 4;
+    uint32_t* s_tmem = reinterpret_cast<uint32_t*>(sm + P_OFF_SMALL + 1328);
     const uint32_t sbase = smem_u32(sm);
 
     auto coords = [&](int item, int& ci, int& h, int& bb) {
@@ -109,16 +119,28 @@ __global__ void __launch_bounds__(NT, 2) prep_gdn_kernel(const __grid_constant__
         h = hb % H;
         bb = hb / H;
     };
-    auto issue_loads = [&](int item, int buf) {
+    auto issue_k = [&](int item, int buf) {
         int ci, h, bb;
         coords(item, ci, h, bb);
         const int hq = h / pp.group;
-        const int t0 = ci * C;
-        mbar_expect_tx(&bar_tma[buf], (uint32_t)(2 + nvt) * 8192u);
-        tma_load_4d(sm + P_OFF_K + buf * 16384, &tm_k, &bar_tma[buf], 0, hq, t0, bb);
-        tma_load_4d(sm + P_OFF_K + buf * 16384 + 8192, &tm_k, &bar_tma[buf], 64, hq, t0, bb);
+        mbar_expect_tx(&bar_tma[buf], 2u * 8192u);
+        tma_load_4d(sm + P_OFF_K + buf * 16384, &tm_k, &bar_tma[buf], 0, hq, ci * C, bb);
+        tma_load_4d(sm + P_OFF_K + buf * 16384 + 8192, &tm_k, &bar_tma[buf], 64, hq, ci * C, bb);
+    };
+    auto issue_q = [&](int item) {
+        int ci, h, bb;
+        coords(item, ci, h, bb);
+        const int hq = h / pp.group;
+        mbar_expect_tx(bar_q, 2u * 8192u);
+        tma_load_4d(sm + P_OFF_Q, &tm_q, bar_q, 0, hq, ci * C, bb);
+        tma_load_4d(sm + P_OFF_Q + 8192, &tm_q, bar_q, 64, hq, ci * C, bb);
+    };
+    auto issue_v = [&](int item) {
+        int ci, h, bb;
+        coords(item, ci, h, bb);
+        mbar_expect_tx(bar_v, (uint32_t)nvt * 8192u);
         for (int vt = 0; vt < nvt; ++vt)
-            tma_load_4d(sm + P_OFF_V + buf * 16384 + vt * 8192, &tm_v, &bar_tma[buf], vt * 64, h, t0, bb);
+            tma_load_4d(sm + P_OFF_V + vt * 8192, &tm_v, bar_v, vt * 64, h, ci * C, bb);
     };
     unsigned short g_a = 0, g_b = 0;
     auto load_gates = [&](int item) {
@@ -140,12 +162,20 @@ __global__ void __launch_bounds__(NT, 2) prep_gdn_kernel(const __grid_constant__
         mbar_init(&bar_tma[0], 1);
         mbar_init(&bar_tma[1], 1);
         mbar_init(bar_mma, 1);
+        mbar_init(bar_q, 1);
+        mbar_init(bar_v, 1);
         fence_barrier_init();
+        prefetch_tmap(&tm_q);
         prefetch_tmap(&tm_k);
         prefetch_tmap(&tm_v);
         prefetch_tmap(&tm_wout);
         prefetch_tmap(&tm_pout);
-        if ((int)blockIdx.x < pp.nitems) issue_loads(blockIdx.x, 0);
+        prefetch_tmap(&tm_aqout);
+        if ((int)blockIdx.x < pp.nitems) {
+            issue_k(blockIdx.x, 0);
+            issue_q(blockIdx.x);
+            issue_v(blockIdx.x);
+        }
     }
     if ((int)blockIdx.x < pp.nitems) load_gates(blockIdx.x);
     if (warp == 0) tmem_alloc(s_tmem, P_TM_COLS);
@@ -154,7 +184,7 @@ __global__ void __launch_bounds__(NT, 2) prep_gdn_kernel(const __grid_constant__
     tc_fence_after();
     const uint32_t tmem = *s_tmem;
     const uint32_t lane_base = (uint32_t)((warp & 3) * 32) << 16;
-    uint32_t ph_tma0 = 0, ph_tma1 = 0, ph_mma = 0;
+    uint32_t ph_tma0 = 0, ph_tma1 = 0, ph_mma = 0, ph_q = 0, ph_v = 0;
     bool ok = true;
 
 #define GDR_WAIT(bar, ph)                                                   \
@@ -171,7 +201,7 @@ __global__ void __launch_bounds__(NT, 2) prep_gdn_kernel(const __grid_constant__
         const int t0 = ci * C;
         const int n = min(C, T - t0);
         const uint32_t kb = sbase + P_OFF_K + buf * 16384u;
-        const uint32_t vb = sbase + P_OFF_V + buf * 16384u;
+        const uint32_t vb = sbase + P_OFF_V;
         GDR_TRACE_P(0);
         // this item's gates (prefetched into registers) -> shared memory
         if (tid < C) {
@@ -179,9 +209,9 @@ __global__ void __launch_bounds__(NT, 2) prep_gdn_kernel(const __grid_constant__
             s_alpha[tid] = valid ? bits_to_f32(g_a) : 1.f;
             s_beta[tid] = valid ? bits_to_f32(g_b) : 0.f;
         }
-        // the next item's inputs: its buffer was last read by this CTA's previous P2
+        // the next item's K: its buffer was last read by this CTA's previous P2
         const int next = item + gridDim.x;
-        if (tid == 0 && next < pp.nitems) issue_loads(next, buf ^ 1);
+        if (tid == 0 && next < pp.nitems) issue_k(next, buf ^ 1);
         if (next < pp.nitems) load_gates(next);
         __syncthreads();
 
@@ -204,9 +234,10 @@ __global__ void __launch_bounds__(NT, 2) prep_gdn_kernel(const __grid_constant__
         }
         if (buf == 0) GDR_WAIT(&bar_tma[0], ph_tma0);  // also publishes the scan
         else GDR_WAIT(&bar_tma[1], ph_tma1);
+        GDR_WAIT(bar_q, ph_q);
         GDR_TRACE_P(1);
 
-        // ---- D1 = K K^T -----------------------------------------------------
+        // ---- D1 = K K^T (lanes 0..63), Q K^T (lanes 64..127, columns 64..127) ----
         if (tid == 0) {
             tc_fence_after();
             const uint32_t id = idesc_bf16(128, 64, 0, 0);
@@ -215,6 +246,8 @@ __global__ void __launch_bounds__(NT, 2) prep_gdn_kernel(const __grid_constant__
                 const uint32_t koff = (ks >> 2) * 8192u + (ks & 3) * 32u;
                 mma_bf16(tmem + P_TM_D1, sdesc_sw128(kb + koff, 16, 1024), sdesc_sw128(kb + koff, 16, 1024),
                          id, ks > 0);
+                mma_bf16(tmem + P_TM_DQ, sdesc_sw128(sbase + P_OFF_Q - 8192 + koff, 16, 1024),
+                         sdesc_sw128(kb + koff, 16, 1024), id, ks > 0);
             }
             mma_commit(bar_mma);
             // the previous item's stores must have left the staging tiles (A32, T32)
@@ -255,8 +288,31 @@ __global__ void __launch_bounds__(NT, 2) prep_gdn_kernel(const __grid_constant__
                     for (int j = 0; j < 16; ++j) at[j * 16 + rr] = d[j];
                 }
             }
+        } else {
+            // Aq_tj = (q_t . k_j) 2^(l_t - l_j), j <= t (bf16) -> staging over Q's first tile
+            const int t = row - 64;
+            float d[32];
+            tmem_ld32(tmem + lane_base + P_TM_DQ + wg * 32, d);
+            const float lt = s_l[t];
+#pragma unroll
+            for (int c8 = 0; c8 < 4; ++c8) {
+                const int j0 = wg * 32 + c8 * 8;
+                const float4 la = *reinterpret_cast<const float4*>(s_l + j0);
+                const float4 lb = *reinterpret_cast<const float4*>(s_l + j0 + 4);
+                const float lj[8] = {la.x, la.y, la.z, la.w, lb.x, lb.y, lb.z, lb.w};
+                float x[8];
+#pragma unroll
+                for (int e = 0; e < 8; ++e)
+                    x[e] = j0 + e <= t ? d[c8 * 8 + e] * ex2_approx(fminf(lt - lj[e], 0.f)) : 0.f;
+                st_chunk(sm + P_OFF_Q, sw128_chunk(t, wg * 4 + c8, 64), x);
+            }
         }
+        fence_proxy_async();
         __syncthreads();
+        if (tid == 0) {
+            tma_store_4d(&tm_aqout, sm + P_OFF_Q, 0, h, t0, bb);
+            bulk_commit_group();
+        }
         GDR_TRACE_P(3);
 
         // ---- T = (I + A)^-1; L = T Diag(beta g), PRE = T Diag(beta) (bf16) ----------
@@ -288,11 +344,14 @@ __global__ void __launch_bounds__(NT, 2) prep_gdn_kernel(const __grid_constant__
         }
         fence_proxy_async();
         tc_fence_before();
-        __syncthreads();
+        GDR_WAIT(bar_v, ph_v);  // V landed during the solve (also publishes L, PRE)
 
         // ---- D2 = L K (-> W), D3 = PRE V (-> P) ----------------------------------
         if (tid == 0) {
             tc_fence_after();
+            // the Aq store has read its staging tile: the next item's Q may land there
+            bulk_wait_group_read0();
+            if (next < pp.nitems) issue_q(next);
             const uint32_t idW = idesc_bf16(128, 128, 0, 1);
             const uint32_t idP = idesc_bf16(128, dv, 0, 1);
 #pragma unroll
@@ -307,6 +366,7 @@ __global__ void __launch_bounds__(NT, 2) prep_gdn_kernel(const __grid_constant__
         GDR_TRACE_P(5);
         GDR_WAIT(bar_mma, ph_mma);
         tc_fence_after();
+        if (tid == 0 && next < pp.nitems) issue_v(next);  // the P product has read V
         GDR_TRACE_P(6);
 
         // ---- -W and P -> staging tiles (rows 0..63; each warpgroup half the columns)
@@ -360,23 +420,23 @@ finish:
 // ---- pass 2 shared memory ---------------------------------------------------
 // Inputs are triple-buffered (chunk ci + 2 loads while chunk ci runs); a stage
 // holds [Q ; -W] (Q in rows 0..63, -W in rows 64..127, two 64-column blocks
-// of 16 KB), K and this CTA's 64 columns of P.
+// of 16 KB), K, this CTA's 64 columns of P and Aq (from the first pass; rows
+// 0..63 of the Aq U operand, whose rows 64..127 are the next 8 KB, unused).
 constexpr int S_NBUF = 3;
-constexpr uint32_t S_STAGE = 57344;
+constexpr uint32_t S_STAGE = 65536;
 constexpr uint32_t S_ST_QW = 0;         // [Q ; -W] bf16 [128 x 128]
 constexpr uint32_t S_ST_K = 32768;      // K bf16 [64 x 128]
 constexpr uint32_t S_ST_P = 49152;      // P slice bf16 [64 x 64]
+constexpr uint32_t S_ST_AQ = 57344;     // Aq bf16 [64 x 64]
 constexpr uint32_t S_OFF_SBF = S_NBUF * S_STAGE;     // S bf16 [128 x 64] (B operand, MN-major)
-constexpr uint32_t S_OFF_AQ = S_OFF_SBF + 16384;     // Aq bf16 [64 x 64] (rows 0..63 of the
-                                                     // Aq U A operand; U below are its rows 64..127)
-constexpr uint32_t S_OFF_U = S_OFF_AQ + 8192;        // U bf16 [64 x 64] (B operand of Aq U)
+constexpr uint32_t S_OFF_U = S_OFF_SBF + 16384;      // U bf16 [64 x 64] (B operand of Aq U)
 constexpr uint32_t S_OFF_U2 = S_OFF_U + 8192;        // Diag(g_{n-1}/g) U (B operand of K^T U)
 constexpr uint32_t S_OFF_SMALL = S_OFF_U2 + 8192;
-constexpr uint32_t S_SMEM_BYTES = S_OFF_SMALL + 3072 + 1024;
+constexpr uint32_t S_SMEM_BYTES = S_OFF_SMALL + 2048 + 1024;
 // TMEM columns: D3 [Q S ; -W S] and D5 (Aq U, lanes 0..63) alternate between
 // two column sets by chunk parity, so chunk ci's outputs are written while
-// chunk ci + 1 runs; D1 = [Q ; -W] K^T (lanes 0..63: Q K^T); D4 = K^T U'.
-constexpr uint32_t S_TM_D3 = 0, S_TM_D1 = 128, S_TM_D4 = 192, S_TM_D5 = 256, S_TM_COLS = 512;
+// chunk ci + 1 runs; D4 = K^T U'.
+constexpr uint32_t S_TM_D3 = 0, S_TM_D4 = 192, S_TM_D5 = 256, S_TM_COLS = 512;
 // Threads: warps 0..7 compute (thread t < 256: state row t & 127, columns
 // 32 (t >> 7) .. + 31 of the CTA's 64); warp 8 issues every MMA and TMA load.
 constexpr int S_NT = 288;
@@ -403,15 +463,15 @@ __device__ __forceinline__ void mbar_arrive(uint64_t* bar) {
 // state are on the chain from one chunk to the next:
 //   D3 = [Q ; -W] S             (U = P - W S, lanes 64..127, by warps 2, 3, 6, 7)
 //   D4 = K^T Diag(g_{n-1}/g) U  (S <- g_{n-1} S + D4, all compute warps)
-// The output's products are queued between them and after them:
-//   D1 = [Q ; -W] K^T           (Aq = masked (Q K^T) . 2^(l_r - l_j), lanes 0..63,
-//                                by warps 0, 1, 4, 5 while warps 2, 3, 6, 7 form U)
-//   D5 = [Aq ; U] U             (lanes 0..63: Aq U; with Q S it gives O of the
-//                                chunk, written during the next chunk)
-// Warp 8 issues them in that order, each when its operands are in shared
-// memory (mbarriers u_ready, aq_ready, s_ready), so no compute warp waits on
-// MMA issue. Decay ratios are formed per element from the log2 prefix l
-// (exact for any alpha in (0, 1]: every factor used is at most 1).
+// The output's product follows D4:
+//   D5 = [Aq ; .] U             (lanes 0..63: Aq U, Aq = masked (Q K^T) . 2^(l_r - l_j)
+//                                formed by the first pass; with Q S it gives O of
+//                                the chunk, written during the next chunk)
+// Warp 8 issues them, each when its operands are in shared memory (mbarriers
+// u_ready, s_ready), so no compute warp waits on MMA issue. D5 commits to one
+// barrier per TMEM column set: a barrier completes every second chunk, so the
+// warps that wait for one chunk's output can never see the next completion of
+// the same barrier first.
 // Optional checkpoints for the backward pass, written off the chunk chain:
 // the fp32 state at every chunk start ([B, H, nchunks, 128, d_v]) and
 // U = P - W S of every token in fp32 ([B, T, H, d_v]; U = beta v - r, with r
@@ -427,7 +487,7 @@ template <bool CKPT>
 __global__ void __launch_bounds__(S_NT, 1) state_gdn_kernel(
     const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ CUtensorMap tm_k,
     const __grid_constant__ CUtensorMap tm_w, const __grid_constant__ CUtensorMap tm_p,
-    const Params p, const Ckpt ck) {
+    const __grid_constant__ CUtensorMap tm_aq, const Params p, const Ckpt ck) {
     extern __shared__ uint8_t smem_raw[];
     uint8_t* sm = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) &
                                              ~uintptr_t(1023));
@@ -442,37 +502,35 @@ __global__ void __launch_bounds__(S_NT, 1) state_gdn_kernel(
     const int nchunks = (T + C - 1) / C;
 
     // per-chunk factors, three sets by chunk % 3 (written one chunk ahead,
-    // read up to one chunk behind): l (log2 prefix), g = 2^l,
+    // read up to one chunk behind): g = 2^l (l the log2 prefix),
     // gcr = 2^(l_{n-1} - l), and g_{n-1}
-    float* s_l3 = reinterpret_cast<float*>(sm + S_OFF_SMALL);   // [3][64]
-    float* s_g3 = s_l3 + 192;                                    // [3][64]
-    float* s_gcr3 = s_l3 + 384;                                  // [3][64]
-    float* s_gC3 = s_l3 + 576;                                   // [3][4]
-    uint64_t* bar_tma = reinterpret_cast<uint64_t*>(sm + S_OFF_SMALL + 2752);  // [3]
+    float* s_g3 = reinterpret_cast<float*>(sm + S_OFF_SMALL);   // [3][64]
+    float* s_gcr3 = s_g3 + 192;                                  // [3][64]
+    float* s_gC3 = s_g3 + 384;                                   // [3][4]
+    uint64_t* bar_tma = reinterpret_cast<uint64_t*>(sm + S_OFF_SMALL + 1600);  // [3]
     uint64_t* bar_w = bar_tma + 3;      // MMA commits
-    uint64_t* bar_q = bar_tma + 4;
-    uint64_t* bar_k = bar_tma + 5;
-    uint64_t* bar_a = bar_tma + 6;
-    uint64_t* bar_drain = bar_tma + 7;
-    uint64_t* u_ready = bar_tma + 8;    // operands written (compute -> issuer)
-    uint64_t* aq_ready = bar_tma + 9;
-    uint64_t* s_ready = bar_tma + 10;
-    uint32_t* s_tmem = reinterpret_cast<uint32_t*>(sm + S_OFF_SMALL + 2880);
+    uint64_t* bar_k = bar_tma + 4;
+    uint64_t* bar_drain = bar_tma + 5;
+    uint64_t* u_ready = bar_tma + 6;    // operands written (compute -> issuer)
+    uint64_t* s_ready = bar_tma + 7;
+    uint64_t* bar_a0 = bar_tma + 8;     // D5 commits, one per TMEM column set
+    auto bar_a = [&](int set) { return bar_a0 + set; };
+    uint32_t* s_tmem = reinterpret_cast<uint32_t*>(sm + S_OFF_SMALL + 1696);
     if (tid == 0) {
         for (int i = 0; i < 3; ++i) mbar_init(&bar_tma[i], 1);
         mbar_init(bar_w, 1);
-        mbar_init(bar_q, 1);
         mbar_init(bar_k, 1);
-        mbar_init(bar_a, 1);
+        mbar_init(bar_a(0), 1);
+        mbar_init(bar_a(1), 1);
         mbar_init(bar_drain, 1);
         mbar_init(u_ready, 128);
-        mbar_init(aq_ready, 128);
         mbar_init(s_ready, 1);
         fence_barrier_init();
         prefetch_tmap(&tm_q);
         prefetch_tmap(&tm_k);
         prefetch_tmap(&tm_w);
         prefetch_tmap(&tm_p);
+        prefetch_tmap(&tm_aq);
     }
     if (warp == 0) tmem_alloc(s_tmem, S_TM_COLS);
     tc_fence_before();
@@ -518,11 +576,8 @@ __global__ void __launch_bounds__(S_NT, 1) state_gdn_kernel(
         }
         const float l1 = x, l0v = x - la1;
         const float last = __shfl_sync(0xffffffffu, l1, 31);
-        float* l = s_l3 + s3 * 64;
         float* g = s_g3 + s3 * 64;
         float* gcr = s_gcr3 + s3 * 64;
-        l[2 * lane] = l0v;
-        l[2 * lane + 1] = l1;
         g[2 * lane] = ex2_approx(l0v);
         g[2 * lane + 1] = ex2_approx(l1);
         gcr[2 * lane] = ex2_approx(last - l0v);
@@ -533,7 +588,7 @@ __global__ void __launch_bounds__(S_NT, 1) state_gdn_kernel(
     auto issue_loads = [&](int ci) {
         const int t0 = ci * C, buf = ci % S_NBUF;
         uint8_t* st = sm + buf * S_STAGE;
-        mbar_expect_tx(&bar_tma[buf], 7u * 8192u);
+        mbar_expect_tx(&bar_tma[buf], 8u * 8192u);
         // [Q ; -W]: each 64-column block holds 128 rows (q rows 0..63, -W rows 64..127)
         tma_load_4d(st + S_ST_QW, &tm_q, &bar_tma[buf], 0, hq, t0, bb);
         tma_load_4d(st + S_ST_QW + 16384, &tm_q, &bar_tma[buf], 64, hq, t0, bb);
@@ -542,6 +597,7 @@ __global__ void __launch_bounds__(S_NT, 1) state_gdn_kernel(
         tma_load_4d(st + S_ST_K, &tm_k, &bar_tma[buf], 0, hq, t0, bb);
         tma_load_4d(st + S_ST_K + 8192, &tm_k, &bar_tma[buf], 64, hq, t0, bb);
         tma_load_4d(st + S_ST_P, &tm_p, &bar_tma[buf], v0, h, t0, bb);
+        tma_load_4d(st + S_ST_AQ, &tm_aq, &bar_tma[buf], 0, h, t0, bb);
     };
 
     // the state's bf16 copy is read by the first MMA (async proxy)
@@ -580,27 +636,28 @@ __global__ void __launch_bounds__(S_NT, 1) state_gdn_kernel(
             tc_fence_after();
             if (lane == 0) {
                 const uint32_t idS = idesc_bf16(128, NV, 0, 1);
-                const uint32_t idK = idesc_bf16(128, 64, 0, 0);
                 const uint32_t d3 = S_TM_D3 + (uint32_t)par * 64u;
-                // D3 and D1 k-step by k-step: two independent accumulators in flight
 #pragma unroll
                 for (int ks = 0; ks < 8; ++ks) {
                     const uint32_t koff = (ks >> 2) * 16384u + (ks & 3) * 32u;
-                    const uint32_t kkoff = (ks >> 2) * 8192u + (ks & 3) * 32u;
                     mma_bf16(tmem + d3, sdesc_sw128(qwb + koff, 16, 1024),
                              sdesc_sw128(sbase + S_OFF_SBF + ks * 2048u, 8192, 1024), idS, ks > 0);
-                    if (ks == 7) mma_commit(bar_w);
-                    mma_bf16(tmem + S_TM_D1, sdesc_sw128(qwb + koff, 16, 1024),
-                             sdesc_sw128(kb + kkoff, 16, 1024), idK, ks > 0);
                 }
-                mma_commit(bar_q);
-                // chunk ci + 2's inputs go to the stage of chunk ci - 1, all of whose
-                // readers finished before the state copy of chunk ci was written
-                if (ci + 2 < nchunks) issue_loads(ci + 2);
+                mma_commit(bar_w);
             }
+            __syncwarp();
+            // chunk ci + 2's inputs go to the stage of chunk ci - 1: its Aq tile's
+            // reader (D5 of chunk ci - 1) has finished; every other reader of that
+            // stage finished before the state copy of chunk ci was written
+            if (ci > 0) {
+                iok = __all_sync(0xffffffffu,
+                                 mbar_wait(bar_a((ci - 1) & 1), (uint32_t)(((ci - 1) >> 1) & 1)) && iok);
+                if (!iok) break;
+            }
+            if (lane == 0 && ci + 2 < nchunks) issue_loads(ci + 2);
             if (ci + 2 < nchunks) loads_issued = ci + 3;
             __syncwarp();
-            // ---- D4 = K^T U' once U is written --------------------------------------
+            // ---- D4 = K^T U', then D5 = [Aq ; .] U, once U is written --------------------
             iok = __all_sync(0xffffffffu, mbar_wait(u_ready, ph) && iok);
             if (!iok) break;
             GDR_TRACE_S(1, 256);
@@ -612,21 +669,13 @@ __global__ void __launch_bounds__(S_NT, 1) state_gdn_kernel(
                     mma_bf16(tmem + S_TM_D4, sdesc_sw128(kb + ks * 2048u, 8192, 1024),
                              sdesc_sw128(sbase + S_OFF_U2 + ks * 2048u, 8192, 1024), idM, ks > 0);
                 mma_commit(bar_k);
-            }
-            __syncwarp();
-            // ---- D5 = [Aq ; U] U once Aq is written ---------------------------------
-            iok = __all_sync(0xffffffffu, mbar_wait(aq_ready, ph) && iok);
-            if (!iok) break;
-            GDR_TRACE_S(2, 256);
-            tc_fence_after();
-            if (lane == 0) {
                 const uint32_t idA = idesc_bf16(128, NV, 0, 1);
                 const uint32_t d5 = S_TM_D5 + (uint32_t)par * 64u;
 #pragma unroll
                 for (int ks = 0; ks < 4; ++ks)
-                    mma_bf16(tmem + d5, sdesc_sw128(sbase + S_OFF_AQ + ks * 32u, 16, 1024),
+                    mma_bf16(tmem + d5, sdesc_sw128(stb + S_ST_AQ + ks * 32u, 16, 1024),
                              sdesc_sw128(sbase + S_OFF_U + ks * 2048u, 8192, 1024), idA, ks > 0);
-                mma_commit(bar_a);
+                mma_commit(bar_a(par));
             }
             __syncwarp();
         }
@@ -683,9 +732,9 @@ __global__ void __launch_bounds__(S_NT, 1) state_gdn_kernel(
                     *reinterpret_cast<float4*>(dst + jj) = make_float4(S[jj], S[jj + 1], S[jj + 2], S[jj + 3]);
             }
             if (lo) {
-                // ---- O of the previous chunk, the next decay scan, Aq -----------------------
+                // ---- O of the previous chunk, the next decay scan ---------------------------
                 if (ci > 0) {
-                    w_ok = mbar_wait(bar_a, (uint32_t)((ci - 1) & 1)) && w_ok;
+                    w_ok = mbar_wait(bar_a((ci - 1) & 1), (uint32_t)(((ci - 1) >> 1) & 1)) && w_ok;
                     tc_fence_after();
                     store_o(ci - 1);
                 }
@@ -693,31 +742,6 @@ __global__ void __launch_bounds__(S_NT, 1) state_gdn_kernel(
                     decay_scan(ci + 1);
                     if (ci + 2 < nchunks) load_alpha(ci + 2);
                 }
-                w_ok = mbar_wait(bar_q, ph) && w_ok;
-                tc_fence_after();
-                GDR_TRACE_S(3, 0);
-                {
-                    const int r = row;
-                    float d[32];
-                    tmem_ld32(tmem + lane_base + S_TM_D1 + wg * 32, d);
-                    const float* l = s_l3 + s3 * 64;
-                    const float lr = l[r];
-#pragma unroll
-                    for (int c8 = 0; c8 < 4; ++c8) {
-                        const int j0 = wg * 32 + c8 * 8;
-                        float x[8];
-                        const float4 la = *reinterpret_cast<const float4*>(l + j0);
-                        const float4 lb = *reinterpret_cast<const float4*>(l + j0 + 4);
-                        const float lj[8] = {la.x, la.y, la.z, la.w, lb.x, lb.y, lb.z, lb.w};
-#pragma unroll
-                        for (int e = 0; e < 8; ++e)
-                            x[e] = j0 + e <= r ? d[c8 * 8 + e] * ex2_approx(fminf(lr - lj[e], 0.f)) : 0.f;
-                        st_chunk(sm + S_OFF_AQ, sw128_chunk(r, wg * 4 + c8, 128), x);
-                    }
-                }
-                fence_proxy_async();
-                tc_fence_before();
-                mbar_arrive(aq_ready);
                 GDR_TRACE_S(4, 0);
             } else {
                 // ---- U = P - W S (lanes 64..127 of D3) -> U and U' -------------------------
@@ -773,7 +797,7 @@ __global__ void __launch_bounds__(S_NT, 1) state_gdn_kernel(
         }
         if (ci < nchunks) ok = false;  // a wait gave up
         if (ok && lo && nchunks > 0) {
-            ok = mbar_wait(bar_a, (uint32_t)((nchunks - 1) & 1));
+            ok = mbar_wait(bar_a((nchunks - 1) & 1), (uint32_t)(((nchunks - 1) >> 1) & 1));
             tc_fence_after();
             if (ok) store_o(nchunks - 1);
         }
@@ -794,10 +818,11 @@ __global__ void __launch_bounds__(S_NT, 1) state_gdn_kernel(
 }  // namespace twopass
 
 size_t twopass_workspace_bytes(int B, int T, int H, int dv) {
-    return (size_t)B * T * H * (chunkc::DK + dv) * sizeof(__nv_bfloat16);
+    return (size_t)B * T * H * (chunkc::DK + dv + chunkc::C) * sizeof(__nv_bfloat16);
 }
 
-// maps: q, k, v, then the workspace maps -W ([B,T,H,128]) and P ([B,T,H,d_v]).
+// maps: q, k, v, then the workspace maps -W ([B,T,H,128]), P ([B,T,H,d_v]) and
+// Aq ([B,T,H,64], the chunk's masked, decay-scaled Q K^T block row of each token).
 // ckS, up: the backward pass's checkpoints (struct Ckpt; both or neither), or NULL:
 // with them, o is not written.
 cudaError_t launch_chunk_twopass_gdn(const CUtensorMap* maps, const CUtensorMap* ws_maps, void* ws,
@@ -818,7 +843,8 @@ cudaError_t launch_chunk_twopass_gdn(const CUtensorMap* maps, const CUtensorMap*
     if ((e = cudaGetDevice(&dev)) != cudaSuccess) return e;
     if ((e = cudaDeviceGetAttribute(&nsm, cudaDevAttrMultiProcessorCount, dev)) != cudaSuccess) return e;
     const int grid = min(pp.nitems, 2 * nsm);  // two resident CTAs per SM
-    prep_gdn_kernel<<<grid, NT, P_SMEM_BYTES, st>>>(maps[1], maps[2], ws_maps[0], ws_maps[1], pp);
+    prep_gdn_kernel<<<grid, NT, P_SMEM_BYTES, st>>>(maps[0], maps[1], maps[2], ws_maps[0], ws_maps[1],
+                                                    ws_maps[2], pp);
     e = cudaGetLastError();
     if (e != cudaSuccess) return e;
 
@@ -845,8 +871,10 @@ cudaError_t launch_chunk_twopass_gdn(const CUtensorMap* maps, const CUtensorMap*
     Ckpt ck;
     ck.ckS = ckS;
     ck.up = up;
-    return ckpt ? cudaLaunchKernelEx(&cfg, state_gdn_kernel<true>, maps[0], maps[1], ws_maps[0], ws_maps[1], p, ck)
-                : cudaLaunchKernelEx(&cfg, state_gdn_kernel<false>, maps[0], maps[1], ws_maps[0], ws_maps[1], p, ck);
+    return ckpt ? cudaLaunchKernelEx(&cfg, state_gdn_kernel<true>, maps[0], maps[1], ws_maps[0], ws_maps[1],
+                                     ws_maps[2], p, ck)
+                : cudaLaunchKernelEx(&cfg, state_gdn_kernel<false>, maps[0], maps[1], ws_maps[0], ws_maps[1],
+                                     ws_maps[2], p, ck);
 }
 
 }  // namespace gdr

@@ -160,8 +160,9 @@ gdr_status gdr_chunk_fwd_grouped(const void* q, const void* k, const void* v,
  * path needs for this shape and gate form, or 0 when it has none. Two-pass
  * shapes: dtype GDR_BF16, d_k = 128, d_v in {64, 128}, T >= 1, an erase gate
  * (b_kind != GDR_GATE_NONE). Sizes, in bytes, with N = B*T*H:
- *   scalar alpha, tied scalar beta (Gated DeltaNet): 2 N (d_k + d_v)
- *     (per-token rows of -W = -T Diag(beta g) K and of T Diag(beta) V);
+ *   scalar alpha, tied scalar beta (Gated DeltaNet): 2 N (d_k + d_v + 64)
+ *     (per-token rows of -W = -T Diag(beta g) K, of T Diag(beta) V and of
+ *     the chunk's masked, decay-scaled q k^T block);
  *   every other form: the per-token rows of -W 2^ref, q.g, k.g_{n-1}/g,
  *     the masked (q.rowf)(k.colf)^T block row and P (plus, with independent
  *     b and w, w.k.g_{n-1}/g and the masked (q.rowf)(w.k.colf)^T row), in
@@ -312,8 +313,9 @@ size_t gdr_chunk_bwd_grouped_workspace_size(int B, int T, int H_qk, int H, int d
  * chunk-start states and chunk-end state gradients (2 x B H ceil(T/64) d_k
  * d_v), r_t and dr_t of every token (2 x B T H d_v), and scalar-gate partial
  * sums (3 x ceil(d_k / RB) x B T H, RB = 128 / (d_v / 8 rounded up to a power
- * of two)), and when d_k = d_v = 128 the forward's per-token -W and P rows
- * (B T H (d_k + d_v) bf16), each rounded up to 256 bytes. Host-only;
+ * of two)), and when d_k = d_v = 128 the forward's per-token -W, P and
+ * q k^T block rows
+ * (B T H (d_k + d_v + 64) bf16), each rounded up to 256 bytes. Host-only;
  * launches nothing. */
 size_t gdr_chunk_bwd_workspace_size(int B, int T, int H, int d_k, int d_v);
 

@@ -106,8 +106,9 @@ def test_binding_raises_on_error_status():
 
 
 @pytest.mark.parametrize("shape,kinds,expect", [
-    ((4, 4096, 16, 128, 128), (1, 1, 3), 4 * 4096 * 16 * (128 + 128) * 2),   # GDN form
-    ((1, 100, 2, 128, 64), (1, 1, 3), 1 * 100 * 2 * (128 + 64) * 2),
+    # GDN form: per-token rows of -W (d_k), P (d_v) and the chunk's Aq block (64)
+    ((4, 4096, 16, 128, 128), (1, 1, 3), 4 * 4096 * 16 * (128 + 128 + 64) * 2),
+    ((1, 100, 2, 128, 64), (1, 1, 3), 1 * 100 * 2 * (128 + 64 + 64) * 2),
     ((1, 64, 1, 128, 256), (1, 1, 3), 0),          # d_v > 128: single pass only
     ((1, 64, 1, 128, 128), (2, 1, 3), 3 * 16384 + 8192 + 16384 + 512 + 65536),   # KDA form
     ((1, 100, 2, 128, 64), (2, 2, 2), 4 * 51200 + 3 * 25600 + 2048 + 65536),      # GDN-2 form
@@ -177,7 +178,7 @@ def r256(x):
     # checkpoints of S and G, r and dr per token, scalar-gate partials (16 row blocks of
     # 8), and at d_k = d_v = 128 the forward's -W and P rows (bf16)
     ((4, 4096, 16, 128, 128), 2 * 4 * 16 * 64 * 128 * 128 * 4 + 2 * 4 * 4096 * 16 * 128 * 4
-     + 3 * 16 * 4 * 4096 * 16 * 4 + 4 * 4096 * 16 * (128 + 128) * 2),
+     + 3 * 16 * 4 * 4096 * 16 * 4 + 4 * 4096 * 16 * (128 + 128 + 64) * 2),
     # d_v = 32: 4 threads per row, 32 rows per block, 2 blocks
     ((1, 65, 2, 64, 32), 2 * 2 * 2 * 64 * 32 * 4 + 2 * r256(65 * 2 * 32 * 4) + r256(3 * 2 * 65 * 2 * 4)),
     ((1, 0, 2, 64, 32), 0),

@@ -209,9 +209,9 @@ def test_two_pass_matches_oracle_and_single_pass(cuda_device, family, T, dv):
 
 
 def test_two_pass_workspace_is_used(cuda_device):
-    """The two-pass path writes the per-token rows of -W and P into the
+    """The two-pass path writes the per-token rows of -W, P and Aq into the
     caller's workspace: row t of -W is -(T Diag(beta g) K)_t, so a token whose
-    beta is 0 gets a zero row in both."""
+    beta is 0 gets a zero row in both -W and P; Aq is lower triangular."""
     wl = small("gdn", T=130, B=1, H=2, seed=17)
     inp = make_chunk_inputs(wl)
     inp["b"][0, 5, 1] = 0.0
@@ -219,16 +219,20 @@ def test_two_pass_workspace_is_used(cuda_device):
     q, k, v, a, b = (inp[x].to(dev) for x in ("q", "k", "v", "alpha", "b"))
     from gated_delta_rule_147_b200 import workspace_bytes
     nbytes = workspace_bytes(q, v, a, b, TIED)
-    assert nbytes == 1 * 130 * 2 * (128 + 128) * 2
+    assert nbytes == 1 * 130 * 2 * (128 + 128 + 64) * 2
     ws = torch.full((nbytes,), 0x7F, dtype=torch.uint8, device=dev)
     chunk_fwd(q, k, v, a, b, TIED, None, workspace=ws)
     torch.cuda.synchronize()
     half = 130 * 2 * 128
     wneg = ws[: half * 2].view(torch.bfloat16).view(1, 130, 2, 128).float().cpu()
-    p = ws[half * 2:].view(torch.bfloat16).view(1, 130, 2, 128).float().cpu()
+    p = ws[half * 2: half * 4].view(torch.bfloat16).view(1, 130, 2, 128).float().cpu()
+    aq = ws[half * 4:].view(torch.bfloat16).view(1, 130, 2, 64).float().cpu()
     assert torch.all(wneg[0, 5, 1] == 0) and torch.all(p[0, 5, 1] == 0)
-    assert torch.isfinite(wneg).all() and torch.isfinite(p).all()
+    assert torch.isfinite(wneg).all() and torch.isfinite(p).all() and torch.isfinite(aq).all()
     assert wneg.abs().sum() > 0 and p.abs().sum() > 0
+    for t in (0, 5, 63, 64, 100, 129):  # token t of a chunk: Aq row zero past its own position
+        j = t % 64
+        assert torch.all(aq[0, t, :, j + 1:] == 0) and torch.all(aq[0, t, :, j] != 0)
 
 
 @pytest.mark.parametrize("family", FAMILIES)

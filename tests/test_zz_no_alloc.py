@@ -18,7 +18,7 @@ KIND = {"none": 0, "scalar": 1, "channel": 2, "tied": 3}
 def test_oversize_is_rejected_before_any_device_work():
     cap = _lib.gdr_chunk_fwd_static_capacity()
     assert cap == 64 << 20
-    B, T, H = 8, 8192, 32   # GDN form needs B*T*H*(128 + 128)*2 bytes > 64 MiB
+    B, T, H = 8, 8192, 32   # GDN form needs B*T*H*(128 + 128 + 64)*2 bytes > 64 MiB
     need = _lib.gdr_chunk_fwd_workspace_size(B, T, H, 128, 128, GATE_SCALAR, GATE_SCALAR, GATE_TIED,
                                              GDR_BF16)
     assert need > cap
