@@ -349,9 +349,6 @@ __global__ void __launch_bounds__(NT, 2) prep_gdn_kernel(const __grid_constant__
         // ---- D2 = L K (-> W), D3 = PRE V (-> P) ----------------------------------
         if (tid == 0) {
             tc_fence_after();
-            // the Aq store has read its staging tile: the next item's Q may land there
-            bulk_wait_group_read0();
-            if (next < pp.nitems) issue_q(next);
             const uint32_t idW = idesc_bf16(128, 128, 0, 1);
             const uint32_t idP = idesc_bf16(128, dv, 0, 1);
 #pragma unroll
@@ -366,7 +363,11 @@ __global__ void __launch_bounds__(NT, 2) prep_gdn_kernel(const __grid_constant__
         GDR_TRACE_P(5);
         GDR_WAIT(bar_mma, ph_mma);
         tc_fence_after();
-        if (tid == 0 && next < pp.nitems) issue_v(next);  // the P product has read V
+        if (tid == 0 && next < pp.nitems) {
+            issue_v(next);            // the P product has read V
+            bulk_wait_group_read0();  // the Aq store has left its staging tile over Q
+            issue_q(next);
+        }
         GDR_TRACE_P(6);
 
         // ---- -W and P -> staging tiles (rows 0..63; each warpgroup half the columns)
