@@ -35,8 +35,9 @@ sys.path.insert(0, ROOT)
 
 METRIC = "gated-delta-rule fwd tokens/s and % roofline; decode state GB/s vs HBM peak"
 # Algorithmic work per token-head (2 flops per multiply-add) of the chunkwise
-# contractions at C = 64, d = 128: general gates and tied scalar beta.
-FLOPS_PER_TOKEN_HEAD = {"general": 281259, "tied": 182955}
+# contractions at C = 64, d = 128 with general gates (tied scalar beta:
+# workload_flops derives it from the head dims; 182,955 at d = 128).
+FLOPS_PER_TOKEN_HEAD = {"general": 281259}
 L2_BYTES = 126 * 2**20
 
 
@@ -50,6 +51,7 @@ KERNEL_SOURCES = {
                         _CSRC + "common.cuh"),
     "erasefree": (_CSRC + "chunk_erasefree_sm100.cu", _CSRC + "chunk_common.cuh",
                   _CSRC + "common.cuh"),
+    "twopass256": (_CSRC + "chunk_twopass256_sm100.cu", _CSRC + "chunk_common.cuh", _CSRC + "common.cuh"),
 }
 
 
@@ -58,13 +60,17 @@ KERNEL_NAMES = {
     "twopass": "gdr::twopass::prep_gdn_kernel + gdr::twopass::state_gdn_kernel (one call, two launches)",
     "erasefree": "gdr::erasefree::chunk_fwd_erasefree_kernel",
     "twopass_general": "gdr::twopass_g::prep_general_kernel + state_general_kernel (one call, two launches)",
+    "twopass256": "gdr::twopass256::prep_gdn256_kernel + state_gdn256_kernel (one call, two launches)",
 }
-LAUNCHES_PER_CALL = {"general": 1, "twopass": 2, "erasefree": 1, "twopass_general": 2}
+LAUNCHES_PER_CALL = {"general": 1, "twopass": 2, "erasefree": 1, "twopass_general": 2, "twopass256": 2}
 
 
 def kernel_family(wl) -> str:
     if wl.b == "none":
         return "erasefree"
+    gdn = wl.alpha == "scalar" and wl.b == "scalar" and wl.w == "tied"
+    if wl.dtype == "bf16" and wl.dk == 256 and gdn and wl.dv % 64 == 0 and wl.dv <= 256 and wl.T > 0:
+        return "twopass256"
     if wl.dtype == "bf16" and wl.dk == 128 and wl.dv in (64, 128) and wl.T > 0:
         if wl.alpha == "scalar" and wl.b == "scalar" and wl.w == "tied":
             return "twopass"
@@ -124,8 +130,13 @@ def workload_flops(wl):
         C = 64
         per = 2 * (2 * wl.dk * wl.dv + C * wl.dv + C * wl.dk // 2)
         return per * wl.B * wl.T * wl.H
-    kind = "tied" if wl.w == "tied" and wl.b == "scalar" else "general"
-    return FLOPS_PER_TOKEN_HEAD[kind] * wl.B * wl.T * wl.H
+    if wl.w == "tied" and wl.b == "scalar":
+        # per token-head: K K^T, Q K^T, -W (C d_k each), P, Aq U (C d_v each),
+        # W S, Q S, the state step (d_k d_v each) and the solve (C^2 / 3)
+        C = 64
+        per = round(2 * (3 * wl.dk * wl.dv + C * (3 * wl.dk + 2 * wl.dv) + C * C / 3))
+        return per * wl.B * wl.T * wl.H
+    return FLOPS_PER_TOKEN_HEAD["general"] * wl.B * wl.T * wl.H
 
 
 class ClockSampler:
@@ -434,7 +445,7 @@ def run_ours(args):
         e2e_ms, h2d, d2h = time_chunk_e2e(inp, wl, dev, max(3, args.steps // 2), args.warmup)
         e2e_steps = max(3, args.steps // 2)
         other = {}
-        for name in ("kda", "gdn2", "gla", "gdn_gqa"):
+        for name in ("kda", "gdn2", "gla", "gdn_gqa", "gdn256"):
             w2 = WORKLOADS[name]
             _, _, tot2, per2 = time_chunk(w2, dev, max(3, args.steps // 2), args.warmup, lambda: None)
             a2 = statistics.fmean(per2)

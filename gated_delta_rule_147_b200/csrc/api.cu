@@ -26,6 +26,11 @@ cudaError_t launch_chunk_twopass_gdn(const CUtensorMap* maps, const CUtensorMap*
                                      const void* alpha, const void* beta, const float* S0, void* o,
                                      float* ST, int* d_status, int B, int T, int H, int dv, int group,
                                      cudaStream_t st, float* ckS = nullptr, float* up = nullptr);
+size_t twopass256_workspace_bytes(int B, int T, int H, int dv);
+cudaError_t launch_chunk_twopass_gdn256(const CUtensorMap* maps, const CUtensorMap* ws_maps,
+                                        const void* alpha, const void* beta, const float* S0, void* o,
+                                        float* ST, int* d_status, int B, int T, int H, int dv, int group,
+                                        cudaStream_t st);
 size_t twopass_general_workspace_bytes(int B, int T, int H, int dv, bool untied);
 cudaError_t launch_chunk_twopass_general(const CUtensorMap* maps,
                                          bool (*make_map)(CUtensorMap*, const void*, int, int, int, int),
@@ -100,18 +105,23 @@ namespace {
 // Two-pass paths (per-chunk factors of all chunks in parallel, then the state
 // pass) exist for the tensor-core shape with an erase gate and d_v <= 128:
 // the Gated DeltaNet form (scalar decay, tied scalar beta) has its own pair of
-// kernels, every other gate form the general pair.
-enum TwoPass { TP_NONE = 0, TP_GDN = 1, TP_GENERAL = 2 };
+// kernels, every other gate form the general pair. At d_k = 256 the Gated
+// DeltaNet form has a pair of its own (d_v a multiple of 64 up to 256).
+enum TwoPass { TP_NONE = 0, TP_GDN = 1, TP_GENERAL = 2, TP_GDN256 = 3 };
 
 TwoPass twopass_kind(int T, int d_k, int d_v, int ak, int bk, int wk, int dtype) {
-    if (T <= 0 || dtype != GDR_BF16 || d_k != 128 || !(d_v == 64 || d_v == 128)) return TP_NONE;
+    if (T <= 0 || dtype != GDR_BF16) return TP_NONE;
+    const bool gdn = ak == GDR_GATE_SCALAR && bk == GDR_GATE_SCALAR && wk == GDR_GATE_TIED;
+    if (d_k == 256) return gdn && d_v % 64 == 0 && d_v >= 64 && d_v <= 256 ? TP_GDN256 : TP_NONE;
+    if (d_k != 128 || !(d_v == 64 || d_v == 128)) return TP_NONE;
     if (bk == GDR_GATE_NONE) return TP_NONE;  // erase-free: single pass, no solve
-    if (ak == GDR_GATE_SCALAR && bk == GDR_GATE_SCALAR && wk == GDR_GATE_TIED) return TP_GDN;
+    if (gdn) return TP_GDN;
     return TP_GENERAL;
 }
 
 size_t twopass_bytes(TwoPass kind, int B, int T, int H, int d_v, int bk, int wk) {
     if (kind == TP_GDN) return gdr::twopass_workspace_bytes(B, T, H, d_v);
+    if (kind == TP_GDN256) return gdr::twopass256_workspace_bytes(B, T, H, d_v);
     if (kind == TP_GENERAL)
         return gdr::twopass_general_workspace_bytes(B, T, H, d_v,
                                                     !(wk == GDR_GATE_TIED && bk == GDR_GATE_SCALAR));
@@ -229,6 +239,20 @@ gdr_status chunk_fwd_impl(const void* q, const void* k, const void* v, const voi
         else
             e = gdr::launch_chunk_sm100(maps, q, k, v, alpha, b, w, alpha_kind, b_kind, w_kind, tied, S0, o,
                                         S_T, d_status, B, T, H, d_v, group, st);
+    } else if (tp == TP_GDN256) {
+        if (!encoder()) return GDR_ERR_NO_DEVICE;
+        CUtensorMap maps[3], ws_maps[4];
+        const size_t n = (size_t)B * T * H;
+        const uint8_t* pbase = reinterpret_cast<const uint8_t*>(workspace) + n * d_k * sizeof(uint16_t);
+        const uint8_t* aqbase = pbase + n * d_v * sizeof(uint16_t);
+        const uint8_t* ktbase = aqbase + n * 64 * sizeof(uint16_t);
+        if (!make_map(&maps[0], q, B, T, H_qk, d_k) || !make_map(&maps[1], k, B, T, H_qk, d_k) ||
+            !make_map(&maps[2], v, B, T, H, d_v) || !make_map(&ws_maps[0], workspace, B, T, H, d_k) ||
+            !make_map(&ws_maps[1], pbase, B, T, H, d_v) || !make_map(&ws_maps[2], aqbase, B, T, H, 64) ||
+            !make_map(&ws_maps[3], ktbase, B, T, H, d_k))
+            return GDR_ERR_INVALID_ARG;
+        e = gdr::launch_chunk_twopass_gdn256(maps, ws_maps, alpha, b, S0, o, S_T, d_status, B, T, H, d_v,
+                                             group, st);
     } else {
         e = gdr::launch_recurrent(q, k, v, alpha, b, w, alpha_kind, b_kind, w_kind, S0, o, S_T, B,
                                   T, H, d_k, d_v, dtype, group, st);

@@ -24,6 +24,9 @@ settings; "Erase-then-Delta Attention" abstract for the independent b/w gates;
          alpha; no erase (b = 0), w = 1; S0 = 0; seed 5 (erase-free path)
   gdn_gqa B=2,H=32 value heads with 16 q/k heads (value head h reads q/k
          head h // 2),T=4096,d=128 bf16; gdn gates per value head; seed 6
+  gdn256 B=2,H=16,T=4096,d_k=d_v=256 bf16 (the Gated DeltaNet head width of
+         "How Linear Attention Remembers", Table 1); gdn gates and
+         normalisation; S0 = 0; seed 7
 
 Value recipes: q,k,v ~ N(0,1); alpha = exp(-softplus(x)), x ~ N(0,1);
 sigmoid gates = 1/(1+exp(-x)), x ~ N(0,1). L2 normalisation is
@@ -91,6 +94,10 @@ WORKLOADS = {
     # ("How Linear Attention Remembers", Table 1)
     "gdn_gqa": ChunkWorkload("gdn_gqa", 2, 32, 4096, 128, 128, "bf16", "scalar", "scalar", "tied",
                              False, True, False, "sigmoid", 6, hq=16),
+    # Gated DeltaNet gates at the d_k = d_v = 256 head width ("How Linear
+    # Attention Remembers", Table 1)
+    "gdn256": ChunkWorkload("gdn256", 2, 16, 4096, 256, 256, "bf16", "scalar", "scalar", "tied",
+                            False, True, False, "sigmoid", 7),
 }
 
 

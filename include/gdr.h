@@ -102,7 +102,10 @@ typedef enum {
  * value. The result does not depend on it beyond rounding.
  * Paths: dtype GDR_BF16 with d_k = 128 and d_v a multiple of 64 runs the
  * tcgen05 tensor-core chunk kernel (bf16 operands, fp32 accumulation, fp32
- * state on chip). Every other supported shape (fp32, or 1 <= d_k <= 256 and
+ * state on chip); so does d_k = 256 (the Gated DeltaNet head width of "How
+ * Linear Attention Remembers", Table 1) with the Gated DeltaNet gates (scalar
+ * alpha, scalar beta, w tied), d_v a multiple of 64 up to 256 and a
+ * workspace. Every other supported shape (fp32, or 1 <= d_k <= 256 and
  * 1 <= d_v <= 1024 otherwise) runs an exact fp32 token-by-token CUDA kernel.
  * Decay: any alpha in (0, 1] is in range. With one decay per token (scalar
  * alpha) the tensor-core kernels form every ratio of decay products inside a
@@ -120,8 +123,8 @@ typedef enum {
  * shape and gate form and workspace is not NULL, the forward runs in two
  * passes: first the per-chunk WY factors of every chunk of every head in
  * parallel (written to the workspace), then the state pass over the chunks.
- * Otherwise one kernel does both per chunk. Both give the same result up to
- * rounding. The workspace must be 256-byte aligned and hold at least the
+ * Otherwise one kernel does both per chunk (at d_k = 256: the exact
+ * kernel). Both give the same result up to rounding. The workspace must be 256-byte aligned and hold at least the
  * queried size; its contents on entry are ignored and on exit undefined.
  * Returns GDR_OK, GDR_ERR_INVALID_ARG (B, H < 1, T < 0, bad kinds, NULL
  * data, workspace smaller than required), GDR_ERR_UNSUPPORTED (chunk != 64,
@@ -158,11 +161,14 @@ gdr_status gdr_chunk_fwd_grouped(const void* q, const void* k, const void* v,
 /*
  * gdr_chunk_fwd_workspace_size -- bytes of scratch gdr_chunk_fwd's two-pass
  * path needs for this shape and gate form, or 0 when it has none. Two-pass
- * shapes: dtype GDR_BF16, d_k = 128, d_v in {64, 128}, T >= 1, an erase gate
- * (b_kind != GDR_GATE_NONE). Sizes, in bytes, with N = B*T*H:
+ * shapes: dtype GDR_BF16, T >= 1, and either d_k = 128, d_v in {64, 128}
+ * with an erase gate (b_kind != GDR_GATE_NONE), or d_k = 256, d_v a multiple
+ * of 64 up to 256 with the Gated DeltaNet gates. Sizes, in bytes, with
+ * N = B*T*H:
  *   scalar alpha, tied scalar beta (Gated DeltaNet): 2 N (d_k + d_v + 64)
  *     (per-token rows of -W = -T Diag(beta g) K, of T Diag(beta) V and of
- *     the chunk's masked, decay-scaled q k^T block);
+ *     the chunk's masked, decay-scaled q k^T block); at d_k = 256 also the
+ *     rows of K~ = Diag(g_{n-1}/g) K: 2 N (2 d_k + d_v + 64);
  *   every other form: the per-token rows of -W 2^ref, q.g, k.g_{n-1}/g,
  *     the masked (q.rowf)(k.colf)^T block row and P (plus, with independent
  *     b and w, w.k.g_{n-1}/g and the masked (q.rowf)(w.k.colf)^T row), in

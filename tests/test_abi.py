@@ -110,6 +110,11 @@ def test_binding_raises_on_error_status():
     ((4, 4096, 16, 128, 128), (1, 1, 3), 4 * 4096 * 16 * (128 + 128 + 64) * 2),
     ((1, 100, 2, 128, 64), (1, 1, 3), 1 * 100 * 2 * (128 + 64 + 64) * 2),
     ((1, 64, 1, 128, 256), (1, 1, 3), 0),          # d_v > 128: single pass only
+    # d_k = 256, GDN form: -W (256), P (d_v), Aq (64) and K~ = Diag(g_{n-1}/g) K (256)
+    ((2, 100, 3, 256, 256), (1, 1, 3), 2 * 100 * 3 * (256 + 256 + 64 + 256) * 2),
+    ((1, 65, 1, 256, 64), (1, 1, 3), 65 * (256 + 64 + 64 + 256) * 2),
+    ((1, 64, 1, 256, 320), (1, 1, 3), 0),          # d_v > 256: exact path
+    ((1, 64, 1, 256, 128), (2, 1, 3), 0),          # d_k = 256, other gate forms: exact path
     ((1, 64, 1, 128, 128), (2, 1, 3), 3 * 16384 + 8192 + 16384 + 512 + 65536),   # KDA form
     ((1, 100, 2, 128, 64), (2, 2, 2), 4 * 51200 + 3 * 25600 + 2048 + 65536),      # GDN-2 form
     ((1, 64, 1, 128, 128), (2, 0, 0), 0),          # no erase: single pass only

@@ -24,7 +24,8 @@ def test_algorithmic_work(name, mb, gf):
 def test_kernel_families():
     fam = {n: bench.kernel_family(w) for n, w in WORKLOADS.items()}
     assert fam == {"tiny": "general", "gdn": "twopass", "kda": "twopass_general",
-                   "gdn2": "twopass_general", "gla": "erasefree", "gdn_gqa": "twopass"}
+                   "gdn2": "twopass_general", "gla": "erasefree", "gdn_gqa": "twopass",
+                   "gdn256": "twopass256"}
     assert set(bench.LAUNCHES_PER_CALL) == set(bench.KERNEL_SOURCES) == set(bench.KERNEL_NAMES)
 
 
@@ -80,3 +81,12 @@ def test_reference_arm_prints_the_contract_line():
         assert key in d, key
     assert d["impl"] == "reference" and d["value"] > 0 and d["steps"] == 1
     assert d["e2e"]["h2d_bytes_per_step"] == 0 and d["cpu_baseline"]["kind"] == "oracle"
+
+
+def test_tied_flops_follow_the_head_dims():
+    """The tied (Gated DeltaNet) count at d = 128 is 182,955 flops per
+    token-head; at d = 256 each d_k d_v term grows 4x, each C d term 2x."""
+    per = lambda wl: bench.workload_flops(wl) / (wl.B * wl.T * wl.H)
+    assert per(WORKLOADS["gdn"]) == 182955
+    C = 64
+    assert per(WORKLOADS["gdn256"]) == round(2 * (3 * 256 * 256 + C * 5 * 256 + C * C / 3))

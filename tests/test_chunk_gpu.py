@@ -347,3 +347,81 @@ def test_erase_free_wide_ctas(cuda_device, dv, akind, wkind):
     o_ref, ST_ref = run_oracle(inp)
     assert_close(o, o_ref, TOL["bf16"], "o")
     assert_close(ST, ST_ref, TOL["bf16"], "S_T")
+
+
+# ---- d_k = 256 (Gated DeltaNet head width, "How Linear Attention Remembers", Table 1) ----
+
+@pytest.mark.parametrize("dv,T", [(256, 200), (256, 64), (128, 65), (64, 1), (192, 130)])
+def test_dk256_tensor_core_path(cuda_device, dv, T):
+    """Gated DeltaNet gates at d_k = 256 run on the d_k = 256 two-pass
+    kernels: several chunks, a ragged tail, every d_v tile count."""
+    wl = WORKLOADS["gdn256"].with_(B=2, H=3, T=T, dv=dv, s0=True, seed=900 + T + dv)
+    inp = make_chunk_inputs(wl)
+    o, ST = run_chunk(inp, cuda_device)
+    o_ref, ST_ref = run_oracle(inp)
+    assert_close(o, o_ref, TOL["bf16"], "o")
+    assert_close(ST, ST_ref, TOL["bf16"], "S_T")
+
+
+def test_dk256_slow_decay_and_grouped_heads(cuda_device):
+    """alpha close to 1 over ten chunks (the state crosses every chunk
+    boundary), and value heads sharing q/k heads in pairs."""
+    wl = WORKLOADS["gdn256"].with_(B=1, H=4, T=640, s0=True, seed=910)
+    inp = make_chunk_inputs(wl)
+    inp["alpha"] = (inp["alpha"].float() ** 0.02).to(inp["alpha"].dtype)
+    qg, kg = inp["q"][:, :, ::2].contiguous(), inp["k"][:, :, ::2].contiguous()
+    inp_g = dict(inp, q=qg, k=kg)
+    o, ST = run_chunk(inp_g, cuda_device)
+    o_ref, ST_ref = run_oracle(inp_g)
+    assert_close(o, o_ref, TOL["bf16"], "o")
+    assert_close(ST, ST_ref, TOL["bf16"], "S_T")
+
+
+def test_dk256_workspace_is_used(cuda_device):
+    """The d_k = 256 path writes -W, P, Aq and K~ = Diag(g_{n-1}/g) K into the
+    caller's workspace: a token with beta = 0 gets zero rows of -W and P, Aq is
+    lower triangular, and K~ of a chunk's last token equals its k."""
+    T, H = 130, 2
+    wl = WORKLOADS["gdn256"].with_(B=1, H=H, T=T, seed=917)
+    inp = make_chunk_inputs(wl)
+    inp["b"][0, 5, 1] = 0.0
+    dev = cuda_device
+    q, k, v, a, b = (inp[x].to(dev) for x in ("q", "k", "v", "alpha", "b"))
+    from gated_delta_rule_147_b200 import workspace_bytes
+    nbytes = workspace_bytes(q, v, a, b, TIED)
+    assert nbytes == T * H * (256 + 256 + 64 + 256) * 2
+    ws = torch.full((nbytes,), 0x7F, dtype=torch.uint8, device=dev)
+    chunk_fwd(q, k, v, a, b, TIED, None, workspace=ws)
+    torch.cuda.synchronize()
+    n = T * H
+    parts, off = {}, 0
+    for name, d in (("wneg", 256), ("p", 256), ("aq", 64), ("kt", 256)):
+        parts[name] = ws[off: off + n * d * 2].view(torch.bfloat16).view(1, T, H, d).float().cpu()
+        off += n * d * 2
+    assert all(torch.isfinite(x).all() for x in parts.values())
+    assert torch.all(parts["wneg"][0, 5, 1] == 0) and torch.all(parts["p"][0, 5, 1] == 0)
+    assert parts["wneg"].abs().sum() > 0 and parts["p"].abs().sum() > 0
+    for t in (0, 5, 63, 64, 100, 129):
+        j = t % 64
+        assert torch.all(parts["aq"][0, t, :, j + 1:] == 0) and torch.all(parts["aq"][0, t, :, j] != 0)
+    kk = inp["k"].float()
+    for t in (63, 127, 129):  # the last token of each chunk: g_{n-1} / g = 1
+        assert torch.equal(parts["kt"][0, t], kk[0, t])
+    # an earlier token is scaled by a decay ratio in (0, 1]
+    m = kk[0, 10].abs() > 1e-3
+    r = parts["kt"][0, 10][m] / kk[0, 10][m]
+    assert m.sum() > 100 and torch.all((r > 0) & (r <= 1.0 + 1e-2))
+
+
+def test_dk256_full_size_sampled_heads(cuda_device):
+    """The d_k = d_v = 256 workload in the launch configuration the benchmark
+    times; the oracle checks sampled heads over the whole sequence."""
+    wl = WORKLOADS["gdn256"]
+    inp = make_chunk_inputs(wl)
+    o, ST = run_chunk(inp, cuda_device)
+    heads = [(0, 3), (1, 14)]
+    o_ref, ST_ref = run_oracle(inp, heads)
+    o_s, ST_s = gather_heads(o, ST, heads)
+    assert_close(o_s, o_ref, TOL["bf16"], f"o {heads}")
+    assert_close(ST_s, ST_ref, TOL["bf16"], f"S_T {heads}")
+    assert np.all(np.isfinite(o))

@@ -69,6 +69,7 @@ def _fwd_guarded(inp, dev, workspace_mode, group=1):
     ("kda", 128, "auto"), ("gdn2", 64, "auto"),      # two-pass, general kernels
     ("gdn", 256, None), ("gdn2", 128, None),         # single-pass kernels
     ("gla", 256, "auto"), ("gla", 64, "auto"),       # erase-free kernel
+    ("gdn256", 256, "auto"), ("gdn256", 64, "auto"), # two-pass, d_k = 256 kernels
 ])
 def test_forward_writes_stay_in_bounds(cuda_device, family, dv, workspace_mode, T):
     wl = WORKLOADS[family].with_(B=2, H=3, T=T, dv=dv, s0=True, seed=1300 + T + dv)
