@@ -74,7 +74,13 @@ struct GPrepParams {
     int* d_status;
     int T, H, dv, akind, bkind, wkind;
     int group;  // value heads per q/k head (q, k read at token-head index / group)
+    const __nv_bfloat16* v;
+    int prefetch_ahead;  // CTAs between this one and the one whose inputs it pulls into L2 (0: none)
 };
+
+__device__ __forceinline__ void prefetch_l2(const void* p) {
+    asm volatile("{\n\t.reg .u64 g;\n\tcvta.to.global.u64 g, %0;\n\tprefetch.global.L2 [g];\n\t}" ::"l"(p));
+}
 
 __device__ __forceinline__ void ld8b(const __nv_bfloat16* p, uint2& u) {
     u = *reinterpret_cast<const uint2*>(p);
@@ -173,6 +179,39 @@ __global__ void __launch_bounds__(NT, 2) prep_general_kernel(
     const uint32_t sbase = smem_u32(sm);
     auto bits_to_f32 = [](unsigned short u) { return __uint_as_float((uint32_t)u << 16); };
 
+    // The CTA launched about `prefetch_ahead` CTAs later (the block scheduler
+    // hands out CTAs in linear order as earlier ones finish) reads its q, k,
+    // v and channel gates with plain loads right at its start: pull its rows
+    // into L2 now, so its build waits on L2 rather than HBM latency.
+    if (pp.prefetch_ahead > 0) {
+        const long long lin = (long long)blockIdx.x + (long long)gridDim.x * (blockIdx.y + (long long)gridDim.y * blockIdx.z) +
+                              pp.prefetch_ahead;
+        const long long tot = (long long)gridDim.x * gridDim.y * gridDim.z;
+        if (lin < tot) {
+            const int nx = (int)(lin % gridDim.x);
+            const long long yz = lin / gridDim.x;
+            const int ny = (int)(yz % gridDim.y), nz = (int)(yz / gridDim.y);
+            const int r = tid & 63, t = (pp.c_begin + nx) * C + r;
+            if (t < T) {
+                const size_t tok = (size_t)nz * T + t;
+                const int part = tid >> 6;
+                const char* row = nullptr;
+                int bytes = 0;
+                if (part == 0) { row = (const char*)(pp.q + (tok * (H / pp.group) + ny / pp.group) * DK); bytes = 2 * DK; }
+                else if (part == 1) { row = (const char*)(pp.k + (tok * (H / pp.group) + ny / pp.group) * DK); bytes = 2 * DK; }
+                else if (part == 2) { row = (const char*)(pp.v + (tok * H + ny) * dv); bytes = 2 * dv; }
+                else if (ACH) { row = (const char*)(pp.alpha + (tok * H + ny) * DK); bytes = 2 * DK; }
+                for (int off = 0; row && off < bytes; off += 128) prefetch_l2(row + off);
+                if (part < 2) {
+                    const bool chan = part == 0 ? pp.bkind == GDR_GATE_CHANNEL : pp.wkind == GDR_GATE_CHANNEL;
+                    const __nv_bfloat16* g = part == 0 ? pp.bg : pp.wg;
+                    if (chan && !(TIED && part == 1))
+                        for (int off = 0; off < 2 * DK; off += 128)
+                            prefetch_l2((const char*)(g + (tok * H + ny) * DK) + off);
+                }
+            }
+        }
+    }
     GDR_TRACE_G(0);
     if (tid == 0) {
         mbar_init(bar_v, 1);
@@ -1063,6 +1102,8 @@ cudaError_t launch_chunk_twopass_general(const CUtensorMap* maps, MapFn make_map
     pp.T = T; pp.H = H; pp.dv = dv;
     pp.akind = akind; pp.bkind = bkind; pp.wkind = wkind;
     pp.group = group;
+    pp.v = reinterpret_cast<const __nv_bfloat16*>(v);
+    pp.prefetch_ahead = 0;
     CUtensorMap sm_maps[8];
     const int dims[7] = {128, 128, 128, 64, dv, 128, 64};
     for (int i = 0; i < 7; ++i) {
@@ -1075,9 +1116,15 @@ cudaError_t launch_chunk_twopass_general(const CUtensorMap* maps, MapFn make_map
     const CUtensorMap& bq_map = tied ? sm_maps[3] : sm_maps[6];
 
     const int nchunks = (T + C - 1) / C;
-    auto prep_range = [&](int c0, int c1, cudaStream_t stream) -> cudaError_t {
+    int nsm_p = 0, dev_p = 0;
+    if (cudaGetDevice(&dev_p) != cudaSuccess ||
+        cudaDeviceGetAttribute(&nsm_p, cudaDevAttrMultiProcessorCount, dev_p) != cudaSuccess)
+        nsm_p = 0;
+    // resident first-pass CTAs: two per SM, less the SMs a concurrent state pass holds
+    auto prep_range = [&](int c0, int c1, cudaStream_t stream, int busy_sms) -> cudaError_t {
         GPrepParams pr = pp;
         pr.c_begin = c0;
+        pr.prefetch_ahead = max(0, 2 * (nsm_p - busy_sms));
         const dim3 pgrid(c1 - c0, H, B);
         auto go = [&](auto kern) -> cudaError_t {
             cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, G_SMEM_BYTES);
@@ -1129,7 +1176,7 @@ cudaError_t launch_chunk_twopass_general(const CUtensorMap* maps, MapFn make_map
         if (aux_lock.owns_lock()) nseg = min(kMaxSegments, nchunks / kSegMin);
     }
     if (nseg == 1) {
-        cudaError_t e = prep_range(0, nchunks, st);
+        cudaError_t e = prep_range(0, nchunks, st, 0);
         if (e != cudaSuccess) return e;
         return state_range(0, nchunks, S0, ST);
     }
@@ -1139,7 +1186,7 @@ cudaError_t launch_chunk_twopass_general(const CUtensorMap* maps, MapFn make_map
     if (e == cudaSuccess) e = cudaStreamWaitEvent(aux->stream, evs[kMaxSegments], 0);
     for (int sgi = 0; sgi < nseg && e == cudaSuccess; ++sgi) {
         const int c0 = (int)((long long)nchunks * sgi / nseg), c1 = (int)((long long)nchunks * (sgi + 1) / nseg);
-        e = prep_range(c0, c1, sgi == 0 ? st : aux->stream);
+        e = prep_range(c0, c1, sgi == 0 ? st : aux->stream, sgi == 0 ? 0 : (int)(sgrid.x * sgrid.y * sgrid.z));
         if (e == cudaSuccess && sgi > 0) e = cudaEventRecord(evs[sgi], aux->stream);
     }
     for (int sgi = 0; sgi < nseg && e == cudaSuccess; ++sgi) {
