@@ -276,24 +276,23 @@ def time_chunk_e2e(inp, wl, dev, steps, warmup):
     return e0.elapsed_time(e1), h2d, d2h
 
 
-# fp32 CUDA-core peak: 148 SMs x 128 FP32 lanes x 2 flop (FMA) x 1965 MHz
-ALU_FP32_TFLOPS = 148 * 128 * 2 * 1965e6 / 1e12
-# the scans of the backward, per state element and token: forward (decay,
-# erase read, erase + write: 4 multiply-adds) and backward (G += q^T dO, k G,
-# u G, G <- alpha (G - e^T (k G)): 5 multiply-adds), 2 flop each. On the
-# tensor-core path of the Gated DeltaNet form the forward direction is done by
-# the forward kernels and only the backward one (5 multiply-adds) is scanned.
-BWD_SCAN_FLOPS_PER_ELEMENT = 2 * 9
-BWD_GRAD_SCAN_FLOPS_PER_ELEMENT = 2 * 5
-# tensor-core products of the chunk kernel per (chunk, head), d = 128, C = 64:
-# [dO;DR][S0|V|R]^T (128x256x128), [Q;U]K^T (128x64x128), P[U;K], P^T[Q;E],
-# [V';-R']G_e^T (128x128x128 each)
+# Tensor-core products of the Gated DeltaNet backward (d = 128, C = 64), per
+# token-head, 2 flop per multiply-add:
+# - the forward two-pass kernels, which checkpoint the state and U: the
+#   forward's own count (182,955; workload_flops);
+# - the chunkwise state-gradient pass: K K^T, Q K^T and X = (Diag(g_{n-1}/g)
+#   T)^T K (C d_k each), Aq T (C^2) and the solve (C^2 / 3) in its first pass;
+#   AqT^T dO (C d_v), X G, Q~^T dO and K^T Y' (d_k d_v each) in its state pass;
+BWD_GRAD_FLOPS_PER_TOKEN_HEAD = round(2 * (3 * 64 * 128 + 64 * 64 + 64 * 128 + 3 * 128 * 128) + 2 * 64 * 64 / 3)
+# - the chunk kernel, per (chunk, head): [dO;DR][S0|V|R]^T (128x256x128),
+#   [Q;U]K^T (128x64x128), P[U;K], P^T[Q;E], [V';-R']G_e^T (128x128x128 each)
 BWD_TC_FLOPS_PER_CHUNK = 2 * 128 * (256 * 128 + 64 * 128 + 3 * 128 * 128)
 
 
 def time_backward(dev, steps, warmup, pk):
     """The backward pass (gdr_chunk_bwd) on the Gated DeltaNet workload: CUDA
-    events per call (the fp32 scans, then the tensor-core chunk kernel)."""
+    events per call (forward checkpoints, the chunkwise state-gradient pass and
+    the chunk kernel, all on tensor cores)."""
     import torch
     from gated_delta_rule_147_b200 import TIED, chunk_bwd, gdr_chunk_bwd_workspace_size
     from gated_delta_rule_147_b200.inputs import WORKLOADS, make_cotangents
@@ -323,24 +322,22 @@ def time_backward(dev, steps, warmup, pk):
     state = wl.B * wl.H * wl.dk * wl.dv * 4
     # read q, k, v, dO (bf16), alpha, beta (bf16), dS_T; write dq, dk, dv (fp32), dalpha, dbeta, dS0
     bytes_ = th * (2 * (2 * wl.dk + 2 * wl.dv) + 2 * 2 + 4 * (2 * wl.dk + wl.dv) + 2 * 4) + 2 * state
-    scan_flops = BWD_GRAD_SCAN_FLOPS_PER_ELEMENT * wl.dk * wl.dv * th
-    tc_flops = BWD_TC_FLOPS_PER_CHUNK * wl.B * wl.H * ((wl.T + 63) // 64)
-    achieved = scan_flops / (ms * 1e-3) / 1e12
+    nch = wl.B * wl.H * ((wl.T + 63) // 64)
+    tc_flops = BWD_TC_FLOPS_PER_CHUNK * nch
+    flops = (workload_flops(wl) + BWD_GRAD_FLOPS_PER_TOKEN_HEAD * th) + tc_flops
+    achieved = flops / (ms * 1e-3) / 1e12
     return {"workload": f"Gated DeltaNet backward B={wl.B} H={wl.H} T={wl.T} d_k=d_v={wl.dk} bf16 "
                         f"inputs, fp32 gradients, dO and dS_T ~ N(0, 1)",
-            "ms_per_call": ms, "tokens_per_s": wl.B * wl.T / (ms * 1e-3), "launches_per_call": 4,
+            "ms_per_call": ms, "tokens_per_s": wl.B * wl.T / (ms * 1e-3), "launches_per_call": 5,
             "kernel": "gdr::twopass::prep_gdn_kernel + state_gdn_kernel<1> (forward, checkpoints S and U) + "
-                      "gdr::bwd::bwd_scan_staged_kernel (fp32 gradient scan) + gdr::bwdtc::bwd_chunk_tc_kernel "
-                      "(tcgen05 chunk products)",
-            "roofline": {"bound": "alu", "achieved": achieved, "peak": ALU_FP32_TFLOPS,
-                         "unit": "TFLOP/s", "frac": achieved / ALU_FP32_TFLOPS,
-                         "peak_source": "derived: 148 SMs x 128 fp32 lanes x 2 x 1965 MHz",
-                         "note": "the gradient scan's flops over the whole call (the scan takes most of it)",
-                         "algorithmic_flops": scan_flops, "algorithmic_bytes": bytes_,
+                      "gdr::bwdgrad::prep_grad_kernel + state_grad_kernel (chunkwise state gradient) + "
+                      "gdr::bwdtc::bwd_chunk_tc_kernel (chunk gradients)",
+            "roofline": {"bound": "tensor", "achieved": achieved, "peak": pk["bf16_tflops"],
+                         "unit": "TFLOP/s", "frac": achieved / pk["bf16_tflops"],
+                         "note": "bf16 tensor-core products of all five launches over the whole call",
+                         "algorithmic_flops": flops, "algorithmic_bytes": bytes_,
                          "hbm_frac": bytes_ / (ms * 1e-3) / 1e9 / pk["hbm_gbs"]},
-            "tensor_products": {"kernel": "gdr::bwdtc::bwd_chunk_tc_kernel", "flops_per_call": tc_flops,
-                                "peak_tflops": pk["bf16_tflops"],
-                                "duration": "per launch in the ncu launch list summary of this workload"}}
+            "chunk_kernel_flops_per_call": tc_flops}
 
 
 def time_decode(dev, nsteps, warmup):

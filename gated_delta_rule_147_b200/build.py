@@ -17,7 +17,7 @@ ROOT = os.path.dirname(HERE)
 CSRC = os.path.join(HERE, "csrc")
 OBJDIR = os.path.join(ROOT, "_build")
 SOURCES = ["api.cu", "decode.cu", "recurrent.cu", "chunk_sm100.cu", "chunk_erasefree_sm100.cu",
-           "chunk_bwd.cu", "chunk_bwd_tc_sm100.cu",
+           "chunk_bwd.cu", "chunk_bwd_tc_sm100.cu", "chunk_bwd_grad_sm100.cu",
            "chunk_twopass_sm100.cu", "chunk_twopass256_sm100.cu", "chunk_twopass_general_sm100.cu", "selftest.cu",
            "static_scratch.cu"]
 HEADERS = ["common.cuh", "chunk_common.cuh", "rcp_seed.h"]

@@ -31,6 +31,12 @@
 //     scalar gate's gradient, from the per-row-block partial sums of pass 2;
 //     bwd_group_sum_kernel (grouped heads only): dq, dk of each q/k head
 //     summed over the value heads that share it.
+// The Gated DeltaNet form in bf16 at d_k = d_v = 128 runs every part on
+// tensor cores instead: the forward two-pass kernels checkpoint the state at
+// every chunk start and U = beta v - r of every token, the chunkwise
+// state-gradient pass (chunk_bwd_grad_sm100.cu) gives G at every chunk end,
+// dr, dv and dS0, and the tensor-core chunk kernel (chunk_bwd_tc_sm100.cu)
+// the other gradients.
 #include "common.cuh"
 
 namespace gdr {
@@ -45,6 +51,10 @@ cudaError_t launch_chunk_twopass_gdn(const CUtensorMap* maps, const CUtensorMap*
                                      const void* alpha, const void* beta, const float* S0, void* o,
                                      float* ST, int* d_status, int B, int T, int H, int dv, int group,
                                      cudaStream_t st, float* ckS, float* up);
+cudaError_t launch_bwd_grad_tc(const CUtensorMap* q_map, const CUtensorMap* k_map, const CUtensorMap* do_map,
+                               const CUtensorMap* ws_maps, const void* alpha, const void* beta,
+                               const float* dST, float* ckG, float* DR, float* dv, float* dS0,
+                               int* d_status, int B, int T, int H, int dvn, int group, cudaStream_t st);
 
 namespace bwd {
 
@@ -62,9 +72,7 @@ struct Params {
     const float *S0, *dST;
     float *dq, *dk, *dv, *dalpha, *db, *dw, *dS0;
     float *ckS, *ckG, *R, *DR, *GP;  // workspace
-    int* d_status;                   // bounded waits of the tensor-core pass 2
-    int grad_scan_only;              // 1: the scans run only the backward direction (the
-                                     // forward two-pass kernels gave S and U = beta v - r)
+    int* d_status;                   // bounded waits of the tensor-core kernels
     float *dq_out, *dk_out;          // grouped heads: the caller's dq, dk (dq, dk are then workspace)
     int B, T, H, Hq, group, dk_, dv_, akind, bkind, wkind, nchunks, tpr, nrb;
 };
@@ -201,8 +209,7 @@ __device__ __forceinline__ void load_rows4(const Params& p, size_t tok, size_t t
 }
 
 // ----------------------------------------------------------------- pass 1 --
-// blockIdx.z = 2 b + direction (b alone, backward direction, when
-// grad_scan_only); warp w of CTA x owns columns
+// blockIdx.z = 2 b + direction; warp w of CTA x owns columns
 // 8 (kScanWarps x + w) .. + 8 (those below d_v), lane l owns rows 4 l .. 4 l + 3.
 template <typename TI>
 __global__ void __launch_bounds__(kScanWarps * 32) bwd_scan_kernel(Params p) {
@@ -210,8 +217,8 @@ __global__ void __launch_bounds__(kScanWarps * 32) bwd_scan_kernel(Params p) {
     const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
     const int c0 = NC * (kScanWarps * blockIdx.x + warp);
     if (c0 >= p.dv_) return;  // no block-wide barriers in this kernel
-    const int b = p.grad_scan_only ? (int)blockIdx.z : (int)(blockIdx.z >> 1);
-    const int dir = p.grad_scan_only ? 1 : (int)(blockIdx.z & 1), h = blockIdx.y;
+    const int b = (int)(blockIdx.z >> 1);
+    const int dir = (int)(blockIdx.z & 1), h = blockIdx.y;
     const size_t head = (size_t)b * p.H + h;
     const int i0 = 4 * lane;
     auto tok_of = [&](int t) { return ((size_t)b * p.T + t) * p.H + h; };
@@ -363,11 +370,9 @@ __device__ __forceinline__ void lds4<__nv_bfloat16>(const __nv_bfloat16* src, fl
     x[2] = __uint_as_float(u.y << 16); x[3] = __uint_as_float(u.y & 0xffff0000u);
 }
 
-// NC state columns per warp: 8, or 4 when only the backward direction runs
-// (half the warps otherwise, and the scan is then bound by latency).
-template <typename TI, int NC>
+template <typename TI>
 __global__ void __launch_bounds__(kScanWarps * 32) bwd_scan_staged_kernel(Params p) {
-    static_assert(NC == 4 || NC == 8, "4 or 8 columns per warp");
+    constexpr int NC = kScanCols;
     constexpr int CTA_COLS = kScanWarps * NC;
     auto st_cols = [](float* dst, const float* x, float sign) {  // NC columns, 16-byte stores
 #pragma unroll
@@ -381,8 +386,8 @@ __global__ void __launch_bounds__(kScanWarps * 32) bwd_scan_staged_kernel(Params
     const int c0 = cb + NC * warp;
     const bool active = c0 < p.dv_;       // idle warps still copy and meet the barriers
     const int ncols = min(CTA_COLS, p.dv_ - cb);
-    const int b = p.grad_scan_only ? (int)blockIdx.z : (int)(blockIdx.z >> 1);
-    const int dir = p.grad_scan_only ? 1 : (int)(blockIdx.z & 1), h = blockIdx.y;
+    const int b = (int)(blockIdx.z >> 1);
+    const int dir = (int)(blockIdx.z & 1), h = blockIdx.y;
     const size_t head = (size_t)b * p.H + h;
     const int i0 = 4 * lane;
     const bool rows_ok = i0 < p.dk_;       // d_k is a multiple of 4 here
@@ -887,34 +892,21 @@ WsLayout ws_layout(int B, int T, int H, int dk, int dv, bool grouped) {
 // tc_maps (q, k, v, dO tensor maps) selects the tensor-core path of the Gated
 // DeltaNet form: the forward two-pass kernels (their factors in fw, maps
 // fw_maps) checkpoint the state at every chunk start and U = beta v - r of
-// every token, the scans run only the backward direction, and the tensor-core
-// pass 2 writes the scalar gate gradients itself.
+// every token; the chunkwise gradient pass (its factors in the same
+// workspace region once the forward is done, maps gw_maps) gives the state
+// gradient at every chunk end, dr, dv and dS0; the tensor-core pass 2 writes
+// the scalar gate gradients itself.
 template <typename TI>
 cudaError_t launch_typed(Params p, const CUtensorMap* tc_maps, const CUtensorMap* fw_maps, void* fw,
-                         cudaStream_t st) {
+                         const CUtensorMap* gw_maps, cudaStream_t st) {
     cudaError_t e;
     if (tc_maps) {
         e = launch_chunk_twopass_gdn(tc_maps, fw_maps, fw, p.alpha, p.b, p.S0, nullptr, nullptr,
                                      p.d_status, p.B, p.T, p.H, p.dv_, p.group, st, p.ckS, p.R);
         if (e != cudaSuccess) return e;
-        p.grad_scan_only = 1;
-    }
-    const int ncw = p.grad_scan_only ? 4 : kScanCols;  // state columns per scan warp
-    const dim3 sgrid((p.dv_ + ncw * kScanWarps - 1) / (ncw * kScanWarps), p.H,
-                     p.grad_scan_only ? p.B : 2 * p.B);
-    if ((p.dk_ * sizeof(TI)) % 16 == 0) {
-        if (p.grad_scan_only)
-            bwd_scan_staged_kernel<TI, 4><<<sgrid, kScanWarps * 32, 0, st>>>(p);
-        else
-            bwd_scan_staged_kernel<TI, kScanCols><<<sgrid, kScanWarps * 32, 0, st>>>(p);
-    } else {
-        const dim3 g8((p.dv_ + kScanCols * kScanWarps - 1) / (kScanCols * kScanWarps), p.H,
-                      p.grad_scan_only ? p.B : 2 * p.B);
-        bwd_scan_kernel<TI><<<g8, kScanWarps * 32, 0, st>>>(p);
-    }
-    e = cudaGetLastError();
-    if (e != cudaSuccess) return e;
-    if (tc_maps) {
+        e = launch_bwd_grad_tc(&tc_maps[0], &tc_maps[1], &tc_maps[3], gw_maps, p.alpha, p.b, p.dST, p.ckG,
+                               p.DR, p.dv, p.dS0, p.d_status, p.B, p.T, p.H, p.dv_, p.group, st);
+        if (e != cudaSuccess) return e;
         e = launch_bwd_chunk_tc(tc_maps, p.ckS, p.ckG, p.R, p.DR, p.alpha, p.b, p.v, true, p.dq, p.dk,
                                 p.dalpha, p.db, p.d_status, p.B, p.T, p.H, p.group, p.nchunks, st);
         if (e != cudaSuccess) return e;
@@ -925,6 +917,13 @@ cudaError_t launch_typed(Params p, const CUtensorMap* tc_maps, const CUtensorMap
         }
         return e;
     }
+    const dim3 sgrid((p.dv_ + kScanCols * kScanWarps - 1) / (kScanCols * kScanWarps), p.H, 2 * p.B);
+    if ((p.dk_ * sizeof(TI)) % 16 == 0)
+        bwd_scan_staged_kernel<TI><<<sgrid, kScanWarps * 32, 0, st>>>(p);
+    else
+        bwd_scan_kernel<TI><<<sgrid, kScanWarps * 32, 0, st>>>(p);
+    e = cudaGetLastError();
+    if (e != cudaSuccess) return e;
     const uint32_t smem = chunk_smem(p.tpr).total;
     void (*kern)(Params) = bwd_chunk_kernel<TI>;
     e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
@@ -1049,10 +1048,9 @@ gdr_status gdr_chunk_bwd_grouped(const void* q, const void* k, const void* v, co
     const int RB = gdr::bwd::kChunkThreads / p.tpr;
     p.nrb = (d_k + RB - 1) / RB;
     p.d_status = d_status;
-    p.grad_scan_only = 0;
     // the Gated DeltaNet form on tensor cores: scalar decay, tied scalar beta,
     // bf16, d_k = d_v = 128
-    CUtensorMap maps[4], fw_maps[3];
+    CUtensorMap maps[4], fw_maps[3], gw_maps[3];
     const CUtensorMap* tc_maps = nullptr;
     void* fw = ws + wl.FW;
     if (dtype == GDR_BF16 && d_k == 128 && d_v == 128 && alpha_kind == GDR_GATE_SCALAR &&
@@ -1063,14 +1061,19 @@ gdr_status gdr_chunk_bwd_grouped(const void* q, const void* k, const void* v, co
             !gdr::make_tma_map_bf16(&maps[3], dO, B, T, H, d_v) ||
             !gdr::make_tma_map_bf16(&fw_maps[0], fw, B, T, H, d_k) ||
             !gdr::make_tma_map_bf16(&fw_maps[1], ws + wl.FW + (size_t)B * T * H * d_k * 2, B, T, H, d_v) ||
-            !gdr::make_tma_map_bf16(&fw_maps[2], ws + wl.FW + (size_t)B * T * H * (d_k + d_v) * 2, B, T, H, 64))
+            !gdr::make_tma_map_bf16(&fw_maps[2], ws + wl.FW + (size_t)B * T * H * (d_k + d_v) * 2, B, T, H, 64) ||
+            // the gradient pass's factors X, Aq T, Diag(g) Q take the same region
+            // (2 B T H (128 + 64 + 128) bytes) once the forward has read its own
+            !gdr::make_tma_map_bf16(&gw_maps[0], fw, B, T, H, d_k) ||
+            !gdr::make_tma_map_bf16(&gw_maps[1], ws + wl.FW + (size_t)B * T * H * d_k * 2, B, T, H, 64) ||
+            !gdr::make_tma_map_bf16(&gw_maps[2], ws + wl.FW + (size_t)B * T * H * (d_k + 64) * 2, B, T, H, d_k))
             return GDR_ERR_NO_DEVICE;
         tc_maps = maps;
         p.GP = nullptr;
     }
     const cudaError_t e = dtype == GDR_BF16
-                              ? gdr::bwd::launch_typed<__nv_bfloat16>(p, tc_maps, fw_maps, fw, st)
-                              : gdr::bwd::launch_typed<float>(p, nullptr, nullptr, nullptr, st);
+                              ? gdr::bwd::launch_typed<__nv_bfloat16>(p, tc_maps, fw_maps, fw, gw_maps, st)
+                              : gdr::bwd::launch_typed<float>(p, nullptr, nullptr, nullptr, nullptr, st);
     return e == cudaSuccess ? GDR_OK : GDR_ERR_LAUNCH;
 }
 

@@ -726,12 +726,15 @@ __global__ void __launch_bounds__(S_NT, 1) state_gdn_kernel(
             const int par = ci & 1;
             const uint32_t ph = (uint32_t)(ci & 1);
             const int s3 = ci % 3;
-            if (CKPT) {  // the state at this chunk's start, for the backward pass
+            // the state at this chunk's start, for the backward pass (each thread
+            // its row; the warps of lanes 64..127 once U has left)
+            auto store_ck = [&]() {
                 float* dst = ck.ckS + ((((size_t)bb * H + h) * nchunks + ci) * DK + row) * p.dv + v0 + wg * NH;
 #pragma unroll
                 for (int jj = 0; jj < NH; jj += 4)
                     *reinterpret_cast<float4*>(dst + jj) = make_float4(S[jj], S[jj + 1], S[jj + 2], S[jj + 3]);
-            }
+            };
+            if (CKPT && lo) store_ck();
             if (lo) {
                 // ---- O of the previous chunk, the next decay scan ---------------------------
                 if (ci > 0) {
@@ -750,32 +753,37 @@ __global__ void __launch_bounds__(S_NT, 1) state_gdn_kernel(
                 w_ok = mbar_wait(bar_w, ph) && w_ok;
                 tc_fence_after();
                 GDR_TRACE_S(7, 64);
-                {
-                    const int j = row - 64;  // token
-                    float d[32];
-                    tmem_ld32(tmem + lane_base + S_TM_D3 + (uint32_t)par * 64u + wg * 32, d);
-                    const float f = s_gcr3[s3 * 64 + j];
+                const int j = row - 64;  // token
+                float d[32];
+                tmem_ld32(tmem + lane_base + S_TM_D3 + (uint32_t)par * 64u + wg * 32, d);
+                const float f = s_gcr3[s3 * 64 + j];
 #pragma unroll
-                    for (int c8 = 0; c8 < 4; ++c8) {
-                        float x[8];
-                        const uint32_t off = sw128_chunk(j, wg * 4 + c8, 64);
-                        ld_chunk(sm + buf * S_STAGE + S_ST_P, off, x);
+                for (int c8 = 0; c8 < 4; ++c8) {
+                    float x[8];
+                    const uint32_t off = sw128_chunk(j, wg * 4 + c8, 64);
+                    ld_chunk(sm + buf * S_STAGE + S_ST_P, off, x);
 #pragma unroll
-                        for (int e = 0; e < 8; ++e) x[e] += d[c8 * 8 + e];
-                        if (CKPT && ci * C + j < T) {
-                            float* up = ck.up + (((size_t)bb * T + ci * C + j) * H + h) * p.dv + v0 + wg * 32 + c8 * 8;
-                            *reinterpret_cast<float4*>(up) = make_float4(x[0], x[1], x[2], x[3]);
-                            *reinterpret_cast<float4*>(up + 4) = make_float4(x[4], x[5], x[6], x[7]);
-                        }
-                        st_chunk(sm + S_OFF_U, off, x);
-#pragma unroll
-                        for (int e = 0; e < 8; ++e) x[e] *= f;
-                        st_chunk(sm + S_OFF_U2, off, x);
+                    for (int e = 0; e < 8; ++e) {
+                        x[e] += d[c8 * 8 + e];
+                        if (CKPT) d[c8 * 8 + e] = x[e];  // U, kept for the checkpoint below
                     }
+                    st_chunk(sm + S_OFF_U, off, x);
+#pragma unroll
+                    for (int e = 0; e < 8; ++e) x[e] *= f;
+                    st_chunk(sm + S_OFF_U2, off, x);
                 }
                 fence_proxy_async();
                 tc_fence_before();
                 mbar_arrive(u_ready);
+                if (CKPT) {  // U of every token and the chunk's start state, off the chain
+                    if (ci * C + j < T) {
+                        float* up = ck.up + (((size_t)bb * T + ci * C + j) * H + h) * p.dv + v0 + wg * 32;
+#pragma unroll
+                        for (int c4 = 0; c4 < 32; c4 += 4)
+                            *reinterpret_cast<float4*>(up + c4) = make_float4(d[c4], d[c4 + 1], d[c4 + 2], d[c4 + 3]);
+                    }
+                    store_ck();
+                }
             }
             // ---- S = g_{n-1} S + D4 (every compute warp: its lanes, half the columns) ----
             w_ok = mbar_wait(bar_k, ph) && w_ok;

@@ -253,24 +253,31 @@ size_t gdr_chunk_fwd_static_capacity(void);
  *   entry ignored, on exit undefined.
  * Method: the state gradient G follows its own backward recurrence
  *   G_{t-1} = Diag(alpha_t)(I - e^T k) G_t + q_{t-1}^T dO_{t-1}, which does
- *   not involve S, so a first kernel scans the tokens forward (S at every
- *   64-token chunk start, r_t) and backward (G at every
- *   chunk end, dr_t = -k G, dv_t, dS0) at the same time in fp32, one warp
- *   per 8 state columns. A second kernel, parallel over chunks and heads,
- *   forms dq, dk and the gate gradients of each chunk from its start state,
- *   end gradient, r and dr:
+ *   not involve S, so the sequential work is two independent passes: forward
+ *   (S at every 64-token chunk start, r_t) and backward (G at every chunk
+ *   end, dr_t = -k G, dv_t, dS0). A chunk-parallel kernel then forms dq, dk
+ *   and the gate gradients of each chunk from its start state, end
+ *   gradient, r and dr:
  *   - the Gated DeltaNet form in bf16 with d_k = d_v = 128 (alpha and b
- *     scalar, w tied): the forward two-pass tensor-core kernels run first
- *     and give S at every chunk start and r_t (so the scan runs only the
- *     backward direction); then the chunk gradients on tensor cores as
- *     masked, decay-scaled products (bf16 operands: the checkpoints, r and
- *     dr are rounded to bf16; fp32 accumulation), one CTA per (chunk,
- *     head) writing dalpha and db directly; the bounded waits of these
- *     kernels OR GDR_DEVICE_TIMEOUT into *d_status (if not NULL) and end
- *     the kernel, leaving the outputs undefined;
- *   - every other form and dtype: fp32 on CUDA cores, per block of state
- *     rows, rebuilding the chunk's states elementwise; a third kernel then
- *     sums scalar gates' gradients over the key channels; d_status unused.
+ *     scalar, w tied) runs on tensor cores throughout (bf16 operands, fp32
+ *     accumulation) and scans nothing token by token: the forward two-pass
+ *     kernels give S at every chunk start and r_t; the backward recurrence
+ *     of G taken a chunk at a time (per chunk, with Y_j = k_j G_j, T the
+ *     forward's UT transform and Aq its masked q k^T block:
+ *     (I + A)^T Y = Diag(g_{n-1}/g) K G_in + Aq^T dO and
+ *     G_out = g_{n-1} G_in + (Diag(g) Q)^T dO - (Diag(beta g) K)^T Y) gives
+ *     G at every chunk end, dr, dv and dS0 (a first pass over all chunks
+ *     forms the chunk factors, a second walks the chunks in reverse); then
+ *     the chunk gradients as masked, decay-scaled products, one CTA per
+ *     (chunk, head) writing dalpha and db directly. Every gradient of this
+ *     form carries bf16 operand rounding. The bounded waits of these kernels
+ *     OR GDR_DEVICE_TIMEOUT into *d_status (if not NULL) and end the kernel,
+ *     leaving the outputs undefined;
+ *   - every other form and dtype: fp32 on CUDA cores: one kernel scans the
+ *     tokens in both directions at once, one warp per 8 state columns; the
+ *     chunk kernel works per block of state rows, rebuilding the chunk's
+ *     states elementwise; a third kernel sums scalar gates' gradients over
+ *     the key channels; d_status unused.
  *   Deterministic (no atomics) on both paths.
  * Supported: chunk = 64, 1 <= d_k <= 128, d_v a multiple of 8 up to 256,
  *   ceil(T / 64) <= 65535 and B * H <= 65535. Every pointer 16-byte
@@ -320,9 +327,9 @@ size_t gdr_chunk_bwd_grouped_workspace_size(int B, int T, int H_qk, int H, int d
  * d_v), r_t and dr_t of every token (2 x B T H d_v), and scalar-gate partial
  * sums (3 x ceil(d_k / RB) x B T H, RB = 128 / (d_v / 8 rounded up to a power
  * of two)), and when d_k = d_v = 128 the forward's per-token -W, P and
- * q k^T block rows
- * (B T H (d_k + d_v + 64) bf16), each rounded up to 256 bytes. Host-only;
- * launches nothing. */
+ * q k^T block rows (B T H (d_k + d_v + 64) bf16; the gradient pass's
+ * per-token rows of its chunk factors, B T H (128 + 64 + 128) bf16, reuse
+ * that region), each rounded up to 256 bytes. Host-only; launches nothing. */
 size_t gdr_chunk_bwd_workspace_size(int B, int T, int H, int d_k, int d_v);
 
 /*
