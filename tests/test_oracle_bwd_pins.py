@@ -135,3 +135,46 @@ def test_chunkwise_route_agrees(gates, T):
             assert got[n] is None, n
         else:
             np.testing.assert_allclose(got[n], x, atol=1e-10 * max(1.0, np.abs(x).max()), err_msg=n)
+
+
+def _chunk_state_gradient(q, k, alpha, beta, dO, dS_T, chunk):
+    """The Gated DeltaNet state-gradient recurrence G_t = q_t^T dO_t +
+    alpha_{t+1} (I - beta_{t+1} k_{t+1}^T k_{t+1}) G_{t+1}, taken a chunk at a
+    time in reverse (the algebra of the tensor-core gradient pass): with g the
+    decay product from the chunk's start, A the masked key products, Aq the
+    masked q k^T block and Y_j = k_j G_j,
+      (I + A)^T Y = Diag(g_{n-1}/g) K G_in + Aq^T dO,
+      G_out = g_{n-1} G_in + (Diag(g) Q)^T dO - (Diag(beta g) K)^T Y.
+    One head: q, k [T, d_k]; alpha, beta [T]; dO [T, d_v]. Returns dv = beta Y
+    per token and dS0 = the final G_out."""
+    T = q.shape[0]
+    G = dS_T.copy()
+    dv = np.zeros((T, dO.shape[1]))
+    for t0 in reversed(range(0, T, chunk)):
+        K, Q, D = k[t0:t0 + chunk], q[t0:t0 + chunk], dO[t0:t0 + chunk]
+        b = beta[t0:t0 + chunk]
+        g = np.cumprod(alpha[t0:t0 + chunk])
+        ratio = g[:, None] / g[None, :]
+        A = np.tril(b[:, None] * (K @ K.T) * ratio, -1)
+        Aq = np.tril((Q @ K.T) * ratio)
+        Y = np.linalg.solve((np.eye(len(g)) + A).T, (g[-1] / g)[:, None] * (K @ G) + Aq.T @ D)
+        dv[t0:t0 + chunk] = b[:, None] * Y
+        G = g[-1] * G + (g[:, None] * Q).T @ D - (b[:, None] * g[:, None] * K).T @ Y
+    return dv, G
+
+
+@pytest.mark.parametrize("T", [1, 8, 21])
+def test_chunk_state_gradient_algebra_agrees(T):
+    """The chunk form of the state-gradient recurrence (what the tensor-core
+    gradient pass computes) gives the reverse token loop's dv and dS0 exactly,
+    ragged final chunks included."""
+    gates = {"alpha": "scalar", "b": "scalar", "w": "tied"}
+    rng = np.random.default_rng(300 + T)
+    q, k, v, a, b, w, S0 = rand_inputs(rng, 1, T, 1, 5, 4, gates, s0=True, k_unit=False)
+    dO = rng.standard_normal(v.shape)
+    dS_T = rng.standard_normal(S0.shape)
+    ref = oracle.recurrence_bwd(q, k, v, a, b, w, S0, gates, dO, dS_T)
+    dv, dS0 = _chunk_state_gradient(q[0, :, 0], k[0, :, 0], a[0, :, 0], b[0, :, 0], dO[0, :, 0],
+                                    dS_T[0, 0], chunk=8)
+    np.testing.assert_allclose(dv, ref["dv"][0, :, 0], atol=1e-10 * np.abs(ref["dv"]).max())
+    np.testing.assert_allclose(dS0, ref["dS0"][0, 0], atol=1e-10 * np.abs(ref["dS0"]).max())
