@@ -14,14 +14,20 @@ namespace gdr {
 // Block: 256 threads per head. Threads are laid out as RPP row lanes x TPR
 // column groups of 4 floats (one 16-byte load each); a warp reads contiguous
 // 16-byte pieces of one or more rows. Each thread keeps NR rows x 4 columns.
+// A block handles DV value columns of one head (blockIdx.y selects which DV of
+// the head's dvf): every column's reductions over d_k stay inside its block,
+// so a wide head can be split over blocks with no exchange between them.
+// Two resident blocks per SM (128 registers a thread) up to 16 state rows per
+// thread; 32 rows (128 registers of state alone) take one.
 template <typename TI, int DV, int NR>
-__global__ void __launch_bounds__(256) decode_step_kernel(
+__global__ void __launch_bounds__(256, NR <= 16 ? 2 : 1) decode_step_kernel(
     const TI* __restrict__ q, const TI* __restrict__ k, const TI* __restrict__ v,
     const TI* __restrict__ alpha, const TI* __restrict__ bg, const TI* __restrict__ wg, int akind,
-    int bkind, int wkind, float* __restrict__ S, TI* __restrict__ o, int dk, int group) {
+    int bkind, int wkind, float* __restrict__ S, TI* __restrict__ o, int dk, int dvf, int group) {
     constexpr int TPR = DV / 4;
     constexpr int RPP = 256 / TPR;
     const int bh = blockIdx.x;
+    const int c0 = blockIdx.y * DV;  // this block's first value column
     const int tid = threadIdx.x;
     __shared__ float s_alpha[256], s_eka[256], s_qa[256], s_k[256], s_wk[256];
     __shared__ float s_v[DV];
@@ -45,7 +51,7 @@ __global__ void __launch_bounds__(256) decode_step_kernel(
         s_k[i] = ki;
         s_wk[i] = ww * ki;
     }
-    for (int j = tid; j < DV; j += 256) s_v[j] = to_f32(v[(size_t)bh * DV + j]);
+    for (int j = tid; j < DV; j += 256) s_v[j] = to_f32(v[(size_t)bh * dvf + c0 + j]);
     __syncthreads();
     if (tid < 32) {
         float d1 = 0.f, d2 = 0.f;
@@ -66,13 +72,14 @@ __global__ void __launch_bounds__(256) decode_step_kernel(
     }
 
     const int cg = tid % TPR, rl = tid / TPR;
-    float4* Sh = reinterpret_cast<float4*>(S + (size_t)bh * dk * DV);
+    float4* Sh = reinterpret_cast<float4*>(S + (size_t)bh * dk * dvf + c0);
+    const size_t rstride = (size_t)dvf / 4;  // float4 per state row
     float4 sv[NR];
     float4 racc = make_float4(0.f, 0.f, 0.f, 0.f), aacc = racc;
 #pragma unroll
     for (int m = 0; m < NR; ++m) {
         const int row = rl + RPP * m;
-        if (row < dk) sv[m] = __ldcs(Sh + (size_t)row * TPR + cg);
+        if (row < dk) sv[m] = __ldcs(Sh + (size_t)row * rstride + cg);
         else sv[m] = make_float4(0.f, 0.f, 0.f, 0.f);
     }
 #pragma unroll
@@ -104,7 +111,7 @@ __global__ void __launch_bounds__(256) decode_step_kernel(
             n.y = a * sv[m].y - kk * r.y + wk * v4.y;
             n.z = a * sv[m].z - kk * r.z + wk * v4.z;
             n.w = a * sv[m].w - kk * r.w + wk * v4.w;
-            __stcs(Sh + (size_t)row * TPR + cg, n);
+            __stcs(Sh + (size_t)row * rstride + cg, n);
         }
     }
     if (rl == 0) {
@@ -115,7 +122,7 @@ __global__ void __launch_bounds__(256) decode_step_kernel(
             a.x += p.x; a.y += p.y; a.z += p.z; a.w += p.w;
         }
         const float qk = s_dots[0], qwk = s_dots[1];
-        TI* ob = o + (size_t)bh * DV + 4 * cg;
+        TI* ob = o + (size_t)bh * dvf + c0 + 4 * cg;
         ob[0] = from_f32<TI>(a.x - qk * r.x + qwk * v4.x);
         ob[1] = from_f32<TI>(a.y - qk * r.y + qwk * v4.y);
         ob[2] = from_f32<TI>(a.z - qk * r.z + qwk * v4.z);
@@ -126,13 +133,14 @@ __global__ void __launch_bounds__(256) decode_step_kernel(
 template <typename TI, int DV>
 static cudaError_t launch_decode_dv(const void* q, const void* k, const void* v, const void* a,
                                     const void* b, const void* w, int ak, int bk, int wk, float* S,
-                                    void* o, int BH, int dk, int group, cudaStream_t st) {
+                                    void* o, int BH, int dk, int dvf, int group, cudaStream_t st) {
     constexpr int RPP = 256 / (DV / 4);
     const int nr = (dk + RPP - 1) / RPP;
+    const dim3 grid(BH, dvf / DV);
 #define GDR_DEC(NRV)                                                                              \
-    decode_step_kernel<TI, DV, NRV><<<BH, 256, 0, st>>>(                                          \
+    decode_step_kernel<TI, DV, NRV><<<grid, 256, 0, st>>>(                                        \
         (const TI*)q, (const TI*)k, (const TI*)v, (const TI*)a, (const TI*)b, (const TI*)w, ak, bk, \
-        wk, S, (TI*)o, dk, group)
+        wk, S, (TI*)o, dk, dvf, group)
     if (nr <= 4) GDR_DEC(4);
     else if (nr <= 8) GDR_DEC(8);
     else if (nr <= 16) GDR_DEC(16);
@@ -143,8 +151,12 @@ static cudaError_t launch_decode_dv(const void* q, const void* k, const void* v,
 }
 
 // Rows per thread needed for (d_k, d_v); the launcher supports up to 32.
+// Value columns per block: the whole head, except d_v = 256 with d_k > 128
+// (64 state rows per thread), which takes two blocks of 128 columns.
+int decode_cols_per_block(int dk, int dv) { return dv == 256 && dk > 128 ? 128 : dv; }
+
 int decode_rows_per_thread(int dk, int dv) {
-    int rpp = 256 / (dv / 4);
+    int rpp = 256 / (decode_cols_per_block(dk, dv) / 4);
     return (dk + rpp - 1) / rpp;
 }
 
@@ -153,11 +165,14 @@ static cudaError_t launch_decode_t(const void* q, const void* k, const void* v, 
                                    const void* b, const void* w, int ak, int bk, int wk, float* S,
                                    void* o, int BH, int dk, int dv, int group, cudaStream_t st) {
     switch (dv) {
-        case 16: return launch_decode_dv<TI, 16>(q, k, v, a, b, w, ak, bk, wk, S, o, BH, dk, group, st);
-        case 32: return launch_decode_dv<TI, 32>(q, k, v, a, b, w, ak, bk, wk, S, o, BH, dk, group, st);
-        case 64: return launch_decode_dv<TI, 64>(q, k, v, a, b, w, ak, bk, wk, S, o, BH, dk, group, st);
-        case 128: return launch_decode_dv<TI, 128>(q, k, v, a, b, w, ak, bk, wk, S, o, BH, dk, group, st);
-        case 256: return launch_decode_dv<TI, 256>(q, k, v, a, b, w, ak, bk, wk, S, o, BH, dk, group, st);
+        case 16: return launch_decode_dv<TI, 16>(q, k, v, a, b, w, ak, bk, wk, S, o, BH, dk, dv, group, st);
+        case 32: return launch_decode_dv<TI, 32>(q, k, v, a, b, w, ak, bk, wk, S, o, BH, dk, dv, group, st);
+        case 64: return launch_decode_dv<TI, 64>(q, k, v, a, b, w, ak, bk, wk, S, o, BH, dk, dv, group, st);
+        case 128: return launch_decode_dv<TI, 128>(q, k, v, a, b, w, ak, bk, wk, S, o, BH, dk, dv, group, st);
+        case 256:
+            return decode_cols_per_block(dk, dv) == 256
+                       ? launch_decode_dv<TI, 256>(q, k, v, a, b, w, ak, bk, wk, S, o, BH, dk, dv, group, st)
+                       : launch_decode_dv<TI, 128>(q, k, v, a, b, w, ak, bk, wk, S, o, BH, dk, dv, group, st);
         default: return cudaErrorInvalidValue;
     }
 }

@@ -341,7 +341,9 @@ size_t gdr_chunk_bwd_workspace_size(int B, int T, int H, int d_k, int d_v);
  * S is read, and S_new is written from registers.
  * q, k [B, H, d_k]; v, o [B, H, d_v]; gates [B, H] or [B, H, d_k];
  * S [B, H, d_k, d_v] fp32. o must not alias S or the inputs.
- * Supported: 1 <= d_k <= 256, d_v a multiple of 4 with 4 <= d_v <= 256.
+ * Supported: 1 <= d_k <= 256, d_v in {16, 32, 64, 128, 256} (a head of
+ * d_k > 128 and d_v = 256 runs as two blocks of 128 value columns: every
+ * column's reductions over d_k stay inside its block).
  * Alignment: S, o, q, k, v and channel gates must be 16-byte aligned.
  * Returns as gdr_chunk_fwd.
  */

@@ -92,7 +92,6 @@ def decode(**kw):
     (dict(bk=5), _lib.GDR_ERR_INVALID_ARG),
     (dict(dv=48), _lib.GDR_ERR_UNSUPPORTED),
     (dict(dk=512), _lib.GDR_ERR_UNSUPPORTED),
-    (dict(dv=256, dk=256), _lib.GDR_ERR_UNSUPPORTED),     # too many state rows per thread
     (dict(S=P + 4), _lib.GDR_ERR_MISALIGNED),
 ])
 def test_decode_step_rejects_bad_arguments(kw, expect):

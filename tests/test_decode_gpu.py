@@ -35,7 +35,9 @@ def rand_step(rng, B, H, dk, dv, kinds, dtype):
 
 @pytest.mark.parametrize("dtype,dk,dv", [(torch.bfloat16, 128, 128), (torch.float32, 128, 128),
                                          (torch.bfloat16, 64, 32), (torch.float32, 96, 256),
-                                         (torch.float32, 200, 16)])
+                                         (torch.float32, 200, 16),
+                                         # d_k = d_v = 256: each head's columns in two blocks
+                                         (torch.bfloat16, 256, 256), (torch.float32, 200, 256)])
 @pytest.mark.parametrize("kinds", [GEN, {"alpha": "scalar", "b": "scalar", "w": "tied"},
                                    {"alpha": "none", "b": "none", "w": "none"}])
 def test_decode_steps_small(cuda_device, dtype, dk, dv, kinds):
@@ -83,7 +85,7 @@ def test_decode_full_size_sampled_heads(cuda_device):
     assert np.all(np.isfinite(S_dev.cpu().numpy()))
 
 
-@pytest.mark.parametrize("family", ["gdn", "kda", "gdn2"])
+@pytest.mark.parametrize("family", ["gdn", "kda", "gdn2", "gdn256"])
 def test_prefill_then_decode_continues_the_sequence(cuda_device, family):
     """The chunk forward's final state is the decode step's state layout:
     prefill T tokens, then decode m more from S_T; the decode outputs equal

@@ -88,10 +88,10 @@ def test_exact_path_writes_stay_in_bounds(cuda_device, dtype, dk, dv):
     _fwd_guarded(make_chunk_inputs(wl), cuda_device, "auto")
 
 
-@pytest.mark.parametrize("dv", [64, 128, 256])
-def test_decode_writes_stay_in_bounds(cuda_device, dv):
+@pytest.mark.parametrize("dk,dv", [(128, 64), (128, 128), (128, 256), (256, 256)])
+def test_decode_writes_stay_in_bounds(cuda_device, dk, dv):
     dev = cuda_device
-    wl = WORKLOADS["gdn2"].with_(B=3, H=5, T=1, dv=dv, s0=True, seed=1600)
+    wl = WORKLOADS["gdn2"].with_(B=3, H=5, T=1, dk=dk, dv=dv, s0=True, seed=1600)
     inp = make_chunk_inputs(wl)
     q, k, v, a, b, w = (inp[x][:, 0].to(dev).contiguous() for x in ("q", "k", "v", "alpha", "b", "w"))
     S = Guarded(tuple(inp["S0"].shape), torch.float32, dev)
