@@ -61,7 +61,8 @@ namespace bwd {
 constexpr int kC = 64;           // chunk: checkpoint interval of the scans
 constexpr int kSub = 8;          // sub-chunk: states rebuilt in registers
 constexpr int kNSub = kC / kSub;
-constexpr int kMaxDK = 128;      // 4 rows per lane in the scans
+constexpr int kMaxDK = 256;      // 4 rows per lane in the scans up to d_k = 128, 8 beyond
+constexpr int kStagedMaxDK = 128; // the staged scan's shared-memory rows
 constexpr int kMaxDV = 256;      // 8 columns per thread, up to 32 threads per row in pass 2
 constexpr int kScanWarps = 4;    // scan CTA: 4 warps
 constexpr int kScanCols = 8;     // state columns per scan warp
@@ -161,57 +162,69 @@ __device__ __forceinline__ void warp_allsum(float (&x)[NV], int lane) {
     for (int v = 0; v < NV; ++v) x[v] = __shfl_sync(0xffffffffu, s, v * (32 / NV));
 }
 
-// Per-row scalars of rows i0 .. i0 + 3 of one token (neutral beyond d_k). With
-// d_k a multiple of 4 the four rows are one vector load per input.
-struct Rows4 {
-    float q[4], k[4], a[4], bg[4], wg[4];
+// Per-row scalars of rows i0 .. i0 + R - 1 of one token (neutral beyond d_k).
+// With d_k a multiple of 4 every four rows are one vector load per input.
+template <int R>
+struct RowsR {
+    float q[R], k[R], a[R], bg[R], wg[R];
 };
+using Rows4 = RowsR<4>;
 
-template <typename TI>
-__device__ __forceinline__ void load_rows4(const Params& p, size_t tok, size_t tokq, int i0, Rows4& r) {
+template <typename TI, int R>
+__device__ __forceinline__ void load_rows(const Params& p, size_t tok, size_t tokq, int i0, RowsR<R>& r) {
     if ((p.dk_ & 3) == 0) {
-        if (i0 < p.dk_) {
-            const size_t gi = tok * p.dk_ + i0;
-            load4<TI>(p.q, tokq * p.dk_ + i0, r.q);
-            load4<TI>(p.k, tokq * p.dk_ + i0, r.k);
-            if (p.akind == GDR_GATE_CHANNEL) load4<TI>(p.alpha, gi, r.a);
-            else {
-                const float a = p.akind == GDR_GATE_SCALAR ? ld1<TI>(p.alpha, tok) : 1.f;
-                r.a[0] = r.a[1] = r.a[2] = r.a[3] = a;
-            }
-            if (p.bkind == GDR_GATE_CHANNEL) load4<TI>(p.b, gi, r.bg);
-            else {
-                const float bb = p.bkind == GDR_GATE_SCALAR ? ld1<TI>(p.b, tok) : 0.f;
-                r.bg[0] = r.bg[1] = r.bg[2] = r.bg[3] = bb;
-            }
-            if (p.wkind == GDR_GATE_CHANNEL) load4<TI>(p.w, gi, r.wg);
-            else if (p.wkind == GDR_GATE_TIED) {
 #pragma unroll
-                for (int rr = 0; rr < 4; ++rr) r.wg[rr] = r.bg[rr];
+        for (int g = 0; g < R; g += 4) {
+            const int ig = i0 + g;
+            if (ig < p.dk_) {
+                const size_t gi = tok * p.dk_ + ig;
+                load4<TI>(p.q, tokq * p.dk_ + ig, *reinterpret_cast<float(*)[4]>(r.q + g));
+                load4<TI>(p.k, tokq * p.dk_ + ig, *reinterpret_cast<float(*)[4]>(r.k + g));
+                if (p.akind == GDR_GATE_CHANNEL) load4<TI>(p.alpha, gi, *reinterpret_cast<float(*)[4]>(r.a + g));
+                else {
+                    const float a = p.akind == GDR_GATE_SCALAR ? ld1<TI>(p.alpha, tok) : 1.f;
+                    r.a[g] = r.a[g + 1] = r.a[g + 2] = r.a[g + 3] = a;
+                }
+                if (p.bkind == GDR_GATE_CHANNEL) load4<TI>(p.b, gi, *reinterpret_cast<float(*)[4]>(r.bg + g));
+                else {
+                    const float bb = p.bkind == GDR_GATE_SCALAR ? ld1<TI>(p.b, tok) : 0.f;
+                    r.bg[g] = r.bg[g + 1] = r.bg[g + 2] = r.bg[g + 3] = bb;
+                }
+                if (p.wkind == GDR_GATE_CHANNEL) load4<TI>(p.w, gi, *reinterpret_cast<float(*)[4]>(r.wg + g));
+                else if (p.wkind == GDR_GATE_TIED) {
+#pragma unroll
+                    for (int rr = 0; rr < 4; ++rr) r.wg[g + rr] = r.bg[g + rr];
+                } else {
+                    const float ww = p.wkind == GDR_GATE_SCALAR ? ld1<TI>(p.w, tok) : 1.f;
+                    r.wg[g] = r.wg[g + 1] = r.wg[g + 2] = r.wg[g + 3] = ww;
+                }
             } else {
-                const float ww = p.wkind == GDR_GATE_SCALAR ? ld1<TI>(p.w, tok) : 1.f;
-                r.wg[0] = r.wg[1] = r.wg[2] = r.wg[3] = ww;
-            }
-            return;
-        }
 #pragma unroll
-        for (int rr = 0; rr < 4; ++rr) {
-            r.q[rr] = r.k[rr] = r.bg[rr] = r.wg[rr] = 0.f;
-            r.a[rr] = 1.f;
+                for (int rr = 0; rr < 4; ++rr) {
+                    r.q[g + rr] = r.k[g + rr] = r.bg[g + rr] = r.wg[g + rr] = 0.f;
+                    r.a[g + rr] = 1.f;
+                }
+            }
         }
         return;
     }
 #pragma unroll
-    for (int rr = 0; rr < 4; ++rr) {
+    for (int rr = 0; rr < R; ++rr) {
         const Row w1 = load_row<TI>(p, tok, tokq, i0 + rr);
         r.q[rr] = w1.q; r.k[rr] = w1.k; r.a[rr] = w1.a; r.bg[rr] = w1.bg; r.wg[rr] = w1.wg;
     }
 }
 
+template <typename TI>
+__device__ __forceinline__ void load_rows4(const Params& p, size_t tok, size_t tokq, int i0, Rows4& r) {
+    load_rows<TI, 4>(p, tok, tokq, i0, r);
+}
+
 // ----------------------------------------------------------------- pass 1 --
 // blockIdx.z = 2 b + direction; warp w of CTA x owns columns
-// 8 (kScanWarps x + w) .. + 8 (those below d_v), lane l owns rows 4 l .. 4 l + 3.
-template <typename TI>
+// 8 (kScanWarps x + w) .. + 8 (those below d_v), lane l owns rows R l .. R l + R - 1
+// (R = 4 up to d_k = 128, 8 up to d_k = 256).
+template <typename TI, int R>
 __global__ void __launch_bounds__(kScanWarps * 32) bwd_scan_kernel(Params p) {
     constexpr int NC = kScanCols;
     const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
@@ -220,27 +233,27 @@ __global__ void __launch_bounds__(kScanWarps * 32) bwd_scan_kernel(Params p) {
     const int b = (int)(blockIdx.z >> 1);
     const int dir = (int)(blockIdx.z & 1), h = blockIdx.y;
     const size_t head = (size_t)b * p.H + h;
-    const int i0 = 4 * lane;
+    const int i0 = R * lane;
     auto tok_of = [&](int t) { return ((size_t)b * p.T + t) * p.H + h; };
     const int hq = h / p.group;
     auto tokq_of = [&](int t) { return ((size_t)b * p.T + t) * p.Hq + hq; };
     auto ck_at = [&](float* base, int chunk, int i) {
         return base + ((head * p.nchunks + chunk) * p.dk_ + i) * p.dv_ + c0;
     };
-    float X[4][NC];  // S (forward) or G (backward): rows i0 + rr, columns c0 + c
+    float X[R][NC];  // S (forward) or G (backward): rows i0 + rr, columns c0 + c
     const float* init = dir == 0 ? p.S0 : p.dST;
 #pragma unroll
-    for (int rr = 0; rr < 4; ++rr) {
+    for (int rr = 0; rr < R; ++rr) {
         if (init && i0 + rr < p.dk_) load8<float>(init, (head * p.dk_ + i0 + rr) * p.dv_ + c0, X[rr]);
         else
             for (int c = 0; c < NC; ++c) X[rr][c] = 0.f;
     }
     // the next token's inputs are loaded while the current one is computed
     const void* colsrc = dir == 0 ? p.v : p.dO;
-    Rows4 nrw;
+    RowsR<R> nrw;
     float nvec[NC];
     const int tfirst = dir == 0 ? 0 : p.T - 1;
-    load_rows4<TI>(p, tok_of(tfirst), tokq_of(tfirst), i0, nrw);
+    load_rows<TI, R>(p, tok_of(tfirst), tokq_of(tfirst), i0, nrw);
     load8<TI>(colsrc, tok_of(tfirst) * p.dv_ + c0, nvec);
     for (int n = 0; n < p.T; ++n) {
         const int t = dir == 0 ? n : p.T - 1 - n;
@@ -248,20 +261,20 @@ __global__ void __launch_bounds__(kScanWarps * 32) bwd_scan_kernel(Params p) {
         const bool store_ck = dir == 0 ? (t % kC == 0) : (t == p.T - 1 || (t + 1) % kC == 0);
         if (store_ck)  // forward: chunk start; backward: before the chunk's last token
 #pragma unroll
-            for (int rr = 0; rr < 4; ++rr)
+            for (int rr = 0; rr < R; ++rr)
                 if (i0 + rr < p.dk_) {
                     float* dst = ck_at(dir == 0 ? p.ckS : p.ckG, t / kC, i0 + rr);
                     reinterpret_cast<float4*>(dst)[0] = make_float4(X[rr][0], X[rr][1], X[rr][2], X[rr][3]);
                     reinterpret_cast<float4*>(dst)[1] = make_float4(X[rr][4], X[rr][5], X[rr][6], X[rr][7]);
                 }
-        const Rows4 rw = nrw;
+        const RowsR<R> rw = nrw;
         float cv[NC];
 #pragma unroll
         for (int c = 0; c < NC; ++c) cv[c] = nvec[c];
         if (n + 1 < p.T) {
             const int tnext = dir == 0 ? t + 1 : t - 1;
             const size_t tn = tok_of(tnext);
-            load_rows4<TI>(p, tn, tokq_of(tnext), i0, nrw);
+            load_rows<TI, R>(p, tn, tokq_of(tnext), i0, nrw);
             load8<TI>(colsrc, tn * p.dv_ + c0, nvec);
         }
         if (dir == 0) {
@@ -270,7 +283,7 @@ __global__ void __launch_bounds__(kScanWarps * 32) bwd_scan_kernel(Params p) {
 #pragma unroll
             for (int c = 0; c < NC; ++c) r[c] = 0.f;
 #pragma unroll
-            for (int rr = 0; rr < 4; ++rr) {
+            for (int rr = 0; rr < R; ++rr) {
                 const float e = rw.bg[rr] * rw.k[rr];
 #pragma unroll
                 for (int c = 0; c < NC; ++c) {
@@ -280,7 +293,7 @@ __global__ void __launch_bounds__(kScanWarps * 32) bwd_scan_kernel(Params p) {
             }
             warp_allsum<NC>(r, lane);
 #pragma unroll
-            for (int rr = 0; rr < 4; ++rr) {
+            for (int rr = 0; rr < R; ++rr) {
                 const float u = rw.wg[rr] * rw.k[rr];
 #pragma unroll
                 for (int c = 0; c < NC; ++c)
@@ -297,7 +310,7 @@ __global__ void __launch_bounds__(kScanWarps * 32) bwd_scan_kernel(Params p) {
 #pragma unroll
             for (int c = 0; c < 2 * NC; ++c) z[c] = 0.f;
 #pragma unroll
-            for (int rr = 0; rr < 4; ++rr) {
+            for (int rr = 0; rr < R; ++rr) {
                 const float u = rw.wg[rr] * rw.k[rr];
 #pragma unroll
                 for (int c = 0; c < NC; ++c) {
@@ -308,7 +321,7 @@ __global__ void __launch_bounds__(kScanWarps * 32) bwd_scan_kernel(Params p) {
             }
             warp_allsum<2 * NC>(z, lane);
 #pragma unroll
-            for (int rr = 0; rr < 4; ++rr) {
+            for (int rr = 0; rr < R; ++rr) {
                 const float e = rw.bg[rr] * rw.k[rr];
 #pragma unroll
                 for (int c = 0; c < NC; ++c) X[rr][c] = rw.a[rr] * fmaf(-e, z[c], X[rr][c]);
@@ -325,7 +338,7 @@ __global__ void __launch_bounds__(kScanWarps * 32) bwd_scan_kernel(Params p) {
     }
     if (dir == 1 && p.dS0)
 #pragma unroll
-        for (int rr = 0; rr < 4; ++rr)
+        for (int rr = 0; rr < R; ++rr)
             if (i0 + rr < p.dk_) {
                 float* dst = p.dS0 + (head * p.dk_ + i0 + rr) * p.dv_ + c0;
                 reinterpret_cast<float4*>(dst)[0] = make_float4(X[rr][0], X[rr][1], X[rr][2], X[rr][3]);
@@ -342,7 +355,7 @@ constexpr int kNT = 8;
 
 template <typename TI>
 struct ScanStage {
-    TI rows[5][kNT][kMaxDK];                  // q, k, alpha, b, w (channel kinds)
+    TI rows[5][kNT][kStagedMaxDK];            // q, k, alpha, b, w (channel kinds)
     TI cols[kNT][kScanWarps * kScanCols];     // v (forward) or dO (backward)
     float scal[3][kNT];                       // scalar alpha, b, w
 };
@@ -918,10 +931,12 @@ cudaError_t launch_typed(Params p, const CUtensorMap* tc_maps, const CUtensorMap
         return e;
     }
     const dim3 sgrid((p.dv_ + kScanCols * kScanWarps - 1) / (kScanCols * kScanWarps), p.H, 2 * p.B);
-    if ((p.dk_ * sizeof(TI)) % 16 == 0)
+    if (p.dk_ > kStagedMaxDK)
+        bwd_scan_kernel<TI, 8><<<sgrid, kScanWarps * 32, 0, st>>>(p);
+    else if ((p.dk_ * sizeof(TI)) % 16 == 0)
         bwd_scan_staged_kernel<TI><<<sgrid, kScanWarps * 32, 0, st>>>(p);
     else
-        bwd_scan_kernel<TI><<<sgrid, kScanWarps * 32, 0, st>>>(p);
+        bwd_scan_kernel<TI, 4><<<sgrid, kScanWarps * 32, 0, st>>>(p);
     e = cudaGetLastError();
     if (e != cudaSuccess) return e;
     const uint32_t smem = chunk_smem(p.tpr).total;

@@ -279,7 +279,7 @@ size_t gdr_chunk_fwd_static_capacity(void);
  *     states elementwise; a third kernel sums scalar gates' gradients over
  *     the key channels; d_status unused.
  *   Deterministic (no atomics) on both paths.
- * Supported: chunk = 64, 1 <= d_k <= 128, d_v a multiple of 8 up to 256,
+ * Supported: chunk = 64, 1 <= d_k <= 256, d_v a multiple of 8 up to 256,
  *   ceil(T / 64) <= 65535 and B * H <= 65535. Every pointer 16-byte
  *   aligned, except scalar gates and their gradients (element aligned).
  * Returns GDR_OK, GDR_ERR_INVALID_ARG (bad sizes or kinds, a NULL array that

@@ -163,7 +163,7 @@ def bwd(**kw):
     (dict(ws=NULL), _lib.GDR_ERR_INVALID_ARG),
     (dict(ws_bytes=1024), _lib.GDR_ERR_INVALID_ARG),     # workspace too small
     (dict(chunk=32), _lib.GDR_ERR_UNSUPPORTED),
-    (dict(dk=256), _lib.GDR_ERR_UNSUPPORTED),
+    (dict(dk=320), _lib.GDR_ERR_UNSUPPORTED),
     (dict(dv=264), _lib.GDR_ERR_UNSUPPORTED),
     (dict(dv=44), _lib.GDR_ERR_UNSUPPORTED),
     (dict(dO=P + 8), _lib.GDR_ERR_MISALIGNED),

@@ -96,10 +96,11 @@ def test_ragged_lengths(cuda_device, T):
 
 
 @pytest.mark.parametrize("dk,dv", [(128, 64), (64, 128), (40, 48), (16, 16), (100, 112), (128, 8),
-                                   (128, 256), (7, 24)])
+                                   (128, 256), (7, 24), (256, 256), (200, 64), (256, 8)])
 def test_head_shapes(cuda_device, dk, dv):
-    """1 to 32 threads per state row (d_v / 8), some of them idle, and row
-    blocks that run past d_k."""
+    """1 to 32 threads per state row (d_v / 8), some of them idle, row
+    blocks that run past d_k, and d_k above 128 (8 state rows per lane in the
+    scans)."""
     wl = WORKLOADS["kda"].with_(B=1, H=3, T=90, dk=dk, dv=dv, dtype="fp32", s0=True, seed=dk + dv)
     inp = make_chunk_inputs(wl)
     cot = make_cotangents(wl)
@@ -221,3 +222,14 @@ def test_tensor_core_deterministic_and_status(cuda_device):
         if outs[0][n] is not None:
             np.testing.assert_array_equal(outs[0][n], outs[1][n])
     check(outs[0], run_oracle_bwd(inp, cot), wl)
+
+
+@pytest.mark.parametrize("T", [1, 70])
+def test_dk256_gated_deltanet_bf16(cuda_device, T):
+    """The Gated DeltaNet head width d_k = d_v = 256 in bf16 (its forward runs
+    on tensor cores; its backward on the fp32 CUDA-core path, held to the
+    fp32 bar)."""
+    wl = WORKLOADS["gdn256"].with_(B=1, H=2, T=T, s0=True, seed=1900 + T)
+    inp = make_chunk_inputs(wl)
+    cot = make_cotangents(wl)
+    check(run_bwd(inp, cot, cuda_device), run_oracle_bwd(inp, cot), wl, f"T={T} ")
