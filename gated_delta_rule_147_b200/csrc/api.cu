@@ -25,7 +25,7 @@ size_t twopass_workspace_bytes(int B, int T, int H, int dv);
 cudaError_t launch_chunk_twopass_gdn(const CUtensorMap* maps, const CUtensorMap* ws_maps, void* ws,
                                      const void* alpha, const void* beta, const float* S0, void* o,
                                      float* ST, int* d_status, int B, int T, int H, int dv, int group,
-                                     cudaStream_t st, float* ckS = nullptr, float* up = nullptr);
+                                     cudaStream_t st, __nv_bfloat16* ckS = nullptr, __nv_bfloat16* up = nullptr);
 size_t twopass256_workspace_bytes(int B, int T, int H, int dv);
 cudaError_t launch_chunk_twopass_gdn256(const CUtensorMap* maps, const CUtensorMap* ws_maps,
                                         const void* alpha, const void* beta, const float* S0, void* o,

@@ -40,20 +40,19 @@
 #include "common.cuh"
 
 namespace gdr {
-cudaError_t launch_bwd_chunk_tc(const CUtensorMap* maps, const float* ckS, const float* ckG,
-                                const float* R, const float* DR, const void* alpha,
-                                const void* beta, const void* v, bool r_from_u, float* dq, float* dk,
-                                float* dalpha, float* db, int* d_status, int B, int T, int H,
-                                int group, int nchunks, cudaStream_t st);
+cudaError_t launch_bwd_chunk_tc(const CUtensorMap* maps, const CUtensorMap* ck_maps, const void* alpha,
+                                const void* beta, float* dq, float* dk, float* dalpha, float* db,
+                                int* d_status, int B, int T, int H, int group, int nchunks,
+                                cudaStream_t st);
 bool make_tma_map_bf16(CUtensorMap* m, const void* base, int B, int T, int H, int d);
 size_t twopass_workspace_bytes(int B, int T, int H, int dv);
 cudaError_t launch_chunk_twopass_gdn(const CUtensorMap* maps, const CUtensorMap* ws_maps, void* ws,
                                      const void* alpha, const void* beta, const float* S0, void* o,
                                      float* ST, int* d_status, int B, int T, int H, int dv, int group,
-                                     cudaStream_t st, float* ckS, float* up);
+                                     cudaStream_t st, __nv_bfloat16* ckS, __nv_bfloat16* up);
 cudaError_t launch_bwd_grad_tc(const CUtensorMap* q_map, const CUtensorMap* k_map, const CUtensorMap* do_map,
                                const CUtensorMap* ws_maps, const void* alpha, const void* beta,
-                               const float* dST, float* ckG, float* DR, float* dv, float* dS0,
+                               const float* dST, __nv_bfloat16* ckG, __nv_bfloat16* DR, float* dv, float* dS0,
                                int* d_status, int B, int T, int H, int dvn, int group, cudaStream_t st);
 
 namespace bwd {
@@ -908,20 +907,24 @@ WsLayout ws_layout(int B, int T, int H, int dk, int dv, bool grouped) {
 // every token; the chunkwise gradient pass (its factors in the same
 // workspace region once the forward is done, maps gw_maps) gives the state
 // gradient at every chunk end, dr, dv and dS0; the tensor-core pass 2 writes
-// the scalar gate gradients itself.
+// the scalar gate gradients itself. On this path the checkpoints are bf16
+// (the start of each checkpoint region; ck_maps: U, dr, S, G).
 template <typename TI>
 cudaError_t launch_typed(Params p, const CUtensorMap* tc_maps, const CUtensorMap* fw_maps, void* fw,
-                         const CUtensorMap* gw_maps, cudaStream_t st) {
+                         const CUtensorMap* gw_maps, const CUtensorMap* ck_maps, cudaStream_t st) {
     cudaError_t e;
     if (tc_maps) {
         e = launch_chunk_twopass_gdn(tc_maps, fw_maps, fw, p.alpha, p.b, p.S0, nullptr, nullptr,
-                                     p.d_status, p.B, p.T, p.H, p.dv_, p.group, st, p.ckS, p.R);
+                                     p.d_status, p.B, p.T, p.H, p.dv_, p.group, st,
+                                     reinterpret_cast<__nv_bfloat16*>(p.ckS),
+                                     reinterpret_cast<__nv_bfloat16*>(p.R));
         if (e != cudaSuccess) return e;
-        e = launch_bwd_grad_tc(&tc_maps[0], &tc_maps[1], &tc_maps[3], gw_maps, p.alpha, p.b, p.dST, p.ckG,
-                               p.DR, p.dv, p.dS0, p.d_status, p.B, p.T, p.H, p.dv_, p.group, st);
+        e = launch_bwd_grad_tc(&tc_maps[0], &tc_maps[1], &tc_maps[3], gw_maps, p.alpha, p.b, p.dST,
+                               reinterpret_cast<__nv_bfloat16*>(p.ckG), reinterpret_cast<__nv_bfloat16*>(p.DR),
+                               p.dv, p.dS0, p.d_status, p.B, p.T, p.H, p.dv_, p.group, st);
         if (e != cudaSuccess) return e;
-        e = launch_bwd_chunk_tc(tc_maps, p.ckS, p.ckG, p.R, p.DR, p.alpha, p.b, p.v, true, p.dq, p.dk,
-                                p.dalpha, p.db, p.d_status, p.B, p.T, p.H, p.group, p.nchunks, st);
+        e = launch_bwd_chunk_tc(tc_maps, ck_maps, p.alpha, p.b, p.dq, p.dk, p.dalpha, p.db, p.d_status,
+                                p.B, p.T, p.H, p.group, p.nchunks, st);
         if (e != cudaSuccess) return e;
         if (p.group > 1) {
             const size_t n = (size_t)p.B * p.T * p.Hq * p.dk_;
@@ -1065,11 +1068,14 @@ gdr_status gdr_chunk_bwd_grouped(const void* q, const void* k, const void* v, co
     p.d_status = d_status;
     // the Gated DeltaNet form on tensor cores: scalar decay, tied scalar beta,
     // bf16, d_k = d_v = 128
-    CUtensorMap maps[4], fw_maps[3], gw_maps[3];
+    CUtensorMap maps[4], fw_maps[3], gw_maps[3], ck_maps[4];
     const CUtensorMap* tc_maps = nullptr;
     void* fw = ws + wl.FW;
+    // the checkpoints' tensor maps view each as [B H nchunks 128, 128] rows (int32 coordinates)
+    const bool ck_rows_fit = (size_t)B * H * nch * 128 <= (size_t)INT32_MAX;
     if (dtype == GDR_BF16 && d_k == 128 && d_v == 128 && alpha_kind == GDR_GATE_SCALAR &&
-        b_kind == GDR_GATE_SCALAR && w_kind == GDR_GATE_TIED) {
+        b_kind == GDR_GATE_SCALAR && w_kind == GDR_GATE_TIED && ck_rows_fit) {
+        const int ck_rows = B * H * nch * 128;
         if (!gdr::make_tma_map_bf16(&maps[0], q, B, T, H_qk, d_k) ||
             !gdr::make_tma_map_bf16(&maps[1], k, B, T, H_qk, d_k) ||
             !gdr::make_tma_map_bf16(&maps[2], v, B, T, H, d_v) ||
@@ -1081,14 +1087,19 @@ gdr_status gdr_chunk_bwd_grouped(const void* q, const void* k, const void* v, co
             // (2 B T H (128 + 64 + 128) bytes) once the forward has read its own
             !gdr::make_tma_map_bf16(&gw_maps[0], fw, B, T, H, d_k) ||
             !gdr::make_tma_map_bf16(&gw_maps[1], ws + wl.FW + (size_t)B * T * H * d_k * 2, B, T, H, 64) ||
-            !gdr::make_tma_map_bf16(&gw_maps[2], ws + wl.FW + (size_t)B * T * H * (d_k + 64) * 2, B, T, H, d_k))
+            !gdr::make_tma_map_bf16(&gw_maps[2], ws + wl.FW + (size_t)B * T * H * (d_k + 64) * 2, B, T, H, d_k) ||
+            // bf16 checkpoints: U, dr per token; S, G per chunk
+            !gdr::make_tma_map_bf16(&ck_maps[0], ws + wl.R, B, T, H, d_v) ||
+            !gdr::make_tma_map_bf16(&ck_maps[1], ws + wl.DR, B, T, H, d_v) ||
+            !gdr::make_tma_map_bf16(&ck_maps[2], ws + wl.ckS, 1, ck_rows, 1, d_v) ||
+            !gdr::make_tma_map_bf16(&ck_maps[3], ws + wl.ckG, 1, ck_rows, 1, d_v))
             return GDR_ERR_NO_DEVICE;
         tc_maps = maps;
         p.GP = nullptr;
     }
     const cudaError_t e = dtype == GDR_BF16
-                              ? gdr::bwd::launch_typed<__nv_bfloat16>(p, tc_maps, fw_maps, fw, gw_maps, st)
-                              : gdr::bwd::launch_typed<float>(p, nullptr, nullptr, nullptr, nullptr, st);
+                              ? gdr::bwd::launch_typed<__nv_bfloat16>(p, tc_maps, fw_maps, fw, gw_maps, ck_maps, st)
+                              : gdr::bwd::launch_typed<float>(p, nullptr, nullptr, nullptr, nullptr, nullptr, st);
     return e == cudaSuccess ? GDR_OK : GDR_ERR_LAUNCH;
 }
 

@@ -408,8 +408,8 @@ struct GradParams {
     const void* alpha;  // [B, T, H] scalar gates (bf16)
     const void* beta;
     const float* dST;   // [B, H, 128, d_v] or NULL
-    float* ckG;         // [B, H, nchunks, 128, d_v]: G_in of every chunk
-    float* DR;          // [B, T, H, d_v]: dr = -k G
+    __nv_bfloat16* ckG; // [B, H, nchunks, 128, d_v] bf16: G_in of every chunk
+    __nv_bfloat16* DR;  // [B, T, H, d_v] bf16: dr = -k G
     float* dv;          // [B, T, H, d_v]: beta k G
     float* dS0;         // [B, H, 128, d_v] or NULL
     int* d_status;
@@ -626,10 +626,12 @@ __global__ void __launch_bounds__(G_NT, 1) state_grad_kernel(
             // G_in of the chunk (the gradient its last state receives from later
             // tokens), written by each thread for its row off the chunk chain
             auto store_ck = [&]() {
-                float* dst = p.ckG + ((((size_t)bb * H + h) * nchunks + ci) * DK + row) * p.dv_ + v0 + wg * NH;
+                __nv_bfloat16* dst = p.ckG + ((((size_t)bb * H + h) * nchunks + ci) * DK + row) * p.dv_ + v0 + wg * NH;
 #pragma unroll
-                for (int jj = 0; jj < NH; jj += 4)
-                    *reinterpret_cast<float4*>(dst + jj) = make_float4(G[jj], G[jj + 1], G[jj + 2], G[jj + 3]);
+                for (int jj = 0; jj < NH; jj += 8)
+                    *reinterpret_cast<uint4*>(dst + jj) =
+                        make_uint4(pack_bf16x2(G[jj], G[jj + 1]), pack_bf16x2(G[jj + 2], G[jj + 3]),
+                                   pack_bf16x2(G[jj + 4], G[jj + 5]), pack_bf16x2(G[jj + 6], G[jj + 7]));
             };
             if (lo) {
                 // ---- Y of the chunk's tokens: dv, dr, and Y' = -Diag(beta g) Y ----------
@@ -654,12 +656,14 @@ __global__ void __launch_bounds__(G_NT, 1) state_grad_kernel(
                 if (t < T) {
                     const size_t off = (((size_t)bb * T + t) * H + h) * p.dv_ + v0 + wg * 32;
 #pragma unroll
-                    for (int c4 = 0; c4 < 32; c4 += 4) {
+                    for (int c4 = 0; c4 < 32; c4 += 4)
                         *reinterpret_cast<float4*>(p.dv + off + c4) =
                             make_float4(bj * d[c4], bj * d[c4 + 1], bj * d[c4 + 2], bj * d[c4 + 3]);
-                        *reinterpret_cast<float4*>(p.DR + off + c4) =
-                            make_float4(-d[c4], -d[c4 + 1], -d[c4 + 2], -d[c4 + 3]);
-                    }
+#pragma unroll
+                    for (int c8 = 0; c8 < 32; c8 += 8)
+                        *reinterpret_cast<uint4*>(p.DR + off + c8) =
+                            make_uint4(pack_bf16x2(-d[c8], -d[c8 + 1]), pack_bf16x2(-d[c8 + 2], -d[c8 + 3]),
+                                       pack_bf16x2(-d[c8 + 4], -d[c8 + 5]), pack_bf16x2(-d[c8 + 6], -d[c8 + 7]));
                 }
                 store_ck();
             } else {
@@ -709,10 +713,11 @@ size_t bwd_grad_workspace_bytes(int B, int T, int H) {
 }
 
 // maps: q, k ([B,T,H/group,128]) and dO ([B,T,H,128]); ws_maps: X ([B,T,H,128]),
-// AqT ([B,T,H,64]), Q~ ([B,T,H,128]). Writes ckG, DR, dv and (if not NULL) dS0.
+// AqT ([B,T,H,64]), Q~ ([B,T,H,128]). Writes ckG and DR (bf16), dv and (if not
+// NULL) dS0.
 cudaError_t launch_bwd_grad_tc(const CUtensorMap* q_map, const CUtensorMap* k_map, const CUtensorMap* do_map,
                                const CUtensorMap* ws_maps, const void* alpha, const void* beta,
-                               const float* dST, float* ckG, float* DR, float* dv, float* dS0,
+                               const float* dST, __nv_bfloat16* ckG, __nv_bfloat16* DR, float* dv, float* dS0,
                                int* d_status, int B, int T, int H, int dvn, int group, cudaStream_t st) {
     using namespace bwdgrad;
     if (dvn != 128) return cudaErrorInvalidValue;

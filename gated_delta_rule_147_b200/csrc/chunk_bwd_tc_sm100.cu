@@ -4,7 +4,8 @@
 //
 // The gradients of a chunk follow from its start state S0, the state gradient
 // G_e at its end and, per token, the erase read r_t and its gradient dr_t
-// (both from the two scans of the backward pass): with r and dr known the
+// (checkpoints of the backward's forward and gradient passes, bf16; r comes as
+// U = beta v - r): with r and dr known the
 // chunk is a diagonal-decay system without erase, and every gradient is a
 // masked product ("The Eraser Trilogy", "The Rosetta Stone": the masked-
 // matrix form of such a system). With l_t the prefix sum of log2 alpha over
@@ -30,8 +31,9 @@
 //   terms (no decay) to cancel between two separately rounded sums.
 // Every decay factor used is at most 1, so any alpha in (0, 1] is in range.
 //
-// One CTA per (chunk, head, batch), 256 threads; thread 0 issues the MMAs
-// (bf16 operands, fp32 accumulators in tensor memory), three products:
+// One CTA per (chunk, head, batch), 256 threads; thread 0 loads every operand
+// tile by TMA (q, k, v, dO, U, dr, S0, G_e) and issues the MMAs (bf16
+// operands, fp32 accumulators in tensor memory), three products:
 //   D12 = [dO ; DR] [S0 | V | R]^T            (N = 256: dO S0^T, DR S0^T and
 //                                              the four token-by-token blocks)
 //   D7  = [Q ; U] K^T                           (q_t . k_j and e_t . k_j for M)
@@ -47,12 +49,7 @@ namespace bwdtc {
 using namespace chunkc;
 
 struct TcParams {
-    const float *ckS, *ckG, *R, *DR;       // scans: chunk-start states, chunk-end state
-                                           // gradients, r, dr (fp32)
     const __nv_bfloat16 *alpha, *beta;     // scalar gates [B, T, H]
-    const __nv_bfloat16* v;                // [B, T, H, 128]
-    int r_from_u;                          // R holds U = beta v - r (from the forward
-                                           // kernels): r = beta v - U
     float *dq, *dk, *dalpha, *db;          // dq, dk [B, T, H, 128] per value head; gates [B, T, H]
     int* d_status;
     int T, H, group, nchunks;
@@ -62,12 +59,12 @@ struct TcParams {
 constexpr uint32_t R0 = 0;          // [dO ; DR] bf16 [128 x 128] (K-major A of D12);
                                     // after D12: [V' ; -R'] (A of the G_e product)
 constexpr uint32_t R1 = 32768;      // B of D12, per 64-column K block (32 KB): rows 0..127
-                                    // S0 (row = key channel), 128..191 V, 192..255 R;
-                                    // after D12 rows 0..127 hold G_e; after the last
-                                    // product, fp32 staging of du
+                                    // S0 (row = key channel), 128..191 V, 192..255 U,
+                                    // then R; after the last product, fp32 staging of du
 constexpr uint32_t R2 = 98304;      // per 64-channel block (24 KB): Q, U = beta K, K rows
 constexpr uint32_t R3 = 147456;     // [[P1, -P2] ; [P3, -P4]] bf16 [128 x 128]
-constexpr uint32_t SMALL = 180224;
+constexpr uint32_t R4 = 180224;     // G_e, per 64-column K block (16 KB): 128 rows
+constexpr uint32_t SMALL = 212992;
 constexpr uint32_t SMEM_BYTES = SMALL + 8192 + 64 + 1024;
 // D6 takes D12's columns 128..255 once the masked blocks have been formed;
 // D7 sits in D3's columns until then
@@ -79,18 +76,14 @@ __device__ __forceinline__ void put32(uint8_t* tile, int row, int ch0, int rows,
     for (int c = 0; c < 4; ++c) st_chunk(tile, sw128_chunk(row, ch0 + c, rows), x + 8 * c);
 }
 
-__device__ __forceinline__ void ld32f(const float* g, float* x) {
-#pragma unroll
-    for (int c = 0; c < 8; ++c) {
-        const float4 v = reinterpret_cast<const float4*>(g)[c];
-        x[4 * c] = v.x; x[4 * c + 1] = v.y; x[4 * c + 2] = v.z; x[4 * c + 3] = v.w;
-    }
-}
-
 __global__ void __launch_bounds__(256, 1) bwd_chunk_tc_kernel(const __grid_constant__ CUtensorMap tm_q,
                                                               const __grid_constant__ CUtensorMap tm_k,
                                                               const __grid_constant__ CUtensorMap tm_v,
                                                               const __grid_constant__ CUtensorMap tm_do,
+                                                              const __grid_constant__ CUtensorMap tm_u,
+                                                              const __grid_constant__ CUtensorMap tm_dr,
+                                                              const __grid_constant__ CUtensorMap tm_s0,
+                                                              const __grid_constant__ CUtensorMap tm_ge,
                                                               const TcParams p) {
     extern __shared__ uint8_t smem_raw[];
     uint8_t* sm = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) &
@@ -113,6 +106,7 @@ __global__ void __launch_bounds__(256, 1) bwd_chunk_tc_kernel(const __grid_const
     uint64_t* bar_tma = reinterpret_cast<uint64_t*>(sm + SMALL + 8192);
     uint64_t* bar_mma = bar_tma + 1;
     uint64_t* bar_drain = bar_tma + 2;
+    uint64_t* bar_ge = bar_tma + 3;
     uint32_t* s_tmem = reinterpret_cast<uint32_t*>(sm + SMALL + 8192 + 32);
     const uint32_t sbase = smem_u32(sm);
 
@@ -120,14 +114,27 @@ __global__ void __launch_bounds__(256, 1) bwd_chunk_tc_kernel(const __grid_const
         mbar_init(bar_tma, 1);
         mbar_init(bar_mma, 1);
         mbar_init(bar_drain, 1);
+        mbar_init(bar_ge, 1);
         fence_barrier_init();
-        mbar_expect_tx(bar_tma, 8u * 8192u);
+        // checkpoint rows: (head, chunk) -> 128 rows of a [rows, 128] view
+        const int ck_row = (int)((head * p.nchunks + c) * 128);
+        mbar_expect_tx(bar_tma, 16u * 8192u);
 #pragma unroll
         for (int blk = 0; blk < 2; ++blk) {
             tma_load_4d(sm + R0 + blk * 16384, &tm_do, bar_tma, 64 * blk, h, t0, bb);
+            tma_load_4d(sm + R0 + blk * 16384 + 8192, &tm_dr, bar_tma, 64 * blk, h, t0, bb);
+            tma_load_4d(sm + R1 + blk * 32768, &tm_s0, bar_tma, 64 * blk, 0, ck_row, 0);
+            tma_load_4d(sm + R1 + blk * 32768 + 8192, &tm_s0, bar_tma, 64 * blk, 0, ck_row + 64, 0);
             tma_load_4d(sm + R1 + blk * 32768 + 16384, &tm_v, bar_tma, 64 * blk, h, t0, bb);
+            tma_load_4d(sm + R1 + blk * 32768 + 24576, &tm_u, bar_tma, 64 * blk, h, t0, bb);
             tma_load_4d(sm + R2 + blk * 24576, &tm_q, bar_tma, 64 * blk, hq, t0, bb);
             tma_load_4d(sm + R2 + blk * 24576 + 16384, &tm_k, bar_tma, 64 * blk, hq, t0, bb);
+        }
+        mbar_expect_tx(bar_ge, 4u * 8192u);
+#pragma unroll
+        for (int blk = 0; blk < 2; ++blk) {
+            tma_load_4d(sm + R4 + blk * 16384, &tm_ge, bar_ge, 64 * blk, 0, ck_row, 0);
+            tma_load_4d(sm + R4 + blk * 16384 + 8192, &tm_ge, bar_ge, 64 * blk, 0, ck_row + 64, 0);
         }
     }
     if (warp == 0) tmem_alloc(s_tmem, TM_COLS);
@@ -136,43 +143,6 @@ __global__ void __launch_bounds__(256, 1) bwd_chunk_tc_kernel(const __grid_const
         const size_t gi = ((size_t)bb * T + t0 + min(tid, n - 1)) * H + h;
         s_alpha[tid] = valid ? __bfloat162float(p.alpha[gi]) : 1.f;
         s_beta[tid] = valid ? __bfloat162float(p.beta[gi]) : 0.f;
-    }
-    // DR -> rows 64..127 of R0, R -> rows 192..255 of R1, S0 -> rows 0..127 of R1 (bf16)
-    {
-        const int t = tid >> 2, part = tid & 3;  // token, 32 value columns
-        float x[32];
-        const size_t tok = ((size_t)bb * T + t0 + t) * H + h;
-        if (t < n) ld32f(p.DR + tok * 128 + part * 32, x);
-        else
-#pragma unroll
-            for (int e = 0; e < 32; ++e) x[e] = 0.f;
-        put32(sm + R0, 64 + t, part * 4, 128, x);
-        if (t < n) {
-            ld32f(p.R + tok * 128 + part * 32, x);
-            if (p.r_from_u) {
-                const float bt = __bfloat162float(p.beta[tok]);
-                const uint4* vp = reinterpret_cast<const uint4*>(p.v + tok * 128 + part * 32);
-#pragma unroll
-                for (int c4 = 0; c4 < 4; ++c4) {
-                    const uint4 u = vp[c4];
-                    const __nv_bfloat162* hh = reinterpret_cast<const __nv_bfloat162*>(&u);
-#pragma unroll
-                    for (int e = 0; e < 4; ++e) {
-                        const float2 f = __bfloat1622float2(hh[e]);
-                        x[c4 * 8 + 2 * e] = fmaf(bt, f.x, -x[c4 * 8 + 2 * e]);
-                        x[c4 * 8 + 2 * e + 1] = fmaf(bt, f.y, -x[c4 * 8 + 2 * e + 1]);
-                    }
-                }
-            }
-        }
-        put32(sm + R1, 192 + t, part * 4, 256, x);
-        const int i = tid >> 1, half = tid & 1;  // key channel, 64 value columns
-        const float* s0 = p.ckS + ((head * p.nchunks + c) * 128 + i) * 128 + half * 64;
-#pragma unroll
-        for (int q2 = 0; q2 < 2; ++q2) {
-            ld32f(s0 + q2 * 32, x);
-            put32(sm + R1, i, half * 8 + q2 * 4, 256, x);
-        }
     }
     tc_fence_before();
     __syncthreads();
@@ -211,7 +181,8 @@ __global__ void __launch_bounds__(256, 1) bwd_chunk_tc_kernel(const __grid_const
         uint32_t ph_tma = 0;
         GDR_WAIT(bar_tma, ph_tma);
     }
-    // U = beta K (rows of the K tile scaled per token) next to Q and K
+    // U = beta K (rows of the K tile scaled per token) next to Q and K; the
+    // erase reads r = beta v - U in place of U (rows 192..255 of R1, beside V)
     {
         const int t = tid >> 2, part = tid & 3;  // token, 4 of the 16 pieces of its 128 channels
         const float f = s_beta[t];
@@ -219,11 +190,16 @@ __global__ void __launch_bounds__(256, 1) bwd_chunk_tc_kernel(const __grid_const
         for (int q4 = 0; q4 < 4; ++q4) {
             const int ch = part * 4 + q4, blk = ch >> 3;
             const uint32_t off = sw128_chunk(t, ch & 7, 64);
-            float x[8];
+            float x[8], y[8];
             ld_chunk(sm + R2 + blk * 24576 + 16384, off, x);
 #pragma unroll
             for (int e = 0; e < 8; ++e) x[e] *= f;
             st_chunk(sm + R2 + blk * 24576 + 8192, off, x);
+            ld_chunk(sm + R1 + blk * 32768 + 16384, off, x);  // v (rows 128 + t: same swizzle)
+            ld_chunk(sm + R1 + blk * 32768 + 24576, off, y);  // U
+#pragma unroll
+            for (int e = 0; e < 8; ++e) y[e] = fmaf(f, x[e], -y[e]);
+            st_chunk(sm + R1 + blk * 32768 + 24576, off, y);
         }
     }
     fence_proxy_async();
@@ -254,7 +230,7 @@ __global__ void __launch_bounds__(256, 1) bwd_chunk_tc_kernel(const __grid_const
     GDR_WAIT(bar_mma, ph_mma);
     tc_fence_after();
 
-    // ---- masked, decay-scaled blocks -> R3; G_e -> R1 rows 0..127; [V' ; -R'] -> R0 ----
+    // ---- masked, decay-scaled blocks -> R3; [V' ; -R'] -> R0 ----------------------------
     {
         // lanes 0..63 (token t): dO V^T (wg 0) and dO R^T (wg 1), mask j <= t;
         // lanes 64..127: DR V^T and DR R^T, mask j < t
@@ -293,15 +269,6 @@ __global__ void __launch_bounds__(256, 1) bwd_chunk_tc_kernel(const __grid_const
         }
     }
     {
-        // G_e (fp32) -> rows 0..127 of R1, as S0 was
-        const int i = tid >> 1, half = tid & 1;
-        const float* ge = p.ckG + ((head * p.nchunks + c) * 128 + i) * 128 + half * 64;
-        float x[32];
-#pragma unroll
-        for (int q2 = 0; q2 < 2; ++q2) {
-            ld32f(ge + q2 * 32, x);
-            put32(sm + R1, i, half * 8 + q2 * 4, 256, x);
-        }
         // rows t of V and R scaled by Gam_C / Gam_t (R negated) -> R0
         const int t = tid >> 2, part = tid & 3;
         const float f = s_gcr[t];
@@ -321,7 +288,10 @@ __global__ void __launch_bounds__(256, 1) bwd_chunk_tc_kernel(const __grid_const
     }
     fence_proxy_async();
     tc_fence_before();
-    __syncthreads();
+    {
+        uint32_t ph_ge = 0;  // G_e (loaded at the start) has landed
+        GDR_WAIT(bar_ge, ph_ge);
+    }
 
     // ---- D3 = P [U ; K];  D45 = P^T [Q ; U];  D6 = [V' ; -R'] G_e^T ----------------
     if (tid == 0) {
@@ -340,19 +310,21 @@ __global__ void __launch_bounds__(256, 1) bwd_chunk_tc_kernel(const __grid_const
 #pragma unroll
         for (int ks = 0; ks < 8; ++ks)
             mma_bf16(tmem + TM_D6, sdesc_sw128(sbase + R0 + (ks >> 2) * 16384u + (ks & 3) * 32u, 16, 1024),
-                     sdesc_sw128(sbase + R1 + (ks >> 2) * 32768u + (ks & 3) * 32u, 16, 1024), id5, ks > 0);
+                     sdesc_sw128(sbase + R4 + (ks >> 2) * 16384u + (ks & 3) * 32u, 16, 1024), id5, ks > 0);
         mma_commit(bar_mma);
     }
-    // <G_e, S0> over the whole state
+    // <G_e, S0> over the whole state, from the two tiles in shared memory (the
+    // same 128-byte swizzle at 1024-aligned bases pairs equal elements)
     {
-        const float* se = p.ckS + (head * p.nchunks + c) * 16384;
-        const float* ge = p.ckG + (head * p.nchunks + c) * 16384;
         float acc = 0.f;
 #pragma unroll 4
-        for (int e = tid * 4; e < 16384; e += 1024) {
-            const float4 a = *reinterpret_cast<const float4*>(ge + e);
-            const float4 b = *reinterpret_cast<const float4*>(se + e);
-            acc = fmaf(a.x, b.x, fmaf(a.y, b.y, fmaf(a.z, b.z, fmaf(a.w, b.w, acc))));
+        for (int i = tid; i < 2048; i += 256) {
+            const uint32_t blk = (uint32_t)i >> 10, o = ((uint32_t)i & 1023u) * 16u;
+            float a[8], b[8];
+            ld_chunk(sm + R4 + blk * 16384, o, a);
+            ld_chunk(sm + R1 + blk * 32768, o, b);
+#pragma unroll
+            for (int e = 0; e < 8; ++e) acc = fmaf(a[e], b[e], acc);
         }
 #pragma unroll
         for (int off = 16; off > 0; off >>= 1) acc += __shfl_xor_sync(0xffffffffu, acc, off);
@@ -473,6 +445,7 @@ finish:
         // before the block leaves (each wait bounded): the input copies have
         // landed and every issued MMA has finished
         (void)mbar_wait(bar_tma, 0);
+        (void)mbar_wait(bar_ge, 0);
         mma_commit(bar_drain);
         (void)mbar_wait(bar_drain, 0);
         flag_status(p.d_status, GDR_DEVICE_TIMEOUT);
@@ -486,23 +459,23 @@ finish:
 }  // namespace bwdtc
 
 // maps: q, k (q/k heads), v, dO (value heads), bf16 [B, T, H, 128] each.
-cudaError_t launch_bwd_chunk_tc(const CUtensorMap* maps, const float* ckS, const float* ckG,
-                                const float* R, const float* DR, const void* alpha,
-                                const void* beta, const void* v, bool r_from_u, float* dq, float* dk,
-                                float* dalpha, float* db, int* d_status, int B, int T, int H,
-                                int group, int nchunks, cudaStream_t st) {
+// ck_maps: U = beta v - r and dr (bf16 [B, T, H, 128]), the chunk-start states
+// and the chunk-end state gradients (bf16 [B, H, nchunks, 128, 128], each
+// mapped as one [B H nchunks 128, 128] view).
+cudaError_t launch_bwd_chunk_tc(const CUtensorMap* maps, const CUtensorMap* ck_maps, const void* alpha,
+                                const void* beta, float* dq, float* dk, float* dalpha, float* db,
+                                int* d_status, int B, int T, int H, int group, int nchunks,
+                                cudaStream_t st) {
     using namespace bwdtc;
     TcParams p;
-    p.ckS = ckS; p.ckG = ckG; p.R = R; p.DR = DR;
-    p.v = reinterpret_cast<const __nv_bfloat16*>(v);
-    p.r_from_u = r_from_u ? 1 : 0;
     p.alpha = reinterpret_cast<const __nv_bfloat16*>(alpha);
     p.beta = reinterpret_cast<const __nv_bfloat16*>(beta);
     p.dq = dq; p.dk = dk; p.dalpha = dalpha; p.db = db; p.d_status = d_status;
     p.T = T; p.H = H; p.group = group; p.nchunks = nchunks;
     cudaError_t e = cudaFuncSetAttribute(bwd_chunk_tc_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, SMEM_BYTES);
     if (e != cudaSuccess) return e;
-    bwd_chunk_tc_kernel<<<dim3(nchunks, H, B), 256, SMEM_BYTES, st>>>(maps[0], maps[1], maps[2], maps[3], p);
+    bwd_chunk_tc_kernel<<<dim3(nchunks, H, B), 256, SMEM_BYTES, st>>>(maps[0], maps[1], maps[2], maps[3], ck_maps[0],
+                                                                    ck_maps[1], ck_maps[2], ck_maps[3], p);
     return cudaGetLastError();
 }
 

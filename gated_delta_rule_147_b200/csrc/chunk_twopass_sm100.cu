@@ -474,12 +474,13 @@ __device__ __forceinline__ void mbar_arrive(uint64_t* bar) {
 // warps that wait for one chunk's output can never see the next completion of
 // the same barrier first.
 // Optional checkpoints for the backward pass, written off the chunk chain:
-// the fp32 state at every chunk start ([B, H, nchunks, 128, d_v]) and
-// U = P - W S of every token in fp32 ([B, T, H, d_v]; U = beta v - r, with r
-// the token's erase read).
+// the state at every chunk start ([B, H, nchunks, 128, d_v]) and U = P - W S
+// of every token ([B, T, H, d_v]; U = beta v - r, with r the token's erase
+// read), both bf16: the backward reads them only as tensor-core operands and
+// for one inner product per chunk.
 struct Ckpt {
-    float* ckS;
-    float* up;
+    __nv_bfloat16* ckS;
+    __nv_bfloat16* up;
 };
 
 // CKPT: the backward pass's instantiation (checkpoints written, o not written);
@@ -729,10 +730,12 @@ __global__ void __launch_bounds__(S_NT, 1) state_gdn_kernel(
             // the state at this chunk's start, for the backward pass (each thread
             // its row; the warps of lanes 64..127 once U has left)
             auto store_ck = [&]() {
-                float* dst = ck.ckS + ((((size_t)bb * H + h) * nchunks + ci) * DK + row) * p.dv + v0 + wg * NH;
+                __nv_bfloat16* dst = ck.ckS + ((((size_t)bb * H + h) * nchunks + ci) * DK + row) * p.dv + v0 + wg * NH;
 #pragma unroll
-                for (int jj = 0; jj < NH; jj += 4)
-                    *reinterpret_cast<float4*>(dst + jj) = make_float4(S[jj], S[jj + 1], S[jj + 2], S[jj + 3]);
+                for (int jj = 0; jj < NH; jj += 8)
+                    *reinterpret_cast<uint4*>(dst + jj) =
+                        make_uint4(pack_bf16x2(S[jj], S[jj + 1]), pack_bf16x2(S[jj + 2], S[jj + 3]),
+                                   pack_bf16x2(S[jj + 4], S[jj + 5]), pack_bf16x2(S[jj + 6], S[jj + 7]));
             };
             if (CKPT && lo) store_ck();
             if (lo) {
@@ -777,10 +780,12 @@ __global__ void __launch_bounds__(S_NT, 1) state_gdn_kernel(
                 mbar_arrive(u_ready);
                 if (CKPT) {  // U of every token and the chunk's start state, off the chain
                     if (ci * C + j < T) {
-                        float* up = ck.up + (((size_t)bb * T + ci * C + j) * H + h) * p.dv + v0 + wg * 32;
+                        __nv_bfloat16* up = ck.up + (((size_t)bb * T + ci * C + j) * H + h) * p.dv + v0 + wg * 32;
 #pragma unroll
-                        for (int c4 = 0; c4 < 32; c4 += 4)
-                            *reinterpret_cast<float4*>(up + c4) = make_float4(d[c4], d[c4 + 1], d[c4 + 2], d[c4 + 3]);
+                        for (int c8 = 0; c8 < 32; c8 += 8)
+                            *reinterpret_cast<uint4*>(up + c8) =
+                                make_uint4(pack_bf16x2(d[c8], d[c8 + 1]), pack_bf16x2(d[c8 + 2], d[c8 + 3]),
+                                           pack_bf16x2(d[c8 + 4], d[c8 + 5]), pack_bf16x2(d[c8 + 6], d[c8 + 7]));
                     }
                     store_ck();
                 }
@@ -832,12 +837,12 @@ size_t twopass_workspace_bytes(int B, int T, int H, int dv) {
 
 // maps: q, k, v, then the workspace maps -W ([B,T,H,128]), P ([B,T,H,d_v]) and
 // Aq ([B,T,H,64], the chunk's masked, decay-scaled Q K^T block row of each token).
-// ckS, up: the backward pass's checkpoints (struct Ckpt; both or neither), or NULL:
-// with them, o is not written.
+// ckS, up: the backward pass's bf16 checkpoints (struct Ckpt; both or neither),
+// or NULL: with them, o is not written.
 cudaError_t launch_chunk_twopass_gdn(const CUtensorMap* maps, const CUtensorMap* ws_maps, void* ws,
                                      const void* alpha, const void* beta, const float* S0, void* o,
                                      float* ST, int* d_status, int B, int T, int H, int dv, int group,
-                                     cudaStream_t st, float* ckS, float* up) {
+                                     cudaStream_t st, __nv_bfloat16* ckS, __nv_bfloat16* up) {
     using namespace twopass;
     PrepParams pp;
     pp.alpha = alpha; pp.beta = beta;
