@@ -98,6 +98,21 @@ namespace gdr {
 bool make_tma_map_bf16(CUtensorMap* m, const void* base, int B, int T, int H, int d) {
     return make_map(m, base, B, T, H, d);
 }
+
+// 4-D map over a [B, T, H, d] fp32 tensor, box {32 (d), 1 (H), 64 (T), 1 (B)}
+// (128-byte rows), 128-byte swizzle: the tile stores of fp32 outputs.
+bool make_tma_map_f32(CUtensorMap* m, const void* base, int B, int T, int H, int d) {
+    auto enc = encoder();
+    if (!enc) return false;
+    cuuint64_t dims[4] = {(cuuint64_t)d, (cuuint64_t)H, (cuuint64_t)T, (cuuint64_t)B};
+    cuuint64_t strides[3] = {(cuuint64_t)d * 4, (cuuint64_t)H * d * 4, (cuuint64_t)T * H * d * 4};
+    cuuint32_t box[4] = {32, 1, 64, 1};
+    cuuint32_t estr[4] = {1, 1, 1, 1};
+    CUresult r = enc(m, CU_TENSOR_MAP_DATA_TYPE_FLOAT32, 4, const_cast<void*>(base), dims, strides, box, estr,
+                     CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
+                     CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
+    return r == CUDA_SUCCESS;
+}
 }  // namespace gdr
 
 namespace {

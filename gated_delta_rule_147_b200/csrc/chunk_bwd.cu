@@ -45,6 +45,7 @@ cudaError_t launch_bwd_chunk_tc(const CUtensorMap* maps, const CUtensorMap* ck_m
                                 int* d_status, int B, int T, int H, int group, int nchunks,
                                 cudaStream_t st);
 bool make_tma_map_bf16(CUtensorMap* m, const void* base, int B, int T, int H, int d);
+bool make_tma_map_f32(CUtensorMap* m, const void* base, int B, int T, int H, int d);
 size_t twopass_workspace_bytes(int B, int T, int H, int dv);
 cudaError_t launch_chunk_twopass_gdn(const CUtensorMap* maps, const CUtensorMap* ws_maps, void* ws,
                                      const void* alpha, const void* beta, const float* S0, void* o,
@@ -908,7 +909,8 @@ WsLayout ws_layout(int B, int T, int H, int dk, int dv, bool grouped) {
 // workspace region once the forward is done, maps gw_maps) gives the state
 // gradient at every chunk end, dr, dv and dS0; the tensor-core pass 2 writes
 // the scalar gate gradients itself. On this path the checkpoints are bf16
-// (the start of each checkpoint region; ck_maps: U, dr, S, G).
+// (the start of each checkpoint region; ck_maps: U, dr, S, G, then the fp32
+// store maps of dq and dk).
 template <typename TI>
 cudaError_t launch_typed(Params p, const CUtensorMap* tc_maps, const CUtensorMap* fw_maps, void* fw,
                          const CUtensorMap* gw_maps, const CUtensorMap* ck_maps, cudaStream_t st) {
@@ -1068,7 +1070,7 @@ gdr_status gdr_chunk_bwd_grouped(const void* q, const void* k, const void* v, co
     p.d_status = d_status;
     // the Gated DeltaNet form on tensor cores: scalar decay, tied scalar beta,
     // bf16, d_k = d_v = 128
-    CUtensorMap maps[4], fw_maps[3], gw_maps[3], ck_maps[4];
+    CUtensorMap maps[4], fw_maps[3], gw_maps[3], ck_maps[6];
     const CUtensorMap* tc_maps = nullptr;
     void* fw = ws + wl.FW;
     // the checkpoints' tensor maps view each as [B H nchunks 128, 128] rows (int32 coordinates)
@@ -1092,7 +1094,9 @@ gdr_status gdr_chunk_bwd_grouped(const void* q, const void* k, const void* v, co
             !gdr::make_tma_map_bf16(&ck_maps[0], ws + wl.R, B, T, H, d_v) ||
             !gdr::make_tma_map_bf16(&ck_maps[1], ws + wl.DR, B, T, H, d_v) ||
             !gdr::make_tma_map_bf16(&ck_maps[2], ws + wl.ckS, 1, ck_rows, 1, d_v) ||
-            !gdr::make_tma_map_bf16(&ck_maps[3], ws + wl.ckG, 1, ck_rows, 1, d_v))
+            !gdr::make_tma_map_bf16(&ck_maps[3], ws + wl.ckG, 1, ck_rows, 1, d_v) ||
+            !gdr::make_tma_map_f32(&ck_maps[4], p.dq, B, T, H, d_k) ||
+            !gdr::make_tma_map_f32(&ck_maps[5], p.dk, B, T, H, d_k))
             return GDR_ERR_NO_DEVICE;
         tc_maps = maps;
         p.GP = nullptr;

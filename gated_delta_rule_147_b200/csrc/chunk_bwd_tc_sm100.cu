@@ -34,8 +34,11 @@
 // One CTA per (chunk, head, batch), 256 threads; thread 0 loads every operand
 // tile by TMA (q, k, v, dO, U, dr, S0, G_e) and issues the MMAs (bf16
 // operands, fp32 accumulators in tensor memory), three products:
-//   D12 = [dO ; DR] [S0 | V | R]^T            (N = 256: dO S0^T, DR S0^T and
-//                                              the four token-by-token blocks)
+//   D12 = [dO ; DR] [S0 | V | Uf]^T           (N = 256: dO S0^T, DR S0^T and
+//                                              the token-by-token blocks; Uf =
+//                                              beta v - r is the forward's
+//                                              checkpoint, so the R blocks are
+//                                              beta_j (V block) - (Uf block))
 //   D7  = [Q ; U] K^T                           (q_t . k_j and e_t . k_j for M)
 //   D3  = [[P1, -P2] ; [P3, -P4]] [U ; K]       (dq and de without their S0 part)
 //   D45 = [[P1, -P2] ; [P3, -P4]]^T [Q ; E]    (du', dkr')
@@ -59,8 +62,8 @@ struct TcParams {
 constexpr uint32_t R0 = 0;          // [dO ; DR] bf16 [128 x 128] (K-major A of D12);
                                     // after D12: [V' ; -R'] (A of the G_e product)
 constexpr uint32_t R1 = 32768;      // B of D12, per 64-column K block (32 KB): rows 0..127
-                                    // S0 (row = key channel), 128..191 V, 192..255 U,
-                                    // then R; after the last product, fp32 staging of du
+                                    // S0 (row = key channel), 128..191 V, 192..255 Uf;
+                                    // after the last product, fp32 staging of du
 constexpr uint32_t R2 = 98304;      // per 64-channel block (24 KB): Q, U = beta K, K rows
 constexpr uint32_t R3 = 147456;     // [[P1, -P2] ; [P3, -P4]] bf16 [128 x 128]
 constexpr uint32_t R4 = 180224;     // G_e, per 64-column K block (16 KB): 128 rows
@@ -84,6 +87,8 @@ __global__ void __launch_bounds__(256, 1) bwd_chunk_tc_kernel(const __grid_const
                                                               const __grid_constant__ CUtensorMap tm_dr,
                                                               const __grid_constant__ CUtensorMap tm_s0,
                                                               const __grid_constant__ CUtensorMap tm_ge,
+                                                              const __grid_constant__ CUtensorMap tm_dq,
+                                                              const __grid_constant__ CUtensorMap tm_dk,
                                                               const TcParams p) {
     extern __shared__ uint8_t smem_raw[];
     uint8_t* sm = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) &
@@ -107,7 +112,8 @@ __global__ void __launch_bounds__(256, 1) bwd_chunk_tc_kernel(const __grid_const
     uint64_t* bar_mma = bar_tma + 1;
     uint64_t* bar_drain = bar_tma + 2;
     uint64_t* bar_ge = bar_tma + 3;
-    uint32_t* s_tmem = reinterpret_cast<uint32_t*>(sm + SMALL + 8192 + 32);
+    uint64_t* bar_qk = bar_tma + 4;
+    uint32_t* s_tmem = reinterpret_cast<uint32_t*>(sm + SMALL + 8192 + 48);
     const uint32_t sbase = smem_u32(sm);
 
     if (tid == 0) {
@@ -115,10 +121,12 @@ __global__ void __launch_bounds__(256, 1) bwd_chunk_tc_kernel(const __grid_const
         mbar_init(bar_mma, 1);
         mbar_init(bar_drain, 1);
         mbar_init(bar_ge, 1);
+        mbar_init(bar_qk, 1);
         fence_barrier_init();
         // checkpoint rows: (head, chunk) -> 128 rows of a [rows, 128] view
         const int ck_row = (int)((head * p.nchunks + c) * 128);
-        mbar_expect_tx(bar_tma, 16u * 8192u);
+        // the operands of D12 first, then Q and K (D7), then G_e (D6)
+        mbar_expect_tx(bar_tma, 12u * 8192u);
 #pragma unroll
         for (int blk = 0; blk < 2; ++blk) {
             tma_load_4d(sm + R0 + blk * 16384, &tm_do, bar_tma, 64 * blk, h, t0, bb);
@@ -127,8 +135,12 @@ __global__ void __launch_bounds__(256, 1) bwd_chunk_tc_kernel(const __grid_const
             tma_load_4d(sm + R1 + blk * 32768 + 8192, &tm_s0, bar_tma, 64 * blk, 0, ck_row + 64, 0);
             tma_load_4d(sm + R1 + blk * 32768 + 16384, &tm_v, bar_tma, 64 * blk, h, t0, bb);
             tma_load_4d(sm + R1 + blk * 32768 + 24576, &tm_u, bar_tma, 64 * blk, h, t0, bb);
-            tma_load_4d(sm + R2 + blk * 24576, &tm_q, bar_tma, 64 * blk, hq, t0, bb);
-            tma_load_4d(sm + R2 + blk * 24576 + 16384, &tm_k, bar_tma, 64 * blk, hq, t0, bb);
+        }
+        mbar_expect_tx(bar_qk, 4u * 8192u);
+#pragma unroll
+        for (int blk = 0; blk < 2; ++blk) {
+            tma_load_4d(sm + R2 + blk * 24576, &tm_q, bar_qk, 64 * blk, hq, t0, bb);
+            tma_load_4d(sm + R2 + blk * 24576 + 16384, &tm_k, bar_qk, 64 * blk, hq, t0, bb);
         }
         mbar_expect_tx(bar_ge, 4u * 8192u);
 #pragma unroll
@@ -181,32 +193,9 @@ __global__ void __launch_bounds__(256, 1) bwd_chunk_tc_kernel(const __grid_const
         uint32_t ph_tma = 0;
         GDR_WAIT(bar_tma, ph_tma);
     }
-    // U = beta K (rows of the K tile scaled per token) next to Q and K; the
-    // erase reads r = beta v - U in place of U (rows 192..255 of R1, beside V)
-    {
-        const int t = tid >> 2, part = tid & 3;  // token, 4 of the 16 pieces of its 128 channels
-        const float f = s_beta[t];
-#pragma unroll
-        for (int q4 = 0; q4 < 4; ++q4) {
-            const int ch = part * 4 + q4, blk = ch >> 3;
-            const uint32_t off = sw128_chunk(t, ch & 7, 64);
-            float x[8], y[8];
-            ld_chunk(sm + R2 + blk * 24576 + 16384, off, x);
-#pragma unroll
-            for (int e = 0; e < 8; ++e) x[e] *= f;
-            st_chunk(sm + R2 + blk * 24576 + 8192, off, x);
-            ld_chunk(sm + R1 + blk * 32768 + 16384, off, x);  // v (rows 128 + t: same swizzle)
-            ld_chunk(sm + R1 + blk * 32768 + 24576, off, y);  // U
-#pragma unroll
-            for (int e = 0; e < 8; ++e) y[e] = fmaf(f, x[e], -y[e]);
-            st_chunk(sm + R1 + blk * 32768 + 24576, off, y);
-        }
-    }
-    fence_proxy_async();
-    tc_fence_before();
-    __syncthreads();
-
-    // ---- D12 = [dO ; DR] [S0 | V | R]^T ---------------------------------------------
+    // ---- D12 = [dO ; DR] [S0 | V | Uf]^T, issued as soon as its tiles land ---------
+    // (the block of the erase reads, [dO ; DR] R^T with R = Diag(beta) V - Uf, is
+    // formed on the unload from the V and Uf blocks)
     if (tid == 0) {
         tc_fence_after();
         const uint32_t id = idesc_bf16(128, 256, 0, 0);
@@ -217,7 +206,33 @@ __global__ void __launch_bounds__(256, 1) bwd_chunk_tc_kernel(const __grid_const
             mma_bf16(tmem + TM_D12, sdesc_sw128(sbase + R0 + ka, 16, 1024),
                      sdesc_sw128(sbase + R1 + kb, 16, 1024), id, ks > 0);
         }
-        // D7 = [Q ; U] K^T: A rows 0..63 Q, 64..127 U (adjacent in each channel block)
+    }
+    {
+        uint32_t ph_qk = 0;
+        GDR_WAIT(bar_qk, ph_qk);
+    }
+    // U = beta K (rows of the K tile scaled per token) next to Q and K
+    {
+        const int t = tid >> 2, part = tid & 3;  // token, 4 of the 16 pieces of its 128 channels
+        const float f = s_beta[t];
+#pragma unroll
+        for (int q4 = 0; q4 < 4; ++q4) {
+            const int ch = part * 4 + q4, blk = ch >> 3;
+            const uint32_t off = sw128_chunk(t, ch & 7, 64);
+            float x[8];
+            ld_chunk(sm + R2 + blk * 24576 + 16384, off, x);
+#pragma unroll
+            for (int e = 0; e < 8; ++e) x[e] *= f;
+            st_chunk(sm + R2 + blk * 24576 + 8192, off, x);
+        }
+    }
+    fence_proxy_async();
+    tc_fence_before();
+    __syncthreads();
+
+    // ---- D7 = [Q ; U] K^T: A rows 0..63 Q, 64..127 U (adjacent in each channel block) --
+    if (tid == 0) {
+        tc_fence_after();
         const uint32_t id7 = idesc_bf16(128, 64, 0, 0);
 #pragma unroll
         for (int ks = 0; ks < 8; ++ks) {
@@ -233,7 +248,8 @@ __global__ void __launch_bounds__(256, 1) bwd_chunk_tc_kernel(const __grid_const
     // ---- masked, decay-scaled blocks -> R3; [V' ; -R'] -> R0 ----------------------------
     {
         // lanes 0..63 (token t): dO V^T (wg 0) and dO R^T (wg 1), mask j <= t;
-        // lanes 64..127: DR V^T and DR R^T, mask j < t
+        // lanes 64..127: DR V^T and DR R^T, mask j < t; the R^T blocks are
+        // beta_j (V^T block) - (Uf^T block)
         // M_tj of this thread's block (wg 0: u_j terms, wg 1: k_j terms), summed over
         // j < s for every s <= t, then over the warp's rows for each s
         const int t = row & 63;
@@ -246,7 +262,15 @@ __global__ void __launch_bounds__(256, 1) bwd_chunk_tc_kernel(const __grid_const
         for (int half = 0; half < 2; ++half) {
             tmem_ld32_async(tmem + lane_base + TM_D12 + 128 + wg * 64 + half * 32, d);
             tmem_ld32_async(tmem + lane_base + TM_D7 + half * 32, g7);
-            tmem_wait_ld();
+            if (wg) {
+                float dvb[32];
+                tmem_ld32_async(tmem + lane_base + TM_D12 + 128 + half * 32, dvb);
+                tmem_wait_ld();
+#pragma unroll
+                for (int e = 0; e < 32; ++e) d[e] = fmaf(s_beta[half * 32 + e], dvb[e], -d[e]);
+            } else {
+                tmem_wait_ld();
+            }
             float x[32], m[32];
 #pragma unroll
             for (int e = 0; e < 32; ++e) {
@@ -269,21 +293,21 @@ __global__ void __launch_bounds__(256, 1) bwd_chunk_tc_kernel(const __grid_const
         }
     }
     {
-        // rows t of V and R scaled by Gam_C / Gam_t (R negated) -> R0
+        // rows t of V and R = beta V - Uf scaled by Gam_C / Gam_t (R negated) -> R0
         const int t = tid >> 2, part = tid & 3;
-        const float f = s_gcr[t];
+        const float f = s_gcr[t], fb = f * s_beta[t];
 #pragma unroll
         for (int q4 = 0; q4 < 4; ++q4) {
             const int ch = part * 4 + q4;
-            float y[8];
+            float y[8], u[8];
             ld_chunk(sm + R1, sw128_chunk(128 + t, ch, 256), y);
+            ld_chunk(sm + R1, sw128_chunk(192 + t, ch, 256), u);
+#pragma unroll
+            for (int e = 0; e < 8; ++e) u[e] = fmaf(f, u[e], -fb * y[e]);
 #pragma unroll
             for (int e = 0; e < 8; ++e) y[e] *= f;
             st_chunk(sm + R0, sw128_chunk(t, ch, 128), y);
-            ld_chunk(sm + R1, sw128_chunk(192 + t, ch, 256), y);
-#pragma unroll
-            for (int e = 0; e < 8; ++e) y[e] *= -f;
-            st_chunk(sm + R0, sw128_chunk(64 + t, ch, 128), y);
+            st_chunk(sm + R0, sw128_chunk(64 + t, ch, 128), u);
         }
     }
     fence_proxy_async();
@@ -334,55 +358,76 @@ __global__ void __launch_bounds__(256, 1) bwd_chunk_tc_kernel(const __grid_const
     tc_fence_after();
 
     // ---- epilogue -------------------------------------------------------------------
+    // Warps w and w + 2 of a warpgroup cover the same tokens and columns: the
+    // first (TMEM lanes 0..63: dq rows) stages du = D45 + D6 for the second
+    // (lanes 64..127: dk rows) and signals a barrier of the pair; then both
+    // form their gradients at the same time. dq and dk leave as fp32 tiles by
+    // TMA (32 columns x 64 tokens, 128-byte swizzle) from R3 and R0, whose
+    // operands the finished products no longer need; rows past T are not
+    // written.
     {
+        auto stage = [&](uint8_t* box, int t_, const float* x) {
+#pragma unroll
+            for (int c = 0; c < 8; ++c)
+                *reinterpret_cast<float4*>(box + t_ * 128 + ((c ^ (t_ & 7)) << 4)) =
+                    make_float4(x[4 * c], x[4 * c + 1], x[4 * c + 2], x[4 * c + 3]);
+        };
         float* du_f = reinterpret_cast<float*>(sm + R1);  // [64][128 + 4] fp32 (R1 is free)
         constexpr int DUP = 132;
         const int t = row & 63;
-        const size_t tok = ((size_t)bb * T + t0 + t) * H + h;
         const float gam = s_gam[t], be = s_beta[t];
+        const uint32_t pair_bar = 1u + (uint32_t)(wg * 2 + (warp & 1));
         if (row < 64) {
-            // dq = Gam dO S0^T + D3; du = D45 + D6 (staged for lanes 64..127);
-            // sums q . (dO S0^T) and u du^G
-            float red_a = 0.f, red_g = 0.f;
+            // du -> du_f and the sum u du^G
+            float red_g = 0.f;
 #pragma unroll
             for (int half = 0; half < 2; ++half) {
                 const int i0 = wg * 64 + half * 32;
-                float x1[32], d3[32], du[32], dg[32];
-                tmem_ld32_async(tmem + lane_base + TM_D12 + i0, x1);
-                tmem_ld32_async(tmem + lane_base + TM_D3 + i0, d3);
+                float du[32], dg[32], kv[32];
                 tmem_ld32_async(tmem + lane_base + TM_D45 + i0, du);
                 tmem_ld32_async(tmem + lane_base + TM_D6 + i0, dg);
                 tmem_wait_ld();
-                float qv[32], kv[32];
+#pragma unroll
+                for (int c4 = 0; c4 < 4; ++c4) {
+                    const int ch = (i0 >> 3) + c4, blk = ch >> 3;
+                    ld_chunk(sm + R2 + blk * 24576 + 16384, sw128_chunk(t, ch & 7, 64), kv + 8 * c4);
+                }
+#pragma unroll
+                for (int e = 0; e < 32; ++e) red_g = fmaf(be * kv[e], dg[e], red_g);
+#pragma unroll
+                for (int e = 0; e < 32; e += 4)
+                    *reinterpret_cast<float4*>(du_f + t * DUP + i0 + e) =
+                        make_float4(du[e] + dg[e], du[e + 1] + dg[e + 1], du[e + 2] + dg[e + 2], du[e + 3] + dg[e + 3]);
+            }
+            __threadfence_block();
+            named_bar_arrive(pair_bar, 64);
+            s_red[(6 + wg) * 64 + t] = red_g;
+            // dq = Gam dO S0^T + D3 and the sum q . (dO S0^T)
+            float red_a = 0.f;
+#pragma unroll
+            for (int half = 0; half < 2; ++half) {
+                const int i0 = wg * 64 + half * 32;
+                float x1[32], d3[32], qv[32];
+                tmem_ld32_async(tmem + lane_base + TM_D12 + i0, x1);
+                tmem_ld32_async(tmem + lane_base + TM_D3 + i0, d3);
+                tmem_wait_ld();
 #pragma unroll
                 for (int c4 = 0; c4 < 4; ++c4) {
                     const int ch = (i0 >> 3) + c4, blk = ch >> 3;
                     ld_chunk(sm + R2 + blk * 24576, sw128_chunk(t, ch & 7, 64), qv + 8 * c4);
-                    ld_chunk(sm + R2 + blk * 24576 + 16384, sw128_chunk(t, ch & 7, 64), kv + 8 * c4);
                 }
-                float dqv[32];
 #pragma unroll
                 for (int e = 0; e < 32; ++e) {
-                    dqv[e] = fmaf(gam, x1[e], d3[e]);
-                    const float u = be * kv[e];
-                    red_a = fmaf(qv[e], x1[e], red_a);  // q . (dO S0^T)
-                    red_g = fmaf(u, dg[e], red_g);
-                    du_f[t * DUP + i0 + e] = du[e] + dg[e];
+                    red_a = fmaf(qv[e], x1[e], red_a);
+                    x1[e] = fmaf(gam, x1[e], d3[e]);
                 }
-                if (t < n) {
-                    float* dst = p.dq + tok * 128 + i0;
-#pragma unroll
-                    for (int e = 0; e < 32; e += 4)
-                        *reinterpret_cast<float4*>(dst + e) = make_float4(dqv[e], dqv[e + 1], dqv[e + 2], dqv[e + 3]);
-                }
+                stage(sm + R3 + (i0 >> 5) * 8192, t, x1);
             }
             s_red[(0 + wg) * 64 + t] = gam * red_a;
-            s_red[(6 + wg) * 64 + t] = red_g;
-        }
-        __syncthreads();
-        if (row >= 64) {
+        } else {
             // de = Gam DR S0^T + D3; dkr = D45 + D6; dk = dkr + beta (de + du);
             // sums e . (dr S0^T), k dkr^G and k (de + du)
+            named_bar_sync(pair_bar, 64);
             float red_db = 0.f, red_l = 0.f, red_g = 0.f;
 #pragma unroll
             for (int half = 0; half < 2; ++half) {
@@ -399,52 +444,85 @@ __global__ void __launch_bounds__(256, 1) bwd_chunk_tc_kernel(const __grid_const
                     const int ch = (i0 >> 3) + c4, blk = ch >> 3;
                     ld_chunk(sm + R2 + blk * 24576 + 16384, sw128_chunk(t, ch & 7, 64), kv + 8 * c4);
                 }
-                float dkv[32];
 #pragma unroll
-                for (int e = 0; e < 32; ++e) {
-                    const float de = fmaf(gam, x2[e], d3[e]);
-                    const float du = du_f[t * DUP + i0 + e];
-                    dkv[e] = fmaf(be, de + du, dkr[e] + dg[e]);
-                    red_db = fmaf(kv[e], de + du, red_db);
-                    red_l = fmaf(kv[e], x2[e], red_l);  // k . (dr S0^T)
-                    red_g = fmaf(kv[e], dg[e], red_g);
-                }
-                if (t < n) {
-                    float* dst = p.dk + tok * 128 + i0;
+                for (int e = 0; e < 32; e += 4) {
+                    const float4 du4 = *reinterpret_cast<const float4*>(du_f + t * DUP + i0 + e);
+                    const float du[4] = {du4.x, du4.y, du4.z, du4.w};
 #pragma unroll
-                    for (int e = 0; e < 32; e += 4)
-                        *reinterpret_cast<float4*>(dst + e) = make_float4(dkv[e], dkv[e + 1], dkv[e + 2], dkv[e + 3]);
+                    for (int q = 0; q < 4; ++q) {
+                        const float de = fmaf(gam, x2[e + q], d3[e + q]);
+                        red_db = fmaf(kv[e + q], de + du[q], red_db);
+                        red_l = fmaf(kv[e + q], x2[e + q], red_l);  // k . (dr S0^T)
+                        red_g = fmaf(kv[e + q], dg[e + q], red_g);
+                        x2[e + q] = fmaf(be, de + du[q], dkr[e + q] + dg[e + q]);
+                    }
                 }
+                stage(sm + R0 + (i0 >> 5) * 8192, t, x2);
             }
             s_red[(2 + wg) * 64 + t] = gam * be * red_l;
             s_red[(4 + wg) * 64 + t] = red_db;
             s_red[(8 + wg) * 64 + t] = red_g;
         }
+        fence_proxy_async();
         __syncthreads();
-        if (tid < C && tid < n) {
+        if (tid == 32) {
+#pragma unroll
+            for (int box = 0; box < 4; ++box) {
+                tma_store_4d(&tm_dq, sm + R3 + box * 8192, 32 * box, h, t0, bb);
+                tma_store_4d(&tm_dk, sm + R0 + box * 8192, 32 * box, h, t0, bb);
+            }
+            bulk_commit_group();
+        }
+        if (warp == 0) {
             // dlam_s = sum_{t >= s} a_t + sum_{t >= s, j < s} M_tj + Gam_C <G_e, S0>
-            //         + sum_{j < s} c_j   (s = tid)
+            //         + sum_{j < s} c_j: lane l holds s = 2l, 2l + 1; a suffix
+            // scan of a and an exclusive prefix scan of c over the lanes
+            const int lane = tid, s0 = 2 * lane, s1 = s0 + 1;
+            auto a_of = [&](int u) {
+                return u < n ? s_red[u] + s_red[64 + u] + s_red[128 + u] + s_red[192 + u] : 0.f;
+            };
+            auto c_of = [&](int j) { return s_red[384 + j] + s_red[448 + j] + s_red[512 + j] + s_red[576 + j]; };
+            const float a0 = a_of(s0), a1 = a_of(s1), c0 = c_of(s0), c1 = c_of(s1);
+            float suf = a0 + a1, pre = c0 + c1;
+#pragma unroll
+            for (int off = 1; off < 32; off <<= 1) {
+                const float ys = __shfl_down_sync(0xffffffffu, suf, off);
+                const float yp = __shfl_up_sync(0xffffffffu, pre, off);
+                if (lane + off < 32) suf += ys;
+                if (lane >= off) pre += yp;
+            }
+            pre -= c0 + c1;  // exclusive: sum over j < s0
             float ge = 0.f;
 #pragma unroll
             for (int w = 0; w < 8; ++w) ge += s_ge[w];
-            float cum = s_gam[C - 1] * ge;  // padding tokens decay by 1: Gam_{63} = Gam_{n-1}
+            const float base = s_gam[C - 1] * ge;  // padding tokens decay by 1: Gam_{63} = Gam_{n-1}
+            float m0 = 0.f, m1 = 0.f;
 #pragma unroll
-            for (int w = 0; w < 8; ++w) cum += s_M[w * 64 + tid];
-            for (int u = tid; u < n; ++u)
-                cum += s_red[u] + s_red[64 + u] + s_red[128 + u] + s_red[192 + u];
-            for (int j = 0; j < tid; ++j)
-                cum += s_red[384 + j] + s_red[448 + j] + s_red[512 + j] + s_red[576 + j];
-            const size_t gi = ((size_t)bb * T + t0 + tid) * H + h;
-            p.dalpha[gi] = cum / s_alpha[tid];
-            p.db[gi] = s_red[256 + tid] + s_red[320 + tid];
+            for (int w = 0; w < 8; ++w) {
+                m0 += s_M[w * 64 + s0];
+                m1 += s_M[w * 64 + s1];
+            }
+            const float cum0 = base + m0 + suf + pre;
+            const float cum1 = base + m1 + (suf - a0) + (pre + c0);
+            const size_t gi = ((size_t)bb * T + t0 + s0) * H + h;
+            if (s0 < n) {
+                p.dalpha[gi] = cum0 / s_alpha[s0];
+                p.db[gi] = s_red[256 + s0] + s_red[320 + s0];
+            }
+            if (s1 < n) {
+                p.dalpha[gi + H] = cum1 / s_alpha[s1];
+                p.db[gi + H] = s_red[256 + s1] + s_red[320 + s1];
+            }
         }
     }
 
+    if (tid == 32) bulk_wait_group_read0();
 finish:
     if (!ok && tid == 0) {
         // before the block leaves (each wait bounded): the input copies have
         // landed and every issued MMA has finished
         (void)mbar_wait(bar_tma, 0);
+        (void)mbar_wait(bar_qk, 0);
         (void)mbar_wait(bar_ge, 0);
         mma_commit(bar_drain);
         (void)mbar_wait(bar_drain, 0);
@@ -461,7 +539,8 @@ finish:
 // maps: q, k (q/k heads), v, dO (value heads), bf16 [B, T, H, 128] each.
 // ck_maps: U = beta v - r and dr (bf16 [B, T, H, 128]), the chunk-start states
 // and the chunk-end state gradients (bf16 [B, H, nchunks, 128, 128], each
-// mapped as one [B H nchunks 128, 128] view).
+// mapped as one [B H nchunks 128, 128] view), then dq and dk (fp32
+// [B, T, H, 128], box 32 x 64 tokens, for the tile stores).
 cudaError_t launch_bwd_chunk_tc(const CUtensorMap* maps, const CUtensorMap* ck_maps, const void* alpha,
                                 const void* beta, float* dq, float* dk, float* dalpha, float* db,
                                 int* d_status, int B, int T, int H, int group, int nchunks,
@@ -475,7 +554,8 @@ cudaError_t launch_bwd_chunk_tc(const CUtensorMap* maps, const CUtensorMap* ck_m
     cudaError_t e = cudaFuncSetAttribute(bwd_chunk_tc_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, SMEM_BYTES);
     if (e != cudaSuccess) return e;
     bwd_chunk_tc_kernel<<<dim3(nchunks, H, B), 256, SMEM_BYTES, st>>>(maps[0], maps[1], maps[2], maps[3], ck_maps[0],
-                                                                    ck_maps[1], ck_maps[2], ck_maps[3], p);
+                                                                    ck_maps[1], ck_maps[2], ck_maps[3], ck_maps[4],
+                                                                    ck_maps[5], p);
     return cudaGetLastError();
 }
 
