@@ -51,6 +51,15 @@ namespace bwdtc {
 
 using namespace chunkc;
 
+// Named barrier `id` (1..15) over `n` threads (a multiple of 32): producers
+// arrive, consumers wait.
+__device__ __forceinline__ void named_bar_arrive(uint32_t id, uint32_t n) {
+    asm volatile("bar.arrive %0, %1;" ::"r"(id), "r"(n) : "memory");
+}
+__device__ __forceinline__ void named_bar_sync(uint32_t id, uint32_t n) {
+    asm volatile("bar.sync %0, %1;" ::"r"(id), "r"(n) : "memory");
+}
+
 struct TcParams {
     const __nv_bfloat16 *alpha, *beta;     // scalar gates [B, T, H]
     float *dq, *dk, *dalpha, *db;          // dq, dk [B, T, H, 128] per value head; gates [B, T, H]

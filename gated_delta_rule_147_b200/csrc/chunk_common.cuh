@@ -207,15 +207,6 @@ __device__ __forceinline__ void compute_bar() {
     asm volatile("bar.sync 1, 256;" ::: "memory");
 }
 
-// Named barrier `id` (1..15) over `n` threads (a multiple of 32): producers
-// arrive, consumers wait.
-__device__ __forceinline__ void named_bar_arrive(uint32_t id, uint32_t n) {
-    asm volatile("bar.arrive %0, %1;" ::"r"(id), "r"(n) : "memory");
-}
-__device__ __forceinline__ void named_bar_sync(uint32_t id, uint32_t n) {
-    asm volatile("bar.sync %0, %1;" ::"r"(id), "r"(n) : "memory");
-}
-
 // In lane l, the sum over the warp's 32 lanes of x[l] (a reduce-scatter by
 // recursive halving: 31 shuffles for 32 columns). x is destroyed.
 __device__ __forceinline__ float warp_colsum32(float* x, int lane) {
