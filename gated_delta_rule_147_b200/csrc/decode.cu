@@ -34,6 +34,13 @@ __global__ void __launch_bounds__(256, NR <= 16 ? 2 : 1) decode_step_kernel(
     __shared__ float4 s_red[2][RPP][TPR];
     __shared__ float s_dots[2];
 
+    // Launched as a programmatic dependent of the previous work on the stream:
+    // the next step's blocks may be scheduled once every block of this one has
+    // started, and nothing is read before the previous grid has completed and
+    // its writes (the state of the previous step, this step's inputs) are visible.
+    asm volatile("griddepcontrol.launch_dependents;");
+    asm volatile("griddepcontrol.wait;" ::: "memory");
+
     const size_t bhq = (size_t)(bh / group);  // q, k have H / group heads
     for (int i = tid; i < dk; i += 256) {
         const size_t gi = (size_t)bh * dk + i;
@@ -136,18 +143,28 @@ static cudaError_t launch_decode_dv(const void* q, const void* k, const void* v,
                                     void* o, int BH, int dk, int dvf, int group, cudaStream_t st) {
     constexpr int RPP = 256 / (DV / 4);
     const int nr = (dk + RPP - 1) / RPP;
-    const dim3 grid(BH, dvf / DV);
-#define GDR_DEC(NRV)                                                                              \
-    decode_step_kernel<TI, DV, NRV><<<grid, 256, 0, st>>>(                                        \
-        (const TI*)q, (const TI*)k, (const TI*)v, (const TI*)a, (const TI*)b, (const TI*)w, ak, bk, \
-        wk, S, (TI*)o, dk, dvf, group)
+    cudaLaunchConfig_t cfg = {};
+    cfg.gridDim = dim3(BH, dvf / DV);
+    cfg.blockDim = dim3(256, 1, 1);
+    cfg.dynamicSmemBytes = 0;
+    cfg.stream = st;
+    cudaLaunchAttribute attr[1];
+    attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;  // overlap the previous tail
+    attr[0].val.programmaticStreamSerializationAllowed = 1;
+    cfg.attrs = attr;
+    cfg.numAttrs = 1;
+    cudaError_t e;
+#define GDR_DEC(NRV)                                                                                  \
+    e = cudaLaunchKernelEx(&cfg, decode_step_kernel<TI, DV, NRV>, (const TI*)q, (const TI*)k,        \
+                           (const TI*)v, (const TI*)a, (const TI*)b, (const TI*)w, ak, bk, wk, S,     \
+                           (TI*)o, dk, dvf, group)
     if (nr <= 4) GDR_DEC(4);
     else if (nr <= 8) GDR_DEC(8);
     else if (nr <= 16) GDR_DEC(16);
     else if (nr <= 32) GDR_DEC(32);
     else return cudaErrorInvalidValue;
 #undef GDR_DEC
-    return cudaGetLastError();
+    return e;
 }
 
 // Rows per thread needed for (d_k, d_v); the launcher supports up to 32.
