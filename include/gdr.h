@@ -261,13 +261,15 @@ size_t gdr_chunk_fwd_static_capacity(void);
  *   - the Gated DeltaNet form in bf16 with d_k = d_v = 128 (alpha and b
  *     scalar, w tied) runs on tensor cores throughout (bf16 operands, fp32
  *     accumulation) and scans nothing token by token: the forward two-pass
- *     kernels give S at every chunk start and r_t; the backward recurrence
+ *     kernels give S at every chunk start and U_t = beta_t v_t - r_t, both
+ *     stored in bf16 (the chunk kernel uses them only as tensor-core
+ *     operands and for one inner product per chunk); the backward recurrence
  *     of G taken a chunk at a time (per chunk, with Y_j = k_j G_j, T the
  *     forward's UT transform and Aq its masked q k^T block:
  *     (I + A)^T Y = Diag(g_{n-1}/g) K G_in + Aq^T dO and
  *     G_out = g_{n-1} G_in + (Diag(g) Q)^T dO - (Diag(beta g) K)^T Y) gives
- *     G at every chunk end, dr, dv and dS0 (a first pass over all chunks
- *     forms the chunk factors, a second walks the chunks in reverse); then
+ *     G at every chunk end and dr (bf16), dv and dS0 (a first pass over all
+ *     chunks forms the chunk factors, a second walks the chunks in reverse); then
  *     the chunk gradients as masked, decay-scaled products, one CTA per
  *     (chunk, head) writing dalpha and db directly. Every gradient of this
  *     form carries bf16 operand rounding. The bounded waits of these kernels
@@ -324,7 +326,8 @@ size_t gdr_chunk_bwd_grouped_workspace_size(int B, int T, int H_qk, int H, int d
 
 /* Bytes of workspace gdr_chunk_bwd needs (0 for T < 1 or bad sizes): fp32
  * chunk-start states and chunk-end state gradients (2 x B H ceil(T/64) d_k
- * d_v), r_t and dr_t of every token (2 x B T H d_v), and scalar-gate partial
+ * d_v), r_t and dr_t of every token (2 x B T H d_v; the tensor-core form
+ * keeps bf16 copies in the first half of each of these four regions), and scalar-gate partial
  * sums (3 x ceil(d_k / RB) x B T H, RB = 128 / (d_v / 8 rounded up to a power
  * of two)), and when d_k = d_v = 128 the forward's per-token -W, P and
  * q k^T block rows (B T H (d_k + d_v + 64) bf16; the gradient pass's
@@ -345,6 +348,10 @@ size_t gdr_chunk_bwd_workspace_size(int B, int T, int H, int d_k, int d_v);
  * d_k > 128 and d_v = 256 runs as two blocks of 128 value columns: every
  * column's reductions over d_k stay inside its block).
  * Alignment: S, o, q, k, v and channel gates must be 16-byte aligned.
+ * The step is a programmatic dependent launch on `stream`: its blocks may be
+ * scheduled while the previous kernel on the stream finishes, and each waits
+ * for that kernel's completion before reading anything, so stream order is
+ * kept as for any launch.
  * Returns as gdr_chunk_fwd.
  */
 gdr_status gdr_decode_step(const void* q, const void* k, const void* v,
