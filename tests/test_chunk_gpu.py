@@ -337,6 +337,28 @@ def test_grouped_workload_full_size_sampled_heads(cuda_device):
     assert_close(ST_s, ST_ref, TOL["bf16"], f"S_T {heads}")
 
 
+@pytest.mark.parametrize("H", [2, 40])
+def test_erase_free_decay_range(cuda_device, H):
+    """Erase-free chunks whose decay span is beyond the two-factor range are
+    applied token by token, between ordinary chunks and twice in a row (the
+    kernel builds the next chunk's operands while the current chunk's last
+    product runs, and runs a flagged chunk after the previous state update).
+    d_status carries the flag and the result matches the oracle. H = 40 takes
+    the 128-column CTAs."""
+    wl = small("gdn2", T=320, H=H, dv=128, alpha="channel", b="none", w="none", s0=True, seed=741)
+    inp = make_chunk_inputs(wl)
+    a = inp["alpha"].clone()
+    for lo, hi in ((64, 128), (192, 256), (256, 320)):  # chunks 1, 3 and 4: 63 x 4.6 nats > 160
+        a[:, lo:hi] = 0.01
+    inp["alpha"] = a
+    st = torch.zeros(1, dtype=torch.int32, device=cuda_device)
+    o, ST = run_chunk(inp, cuda_device, d_status=st)
+    assert int(st.item()) & GDR_DEVICE_DECAY_RANGE
+    o_ref, ST_ref = run_oracle(inp)
+    assert_close(o, o_ref, TOL["bf16"], "o")
+    assert_close(ST, ST_ref, TOL["bf16"], "S_T")
+
+
 @pytest.mark.parametrize("dv,akind,wkind", [(256, "channel", "none"), (128, "scalar", "channel")])
 def test_erase_free_wide_ctas(cuda_device, dv, akind, wkind):
     """More 64-column tiles than SMs: the erase-free kernel carries 128 value
